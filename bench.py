@@ -1,0 +1,541 @@
+"""Benchmark of the B200 hybrid attention library.
+
+One step = one training pass of the hot path on the Llama-3-8B-shaped layer
+(B=2, H=32, T=8192, d=128, w=128, M=8, bf16 I/O): lz_hybrid_fwd (gated
+chunked forward, window + meta softmax, fused sum) followed by lz_hybrid_bwd
+(every gradient).  Inputs are resident in HBM before timing starts and are
+larger than L2.  The same JSON line also carries the forward-only workloads
+and the decode step (sub-measurements, each with its own roofline).
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lizard|reference]
+Under torchrun every rank runs its own replica of the workload (weak scaling);
+rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+import torch.distributed as dist
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "hybrid GLA+SWA attention tokens/s (fwd, fwd+bwd, decode) on 1 B200; % of roofline"
+
+
+# --------------------------------------------------------------------------
+# ranks
+# --------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend="nccl", timeout_s=120):
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend=backend,
+                                timeout=datetime.timedelta(seconds=timeout_s))
+
+
+def barrier():
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def max_over_ranks(x: float, device) -> float:
+    """Maximum of a per-rank number over all ranks (identity on one rank)."""
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, device) -> float:
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------
+# clocks
+# --------------------------------------------------------------------------
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.out = []
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            uuid = str(device_index)
+        self.cmd = ["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
+                    "-lms", "100", "-i", uuid]
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.out = [ln for ln in (out or "").splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.out:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# roofline bookkeeping
+# --------------------------------------------------------------------------
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": float(pk["hbm_gbs"]), "bf16_tflops": float(pk["bf16_tflops"]),
+                "bf16_tflops_sustained": float(pk.get("bf16_tflops_sustained",
+                                                      pk["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def algorithmic_bytes(kernel: str, wl) -> float | None:
+    """Bytes the method must move per launch of ``kernel`` on workload ``wl``
+    (per (batch, head, token): q, k, v, o at the I/O size, g in fp32; the
+    backward reads q, k, v, g, dO and writes dq, dk, dv, dg).  Intermediate
+    chunk states and scratch are not algorithmic."""
+    e = 2 if wl.io == "bf16" else 4
+    n = wl.B * wl.H * wl.T
+    d = wl.dk
+    if kernel.startswith("gla_fwd") or kernel.startswith("hybrid_fwd"):
+        return n * (4 * d * e + 4 * d)
+    if kernel.startswith("swa_fwd"):
+        return n * (4 * d * e + 4)
+    if kernel.startswith("gla_bwd") or kernel.startswith("hybrid_bwd"):
+        return n * (7 * d * e + 8 * d)
+    if kernel.startswith("gla_state_pass"):
+        return n * (2 * d * e + 4 * d)
+    if kernel.startswith("swa_bwd_q"):
+        return n * (3 * d * e + 4 + 4)
+    if kernel.startswith("swa_bwd_kv"):
+        return n * (6 * d * e + 8)
+    return None
+
+
+def decode_bytes_per_step(dwl) -> float:
+    """fp32 state read + write, K/V ring read, one new row of q, k, v, g, o."""
+    d = dwl.dk
+    per = 2 * d * d * 4 + 2 * dwl.w * d * 2 + 3 * d * 2 + d * 4 + d * 2 + 2 * d * 2
+    return dwl.Bd * dwl.H * per
+
+
+def train_flops(wl) -> float:
+    """Algorithmic flops of one fwd+bwd step (causal half of intra tiles,
+    valid window keys only)."""
+    d, C, n = wl.dk, wl.chunk, wl.B * wl.H * wl.T
+    gla = 3 * (C * 2 * d + 4 * d * d)
+    kbar = min(wl.w, wl.T)  # mean valid window ~ w for T >> w
+    swa = 3 * (2 * (kbar + wl.M) * 2 * d)
+    return n * (gla + swa)
+
+
+# --------------------------------------------------------------------------
+# the step
+# --------------------------------------------------------------------------
+class TrainStep:
+    """Buffers and one fwd+bwd pass through the C ABI."""
+
+    def __init__(self, wl, x, device):
+        import gated_linear_sliding_chunked_b200 as L
+        self.L = L
+        self.wl = wl
+        self.x = x
+        B, H, T, dk, dv, M = wl.B, wl.H, wl.T, wl.dk, wl.dv, wl.M
+        self.dims = L.make_dims(B, H, T, dk, dv, chunk=wl.chunk, w=wl.w, M=M,
+                                io=L.io_of(wl.torch_dtype), scale=wl.scale, alpha=wl.alpha)
+        dt = wl.torch_dtype
+        mk = lambda *s, dtype=dt: torch.empty(*s, dtype=dtype, device=device)
+        self.o = mk(B, H, T, dv)
+        self.lse = mk(B, H, T, dtype=torch.float32)
+        self.dq, self.dk, self.dv = mk(B, H, T, dk), mk(B, H, T, dk), mk(B, H, T, dv)
+        self.dg = mk(B, H, T, dk, dtype=torch.float32)
+        self.dmk = mk(H, M, dk, dtype=torch.float32)
+        self.dmv = mk(H, M, dv, dtype=torch.float32)
+        self.dalpha = mk(4, dtype=torch.float32)
+        nf = L.lz_workspace_bytes(self.dims, L.LZ_WS_HYBRID_FWD)
+        nb = L.lz_workspace_bytes(self.dims, L.LZ_WS_HYBRID_BWD)
+        self.wsf, self.nf = mk(max(nf, 1), dtype=torch.uint8), nf
+        self.wsb, self.nb = mk(max(nb, 1), dtype=torch.uint8), nb
+
+    def run(self, x=None):
+        x = x or self.x
+        L, d = self.L, self.dims
+        L.lz_hybrid_fwd(d, x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], None,
+                        self.o, None, self.lse, None, self.wsf, self.nf)
+        L.lz_hybrid_bwd(d, x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], None,
+                        self.lse, x["dO"], None, self.dq, self.dk, self.dv, self.dg, None,
+                        self.dmk, self.dmv, self.dalpha, self.wsb, self.nb)
+
+    def outputs(self):
+        return [self.o, self.dq, self.dk, self.dv, self.dg, self.dmk, self.dmv, self.dalpha]
+
+
+def time_region(fn, steps, device):
+    """Device time of ``steps`` calls of fn (barrier + synchronize on both
+    sides, CUDA events on the current stream); returns ms per step."""
+    barrier()
+    torch.cuda.synchronize(device)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize(device)
+    barrier()
+    return a.elapsed_time(b) / max(steps, 1)
+
+
+def kernel_table(records):
+    tab = {}
+    for name, ms in records:
+        c, t = tab.get(name, (0, 0.0))
+        tab[name] = (c + 1, t + ms)
+    return tab
+
+
+def roofline_for(tab, wl, peaks, traffic=None):
+    """Roofline object for the kernel with the largest total device time."""
+    if not tab:
+        return None, None
+    dom = max(tab, key=lambda k: tab[k][1])
+    count, total = tab[dom]
+    avg_ms = total / count
+    by = algorithmic_bytes(dom, wl)
+    if by is None:
+        return dom, None
+    achieved = by / (avg_ms * 1e-3) / 1e9
+    return dom, {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
+                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                 "frac": round(achieved / peaks["hbm_gbs"], 4),
+                 "traffic": traffic, "launches": count, "avg_ms": round(avg_ms, 4),
+                 "algorithmic_bytes_per_launch": by,
+                 "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs copy)"}
+
+
+# --------------------------------------------------------------------------
+# sub-measurements
+# --------------------------------------------------------------------------
+def measure_fwd(wl, device, steps, warmup, peaks, seed):
+    import gated_linear_sliding_chunked_b200 as L
+    from gated_linear_sliding_chunked_b200 import inputs as I
+    x = I.make_inputs(wl, seed=seed, device=device)
+    dims = L.make_dims(wl.B, wl.H, wl.T, wl.dk, wl.dv, chunk=wl.chunk, w=wl.w, M=wl.M,
+                       io=L.io_of(wl.torch_dtype), scale=wl.scale, alpha=wl.alpha)
+    o = torch.empty(wl.B, wl.H, wl.T, wl.dv, dtype=wl.torch_dtype, device=device)
+    n = L.lz_workspace_bytes(dims, L.LZ_WS_HYBRID_FWD)
+    ws = torch.empty(max(n, 1), dtype=torch.uint8, device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+
+    def fn():
+        flush.zero_()  # 256 MB write: evicts L2 between iterations
+        L.lz_hybrid_fwd(dims, x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], None,
+                        o, None, None, None, ws, n)
+
+    for _ in range(warmup):
+        fn()
+    L.lz_timing_enable(True)
+    ms = time_region(fn, steps, device)
+    L.lz_timing_enable(False)
+    tab = kernel_table(L.lz_timing_read())
+    lib_ms = sum(t for (c, t) in tab.values()) / steps
+    dom, roof = roofline_for(tab, wl, peaks)
+    del x, o, ws, flush
+    return {"workload": wl.name, "tokens_per_s": wl.B * wl.T / (lib_ms * 1e-3),
+            "ms_per_call": round(lib_ms, 4), "ms_per_iter_incl_l2_flush": round(ms, 4),
+            "l2": "256 MB flush between iterations (not counted in ms_per_call)",
+            "kernels": {k: [c // steps, round(t / c, 4)] for k, (c, t) in tab.items()},
+            "roofline": roof}
+
+
+def measure_decode(device, steps, warmup, peaks, seed, n_steps=1000):
+    import gated_linear_sliding_chunked_b200 as L
+    from gated_linear_sliding_chunked_b200 import inputs as I
+    dwl = I.DECODE
+    st = I.make_decode_state(dwl, seed=seed, device=device)
+    toks = I.make_decode_tokens(dwl, steps=n_steps, seed=seed + 1, device=device)
+    o = torch.empty(dwl.Bd, dwl.H, dwl.dv, dtype=torch.bfloat16, device=device)
+
+    def run_all():
+        for s in range(n_steps):
+            L.lz_gla_decode_step(dwl.Bd, dwl.H, dwl.dk, dwl.dv, dwl.w, dwl.M, L.LZ_BF16,
+                                 dwl.scale, dwl.alpha, st["state"], st["kring"], st["vring"],
+                                 st["pos"], toks["q"][s], toks["k"][s], toks["v"][s],
+                                 toks["g"][s], st["meta_k"], st["meta_v"], o)
+
+    run_all()  # warm-up pass over all steps
+    L.lz_timing_enable(True)
+    ms = time_region(run_all, 1, device)
+    L.lz_timing_enable(False)
+    tab = kernel_table(L.lz_timing_read())
+    per_step_ms = ms / n_steps
+    bytes_step = decode_bytes_per_step(dwl)
+    c, t = tab.get("decode_step", (1, per_step_ms))
+    k_ms = t / c
+    ach = bytes_step / (k_ms * 1e-3) / 1e9
+    del st, toks
+    return {"workload": dwl.name, "steps": n_steps,
+            "tokens_per_s": dwl.Bd / (per_step_ms * 1e-3), "ms_per_step": round(per_step_ms, 5),
+            "kernels": {k: [c2 // n_steps, round(t2 / c2, 5)] for k, (c2, t2) in tab.items()},
+            "roofline": {"kernel": "decode_step", "bound": "hbm", "achieved": round(ach, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(ach / peaks["hbm_gbs"], 4),
+                         "algorithmic_bytes_per_launch": bytes_step,
+                         "avg_ms": round(k_ms, 5)}}
+
+
+# --------------------------------------------------------------------------
+# oracle timing (CPU baseline / reference arm)
+# --------------------------------------------------------------------------
+def oracle_sample(wl, pairs: int, T: int, seed: int = 0):
+    """A bounded sample of the training workload for the fp64 CPU oracle:
+    ``pairs`` (batch, head) problems of the first ``T`` tokens."""
+    from gated_linear_sliding_chunked_b200 import inputs as I
+    small = wl.with_(B=1, H=pairs, T=T)
+    x = I.make_inputs(small, seed=seed, device="cpu")
+    return small, {k: v.to(torch.float64).numpy() for k, v in x.items()}
+
+
+def oracle_train_step(small, xs, nthreads):
+    import oracle
+    fwd = oracle.hybrid_fwd(xs["q"], xs["k"], xs["v"], xs["g"], xs["meta_k"], xs["meta_v"],
+                            small.w, small.scale, small.alpha, nthreads=nthreads)
+    oracle.hybrid_bwd(xs["q"], xs["k"], xs["v"], xs["g"], xs["meta_k"], xs["meta_v"], xs["dO"],
+                      small.w, small.scale, small.alpha, nthreads=nthreads)
+    return fwd
+
+
+def cpu_baseline(wl, budget_s=20.0):
+    """Time the oracle as it stands on this host's cores on a bounded sample;
+    report tokens/s in the workload's units (a token = one position over all
+    H heads, so a sample of P head-sequences of T tokens is P*T/H tokens)."""
+    cores = os.cpu_count() or 1
+    pairs = max(1, min(cores, 16))
+    T = 1024
+    small, xs = oracle_sample(wl, pairs, T)
+    t0 = time.perf_counter()
+    oracle_train_step(small, xs, pairs)
+    dt = time.perf_counter() - t0
+    reps = 1
+    while time.perf_counter() - t0 < min(budget_s, 4 * dt) and reps < 3:
+        oracle_train_step(small, xs, pairs)
+        reps += 1
+    wall = (time.perf_counter() - t0) / reps
+    tokens = pairs * T / wl.H
+    return {"value": tokens / wall, "unit": "tokens/s", "cores": pairs, "kind": "oracle",
+            "sample": f"{pairs} (batch, head) problems x first {T} tokens of the training "
+                      f"workload, fwd+bwd, fp64, std::thread over pairs; {reps} rep(s), "
+                      f"{wall:.2f} s each; tokens = pairs*T/H"}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    from gated_linear_sliding_chunked_b200 import inputs as I
+    if rank != 0:
+        return 0
+    wl = I.TRAIN_BF16
+    cores = os.cpu_count() or 1
+    pairs = max(1, min(cores, 8))
+    T = 512
+    small, xs = oracle_sample(wl, pairs, T)
+    for _ in range(args.warmup):
+        oracle_train_step(small, xs, pairs)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_train_step(small, xs, pairs)
+    wall = (time.perf_counter() - t0) / max(args.steps, 1)
+    tokens = pairs * T / wl.H
+    val = tokens / wall
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
+            "higher_is_better": True, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": wall * 1e3, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "global_batch": wl.B, "seq_len": wl.T,
+                       "parallelism": "host cores (oracle)"},
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": pairs, "kind": "oracle",
+                             "sample": f"{pairs} (batch, head) problems x first {T} tokens per "
+                                       f"step, fwd+bwd in fp64; tokens = pairs*T/H"},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
+# main
+# --------------------------------------------------------------------------
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="lizard", choices=["lizard", "reference"])
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the forward-only and decode sub-measurements")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)
+
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world)
+
+    from gated_linear_sliding_chunked_b200 import build as lbuild
+    if rank == 0:
+        lbuild.build()
+    barrier()
+    import gated_linear_sliding_chunked_b200 as L
+    from gated_linear_sliding_chunked_b200 import inputs as I
+    L.load()
+    peaks = load_peaks()
+
+    wl = I.TRAIN_BF16
+    # each rank draws its own replica (seed = rank): weak scaling
+    xh = I.make_inputs(wl, seed=rank, device="cpu")
+    xh = {k: v.pin_memory() for k, v in xh.items()}
+    xd = {k: v.to(device, non_blocking=True) for k, v in xh.items()}
+    torch.cuda.synchronize(device)
+    step = TrainStep(wl, xd, device)
+
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize(device)
+
+    sampler = ClockSampler(local)
+    L.lz_timing_enable(True)
+    with sampler:
+        ms = time_region(step.run, args.steps, device)
+    L.lz_timing_enable(False)
+    records = L.lz_timing_read()
+    ms_max = max_over_ranks(ms, device)
+    tokens_step = wl.B * wl.T
+    value = tokens_step * world / (ms_max * 1e-3)
+    tab = kernel_table(records)
+    launches = len(records)
+    dom, roof = roofline_for(tab, wl, peaks)
+    flops = train_flops(wl)
+
+    # ---- end to end through the C ABI with host buffers --------------------
+    in_keys = ("q", "k", "v", "g", "meta_k", "meta_v", "dO")
+    h2d = sum(xh[k].numel() * xh[k].element_size() for k in in_keys)
+    outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in step.outputs()]
+    d2h = sum(t.numel() * t.element_size() for t in outs_h)
+    xe = {k: torch.empty_like(v) for k, v in xd.items()}
+
+    def e2e_step():
+        for k in in_keys:
+            xe[k].copy_(xh[k], non_blocking=True)
+        step.run(xe)
+        for hbuf, dbuf in zip(outs_h, step.outputs()):
+            hbuf.copy_(dbuf, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    e2e_step()
+    ms_e2e = max_over_ranks(time_region(e2e_step, e2e_steps, device), device)
+    e2e_val = tokens_step * world / (ms_e2e * 1e-3)
+    del xe
+
+    extras = {}
+    if not args.no_extras:
+        extras["fwd_bf16_T2048"] = measure_fwd(I.FWD_BF16, device, 10, 3, peaks, seed=rank)
+        extras["long_T65536"] = measure_fwd(I.LONG_BF16, device, 3, 1, peaks, seed=rank)
+        extras["decode"] = measure_decode(device, 1, 1, peaks, seed=rank)
+        extras["train_step_breakdown"] = {k: [c // args.steps, round(t / c, 4)]
+                                          for k, (c, t) in tab.items()}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl)
+
+    clocks = sampler.summary()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic (seeded, BASELINE-shaped distributions)",
+            "config": {"workload": wl.name, "global_batch": wl.B * world, "seq_len": wl.T,
+                       "heads": wl.H, "head_dim": wl.dk, "window": wl.w, "meta_tokens": wl.M,
+                       "chunk": wl.chunk, "io": wl.io, "alpha": wl.alpha,
+                       "parallelism": f"replicas x{world} (no data-path collective)",
+                       "l2": "inputs larger than L2 (~0.8 GB read per step), no flush"},
+            "roofline": roof,
+            "effective_tflops": flops / (ms_max * 1e-3) / 1e12,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "extras": extras,
+        }
+        print(json.dumps(line), flush=True)
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,304 @@
+"""Python binding of the B200 hybrid attention library (liblizard.so).
+
+The operator is the hybrid attention of "Lizard: An Efficient Linearization
+Framework for Large Language Models" (gist.science technical summary,
+section 2a): gated linear attention S_t = diag(exp(g_t)) S_{t-1} + k_t v_t^T,
+o_gla_t = q_t^T S_t, plus sliding-window softmax attention with meta-memory
+sink tokens, summed as o = o_gla + alpha * o_swa.
+
+Everything here is argument marshalling: the ``lz_*`` functions have the C
+ABI's names and arguments (include/lizard.h) and take torch tensors for the
+pointers; the helpers without the prefix only allocate outputs and scratch
+with torch and call them.  Every step of the computation runs in the CUDA
+library.  There is no CPU fallback: if liblizard.so is missing, loading it
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "liblizard.so")
+
+LZ_OK, LZ_ERR_INVALID_ARG, LZ_ERR_UNSUPPORTED, LZ_ERR_CUDA, LZ_ERR_TIMEOUT = range(5)
+LZ_F32, LZ_BF16 = 0, 1
+LZ_WS_GLA_FWD, LZ_WS_HYBRID_FWD, LZ_WS_GLA_BWD, LZ_WS_SWA_BWD, LZ_WS_HYBRID_BWD = range(5)
+
+EXPORTS = ("lz_gla_fwd", "lz_gla_bwd", "lz_swa_meta_fwd", "lz_hybrid_fwd", "lz_swa_meta_bwd",
+           "lz_hybrid_bwd", "lz_gla_decode_step", "lz_workspace_bytes", "lz_last_error",
+           "lz_version", "lz_timing_enable", "lz_timing_read")
+
+
+class LzError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"lizard status {status}: {message}")
+        self.status = status
+
+
+class LzDims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int),
+                ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("chunk", ctypes.c_int),
+                ("w", ctypes.c_int), ("M", ctypes.c_int), ("io", ctypes.c_int),
+                ("scale", ctypes.c_float), ("alpha", ctypes.c_float)]
+
+
+_lib = None
+_P = ctypes.c_void_p
+
+
+def load(path: str = LIB_PATH):
+    """Load liblizard.so (raises if it is absent: there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library not built: {path} is missing "
+                           "(run python -m gated_linear_sliding_chunked_b200.build)")
+    lib = ctypes.CDLL(path)
+    D = ctypes.POINTER(LzDims)
+    sz = ctypes.c_size_t
+    lib.lz_workspace_bytes.argtypes = [D, ctypes.c_int]
+    lib.lz_workspace_bytes.restype = sz
+    lib.lz_gla_fwd.argtypes = [D] + [_P] * 7 + [_P, sz, _P]
+    lib.lz_swa_meta_fwd.argtypes = [D] + [_P] * 7 + [_P]
+    lib.lz_hybrid_fwd.argtypes = [D] + [_P] * 11 + [_P, sz, _P]
+    lib.lz_gla_bwd.argtypes = [D] + [_P] * 12 + [_P, sz, _P]
+    lib.lz_swa_meta_bwd.argtypes = [D] + [_P] * 12 + [_P, sz, _P]
+    lib.lz_hybrid_bwd.argtypes = [D] + [_P] * 18 + [_P, sz, _P]
+    lib.lz_gla_decode_step.argtypes = ([ctypes.c_int] * 7 + [ctypes.c_float] * 2 +
+                                       [_P] * 11 + [_P])
+    lib.lz_timing_enable.argtypes = [ctypes.c_int]
+    lib.lz_timing_read.argtypes = [ctypes.c_char_p, sz, ctypes.POINTER(ctypes.c_float),
+                                   ctypes.c_int]
+    for name in EXPORTS:
+        if name in ("lz_last_error", "lz_version"):
+            getattr(lib, name).restype = ctypes.c_char_p
+            getattr(lib, name).argtypes = []
+        elif name != "lz_workspace_bytes":
+            getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int):
+    if status != LZ_OK:
+        raise LzError(status, load().lz_last_error().decode())
+
+
+def io_of(dtype) -> int:
+    if dtype == torch.float32:
+        return LZ_F32
+    if dtype == torch.bfloat16:
+        return LZ_BF16
+    raise TypeError(f"unsupported I/O dtype {dtype}")
+
+
+def make_dims(B, H, T, dk, dv, *, chunk=64, w=1, M=0, io=LZ_BF16, scale=None,
+              alpha=0.5) -> LzDims:
+    if scale is None:
+        scale = 1.0 / math.sqrt(dk)
+    return LzDims(B, H, T, dk, dv, chunk, w, M, io, float(scale), float(alpha))
+
+
+# --------------------------------------------------------------------------
+# C ABI mirrors (pointers from tensors, nothing else)
+# --------------------------------------------------------------------------
+def lz_workspace_bytes(dims: LzDims, which: int) -> int:
+    return int(load().lz_workspace_bytes(ctypes.byref(dims), which))
+
+
+def lz_timing_enable(on: bool):
+    load().lz_timing_enable(1 if on else 0)
+
+
+def lz_timing_read(max_records: int = 1 << 16):
+    """[(kernel name, milliseconds)] of the launches recorded since the last
+    read (waits for them to finish)."""
+    stride = 48
+    names = ctypes.create_string_buffer(stride * max_records)
+    ms = (ctypes.c_float * max_records)()
+    n = load().lz_timing_read(names, stride, ms, max_records)
+    out = []
+    for i in range(min(n, max_records)):
+        nm = names.raw[i * stride:(i + 1) * stride].split(b"\0", 1)[0].decode()
+        out.append((nm, float(ms[i])))
+    return out
+
+
+def lz_gla_fwd(dims, q, k, v, g, h0, o, hT, ws, ws_bytes, stream=None):
+    _check(load().lz_gla_fwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(h0),
+                             _ptr(o), _ptr(hT), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def lz_swa_meta_fwd(dims, q, k, v, meta_k, meta_v, o, lse, stream=None):
+    _check(load().lz_swa_meta_fwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(meta_k),
+                                  _ptr(meta_v), _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def lz_hybrid_fwd(dims, q, k, v, g, meta_k, meta_v, h0, o, hT, lse, o_swa, ws, ws_bytes,
+                  stream=None):
+    _check(load().lz_hybrid_fwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                _ptr(meta_k), _ptr(meta_v), _ptr(h0), _ptr(o), _ptr(hT),
+                                _ptr(lse), _ptr(o_swa), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def lz_gla_bwd(dims, q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, ws, ws_bytes, stream=None):
+    _check(load().lz_gla_bwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(h0),
+                             _ptr(dO), _ptr(dhT), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
+                             _ptr(dh0), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def lz_swa_meta_bwd(dims, q, k, v, meta_k, meta_v, lse, dO, dq, dk, dv, dmeta_k, dmeta_v, ws,
+                    ws_bytes, stream=None):
+    _check(load().lz_swa_meta_bwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(meta_k),
+                                  _ptr(meta_v), _ptr(lse), _ptr(dO), _ptr(dq), _ptr(dk),
+                                  _ptr(dv), _ptr(dmeta_k), _ptr(dmeta_v), _ptr(ws), ws_bytes,
+                                  _stream(stream)))
+
+
+def lz_hybrid_bwd(dims, q, k, v, g, meta_k, meta_v, h0, lse, dO, dhT, dq, dk, dv, dg, dh0,
+                  dmeta_k, dmeta_v, dalpha, ws, ws_bytes, stream=None):
+    _check(load().lz_hybrid_bwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                _ptr(meta_k), _ptr(meta_v), _ptr(h0), _ptr(lse), _ptr(dO),
+                                _ptr(dhT), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dh0),
+                                _ptr(dmeta_k), _ptr(dmeta_v), _ptr(dalpha), _ptr(ws), ws_bytes,
+                                _stream(stream)))
+
+
+def lz_gla_decode_step(Bd, H, dk, dv, w, M, io, scale, alpha, state, kring, vring, pos, q, k,
+                       v, g, meta_k, meta_v, o, stream=None):
+    _check(load().lz_gla_decode_step(Bd, H, dk, dv, w, M, io, float(scale), float(alpha),
+                                     _ptr(state), _ptr(kring), _ptr(vring), _ptr(pos), _ptr(q),
+                                     _ptr(k), _ptr(v), _ptr(g), _ptr(meta_k), _ptr(meta_v),
+                                     _ptr(o), _stream(stream)))
+
+
+# --------------------------------------------------------------------------
+# Allocating helpers (torch owns memory; the library computes)
+# --------------------------------------------------------------------------
+def _dims_from(q, v, *, chunk, w, M, scale, alpha):
+    B, H, T, dk = q.shape
+    return make_dims(B, H, T, dk, v.shape[-1], chunk=chunk, w=w, M=M, io=io_of(q.dtype),
+                     scale=scale, alpha=alpha)
+
+
+def _ws(dims, which, device):
+    n = lz_workspace_bytes(dims, which)
+    return (torch.empty(max(n, 1), dtype=torch.uint8, device=device), n)
+
+
+def _M(meta_k):
+    return 0 if meta_k is None else int(meta_k.shape[1])
+
+
+def gla_fwd(q, k, v, g, h0=None, *, chunk=64, want_hT=False, stream=None):
+    d = _dims_from(q, v, chunk=chunk, w=1, M=0, scale=None, alpha=0.0)
+    o = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=q.device)
+    hT = torch.empty(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], dtype=torch.float32,
+                     device=q.device) if want_hT else None
+    ws, n = _ws(d, LZ_WS_GLA_FWD, q.device)
+    lz_gla_fwd(d, q, k, v, g, h0, o, hT, ws, n, stream)
+    return o, hT
+
+
+def swa_meta_fwd(q, k, v, meta_k, meta_v, *, w, scale=None, want_lse=True, stream=None):
+    d = _dims_from(q, v, chunk=64, w=w, M=_M(meta_k), scale=scale, alpha=1.0)
+    o = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=q.device)
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device) if want_lse else None
+    lz_swa_meta_fwd(d, q, k, v, meta_k, meta_v, o, lse, stream)
+    return o, lse
+
+
+def hybrid_fwd(q, k, v, g, meta_k, meta_v, *, w, alpha, scale=None, chunk=64, h0=None,
+               want_hT=False, want_lse=False, want_o_swa=False, stream=None):
+    d = _dims_from(q, v, chunk=chunk, w=w, M=_M(meta_k), scale=scale, alpha=alpha)
+    dev = q.device
+    o = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=dev)
+    hT = torch.empty(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], dtype=torch.float32,
+                     device=dev) if want_hT else None
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=dev) if want_lse else None
+    osw = torch.empty_like(o) if want_o_swa else None
+    ws, n = _ws(d, LZ_WS_HYBRID_FWD, dev)
+    lz_hybrid_fwd(d, q, k, v, g, meta_k, meta_v, h0, o, hT, lse, osw, ws, n, stream)
+    return {"o": o, "hT": hT, "lse": lse, "o_swa": osw}
+
+
+def gla_bwd(q, k, v, g, dO, h0=None, dhT=None, *, chunk=64, want_dh0=False, stream=None):
+    d = _dims_from(q, v, chunk=chunk, w=1, M=0, scale=None, alpha=0.0)
+    dev = q.device
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dg = torch.empty_like(g)
+    dh0 = torch.empty(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], dtype=torch.float32,
+                      device=dev) if want_dh0 else None
+    ws, n = _ws(d, LZ_WS_GLA_BWD, dev)
+    lz_gla_bwd(d, q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, ws, n, stream)
+    return {"dq": dq, "dk": dk, "dv": dv, "dg": dg, "dh0": dh0}
+
+
+def swa_meta_bwd(q, k, v, meta_k, meta_v, lse, dO, *, w, scale=None, stream=None):
+    M = _M(meta_k)
+    d = _dims_from(q, v, chunk=64, w=w, M=M, scale=scale, alpha=1.0)
+    dev = q.device
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dmk = torch.empty(q.shape[1], M, q.shape[-1], dtype=torch.float32, device=dev) if M else None
+    dmv = torch.empty(q.shape[1], M, v.shape[-1], dtype=torch.float32, device=dev) \
+        if (M and meta_v is not None) else None
+    ws, n = _ws(d, LZ_WS_SWA_BWD, dev)
+    lz_swa_meta_bwd(d, q, k, v, meta_k, meta_v, lse, dO, dq, dk, dv, dmk, dmv, ws, n, stream)
+    return {"dq": dq, "dk": dk, "dv": dv, "dmeta_k": dmk, "dmeta_v": dmv}
+
+
+def hybrid_bwd(q, k, v, g, meta_k, meta_v, lse, dO, *, w, alpha, scale=None, chunk=64,
+               h0=None, dhT=None, want_dh0=False, stream=None):
+    M = _M(meta_k)
+    d = _dims_from(q, v, chunk=chunk, w=w, M=M, scale=scale, alpha=alpha)
+    dev = q.device
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dg = torch.empty_like(g)
+    dh0 = torch.empty(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], dtype=torch.float32,
+                      device=dev) if want_dh0 else None
+    dmk = torch.empty(q.shape[1], M, q.shape[-1], dtype=torch.float32, device=dev) if M else None
+    dmv = torch.empty(q.shape[1], M, v.shape[-1], dtype=torch.float32, device=dev) \
+        if (M and meta_v is not None) else None
+    dalpha = torch.empty(4, dtype=torch.float32, device=dev)
+    ws, n = _ws(d, LZ_WS_HYBRID_BWD, dev)
+    lz_hybrid_bwd(d, q, k, v, g, meta_k, meta_v, h0, lse, dO, dhT, dq, dk, dv, dg, dh0, dmk,
+                  dmv, dalpha, ws, n, stream)
+    return {"dq": dq, "dk": dk, "dv": dv, "dg": dg, "dh0": dh0, "dmeta_k": dmk,
+            "dmeta_v": dmv, "dalpha": dalpha[:1]}
+
+
+def decode_step(state, kring, vring, pos, q, k, v, g, meta_k, meta_v, *, alpha, scale=None,
+                o=None, stream=None):
+    """One in-place generation step; returns o [Bd, H, dv]."""
+    Bd, H, dk = q.shape
+    dv = v.shape[-1]
+    w = kring.shape[2]
+    M = _M(meta_k)
+    if scale is None:
+        scale = 1.0 / math.sqrt(dk)
+    if o is None:
+        o = torch.empty(Bd, H, dv, dtype=q.dtype, device=q.device)
+    lz_gla_decode_step(Bd, H, dk, dv, w, M, io_of(q.dtype), scale, alpha, state, kring, vring,
+                       pos, q, k, v, g, meta_k, meta_v, o, stream)
+    return o

@@ -1,0 +1,126 @@
+// Internal launch interface between the C ABI (lizard_api.cu) and the
+// kernels.  Not part of the public header.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace lz {
+
+// Brackets one kernel launch with CUDA events when lz_timing_enable(1) is in
+// effect on the calling thread (see timing.cu); a no-op otherwise.
+class ScopedTiming {
+ public:
+  ScopedTiming(const char* name, cudaStream_t s);
+  ~ScopedTiming();
+  ScopedTiming(const ScopedTiming&) = delete;
+  ScopedTiming& operator=(const ScopedTiming&) = delete;
+
+ private:
+  cudaStream_t s_;
+  bool on_;
+  const char* name_ = nullptr;
+  cudaEvent_t a_ = nullptr, b_ = nullptr;
+};
+
+// ---- gated branch, SIMT path (fp32 arithmetic; fp32 or bf16 I/O) ----------
+struct GlaFwdParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g;
+  const float* h0;     // nullable
+  void* o;             // nullable: skip outputs (state pass only)
+  float* hT;           // nullable
+  float* states;       // nullable: [BH][nchunks][dk][dv] state before each chunk
+  const float* add;    // nullable: fp32 [B,H,T,dv], o += alpha * add
+  float alpha;
+  int B, H, T, dk, dv;
+};
+constexpr int kSimtChunk = 16;
+cudaError_t launch_gla_fwd_simt(const GlaFwdParams& p, bool bf16, cudaStream_t s);
+
+struct GlaBwdParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g;
+  const void* dO;
+  const float* dhT;      // nullable
+  const float* states;   // [BH][nchunks][dk][dv] from the state pass
+  const float* hT;       // [BH][dk][dv] final state (read only when dhT != NULL)
+  const float* add_dq;   // nullable fp32 [B,H,T,dk] added before the store
+  const float* add_dk;   // nullable
+  const float* add_dv;   // nullable fp32 [B,H,T,dv]
+  void* dq;
+  void* dk;
+  void* dv;
+  float* dg;
+  float* dh0;            // nullable
+  int B, H, T, dkd, dvd;
+};
+cudaError_t launch_gla_bwd_simt(const GlaBwdParams& p, bool bf16, cudaStream_t s);
+
+// ---- window + meta softmax, SIMT path ------------------------------------
+struct SwaFwdParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* mk;   // [H,M,dk] (nullable when M == 0)
+  const void* mv;   // nullable = sink-only
+  void* o;          // nullable, io dtype
+  float* o_f32;     // nullable, fp32
+  float* lse;       // nullable
+  int B, H, T, dk, dv, w, M;
+  float scale;
+};
+cudaError_t launch_swa_fwd_simt(const SwaFwdParams& p, bool bf16, cudaStream_t s);
+
+struct SwaBwdParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* mk;
+  const void* mv;
+  const float* lse;
+  const void* dO;
+  float gscale;      // the window branch sees gscale * dO
+  void* dq;          // io dtype outputs (nullable when the f32 ones are used)
+  void* dk;
+  void* dv;
+  float* dq_f32;     // nullable fp32 outputs
+  float* dk_f32;
+  float* dv_f32;
+  float* Dbuf;       // [B*H*T] scratch: dO_t . o_swa_t (unscaled)
+  float* alpha_part; // [n_qblocks] scratch: per-block sums of Dbuf
+  float* meta_part;  // [n_meta_parts][H][M][dk+dv] scratch
+  float* dmk;        // nullable [H,M,dk]
+  float* dmv;        // nullable [H,M,dv]
+  float* dalpha;     // nullable [1]
+  int B, H, T, dkd, dvd, w, M;
+  float scale;
+};
+int swa_bwd_n_qblocks(int B, int H, int T);
+int swa_bwd_n_meta_parts(int B, int T);
+cudaError_t launch_swa_bwd_simt(const SwaBwdParams& p, bool bf16, cudaStream_t s);
+
+// ---- decode --------------------------------------------------------------
+struct DecodeParams {
+  int Bd, H, w, M;
+  float scale, alpha;
+  float* state;
+  void* kring;
+  void* vring;
+  int64_t* pos;
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* g;
+  const void* mk;
+  const void* mv;
+  void* o;
+};
+cudaError_t launch_decode(const DecodeParams& p, bool bf16, cudaStream_t s);
+
+}  // namespace lz

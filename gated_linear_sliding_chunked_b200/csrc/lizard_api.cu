@@ -1,0 +1,397 @@
+// C ABI of the hybrid attention library: argument validation, workspace
+// layout and kernel launches.  Every entry point validates on the host and
+// returns before any launch when an argument is bad; kernels never trap.
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "../../include/lizard.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+lz_status fail(lz_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return st;
+}
+
+lz_status ok() {
+  g_err.clear();
+  return LZ_OK;
+}
+
+lz_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return ok();
+  return fail(LZ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr size_t kAlign = 256;
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Carves consecutive 256-byte aligned regions out of the caller's scratch.
+struct Carver {
+  char* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <typename T>
+  T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += round_up(count * sizeof(T));
+    return p;
+  }
+};
+
+#define LZ_REQUIRE(cond, ...)                                  \
+  do {                                                         \
+    if (!(cond)) return fail(LZ_ERR_INVALID_ARG, __VA_ARGS__); \
+  } while (0)
+
+lz_status check_ptr(const void* p, const char* name, bool required) {
+  if (!p) {
+    if (required) return fail(LZ_ERR_INVALID_ARG, "%s must not be NULL", name);
+    return LZ_OK;
+  }
+  if (!aligned16(p)) return fail(LZ_ERR_INVALID_ARG, "%s must be 16-byte aligned", name);
+  return LZ_OK;
+}
+
+#define LZ_PTR(p, req)                                   \
+  do {                                                   \
+    lz_status _s = check_ptr((p), #p, (req));            \
+    if (_s != LZ_OK) return _s;                          \
+  } while (0)
+
+// Shape checks shared by the prefill/training entry points.
+lz_status check_dims(const lz_dims* d, bool need_window) {
+  LZ_REQUIRE(d != nullptr, "dims must not be NULL");
+  LZ_REQUIRE(d->B >= 0 && d->H >= 0 && d->T >= 0, "B, H, T must be >= 0 (got %d, %d, %d)",
+             d->B, d->H, d->T);
+  if (d->io != LZ_F32 && d->io != LZ_BF16)
+    return fail(LZ_ERR_UNSUPPORTED, "io dtype %d is not LZ_F32 or LZ_BF16", (int)d->io);
+  if ((d->dk != 64 && d->dk != 128) || (d->dv != 64 && d->dv != 128))
+    return fail(LZ_ERR_UNSUPPORTED, "dk, dv must be 64 or 128 (got %d, %d)", d->dk, d->dv);
+  if (d->chunk != 64 && d->chunk != 128)
+    return fail(LZ_ERR_UNSUPPORTED, "chunk must be 64 or 128 (got %d)", d->chunk);
+  if (need_window) {
+    if (d->w < 1 || d->w > 1024)
+      return fail(LZ_ERR_UNSUPPORTED, "window w must be in [1, 1024] (got %d)", d->w);
+    if (d->M < 0 || d->M > 16)
+      return fail(LZ_ERR_UNSUPPORTED, "meta tokens M must be in [0, 16] (got %d)", d->M);
+  }
+  const double elems = (double)d->B * d->H * d->T * (d->dk > d->dv ? d->dk : d->dv);
+  LZ_REQUIRE(elems < 9.0e15, "problem too large");
+  return LZ_OK;
+}
+
+size_t bht(const lz_dims* d) { return (size_t)d->B * d->H * d->T; }
+size_t nchunks16(const lz_dims* d) {
+  return (size_t)((d->T + lz::kSimtChunk - 1) / lz::kSimtChunk);
+}
+
+// ---- workspace layouts ----------------------------------------------------
+struct GlaBwdWs {
+  float* states;
+  float* hT;
+};
+GlaBwdWs carve_gla_bwd(Carver& c, const lz_dims* d) {
+  GlaBwdWs w;
+  const size_t bh = (size_t)d->B * d->H;
+  w.states = c.take<float>(bh * nchunks16(d) * d->dk * d->dv);
+  w.hT = c.take<float>(bh * d->dk * d->dv);
+  return w;
+}
+
+struct SwaBwdWs {
+  float* Dbuf;
+  float* alpha_part;
+  float* meta_part;
+};
+SwaBwdWs carve_swa_bwd(Carver& c, const lz_dims* d) {
+  SwaBwdWs w;
+  w.Dbuf = c.take<float>(bht(d));
+  w.alpha_part = c.take<float>((size_t)lz::swa_bwd_n_qblocks(d->B, d->H, d->T) + 1);
+  w.meta_part = c.take<float>((size_t)lz::swa_bwd_n_meta_parts(d->B, d->T) * d->H * d->M *
+                              (d->dk + d->dv) + 1);
+  return w;
+}
+
+struct HybridBwdWs {
+  SwaBwdWs swa;
+  GlaBwdWs gla;
+  float* dq;
+  float* dk;
+  float* dv;
+};
+HybridBwdWs carve_hybrid_bwd(Carver& c, const lz_dims* d) {
+  HybridBwdWs w;
+  w.swa = carve_swa_bwd(c, d);
+  w.gla = carve_gla_bwd(c, d);
+  w.dq = c.take<float>(bht(d) * d->dk);
+  w.dk = c.take<float>(bht(d) * d->dk);
+  w.dv = c.take<float>(bht(d) * d->dv);
+  return w;
+}
+
+size_t ws_bytes(const lz_dims* d, int which) {
+  Carver c(nullptr);
+  switch (which) {
+    case LZ_WS_GLA_FWD:
+      return 0;
+    case LZ_WS_HYBRID_FWD:
+      c.take<float>(bht(d) * d->dv);
+      return c.off;
+    case LZ_WS_GLA_BWD:
+      carve_gla_bwd(c, d);
+      return c.off;
+    case LZ_WS_SWA_BWD:
+      carve_swa_bwd(c, d);
+      return c.off;
+    case LZ_WS_HYBRID_BWD:
+      carve_hybrid_bwd(c, d);
+      return c.off;
+    default:
+      return 0;
+  }
+}
+
+lz_status check_ws(const lz_dims* d, int which, const void* ws, size_t have) {
+  const size_t need = ws_bytes(d, which);
+  if (need == 0) return LZ_OK;
+  LZ_REQUIRE(ws != nullptr, "workspace must not be NULL (%zu bytes needed)", need);
+  LZ_REQUIRE(aligned16(ws), "workspace must be 16-byte aligned");
+  LZ_REQUIRE(have >= need, "workspace too small: %zu bytes given, %zu needed", have, need);
+  return LZ_OK;
+}
+
+cudaStream_t as_stream(lz_stream s) { return reinterpret_cast<cudaStream_t>(s); }
+
+lz::SwaFwdParams swa_fwd_params(const lz_dims* d, const void* q, const void* k, const void* v,
+                                const void* mk, const void* mv) {
+  lz::SwaFwdParams p{};
+  p.q = q; p.k = k; p.v = v; p.mk = mk; p.mv = d->M > 0 ? mv : nullptr;
+  p.B = d->B; p.H = d->H; p.T = d->T; p.dk = d->dk; p.dv = d->dv; p.w = d->w; p.M = d->M;
+  p.scale = d->scale;
+  return p;
+}
+
+lz::GlaFwdParams gla_fwd_params(const lz_dims* d, const void* q, const void* k, const void* v,
+                                const float* g, const float* h0) {
+  lz::GlaFwdParams p{};
+  p.q = q; p.k = k; p.v = v; p.g = g; p.h0 = h0;
+  p.B = d->B; p.H = d->H; p.T = d->T; p.dk = d->dk; p.dv = d->dv;
+  return p;
+}
+
+lz::SwaBwdParams swa_bwd_params(const lz_dims* d, const void* q, const void* k, const void* v,
+                                const void* mk, const void* mv, const float* lse,
+                                const void* dO, const SwaBwdWs& w) {
+  lz::SwaBwdParams p{};
+  p.q = q; p.k = k; p.v = v; p.mk = mk; p.mv = d->M > 0 ? mv : nullptr; p.lse = lse; p.dO = dO;
+  p.Dbuf = w.Dbuf; p.alpha_part = w.alpha_part; p.meta_part = w.meta_part;
+  p.B = d->B; p.H = d->H; p.T = d->T; p.dkd = d->dk; p.dvd = d->dv; p.w = d->w; p.M = d->M;
+  p.scale = d->scale;
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lz_last_error(void) { return g_err.c_str(); }
+
+const char* lz_version(void) { return "lizard-b200 0.1 (sm_100a)"; }
+
+size_t lz_workspace_bytes(const lz_dims* d, int which) {
+  if (check_dims(d, which != LZ_WS_GLA_FWD && which != LZ_WS_GLA_BWD) != LZ_OK) return 0;
+  return ws_bytes(d, which);
+}
+
+lz_status lz_gla_fwd(const lz_dims* d, const void* q, const void* k, const void* v,
+                     const float* g, const float* h0, void* o, float* hT, void* ws,
+                     size_t ws_bytes_, lz_stream stream) {
+  lz_status st = check_dims(d, false);
+  if (st != LZ_OK) return st;
+  const bool nz = bht(d) > 0;  // empty tensors may have NULL data
+  LZ_PTR(q, nz); LZ_PTR(k, nz); LZ_PTR(v, nz); LZ_PTR(g, nz); LZ_PTR(o, nz);
+  LZ_PTR(h0, false); LZ_PTR(hT, false);
+  st = check_ws(d, LZ_WS_GLA_FWD, ws, ws_bytes_);
+  if (st != LZ_OK) return st;
+  lz::GlaFwdParams p = gla_fwd_params(d, q, k, v, g, h0);
+  p.o = o;
+  p.hT = hT;
+  return cuda_status(lz::launch_gla_fwd_simt(p, d->io == LZ_BF16, as_stream(stream)),
+                     "lz_gla_fwd");
+}
+
+lz_status lz_swa_meta_fwd(const lz_dims* d, const void* q, const void* k, const void* v,
+                          const void* meta_k, const void* meta_v, void* o, float* lse,
+                          lz_stream stream) {
+  lz_status st = check_dims(d, true);
+  if (st != LZ_OK) return st;
+  const bool nz = bht(d) > 0;  // empty tensors may have NULL data
+  LZ_PTR(q, nz); LZ_PTR(k, nz); LZ_PTR(v, nz); LZ_PTR(o, nz);
+  LZ_PTR(meta_k, d->M > 0 && d->H > 0); LZ_PTR(meta_v, false); LZ_PTR(lse, false);
+  lz::SwaFwdParams p = swa_fwd_params(d, q, k, v, meta_k, meta_v);
+  p.o = o;
+  p.lse = lse;
+  return cuda_status(lz::launch_swa_fwd_simt(p, d->io == LZ_BF16, as_stream(stream)),
+                     "lz_swa_meta_fwd");
+}
+
+lz_status lz_hybrid_fwd(const lz_dims* d, const void* q, const void* k, const void* v,
+                        const float* g, const void* meta_k, const void* meta_v,
+                        const float* h0, void* o, float* hT, float* lse, void* o_swa,
+                        void* ws, size_t ws_bytes_, lz_stream stream) {
+  lz_status st = check_dims(d, true);
+  if (st != LZ_OK) return st;
+  const bool nz = bht(d) > 0;  // empty tensors may have NULL data
+  LZ_PTR(q, nz); LZ_PTR(k, nz); LZ_PTR(v, nz); LZ_PTR(g, nz); LZ_PTR(o, nz);
+  LZ_PTR(meta_k, d->M > 0 && d->H > 0); LZ_PTR(meta_v, false); LZ_PTR(h0, false); LZ_PTR(hT, false);
+  LZ_PTR(lse, false); LZ_PTR(o_swa, false);
+  st = check_ws(d, LZ_WS_HYBRID_FWD, ws, ws_bytes_);
+  if (st != LZ_OK) return st;
+  const cudaStream_t s = as_stream(stream);
+  const bool bf = d->io == LZ_BF16;
+  Carver c(ws);
+  float* osw = c.take<float>(bht(d) * d->dv);
+  lz::SwaFwdParams sp = swa_fwd_params(d, q, k, v, meta_k, meta_v);
+  sp.o = o_swa;
+  sp.o_f32 = osw;
+  sp.lse = lse;
+  cudaError_t e = lz::launch_swa_fwd_simt(sp, bf, s);
+  if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_fwd (window branch)");
+  lz::GlaFwdParams gp = gla_fwd_params(d, q, k, v, g, h0);
+  gp.o = o;
+  gp.hT = hT;
+  gp.add = osw;
+  gp.alpha = d->alpha;
+  return cuda_status(lz::launch_gla_fwd_simt(gp, bf, s), "lz_hybrid_fwd (gated branch)");
+}
+
+static cudaError_t gla_bwd_launch(const lz_dims* d, const void* q, const void* k, const void* v,
+                                  const float* g, const float* h0, const void* dO,
+                                  const float* dhT, void* dq, void* dk, void* dv, float* dg,
+                                  float* dh0, const GlaBwdWs& w, const float* add_dq,
+                                  const float* add_dk, const float* add_dv, cudaStream_t s) {
+  const bool bf = d->io == LZ_BF16;
+  lz::GlaFwdParams fp = gla_fwd_params(d, q, k, v, g, h0);
+  fp.states = w.states;
+  fp.hT = w.hT;
+  cudaError_t e = lz::launch_gla_fwd_simt(fp, bf, s);
+  if (e != cudaSuccess) return e;
+  lz::GlaBwdParams p{};
+  p.q = q; p.k = k; p.v = v; p.g = g; p.dO = dO; p.dhT = dhT;
+  p.states = w.states; p.hT = w.hT;
+  p.add_dq = add_dq; p.add_dk = add_dk; p.add_dv = add_dv;
+  p.dq = dq; p.dk = dk; p.dv = dv; p.dg = dg; p.dh0 = dh0;
+  p.B = d->B; p.H = d->H; p.T = d->T; p.dkd = d->dk; p.dvd = d->dv;
+  return lz::launch_gla_bwd_simt(p, bf, s);
+}
+
+lz_status lz_gla_bwd(const lz_dims* d, const void* q, const void* k, const void* v,
+                     const float* g, const float* h0, const void* dO, const float* dhT,
+                     void* dq, void* dk, void* dv, float* dg, float* dh0, void* ws,
+                     size_t ws_bytes_, lz_stream stream) {
+  lz_status st = check_dims(d, false);
+  if (st != LZ_OK) return st;
+  const bool nz = bht(d) > 0;  // empty tensors may have NULL data
+  LZ_PTR(q, nz); LZ_PTR(k, nz); LZ_PTR(v, nz); LZ_PTR(g, nz); LZ_PTR(dO, nz);
+  LZ_PTR(dq, nz); LZ_PTR(dk, nz); LZ_PTR(dv, nz); LZ_PTR(dg, nz);
+  LZ_PTR(h0, false); LZ_PTR(dhT, false); LZ_PTR(dh0, false);
+  st = check_ws(d, LZ_WS_GLA_BWD, ws, ws_bytes_);
+  if (st != LZ_OK) return st;
+  Carver c(ws);
+  GlaBwdWs w = carve_gla_bwd(c, d);
+  return cuda_status(gla_bwd_launch(d, q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, w,
+                                    nullptr, nullptr, nullptr, as_stream(stream)),
+                     "lz_gla_bwd");
+}
+
+lz_status lz_swa_meta_bwd(const lz_dims* d, const void* q, const void* k, const void* v,
+                          const void* meta_k, const void* meta_v, const float* lse,
+                          const void* dO, void* dq, void* dk, void* dv, float* dmeta_k,
+                          float* dmeta_v, void* ws, size_t ws_bytes_, lz_stream stream) {
+  lz_status st = check_dims(d, true);
+  if (st != LZ_OK) return st;
+  const bool nz = bht(d) > 0;  // empty tensors may have NULL data
+  LZ_PTR(q, nz); LZ_PTR(k, nz); LZ_PTR(v, nz); LZ_PTR(lse, nz); LZ_PTR(dO, nz);
+  LZ_PTR(dq, nz); LZ_PTR(dk, nz); LZ_PTR(dv, nz);
+  LZ_PTR(meta_k, d->M > 0 && d->H > 0); LZ_PTR(meta_v, false);
+  LZ_PTR(dmeta_k, false); LZ_PTR(dmeta_v, false);
+  st = check_ws(d, LZ_WS_SWA_BWD, ws, ws_bytes_);
+  if (st != LZ_OK) return st;
+  Carver c(ws);
+  SwaBwdWs w = carve_swa_bwd(c, d);
+  lz::SwaBwdParams p = swa_bwd_params(d, q, k, v, meta_k, meta_v, lse, dO, w);
+  p.gscale = 1.f;
+  p.dq = dq; p.dk = dk; p.dv = dv;
+  p.dmk = dmeta_k; p.dmv = dmeta_v;
+  return cuda_status(lz::launch_swa_bwd_simt(p, d->io == LZ_BF16, as_stream(stream)),
+                     "lz_swa_meta_bwd");
+}
+
+lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const void* v,
+                        const float* g, const void* meta_k, const void* meta_v,
+                        const float* h0, const float* lse, const void* dO, const float* dhT,
+                        void* dq, void* dk, void* dv, float* dg, float* dh0, float* dmeta_k,
+                        float* dmeta_v, float* dalpha, void* ws, size_t ws_bytes_,
+                        lz_stream stream) {
+  lz_status st = check_dims(d, true);
+  if (st != LZ_OK) return st;
+  const bool nz = bht(d) > 0;  // empty tensors may have NULL data
+  LZ_PTR(q, nz); LZ_PTR(k, nz); LZ_PTR(v, nz); LZ_PTR(g, nz); LZ_PTR(lse, nz);
+  LZ_PTR(dO, nz); LZ_PTR(dq, nz); LZ_PTR(dk, nz); LZ_PTR(dv, nz); LZ_PTR(dg, nz);
+  LZ_PTR(meta_k, d->M > 0 && d->H > 0); LZ_PTR(meta_v, false); LZ_PTR(h0, false); LZ_PTR(dhT, false);
+  LZ_PTR(dh0, false); LZ_PTR(dmeta_k, false); LZ_PTR(dmeta_v, false);
+  if (dalpha && (reinterpret_cast<uintptr_t>(dalpha) & 3u))
+    return fail(LZ_ERR_INVALID_ARG, "dalpha must be 4-byte aligned");
+  st = check_ws(d, LZ_WS_HYBRID_BWD, ws, ws_bytes_);
+  if (st != LZ_OK) return st;
+  const cudaStream_t s = as_stream(stream);
+  Carver c(ws);
+  HybridBwdWs w = carve_hybrid_bwd(c, d);
+  lz::SwaBwdParams p = swa_bwd_params(d, q, k, v, meta_k, meta_v, lse, dO, w.swa);
+  p.gscale = d->alpha;
+  p.dq_f32 = w.dq; p.dk_f32 = w.dk; p.dv_f32 = w.dv;
+  p.dmk = dmeta_k; p.dmv = dmeta_v; p.dalpha = dalpha;
+  cudaError_t e = lz::launch_swa_bwd_simt(p, d->io == LZ_BF16, s);
+  if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (window branch)");
+  return cuda_status(gla_bwd_launch(d, q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, w.gla,
+                                    w.dq, w.dk, w.dv, s),
+                     "lz_hybrid_bwd (gated branch)");
+}
+
+lz_status lz_gla_decode_step(int Bd, int H, int dk, int dv, int w, int M, lz_dtype io,
+                             float scale, float alpha, float* state, void* kring,
+                             void* vring, int64_t* pos, const void* q, const void* k,
+                             const void* v, const float* g, const void* meta_k,
+                             const void* meta_v, void* o, lz_stream stream) {
+  LZ_REQUIRE(Bd >= 0 && H >= 0, "Bd, H must be >= 0 (got %d, %d)", Bd, H);
+  if (io != LZ_F32 && io != LZ_BF16)
+    return fail(LZ_ERR_UNSUPPORTED, "io dtype %d is not LZ_F32 or LZ_BF16", (int)io);
+  if (dk != 128 || dv != 128)
+    return fail(LZ_ERR_UNSUPPORTED, "decode supports dk = dv = 128 (got %d, %d)", dk, dv);
+  if (w < 1 || w > 1024) return fail(LZ_ERR_UNSUPPORTED, "w must be in [1, 1024] (got %d)", w);
+  if (M < 0 || M > 16) return fail(LZ_ERR_UNSUPPORTED, "M must be in [0, 16] (got %d)", M);
+  const bool nz = (size_t)Bd * H > 0;  // empty tensors may have NULL data
+  LZ_PTR(state, nz); LZ_PTR(kring, nz); LZ_PTR(vring, nz); LZ_PTR(pos, Bd > 0);
+  LZ_PTR(q, nz); LZ_PTR(k, nz); LZ_PTR(v, nz); LZ_PTR(g, nz); LZ_PTR(o, nz);
+  LZ_PTR(meta_k, M > 0 && H > 0); LZ_PTR(meta_v, false);
+  lz::DecodeParams p{};
+  p.Bd = Bd; p.H = H; p.w = w; p.M = M; p.scale = scale; p.alpha = alpha;
+  p.state = state; p.kring = kring; p.vring = vring; p.pos = pos;
+  p.q = q; p.k = k; p.v = v; p.g = g; p.mk = meta_k; p.mv = M > 0 ? meta_v : nullptr; p.o = o;
+  return cuda_status(lz::launch_decode(p, io == LZ_BF16, as_stream(stream)),
+                     "lz_gla_decode_step");
+}
+
+}  // extern "C"

@@ -1,0 +1,182 @@
+/*
+ * lizard.h -- C ABI of the B200 (sm_100a) hybrid attention library.
+ *
+ * The operator is the hybrid attention of "Lizard: An Efficient Linearization
+ * Framework for Large Language Models" (gist.science technical summary,
+ * section 2a "hybrid attention architecture"):
+ *
+ *   gated linear attention   S_t = diag(exp(g_t)) S_{t-1} + k_t v_t^T,
+ *                            o_gla_t = q_t^T S_t            (state update eq.)
+ *   anchor window softmax    o_swa_t = softmax over keys j in [t-w+1, t] plus
+ *                            M learnable meta tokens that sit in the
+ *                            denominator as attention sinks
+ *   output                   o_t = o_gla_t + alpha * o_swa_t  (weighted sum)
+ *
+ * and the gradient needed by its first training stage (section 2b), plus the
+ * constant-memory generation step that the fixed-size state allows.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every pointer is DEVICE memory owned by the caller.  The library never
+ *   allocates, frees or synchronizes; every call is asynchronous on `stream`
+ *   (a cudaStream_t passed as void*; NULL means the legacy default stream).
+ * - Layouts are contiguous row-major:
+ *     q, k, g, dq, dk, dg     [B, H, T, dk]
+ *     v, o, o_swa, dO, dv     [B, H, T, dv]
+ *     h0, hT, dh0, dhT        [B, H, dk, dv]   (fp32)
+ *     lse                     [B, H, T]        (fp32, natural log)
+ *     meta_k, dmeta_k         [H, M, dk]
+ *     meta_v, dmeta_v         [H, M, dv]
+ *   q, k, v, o, o_swa, meta_k, meta_v, dO, dq, dk, dv use the I/O dtype
+ *   `io`; the log-gates g, states, lse and every meta gradient are fp32.
+ * - g holds log-gates (g <= 0; gate = exp(g) in (0, 1]).  g > 0 is not
+ *   checked: it is a precondition, and NaN/Inf propagate.
+ * - Every pointer must be 16-byte aligned.  Supported: dk, dv in {64, 128};
+ *   chunk in {64, 128} (a tiling choice: results agree up to rounding);
+ *   1 <= w <= 1024; 0 <= M <= 16; T >= 0 (no multiple-of-anything rule).
+ * - Inputs must not alias outputs (the decode state/rings/pos are the
+ *   in-place exceptions).  Gradients are written, not accumulated.
+ * - On a bad argument the call returns LZ_ERR_INVALID_ARG or
+ *   LZ_ERR_UNSUPPORTED before launching anything; a failed launch returns
+ *   LZ_ERR_CUDA.  lz_last_error() then describes the failure (thread-local).
+ *   Kernels never trap.
+ */
+#ifndef LIZARD_H
+#define LIZARD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LZ_OK = 0,
+  LZ_ERR_INVALID_ARG = 1,  /* NULL / misaligned pointer, bad size, short workspace */
+  LZ_ERR_UNSUPPORTED = 2,  /* valid but outside the supported shapes/dtypes */
+  LZ_ERR_CUDA = 3,         /* a kernel launch or CUDA runtime call failed */
+  LZ_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up */
+} lz_status;
+
+typedef enum { LZ_F32 = 0, LZ_BF16 = 1 } lz_dtype;
+
+typedef void* lz_stream; /* cudaStream_t */
+
+/* Problem description shared by the prefill/training entry points. */
+typedef struct {
+  int B, H, T;    /* batch, heads, sequence length */
+  int dk, dv;     /* key and value head dims */
+  int chunk;      /* chunk length of the gated branch (64 or 128) */
+  int w;          /* window: keys t-w+1 .. t (w keys, the current one included) */
+  int M;          /* number of meta-memory tokens (0 = none) */
+  lz_dtype io;    /* dtype of q, k, v, o, meta, dO, dq, dk, dv */
+  float scale;    /* softmax logit scale (usually 1/sqrt(dk)); meta logits too */
+  float alpha;    /* weight of the window branch in the hybrid sum */
+} lz_dims;
+
+/* Bytes of scratch the call needs (0 is possible); `which` is one of the
+ * LZ_WS_* values.  The scratch is caller-owned device memory, 256-byte
+ * aligned, and may be reused once the call's stream work has finished. */
+enum { LZ_WS_GLA_FWD = 0, LZ_WS_HYBRID_FWD = 1, LZ_WS_GLA_BWD = 2,
+       LZ_WS_SWA_BWD = 3, LZ_WS_HYBRID_BWD = 4 };
+size_t lz_workspace_bytes(const lz_dims* d, int which);
+
+/* Gated linear attention forward (section 2a, state update equation).
+ *   o = q^T S_t per token; h0 (nullable = zeros) is the state before token 0;
+ *   hT (nullable) receives the state after the last token.  Fields used: B,
+ *   H, T, dk, dv, chunk, io. */
+lz_status lz_gla_fwd(const lz_dims* d, const void* q, const void* k,
+                     const void* v, const float* g, const float* h0, void* o,
+                     float* hT, void* ws, size_t ws_bytes, lz_stream stream);
+
+/* Sliding-window softmax with meta-memory sinks (section 2a, anchor window
+ * attention).  meta_k may be NULL only when M == 0.  meta_v == NULL selects
+ * the sink-only reading (meta tokens enter the denominator only).  o gets
+ * o_swa; lse (nullable) gets log(sum of exp(logits)) per query, which the
+ * backward needs.  Fields used: B, H, T, dk, dv, w, M, io, scale. */
+lz_status lz_swa_meta_fwd(const lz_dims* d, const void* q, const void* k,
+                          const void* v, const void* meta_k,
+                          const void* meta_v, void* o, float* lse,
+                          lz_stream stream);
+
+/* Hybrid forward o = o_gla + alpha * o_swa (section 2a, final output).
+ *   hT, lse, o_swa are nullable extra outputs (lse and o_swa are what
+ *   lz_hybrid_bwd needs).  All lz_dims fields are used. */
+lz_status lz_hybrid_fwd(const lz_dims* d, const void* q, const void* k,
+                        const void* v, const float* g, const void* meta_k,
+                        const void* meta_v, const float* h0, void* o,
+                        float* hT, float* lse, void* o_swa, void* ws,
+                        size_t ws_bytes, lz_stream stream);
+
+/* Gradient of lz_gla_fwd (needed by the attention-distillation stage,
+ * section 2b).  dO = dL/do; dhT (nullable) = dL/dhT.  Writes dq, dk, dv (io
+ * dtype), dg (fp32) and dh0 (nullable, fp32).  h0 may be NULL (zeros). */
+lz_status lz_gla_bwd(const lz_dims* d, const void* q, const void* k,
+                     const void* v, const float* g, const float* h0,
+                     const void* dO, const float* dhT, void* dq, void* dk,
+                     void* dv, float* dg, float* dh0, void* ws,
+                     size_t ws_bytes, lz_stream stream);
+
+/* Gradient of lz_swa_meta_fwd.  dO = dL/d(o_swa); lse from the forward.
+ * Writes dq, dk, dv (io dtype) and, when M > 0, dmeta_k (fp32, summed over
+ * batch and sequence) and dmeta_v (fp32; ignored in sink-only mode). */
+lz_status lz_swa_meta_bwd(const lz_dims* d, const void* q, const void* k,
+                          const void* v, const void* meta_k,
+                          const void* meta_v, const float* lse,
+                          const void* dO, void* dq, void* dk, void* dv,
+                          float* dmeta_k, float* dmeta_v, void* ws,
+                          size_t ws_bytes, lz_stream stream);
+
+/* Gradient of lz_hybrid_fwd in one call: the gated branch sees dO, the
+ * window branch alpha * dO.  lse from the forward.  dalpha (nullable, one
+ * fp32) receives sum over (b,h,t) of dO_t . o_swa_t. */
+lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k,
+                        const void* v, const float* g, const void* meta_k,
+                        const void* meta_v, const float* h0, const float* lse,
+                        const void* dO, const float* dhT, void* dq, void* dk,
+                        void* dv, float* dg, float* dh0, float* dmeta_k,
+                        float* dmeta_v, float* dalpha, void* ws,
+                        size_t ws_bytes, lz_stream stream);
+
+/* One constant-memory generation step for Bd sequences (section 2a: the
+ * fixed-size state replaces the growing KV cache), all in place:
+ *   state [Bd,H,dk,dv] fp32; kring [Bd,H,w,dk], vring [Bd,H,w,dv] (io
+ *   dtype); pos [Bd] int64 = tokens seen so far per sequence.
+ * Per sequence with p = pos[b]: k, v go to ring slot p mod w; the state is
+ * decayed by exp(g) and gets k v^T; o_gla = q^T S; the window is the last
+ * min(p+1, w) tokens (the new one included) plus the M meta tokens; o =
+ * o_gla + alpha * o_swa; pos[b] = p + 1.
+ *   q, k [Bd,H,dk], v, o [Bd,H,dv] io dtype; g [Bd,H,dk] fp32.  meta_v NULL
+ *   = sink-only.  Supported: dk = dv = 128, io = LZ_BF16 or LZ_F32. */
+lz_status lz_gla_decode_step(int Bd, int H, int dk, int dv, int w, int M,
+                             lz_dtype io, float scale, float alpha,
+                             float* state, void* kring, void* vring,
+                             int64_t* pos, const void* q, const void* k,
+                             const void* v, const float* g,
+                             const void* meta_k, const void* meta_v, void* o,
+                             lz_stream stream);
+
+/* Per-launch device timing for benchmarks (no counterpart on the pages; a
+ * measurement aid).  lz_timing_enable(1) makes every later kernel launch of
+ * this library from the calling host thread record a pair of CUDA events
+ * around itself on its own stream; lz_timing_enable(0) stops it (the
+ * default).  lz_timing_read waits for the recorded launches, writes up to
+ * max_records kernel names (NUL-terminated, name_stride bytes apart; names
+ * may be NULL) and elapsed milliseconds (ms may be NULL), clears the record
+ * and returns how many launches were recorded.  Both return 0 / a count and
+ * never fail. */
+int lz_timing_enable(int on);
+int lz_timing_read(char* names, size_t name_stride, float* ms, int max_records);
+
+/* Thread-local description of the last non-OK status ("" if none). */
+const char* lz_last_error(void);
+
+/* Library version string. */
+const char* lz_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIZARD_H */

@@ -1,0 +1,144 @@
+"""The C-ABI library loads, exports every entry point include/lizard.h
+declares, and rejects bad arguments on the host before any launch.  No
+compute call is made (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_linear_sliding_chunked_b200 as L
+from gated_linear_sliding_chunked_b200 import build as lbuild
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "lizard.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lz_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    lbuild.build()
+    return L.load()
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("lz_gla_fwd", "lz_gla_bwd", "lz_swa_meta_fwd", "lz_hybrid_fwd",
+              "lz_gla_decode_step", "lz_swa_meta_bwd", "lz_hybrid_bwd", "lz_workspace_bytes",
+              "lz_last_error"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_version(lib):
+    assert b"sm_100a" in lib.lz_version()
+
+
+FAKE = 0x7F0000000000  # never dereferenced: validation fails first
+
+
+def _dims(**kw):
+    base = dict(B=1, H=2, T=64, dk=64, dv=64, chunk=64, w=8, M=2, io=L.LZ_BF16, scale=0.125,
+                alpha=0.5)
+    base.update(kw)
+    return L.LzDims(*[base[f] for f, _ in L.LzDims._fields_])
+
+
+def _call_hybrid(lib, d, **ptrs):
+    p = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, mk=FAKE, mv=FAKE, h0=None, o=FAKE, hT=None,
+             lse=None, osw=None, ws=FAKE)
+    p.update(ptrs)
+    return lib.lz_hybrid_fwd(ctypes.byref(d), p["q"], p["k"], p["v"], p["g"], p["mk"], p["mv"],
+                             p["h0"], p["o"], p["hT"], p["lse"], p["osw"], p["ws"],
+                             ptrs.get("ws_bytes", 1 << 40), 0)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=96), L.LZ_ERR_UNSUPPORTED),
+    (dict(dv=32), L.LZ_ERR_UNSUPPORTED),
+    (dict(chunk=48), L.LZ_ERR_UNSUPPORTED),
+    (dict(w=0), L.LZ_ERR_UNSUPPORTED),
+    (dict(w=1025), L.LZ_ERR_UNSUPPORTED),
+    (dict(M=17), L.LZ_ERR_UNSUPPORTED),
+    (dict(M=-1), L.LZ_ERR_UNSUPPORTED),
+    (dict(io=7), L.LZ_ERR_UNSUPPORTED),
+    (dict(T=-1), L.LZ_ERR_INVALID_ARG),
+    (dict(B=-2), L.LZ_ERR_INVALID_ARG),
+])
+def test_bad_shapes_rejected(lib, kw, status):
+    assert _call_hybrid(lib, _dims(**kw)) == status
+    assert lib.lz_last_error()
+
+
+@pytest.mark.parametrize("which", ["q", "k", "v", "g", "o", "mk"])
+def test_null_required_pointer_rejected(lib, which):
+    assert _call_hybrid(lib, _dims(), **{which: None}) == L.LZ_ERR_INVALID_ARG
+    assert b"NULL" in lib.lz_last_error()
+
+
+def test_meta_k_may_be_null_without_meta(lib):
+    # M == 0: meta_k NULL passes validation; the workspace check then fails
+    # because no workspace is given, still before any launch.
+    st = _call_hybrid(lib, _dims(M=0), mk=None, mv=None, ws=None)
+    assert st == L.LZ_ERR_INVALID_ARG and b"workspace" in lib.lz_last_error()
+
+
+@pytest.mark.parametrize("which", ["q", "v", "g", "o", "h0", "lse"])
+def test_misaligned_pointer_rejected(lib, which):
+    assert _call_hybrid(lib, _dims(), **{which: FAKE + 4}) == L.LZ_ERR_INVALID_ARG
+    assert b"aligned" in lib.lz_last_error()
+
+
+def test_short_workspace_rejected(lib):
+    d = _dims()
+    need = L.lz_workspace_bytes(d, L.LZ_WS_HYBRID_FWD)
+    assert need > 0
+    assert _call_hybrid(lib, d, ws_bytes=need - 1) == L.LZ_ERR_INVALID_ARG
+    assert b"too small" in lib.lz_last_error()
+
+
+def test_workspace_sizes_grow_with_problem(lib):
+    small = L.lz_workspace_bytes(_dims(T=64), L.LZ_WS_HYBRID_BWD)
+    big = L.lz_workspace_bytes(_dims(T=4096), L.LZ_WS_HYBRID_BWD)
+    assert 0 < small < big
+    assert L.lz_workspace_bytes(_dims(dk=96), L.LZ_WS_HYBRID_BWD) == 0
+
+
+def test_decode_validation(lib):
+    f = lib.lz_gla_decode_step
+    args = [FAKE] * 11
+    assert f(4, 2, 64, 128, 16, 2, L.LZ_BF16, 0.1, 0.5, *args, 0) == L.LZ_ERR_UNSUPPORTED
+    assert f(4, 2, 128, 128, 0, 2, L.LZ_BF16, 0.1, 0.5, *args, 0) == L.LZ_ERR_UNSUPPORTED
+    assert f(4, 2, 128, 128, 16, 17, L.LZ_BF16, 0.1, 0.5, *args, 0) == L.LZ_ERR_UNSUPPORTED
+    assert f(-1, 2, 128, 128, 16, 2, L.LZ_BF16, 0.1, 0.5, *args, 0) == L.LZ_ERR_INVALID_ARG
+    bad = list(args)
+    bad[0] = None  # state
+    assert f(4, 2, 128, 128, 16, 2, L.LZ_BF16, 0.1, 0.5, *bad, 0) == L.LZ_ERR_INVALID_ARG
+    bad = list(args)
+    bad[3] = FAKE + 8  # pos misaligned
+    assert f(4, 2, 128, 128, 16, 2, L.LZ_BF16, 0.1, 0.5, *bad, 0) == L.LZ_ERR_INVALID_ARG
+
+
+def test_backward_validation(lib):
+    d = _dims()
+    P = [FAKE] * 18
+    # lse is required by the hybrid backward
+    P2 = list(P)
+    P2[7] = None
+    assert lib.lz_hybrid_bwd(ctypes.byref(d), *P2, FAKE, 1 << 40, 0) == L.LZ_ERR_INVALID_ARG
+    # dalpha only needs 4-byte alignment, but not 2
+    P3 = list(P)
+    P3[17] = FAKE + 2
+    assert lib.lz_hybrid_bwd(ctypes.byref(d), *P3, FAKE, 1 << 40, 0) == L.LZ_ERR_INVALID_ARG
+    assert lib.lz_gla_bwd(ctypes.byref(_dims(dk=32)), *([FAKE] * 12), FAKE, 1 << 40, 0) == \
+        L.LZ_ERR_UNSUPPORTED

@@ -1,0 +1,131 @@
+"""Backward parity: every gradient of the CUDA library vs the fp64 oracle's
+hand-written backward (itself pinned to finite differences)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import gated_linear_sliding_chunked_b200 as L
+from gated_linear_sliding_chunked_b200 import inputs as I
+import oracle
+from parity_util import assert_close, np64, oracle_inputs, small_problem
+
+pytestmark = pytest.mark.gpu
+
+DTYPES = [torch.float32, torch.bfloat16]
+
+
+@pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
+@pytest.mark.parametrize("T,dk,dv", [(1, 64, 64), (37, 64, 64), (130, 128, 128),
+                                     (200, 64, 128), (257, 128, 64)])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_gla_bwd(dtype, T, dk, dv, with_state):
+    cpu, dev = small_problem(20 + T, 2, 2, T, dk, dv, 0, dtype, train=True, h0=with_state)
+    dhT = dev["dhT"] if with_state else None
+    res = L.gla_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["dO"], dev.get("h0"), dhT,
+                    want_dh0=True)
+    x = oracle_inputs(cpu, ("q", "k", "v", "g", "dO", "h0", "dhT"))
+    ref = oracle.gla_bwd(x["q"], x["k"], x["v"], x["g"], x["dO"], x["h0"],
+                         x["dhT"] if with_state else None)
+    for name in ("dq", "dk", "dv", "dg", "dh0"):
+        assert_close(name, res[name], ref[name], dtype)
+
+
+@pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
+@pytest.mark.parametrize("T,w,M,sink", [(1, 1, 2, False), (50, 1, 0, False),
+                                        (130, 33, 4, False), (130, 33, 4, True),
+                                        (150, 200, 0, False), (290, 128, 16, False)])
+def test_swa_meta_bwd(dtype, T, w, M, sink):
+    cpu, dev = small_problem(40 + T + w, 2, 2, T, 128, 128, M, dtype, train=True)
+    mk = dev["meta_k"] if M else None
+    mv = dev["meta_v"] if (M and not sink) else None
+    _, lse = L.swa_meta_fwd(dev["q"], dev["k"], dev["v"], mk, mv, w=w)
+    res = L.swa_meta_bwd(dev["q"], dev["k"], dev["v"], mk, mv, lse, dev["dO"], w=w)
+    x = oracle_inputs(cpu, ("q", "k", "v", "meta_k", "meta_v", "dO"))
+    ref = oracle.swa_meta_bwd(x["q"], x["k"], x["v"], x["meta_k"] if M else None,
+                              x["meta_v"] if (M and not sink) else None, x["dO"], w,
+                              1 / math.sqrt(128))
+    for name in ("dq", "dk", "dv"):
+        assert_close(name, res[name], ref[name], dtype)
+    if M:
+        assert_close("dmeta_k", res["dmeta_k"], ref["dmeta_k"], dtype)
+        if not sink:
+            assert_close("dmeta_v", res["dmeta_v"], ref["dmeta_v"], dtype)
+
+
+@pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
+@pytest.mark.parametrize("alpha", [0.0, 0.5, 2.0])
+def test_hybrid_bwd(dtype, alpha):
+    T, w, M = 210, 40, 6
+    cpu, dev = small_problem(77, 2, 2, T, 128, 128, M, dtype, train=True, h0=True)
+    fwd = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
+                       w=w, alpha=alpha, h0=dev["h0"], want_lse=True)
+    res = L.hybrid_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
+                       fwd["lse"], dev["dO"], w=w, alpha=alpha, h0=dev["h0"], dhT=dev["dhT"],
+                       want_dh0=True)
+    x = oracle_inputs(cpu, ("q", "k", "v", "g", "meta_k", "meta_v", "dO", "h0", "dhT"))
+    ref = oracle.hybrid_bwd(x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], x["dO"], w,
+                            1 / math.sqrt(128), alpha, x["h0"], x["dhT"])
+    for name in ("dq", "dk", "dv", "dg", "dh0", "dmeta_k", "dmeta_v"):
+        assert_close(name, res[name], ref[name], dtype)
+    assert_close("dalpha", res["dalpha"].cpu().double().numpy(), np.array([ref["dalpha"]]), dtype)
+
+
+def test_gla_bwd_full_forgetting():
+    """g = -30 everywhere: the elementwise-exponent path of the backward."""
+    cpu, dev = small_problem(3, 1, 2, 45, 64, 64, 0, torch.float32, train=True)
+    g = torch.full((1, 2, 45, 64), -30.0)
+    g[..., ::2, :] = -0.05
+    res = L.gla_bwd(dev["q"], dev["k"], dev["v"], g.cuda(), dev["dO"])
+    x = oracle_inputs(cpu, ("q", "k", "v", "dO"))
+    ref = oracle.gla_bwd(x["q"], x["k"], x["v"], g.double().numpy(), x["dO"])
+    for name in ("dq", "dk", "dv", "dg"):
+        assert_close(name, res[name], ref[name], torch.float32)
+
+
+def test_bwd_determinism():
+    cpu, dev = small_problem(8, 2, 2, 300, 128, 128, 4, torch.bfloat16, train=True)
+    fwd = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
+                       w=64, alpha=0.5, want_lse=True)
+    runs = [L.hybrid_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
+                         fwd["lse"], dev["dO"], w=64, alpha=0.5) for _ in range(2)]
+    for name in ("dq", "dk", "dv", "dg", "dmeta_k", "dmeta_v", "dalpha"):
+        assert torch.equal(runs[0][name], runs[1][name]), name
+
+
+def test_workload_train_sampled():
+    """Llama-3-8B-shaped training layer (B=2, H=32, T=8192): fwd + bwd at full
+    size on the GPU; every per-token gradient checked on sampled heads, meta
+    gradients for one head exactly (both batch rows), dalpha over all heads."""
+    wl = I.TRAIN_BF16
+    x = I.make_inputs(wl, seed=0, device="cpu")
+    dev = {k: v.cuda() for k, v in x.items()}
+    fwd = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
+                       w=wl.w, alpha=wl.alpha, chunk=wl.chunk, want_lse=True)
+    res = L.hybrid_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
+                       fwd["lse"], dev["dO"], w=wl.w, alpha=wl.alpha, chunk=wl.chunk)
+    torch.cuda.synchronize()
+    h = 5
+    for b in range(wl.B):
+        sl = lambda t: np64(t[b:b + 1, h:h + 1])
+        ref = oracle.hybrid_bwd(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["g"]),
+                                np64(x["meta_k"][h:h + 1]), np64(x["meta_v"][h:h + 1]),
+                                sl(x["dO"]), wl.w, wl.scale, wl.alpha)
+        for name in ("dq", "dk", "dv", "dg"):
+            assert_close(f"{name}[{b},{h}]", res[name][b:b + 1, h:h + 1], ref[name],
+                         torch.bfloat16)
+        if b == 0:
+            mk_acc, mv_acc = ref["dmeta_k"].copy(), ref["dmeta_v"].copy()
+        else:
+            mk_acc += ref["dmeta_k"]
+            mv_acc += ref["dmeta_v"]
+    assert_close("dmeta_k[h]", res["dmeta_k"][h:h + 1], mk_acc, torch.bfloat16)
+    assert_close("dmeta_v[h]", res["dmeta_v"][h:h + 1], mv_acc, torch.bfloat16)
+    # dalpha = sum over every (b, h, t) of dO . o_swa, with o_swa from the oracle
+    xs = {k: np64(v) for k, v in x.items() if k in ("q", "k", "v", "meta_k", "meta_v", "dO")}
+    o_swa, _ = oracle.swa_meta_fwd(xs["q"], xs["k"], xs["v"], xs["meta_k"], xs["meta_v"], wl.w,
+                                   wl.scale)
+    dal = float(np.sum(xs["dO"] * o_swa))
+    assert_close("dalpha", res["dalpha"].cpu().double().numpy(), np.array([dal]),
+                 torch.bfloat16)

@@ -1,0 +1,107 @@
+"""Decode-step parity: the constant-memory generation step vs the oracle, the
+decode-equals-prefill identity on the GPU, and save/restore of the state."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import gated_linear_sliding_chunked_b200 as L
+from gated_linear_sliding_chunked_b200 import inputs as I
+import oracle
+from parity_util import assert_close, np64, small_problem
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("w,M,sink", [(1, 0, False), (5, 2, False), (16, 3, True),
+                                      (40, 16, False)])
+def test_decode_equals_prefill(dtype, w, M, sink):
+    """T steps from an empty state reproduce the hybrid forward on the same
+    tokens (the window wraps around the ring when T > w)."""
+    Bd, H, T = 3, 2, 37
+    cpu, dev = small_problem(50 + w + M, Bd, H, T, 128, 128, M, dtype)
+    mk = dev["meta_k"] if M else None
+    mv = dev["meta_v"] if (M and not sink) else None
+    alpha = 0.7
+    pre = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], mk, mv, w=w, alpha=alpha,
+                       want_hT=True)
+    state = torch.zeros(Bd, H, 128, 128, device="cuda")
+    kring = torch.zeros(Bd, H, w, 128, dtype=dtype, device="cuda")
+    vring = torch.zeros_like(kring)
+    pos = torch.zeros(Bd, dtype=torch.int64, device="cuda")
+    outs = []
+    for t in range(T):
+        sl = lambda n: dev[n][:, :, t].contiguous()
+        outs.append(L.decode_step(state, kring, vring, pos, sl("q"), sl("k"), sl("v"), sl("g"),
+                                  mk, mv, alpha=alpha).clone())
+    dec = torch.stack(outs, dim=2)
+    x = {k: np64(v) for k, v in cpu.items()}
+    ref = oracle.hybrid_fwd(x["q"], x["k"], x["v"], x["g"], x["meta_k"] if M else None,
+                            x["meta_v"] if (M and not sink) else None, w, 1 / math.sqrt(128),
+                            alpha)
+    assert_close("decode o", dec, ref["o"], dtype)
+    assert_close("decode state", state, ref["hT"], dtype)
+    assert_close("prefill o", pre["o"], ref["o"], dtype)
+    assert torch.all(pos.cpu() == T)
+
+
+def test_decode_workload_sampled():
+    """Decode workload shape (Bd=128, H=32, w=128, M=8, bf16 I/O, fp32 state)
+    from a random full-window state: 6 steps on the GPU; sampled
+    (sequence, head) pairs replayed in the oracle step by step."""
+    wl = I.DECODE
+    st = I.make_decode_state(wl, seed=0, device="cpu")
+    toks = I.make_decode_tokens(wl, steps=6, seed=1, device="cpu")
+    d = {k: v.cuda() for k, v in st.items()}
+    outs = []
+    for s in range(6):
+        outs.append(L.decode_step(d["state"], d["kring"], d["vring"], d["pos"],
+                                  toks["q"][s].cuda(), toks["k"][s].cuda(), toks["v"][s].cuda(),
+                                  toks["g"][s].cuda(), d["meta_k"], d["meta_v"],
+                                  alpha=wl.alpha).clone())
+    torch.cuda.synchronize()
+    seqs = [0, 77, 127]
+    heads = [0, 13, 31]
+    ost = {"state": np64(st["state"][seqs][:, heads]), "kring": np64(st["kring"][seqs][:, heads]),
+           "vring": np64(st["vring"][seqs][:, heads]), "pos": st["pos"][seqs].numpy()}
+    mk = np64(st["meta_k"][heads])
+    mv = np64(st["meta_v"][heads])
+    for s in range(6):
+        sel = lambda t: np64(t[s][seqs][:, heads])
+        ost = oracle.decode_step(ost["state"], ost["kring"], ost["vring"], ost["pos"],
+                                 sel(toks["q"]), sel(toks["k"]), sel(toks["v"]), sel(toks["g"]),
+                                 mk, mv, wl.scale, wl.alpha)
+        assert_close(f"o step {s}", outs[s][seqs][:, heads], ost["o"], torch.bfloat16)
+    assert_close("state", d["state"][seqs][:, heads], ost["state"], torch.bfloat16)
+    assert np.array_equal(np64(d["kring"][seqs][:, heads]), ost["kring"])
+    assert np.array_equal(np64(d["vring"][seqs][:, heads]), ost["vring"])
+    assert torch.all(d["pos"].cpu() == wl.pos0 + 6)
+
+
+def test_decode_state_save_restore_bitwise():
+    Bd, H, w, M = 4, 2, 8, 2
+    cpu, dev = small_problem(90, Bd, H, 12, 128, 128, M, torch.bfloat16)
+    state = torch.randn(Bd, H, 128, 128, device="cuda") * 0.1
+    kring = (torch.randn(Bd, H, w, 128, device="cuda") * 0.1).bfloat16()
+    vring = (torch.randn(Bd, H, w, 128, device="cuda") * 0.1).bfloat16()
+    pos = torch.tensor([0, 3, 8, 100], dtype=torch.int64, device="cuda")
+
+    def run(st, kr, vr, ps, t0, t1):
+        o = []
+        for t in range(t0, t1):
+            sl = lambda n: dev[n][:, :, t].contiguous()
+            o.append(L.decode_step(st, kr, vr, ps, sl("q"), sl("k"), sl("v"), sl("g"),
+                                   dev["meta_k"], dev["meta_v"], alpha=0.5).clone())
+        return o
+
+    a = [x.clone() for x in (state, kring, vring, pos)]
+    run(*a, 0, 6)
+    saved = [x.clone() for x in a]
+    out1 = run(*a, 6, 12)
+    out2 = run(*saved, 6, 12)
+    for x, y in zip(out1, out2):
+        assert torch.equal(x, y)
+    for x, y in zip(a, saved):
+        assert torch.equal(x, y)
