@@ -92,9 +92,17 @@ __global__ void __launch_bounds__(NT) decode_kernel(DecodeParams p) {
   const IO* mv = p.mv ? (const IO*)p.mv + (size_t)h * M * D : nullptr;
   const int nkeys = nwin + M;
   const int half = lane >> 4, l16 = lane & 15;
-  for (int key = warp * 2 + half; key < nkeys; key += 2 * (NT / 32)) {
+  // The trip count depends on the warp only (both half-warps iterate together)
+  // because the full-mask shuffles below need all 32 lanes every iteration.
+  for (int base = warp * 2; base < nkeys; base += 2 * (NT / 32)) {
+    const int key = base + half;
+    const bool have = key < nkeys;
     float x[8];
-    if (key == 0) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = 0.f;
+    if (!have) {
+      // second half-warp past the last key: contributes zeros
+    } else if (key == 0) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) x[e] = ks[l16 * 8 + e];
     } else if (key < nwin) {
@@ -110,7 +118,7 @@ __global__ void __launch_bounds__(NT) decode_kernel(DecodeParams p) {
     a += __shfl_xor_sync(0xffffffffu, a, 4);
     a += __shfl_xor_sync(0xffffffffu, a, 2);
     a += __shfl_xor_sync(0xffffffffu, a, 1);
-    if (l16 == 0) sc[key] = a * p.scale;
+    if (have && l16 == 0) sc[key] = a * p.scale;
   }
   __syncthreads();
   if (warp == 0) {
