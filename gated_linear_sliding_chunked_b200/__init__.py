@@ -30,7 +30,10 @@ LZ_WS_GLA_FWD, LZ_WS_HYBRID_FWD, LZ_WS_GLA_BWD, LZ_WS_SWA_BWD, LZ_WS_HYBRID_BWD 
 
 EXPORTS = ("lz_gla_fwd", "lz_gla_bwd", "lz_swa_meta_fwd", "lz_hybrid_fwd", "lz_swa_meta_bwd",
            "lz_hybrid_bwd", "lz_gla_decode_step", "lz_workspace_bytes", "lz_last_error",
-           "lz_version", "lz_timing_enable", "lz_timing_read")
+           "lz_version", "lz_timing_enable", "lz_timing_read", "lz_swa_meta_bwd_noalloc")
+
+# size of the static scratch array behind lz_swa_meta_bwd_noalloc
+LZ_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class LzError(RuntimeError):
@@ -69,6 +72,7 @@ def load(path: str = LIB_PATH):
     lib.lz_gla_bwd.argtypes = [D] + [_P] * 12 + [_P, sz, _P]
     lib.lz_swa_meta_bwd.argtypes = [D] + [_P] * 12 + [_P, sz, _P]
     lib.lz_hybrid_bwd.argtypes = [D] + [_P] * 18 + [_P, sz, _P]
+    lib.lz_swa_meta_bwd_noalloc.argtypes = [D] + [_P] * 12 + [_P]
     lib.lz_gla_decode_step.argtypes = ([ctypes.c_int] * 7 + [ctypes.c_float] * 2 +
                                        [_P] * 11 + [_P])
     lib.lz_timing_enable.argtypes = [ctypes.c_int]
@@ -174,6 +178,18 @@ def lz_swa_meta_bwd(dims, q, k, v, meta_k, meta_v, lse, dO, dq, dk, dv, dmeta_k,
                                   _ptr(meta_v), _ptr(lse), _ptr(dO), _ptr(dq), _ptr(dk),
                                   _ptr(dv), _ptr(dmeta_k), _ptr(dmeta_v), _ptr(ws), ws_bytes,
                                   _stream(stream)))
+
+
+def lz_swa_meta_bwd_noalloc(dims, q, k, v, meta_k, meta_v, lse, dO, dq, dk, dv, dmeta_k,
+                            dmeta_v, stream=None):
+    """lz_swa_meta_bwd without caller scratch: for callers that cannot
+    allocate device memory; uses the library's static scratch array (see
+    include/lizard.h for the size limit and the rule against overlapping
+    calls)."""
+    _check(load().lz_swa_meta_bwd_noalloc(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v),
+                                          _ptr(meta_k), _ptr(meta_v), _ptr(lse), _ptr(dO),
+                                          _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dmeta_k),
+                                          _ptr(dmeta_v), _stream(stream)))
 
 
 def lz_hybrid_bwd(dims, q, k, v, g, meta_k, meta_v, h0, lse, dO, dhT, dq, dk, dv, dg, dh0,

@@ -24,6 +24,9 @@ class ScopedTiming {
   cudaEvent_t a_ = nullptr, b_ = nullptr;
 };
 
+// Records `message` as the thread's last error and returns `status`.
+int set_last_error(int status, const char* message);
+
 // ---- gated branch, SIMT path (fp32 arithmetic; fp32 or bf16 I/O) ----------
 struct GlaFwdParams {
   const void* q;

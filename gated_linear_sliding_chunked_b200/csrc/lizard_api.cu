@@ -27,6 +27,19 @@ lz_status ok() {
   return LZ_OK;
 }
 
+}  // namespace
+
+namespace lz {
+// Lets other translation units of the library report a failure through
+// lz_last_error().
+int set_last_error(int status, const char* message) {
+  g_err = message ? message : "";
+  return status;
+}
+}  // namespace lz
+
+namespace {
+
 lz_status cuda_status(cudaError_t e, const char* what) {
   if (e == cudaSuccess) return ok();
   return fail(LZ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));

@@ -128,6 +128,34 @@ lz_status lz_swa_meta_bwd(const lz_dims* d, const void* q, const void* k,
                           float* dmeta_k, float* dmeta_v, void* ws,
                           size_t ws_bytes, lz_stream stream);
 
+/* Scratch-free variant of lz_swa_meta_bwd, for callers that cannot allocate
+ * device memory when they run the backward (for example an engine plugin
+ * whose enqueue step must not call cudaMalloc, or a host framework that has
+ * reserved all device memory for its own pool).  The paper has no
+ * counterpart: this is a deployment convenience.
+ *
+ * Arguments, layouts and results are those of lz_swa_meta_bwd; the scratch
+ * comes from a static device array of LZ_NOALLOC_SCRATCH_BYTES (16 MiB) that
+ * the library holds on every GPU that loads it until the process exits.
+ * A problem whose lz_workspace_bytes(d, LZ_WS_SWA_BWD) exceeds that size is
+ * rejected with LZ_ERR_UNSUPPORTED (nothing launched).  The call allocates
+ * nothing (no cudaMalloc/cudaFree, no allocating library routine).
+ *
+ * The first call on a device (the device current on the calling thread,
+ * which must be the stream's device) looks up the array's device address
+ * once; make that first call before any stream capture.  All calls share
+ * the one array: calls that may overlap on the GPU (different streams, or
+ * several host threads, on the same device) race and must be serialized by
+ * the caller.  The array keeps the previous call's contents; every part of
+ * it is written before it is read, so nothing needs clearing. */
+#define LZ_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+lz_status lz_swa_meta_bwd_noalloc(const lz_dims* d, const void* q,
+                                  const void* k, const void* v,
+                                  const void* meta_k, const void* meta_v,
+                                  const float* lse, const void* dO, void* dq,
+                                  void* dk, void* dv, float* dmeta_k,
+                                  float* dmeta_v, lz_stream stream);
+
 /* Gradient of lz_hybrid_fwd in one call: the gated branch sees dO, the
  * window branch alpha * dO.  lse from the forward.  dalpha (nullable, one
  * fp32) receives sum over (b,h,t) of dO_t . o_swa_t. */

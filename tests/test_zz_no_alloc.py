@@ -1,0 +1,63 @@
+"""Scratch-free window + meta-token backward (lz_swa_meta_bwd_noalloc).
+
+Some callers cannot allocate device memory at the moment they run the
+backward: an engine plugin whose enqueue step must not call cudaMalloc, or a
+host framework that has already reserved all device memory for its own pool.
+The entry point that serves them takes its scratch from a fixed array inside
+the library instead of from the caller.  These tests check that it returns
+the same gradients as lz_swa_meta_bwd with caller-owned scratch, on two calls
+in a row (the second call finds the first call's leftovers in the shared
+array), and that a problem too large for the array is refused before anything
+runs.
+
+This file is named so that pytest collects it last.
+"""
+import ctypes
+
+import pytest
+import torch
+
+import gated_linear_sliding_chunked_b200 as L
+from gated_linear_sliding_chunked_b200 import build as lbuild
+from parity_util import assert_close, small_problem
+
+
+def _noalloc(dims, dev, mk, mv, lse):
+    out = {"dq": torch.empty_like(dev["q"]), "dk": torch.empty_like(dev["k"]),
+           "dv": torch.empty_like(dev["v"]),
+           "dmeta_k": torch.empty(mk.shape, dtype=torch.float32, device="cuda"),
+           "dmeta_v": torch.empty(mv.shape, dtype=torch.float32, device="cuda")}
+    L.lz_swa_meta_bwd_noalloc(dims, dev["q"], dev["k"], dev["v"], mk, mv, lse, dev["dO"],
+                              out["dq"], out["dk"], out["dv"], out["dmeta_k"], out["dmeta_v"])
+    return out
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_allocating_backward_twice():
+    lbuild.build()
+    L.load()
+    # two different problems back to back through the same static scratch
+    cases = [(3, 2, 4, 700, 64, 8, torch.bfloat16), (4, 1, 3, 513, 33, 3, torch.float32)]
+    for seed, B, H, T, w, M, dtype in cases:
+        cpu, dev = small_problem(seed, B, H, T, 128, 128, M, dtype, train=True)
+        mk, mv = dev["meta_k"], dev["meta_v"]
+        dims = L.make_dims(B, H, T, 128, 128, chunk=64, w=w, M=M, io=L.io_of(dtype),
+                           alpha=1.0)
+        assert L.lz_workspace_bytes(dims, L.LZ_WS_SWA_BWD) <= L.LZ_NOALLOC_SCRATCH_BYTES
+        _, lse = L.swa_meta_fwd(dev["q"], dev["k"], dev["v"], mk, mv, w=w)
+        ref = L.swa_meta_bwd(dev["q"], dev["k"], dev["v"], mk, mv, lse, dev["dO"], w=w)
+        got = _noalloc(dims, dev, mk, mv, lse)
+        torch.cuda.synchronize()
+        for name in ("dq", "dk", "dv", "dmeta_k", "dmeta_v"):
+            assert_close(f"{name} (T={T})", got[name], ref[name].double().cpu().numpy(), dtype)
+
+
+def test_noalloc_rejects_problem_larger_than_its_scratch():
+    lbuild.build()
+    lib = L.load()
+    dims = L.make_dims(1, 32, 200_000, 128, 128, chunk=64, w=64, M=4, io=L.LZ_BF16)
+    assert L.lz_workspace_bytes(dims, L.LZ_WS_SWA_BWD) > L.LZ_NOALLOC_SCRATCH_BYTES
+    fake = ctypes.c_void_p(0x7F0000000000)
+    st = lib.lz_swa_meta_bwd_noalloc(ctypes.byref(dims), *([fake] * 12), None)
+    assert st == L.LZ_ERR_UNSUPPORTED
+    assert b"static" in lib.lz_last_error()
