@@ -515,7 +515,7 @@ def main(argv=None):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "data": "synthetic (seeded, BASELINE-shaped distributions)",
+            "dtype": "bf16", "data": "synthetic (seeded, BASELINE-shaped distributions)",
             "config": {"workload": wl.name, "global_batch": wl.B * world, "seq_len": wl.T,
                        "heads": wl.H, "head_dim": wl.dk, "window": wl.w, "meta_tokens": wl.M,
                        "chunk": wl.chunk, "io": wl.io, "alpha": wl.alpha,

@@ -37,12 +37,21 @@ struct GlaFwdParams {
   void* o;             // nullable: skip outputs (state pass only)
   float* hT;           // nullable
   float* states;       // nullable: [BH][nchunks][dk][dv] state before each chunk
+  void* states16;      // nullable (tensor-core kernel): the same in bf16, 64-token chunks
   const float* add;    // nullable: fp32 [B,H,T,dv], o += alpha * add
+  const void* add16;   // nullable (tensor-core kernel): the same in bf16; may alias o
   float alpha;
   int B, H, T, dk, dv;
 };
 constexpr int kSimtChunk = 16;
 cudaError_t launch_gla_fwd_simt(const GlaFwdParams& p, bool bf16, cudaStream_t s);
+
+// ---- gated branch, tensor-core forward (bf16 I/O, dk = 128) --------------
+// Same params; `states` (if set) receives the fp32 state before every
+// 64-token chunk: [BH][ceil(T/64)][dk][dv].
+bool gla_fwd_mma_supported(int dk, int dv, bool bf16);
+int gla_fwd_mma_chunk();
+cudaError_t launch_gla_fwd_mma(const GlaFwdParams& p, cudaStream_t s);
 
 struct GlaBwdParams {
   const void* q;
@@ -52,10 +61,12 @@ struct GlaBwdParams {
   const void* dO;
   const float* dhT;      // nullable
   const float* states;   // [BH][nchunks][dk][dv] from the state pass
+  const void* states16;  // tensor-core kernel: bf16 states per 64-token chunk
   const float* hT;       // [BH][dk][dv] final state (read only when dhT != NULL)
   const float* add_dq;   // nullable fp32 [B,H,T,dk] added before the store
   const float* add_dk;   // nullable
   const float* add_dv;   // nullable fp32 [B,H,T,dv]
+  bool add_in_place;     // tensor-core kernel: dq, dk, dv already hold bf16 terms to add
   void* dq;
   void* dk;
   void* dv;
@@ -64,6 +75,11 @@ struct GlaBwdParams {
   int B, H, T, dkd, dvd;
 };
 cudaError_t launch_gla_bwd_simt(const GlaBwdParams& p, bool bf16, cudaStream_t s);
+
+// ---- gated branch, tensor-core backward (bf16 I/O, dk = dv = 128) --------
+// Needs states16 and hT from the tensor-core forward run as a state pass.
+bool gla_bwd_mma_supported(int dk, int dv, bool bf16);
+cudaError_t launch_gla_bwd_mma(const GlaBwdParams& p, cudaStream_t s);
 
 // ---- window + meta softmax, SIMT path ------------------------------------
 struct SwaFwdParams {
@@ -79,6 +95,9 @@ struct SwaFwdParams {
   float scale;
 };
 cudaError_t launch_swa_fwd_simt(const SwaFwdParams& p, bool bf16, cudaStream_t s);
+// tensor-core forward (bf16 I/O, dk = dv = 128)
+bool swa_fwd_mma_supported(int dk, int dv, bool bf16);
+cudaError_t launch_swa_fwd_mma(const SwaFwdParams& p, cudaStream_t s);
 
 struct SwaBwdParams {
   const void* q;
@@ -107,6 +126,11 @@ struct SwaBwdParams {
 int swa_bwd_n_qblocks(int B, int H, int T);
 int swa_bwd_n_meta_parts(int B, int T);
 cudaError_t launch_swa_bwd_simt(const SwaBwdParams& p, bool bf16, cudaStream_t s);
+// fixed-order sums of the meta-gradient and dalpha partials
+cudaError_t launch_swa_bwd_reduce(const SwaBwdParams& p, int nparts, int nalpha, cudaStream_t s);
+// tensor-core backward (bf16 I/O, dk = dv = 128); same scratch layout
+bool swa_bwd_mma_supported(int dk, int dv, bool bf16);
+cudaError_t launch_swa_bwd_mma(const SwaBwdParams& p, cudaStream_t s);
 
 // ---- decode --------------------------------------------------------------
 struct DecodeParams {

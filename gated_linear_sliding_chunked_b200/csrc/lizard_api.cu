@@ -12,6 +12,26 @@ namespace {
 
 thread_local std::string g_err;
 
+// The window branch's forward: tensor cores for bf16 with dk = dv = 128,
+// fp32 SIMT otherwise.
+cudaError_t swa_forward(const lz::SwaFwdParams& p, bool bf16, cudaStream_t s) {
+  if (lz::swa_fwd_mma_supported(p.dk, p.dv, bf16)) return lz::launch_swa_fwd_mma(p, s);
+  return lz::launch_swa_fwd_simt(p, bf16, s);
+}
+
+// The window branch's backward: tensor cores for bf16 with dk = dv = 128.
+cudaError_t swa_backward(const lz::SwaBwdParams& p, bool bf16, cudaStream_t s) {
+  if (lz::swa_bwd_mma_supported(p.dkd, p.dvd, bf16)) return lz::launch_swa_bwd_mma(p, s);
+  return lz::launch_swa_bwd_simt(p, bf16, s);
+}
+
+// The forward of the gated branch: tensor cores for bf16 with dk = 128,
+// fp32 SIMT otherwise.
+cudaError_t gla_forward(const lz::GlaFwdParams& p, bool bf16, cudaStream_t s) {
+  if (p.o && lz::gla_fwd_mma_supported(p.dk, p.dv, bf16)) return lz::launch_gla_fwd_mma(p, s);
+  return lz::launch_gla_fwd_simt(p, bf16, s);
+}
+
 lz_status fail(lz_status st, const char* fmt, ...) {
   char buf[512];
   va_list ap;
@@ -111,14 +131,35 @@ size_t nchunks16(const lz_dims* d) {
 }
 
 // ---- workspace layouts ----------------------------------------------------
+bool bwd_uses_mma(const lz_dims* d) {
+  return lz::gla_bwd_mma_supported(d->dk, d->dv, d->io == LZ_BF16);
+}
+
+// Tensor-core hybrid path: the window branch's bf16 results go straight into
+// the caller's output buffers and the gated kernels add to them in place.
+bool hybrid_uses_mma(const lz_dims* d) {
+  const bool bf = d->io == LZ_BF16;
+  return lz::gla_fwd_mma_supported(d->dk, d->dv, bf) && lz::swa_fwd_mma_supported(d->dk, d->dv, bf) &&
+         lz::swa_bwd_mma_supported(d->dk, d->dv, bf) && lz::gla_bwd_mma_supported(d->dk, d->dv, bf);
+}
+
+// Gated backward scratch: the states before every chunk (fp32 per 16-token
+// chunk for the SIMT kernel, bf16 per 64-token chunk for the tensor-core
+// kernel) and the final state.
 struct GlaBwdWs {
   float* states;
+  void* states16;
   float* hT;
 };
 GlaBwdWs carve_gla_bwd(Carver& c, const lz_dims* d) {
-  GlaBwdWs w;
+  GlaBwdWs w{};
   const size_t bh = (size_t)d->B * d->H;
-  w.states = c.take<float>(bh * nchunks16(d) * d->dk * d->dv);
+  if (bwd_uses_mma(d)) {
+    const size_t n64 = (size_t)((d->T + lz::gla_fwd_mma_chunk() - 1) / lz::gla_fwd_mma_chunk());
+    w.states16 = c.take<uint16_t>(bh * n64 * d->dk * d->dv);  // bf16
+  } else {
+    w.states = c.take<float>(bh * nchunks16(d) * d->dk * d->dv);
+  }
   w.hT = c.take<float>(bh * d->dk * d->dv);
   return w;
 }
@@ -140,17 +181,19 @@ SwaBwdWs carve_swa_bwd(Carver& c, const lz_dims* d) {
 struct HybridBwdWs {
   SwaBwdWs swa;
   GlaBwdWs gla;
-  float* dq;
+  float* dq;  // fp32 window-branch gradients (SIMT path only)
   float* dk;
   float* dv;
 };
 HybridBwdWs carve_hybrid_bwd(Carver& c, const lz_dims* d) {
-  HybridBwdWs w;
+  HybridBwdWs w{};
   w.swa = carve_swa_bwd(c, d);
   w.gla = carve_gla_bwd(c, d);
-  w.dq = c.take<float>(bht(d) * d->dk);
-  w.dk = c.take<float>(bht(d) * d->dk);
-  w.dv = c.take<float>(bht(d) * d->dv);
+  if (!hybrid_uses_mma(d)) {
+    w.dq = c.take<float>(bht(d) * d->dk);
+    w.dk = c.take<float>(bht(d) * d->dk);
+    w.dv = c.take<float>(bht(d) * d->dv);
+  }
   return w;
 }
 
@@ -160,7 +203,7 @@ size_t ws_bytes(const lz_dims* d, int which) {
     case LZ_WS_GLA_FWD:
       return 0;
     case LZ_WS_HYBRID_FWD:
-      c.take<float>(bht(d) * d->dv);
+      if (!hybrid_uses_mma(d)) c.take<float>(bht(d) * d->dv);  // fp32 window output
       return c.off;
     case LZ_WS_GLA_BWD:
       carve_gla_bwd(c, d);
@@ -241,8 +284,7 @@ lz_status lz_gla_fwd(const lz_dims* d, const void* q, const void* k, const void*
   lz::GlaFwdParams p = gla_fwd_params(d, q, k, v, g, h0);
   p.o = o;
   p.hT = hT;
-  return cuda_status(lz::launch_gla_fwd_simt(p, d->io == LZ_BF16, as_stream(stream)),
-                     "lz_gla_fwd");
+  return cuda_status(gla_forward(p, d->io == LZ_BF16, as_stream(stream)), "lz_gla_fwd");
 }
 
 lz_status lz_swa_meta_fwd(const lz_dims* d, const void* q, const void* k, const void* v,
@@ -256,8 +298,7 @@ lz_status lz_swa_meta_fwd(const lz_dims* d, const void* q, const void* k, const 
   lz::SwaFwdParams p = swa_fwd_params(d, q, k, v, meta_k, meta_v);
   p.o = o;
   p.lse = lse;
-  return cuda_status(lz::launch_swa_fwd_simt(p, d->io == LZ_BF16, as_stream(stream)),
-                     "lz_swa_meta_fwd");
+  return cuda_status(swa_forward(p, d->io == LZ_BF16, as_stream(stream)), "lz_swa_meta_fwd");
 }
 
 lz_status lz_hybrid_fwd(const lz_dims* d, const void* q, const void* k, const void* v,
@@ -274,40 +315,47 @@ lz_status lz_hybrid_fwd(const lz_dims* d, const void* q, const void* k, const vo
   if (st != LZ_OK) return st;
   const cudaStream_t s = as_stream(stream);
   const bool bf = d->io == LZ_BF16;
+  const bool mma = hybrid_uses_mma(d);
   Carver c(ws);
-  float* osw = c.take<float>(bht(d) * d->dv);
+  float* osw = mma ? nullptr : c.take<float>(bht(d) * d->dv);
   lz::SwaFwdParams sp = swa_fwd_params(d, q, k, v, meta_k, meta_v);
-  sp.o = o_swa;
+  // tensor-core path: bf16 window output into o_swa if requested, else into o
+  sp.o = mma ? (o_swa ? o_swa : o) : o_swa;
   sp.o_f32 = osw;
   sp.lse = lse;
-  cudaError_t e = lz::launch_swa_fwd_simt(sp, bf, s);
+  cudaError_t e = swa_forward(sp, bf, s);
   if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_fwd (window branch)");
   lz::GlaFwdParams gp = gla_fwd_params(d, q, k, v, g, h0);
   gp.o = o;
   gp.hT = hT;
   gp.add = osw;
+  gp.add16 = mma ? sp.o : nullptr;
   gp.alpha = d->alpha;
-  return cuda_status(lz::launch_gla_fwd_simt(gp, bf, s), "lz_hybrid_fwd (gated branch)");
+  return cuda_status(gla_forward(gp, bf, s), "lz_hybrid_fwd (gated branch)");
 }
 
 static cudaError_t gla_bwd_launch(const lz_dims* d, const void* q, const void* k, const void* v,
                                   const float* g, const float* h0, const void* dO,
                                   const float* dhT, void* dq, void* dk, void* dv, float* dg,
                                   float* dh0, const GlaBwdWs& w, const float* add_dq,
-                                  const float* add_dk, const float* add_dv, cudaStream_t s) {
+                                  const float* add_dk, const float* add_dv, bool add_in_place,
+                                  cudaStream_t s) {
   const bool bf = d->io == LZ_BF16;
+  const bool mma = bwd_uses_mma(d);
   lz::GlaFwdParams fp = gla_fwd_params(d, q, k, v, g, h0);
   fp.states = w.states;
+  fp.states16 = w.states16;
   fp.hT = w.hT;
-  cudaError_t e = lz::launch_gla_fwd_simt(fp, bf, s);
+  cudaError_t e = mma ? lz::launch_gla_fwd_mma(fp, s) : lz::launch_gla_fwd_simt(fp, bf, s);
   if (e != cudaSuccess) return e;
   lz::GlaBwdParams p{};
   p.q = q; p.k = k; p.v = v; p.g = g; p.dO = dO; p.dhT = dhT;
-  p.states = w.states; p.hT = w.hT;
+  p.states = w.states; p.states16 = w.states16; p.hT = w.hT;
   p.add_dq = add_dq; p.add_dk = add_dk; p.add_dv = add_dv;
+  p.add_in_place = add_in_place;
   p.dq = dq; p.dk = dk; p.dv = dv; p.dg = dg; p.dh0 = dh0;
   p.B = d->B; p.H = d->H; p.T = d->T; p.dkd = d->dk; p.dvd = d->dv;
-  return lz::launch_gla_bwd_simt(p, bf, s);
+  return mma ? lz::launch_gla_bwd_mma(p, s) : lz::launch_gla_bwd_simt(p, bf, s);
 }
 
 lz_status lz_gla_bwd(const lz_dims* d, const void* q, const void* k, const void* v,
@@ -325,7 +373,7 @@ lz_status lz_gla_bwd(const lz_dims* d, const void* q, const void* k, const void*
   Carver c(ws);
   GlaBwdWs w = carve_gla_bwd(c, d);
   return cuda_status(gla_bwd_launch(d, q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, w,
-                                    nullptr, nullptr, nullptr, as_stream(stream)),
+                                    nullptr, nullptr, nullptr, false, as_stream(stream)),
                      "lz_gla_bwd");
 }
 
@@ -348,8 +396,7 @@ lz_status lz_swa_meta_bwd(const lz_dims* d, const void* q, const void* k, const 
   p.gscale = 1.f;
   p.dq = dq; p.dk = dk; p.dv = dv;
   p.dmk = dmeta_k; p.dmv = dmeta_v;
-  return cuda_status(lz::launch_swa_bwd_simt(p, d->io == LZ_BF16, as_stream(stream)),
-                     "lz_swa_meta_bwd");
+  return cuda_status(swa_backward(p, d->io == LZ_BF16, as_stream(stream)), "lz_swa_meta_bwd");
 }
 
 lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const void* v,
@@ -372,14 +419,18 @@ lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const vo
   const cudaStream_t s = as_stream(stream);
   Carver c(ws);
   HybridBwdWs w = carve_hybrid_bwd(c, d);
+  const bool mma = hybrid_uses_mma(d);
   lz::SwaBwdParams p = swa_bwd_params(d, q, k, v, meta_k, meta_v, lse, dO, w.swa);
   p.gscale = d->alpha;
+  // tensor-core path: bf16 window gradients straight into dq, dk, dv; the
+  // gated backward then adds its own terms in place
+  p.dq = dq; p.dk = dk; p.dv = dv;
   p.dq_f32 = w.dq; p.dk_f32 = w.dk; p.dv_f32 = w.dv;
   p.dmk = dmeta_k; p.dmv = dmeta_v; p.dalpha = dalpha;
-  cudaError_t e = lz::launch_swa_bwd_simt(p, d->io == LZ_BF16, s);
+  cudaError_t e = swa_backward(p, d->io == LZ_BF16, s);
   if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (window branch)");
   return cuda_status(gla_bwd_launch(d, q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, w.gla,
-                                    w.dq, w.dk, w.dv, s),
+                                    w.dq, w.dk, w.dv, mma, s),
                      "lz_hybrid_bwd (gated branch)");
 }
 

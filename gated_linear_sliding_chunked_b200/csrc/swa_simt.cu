@@ -525,6 +525,16 @@ cudaError_t bwd_launch(const SwaBwdParams& p, cudaStream_t s) {
 }  // namespace
 
 int swa_bwd_n_qblocks(int B, int H, int T) { return ((T + QR - 1) / QR) * B * H; }
+
+cudaError_t launch_swa_bwd_reduce(const SwaBwdParams& p, int nparts, int nalpha, cudaStream_t s) {
+  const int total = p.H * p.M * (p.dkd + p.dvd);
+  const int blocks = max(1, (total + 255) / 256);
+  {
+    ScopedTiming tm("swa_bwd_reduce", s);
+    swa_bwd_reduce_kernel<<<blocks, 256, 0, s>>>(p, nparts, nalpha);
+  }
+  return cudaGetLastError();
+}
 int swa_bwd_n_meta_parts(int B, int T) { return B * ((T + SLAB - 1) / SLAB); }
 
 cudaError_t launch_swa_fwd_simt(const SwaFwdParams& p, bool bf16, cudaStream_t s) {

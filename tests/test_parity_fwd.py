@@ -65,22 +65,27 @@ def test_hybrid_fwd(dtype, alpha):
                      (dtype if name == "hT" else torch.float32))
 
 
-def test_gate_edge_cases():
-    """g = 0 (no decay), g = -30 (full forgetting, the elementwise path) and a
-    mixture inside one chunk."""
-    T = 70
-    cpu, dev = small_problem(3, 1, 2, T, 64, 64, 0, torch.float32)
-    for fill in (0.0, -30.0, "mixed"):
-        g = torch.zeros(1, 2, T, 64)
+@pytest.mark.parametrize("dtype,d", [(torch.float32, 64), (torch.bfloat16, 128)],
+                         ids=["f32-d64", "bf16-d128"])
+def test_gate_edge_cases(dtype, d):
+    """g = 0 (no decay), g = -30 (full forgetting: the elementwise path), a
+    mixture inside one chunk, and one decaying key dim among slow ones."""
+    T = 150
+    cpu, dev = small_problem(3, 1, 2, T, d, d, 0, dtype)
+    for fill in (0.0, -30.0, "mixed", "one-dim"):
+        g = torch.zeros(1, 2, T, d)
         if fill == "mixed":
             g[..., ::3, :] = -30.0
             g[..., 1::3, :] = -0.01
+        elif fill == "one-dim":
+            g[..., :] = -0.02
+            g[..., 70:90, 5] = -9.0
         else:
             g.fill_(fill)
         o, hT = L.gla_fwd(dev["q"], dev["k"], dev["v"], g.cuda(), want_hT=True)
         ro, rhT = oracle.gla_fwd(np64(cpu["q"]), np64(cpu["k"]), np64(cpu["v"]), g.double().numpy())
-        assert_close(f"o[g={fill}]", o, ro, torch.float32)
-        assert_close(f"hT[g={fill}]", hT, rhT, torch.float32)
+        assert_close(f"o[g={fill}]", o, ro, dtype)
+        assert_close(f"hT[g={fill}]", hT, rhT, dtype)
 
 
 def test_empty_sequence_keeps_state():
