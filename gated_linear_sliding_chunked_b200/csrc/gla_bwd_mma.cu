@@ -93,38 +93,45 @@ static_assert(sizeof(BwdSmem) <= 232448, "shared memory per block exceeds 227 KB
 
 __device__ __forceinline__ int pair_index(int I, int J) { return I * (I + 1) / 2 + J; }
 
-// Transposed diagonal scores A^T[t][u] = sum_i q_u,i k_t,i exp(sum_{x=t+1..u} g_x,i)
-// for u >= t inside sub-block I (this CTA's key dims only), at the lane's
-// fragment positions.  q, k: stage tiles [C][DKH]; g: global, first row of
-// the chunk, row stride DK, already offset to this CTA's dims.
-__device__ __noinline__ void diag_at_elementwise(const bf16* q, const bf16* k, const float* g,
-                                                 int rows, int I, int lane, float (*acc)[4]) {
-  const int gr = lane >> 2, gc = (lane & 3) * 2;
-  for (int nt = 0; nt < 2; ++nt)
-    for (int e = 0; e < 4; ++e) {
-      const int t = gr + (e >> 1) * 8, u = nt * 8 + gc + (e & 1);
-      const int rt = SB * I + t, ru = SB * I + u;
-      float a = 0.f;
-      if (u >= t && ru < rows) {
-        for (int i = 0; i < DKH; ++i) {
-          float lg = 0.f;
-          for (int x = rt + 1; x <= ru; ++x) lg += g[(size_t)x * DK + i];
-          a += __bfloat162float(q[ru * DKH + i]) * __bfloat162float(k[rt * DKH + i]) * __expf(lg);
-        }
-      }
-      acc[nt][e] = a;
-    }
+// exp(sum_{x = s+1 .. t} g_x,i) for chunk rows s <= t (g: global, the
+// chunk's first row, already offset to this CTA's key dims).  Used only by
+// the strong-decay fallback of the diagonal blocks; it returns a scalar so
+// that no register array of the caller has its address taken.
+__device__ __noinline__ float gate_ratio(const float* g, int rows, int t, int s, int i) {
+  float lg = 0.f;
+  for (int x = s + 1; x <= t && x < rows; ++x) lg += g[(size_t)x * DK + i];
+  return __expf(lg);
 }
 
-// Same for B-side products: E[t][s] = exp(sum_{x=s+1..t} g_x) is needed
-// elementwise only through A; B carries no gate, so dq/dk intra terms of a
-// slow diagonal block are rebuilt from these per-dim factors.
-__device__ __noinline__ void diag_gate_elementwise(const float* g, int rows, int I, int t, int s,
-                                                   int i, float* out) {
-  // exp(sum_{x=s+1..t} g_x,i) for one (t, s, i); t, s relative to sub-block I
-  float lg = 0.f;
-  for (int x = SB * I + s + 1; x <= SB * I + t && x < rows; ++x) lg += g[(size_t)x * DK + i];
-  *out = __expf(lg);
+// Diagonal-block intra term of a strong-decay chunk at (row t, key dim il):
+// role 0 (dq): sum_{s in block, s <= t} (dO_t . v_s) k_s,il exp(b_t - b_s)
+// role 1 (dk): sum_{u in block, u >= t} (dO_u . v_t) q_u,il exp(b_u - b_t)
+__device__ __noinline__ float diag_intra_term(const bf16* dO, const bf16* v, const bf16* kq,
+                                              const float* g, int rows, int I, int t, int il,
+                                              int role) {
+  float x = 0.f;
+  const int lo = role == 0 ? SB * I : t, hi = role == 0 ? t : SB * I + SB - 1;
+  for (int r = lo; r <= hi; ++r) {
+    const int rq = role == 0 ? t : r, rv = role == 0 ? r : t;
+    float b = 0.f;
+    for (int j = 0; j < DV; ++j) b += __bfloat162float(dO[rq * VP + j]) * __bfloat162float(v[rv * VP + j]);
+    x += b * __bfloat162float(kq[r * DKH + il]) *
+         (role == 0 ? gate_ratio(g, rows, t, r, il) : gate_ratio(g, rows, r, t, il));
+  }
+  return x;
+}
+
+// A^T[t][u] = sum_i q_u,i k_t,i exp(b_u,i - b_t,i) over this CTA's key dims,
+// chunk rows t <= u < rows (strong-decay fallback of the diagonal blocks).
+__device__ __noinline__ float diag_at_entry(const bf16* q, const bf16* k, const float* g, int rows,
+                                            int t, int u) {
+  float a = 0.f;
+  for (int i = 0; i < DKH; ++i) {
+    float lg = 0.f;
+    for (int x = t + 1; x <= u && x < rows; ++x) lg += g[(size_t)x * DK + i];
+    a += __bfloat162float(q[u * DKH + i]) * __bfloat162float(k[t * DKH + i]) * __expf(lg);
+  }
+  return a;
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
@@ -308,361 +315,249 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     }
     const bool scaled = flags & 1, slow = flags & 2;
 
-    float dv[16][4];  // warps 4..7: partial dv of rows I, all 128 value columns
-    if (warp < 4) {
-      // ================= dq, dk of rows I (this CTA's key dims) =============
-      const int I = warp;
-      float acc[8][4];
-      // ---- B[I][J <= I] with dO rows I as A ---------------------------------
-      {
-        uint32_t da[8][4];
+    // warp -> (row block I, role): role 0 computes dq and dv of value columns
+    // [0, 64); role 1 computes dk and dv of value columns [64, 128)
+    const int I = warp & 3, role = warp >> 2;
+    const float* gch = g + (size_t)c0 * DK + i0;  // this chunk, this CTA's dims
+    // in-place terms (the window branch's gradients) for this warp's outputs,
+    // loaded now so that the loads overlap the products below
+    uint32_t pre[8][2], prev[8][2];
+    if (p.add_in_place) {
+      const bf16* src = (const bf16*)(role == 0 ? p.dq : p.dk);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          ldsm_x4(smem_u32(&sm.dO[st][(16 * I + (lane & 15)) * VP + kk * 16 + (lane >> 4) * 8]),
-                  da[kk][0], da[kk][1], da[kk][2], da[kk][3]);
-        float bs[NSB][2][4];
+      for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-        for (int J = 0; J < NSB; ++J) {
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) bs[J][nt][e] = 0.f;
-          if (J > I) continue;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(smem_u32(&sm.v[st][(16 * J + (lane & 7) + ((lane >> 4) << 3)) * VP + kk * 16 +
-                                       ((lane >> 3) & 1) * 8]),
-                    b0, b1, b2, b3);
-            mma_bf16(bs[J][0], da[kk], b0, b1);
-            mma_bf16(bs[J][1], da[kk], b2, b3);
-          }
-          if (J == I) {
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int t = gr + (e >> 1) * 8, sk = nt * 8 + gc + (e & 1);
-                if (sk > t) bs[J][nt][e] = 0.f;
-              }
-          }
+        for (int hh = 0; hh < 2; ++hh) {
+          const int t = 16 * I + gr + 8 * hh;
+          pre[nt][hh] = c0 + t < T ? *reinterpret_cast<const uint32_t*>(
+                                         &src[tk + (size_t)(c0 + t) * DK + i0 + nt * 8 + gc])
+                                   : 0u;
+          prev[nt][hh] = (role == half && c0 + t < T)
+                             ? *reinterpret_cast<const uint32_t*>(
+                                   &((const bf16*)p.dv)[tv + (size_t)(c0 + t) * DV + 64 * half + nt * 8 + gc])
+                             : 0u;
         }
-        // ---- dq accumulator: inter (dO S_prev^T, scaled by ci per dim) -----
+    }
+    // role 0: A rows = dO rows I, score partner = v rows J <= I, inter B = S_prev,
+    //         intra B = Kf_J (factor F_IJ), output scale Eq
+    // role 1: A rows = v rows I,  score partner = dO rows J >= I, inter B = G,
+    //         intra B = Qf_J (factor F_JI), output scale Ek
+    const bf16* arows = role == 0 ? sm.dO[st] : sm.v[st];
+    const bf16* prows = role == 0 ? sm.v[st] : sm.dO[st];
+    const bf16* inter_b = role == 0 ? sm.sp : sm.g16;
+    const bf16* intra_b = role == 0 ? sm.kf : sm.qf;
+    const float* colf = role == 0 ? sm.ci[I] : sm.ck[I];
+    const bf16* oscale = role == 0 ? sm.eqf : sm.ekf;
+    float acc[8][4];
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
+    for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-        const float* ciI = sm.ci[I];
+      for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+    // ---- inter: (dO S_prev^T | v G^T), then per-dim factor (ci | ck) --------
+#pragma unroll 2
+    for (int kk = 0; kk < 8; ++kk) {
+      uint32_t a[4];
+      ldsm_x4(smem_u32(&arows[(16 * I + (lane & 15)) * VP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
+              a[3]);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-          for (int ntp = 0; ntp < 4; ++ntp) {
-            uint32_t b0, b1, b2, b3;
-            const int n = ntp * 16 + (lane & 7) + ((lane >> 4) << 3);
-            ldsm_x4(smem_u32(&sm.sp[swz(n, kk * 16 + ((lane >> 3) & 1) * 8)]), b0, b1, b2, b3);
-            const float f0 = ciI[ntp * 16 + gr], f1 = ciI[ntp * 16 + 8 + gr];
-            b0 = scale_bf16x2(b0, f0, f0);
-            b1 = scale_bf16x2(b1, f0, f0);
-            b2 = scale_bf16x2(b2, f1, f1);
-            b3 = scale_bf16x2(b3, f1, f1);
-            mma_bf16(acc[2 * ntp], da[kk], b0, b1);
-            mma_bf16(acc[2 * ntp + 1], da[kk], b2, b3);
-          }
-        }
-        // ---- seed part: column sums of q * dq_inter over this warp's rows ----
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-          const int il = nt * 8 + gc;
-          float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int t = 16 * I + gr + 8 * hh;
-            const float2 eq = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.eqf[t * KP + il]));
-            const float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.q[st][t * DKH + il]));
-            s0 += qv.x * acc[nt][2 * hh] * eq.x;
-            s1 += qv.y * acc[nt][2 * hh + 1] * eq.y;
-          }
-#pragma unroll
-          for (int o = 4; o < 32; o <<= 1) {
-            s0 += __shfl_xor_sync(0xffffffffu, s0, o);
-            s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-          }
-          if (gr == 0) {
-            sm.qdqi[I][il] = s0;
-            sm.qdqi[I][il + 1] = s1;
-          }
-        }
-        // ---- dq intra: sum_J B[I][J] (Kf_J * F_IJ) --------------------------
-#pragma unroll
-        for (int J = 0; J < NSB; ++J) {
-          if (J > I) continue;
-          if (J == I && slow) continue;  // handled elementwise below
-          const uint32_t pa[4] = {pack_bf16(bs[J][0][0], bs[J][0][1]), pack_bf16(bs[J][0][2], bs[J][0][3]),
-                                  pack_bf16(bs[J][1][0], bs[J][1][1]), pack_bf16(bs[J][1][2], bs[J][1][3])};
-          const float* fac = sm.fac[pair_index(I, J)];
-#pragma unroll
-          for (int ntp = 0; ntp < 4; ++ntp) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(smem_u32(&sm.kf[(16 * J + (lane & 7) + ((lane >> 3) & 1) * 8) * KP + ntp * 16 +
-                                      (lane >> 4) * 8]),
-                      b0, b1, b2, b3);
-            if (scaled) {
-              const float f0 = fac[ntp * 16 + gr], f1 = fac[ntp * 16 + 8 + gr];
-              b0 = scale_bf16x2(b0, f0, f0);
-              b1 = scale_bf16x2(b1, f0, f0);
-              b2 = scale_bf16x2(b2, f1, f1);
-              b3 = scale_bf16x2(b3, f1, f1);
-            }
-            mma_bf16(acc[2 * ntp], pa, b0, b1);
-            mma_bf16(acc[2 * ntp + 1], pa, b2, b3);
-          }
-        }
-        // ---- dq = Eq * acc (+ slow diagonal term), store, stage q*dq -------
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int t = 16 * I + gr + 8 * hh;
-            const int il = nt * 8 + gc;
-            const float2 eq = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.eqf[t * KP + il]));
-            float x0 = acc[nt][2 * hh] * eq.x, x1 = acc[nt][2 * hh + 1] * eq.y;
-            if (slow) {
-              // diagonal block: sum_{s in I, s <= t} B[t][s] k_s exp(b_t - b_s)
-              for (int s2 = 0; s2 <= gr + 8 * hh; ++s2) {
-                const int rs = 16 * I + s2;
-                // B[t][s] lives in another lane's registers: rebuild it
-                float bts = 0.f;
-                for (int j = 0; j < DV; ++j)
-                  bts += __bfloat162float(sm.dO[st][t * VP + j]) * __bfloat162float(sm.v[st][rs * VP + j]);
-                float e0, e1;
-                diag_gate_elementwise(g + (size_t)c0 * DK + i0, rows, I, gr + 8 * hh, s2, il, &e0);
-                diag_gate_elementwise(g + (size_t)c0 * DK + i0, rows, I, gr + 8 * hh, s2, il + 1, &e1);
-                x0 += bts * __bfloat162float(sm.k[st][rs * DKH + il]) * e0;
-                x1 += bts * __bfloat162float(sm.k[st][rs * DKH + il + 1]) * e1;
-              }
-            }
-            if (c0 + t < T) {
-              const size_t off = tk + (size_t)(c0 + t) * DK + i0 + il;
-              float y0 = x0, y1 = x1;
-              if (p.add_dq) {
-                const float2 a = *reinterpret_cast<const float2*>(&p.add_dq[off]);
-                y0 += a.x;
-                y1 += a.y;
-              } else if (p.add_in_place) {
-                const float2 a = unpack_bf16(*reinterpret_cast<const uint32_t*>(&((const bf16*)p.dq)[off]));
-                y0 += a.x;
-                y1 += a.y;
-              }
-              *reinterpret_cast<uint32_t*>(&((bf16*)p.dq)[off]) = pack_bf16(y0, y1);
-            }
-            const float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.q[st][t * DKH + il]));
-            sm.red[t * RP + il] = qv.x * x0;
-            sm.red[t * RP + il + 1] = qv.y * x1;
-          }
+      for (int ntp = 0; ntp < 4; ++ntp) {
+        uint32_t b0, b1, b2, b3;
+        const int n = ntp * 16 + (lane & 7) + ((lane >> 4) << 3);
+        ldsm_x4(smem_u32(&inter_b[swz(n, kk * 16 + ((lane >> 3) & 1) * 8)]), b0, b1, b2, b3);
+        mma_bf16(acc[2 * ntp], a, b0, b1);
+        mma_bf16(acc[2 * ntp + 1], a, b2, b3);
       }
-      // ---- B^T[I][J >= I] with v rows I as A ---------------------------------
-      {
-        uint32_t va[8][4];
+    }
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          ldsm_x4(smem_u32(&sm.v[st][(16 * I + (lane & 15)) * VP + kk * 16 + (lane >> 4) * 8]),
-                  va[kk][0], va[kk][1], va[kk][2], va[kk][3]);
-        float bt[NSB][2][4];
+    for (int nt = 0; nt < 8; ++nt) {
+      const float2 f = *reinterpret_cast<const float2*>(&colf[nt * 8 + gc]);
+      acc[nt][0] *= f.x;
+      acc[nt][1] *= f.y;
+      acc[nt][2] *= f.x;
+      acc[nt][3] *= f.y;
+    }
+    if (role == 0) {
+      // ---- seed part of dg: column sums of q * dq_inter over these rows ------
 #pragma unroll
-        for (int J = 0; J < NSB; ++J) {
+      for (int nt = 0; nt < 8; ++nt) {
+        const int il = nt * 8 + gc;
+        float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) bt[J][nt][e] = 0.f;
-          if (J < I) continue;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(smem_u32(&sm.dO[st][(16 * J + (lane & 7) + ((lane >> 4) << 3)) * VP + kk * 16 +
-                                        ((lane >> 3) & 1) * 8]),
-                    b0, b1, b2, b3);
-            mma_bf16(bt[J][0], va[kk], b0, b1);
-            mma_bf16(bt[J][1], va[kk], b2, b3);
-          }
-          if (J == I) {
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int t = gr + (e >> 1) * 8, u = nt * 8 + gc + (e & 1);
-                if (u < t) bt[J][nt][e] = 0.f;
-              }
-          }
+        for (int hh = 0; hh < 2; ++hh) {
+          const int t = 16 * I + gr + 8 * hh;
+          const float2 eq = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.eqf[t * KP + il]));
+          const float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.q[st][t * DKH + il]));
+          s0 += qv.x * acc[nt][2 * hh] * eq.x;
+          s1 += qv.y * acc[nt][2 * hh + 1] * eq.y;
         }
-        // ---- dk accumulator: inter (v G^T, scaled by ck per dim) ------------
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-        const float* ckI = sm.ck[I];
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-          for (int ntp = 0; ntp < 4; ++ntp) {
-            uint32_t b0, b1, b2, b3;
-            const int n = ntp * 16 + (lane & 7) + ((lane >> 4) << 3);
-            ldsm_x4(smem_u32(&sm.g16[swz(n, kk * 16 + ((lane >> 3) & 1) * 8)]), b0, b1, b2, b3);
-            const float f0 = ckI[ntp * 16 + gr], f1 = ckI[ntp * 16 + 8 + gr];
-            b0 = scale_bf16x2(b0, f0, f0);
-            b1 = scale_bf16x2(b1, f0, f0);
-            b2 = scale_bf16x2(b2, f1, f1);
-            b3 = scale_bf16x2(b3, f1, f1);
-            mma_bf16(acc[2 * ntp], va[kk], b0, b1);
-            mma_bf16(acc[2 * ntp + 1], va[kk], b2, b3);
-          }
+        for (int o = 4; o < 32; o <<= 1) {
+          s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+          s1 += __shfl_xor_sync(0xffffffffu, s1, o);
         }
-        // ---- dk intra: sum_{J >= I} B^T[I][J] (Qf_J * F_JI) -----------------
-#pragma unroll
-        for (int J = 0; J < NSB; ++J) {
-          if (J < I) continue;
-          if (J == I && slow) continue;
-          const uint32_t pa[4] = {pack_bf16(bt[J][0][0], bt[J][0][1]), pack_bf16(bt[J][0][2], bt[J][0][3]),
-                                  pack_bf16(bt[J][1][0], bt[J][1][1]), pack_bf16(bt[J][1][2], bt[J][1][3])};
-          const float* fac = sm.fac[pair_index(J, I)];
-#pragma unroll
-          for (int ntp = 0; ntp < 4; ++ntp) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(smem_u32(&sm.qf[(16 * J + (lane & 7) + ((lane >> 3) & 1) * 8) * KP + ntp * 16 +
-                                      (lane >> 4) * 8]),
-                      b0, b1, b2, b3);
-            if (scaled) {
-              const float f0 = fac[ntp * 16 + gr], f1 = fac[ntp * 16 + 8 + gr];
-              b0 = scale_bf16x2(b0, f0, f0);
-              b1 = scale_bf16x2(b1, f0, f0);
-              b2 = scale_bf16x2(b2, f1, f1);
-              b3 = scale_bf16x2(b3, f1, f1);
-            }
-            mma_bf16(acc[2 * ntp], pa, b0, b1);
-            mma_bf16(acc[2 * ntp + 1], pa, b2, b3);
-          }
-        }
-        // ---- dk = Ek * acc (+ slow diagonal term), store, stage -k*dk -------
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int t = 16 * I + gr + 8 * hh;
-            const int il = nt * 8 + gc;
-            const float2 ek = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.ekf[t * KP + il]));
-            float x0 = acc[nt][2 * hh] * ek.x, x1 = acc[nt][2 * hh + 1] * ek.y;
-            if (slow) {
-              // diagonal block: sum_{u in I, u >= t} B[u][t] q_u exp(b_u - b_t)
-              for (int u2 = gr + 8 * hh; u2 < SB; ++u2) {
-                const int ru = 16 * I + u2;
-                float but = 0.f;
-                for (int j = 0; j < DV; ++j)
-                  but += __bfloat162float(sm.dO[st][ru * VP + j]) * __bfloat162float(sm.v[st][t * VP + j]);
-                float e0, e1;
-                diag_gate_elementwise(g + (size_t)c0 * DK + i0, rows, I, u2, gr + 8 * hh, il, &e0);
-                diag_gate_elementwise(g + (size_t)c0 * DK + i0, rows, I, u2, gr + 8 * hh, il + 1, &e1);
-                x0 += but * __bfloat162float(sm.q[st][ru * DKH + il]) * e0;
-                x1 += but * __bfloat162float(sm.q[st][ru * DKH + il + 1]) * e1;
-              }
-            }
-            if (c0 + t < T) {
-              const size_t off = tk + (size_t)(c0 + t) * DK + i0 + il;
-              float y0 = x0, y1 = x1;
-              if (p.add_dk) {
-                const float2 a = *reinterpret_cast<const float2*>(&p.add_dk[off]);
-                y0 += a.x;
-                y1 += a.y;
-              } else if (p.add_in_place) {
-                const float2 a = unpack_bf16(*reinterpret_cast<const uint32_t*>(&((const bf16*)p.dk)[off]));
-                y0 += a.x;
-                y1 += a.y;
-              }
-              *reinterpret_cast<uint32_t*>(&((bf16*)p.dk)[off]) = pack_bf16(y0, y1);
-            }
-            const float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.k[st][t * DKH + il]));
-            sm.red[t * RP + il] -= kv.x * x0;
-            sm.red[t * RP + il + 1] -= kv.y * x1;
-          }
+        if (gr == 0) *reinterpret_cast<float2*>(&sm.qdqi[I][il]) = make_float2(s0, s1);
       }
-    } else {
-      // ================= partial dv of rows I over this CTA's key dims ======
-      const int I = warp - 4;
-      float at[NSB][2][4];
+    }
+    // ---- intra: one 16x16 score block at a time, consumed right away -------
+    const int jlo = role == 0 ? 0 : I, jhi = role == 0 ? I : NSB - 1;
+    for (int J = jlo; J <= jhi; ++J) {
+      float sc[2][4];
 #pragma unroll
-      for (int J = 0; J < NSB; ++J) {
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
+#pragma unroll 2
+      for (int kk = 0; kk < 8; ++kk) {
+        uint32_t a[4], b0, b1, b2, b3;
+        ldsm_x4(smem_u32(&arows[(16 * I + (lane & 15)) * VP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
+                a[3]);
+        ldsm_x4(smem_u32(&prows[(16 * J + (lane & 7) + ((lane >> 4) << 3)) * VP + kk * 16 +
+                                ((lane >> 3) & 1) * 8]),
+                b0, b1, b2, b3);
+        mma_bf16(sc[0], a, b0, b1);
+        mma_bf16(sc[1], a, b2, b3);
+      }
+      if (J == I) {
+        if (slow) continue;  // the diagonal block of a strong-decay chunk: below
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) at[J][nt][e] = 0.f;
-        if (J < I) continue;
-        const float* fac = sm.fac[pair_index(J, I)];
-#pragma unroll
-        for (int kk = 0; kk < DKH / 16; ++kk) {
-          uint32_t a[4];
-          ldsm_x4(smem_u32(&sm.kf[(16 * I + (lane & 15)) * KP + kk * 16 + (lane >> 4) * 8]), a[0], a[1],
-                  a[2], a[3]);
-          if (scaled) {
-            const float2 f0 = *reinterpret_cast<const float2*>(&fac[kk * 16 + gc]);
-            const float2 f1 = *reinterpret_cast<const float2*>(&fac[kk * 16 + 8 + gc]);
-            a[0] = scale_bf16x2(a[0], f0.x, f0.y);
-            a[1] = scale_bf16x2(a[1], f0.x, f0.y);
-            a[2] = scale_bf16x2(a[2], f1.x, f1.y);
-            a[3] = scale_bf16x2(a[3], f1.x, f1.y);
+          for (int e = 0; e < 4; ++e) {
+            const int t = gr + (e >> 1) * 8, u = nt * 8 + gc + (e & 1);
+            if (role == 0 ? (u > t) : (u < t)) sc[nt][e] = 0.f;
           }
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(smem_u32(&sm.qf[(16 * J + (lane & 7) + ((lane >> 4) << 3)) * KP + kk * 16 +
-                                  ((lane >> 3) & 1) * 8]),
+      }
+      const uint32_t pa[4] = {pack_bf16(sc[0][0], sc[0][1]), pack_bf16(sc[0][2], sc[0][3]),
+                              pack_bf16(sc[1][0], sc[1][1]), pack_bf16(sc[1][2], sc[1][3])};
+      const float* fac = sm.fac[role == 0 ? pair_index(I, J) : pair_index(J, I)];
+#pragma unroll
+      for (int ntp = 0; ntp < 4; ++ntp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(smem_u32(&intra_b[(16 * J + (lane & 7) + ((lane >> 3) & 1) * 8) * KP + ntp * 16 +
+                                    (lane >> 4) * 8]),
                   b0, b1, b2, b3);
-          mma_bf16(at[J][0], a, b0, b1);
-          mma_bf16(at[J][1], a, b2, b3);
+        if (scaled) {
+          const float f0 = fac[ntp * 16 + gr], f1 = fac[ntp * 16 + 8 + gr];
+          b0 = scale_bf16x2(b0, f0, f0);
+          b1 = scale_bf16x2(b1, f0, f0);
+          b2 = scale_bf16x2(b2, f1, f1);
+          b3 = scale_bf16x2(b3, f1, f1);
         }
-        if (J == I) {
-          if (slow) {
-            diag_at_elementwise(sm.q[st], sm.k[st], g + (size_t)c0 * DK + i0, rows, I, lane, at[J]);
-          } else {
+        mma_bf16(acc[2 * ntp], pa, b0, b1);
+        mma_bf16(acc[2 * ntp + 1], pa, b2, b3);
+      }
+    }
+    // ---- finalize (dq | dk) = (Eq | Ek) * acc, store, stage for dg ---------
+    float kdk[8][4];  // role 1: k * dk, subtracted into red after a barrier
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+    for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int t = gr + (e >> 1) * 8, u = nt * 8 + gc + (e & 1);
-                if (u < t) at[J][nt][e] = 0.f;
-              }
+      for (int hh = 0; hh < 2; ++hh) {
+        const int t = 16 * I + gr + 8 * hh;
+        const int il = nt * 8 + gc;
+        const float2 os = unpack_bf16(*reinterpret_cast<const uint32_t*>(&oscale[t * KP + il]));
+        float x0 = acc[nt][2 * hh] * os.x, x1 = acc[nt][2 * hh + 1] * os.y;
+        if (slow) {
+          x0 += diag_intra_term(sm.dO[st], sm.v[st], role == 0 ? sm.k[st] : sm.q[st], gch, rows, I, t, il,
+                                role);
+          x1 += diag_intra_term(sm.dO[st], sm.v[st], role == 0 ? sm.k[st] : sm.q[st], gch, rows, I, t,
+                                il + 1, role);
+        }
+        if (c0 + t < T) {
+          const size_t off = tk + (size_t)(c0 + t) * DK + i0 + il;
+          const float* addf = role == 0 ? p.add_dq : p.add_dk;
+          float y0 = x0, y1 = x1;
+          if (addf) {
+            const float2 a = *reinterpret_cast<const float2*>(&addf[off]);
+            y0 += a.x;
+            y1 += a.y;
+          } else if (p.add_in_place) {
+            const float2 a = unpack_bf16(pre[nt][hh]);
+            y0 += a.x;
+            y1 += a.y;
           }
+          *reinterpret_cast<uint32_t*>(&((bf16*)(role == 0 ? p.dq : p.dk))[off]) = pack_bf16(y0, y1);
+        }
+        const float2 xv = unpack_bf16(*reinterpret_cast<const uint32_t*>(
+            &(role == 0 ? sm.q[st] : sm.k[st])[t * DKH + il]));
+        if (role == 0) {
+          *reinterpret_cast<float2*>(&sm.red[t * RP + il]) = make_float2(xv.x * x0, xv.y * x1);
+        } else {
+          kdk[nt][2 * hh] = xv.x * x0;
+          kdk[nt][2 * hh + 1] = xv.y * x1;
         }
       }
+
+    // ---- partial dv of rows I, value columns [64 role, 64 role + 64) ---------
+    float dvh[8][4];
 #pragma unroll
-      for (int nt = 0; nt < 16; ++nt)
+    for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) dv[nt][e] = 0.f;
-      // inter: (k e^{b_l - b})_I G   (k over this CTA's key dims)
+      for (int e = 0; e < 4; ++e) dvh[nt][e] = 0.f;
+    // inter: (k e^{b_l - b})_I G[:, this role's columns]
+#pragma unroll
+    for (int kk = 0; kk < DKH / 16; ++kk) {
+      uint32_t a[4];
+      ldsm_x4(smem_u32(&sm.ks[(16 * I + (lane & 15)) * KP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
+              a[3]);
+#pragma unroll
+      for (int ntp = 0; ntp < 4; ++ntp) {
+        uint32_t b0, b1, b2, b3;
+        const int kr = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        ldsm_x4_t(smem_u32(&sm.g16[swz(kr, 64 * role + ntp * 16 + (lane >> 4) * 8)]), b0, b1, b2, b3);
+        mma_bf16(dvh[2 * ntp], a, b0, b1);
+        mma_bf16(dvh[2 * ntp + 1], a, b2, b3);
+      }
+    }
+    // intra: A^T[I][J] dO_J for J >= I, one score block at a time
+    for (int J = I; J < NSB; ++J) {
+      float at[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) at[nt][e] = 0.f;
+      const float* fac = sm.fac[pair_index(J, I)];
 #pragma unroll
       for (int kk = 0; kk < DKH / 16; ++kk) {
         uint32_t a[4];
-        ldsm_x4(smem_u32(&sm.ks[(16 * I + (lane & 15)) * KP + kk * 16 + (lane >> 4) * 8]), a[0], a[1],
-                a[2], a[3]);
-#pragma unroll
-        for (int ntp = 0; ntp < 8; ++ntp) {
-          uint32_t b0, b1, b2, b3;
-          const int kr = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-          ldsm_x4_t(smem_u32(&sm.g16[swz(kr, ntp * 16 + (lane >> 4) * 8)]), b0, b1, b2, b3);
-          mma_bf16(dv[2 * ntp], a, b0, b1);
-          mma_bf16(dv[2 * ntp + 1], a, b2, b3);
+        ldsm_x4(smem_u32(&sm.kf[(16 * I + (lane & 15)) * KP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
+                a[3]);
+        if (scaled) {
+          const float2 f0 = *reinterpret_cast<const float2*>(&fac[kk * 16 + gc]);
+          const float2 f1 = *reinterpret_cast<const float2*>(&fac[kk * 16 + 8 + gc]);
+          a[0] = scale_bf16x2(a[0], f0.x, f0.y);
+          a[1] = scale_bf16x2(a[1], f0.x, f0.y);
+          a[2] = scale_bf16x2(a[2], f1.x, f1.y);
+          a[3] = scale_bf16x2(a[3], f1.x, f1.y);
         }
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(smem_u32(&sm.qf[(16 * J + (lane & 7) + ((lane >> 4) << 3)) * KP + kk * 16 +
+                                ((lane >> 3) & 1) * 8]),
+                b0, b1, b2, b3);
+        mma_bf16(at[0], a, b0, b1);
+        mma_bf16(at[1], a, b2, b3);
       }
-      // intra: sum_{J >= I} A^T[I][J] dO_J
+      if (J == I) {
 #pragma unroll
-      for (int J = 0; J < NSB; ++J) {
-        if (J < I) continue;
-        const uint32_t pa[4] = {pack_bf16(at[J][0][0], at[J][0][1]), pack_bf16(at[J][0][2], at[J][0][3]),
-                                pack_bf16(at[J][1][0], at[J][1][1]), pack_bf16(at[J][1][2], at[J][1][3])};
+        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int ntp = 0; ntp < 8; ++ntp) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(smem_u32(&sm.dO[st][(16 * J + (lane & 7) + ((lane >> 3) & 1) * 8) * VP + ntp * 16 +
-                                        (lane >> 4) * 8]),
-                    b0, b1, b2, b3);
-          mma_bf16(dv[2 * ntp], pa, b0, b1);
-          mma_bf16(dv[2 * ntp + 1], pa, b2, b3);
-        }
+          for (int e = 0; e < 4; ++e) {
+            const int t = gr + (e >> 1) * 8, u = nt * 8 + gc + (e & 1);
+            const int rt = 16 * I + t, ru = 16 * I + u;
+            if (u < t) at[nt][e] = 0.f;
+            else if (slow) at[nt][e] = ru < rows ? diag_at_entry(sm.q[st], sm.k[st], gch, rows, rt, ru) : 0.f;
+          }
+      }
+      const uint32_t pa[4] = {pack_bf16(at[0][0], at[0][1]), pack_bf16(at[0][2], at[0][3]),
+                              pack_bf16(at[1][0], at[1][1]), pack_bf16(at[1][2], at[1][3])};
+#pragma unroll
+      for (int ntp = 0; ntp < 4; ++ntp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(smem_u32(&sm.dO[st][(16 * J + (lane & 7) + ((lane >> 3) & 1) * 8) * VP + 64 * role +
+                                      ntp * 16 + (lane >> 4) * 8]),
+                  b0, b1, b2, b3);
+        mma_bf16(dvh[2 * ntp], pa, b0, b1);
+        mma_bf16(dvh[2 * ntp + 1], pa, b2, b3);
       }
     }
 
@@ -713,9 +608,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
         }
       }
     }
-    __syncthreads();  // red staged; every reader of sp, g16 and the operands is done
+    __syncthreads();  // q*dq staged; every reader of sp, g16 and the operands is done
     if (c > 0) issue_sp(c - 1);
     write_g16();
+    if (role == 1) {
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int t = 16 * I + gr + 8 * hh, il = nt * 8 + gc;
+          float2* r = reinterpret_cast<float2*>(&sm.red[t * RP + il]);
+          const float2 x = *r;
+          *r = make_float2(x.x - kdk[nt][2 * hh], x.y - kdk[nt][2 * hh + 1]);
+        }
+    }
+    __syncthreads();
 
     // ---- dg: exact seed at the chunk's first row, then a running sum inside --
     {
@@ -743,39 +650,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
 
     // ---- dv: exchange the peer's 64 columns through distributed smem --------
     cluster.sync();  // both CTAs are done with red
-    if (warp >= 4) {
-      const int I = warp - 4;
-      const int pcol = 64 * (half ^ 1);
+    if (role != half) {  // these warps hold the peer's value columns
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int t = 16 * I + gr + 8 * hh, cl = nt * 8 + gc;
-          const int ntg = (pcol >> 3) + nt;
-          *reinterpret_cast<float2*>(&peer_red[t * RP + cl]) =
-              make_float2(dv[ntg][2 * hh], dv[ntg][2 * hh + 1]);
+          *reinterpret_cast<float2*>(&peer_red[t * RP + cl]) = make_float2(dvh[nt][2 * hh], dvh[nt][2 * hh + 1]);
         }
     }
     cluster.sync();  // the peer's share has landed in red
-    if (warp >= 4) {
-      const int I = warp - 4;
+    if (role == half) {
       const int mcol = 64 * half;
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int t = 16 * I + gr + 8 * hh, cl = nt * 8 + gc;
-          const int ntg = (mcol >> 3) + nt;
           if (c0 + t >= T) continue;
           const float2 pr = *reinterpret_cast<const float2*>(&sm.red[t * RP + cl]);
-          float y0 = dv[ntg][2 * hh] + pr.x, y1 = dv[ntg][2 * hh + 1] + pr.y;
+          float y0 = dvh[nt][2 * hh] + pr.x, y1 = dvh[nt][2 * hh + 1] + pr.y;
           const size_t off = tv + (size_t)(c0 + t) * DV + mcol + cl;
           if (p.add_dv) {
             const float2 a = *reinterpret_cast<const float2*>(&p.add_dv[off]);
             y0 += a.x;
             y1 += a.y;
           } else if (p.add_in_place) {
-            const float2 a = unpack_bf16(*reinterpret_cast<const uint32_t*>(&((const bf16*)p.dv)[off]));
+            const float2 a = unpack_bf16(prev[nt][hh]);
             y0 += a.x;
             y1 += a.y;
           }

@@ -64,29 +64,21 @@ static_assert(sizeof(FwdSmem<64>) <= 232448, "shared memory per block exceeds 22
 
 __device__ __forceinline__ int pair_index(int I, int J) { return I * (I + 1) / 2 + J; }
 
-// Diagonal-block scores with one exponential per (t, s, key dim):
-// A[t][s] = sum_i q_t,i k_s,i exp(sum_{u=s+1..t} g_u,i) for the lane's
-// fragment positions of sub-block I (zero above the diagonal).  Used only
-// when a sub-block's gate decay leaves the range of the factorized form.
-// g points at the chunk's first row in global memory.
-__device__ __noinline__ void diag_scores_elementwise(const bf16* q, const bf16* k, const float* g,
-                                                     int rows, int I, int lane,
-                                                     float (*acc)[4]) {
-  const int gr = lane >> 2, gc = (lane & 3) * 2;
-  for (int nt = 0; nt < 2; ++nt)
-    for (int e = 0; e < 4; ++e) {
-      const int t = gr + (e >> 1) * 8, sk = nt * 8 + gc + (e & 1);
-      float a = 0.f;
-      const int rt = SB * I + t, rs = SB * I + sk;
-      if (sk <= t && rt < rows) {
-        for (int i = 0; i < DK; ++i) {
-          float lg = 0.f;
-          for (int u = rs + 1; u <= rt; ++u) lg += g[(size_t)u * DK + i];
-          a += __bfloat162float(q[rt * DK + i]) * __bfloat162float(k[rs * DK + i]) * __expf(lg);
-        }
-      }
-      acc[nt][e] = a;
-    }
+// Diagonal-block score with one exponential per key dim:
+// A[t][s] = sum_i q_t,i k_s,i exp(sum_{u=s+1..t} g_u,i) for rows t, s of
+// the chunk (s <= t < rows).  Used only when a sub-block's gate decay leaves
+// the range of the factorized form; g points at the chunk's first row in
+// global memory.  Returns a scalar so that no register array of the caller
+// has its address taken.
+__device__ __noinline__ float diag_score_elementwise(const bf16* q, const bf16* k, const float* g,
+                                                     int rt, int rs) {
+  float a = 0.f;
+  for (int i = 0; i < DK; ++i) {
+    float lg = 0.f;
+    for (int u = rs + 1; u <= rt; ++u) lg += g[(size_t)u * DK + i];
+    a += __bfloat162float(q[rt * DK + i]) * __bfloat162float(k[rs * DK + i]) * __expf(lg);
+  }
+  return a;
 }
 
 template <int DVT>
@@ -349,8 +341,16 @@ __global__ void __launch_bounds__(NT, 1) gla_fwd_mma_kernel(GlaFwdParams p) {
         }
         if (J == I) {
           if (slow) {
-            diag_scores_elementwise(sm.q[st], sm.k[st], g + (size_t)c0 * DK, T - c0, I, lane,
-                                    acc[J]);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int t = gr + (e >> 1) * 8, sk = nt * 8 + gc + (e & 1);
+                const int rt = 16 * I + t, rs = 16 * I + sk;
+                acc[J][nt][e] = (sk <= t && rt < T - c0)
+                                    ? diag_score_elementwise(sm.q[st], sm.k[st], g + (size_t)c0 * DK, rt, rs)
+                                    : 0.f;
+              }
           } else {
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
