@@ -12,12 +12,11 @@
 //   dk_t = e^{b_l - b_t} (G v_t) + sum_{u>=t} B[u][t] q_u e^{b_u - b_t}
 //   dv_t = (k_t e^{b_l - b_t})^T G + sum_{u>=t} A[u][t] dO_u
 //   G   <- diag(e^{b_l}) G + sum_u (q_u e^{b_u})^T dO_u
-//   dg   : from the gate's direct gradient e^{g_t} <dS_t, S_{t-1}> per key dim,
-//          which at the chunk's first row is
-//            seed = e^{b_l} <G, S_prev> + sum_u q_u * dq_inter_u
-//          (dq_inter_u = e^{b_u} S_prev dO_u), and inside the chunk
-//            dg_t = seed - sum_{u<t} (q_u dq_u - k_u dk_u)
-//          so rounding errors add up over one chunk, not the whole sequence.
+//   dg   : the gate's direct gradient is dg_t = e^{g_t} <dS_t, S_{t-1}> per key
+//          dim; at the chunk's first row that is <G_new, S_prev> with G_new
+//          the carried gradient after this chunk's update, and inside the
+//          chunk dg_t = dg_first - sum_{u<t} (q_u dq_u - k_u dk_u), so
+//          rounding errors add up over one chunk, not the whole sequence.
 //
 // Work split: a cluster of two CTAs per (batch, head); CTA r owns key dims
 // [64r, 64r+64).  dq, dk, dg and its half of G are complete inside the CTA;
@@ -63,6 +62,10 @@ __device__ constexpr float kMinBlockDecay = 8.75651076e-27f;  // e^-60
 __device__ __forceinline__ int swz(int row, int col) {
   return row * 128 + ((((col >> 3) ^ row) & 15) << 3) + (col & 7);
 }
+// [rows][64] bf16 tile, same idea (8 chunks per row)
+__device__ __forceinline__ int swz64(int row, int col) {
+  return row * 64 + ((((col >> 3) ^ row) & 7) << 3) + (col & 7);
+}
 
 struct BwdSmem {
   bf16 q[2][C * DKH];
@@ -84,8 +87,7 @@ struct BwdSmem {
   float ci[NSB][DKH];
   float ck[NSB][DKH];
   float ec[DKH];
-  float qdqi[NSB][DKH];  // per sub-block column sums of q * dq_inter
-  float gsp[2][DKH];     // <G, S_prev> per key dim, two value halves
+  float gsp[2][DKH];     // <G_new, S_prev> per key dim, two value halves
   float tot[NSB][DKH];
 };
 
@@ -115,7 +117,7 @@ __device__ __noinline__ float diag_intra_term(const bf16* dO, const bf16* v, con
     const int rq = role == 0 ? t : r, rv = role == 0 ? r : t;
     float b = 0.f;
     for (int j = 0; j < DV; ++j) b += __bfloat162float(dO[rq * VP + j]) * __bfloat162float(v[rv * VP + j]);
-    x += b * __bfloat162float(kq[r * DKH + il]) *
+    x += b * __bfloat162float(kq[swz64(r, il)]) *
          (role == 0 ? gate_ratio(g, rows, t, r, il) : gate_ratio(g, rows, r, t, il));
   }
   return x;
@@ -129,7 +131,7 @@ __device__ __noinline__ float diag_at_entry(const bf16* q, const bf16* k, const 
   for (int i = 0; i < DKH; ++i) {
     float lg = 0.f;
     for (int x = t + 1; x <= u && x < rows; ++x) lg += g[(size_t)x * DK + i];
-    a += __bfloat162float(q[u * DKH + i]) * __bfloat162float(k[t * DKH + i]) * __expf(lg);
+    a += __bfloat162float(q[swz64(u, i)]) * __bfloat162float(k[swz64(t, i)]) * __expf(lg);
   }
   return a;
 }
@@ -161,8 +163,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       const int r = x / (DKH / 8), cc = x % (DKH / 8);
       const bool ok = c0 + r < T;
       const size_t off = (size_t)(ok ? c0 + r : 0) * DK + i0 + cc * 8;
-      cp_async16(&sm.q[st][r * DKH + cc * 8], q + off, ok ? 16 : 0);
-      cp_async16(&sm.k[st][r * DKH + cc * 8], k + off, ok ? 16 : 0);
+      cp_async16(&sm.q[st][swz64(r, cc * 8)], q + off, ok ? 16 : 0);
+      cp_async16(&sm.k[st][swz64(r, cc * 8)], k + off, ok ? 16 : 0);
     }
     for (int x = tid; x < C * DV / 8; x += NT) {
       const int r = x / (DV / 8), cc = x % (DV / 8);
@@ -298,8 +300,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       if (K == 0) sm.ec[i] = d0 * d1 * d2 * d3;
 #pragma unroll
       for (int r = 0; r < SB; ++r) {
-        const float qv = __bfloat162float(sm.q[st][(r0 + r) * DKH + i]);
-        const float kv = __bfloat162float(sm.k[st][(r0 + r) * DKH + i]);
+        const float qv = __bfloat162float(sm.q[st][swz64(r0 + r, i)]);
+        const float kv = __bfloat162float(sm.k[st][swz64(r0 + r, i)]);
         const float eq = qfac[r] * rq, ek = kfac[r] * rk;
         const int o = (r0 + r) * KP + i;
         sm.qf[o] = __float2bfloat16_rn(qv * eq);
@@ -318,6 +320,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     // warp -> (row block I, role): role 0 computes dq and dv of value columns
     // [0, 64); role 1 computes dk and dv of value columns [64, 128)
     const int I = warp & 3, role = warp >> 2;
+    const int Ivp = role == 0 ? I : NSB - 1 - I;  // dv row block (see below)
     const float* gch = g + (size_t)c0 * DK + i0;  // this chunk, this CTA's dims
     // in-place terms (the window branch's gradients) for this warp's outputs,
     // loaded now so that the loads overlap the products below
@@ -332,9 +335,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
           pre[nt][hh] = c0 + t < T ? *reinterpret_cast<const uint32_t*>(
                                          &src[tk + (size_t)(c0 + t) * DK + i0 + nt * 8 + gc])
                                    : 0u;
-          prev[nt][hh] = (role == half && c0 + t < T)
+          const int tv2 = 16 * Ivp + gr + 8 * hh;
+          prev[nt][hh] = (role == half && c0 + tv2 < T)
                              ? *reinterpret_cast<const uint32_t*>(
-                                   &((const bf16*)p.dv)[tv + (size_t)(c0 + t) * DV + 64 * half + nt * 8 + gc])
+                                   &((const bf16*)p.dv)[tv + (size_t)(c0 + tv2) * DV + 64 * half + nt * 8 + gc])
                              : 0u;
         }
     }
@@ -376,47 +380,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       acc[nt][2] *= f.x;
       acc[nt][3] *= f.y;
     }
-    if (role == 0) {
-      // ---- seed part of dg: column sums of q * dq_inter over these rows ------
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        const int il = nt * 8 + gc;
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int t = 16 * I + gr + 8 * hh;
-          const float2 eq = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.eqf[t * KP + il]));
-          const float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.q[st][t * DKH + il]));
-          s0 += qv.x * acc[nt][2 * hh] * eq.x;
-          s1 += qv.y * acc[nt][2 * hh + 1] * eq.y;
-        }
-#pragma unroll
-        for (int o = 4; o < 32; o <<= 1) {
-          s0 += __shfl_xor_sync(0xffffffffu, s0, o);
-          s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-        }
-        if (gr == 0) *reinterpret_cast<float2*>(&sm.qdqi[I][il]) = make_float2(s0, s1);
-      }
-    }
     // ---- intra: one 16x16 score block at a time, consumed right away -------
     const int jlo = role == 0 ? 0 : I, jhi = role == 0 ? I : NSB - 1;
     for (int J = jlo; J <= jhi; ++J) {
-      float sc[2][4];
+      float sc[2][4], sc2[2][4];  // two partial sums over k for independent MMA chains
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
-#pragma unroll 2
-      for (int kk = 0; kk < 8; ++kk) {
-        uint32_t a[4], b0, b1, b2, b3;
+        for (int e = 0; e < 4; ++e) sc[nt][e] = sc2[nt][e] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < 8; kk += 2) {
+        uint32_t a[4], b0, b1, b2, b3, c[4], d0, d1, d2, d3;
         ldsm_x4(smem_u32(&arows[(16 * I + (lane & 15)) * VP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
                 a[3]);
         ldsm_x4(smem_u32(&prows[(16 * J + (lane & 7) + ((lane >> 4) << 3)) * VP + kk * 16 +
                                 ((lane >> 3) & 1) * 8]),
                 b0, b1, b2, b3);
+        ldsm_x4(smem_u32(&arows[(16 * I + (lane & 15)) * VP + kk * 16 + 16 + (lane >> 4) * 8]), c[0], c[1],
+                c[2], c[3]);
+        ldsm_x4(smem_u32(&prows[(16 * J + (lane & 7) + ((lane >> 4) << 3)) * VP + kk * 16 + 16 +
+                                ((lane >> 3) & 1) * 8]),
+                d0, d1, d2, d3);
         mma_bf16(sc[0], a, b0, b1);
         mma_bf16(sc[1], a, b2, b3);
+        mma_bf16(sc2[0], c, d0, d1);
+        mma_bf16(sc2[1], c, d2, d3);
       }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[nt][e] += sc2[nt][e];
       if (J == I) {
         if (slow) continue;  // the diagonal block of a strong-decay chunk: below
 #pragma unroll
@@ -479,7 +472,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
           *reinterpret_cast<uint32_t*>(&((bf16*)(role == 0 ? p.dq : p.dk))[off]) = pack_bf16(y0, y1);
         }
         const float2 xv = unpack_bf16(*reinterpret_cast<const uint32_t*>(
-            &(role == 0 ? sm.q[st] : sm.k[st])[t * DKH + il]));
+            &(role == 0 ? sm.q[st] : sm.k[st])[swz64(t, il)]));
         if (role == 0) {
           *reinterpret_cast<float2*>(&sm.red[t * RP + il]) = make_float2(xv.x * x0, xv.y * x1);
         } else {
@@ -488,17 +481,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
         }
       }
 
-    // ---- partial dv of rows I, value columns [64 role, 64 role + 64) ---------
+    // ---- partial dv of row block Iv, value columns [64 role, 64 role + 64) ---
+    // (role 1 takes the mirrored row block so that every warp multiplies
+    // 5 score blocks: dq/dk of I take I+1 / 4-I, dv of Iv takes 4-Iv)
+    const int Iv = role == 0 ? I : NSB - 1 - I;
     float dvh[8][4];
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) dvh[nt][e] = 0.f;
-    // inter: (k e^{b_l - b})_I G[:, this role's columns]
+    // inter: (k e^{b_l - b})_Iv G[:, this role's columns]
 #pragma unroll
     for (int kk = 0; kk < DKH / 16; ++kk) {
       uint32_t a[4];
-      ldsm_x4(smem_u32(&sm.ks[(16 * I + (lane & 15)) * KP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
+      ldsm_x4(smem_u32(&sm.ks[(16 * Iv + (lane & 15)) * KP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
               a[3]);
 #pragma unroll
       for (int ntp = 0; ntp < 4; ++ntp) {
@@ -509,18 +505,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
         mma_bf16(dvh[2 * ntp + 1], a, b2, b3);
       }
     }
-    // intra: A^T[I][J] dO_J for J >= I, one score block at a time
-    for (int J = I; J < NSB; ++J) {
+    // intra: A^T[Iv][J] dO_J for J >= Iv, one score block at a time
+    for (int J = Iv; J < NSB; ++J) {
       float at[2][4];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) at[nt][e] = 0.f;
-      const float* fac = sm.fac[pair_index(J, I)];
+      const float* fac = sm.fac[pair_index(J, Iv)];
 #pragma unroll
       for (int kk = 0; kk < DKH / 16; ++kk) {
         uint32_t a[4];
-        ldsm_x4(smem_u32(&sm.kf[(16 * I + (lane & 15)) * KP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
+        ldsm_x4(smem_u32(&sm.kf[(16 * Iv + (lane & 15)) * KP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
                 a[3]);
         if (scaled) {
           const float2 f0 = *reinterpret_cast<const float2*>(&fac[kk * 16 + gc]);
@@ -537,13 +533,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
         mma_bf16(at[0], a, b0, b1);
         mma_bf16(at[1], a, b2, b3);
       }
-      if (J == I) {
+      if (J == Iv) {
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int t = gr + (e >> 1) * 8, u = nt * 8 + gc + (e & 1);
-            const int rt = 16 * I + t, ru = 16 * I + u;
+            const int rt = 16 * Iv + t, ru = 16 * Iv + u;
             if (u < t) at[nt][e] = 0.f;
             else if (slow) at[nt][e] = ru < rows ? diag_at_entry(sm.q[st], sm.k[st], gch, rows, rt, ru) : 0.f;
           }
@@ -561,26 +557,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       }
     }
 
-    // ---- <G, S_prev> per key dim (G still the gradient carried into the chunk)
-    {
-      float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        const int j = 64 * gnh + nt * 8 + gc;
-        const float2 s0 = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.sp[swz(16 * mt + gr, j)]));
-        const float2 s1 = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.sp[swz(16 * mt + gr + 8, j)]));
-        a0 += G[nt][0] * s0.x + G[nt][1] * s0.y;
-        a1 += G[nt][2] * s1.x + G[nt][3] * s1.y;
-      }
-      a0 += __shfl_xor_sync(0xffffffffu, a0, 1);
-      a0 += __shfl_xor_sync(0xffffffffu, a0, 2);
-      a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
-      a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
-      if ((lane & 3) == 0) {
-        sm.gsp[gnh][16 * mt + gr] = a0;
-        sm.gsp[gnh][16 * mt + gr + 8] = a1;
-      }
-    }
     // ---- carried gradient: G = diag(e^{b_l}) G + (q e^{b})^T dO --------------
     {
       const float d0 = sm.ec[16 * mt + gr], d1 = sm.ec[16 * mt + gr + 8];
@@ -606,6 +582,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
           mma_bf16(G[2 * ntp], a, b0, b1);
           mma_bf16(G[2 * ntp + 1], a, b2, b3);
         }
+      }
+    }
+    // ---- <G_new, S_prev> per key dim: dg at the chunk's first row -----------
+    {
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const int j = 64 * gnh + nt * 8 + gc;
+        const float2 s0 = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.sp[swz(16 * mt + gr, j)]));
+        const float2 s1 = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.sp[swz(16 * mt + gr + 8, j)]));
+        a0 += G[nt][0] * s0.x + G[nt][1] * s0.y;
+        a1 += G[nt][2] * s1.x + G[nt][3] * s1.y;
+      }
+      a0 += __shfl_xor_sync(0xffffffffu, a0, 1);
+      a0 += __shfl_xor_sync(0xffffffffu, a0, 2);
+      a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
+      a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
+      if ((lane & 3) == 0) {
+        sm.gsp[gnh][16 * mt + gr] = a0;
+        sm.gsp[gnh][16 * mt + gr + 8] = a1;
       }
     }
     __syncthreads();  // q*dq staged; every reader of sp, g16 and the operands is done
@@ -636,8 +632,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       }
       sm.tot[qq][col] = run;
       __syncthreads();
-      float base = sm.ec[col] * (sm.gsp[0][col] + sm.gsp[1][col]) + sm.qdqi[0][col] +
-                   sm.qdqi[1][col] + sm.qdqi[2][col] + sm.qdqi[3][col];
+      float base = sm.gsp[0][col] + sm.gsp[1][col];
 #pragma unroll
       for (int q2 = 0; q2 < NSB; ++q2)
         if (q2 < qq) base -= sm.tot[q2][col];
@@ -655,7 +650,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          const int t = 16 * I + gr + 8 * hh, cl = nt * 8 + gc;
+          const int t = 16 * Iv + gr + 8 * hh, cl = nt * 8 + gc;
           *reinterpret_cast<float2*>(&peer_red[t * RP + cl]) = make_float2(dvh[nt][2 * hh], dvh[nt][2 * hh + 1]);
         }
     }
@@ -666,7 +661,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          const int t = 16 * I + gr + 8 * hh, cl = nt * 8 + gc;
+          const int t = 16 * Iv + gr + 8 * hh, cl = nt * 8 + gc;
           if (c0 + t >= T) continue;
           const float2 pr = *reinterpret_cast<const float2*>(&sm.red[t * RP + cl]);
           float y0 = dvh[nt][2 * hh] + pr.x, y1 = dvh[nt][2 * hh + 1] + pr.y;

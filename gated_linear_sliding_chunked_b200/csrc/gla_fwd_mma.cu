@@ -40,6 +40,7 @@ constexpr int DK = 128;
 constexpr int NT = 256;
 constexpr int QKP = DK + 8;  // padded bf16 row of the ldmatrix operands
 constexpr int NPAIR = NSB * (NSB + 1) / 2;
+constexpr int PTP = C + 8;   // padded row of a query sub-block's score tile
 // a sub-block whose decay is below this in some key dim takes the
 // elementwise path for its diagonal scores
 __device__ constexpr float kMinBlockDecay = 8.75651076e-27f;  // e^-60
@@ -58,11 +59,17 @@ struct FwdSmem {
   float dec[NSB][DK];       // sub-block decays D_K
   float fac[NPAIR][DK];     // score factors F_IJ (1 for tame key dims)
   float ec[DK];             // chunk decay e^{b_l}
+  bf16 pt[NSB][SB * PTP];   // bf16 scores of each query sub-block (shared by its warp pair)
 };
 
 static_assert(sizeof(FwdSmem<64>) <= 232448, "shared memory per block exceeds 227 KB");
 
 __device__ __forceinline__ int pair_index(int I, int J) { return I * (I + 1) / 2 + J; }
+
+// barrier for the two warps (64 threads) that share query sub-block I
+__device__ __forceinline__ void pair_sync(int I) {
+  asm volatile("bar.sync %0, 64;\n" ::"r"(1 + I) : "memory");
+}
 
 // Diagonal-block score with one exponential per key dim:
 // A[t][s] = sum_i q_t,i k_s,i exp(sum_{u=s+1..t} g_u,i) for rows t, s of
@@ -270,17 +277,26 @@ __global__ void __launch_bounds__(NT, 1) gla_fwd_mma_kernel(GlaFwdParams p) {
           }
         if (K == 0) sm.ec[i2 + h2] = d0 * d1 * d2 * d3;
       }
+      if (p.o) {
 #pragma unroll
-      for (int r = 0; r < SB; ++r) {
-        const float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.q[st][(r0 + r) * DK + i2]));
-        const float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.k[st][(r0 + r) * DK + i2]));
-        const float qx = qv.x * qfac[r].x, qy = qv.y * qfac[r].y;
-        const float kx = kv.x * kfac[r].x, ky = kv.y * kfac[r].y;
-        const int o = (r0 + r) * QKP + i2;
-        *reinterpret_cast<uint32_t*>(&sm.qf[o]) = pack_bf16(qx * rq[0], qy * rq[1]);
-        *reinterpret_cast<uint32_t*>(&sm.qi[o]) = pack_bf16(qx * eqk[0], qy * eqk[1]);
-        *reinterpret_cast<uint32_t*>(&sm.kf[o]) = pack_bf16(kx * rk[0], ky * rk[1]);
-        *reinterpret_cast<uint32_t*>(&sm.ks[o]) = pack_bf16(kx * ksk[0], ky * ksk[1]);
+        for (int r = 0; r < SB; ++r) {
+          const float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.q[st][(r0 + r) * DK + i2]));
+          const float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.k[st][(r0 + r) * DK + i2]));
+          const float qx = qv.x * qfac[r].x, qy = qv.y * qfac[r].y;
+          const float kx = kv.x * kfac[r].x, ky = kv.y * kfac[r].y;
+          const int o = (r0 + r) * QKP + i2;
+          *reinterpret_cast<uint32_t*>(&sm.qf[o]) = pack_bf16(qx * rq[0], qy * rq[1]);
+          *reinterpret_cast<uint32_t*>(&sm.qi[o]) = pack_bf16(qx * eqk[0], qy * eqk[1]);
+          *reinterpret_cast<uint32_t*>(&sm.kf[o]) = pack_bf16(kx * rk[0], ky * rk[1]);
+          *reinterpret_cast<uint32_t*>(&sm.ks[o]) = pack_bf16(kx * ksk[0], ky * ksk[1]);
+        }
+      } else {  // state pass: only the state-update key operand
+#pragma unroll
+        for (int r = 0; r < SB; ++r) {
+          const float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.k[st][(r0 + r) * DK + i2]));
+          *reinterpret_cast<uint32_t*>(&sm.ks[(r0 + r) * QKP + i2]) =
+              pack_bf16(kv.x * kfac[r].x * ksk[0], kv.y * kfac[r].y * ksk[1]);
+        }
       }
       const int w = __syncthreads_or(any_wild);
       const int b = __syncthreads_or(wild_bad);
@@ -319,8 +335,9 @@ __global__ void __launch_bounds__(NT, 1) gla_fwd_mma_kernel(GlaFwdParams p) {
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
           for (int e = 0; e < 4; ++e) acc[J][nt][e] = 0.f;
-        if (J > I) continue;
+        if (J > I || (J & 1) != nh) continue;  // the pair splits the score blocks
         const float* fac = sm.fac[pair_index(I, J)];
+        float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // odd k steps
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
           uint32_t a[4] = {qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]};
@@ -336,9 +353,14 @@ __global__ void __launch_bounds__(NT, 1) gla_fwd_mma_kernel(GlaFwdParams p) {
           ldsm_x4(smem_u32(&sm.kf[(16 * J + (lane & 7) + ((lane >> 4) << 3)) * QKP + kk * 16 +
                                   ((lane >> 3) & 1) * 8]),
                   b0, b1, b2, b3);
-          mma_bf16(acc[J][0], a, b0, b1);
-          mma_bf16(acc[J][1], a, b2, b3);
+          float (*dst)[4] = (kk & 1) ? acc2 : acc[J];
+          mma_bf16(dst[0], a, b0, b1);
+          mma_bf16(dst[1], a, b2, b3);
         }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[J][nt][e] += acc2[nt][e];
         if (J == I) {
           if (slow) {
 #pragma unroll
@@ -367,14 +389,25 @@ __global__ void __launch_bounds__(NT, 1) gla_fwd_mma_kernel(GlaFwdParams p) {
       for (int nt = 0; nt < ONT; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+      // share this warp's score blocks with its pair through shared memory
+      bf16* pt = sm.pt[I];
+#pragma unroll
+      for (int J = 0; J < NSB; ++J) {
+        if (J > I || (J & 1) != nh) continue;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+            *reinterpret_cast<uint32_t*>(&pt[(gr + 8 * hh) * PTP + 16 * J + nt * 8 + gc]) =
+                pack_bf16(acc[J][nt][2 * hh], acc[J][nt][2 * hh + 1]);
+      }
+      pair_sync(I);
       // intra: P V over the key sub-blocks J <= I
 #pragma unroll
       for (int J = 0; J < NSB; ++J) {
         if (J > I) continue;
-        const uint32_t pa[4] = {pack_bf16(acc[J][0][0], acc[J][0][1]),
-                                pack_bf16(acc[J][0][2], acc[J][0][3]),
-                                pack_bf16(acc[J][1][0], acc[J][1][1]),
-                                pack_bf16(acc[J][1][2], acc[J][1][3])};
+        uint32_t pa[4];
+        ldsm_x4(smem_u32(&pt[(lane & 15) * PTP + 16 * J + (lane >> 4) * 8]), pa[0], pa[1], pa[2], pa[3]);
 #pragma unroll
         for (int ntp = 0; ntp < ONT / 2; ++ntp) {
           uint32_t b0, b1, b2, b3;
