@@ -1,0 +1,506 @@
+// Two-pass chunked gated linear attention forward on the tensor cores (bf16
+// I/O, fp32 accumulation, dk = dv = 128).
+//
+// Recurrence (Lizard technical summary, section 2a, state update equation):
+//   S_t = diag(exp(g_t)) S_{t-1} + k_t v_t^T,   o_t = q_t^T S_t.
+// Over 64-token chunks with b_t the running log-gate inside the chunk and b_l
+// its last value:
+//   S_next = diag(e^{b_l}) S_prev + sum_s (k_s e^{b_l - b_s}) v_s^T
+//   o_t    = (q_t e^{b_t})^T S_prev + sum_{s<=t} A[t][s] v_s,
+//   A[t][s] = sum_i q_t,i k_s,i e^{b_t,i - b_s,i}.
+// Only the state carries a dependence between chunks, so the work is split:
+//   pass 1 (gla_states_kernel): one CTA per (batch, head, 32 value columns)
+//     walks the chunks and writes the bf16 state before every chunk (and the
+//     final fp32 state);
+//   pass 2 (gla_out_kernel): one CTA per (chunk, batch, head) computes the
+//     chunk's outputs from its incoming state, all chunks in parallel.
+// Gate factors are the bounded ones of the single-pass kernel: per key dim
+// one reference row when each 32-row half decays by at most e^-60 ("tame"),
+// else 16-row sub-block references with per-pair factors F_IJ; diagonal
+// blocks that decay past e^-60 take exp(b_t - b_s) per element.
+#include "common.cuh"
+#include "kernels.h"
+#include "mma.cuh"
+
+namespace lz {
+namespace {
+
+constexpr int C = 64;
+constexpr int SB = 16;
+constexpr int NSB = C / SB;
+constexpr int DK = 128;
+constexpr int DV = 128;
+constexpr int NT = 256;
+constexpr int QKP = DK + 8;
+constexpr int VP = DV + 8;
+constexpr int NPAIR = NSB * (NSB + 1) / 2;
+__device__ constexpr float kMinBlockDecay = 8.75651076e-27f;  // e^-60
+
+__device__ __forceinline__ int pair_index(int I, int J) { return I * (I + 1) / 2 + J; }
+
+// ===========================================================================
+// Pass 1: the state walk
+// ===========================================================================
+constexpr int DVS = 32;          // value columns per CTA
+constexpr int SVP = DVS + 8;     // padded row of the v slice
+
+struct StateSmem {
+  bf16 k[2][C * DK];
+  bf16 v[2][C * SVP];
+  float g[C * DK];
+  bf16 ks[C * QKP];              // k e^{b_l - b}
+  float dec[NSB][DK];
+  float ec[DK];
+};
+static_assert(sizeof(StateSmem) <= 115712, "two state-pass CTAs must fit one SM");
+
+__global__ void __launch_bounds__(NT, 2) gla_states_kernel(GlaFwdParams p) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  StateSmem& sm = *reinterpret_cast<StateSmem*>(smem_raw);
+  constexpr int SNT = DVS / 8;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gr = lane >> 2, gc = (lane & 3) * 2;
+  const int j0 = blockIdx.x * DVS;
+  const int bh = blockIdx.y;
+  const int T = p.T;
+  const bf16* k = (const bf16*)p.k + (size_t)bh * T * DK;
+  const bf16* v = (const bf16*)p.v + (size_t)bh * T * DV;
+  const float* g = p.g + (size_t)bh * T * DK;
+  const int nchunks = (T + C - 1) / C;
+
+  auto issue_kv = [&](int c, int st) {
+    const int c0 = c * C;
+    for (int x = tid; x < C * DK / 8; x += NT) {
+      const int r = x / (DK / 8), cc = x % (DK / 8);
+      const bool ok = c0 + r < T;
+      cp_async16(&sm.k[st][r * DK + cc * 8], k + (size_t)(ok ? c0 + r : 0) * DK + cc * 8, ok ? 16 : 0);
+    }
+    for (int x = tid; x < C * DVS / 8; x += NT) {
+      const int r = x / (DVS / 8), cc = x % (DVS / 8);
+      const bool ok = c0 + r < T;
+      cp_async16(&sm.v[st][r * SVP + cc * 8], v + (size_t)(ok ? c0 + r : 0) * DV + j0 + cc * 8,
+                 ok ? 16 : 0);
+    }
+    cp_async_commit();
+  };
+  auto issue_g = [&](int c) {
+    const int c0 = c * C;
+    for (int x = tid; x < C * DK / 4; x += NT) {
+      const int r = x / (DK / 4), cc = x % (DK / 4);
+      const bool ok = c0 + r < T;
+      cp_async16(&sm.g[r * DK + cc * 4], g + (size_t)(ok ? c0 + r : 0) * DK + cc * 4, ok ? 16 : 0);
+    }
+    cp_async_commit();
+  };
+
+  // state rows 16w .. 16w+15, this CTA's 32 value columns, fp32 in registers
+  float s[SNT][4];
+#pragma unroll
+  for (int nt = 0; nt < SNT; ++nt)
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int i = 16 * warp + gr + 8 * hh, j = j0 + nt * 8 + gc;
+      float a = 0.f, b = 0.f;
+      if (p.h0) {
+        const float* hp = p.h0 + ((size_t)bh * DK + i) * DV + j;
+        a = hp[0];
+        b = hp[1];
+      }
+      s[nt][2 * hh] = a;
+      s[nt][2 * hh + 1] = b;
+    }
+
+  if (nchunks > 0) {
+    issue_kv(0, 0);
+    issue_g(0);
+  }
+  for (int c = 0; c < nchunks; ++c) {
+    const int st = c & 1;
+    cp_async_wait<0>();
+    __syncthreads();
+    if (c + 1 < nchunks) issue_kv(c + 1, st ^ 1);
+    {  // state before this chunk
+      bf16* dst = (bf16*)p.states16 + ((size_t)bh * nchunks + c) * DK * DV + j0;
+#pragma unroll
+      for (int nt = 0; nt < SNT; ++nt)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int i = 16 * warp + gr + 8 * hh, j = nt * 8 + gc;
+          *reinterpret_cast<uint32_t*>(&dst[(size_t)i * DV + j]) = pack_bf16(s[nt][2 * hh], s[nt][2 * hh + 1]);
+        }
+    }
+    // prep: thread -> (sub-block K, key dims i2, i2+1); k side only
+    const int K = tid >> 6, i2 = (tid & 63) * 2, r0 = K * SB;
+    float2 kfac[SB];
+    {
+      float2 run = make_float2(1.f, 1.f);
+#pragma unroll
+      for (int r = SB - 1; r >= 0; --r) {  // prod_{u = r+1 .. end} e_u
+        kfac[r] = run;
+        const float2 gg = *reinterpret_cast<const float2*>(&sm.g[(r0 + r) * DK + i2]);
+        run.x *= __expf(gg.x);
+        run.y *= __expf(gg.y);
+      }
+      *reinterpret_cast<float2*>(&sm.dec[K][i2]) = run;
+    }
+    __syncthreads();
+    if (c + 1 < nchunks) issue_g(c + 1);
+    {
+      float2 f = make_float2(1.f, 1.f);
+#pragma unroll
+      for (int J = 0; J < NSB; ++J)
+        if (J > K) {
+          const float2 d = *reinterpret_cast<const float2*>(&sm.dec[J][i2]);
+          f.x *= d.x;
+          f.y *= d.y;
+        }
+      if (K == 0) {
+        float2 e = make_float2(1.f, 1.f);
+#pragma unroll
+        for (int J = 0; J < NSB; ++J) {
+          const float2 d = *reinterpret_cast<const float2*>(&sm.dec[J][i2]);
+          e.x *= d.x;
+          e.y *= d.y;
+        }
+        *reinterpret_cast<float2*>(&sm.ec[i2]) = e;
+      }
+#pragma unroll
+      for (int r = 0; r < SB; ++r) {
+        const float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.k[st][(r0 + r) * DK + i2]));
+        *reinterpret_cast<uint32_t*>(&sm.ks[(r0 + r) * QKP + i2]) =
+            pack_bf16(kv.x * kfac[r].x * f.x, kv.y * kfac[r].y * f.y);
+      }
+    }
+    __syncthreads();
+    // S = diag(e^{b_l}) S + Ks^T V
+    {
+      const float d0 = sm.ec[16 * warp + gr], d1 = sm.ec[16 * warp + gr + 8];
+#pragma unroll
+      for (int nt = 0; nt < SNT; ++nt) {
+        s[nt][0] *= d0;
+        s[nt][1] *= d0;
+        s[nt][2] *= d1;
+        s[nt][3] *= d1;
+      }
+#pragma unroll
+      for (int kk = 0; kk < C / 16; ++kk) {
+        uint32_t a[4];
+        ldsm_x4_t(smem_u32(&sm.ks[(16 * kk + (lane & 7) + ((lane >> 4) << 3)) * QKP + 16 * warp +
+                                  ((lane >> 3) & 1) * 8]),
+                  a[0], a[1], a[2], a[3]);
+#pragma unroll
+        for (int ntp = 0; ntp < SNT / 2; ++ntp) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(smem_u32(&sm.v[st][(16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8) * SVP + ntp * 16 +
+                                       (lane >> 4) * 8]),
+                    b0, b1, b2, b3);
+          mma_bf16(s[2 * ntp], a, b0, b1);
+          mma_bf16(s[2 * ntp + 1], a, b2, b3);
+        }
+      }
+    }
+  }
+  if (p.hT) {
+#pragma unroll
+    for (int nt = 0; nt < SNT; ++nt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int i = 16 * warp + gr + 8 * hh, j = j0 + nt * 8 + gc;
+        *reinterpret_cast<float2*>(&p.hT[((size_t)bh * DK + i) * DV + j]) =
+            make_float2(s[nt][2 * hh], s[nt][2 * hh + 1]);
+      }
+  }
+}
+
+// ===========================================================================
+// Pass 2: chunk outputs, all chunks in parallel
+// ===========================================================================
+struct OutSmem {
+  bf16 q[C * QKP];     // raw q, then the score operand Qf in place
+  bf16 k[C * QKP];     // raw k, then Kf in place
+  bf16 qi[C * QKP];    // q e^{b}
+  bf16 v[C * VP];
+  bf16 sp[DK * VP];    // state before the chunk
+  float dec[NSB][DK];
+  float fac[NPAIR][DK];
+};
+static_assert(sizeof(OutSmem) <= 115712, "two output CTAs must fit one SM");
+
+// A[t][s] with one exponential per key dim (strong-decay diagonal blocks);
+// q, k, g: global rows of the chunk.
+__device__ __noinline__ float diag_score_global(const bf16* q, const bf16* k, const float* g, int rt,
+                                                int rs) {
+  float a = 0.f;
+  for (int i = 0; i < DK; ++i) {
+    float lg = 0.f;
+    for (int u = rs + 1; u <= rt; ++u) lg += g[(size_t)u * DK + i];
+    a += __bfloat162float(q[(size_t)rt * DK + i]) * __bfloat162float(k[(size_t)rs * DK + i]) * __expf(lg);
+  }
+  return a;
+}
+
+__global__ void __launch_bounds__(NT, 2) gla_out_kernel(GlaFwdParams p) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  OutSmem& sm = *reinterpret_cast<OutSmem*>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gr = lane >> 2, gc = (lane & 3) * 2;
+  const int c = blockIdx.x, bh = blockIdx.y;
+  const int T = p.T;
+  const int c0 = c * C;
+  const int rows = min(C, T - c0);
+  const int nchunks = gridDim.x;
+  const bf16* q = (const bf16*)p.q + ((size_t)bh * T + c0) * DK;
+  const bf16* k = (const bf16*)p.k + ((size_t)bh * T + c0) * DK;
+  const bf16* v = (const bf16*)p.v + ((size_t)bh * T + c0) * DV;
+  const float* g = p.g + ((size_t)bh * T + c0) * DK;
+  const bf16* sp = (const bf16*)p.states16 + ((size_t)bh * nchunks + c) * DK * DV;
+
+  for (int x = tid; x < C * DK / 8; x += NT) {
+    const int r = x / (DK / 8), cc = x % (DK / 8);
+    const bool ok = r < rows;
+    const size_t off = (size_t)(ok ? r : 0) * DK + cc * 8;
+    cp_async16(&sm.q[r * QKP + cc * 8], q + off, ok ? 16 : 0);
+    cp_async16(&sm.k[r * QKP + cc * 8], k + off, ok ? 16 : 0);
+  }
+  for (int x = tid; x < C * DV / 8; x += NT) {
+    const int r = x / (DV / 8), cc = x % (DV / 8);
+    const bool ok = r < rows;
+    cp_async16(&sm.v[r * VP + cc * 8], v + (size_t)(ok ? r : 0) * DV + cc * 8, ok ? 16 : 0);
+  }
+  for (int x = tid; x < DK * DV / 8; x += NT) {
+    const int r = x / (DV / 8), cc = x % (DV / 8);
+    cp_async16(&sm.sp[r * VP + cc * 8], sp + (size_t)r * DV + cc * 8, 16);
+  }
+  cp_async_commit();
+
+  // ---- prep 1 (gates straight from global): thread -> (sub-block K, dims i2, i2+1)
+  const int K = tid >> 6, i2 = (tid & 63) * 2, r0 = K * SB;
+  float2 qfac[SB], kfac[SB];
+  {
+    float2 e[SB];
+#pragma unroll
+    for (int r = 0; r < SB; ++r) {
+      const float2 gg = r0 + r < rows ? *reinterpret_cast<const float2*>(&g[(size_t)(r0 + r) * DK + i2])
+                                      : make_float2(0.f, 0.f);
+      e[r] = make_float2(__expf(gg.x), __expf(gg.y));
+    }
+    float2 run = make_float2(1.f, 1.f);
+#pragma unroll
+    for (int r = SB - 1; r >= 0; --r) {
+      kfac[r] = run;
+      run.x *= e[r].x;
+      run.y *= e[r].y;
+    }
+    run = make_float2(1.f, 1.f);
+#pragma unroll
+    for (int r = 0; r < SB; ++r) {
+      run.x *= e[r].x;
+      run.y *= e[r].y;
+      qfac[r] = run;
+    }
+    *reinterpret_cast<float2*>(&sm.dec[K][i2]) = run;
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  // ---- prep 2: operands and score factors ----------------------------------
+  int flags;
+  {
+    float2 D[NSB];
+#pragma unroll
+    for (int J = 0; J < NSB; ++J) D[J] = *reinterpret_cast<const float2*>(&sm.dec[J][i2]);
+    bool wild_bad = false, any_wild = false;
+    float rq[2], rk[2], eqk[2];
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const float d0 = h2 ? D[0].y : D[0].x, d1 = h2 ? D[1].y : D[1].x;
+      const float d2 = h2 ? D[2].y : D[2].x, d3 = h2 ? D[3].y : D[3].x;
+      const bool tame = (d0 * d1 >= kMinBlockDecay) && (d2 * d3 >= kMinBlockDecay);
+      any_wild |= !tame;
+      if (!tame)
+        wild_bad |= !(d0 >= kMinBlockDecay && d1 >= kMinBlockDecay && d2 >= kMinBlockDecay &&
+                      d3 >= kMinBlockDecay);
+      const float dk[NSB] = {d0, d1, d2, d3};
+      float rqK = 1.f, rkK = 1.f;
+      if (tame) {
+        rqK = K == 0 ? 1.f / (d0 * d1) : K == 1 ? 1.f / d1 : K == 2 ? 1.f : d2;
+        rkK = K == 0 ? d1 : K == 1 ? 1.f : K == 2 ? 1.f / d2 : 1.f / (d2 * d3);
+      }
+      float eq = 1.f;
+#pragma unroll
+      for (int J = 0; J < NSB; ++J)
+        if (J < K) eq *= dk[J];
+      rq[h2] = rqK;
+      rk[h2] = rkK;
+      eqk[h2] = eq;
+#pragma unroll
+      for (int I = 0; I < NSB; ++I)
+#pragma unroll
+        for (int J = 0; J <= I; ++J) {
+          if (pair_index(I, J) % NSB != K) continue;
+          float f = 1.f;
+          if (!tame) {
+            if (J == I) {
+              f = 1.f / fmaxf(dk[I], 1e-30f);
+            } else {
+#pragma unroll
+              for (int Kp = 0; Kp < NSB; ++Kp)
+                if (Kp > J && Kp < I) f *= dk[Kp];
+            }
+          }
+          sm.fac[pair_index(I, J)][i2 + h2] = f;
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < SB; ++r) {
+      const int o = (r0 + r) * QKP + i2;
+      const float2 qv = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.q[o]));
+      const float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.k[o]));
+      const float qx = qv.x * qfac[r].x, qy = qv.y * qfac[r].y;
+      const float kx = kv.x * kfac[r].x, ky = kv.y * kfac[r].y;
+      *reinterpret_cast<uint32_t*>(&sm.q[o]) = pack_bf16(qx * rq[0], qy * rq[1]);
+      *reinterpret_cast<uint32_t*>(&sm.qi[o]) = pack_bf16(qx * eqk[0], qy * eqk[1]);
+      *reinterpret_cast<uint32_t*>(&sm.k[o]) = pack_bf16(kx * rk[0], ky * rk[1]);
+    }
+    const int w = __syncthreads_or(any_wild);
+    const int b = __syncthreads_or(wild_bad);
+    flags = (w ? 1 : 0) | (b ? 2 : 0);
+  }
+  const bool scaled = flags & 1, slow = flags & 2;
+
+  // ---- outputs: warp -> (query sub-block I, value half nh) --------------------
+  const int I = warp >> 1, nh = warp & 1;
+  float2 addv[8][2];
+  if (p.add16) {
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int t = 16 * I + gr + 8 * hh;
+        addv[nt][hh] = t < rows ? unpack_bf16(*reinterpret_cast<const uint32_t*>(
+                                      &((const bf16*)p.add16)[((size_t)bh * T + c0 + t) * DV + 64 * nh + nt * 8 + gc]))
+                                : make_float2(0.f, 0.f);
+      }
+  }
+  float o[8][4];
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+  // inter: (q e^{b}) S_prev
+#pragma unroll 2
+  for (int kk = 0; kk < DK / 16; ++kk) {
+    uint32_t a[4];
+    ldsm_x4(smem_u32(&sm.qi[(16 * I + (lane & 15)) * QKP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
+            a[3]);
+#pragma unroll
+    for (int ntp = 0; ntp < 4; ++ntp) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(smem_u32(&sm.sp[(16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8) * VP + 64 * nh + ntp * 16 +
+                                (lane >> 4) * 8]),
+                b0, b1, b2, b3);
+      mma_bf16(o[2 * ntp], a, b0, b1);
+      mma_bf16(o[2 * ntp + 1], a, b2, b3);
+    }
+  }
+  // intra: one score block at a time (J <= I), P V right away
+  for (int J = 0; J <= I; ++J) {
+    float sc[2][4], sc2[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sc[nt][e] = sc2[nt][e] = 0.f;
+    const float* fac = sm.fac[pair_index(I, J)];
+#pragma unroll
+    for (int kk = 0; kk < DK / 16; ++kk) {
+      uint32_t a[4];
+      ldsm_x4(smem_u32(&sm.q[(16 * I + (lane & 15)) * QKP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
+              a[3]);
+      if (scaled) {
+        const float2 f0 = *reinterpret_cast<const float2*>(&fac[kk * 16 + gc]);
+        const float2 f1 = *reinterpret_cast<const float2*>(&fac[kk * 16 + 8 + gc]);
+        a[0] = scale_bf16x2(a[0], f0.x, f0.y);
+        a[1] = scale_bf16x2(a[1], f0.x, f0.y);
+        a[2] = scale_bf16x2(a[2], f1.x, f1.y);
+        a[3] = scale_bf16x2(a[3], f1.x, f1.y);
+      }
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(smem_u32(&sm.k[(16 * J + (lane & 7) + ((lane >> 4) << 3)) * QKP + kk * 16 +
+                             ((lane >> 3) & 1) * 8]),
+              b0, b1, b2, b3);
+      float (*dst)[4] = (kk & 1) ? sc2 : sc;
+      mma_bf16(dst[0], a, b0, b1);
+      mma_bf16(dst[1], a, b2, b3);
+    }
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int t = gr + (e >> 1) * 8, sk = nt * 8 + gc + (e & 1);
+        float x = sc[nt][e] + sc2[nt][e];
+        if (J == I) {
+          if (sk > t) x = 0.f;
+          else if (slow) x = 16 * I + t < rows ? diag_score_global(q, k, g, 16 * I + t, 16 * I + sk) : 0.f;
+        }
+        sc[nt][e] = x;
+      }
+    const uint32_t pa[4] = {pack_bf16(sc[0][0], sc[0][1]), pack_bf16(sc[0][2], sc[0][3]),
+                            pack_bf16(sc[1][0], sc[1][1]), pack_bf16(sc[1][2], sc[1][3])};
+#pragma unroll
+    for (int ntp = 0; ntp < 4; ++ntp) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(smem_u32(&sm.v[(16 * J + (lane & 7) + ((lane >> 3) & 1) * 8) * VP + 64 * nh + ntp * 16 +
+                               (lane >> 4) * 8]),
+                b0, b1, b2, b3);
+      mma_bf16(o[2 * ntp], pa, b0, b1);
+      mma_bf16(o[2 * ntp + 1], pa, b2, b3);
+    }
+  }
+  // epilogue: o = o_gla + alpha * add
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int t = 16 * I + gr + 8 * hh;
+      if (t >= rows) continue;
+      const size_t off = ((size_t)bh * T + c0 + t) * DV + 64 * nh + nt * 8 + gc;
+      float x0 = o[nt][2 * hh], x1 = o[nt][2 * hh + 1];
+      if (p.add16) {
+        x0 += p.alpha * addv[nt][hh].x;
+        x1 += p.alpha * addv[nt][hh].y;
+      }
+      *reinterpret_cast<uint32_t*>(&((bf16*)p.o)[off]) = pack_bf16(x0, x1);
+    }
+}
+
+}  // namespace
+
+bool gla_chunk_mma_supported(int dk, int dv, bool bf16) { return bf16 && dk == DK && dv == DV; }
+
+cudaError_t launch_gla_states(const GlaFwdParams& p, cudaStream_t s) {
+  if (p.B * p.H == 0) return cudaSuccess;
+  const size_t bytes = sizeof(StateSmem);
+  cudaError_t e = cudaFuncSetAttribute(gla_states_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)bytes);
+  if (e != cudaSuccess) return e;
+  {
+    ScopedTiming tm("gla_states_mma", s);
+    gla_states_kernel<<<dim3(DV / DVS, p.B * p.H), NT, bytes, s>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gla_out(const GlaFwdParams& p, cudaStream_t s) {
+  const int nchunks = (p.T + C - 1) / C;
+  if (p.B * p.H == 0 || nchunks == 0) return cudaSuccess;
+  const size_t bytes = sizeof(OutSmem);
+  cudaError_t e =
+      cudaFuncSetAttribute(gla_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  {
+    ScopedTiming tm("gla_out_mma", s);
+    gla_out_kernel<<<dim3(nchunks, p.B * p.H), NT, bytes, s>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace lz

@@ -76,6 +76,14 @@ struct GlaBwdParams {
 };
 cudaError_t launch_gla_bwd_simt(const GlaBwdParams& p, bool bf16, cudaStream_t s);
 
+// ---- gated branch, two-pass tensor-core forward (bf16, dk = dv = 128) -----
+// launch_gla_states writes states16 ([BH][ceil(T/64)][dk][dv] bf16, the state
+// before every 64-token chunk) and hT; launch_gla_out then computes o (adding
+// alpha * add16 when set) from them, all chunks in parallel.
+bool gla_chunk_mma_supported(int dk, int dv, bool bf16);
+cudaError_t launch_gla_states(const GlaFwdParams& p, cudaStream_t s);
+cudaError_t launch_gla_out(const GlaFwdParams& p, cudaStream_t s);
+
 // ---- gated branch, tensor-core backward (bf16 I/O, dk = dv = 128) --------
 // Needs states16 and hT from the tensor-core forward run as a state pass.
 bool gla_bwd_mma_supported(int dk, int dv, bool bf16);

@@ -25,9 +25,17 @@ cudaError_t swa_backward(const lz::SwaBwdParams& p, bool bf16, cudaStream_t s) {
   return lz::launch_swa_bwd_simt(p, bf16, s);
 }
 
-// The forward of the gated branch: tensor cores for bf16 with dk = 128,
-// fp32 SIMT otherwise.
-cudaError_t gla_forward(const lz::GlaFwdParams& p, bool bf16, cudaStream_t s) {
+// The forward of the gated branch.  bf16 with dk = dv = 128: a state pass
+// (bf16 states into `states16` scratch) then all chunks' outputs in
+// parallel; bf16 with dk = 128 and other dv: the single-pass tensor-core
+// kernel; otherwise fp32 SIMT.
+cudaError_t gla_forward(lz::GlaFwdParams p, bool bf16, void* states16, cudaStream_t s) {
+  if (lz::gla_chunk_mma_supported(p.dk, p.dv, bf16)) {
+    p.states16 = states16;
+    cudaError_t e = lz::launch_gla_states(p, s);
+    if (e != cudaSuccess) return e;
+    return lz::launch_gla_out(p, s);
+  }
   if (p.o && lz::gla_fwd_mma_supported(p.dk, p.dv, bf16)) return lz::launch_gla_fwd_mma(p, s);
   return lz::launch_gla_fwd_simt(p, bf16, s);
 }
@@ -126,6 +134,15 @@ lz_status check_dims(const lz_dims* d, bool need_window) {
 }
 
 size_t bht(const lz_dims* d) { return (size_t)d->B * d->H * d->T; }
+
+bool fwd_uses_chunks(const lz_dims* d) {
+  return lz::gla_chunk_mma_supported(d->dk, d->dv, d->io == LZ_BF16);
+}
+// bf16 state before every 64-token chunk (two-pass forward, tensor-core backward)
+size_t states16_count(const lz_dims* d) {
+  const size_t n64 = (size_t)((d->T + lz::gla_fwd_mma_chunk() - 1) / lz::gla_fwd_mma_chunk());
+  return (size_t)d->B * d->H * n64 * d->dk * d->dv;
+}
 size_t nchunks16(const lz_dims* d) {
   return (size_t)((d->T + lz::kSimtChunk - 1) / lz::kSimtChunk);
 }
@@ -155,8 +172,7 @@ GlaBwdWs carve_gla_bwd(Carver& c, const lz_dims* d) {
   GlaBwdWs w{};
   const size_t bh = (size_t)d->B * d->H;
   if (bwd_uses_mma(d)) {
-    const size_t n64 = (size_t)((d->T + lz::gla_fwd_mma_chunk() - 1) / lz::gla_fwd_mma_chunk());
-    w.states16 = c.take<uint16_t>(bh * n64 * d->dk * d->dv);  // bf16
+    w.states16 = c.take<uint16_t>(states16_count(d));  // bf16
   } else {
     w.states = c.take<float>(bh * nchunks16(d) * d->dk * d->dv);
   }
@@ -201,9 +217,11 @@ size_t ws_bytes(const lz_dims* d, int which) {
   Carver c(nullptr);
   switch (which) {
     case LZ_WS_GLA_FWD:
-      return 0;
+      if (fwd_uses_chunks(d)) c.take<uint16_t>(states16_count(d));
+      return c.off;
     case LZ_WS_HYBRID_FWD:
       if (!hybrid_uses_mma(d)) c.take<float>(bht(d) * d->dv);  // fp32 window output
+      if (fwd_uses_chunks(d)) c.take<uint16_t>(states16_count(d));
       return c.off;
     case LZ_WS_GLA_BWD:
       carve_gla_bwd(c, d);
@@ -284,7 +302,9 @@ lz_status lz_gla_fwd(const lz_dims* d, const void* q, const void* k, const void*
   lz::GlaFwdParams p = gla_fwd_params(d, q, k, v, g, h0);
   p.o = o;
   p.hT = hT;
-  return cuda_status(gla_forward(p, d->io == LZ_BF16, as_stream(stream)), "lz_gla_fwd");
+  Carver c(ws);
+  void* states16 = fwd_uses_chunks(d) ? c.take<uint16_t>(states16_count(d)) : nullptr;
+  return cuda_status(gla_forward(p, d->io == LZ_BF16, states16, as_stream(stream)), "lz_gla_fwd");
 }
 
 lz_status lz_swa_meta_fwd(const lz_dims* d, const void* q, const void* k, const void* v,
@@ -318,6 +338,7 @@ lz_status lz_hybrid_fwd(const lz_dims* d, const void* q, const void* k, const vo
   const bool mma = hybrid_uses_mma(d);
   Carver c(ws);
   float* osw = mma ? nullptr : c.take<float>(bht(d) * d->dv);
+  void* states16 = fwd_uses_chunks(d) ? c.take<uint16_t>(states16_count(d)) : nullptr;
   lz::SwaFwdParams sp = swa_fwd_params(d, q, k, v, meta_k, meta_v);
   // tensor-core path: bf16 window output into o_swa if requested, else into o
   sp.o = mma ? (o_swa ? o_swa : o) : o_swa;
@@ -331,7 +352,7 @@ lz_status lz_hybrid_fwd(const lz_dims* d, const void* q, const void* k, const vo
   gp.add = osw;
   gp.add16 = mma ? sp.o : nullptr;
   gp.alpha = d->alpha;
-  return cuda_status(gla_forward(gp, bf, s), "lz_hybrid_fwd (gated branch)");
+  return cuda_status(gla_forward(gp, bf, states16, s), "lz_hybrid_fwd (gated branch)");
 }
 
 static cudaError_t gla_bwd_launch(const lz_dims* d, const void* q, const void* k, const void* v,
@@ -346,7 +367,7 @@ static cudaError_t gla_bwd_launch(const lz_dims* d, const void* q, const void* k
   fp.states = w.states;
   fp.states16 = w.states16;
   fp.hT = w.hT;
-  cudaError_t e = mma ? lz::launch_gla_fwd_mma(fp, s) : lz::launch_gla_fwd_simt(fp, bf, s);
+  cudaError_t e = mma ? lz::launch_gla_states(fp, s) : lz::launch_gla_fwd_simt(fp, bf, s);
   if (e != cudaSuccess) return e;
   lz::GlaBwdParams p{};
   p.q = q; p.k = k; p.v = v; p.g = g; p.dO = dO; p.dhT = dhT;
