@@ -204,6 +204,7 @@ class TrainStep:
         dt = wl.torch_dtype
         mk = lambda *s, dtype=dt: torch.empty(*s, dtype=dtype, device=device)
         self.o = mk(B, H, T, dv)
+        self.osw = mk(B, H, T, dv)  # window output saved for the backward
         self.lse = mk(B, H, T, dtype=torch.float32)
         self.dq, self.dk, self.dv = mk(B, H, T, dk), mk(B, H, T, dk), mk(B, H, T, dv)
         self.dg = mk(B, H, T, dk, dtype=torch.float32)
@@ -219,9 +220,9 @@ class TrainStep:
         x = x or self.x
         L, d = self.L, self.dims
         L.lz_hybrid_fwd(d, x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], None,
-                        self.o, None, self.lse, None, self.wsf, self.nf)
+                        self.o, None, self.lse, self.osw, self.wsf, self.nf)
         L.lz_hybrid_bwd(d, x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], None,
-                        self.lse, x["dO"], None, self.dq, self.dk, self.dv, self.dg, None,
+                        self.lse, self.osw, x["dO"], None, self.dq, self.dk, self.dv, self.dg, None,
                         self.dmk, self.dmv, self.dalpha, self.wsb, self.nb)
 
     def outputs(self):

@@ -70,9 +70,9 @@ def load(path: str = LIB_PATH):
     lib.lz_swa_meta_fwd.argtypes = [D] + [_P] * 7 + [_P]
     lib.lz_hybrid_fwd.argtypes = [D] + [_P] * 11 + [_P, sz, _P]
     lib.lz_gla_bwd.argtypes = [D] + [_P] * 12 + [_P, sz, _P]
-    lib.lz_swa_meta_bwd.argtypes = [D] + [_P] * 12 + [_P, sz, _P]
-    lib.lz_hybrid_bwd.argtypes = [D] + [_P] * 18 + [_P, sz, _P]
-    lib.lz_swa_meta_bwd_noalloc.argtypes = [D] + [_P] * 12 + [_P]
+    lib.lz_swa_meta_bwd.argtypes = [D] + [_P] * 13 + [_P, sz, _P]
+    lib.lz_hybrid_bwd.argtypes = [D] + [_P] * 19 + [_P, sz, _P]
+    lib.lz_swa_meta_bwd_noalloc.argtypes = [D] + [_P] * 13 + [_P]
     lib.lz_gla_decode_step.argtypes = ([ctypes.c_int] * 7 + [ctypes.c_float] * 2 +
                                        [_P] * 11 + [_P])
     lib.lz_timing_enable.argtypes = [ctypes.c_int]
@@ -172,30 +172,32 @@ def lz_gla_bwd(dims, q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, ws, ws_bytes,
                              _ptr(dh0), _ptr(ws), ws_bytes, _stream(stream)))
 
 
-def lz_swa_meta_bwd(dims, q, k, v, meta_k, meta_v, lse, dO, dq, dk, dv, dmeta_k, dmeta_v, ws,
-                    ws_bytes, stream=None):
+def lz_swa_meta_bwd(dims, q, k, v, meta_k, meta_v, lse, o, dO, dq, dk, dv, dmeta_k, dmeta_v,
+                    ws, ws_bytes, stream=None):
     _check(load().lz_swa_meta_bwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(meta_k),
-                                  _ptr(meta_v), _ptr(lse), _ptr(dO), _ptr(dq), _ptr(dk),
+                                  _ptr(meta_v), _ptr(lse), _ptr(o), _ptr(dO), _ptr(dq), _ptr(dk),
                                   _ptr(dv), _ptr(dmeta_k), _ptr(dmeta_v), _ptr(ws), ws_bytes,
                                   _stream(stream)))
 
 
-def lz_swa_meta_bwd_noalloc(dims, q, k, v, meta_k, meta_v, lse, dO, dq, dk, dv, dmeta_k,
+def lz_swa_meta_bwd_noalloc(dims, q, k, v, meta_k, meta_v, lse, o, dO, dq, dk, dv, dmeta_k,
                             dmeta_v, stream=None):
     """lz_swa_meta_bwd without caller scratch: for callers that cannot
     allocate device memory; uses the library's static scratch array (see
     include/lizard.h for the size limit and the rule against overlapping
     calls)."""
     _check(load().lz_swa_meta_bwd_noalloc(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v),
-                                          _ptr(meta_k), _ptr(meta_v), _ptr(lse), _ptr(dO),
+                                          _ptr(meta_k), _ptr(meta_v), _ptr(lse), _ptr(o),
+                                          _ptr(dO),
                                           _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dmeta_k),
                                           _ptr(dmeta_v), _stream(stream)))
 
 
-def lz_hybrid_bwd(dims, q, k, v, g, meta_k, meta_v, h0, lse, dO, dhT, dq, dk, dv, dg, dh0,
-                  dmeta_k, dmeta_v, dalpha, ws, ws_bytes, stream=None):
+def lz_hybrid_bwd(dims, q, k, v, g, meta_k, meta_v, h0, lse, o_swa, dO, dhT, dq, dk, dv, dg,
+                  dh0, dmeta_k, dmeta_v, dalpha, ws, ws_bytes, stream=None):
     _check(load().lz_hybrid_bwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
-                                _ptr(meta_k), _ptr(meta_v), _ptr(h0), _ptr(lse), _ptr(dO),
+                                _ptr(meta_k), _ptr(meta_v), _ptr(h0), _ptr(lse), _ptr(o_swa),
+                                _ptr(dO),
                                 _ptr(dhT), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dh0),
                                 _ptr(dmeta_k), _ptr(dmeta_v), _ptr(dalpha), _ptr(ws), ws_bytes,
                                 _stream(stream)))
@@ -271,7 +273,8 @@ def gla_bwd(q, k, v, g, dO, h0=None, dhT=None, *, chunk=64, want_dh0=False, stre
     return {"dq": dq, "dk": dk, "dv": dv, "dg": dg, "dh0": dh0}
 
 
-def swa_meta_bwd(q, k, v, meta_k, meta_v, lse, dO, *, w, scale=None, stream=None):
+def swa_meta_bwd(q, k, v, meta_k, meta_v, lse, dO, *, w, scale=None, o=None, stream=None):
+    """o: the forward output (optional; see lz_swa_meta_bwd)."""
     M = _M(meta_k)
     d = _dims_from(q, v, chunk=64, w=w, M=M, scale=scale, alpha=1.0)
     dev = q.device
@@ -280,12 +283,13 @@ def swa_meta_bwd(q, k, v, meta_k, meta_v, lse, dO, *, w, scale=None, stream=None
     dmv = torch.empty(q.shape[1], M, v.shape[-1], dtype=torch.float32, device=dev) \
         if (M and meta_v is not None) else None
     ws, n = _ws(d, LZ_WS_SWA_BWD, dev)
-    lz_swa_meta_bwd(d, q, k, v, meta_k, meta_v, lse, dO, dq, dk, dv, dmk, dmv, ws, n, stream)
+    lz_swa_meta_bwd(d, q, k, v, meta_k, meta_v, lse, o, dO, dq, dk, dv, dmk, dmv, ws, n, stream)
     return {"dq": dq, "dk": dk, "dv": dv, "dmeta_k": dmk, "dmeta_v": dmv}
 
 
 def hybrid_bwd(q, k, v, g, meta_k, meta_v, lse, dO, *, w, alpha, scale=None, chunk=64,
-               h0=None, dhT=None, want_dh0=False, stream=None):
+               h0=None, dhT=None, o_swa=None, want_dh0=False, stream=None):
+    """o_swa: the forward's window output (optional; see lz_hybrid_bwd)."""
     M = _M(meta_k)
     d = _dims_from(q, v, chunk=chunk, w=w, M=M, scale=scale, alpha=alpha)
     dev = q.device
@@ -298,8 +302,8 @@ def hybrid_bwd(q, k, v, g, meta_k, meta_v, lse, dO, *, w, alpha, scale=None, chu
         if (M and meta_v is not None) else None
     dalpha = torch.empty(4, dtype=torch.float32, device=dev)
     ws, n = _ws(d, LZ_WS_HYBRID_BWD, dev)
-    lz_hybrid_bwd(d, q, k, v, g, meta_k, meta_v, h0, lse, dO, dhT, dq, dk, dv, dg, dh0, dmk,
-                  dmv, dalpha, ws, n, stream)
+    lz_hybrid_bwd(d, q, k, v, g, meta_k, meta_v, h0, lse, o_swa, dO, dhT, dq, dk, dv, dg, dh0,
+                  dmk, dmv, dalpha, ws, n, stream)
     return {"dq": dq, "dk": dk, "dv": dv, "dg": dg, "dh0": dh0, "dmeta_k": dmk,
             "dmeta_v": dmv, "dalpha": dalpha[:1]}
 

@@ -27,6 +27,7 @@ class ScopedTiming {
 // Records `message` as the thread's last error and returns `status`.
 int set_last_error(int status, const char* message);
 
+
 // ---- gated branch, SIMT path (fp32 arithmetic; fp32 or bf16 I/O) ----------
 struct GlaFwdParams {
   const void* q;
@@ -114,6 +115,8 @@ struct SwaBwdParams {
   const void* mk;
   const void* mv;
   const float* lse;
+  const void* osw;   // nullable: the window branch's forward output; when given
+                     // D_t = dO_t . osw_t is read off it instead of recomputed
   const void* dO;
   float gscale;      // the window branch sees gscale * dO
   void* dq;          // io dtype outputs (nullable when the f32 ones are used)
@@ -131,6 +134,8 @@ struct SwaBwdParams {
   int B, H, T, dkd, dvd, w, M;
   float scale;
 };
+// query rows per CTA of the meta-gradient pass (one partial per slab)
+constexpr int kSwaBwdSlab = 512;
 int swa_bwd_n_qblocks(int B, int H, int T);
 int swa_bwd_n_meta_parts(int B, int T);
 cudaError_t launch_swa_bwd_simt(const SwaBwdParams& p, bool bf16, cudaStream_t s);

@@ -267,9 +267,10 @@ lz::GlaFwdParams gla_fwd_params(const lz_dims* d, const void* q, const void* k, 
 
 lz::SwaBwdParams swa_bwd_params(const lz_dims* d, const void* q, const void* k, const void* v,
                                 const void* mk, const void* mv, const float* lse,
-                                const void* dO, const SwaBwdWs& w) {
+                                const void* osw, const void* dO, const SwaBwdWs& w) {
   lz::SwaBwdParams p{};
   p.q = q; p.k = k; p.v = v; p.mk = mk; p.mv = d->M > 0 ? mv : nullptr; p.lse = lse; p.dO = dO;
+  p.osw = osw;
   p.Dbuf = w.Dbuf; p.alpha_part = w.alpha_part; p.meta_part = w.meta_part;
   p.B = d->B; p.H = d->H; p.T = d->T; p.dkd = d->dk; p.dvd = d->dv; p.w = d->w; p.M = d->M;
   p.scale = d->scale;
@@ -400,20 +401,21 @@ lz_status lz_gla_bwd(const lz_dims* d, const void* q, const void* k, const void*
 
 lz_status lz_swa_meta_bwd(const lz_dims* d, const void* q, const void* k, const void* v,
                           const void* meta_k, const void* meta_v, const float* lse,
-                          const void* dO, void* dq, void* dk, void* dv, float* dmeta_k,
-                          float* dmeta_v, void* ws, size_t ws_bytes_, lz_stream stream) {
+                          const void* o, const void* dO, void* dq, void* dk, void* dv,
+                          float* dmeta_k, float* dmeta_v, void* ws, size_t ws_bytes_,
+                          lz_stream stream) {
   lz_status st = check_dims(d, true);
   if (st != LZ_OK) return st;
   const bool nz = bht(d) > 0;  // empty tensors may have NULL data
   LZ_PTR(q, nz); LZ_PTR(k, nz); LZ_PTR(v, nz); LZ_PTR(lse, nz); LZ_PTR(dO, nz);
   LZ_PTR(dq, nz); LZ_PTR(dk, nz); LZ_PTR(dv, nz);
-  LZ_PTR(meta_k, d->M > 0 && d->H > 0); LZ_PTR(meta_v, false);
+  LZ_PTR(meta_k, d->M > 0 && d->H > 0); LZ_PTR(meta_v, false); LZ_PTR(o, false);
   LZ_PTR(dmeta_k, false); LZ_PTR(dmeta_v, false);
   st = check_ws(d, LZ_WS_SWA_BWD, ws, ws_bytes_);
   if (st != LZ_OK) return st;
   Carver c(ws);
   SwaBwdWs w = carve_swa_bwd(c, d);
-  lz::SwaBwdParams p = swa_bwd_params(d, q, k, v, meta_k, meta_v, lse, dO, w);
+  lz::SwaBwdParams p = swa_bwd_params(d, q, k, v, meta_k, meta_v, lse, o, dO, w);
   p.gscale = 1.f;
   p.dq = dq; p.dk = dk; p.dv = dv;
   p.dmk = dmeta_k; p.dmv = dmeta_v;
@@ -422,7 +424,8 @@ lz_status lz_swa_meta_bwd(const lz_dims* d, const void* q, const void* k, const 
 
 lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const void* v,
                         const float* g, const void* meta_k, const void* meta_v,
-                        const float* h0, const float* lse, const void* dO, const float* dhT,
+                        const float* h0, const float* lse, const void* o_swa,
+                        const void* dO, const float* dhT,
                         void* dq, void* dk, void* dv, float* dg, float* dh0, float* dmeta_k,
                         float* dmeta_v, float* dalpha, void* ws, size_t ws_bytes_,
                         lz_stream stream) {
@@ -432,7 +435,7 @@ lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const vo
   LZ_PTR(q, nz); LZ_PTR(k, nz); LZ_PTR(v, nz); LZ_PTR(g, nz); LZ_PTR(lse, nz);
   LZ_PTR(dO, nz); LZ_PTR(dq, nz); LZ_PTR(dk, nz); LZ_PTR(dv, nz); LZ_PTR(dg, nz);
   LZ_PTR(meta_k, d->M > 0 && d->H > 0); LZ_PTR(meta_v, false); LZ_PTR(h0, false); LZ_PTR(dhT, false);
-  LZ_PTR(dh0, false); LZ_PTR(dmeta_k, false); LZ_PTR(dmeta_v, false);
+  LZ_PTR(dh0, false); LZ_PTR(dmeta_k, false); LZ_PTR(dmeta_v, false); LZ_PTR(o_swa, false);
   if (dalpha && (reinterpret_cast<uintptr_t>(dalpha) & 3u))
     return fail(LZ_ERR_INVALID_ARG, "dalpha must be 4-byte aligned");
   st = check_ws(d, LZ_WS_HYBRID_BWD, ws, ws_bytes_);
@@ -441,7 +444,7 @@ lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const vo
   Carver c(ws);
   HybridBwdWs w = carve_hybrid_bwd(c, d);
   const bool mma = hybrid_uses_mma(d);
-  lz::SwaBwdParams p = swa_bwd_params(d, q, k, v, meta_k, meta_v, lse, dO, w.swa);
+  lz::SwaBwdParams p = swa_bwd_params(d, q, k, v, meta_k, meta_v, lse, o_swa, dO, w.swa);
   p.gscale = d->alpha;
   // tensor-core path: bf16 window gradients straight into dq, dk, dv; the
   // gated backward then adds its own terms in place

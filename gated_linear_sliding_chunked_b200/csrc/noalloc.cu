@@ -34,7 +34,8 @@ std::unordered_map<int, void*> g_addr;  // device ordinal -> device address of t
 extern "C" lz_status lz_swa_meta_bwd_noalloc(const lz_dims* d, const void* q, const void* k,
                                             const void* v, const void* meta_k,
                                             const void* meta_v, const float* lse,
-                                            const void* dO, void* dq, void* dk, void* dv,
+                                            const void* o, const void* dO, void* dq,
+                                            void* dk, void* dv,
                                             float* dmeta_k, float* dmeta_v, lz_stream stream) {
   if (d == nullptr)
     return (lz_status)lz::set_last_error(LZ_ERR_INVALID_ARG, "dims must not be NULL");
@@ -80,6 +81,6 @@ extern "C" lz_status lz_swa_meta_bwd_noalloc(const lz_dims* d, const void* q, co
   }
   // Every region of this scratch is written before it is read, so the
   // previous call's leftovers need no clearing.
-  return lz_swa_meta_bwd(d, q, k, v, meta_k, meta_v, lse, dO, dq, dk, dv, dmeta_k, dmeta_v,
+  return lz_swa_meta_bwd(d, q, k, v, meta_k, meta_v, lse, o, dO, dq, dk, dv, dmeta_k, dmeta_v,
                          scratch, kScratchBytes, stream);
 }

@@ -9,9 +9,10 @@
 // (Lizard technical summary, section 2a: window keys j in [t-w+1, t] plus M
 // always-visible meta tokens in the softmax).
 //
-// Kernel 1 (query-major): CTA = one (batch, head) and a slab of up to 1024
-// query rows, walked in 64-row tiles by 4 warps x 16 rows; two sweeps over
-// the key tiles: the first accumulates D, the second dS and dq.  Meta-token
+// Kernel 1 (query-major): CTA = one (batch, head) and a slab of query rows,
+// walked in 64-row tiles by 4 warps x 16 rows.  With the forward output at
+// hand D_t = dO_t . o_t comes straight off it and one sweep over the key
+// tiles gives dS and dq; without it a first sweep accumulates D.  Meta-token
 // gradients accumulate in registers over the slab and are written as one
 // partial per CTA; D goes to scratch for kernel 2.
 // Kernel 2 (key-major): CTA = 64 keys of one (batch, head), 4 warps x 16
@@ -30,7 +31,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int QTILE = 64;   // kernel 1 query rows per tile
 constexpr int KT1 = 32;     // kernel 1 keys per tile
 constexpr int MT = 16;      // meta tile
-constexpr int SLAB = 1024;  // kernel 1 query rows per CTA (matches the partial layout)
+constexpr int SLAB = kSwaBwdSlab;  // kernel 1 query rows per CTA (one meta partial each)
 constexpr int NT = 128;
 
 template <int N>
@@ -48,6 +49,7 @@ struct QSmem {
   bf16 dsm[QTILE * 24];   // meta dS (bf16), rows x 16 (+8 pad)
   bf16 pm[QTILE * 24];    // meta P (bf16)
   float lse2[QTILE];
+  float drow[QTILE];      // D_t from the saved forward output
 };
 
 static_assert(sizeof(QSmem) <= 232448, "shared memory per block exceeds 227 KB");
@@ -121,6 +123,28 @@ __global__ void __launch_bounds__(NT, 2) swa_bwd_q_mma_kernel(SwaBwdParams p) {
     cp_async_commit();
     cp_async_wait<0>();
     __syncthreads();
+    if (p.osw) {  // D_t = dO_t . o_t, two threads per row
+      const int r = tid >> 1, c0 = (tid & 1) * (D / 2);
+      float acc = 0.f;
+      if (t0 + r < T) {
+        const uint4* op = reinterpret_cast<const uint4*>((const bf16*)p.osw + ((size_t)bh * T + t0 + r) * D + c0);
+#pragma unroll
+        for (int x = 0; x < D / 16; ++x) {
+          const uint4 ov = __ldg(op + x);
+          const uint4 dv4 = *reinterpret_cast<const uint4*>(&sm.dO[r * RPAD + c0 + 8 * x]);
+          const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, dw[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+#pragma unroll
+          for (int y = 0; y < 4; ++y) {
+            const float2 a = unpack_bf16(ow[y]), bb = unpack_bf16(dw[y]);
+            acc = fmaf(a.x, bb.x, acc);
+            acc = fmaf(a.y, bb.y, acc);
+          }
+        }
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      if ((tid & 1) == 0) sm.drow[r] = acc;
+      __syncthreads();
+    }
     const int row0 = t0 + 16 * warp + gr;
     uint32_t qa[D / 16][4], da[D / 16][4];
 #pragma unroll
@@ -132,6 +156,10 @@ __global__ void __launch_bounds__(NT, 2) swa_bwd_q_mma_kernel(SwaBwdParams p) {
     }
     const float l2[2] = {sm.lse2[16 * warp + gr], sm.lse2[16 * warp + gr + 8]};
     float Drow[2] = {0.f, 0.f};
+    if (p.osw) {
+      Drow[0] = sm.drow[16 * warp + gr];
+      Drow[1] = sm.drow[16 * warp + gr + 8];
+    }
     float dq[D / 8][4];
 #pragma unroll
     for (int nt = 0; nt < D / 8; ++nt)
@@ -168,7 +196,7 @@ __global__ void __launch_bounds__(NT, 2) swa_bwd_q_mma_kernel(SwaBwdParams p) {
     auto meta_valid = [=](int hh, int j) { return j < M && row0 + 8 * hh < T; };
     const bf16* mvs = p.mv ? sm.mv : nullptr;
 
-    for (int sweep = 0; sweep < 2; ++sweep) {
+    for (int sweep = p.osw ? 1 : 0; sweep < 2; ++sweep) {
       if (M > 0) {  // meta tile
         float s[MT / 8][4], dp[MT / 8][4];
         tile_pdp(sm.mk, mvs, IntTag<MT>{}, meta_valid, s, dp);

@@ -347,7 +347,7 @@ __global__ void __launch_bounds__(KVW * 32) swa_bwd_kv_kernel(SwaBwdParams p) {
 // Meta gradients: per (batch, head, slab of rows) partial sums, written to
 // scratch; one warp per meta token (M <= 16, 8 warps, two tokens each).
 // ---------------------------------------------------------------------------
-constexpr int SLAB = 1024;
+constexpr int SLAB = kSwaBwdSlab;
 constexpr int MW = 8;  // warps in the meta kernel
 
 template <typename IO, int DK, int DV>

@@ -119,13 +119,17 @@ lz_status lz_gla_bwd(const lz_dims* d, const void* q, const void* k,
                      size_t ws_bytes, lz_stream stream);
 
 /* Gradient of lz_swa_meta_fwd.  dO = dL/d(o_swa); lse from the forward.
+ * o (nullable) is the forward's output o_swa: when given, the softmax
+ * backward's row term D_t = dO_t . o_t is read off it (the bf16 tensor-core
+ * path then walks the window once instead of twice); when NULL it is
+ * rebuilt from the scores.  Both give the same result up to rounding.
  * Writes dq, dk, dv (io dtype) and, when M > 0, dmeta_k (fp32, summed over
  * batch and sequence) and dmeta_v (fp32; ignored in sink-only mode). */
 lz_status lz_swa_meta_bwd(const lz_dims* d, const void* q, const void* k,
                           const void* v, const void* meta_k,
                           const void* meta_v, const float* lse,
-                          const void* dO, void* dq, void* dk, void* dv,
-                          float* dmeta_k, float* dmeta_v, void* ws,
+                          const void* o, const void* dO, void* dq, void* dk,
+                          void* dv, float* dmeta_k, float* dmeta_v, void* ws,
                           size_t ws_bytes, lz_stream stream);
 
 /* Scratch-free variant of lz_swa_meta_bwd, for callers that cannot allocate
@@ -152,17 +156,20 @@ lz_status lz_swa_meta_bwd(const lz_dims* d, const void* q, const void* k,
 lz_status lz_swa_meta_bwd_noalloc(const lz_dims* d, const void* q,
                                   const void* k, const void* v,
                                   const void* meta_k, const void* meta_v,
-                                  const float* lse, const void* dO, void* dq,
-                                  void* dk, void* dv, float* dmeta_k,
-                                  float* dmeta_v, lz_stream stream);
+                                  const float* lse, const void* o,
+                                  const void* dO, void* dq, void* dk, void* dv,
+                                  float* dmeta_k, float* dmeta_v,
+                                  lz_stream stream);
 
 /* Gradient of lz_hybrid_fwd in one call: the gated branch sees dO, the
- * window branch alpha * dO.  lse from the forward.  dalpha (nullable, one
- * fp32) receives sum over (b,h,t) of dO_t . o_swa_t. */
+ * window branch alpha * dO.  lse from the forward; o_swa (nullable) the
+ * forward's window output, used as in lz_swa_meta_bwd.  dalpha (nullable,
+ * one fp32) receives sum over (b,h,t) of dO_t . o_swa_t. */
 lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k,
                         const void* v, const float* g, const void* meta_k,
                         const void* meta_v, const float* h0, const float* lse,
-                        const void* dO, const float* dhT, void* dq, void* dk,
+                        const void* o_swa, const void* dO, const float* dhT,
+                        void* dq, void* dk,
                         void* dv, float* dg, float* dh0, float* dmeta_k,
                         float* dmeta_v, float* dalpha, void* ws,
                         size_t ws_bytes, lz_stream stream);

@@ -131,14 +131,14 @@ def test_decode_validation(lib):
 
 def test_backward_validation(lib):
     d = _dims()
-    P = [FAKE] * 18
+    P = [FAKE] * 19
     # lse is required by the hybrid backward
     P2 = list(P)
     P2[7] = None
     assert lib.lz_hybrid_bwd(ctypes.byref(d), *P2, FAKE, 1 << 40, 0) == L.LZ_ERR_INVALID_ARG
     # dalpha only needs 4-byte alignment, but not 2
     P3 = list(P)
-    P3[17] = FAKE + 2
+    P3[18] = FAKE + 2
     assert lib.lz_hybrid_bwd(ctypes.byref(d), *P3, FAKE, 1 << 40, 0) == L.LZ_ERR_INVALID_ARG
     assert lib.lz_gla_bwd(ctypes.byref(_dims(dk=32)), *([FAKE] * 12), FAKE, 1 << 40, 0) == \
         L.LZ_ERR_UNSUPPORTED

@@ -35,13 +35,17 @@ def test_gla_bwd(dtype, T, dk, dv, with_state):
 @pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
 @pytest.mark.parametrize("T,w,M,sink", [(1, 1, 2, False), (50, 1, 0, False),
                                         (130, 33, 4, False), (130, 33, 4, True),
-                                        (150, 200, 0, False), (290, 128, 16, False)])
-def test_swa_meta_bwd(dtype, T, w, M, sink):
+                                        (150, 200, 0, False), (290, 128, 16, False),
+                                        (1100, 128, 8, False)])
+@pytest.mark.parametrize("with_o", [False, True], ids=["rebuild-D", "saved-o"])
+def test_swa_meta_bwd(dtype, T, w, M, sink, with_o):
+    """with_o: the forward output is passed, so D = dO . o comes off it."""
     cpu, dev = small_problem(40 + T + w, 2, 2, T, 128, 128, M, dtype, train=True)
     mk = dev["meta_k"] if M else None
     mv = dev["meta_v"] if (M and not sink) else None
-    _, lse = L.swa_meta_fwd(dev["q"], dev["k"], dev["v"], mk, mv, w=w)
-    res = L.swa_meta_bwd(dev["q"], dev["k"], dev["v"], mk, mv, lse, dev["dO"], w=w)
+    o, lse = L.swa_meta_fwd(dev["q"], dev["k"], dev["v"], mk, mv, w=w)
+    res = L.swa_meta_bwd(dev["q"], dev["k"], dev["v"], mk, mv, lse, dev["dO"], w=w,
+                         o=o if with_o else None)
     x = oracle_inputs(cpu, ("q", "k", "v", "meta_k", "meta_v", "dO"))
     ref = oracle.swa_meta_bwd(x["q"], x["k"], x["v"], x["meta_k"] if M else None,
                               x["meta_v"] if (M and not sink) else None, x["dO"], w,
@@ -56,14 +60,15 @@ def test_swa_meta_bwd(dtype, T, w, M, sink):
 
 @pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
 @pytest.mark.parametrize("alpha", [0.0, 0.5, 2.0])
-def test_hybrid_bwd(dtype, alpha):
+@pytest.mark.parametrize("saved", [False, True], ids=["rebuild-D", "saved-o_swa"])
+def test_hybrid_bwd(dtype, alpha, saved):
     T, w, M = 210, 40, 6
     cpu, dev = small_problem(77, 2, 2, T, 128, 128, M, dtype, train=True, h0=True)
     fwd = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
-                       w=w, alpha=alpha, h0=dev["h0"], want_lse=True)
+                       w=w, alpha=alpha, h0=dev["h0"], want_lse=True, want_o_swa=saved)
     res = L.hybrid_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
                        fwd["lse"], dev["dO"], w=w, alpha=alpha, h0=dev["h0"], dhT=dev["dhT"],
-                       want_dh0=True)
+                       o_swa=fwd["o_swa"], want_dh0=True)
     x = oracle_inputs(cpu, ("q", "k", "v", "g", "meta_k", "meta_v", "dO", "h0", "dhT"))
     ref = oracle.hybrid_bwd(x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], x["dO"], w,
                             1 / math.sqrt(128), alpha, x["h0"], x["dhT"])
@@ -102,9 +107,10 @@ def test_workload_train_sampled():
     x = I.make_inputs(wl, seed=0, device="cpu")
     dev = {k: v.cuda() for k, v in x.items()}
     fwd = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
-                       w=wl.w, alpha=wl.alpha, chunk=wl.chunk, want_lse=True)
+                       w=wl.w, alpha=wl.alpha, chunk=wl.chunk, want_lse=True, want_o_swa=True)
     res = L.hybrid_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
-                       fwd["lse"], dev["dO"], w=wl.w, alpha=wl.alpha, chunk=wl.chunk)
+                       fwd["lse"], dev["dO"], w=wl.w, alpha=wl.alpha, chunk=wl.chunk,
+                       o_swa=fwd["o_swa"])
     torch.cuda.synchronize()
     h = 5
     for b in range(wl.B):

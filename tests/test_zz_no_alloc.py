@@ -27,7 +27,7 @@ def _noalloc(dims, dev, mk, mv, lse):
            "dv": torch.empty_like(dev["v"]),
            "dmeta_k": torch.empty(mk.shape, dtype=torch.float32, device="cuda"),
            "dmeta_v": torch.empty(mv.shape, dtype=torch.float32, device="cuda")}
-    L.lz_swa_meta_bwd_noalloc(dims, dev["q"], dev["k"], dev["v"], mk, mv, lse, dev["dO"],
+    L.lz_swa_meta_bwd_noalloc(dims, dev["q"], dev["k"], dev["v"], mk, mv, lse, None, dev["dO"],
                               out["dq"], out["dk"], out["dv"], out["dmeta_k"], out["dmeta_v"])
     return out
 
@@ -58,6 +58,6 @@ def test_noalloc_rejects_problem_larger_than_its_scratch():
     dims = L.make_dims(1, 32, 200_000, 128, 128, chunk=64, w=64, M=4, io=L.LZ_BF16)
     assert L.lz_workspace_bytes(dims, L.LZ_WS_SWA_BWD) > L.LZ_NOALLOC_SCRATCH_BYTES
     fake = ctypes.c_void_p(0x7F0000000000)
-    st = lib.lz_swa_meta_bwd_noalloc(ctypes.byref(dims), *([fake] * 12), None)
+    st = lib.lz_swa_meta_bwd_noalloc(ctypes.byref(dims), *([fake] * 13), None)
     assert st == L.LZ_ERR_UNSUPPORTED
     assert b"static" in lib.lz_last_error()
