@@ -79,27 +79,71 @@ CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.a
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+    """SM clocks and throttle reasons sampled while the timed region runs:
+    NVML read from a background thread every 10 ms (read-only queries),
+    else nvidia-smi every 100 ms."""
+
+    # clocks-event-reason bits (nvml.h): the slowdowns that reject a run,
+    # and the power cap that is kept and noted
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4}
 
     def __init__(self, device_index: int):
+        self.device_index = device_index
+        self.samples = []  # (sm_mhz, max_mhz, reason bits or names)
         self.proc = None
-        self.out = []
-        try:
-            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
-        except Exception:
-            uuid = str(device_index)
-        self.cmd = ["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
-                    "-lms", "100", "-i", uuid]
+        self.thread = None
+        self.stop = None
+        self.source = None
+
+    def _nvml_loop(self, handle, nv):
+        import time
+        while not self.stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                self.samples.append((float(sm), float(mx),
+                                     {n for n, b in self.REASONS.items() if bits & b}))
+            except Exception:
+                pass
+            time.sleep(0.01)
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE,
-                                         stderr=subprocess.DEVNULL, text=True)
+            import pynvml as nv
+            nv.nvmlInit()
+            try:
+                uuid = "GPU-" + str(torch.cuda.get_device_properties(self.device_index).uuid)
+                handle = nv.nvmlDeviceGetHandleByUUID(uuid)
+            except Exception:
+                handle = nv.nvmlDeviceGetHandleByIndex(self.device_index)
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._nvml_loop, args=(handle, nv), daemon=True)
+            self.thread.start()
+            self.source = "nvml, 10 ms"
+            return self
+        except Exception:
+            self.thread = None
+        try:
+            try:
+                uuid = "GPU-" + str(torch.cuda.get_device_properties(self.device_index).uuid)
+            except Exception:
+                uuid = str(self.device_index)
+            cmd = ["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "100", "-i", uuid]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            self.source = "nvidia-smi, 100 ms"
         except Exception:
             self.proc = None
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -107,27 +151,28 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
                 out = ""
-            self.out = [ln for ln in (out or "").splitlines() if ln.strip()]
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for ln in (out or "").splitlines():
+                f = [x.strip() for x in ln.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm, mx = float(f[1]), float(f[2])
+                except ValueError:
+                    continue
+                self.samples.append((sm, mx, {n for n, v in zip(names, f[5:9])
+                                              if v.lower().startswith("active")}))
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.out:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
-            except ValueError:
-                continue
-            for nm, val in zip(names, f[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(nm)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "source": self.source}
+        reasons = set()
+        for _, _, r in self.samples:
+            reasons |= r
+        return {"sm_mhz": statistics.median(x[0] for x in self.samples),
+                "sm_max_mhz": max(x[1] for x in self.samples), "reasons": sorted(reasons),
+                "samples": len(self.samples), "source": self.source}
 
 
 # --------------------------------------------------------------------------
@@ -205,6 +250,9 @@ class TrainStep:
         mk = lambda *s, dtype=dt: torch.empty(*s, dtype=dtype, device=device)
         self.o = mk(B, H, T, dv)
         self.osw = mk(B, H, T, dv)  # window output saved for the backward
+        ncs = L.lz_workspace_bytes(self.dims, L.LZ_WS_CHUNK_STATES)
+        # gated chunk states saved by the forward for the backward
+        self.cs = mk(ncs, dtype=torch.uint8) if ncs else None
         self.lse = mk(B, H, T, dtype=torch.float32)
         self.dq, self.dk, self.dv = mk(B, H, T, dk), mk(B, H, T, dk), mk(B, H, T, dv)
         self.dg = mk(B, H, T, dk, dtype=torch.float32)
@@ -220,10 +268,11 @@ class TrainStep:
         x = x or self.x
         L, d = self.L, self.dims
         L.lz_hybrid_fwd(d, x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], None,
-                        self.o, None, self.lse, self.osw, self.wsf, self.nf)
+                        self.o, None, self.lse, self.osw, self.cs, self.wsf, self.nf)
         L.lz_hybrid_bwd(d, x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], None,
-                        self.lse, self.osw, x["dO"], None, self.dq, self.dk, self.dv, self.dg, None,
-                        self.dmk, self.dmv, self.dalpha, self.wsb, self.nb)
+                        self.lse, self.osw, self.cs, None, x["dO"], None, self.dq, self.dk,
+                        self.dv, self.dg, None, self.dmk, self.dmv, self.dalpha, self.wsb,
+                        self.nb)
 
     def outputs(self):
         return [self.o, self.dq, self.dk, self.dv, self.dg, self.dmk, self.dmv, self.dalpha]
@@ -275,7 +324,7 @@ def roofline_for(tab, wl, peaks, traffic=None):
 # --------------------------------------------------------------------------
 # sub-measurements
 # --------------------------------------------------------------------------
-def measure_fwd(wl, device, steps, warmup, peaks, seed):
+def measure_fwd(wl, device, steps, warmup, peaks, seed, tcgen05_window=False):
     import gated_linear_sliding_chunked_b200 as L
     from gated_linear_sliding_chunked_b200 import inputs as I
     x = I.make_inputs(wl, seed=seed, device=device)
@@ -289,13 +338,15 @@ def measure_fwd(wl, device, steps, warmup, peaks, seed):
     def fn():
         flush.zero_()  # 256 MB write: evicts L2 between iterations
         L.lz_hybrid_fwd(dims, x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], None,
-                        o, None, None, None, ws, n)
+                        o, None, None, None, None, ws, n)
 
+    prev = L.lz_prefer_tcgen05(tcgen05_window)
     for _ in range(warmup):
         fn()
     L.lz_timing_enable(True)
     ms = time_region(fn, steps, device)
     L.lz_timing_enable(False)
+    L.lz_prefer_tcgen05(prev)
     tab = kernel_table(L.lz_timing_read())
     lib_ms = sum(t for (c, t) in tab.values()) / steps
     dom, roof = roofline_for(tab, wl, peaks)
@@ -423,6 +474,63 @@ def run_reference(args):
 # --------------------------------------------------------------------------
 # main
 # --------------------------------------------------------------------------
+PROFILE_CASES = {
+    "train": "hybrid fwd + bwd, B2 H32 T8192 (the timed step)",
+    "train-small": "hybrid fwd + bwd, B4 H16 T2048 w64 M4 (for full ncu captures)",
+    "fwd": "hybrid fwd, B4 H16 T2048",
+    "long": "hybrid fwd, B1 H32 T65536",
+    "decode": "one decode step, Bd128 H32",
+}
+
+
+def run_profile_case(args):
+    """Runs one workload's step (args.warmup + args.steps times) on cuda:0,
+    for a profiler to capture; prints one status line."""
+    import gated_linear_sliding_chunked_b200 as L
+    from gated_linear_sliding_chunked_b200 import build as lbuild
+    from gated_linear_sliding_chunked_b200 import inputs as I
+    lbuild.build()
+    L.load()
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    L.lz_prefer_tcgen05(args.tcgen05_window)
+    case = args.profile_case
+    if case in ("train", "train-small"):
+        wl = I.TRAIN_BF16 if case == "train" else I.FWD_BF16.with_(train=True)
+        step = TrainStep(wl, I.make_inputs(wl, seed=0, device=device), device)
+        fn = step.run
+    elif case in ("fwd", "long"):
+        wl = I.FWD_BF16 if case == "fwd" else I.LONG_BF16
+        x = I.make_inputs(wl, seed=0, device=device)
+        dims = L.make_dims(wl.B, wl.H, wl.T, wl.dk, wl.dv, chunk=wl.chunk, w=wl.w, M=wl.M,
+                           io=L.io_of(wl.torch_dtype), scale=wl.scale, alpha=wl.alpha)
+        o = torch.empty(wl.B, wl.H, wl.T, wl.dv, dtype=wl.torch_dtype, device=device)
+        n = L.lz_workspace_bytes(dims, L.LZ_WS_HYBRID_FWD)
+        ws = torch.empty(max(n, 1), dtype=torch.uint8, device=device)
+
+        def fn():
+            L.lz_hybrid_fwd(dims, x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"],
+                            None, o, None, None, None, None, ws, n)
+    else:
+        dwl = I.DECODE
+        st = I.make_decode_state(dwl, seed=0, device=device)
+        tk = I.make_decode_tokens(dwl, steps=1, seed=1, device=device)
+        o = torch.empty(dwl.Bd, dwl.H, dwl.dv, dtype=torch.bfloat16, device=device)
+
+        def fn():
+            L.lz_gla_decode_step(dwl.Bd, dwl.H, dwl.dk, dwl.dv, dwl.w, dwl.M, L.LZ_BF16,
+                                 dwl.scale, dwl.alpha, st["state"], st["kring"], st["vring"],
+                                 st["pos"], tk["q"][0], tk["k"][0], tk["v"][0], tk["g"][0],
+                                 st["meta_k"], st["meta_v"], o)
+    for _ in range(args.warmup + args.steps):
+        fn()
+    torch.cuda.synchronize(device)
+    L.lz_device_check()
+    print(f"profile-case {case}: {PROFILE_CASES[case]}; {args.warmup + args.steps} steps ok",
+          flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -432,7 +540,14 @@ def main(argv=None):
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the forward-only and decode sub-measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
+                    help="run only this workload's step (warm-up + steps) for a profiler "
+                         "and print one status line; no measurement")
+    ap.add_argument("--tcgen05-window", action="store_true",
+                    help="with --profile-case: run the window forward on the tcgen05 kernel")
     args = ap.parse_args(argv)
+    if args.profile_case:
+        return run_profile_case(args)
     args.warmup = max(args.warmup, 3)
 
     if args.impl == "reference":
@@ -502,6 +617,11 @@ def main(argv=None):
     if not args.no_extras:
         extras["fwd_bf16_T2048"] = measure_fwd(I.FWD_BF16, device, 10, 3, peaks, seed=rank)
         extras["long_T65536"] = measure_fwd(I.LONG_BF16, device, 3, 1, peaks, seed=rank)
+        # the same forwards with the tcgen05 window kernel (a comparison)
+        extras["fwd_bf16_T2048_tcgen05_window"] = measure_fwd(I.FWD_BF16, device, 10, 3, peaks,
+                                                              seed=rank, tcgen05_window=True)
+        extras["long_T65536_tcgen05_window"] = measure_fwd(I.LONG_BF16, device, 3, 1, peaks,
+                                                           seed=rank, tcgen05_window=True)
         extras["decode"] = measure_decode(device, 1, 1, peaks, seed=rank)
         extras["train_step_breakdown"] = {k: [c // args.steps, round(t / c, 4)]
                                           for k, (c, t) in tab.items()}
@@ -516,7 +636,7 @@ def main(argv=None):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic (seeded, BASELINE-shaped distributions)",
+            "dtype": "bf16", "data": "synthetic (seeded; the workload's shapes and distributions)",
             "config": {"workload": wl.name, "global_batch": wl.B * world, "seq_len": wl.T,
                        "heads": wl.H, "head_dim": wl.dk, "window": wl.w, "meta_tokens": wl.M,
                        "chunk": wl.chunk, "io": wl.io, "alpha": wl.alpha,

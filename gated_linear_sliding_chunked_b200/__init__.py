@@ -26,11 +26,13 @@ LIB_PATH = os.path.join(_PKG, "liblizard.so")
 
 LZ_OK, LZ_ERR_INVALID_ARG, LZ_ERR_UNSUPPORTED, LZ_ERR_CUDA, LZ_ERR_TIMEOUT = range(5)
 LZ_F32, LZ_BF16 = 0, 1
-LZ_WS_GLA_FWD, LZ_WS_HYBRID_FWD, LZ_WS_GLA_BWD, LZ_WS_SWA_BWD, LZ_WS_HYBRID_BWD = range(5)
+(LZ_WS_GLA_FWD, LZ_WS_HYBRID_FWD, LZ_WS_GLA_BWD, LZ_WS_SWA_BWD, LZ_WS_HYBRID_BWD,
+ LZ_WS_CHUNK_STATES) = range(6)
 
 EXPORTS = ("lz_gla_fwd", "lz_gla_bwd", "lz_swa_meta_fwd", "lz_hybrid_fwd", "lz_swa_meta_bwd",
            "lz_hybrid_bwd", "lz_gla_decode_step", "lz_workspace_bytes", "lz_last_error",
-           "lz_version", "lz_timing_enable", "lz_timing_read", "lz_swa_meta_bwd_noalloc")
+           "lz_version", "lz_timing_enable", "lz_timing_read", "lz_swa_meta_bwd_noalloc",
+           "lz_device_check", "lz_prefer_tcgen05")
 
 # size of the static scratch array behind lz_swa_meta_bwd_noalloc
 LZ_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -66,15 +68,17 @@ def load(path: str = LIB_PATH):
     sz = ctypes.c_size_t
     lib.lz_workspace_bytes.argtypes = [D, ctypes.c_int]
     lib.lz_workspace_bytes.restype = sz
-    lib.lz_gla_fwd.argtypes = [D] + [_P] * 7 + [_P, sz, _P]
+    lib.lz_gla_fwd.argtypes = [D] + [_P] * 8 + [_P, sz, _P]
     lib.lz_swa_meta_fwd.argtypes = [D] + [_P] * 7 + [_P]
-    lib.lz_hybrid_fwd.argtypes = [D] + [_P] * 11 + [_P, sz, _P]
-    lib.lz_gla_bwd.argtypes = [D] + [_P] * 12 + [_P, sz, _P]
+    lib.lz_hybrid_fwd.argtypes = [D] + [_P] * 12 + [_P, sz, _P]
+    lib.lz_gla_bwd.argtypes = [D] + [_P] * 14 + [_P, sz, _P]
     lib.lz_swa_meta_bwd.argtypes = [D] + [_P] * 13 + [_P, sz, _P]
-    lib.lz_hybrid_bwd.argtypes = [D] + [_P] * 19 + [_P, sz, _P]
+    lib.lz_hybrid_bwd.argtypes = [D] + [_P] * 21 + [_P, sz, _P]
     lib.lz_swa_meta_bwd_noalloc.argtypes = [D] + [_P] * 13 + [_P]
     lib.lz_gla_decode_step.argtypes = ([ctypes.c_int] * 7 + [ctypes.c_float] * 2 +
                                        [_P] * 11 + [_P])
+    lib.lz_device_check.argtypes = [_P]
+    lib.lz_prefer_tcgen05.argtypes = [ctypes.c_int]
     lib.lz_timing_enable.argtypes = [ctypes.c_int]
     lib.lz_timing_read.argtypes = [ctypes.c_char_p, sz, ctypes.POINTER(ctypes.c_float),
                                    ctypes.c_int]
@@ -131,6 +135,18 @@ def lz_workspace_bytes(dims: LzDims, which: int) -> int:
     return int(load().lz_workspace_bytes(ctypes.byref(dims), which))
 
 
+def lz_device_check(stream=None):
+    """Raises LzError(LZ_ERR_TIMEOUT) if a bounded device wait of a library
+    kernel gave up since the last check (synchronizes the stream)."""
+    _check(load().lz_device_check(_stream(stream)))
+
+
+def lz_prefer_tcgen05(on: bool) -> bool:
+    """Selects the tcgen05 window-forward kernel (where it applies) for the
+    calling thread; returns the previous setting."""
+    return bool(load().lz_prefer_tcgen05(1 if on else 0))
+
+
 def lz_timing_enable(on: bool):
     load().lz_timing_enable(1 if on else 0)
 
@@ -149,9 +165,10 @@ def lz_timing_read(max_records: int = 1 << 16):
     return out
 
 
-def lz_gla_fwd(dims, q, k, v, g, h0, o, hT, ws, ws_bytes, stream=None):
+def lz_gla_fwd(dims, q, k, v, g, h0, o, hT, chunk_states, ws, ws_bytes, stream=None):
     _check(load().lz_gla_fwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(h0),
-                             _ptr(o), _ptr(hT), _ptr(ws), ws_bytes, _stream(stream)))
+                             _ptr(o), _ptr(hT), _ptr(chunk_states), _ptr(ws), ws_bytes,
+                             _stream(stream)))
 
 
 def lz_swa_meta_fwd(dims, q, k, v, meta_k, meta_v, o, lse, stream=None):
@@ -159,17 +176,20 @@ def lz_swa_meta_fwd(dims, q, k, v, meta_k, meta_v, o, lse, stream=None):
                                   _ptr(meta_v), _ptr(o), _ptr(lse), _stream(stream)))
 
 
-def lz_hybrid_fwd(dims, q, k, v, g, meta_k, meta_v, h0, o, hT, lse, o_swa, ws, ws_bytes,
-                  stream=None):
+def lz_hybrid_fwd(dims, q, k, v, g, meta_k, meta_v, h0, o, hT, lse, o_swa, chunk_states, ws,
+                  ws_bytes, stream=None):
     _check(load().lz_hybrid_fwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
                                 _ptr(meta_k), _ptr(meta_v), _ptr(h0), _ptr(o), _ptr(hT),
-                                _ptr(lse), _ptr(o_swa), _ptr(ws), ws_bytes, _stream(stream)))
+                                _ptr(lse), _ptr(o_swa), _ptr(chunk_states), _ptr(ws), ws_bytes,
+                                _stream(stream)))
 
 
-def lz_gla_bwd(dims, q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, ws, ws_bytes, stream=None):
+def lz_gla_bwd(dims, q, k, v, g, h0, dO, dhT, chunk_states, hT, dq, dk, dv, dg, dh0, ws,
+               ws_bytes, stream=None):
     _check(load().lz_gla_bwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(h0),
-                             _ptr(dO), _ptr(dhT), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg),
-                             _ptr(dh0), _ptr(ws), ws_bytes, _stream(stream)))
+                             _ptr(dO), _ptr(dhT), _ptr(chunk_states), _ptr(hT), _ptr(dq),
+                             _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dh0), _ptr(ws), ws_bytes,
+                             _stream(stream)))
 
 
 def lz_swa_meta_bwd(dims, q, k, v, meta_k, meta_v, lse, o, dO, dq, dk, dv, dmeta_k, dmeta_v,
@@ -193,11 +213,11 @@ def lz_swa_meta_bwd_noalloc(dims, q, k, v, meta_k, meta_v, lse, o, dO, dq, dk, d
                                           _ptr(dmeta_v), _stream(stream)))
 
 
-def lz_hybrid_bwd(dims, q, k, v, g, meta_k, meta_v, h0, lse, o_swa, dO, dhT, dq, dk, dv, dg,
-                  dh0, dmeta_k, dmeta_v, dalpha, ws, ws_bytes, stream=None):
+def lz_hybrid_bwd(dims, q, k, v, g, meta_k, meta_v, h0, lse, o_swa, chunk_states, hT, dO, dhT,
+                  dq, dk, dv, dg, dh0, dmeta_k, dmeta_v, dalpha, ws, ws_bytes, stream=None):
     _check(load().lz_hybrid_bwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
                                 _ptr(meta_k), _ptr(meta_v), _ptr(h0), _ptr(lse), _ptr(o_swa),
-                                _ptr(dO),
+                                _ptr(chunk_states), _ptr(hT), _ptr(dO),
                                 _ptr(dhT), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dh0),
                                 _ptr(dmeta_k), _ptr(dmeta_v), _ptr(dalpha), _ptr(ws), ws_bytes,
                                 _stream(stream)))
@@ -229,14 +249,24 @@ def _M(meta_k):
     return 0 if meta_k is None else int(meta_k.shape[1])
 
 
-def gla_fwd(q, k, v, g, h0=None, *, chunk=64, want_hT=False, stream=None):
+def _chunk_states(dims, device):
+    """Buffer for the forward's chunk states, or None where the kernels keep
+    none (LZ_WS_CHUNK_STATES)."""
+    n = lz_workspace_bytes(dims, LZ_WS_CHUNK_STATES)
+    return torch.empty(n, dtype=torch.uint8, device=device) if n else None
+
+
+def gla_fwd(q, k, v, g, h0=None, *, chunk=64, want_hT=False, want_chunk_states=False,
+            stream=None):
+    """Returns (o, hT), or (o, hT, chunk_states) with want_chunk_states."""
     d = _dims_from(q, v, chunk=chunk, w=1, M=0, scale=None, alpha=0.0)
     o = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=q.device)
     hT = torch.empty(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], dtype=torch.float32,
                      device=q.device) if want_hT else None
+    cs = _chunk_states(d, q.device) if want_chunk_states else None
     ws, n = _ws(d, LZ_WS_GLA_FWD, q.device)
-    lz_gla_fwd(d, q, k, v, g, h0, o, hT, ws, n, stream)
-    return o, hT
+    lz_gla_fwd(d, q, k, v, g, h0, o, hT, cs, ws, n, stream)
+    return (o, hT, cs) if want_chunk_states else (o, hT)
 
 
 def swa_meta_fwd(q, k, v, meta_k, meta_v, *, w, scale=None, want_lse=True, stream=None):
@@ -248,7 +278,8 @@ def swa_meta_fwd(q, k, v, meta_k, meta_v, *, w, scale=None, want_lse=True, strea
 
 
 def hybrid_fwd(q, k, v, g, meta_k, meta_v, *, w, alpha, scale=None, chunk=64, h0=None,
-               want_hT=False, want_lse=False, want_o_swa=False, stream=None):
+               want_hT=False, want_lse=False, want_o_swa=False, want_chunk_states=False,
+               stream=None):
     d = _dims_from(q, v, chunk=chunk, w=w, M=_M(meta_k), scale=scale, alpha=alpha)
     dev = q.device
     o = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=dev)
@@ -256,12 +287,15 @@ def hybrid_fwd(q, k, v, g, meta_k, meta_v, *, w, alpha, scale=None, chunk=64, h0
                      device=dev) if want_hT else None
     lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=dev) if want_lse else None
     osw = torch.empty_like(o) if want_o_swa else None
+    cs = _chunk_states(d, dev) if want_chunk_states else None
     ws, n = _ws(d, LZ_WS_HYBRID_FWD, dev)
-    lz_hybrid_fwd(d, q, k, v, g, meta_k, meta_v, h0, o, hT, lse, osw, ws, n, stream)
-    return {"o": o, "hT": hT, "lse": lse, "o_swa": osw}
+    lz_hybrid_fwd(d, q, k, v, g, meta_k, meta_v, h0, o, hT, lse, osw, cs, ws, n, stream)
+    return {"o": o, "hT": hT, "lse": lse, "o_swa": osw, "chunk_states": cs}
 
 
-def gla_bwd(q, k, v, g, dO, h0=None, dhT=None, *, chunk=64, want_dh0=False, stream=None):
+def gla_bwd(q, k, v, g, dO, h0=None, dhT=None, *, chunk=64, chunk_states=None, hT=None,
+            want_dh0=False, stream=None):
+    """chunk_states, hT: the forward's (optional; see lz_gla_bwd)."""
     d = _dims_from(q, v, chunk=chunk, w=1, M=0, scale=None, alpha=0.0)
     dev = q.device
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -269,7 +303,7 @@ def gla_bwd(q, k, v, g, dO, h0=None, dhT=None, *, chunk=64, want_dh0=False, stre
     dh0 = torch.empty(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], dtype=torch.float32,
                       device=dev) if want_dh0 else None
     ws, n = _ws(d, LZ_WS_GLA_BWD, dev)
-    lz_gla_bwd(d, q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, ws, n, stream)
+    lz_gla_bwd(d, q, k, v, g, h0, dO, dhT, chunk_states, hT, dq, dk, dv, dg, dh0, ws, n, stream)
     return {"dq": dq, "dk": dk, "dv": dv, "dg": dg, "dh0": dh0}
 
 
@@ -288,8 +322,9 @@ def swa_meta_bwd(q, k, v, meta_k, meta_v, lse, dO, *, w, scale=None, o=None, str
 
 
 def hybrid_bwd(q, k, v, g, meta_k, meta_v, lse, dO, *, w, alpha, scale=None, chunk=64,
-               h0=None, dhT=None, o_swa=None, want_dh0=False, stream=None):
-    """o_swa: the forward's window output (optional; see lz_hybrid_bwd)."""
+               h0=None, dhT=None, o_swa=None, chunk_states=None, hT=None, want_dh0=False,
+               stream=None):
+    """o_swa, chunk_states, hT: the forward's (optional; see lz_hybrid_bwd)."""
     M = _M(meta_k)
     d = _dims_from(q, v, chunk=chunk, w=w, M=M, scale=scale, alpha=alpha)
     dev = q.device
@@ -302,8 +337,8 @@ def hybrid_bwd(q, k, v, g, meta_k, meta_v, lse, dO, *, w, alpha, scale=None, chu
         if (M and meta_v is not None) else None
     dalpha = torch.empty(4, dtype=torch.float32, device=dev)
     ws, n = _ws(d, LZ_WS_HYBRID_BWD, dev)
-    lz_hybrid_bwd(d, q, k, v, g, meta_k, meta_v, h0, lse, o_swa, dO, dhT, dq, dk, dv, dg, dh0,
-                  dmk, dmv, dalpha, ws, n, stream)
+    lz_hybrid_bwd(d, q, k, v, g, meta_k, meta_v, h0, lse, o_swa, chunk_states, hT, dO, dhT, dq,
+                  dk, dv, dg, dh0, dmk, dmv, dalpha, ws, n, stream)
     return {"dq": dq, "dk": dk, "dv": dv, "dg": dg, "dh0": dh0, "dmeta_k": dmk,
             "dmeta_v": dmv, "dalpha": dalpha[:1]}
 

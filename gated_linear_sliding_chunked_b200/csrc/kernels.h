@@ -27,6 +27,10 @@ class ScopedTiming {
 // Records `message` as the thread's last error and returns `status`.
 int set_last_error(int status, const char* message);
 
+// Device address of the library's status word on the current device: the
+// tcgen05 kernels add one per bounded wait that gave up.  NULL if the
+// address cannot be had (the caller then refuses to launch).
+unsigned int* device_status_word();
 
 // ---- gated branch, SIMT path (fp32 arithmetic; fp32 or bf16 I/O) ----------
 struct GlaFwdParams {
@@ -102,11 +106,15 @@ struct SwaFwdParams {
   float* lse;       // nullable
   int B, H, T, dk, dv, w, M;
   float scale;
+  unsigned int* status;  // device status word (set by the tcgen05 launcher)
 };
 cudaError_t launch_swa_fwd_simt(const SwaFwdParams& p, bool bf16, cudaStream_t s);
-// tensor-core forward (bf16 I/O, dk = dv = 128)
+// warp-level tensor-core forward (bf16 I/O, dk = dv = 128)
 bool swa_fwd_mma_supported(int dk, int dv, bool bf16);
 cudaError_t launch_swa_fwd_mma(const SwaFwdParams& p, cudaStream_t s);
+// tcgen05 forward (bf16 I/O, dk = dv = 128, w <= 129)
+bool swa_fwd_tc_supported(int dk, int dv, bool bf16, int w);
+cudaError_t launch_swa_fwd_tc(const SwaFwdParams& p, cudaStream_t s);
 
 struct SwaBwdParams {
   const void* q;

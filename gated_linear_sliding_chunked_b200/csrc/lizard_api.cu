@@ -11,10 +11,13 @@
 namespace {
 
 thread_local std::string g_err;
+thread_local bool g_prefer_tc = false;  // lz_prefer_tcgen05
 
-// The window branch's forward: tensor cores for bf16 with dk = dv = 128,
-// fp32 SIMT otherwise.
+// The window branch's forward: warp-level MMA for bf16 with dk = dv = 128
+// (tcgen05 instead when the calling thread prefers it and w <= 129), fp32
+// SIMT otherwise.
 cudaError_t swa_forward(const lz::SwaFwdParams& p, bool bf16, cudaStream_t s) {
+  if (g_prefer_tc && lz::swa_fwd_tc_supported(p.dk, p.dv, bf16, p.w)) return lz::launch_swa_fwd_tc(p, s);
   if (lz::swa_fwd_mma_supported(p.dk, p.dv, bf16)) return lz::launch_swa_fwd_mma(p, s);
   return lz::launch_swa_fwd_simt(p, bf16, s);
 }
@@ -232,9 +235,27 @@ size_t ws_bytes(const lz_dims* d, int which) {
     case LZ_WS_HYBRID_BWD:
       carve_hybrid_bwd(c, d);
       return c.off;
+    case LZ_WS_CHUNK_STATES:
+      return fwd_uses_chunks(d) && bwd_uses_mma(d) ? states16_count(d) * sizeof(uint16_t) : 0;
     default:
       return 0;
   }
+}
+
+// The forward's chunk states handed to a backward call: used only where the
+// kernels keep bf16 chunk states (*states is cleared otherwise); the final
+// state must come with them when dL/dhT is given.
+lz_status check_saved_states(const lz_dims* d, const float* dhT, const void** states,
+                             const float* hT) {
+  const void* chunk_states = *states;
+  if (chunk_states == nullptr) return LZ_OK;
+  LZ_PTR(chunk_states, false);
+  if (ws_bytes(d, LZ_WS_CHUNK_STATES) == 0) {
+    *states = nullptr;
+    return LZ_OK;
+  }
+  LZ_PTR(hT, dhT != nullptr);
+  return LZ_OK;
 }
 
 lz_status check_ws(const lz_dims* d, int which, const void* ws, size_t have) {
@@ -285,19 +306,25 @@ const char* lz_last_error(void) { return g_err.c_str(); }
 
 const char* lz_version(void) { return "lizard-b200 0.1 (sm_100a)"; }
 
+int lz_prefer_tcgen05(int on) {
+  const int prev = g_prefer_tc ? 1 : 0;
+  g_prefer_tc = on != 0;
+  return prev;
+}
+
 size_t lz_workspace_bytes(const lz_dims* d, int which) {
   if (check_dims(d, which != LZ_WS_GLA_FWD && which != LZ_WS_GLA_BWD) != LZ_OK) return 0;
   return ws_bytes(d, which);
 }
 
 lz_status lz_gla_fwd(const lz_dims* d, const void* q, const void* k, const void* v,
-                     const float* g, const float* h0, void* o, float* hT, void* ws,
-                     size_t ws_bytes_, lz_stream stream) {
+                     const float* g, const float* h0, void* o, float* hT,
+                     void* chunk_states, void* ws, size_t ws_bytes_, lz_stream stream) {
   lz_status st = check_dims(d, false);
   if (st != LZ_OK) return st;
   const bool nz = bht(d) > 0;  // empty tensors may have NULL data
   LZ_PTR(q, nz); LZ_PTR(k, nz); LZ_PTR(v, nz); LZ_PTR(g, nz); LZ_PTR(o, nz);
-  LZ_PTR(h0, false); LZ_PTR(hT, false);
+  LZ_PTR(h0, false); LZ_PTR(hT, false); LZ_PTR(chunk_states, false);
   st = check_ws(d, LZ_WS_GLA_FWD, ws, ws_bytes_);
   if (st != LZ_OK) return st;
   lz::GlaFwdParams p = gla_fwd_params(d, q, k, v, g, h0);
@@ -305,6 +332,7 @@ lz_status lz_gla_fwd(const lz_dims* d, const void* q, const void* k, const void*
   p.hT = hT;
   Carver c(ws);
   void* states16 = fwd_uses_chunks(d) ? c.take<uint16_t>(states16_count(d)) : nullptr;
+  if (states16 && chunk_states && ws_bytes(d, LZ_WS_CHUNK_STATES) > 0) states16 = chunk_states;
   return cuda_status(gla_forward(p, d->io == LZ_BF16, states16, as_stream(stream)), "lz_gla_fwd");
 }
 
@@ -325,13 +353,13 @@ lz_status lz_swa_meta_fwd(const lz_dims* d, const void* q, const void* k, const 
 lz_status lz_hybrid_fwd(const lz_dims* d, const void* q, const void* k, const void* v,
                         const float* g, const void* meta_k, const void* meta_v,
                         const float* h0, void* o, float* hT, float* lse, void* o_swa,
-                        void* ws, size_t ws_bytes_, lz_stream stream) {
+                        void* chunk_states, void* ws, size_t ws_bytes_, lz_stream stream) {
   lz_status st = check_dims(d, true);
   if (st != LZ_OK) return st;
   const bool nz = bht(d) > 0;  // empty tensors may have NULL data
   LZ_PTR(q, nz); LZ_PTR(k, nz); LZ_PTR(v, nz); LZ_PTR(g, nz); LZ_PTR(o, nz);
   LZ_PTR(meta_k, d->M > 0 && d->H > 0); LZ_PTR(meta_v, false); LZ_PTR(h0, false); LZ_PTR(hT, false);
-  LZ_PTR(lse, false); LZ_PTR(o_swa, false);
+  LZ_PTR(lse, false); LZ_PTR(o_swa, false); LZ_PTR(chunk_states, false);
   st = check_ws(d, LZ_WS_HYBRID_FWD, ws, ws_bytes_);
   if (st != LZ_OK) return st;
   const cudaStream_t s = as_stream(stream);
@@ -340,6 +368,7 @@ lz_status lz_hybrid_fwd(const lz_dims* d, const void* q, const void* k, const vo
   Carver c(ws);
   float* osw = mma ? nullptr : c.take<float>(bht(d) * d->dv);
   void* states16 = fwd_uses_chunks(d) ? c.take<uint16_t>(states16_count(d)) : nullptr;
+  if (states16 && chunk_states && ws_bytes(d, LZ_WS_CHUNK_STATES) > 0) states16 = chunk_states;
   lz::SwaFwdParams sp = swa_fwd_params(d, q, k, v, meta_k, meta_v);
   // tensor-core path: bf16 window output into o_swa if requested, else into o
   sp.o = mma ? (o_swa ? o_swa : o) : o_swa;
@@ -358,21 +387,29 @@ lz_status lz_hybrid_fwd(const lz_dims* d, const void* q, const void* k, const vo
 
 static cudaError_t gla_bwd_launch(const lz_dims* d, const void* q, const void* k, const void* v,
                                   const float* g, const float* h0, const void* dO,
-                                  const float* dhT, void* dq, void* dk, void* dv, float* dg,
+                                  const float* dhT, const void* saved_states,
+                                  const float* saved_hT, void* dq, void* dk, void* dv, float* dg,
                                   float* dh0, const GlaBwdWs& w, const float* add_dq,
                                   const float* add_dk, const float* add_dv, bool add_in_place,
                                   cudaStream_t s) {
   const bool bf = d->io == LZ_BF16;
   const bool mma = bwd_uses_mma(d);
-  lz::GlaFwdParams fp = gla_fwd_params(d, q, k, v, g, h0);
-  fp.states = w.states;
-  fp.states16 = w.states16;
-  fp.hT = w.hT;
-  cudaError_t e = mma ? lz::launch_gla_states(fp, s) : lz::launch_gla_fwd_simt(fp, bf, s);
-  if (e != cudaSuccess) return e;
+  const void* states16 = w.states16;
+  const float* hT = w.hT;
+  if (saved_states) {  // the forward's chunk states: no state pass
+    states16 = saved_states;
+    hT = saved_hT;
+  } else {
+    lz::GlaFwdParams fp = gla_fwd_params(d, q, k, v, g, h0);
+    fp.states = w.states;
+    fp.states16 = w.states16;
+    fp.hT = w.hT;
+    cudaError_t e = mma ? lz::launch_gla_states(fp, s) : lz::launch_gla_fwd_simt(fp, bf, s);
+    if (e != cudaSuccess) return e;
+  }
   lz::GlaBwdParams p{};
   p.q = q; p.k = k; p.v = v; p.g = g; p.dO = dO; p.dhT = dhT;
-  p.states = w.states; p.states16 = w.states16; p.hT = w.hT;
+  p.states = w.states; p.states16 = states16; p.hT = hT;
   p.add_dq = add_dq; p.add_dk = add_dk; p.add_dv = add_dv;
   p.add_in_place = add_in_place;
   p.dq = dq; p.dk = dk; p.dv = dv; p.dg = dg; p.dh0 = dh0;
@@ -382,19 +419,22 @@ static cudaError_t gla_bwd_launch(const lz_dims* d, const void* q, const void* k
 
 lz_status lz_gla_bwd(const lz_dims* d, const void* q, const void* k, const void* v,
                      const float* g, const float* h0, const void* dO, const float* dhT,
-                     void* dq, void* dk, void* dv, float* dg, float* dh0, void* ws,
-                     size_t ws_bytes_, lz_stream stream) {
+                     const void* chunk_states, const float* hT, void* dq, void* dk, void* dv,
+                     float* dg, float* dh0, void* ws, size_t ws_bytes_, lz_stream stream) {
   lz_status st = check_dims(d, false);
   if (st != LZ_OK) return st;
   const bool nz = bht(d) > 0;  // empty tensors may have NULL data
   LZ_PTR(q, nz); LZ_PTR(k, nz); LZ_PTR(v, nz); LZ_PTR(g, nz); LZ_PTR(dO, nz);
   LZ_PTR(dq, nz); LZ_PTR(dk, nz); LZ_PTR(dv, nz); LZ_PTR(dg, nz);
   LZ_PTR(h0, false); LZ_PTR(dhT, false); LZ_PTR(dh0, false);
+  st = check_saved_states(d, dhT, &chunk_states, hT);
+  if (st != LZ_OK) return st;
   st = check_ws(d, LZ_WS_GLA_BWD, ws, ws_bytes_);
   if (st != LZ_OK) return st;
   Carver c(ws);
   GlaBwdWs w = carve_gla_bwd(c, d);
-  return cuda_status(gla_bwd_launch(d, q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, w,
+  return cuda_status(gla_bwd_launch(d, q, k, v, g, h0, dO, dhT, chunk_states, hT, dq, dk, dv,
+                                    dg, dh0, w,
                                     nullptr, nullptr, nullptr, false, as_stream(stream)),
                      "lz_gla_bwd");
 }
@@ -425,7 +465,8 @@ lz_status lz_swa_meta_bwd(const lz_dims* d, const void* q, const void* k, const 
 lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const void* v,
                         const float* g, const void* meta_k, const void* meta_v,
                         const float* h0, const float* lse, const void* o_swa,
-                        const void* dO, const float* dhT,
+                        const void* chunk_states, const float* hT, const void* dO,
+                        const float* dhT,
                         void* dq, void* dk, void* dv, float* dg, float* dh0, float* dmeta_k,
                         float* dmeta_v, float* dalpha, void* ws, size_t ws_bytes_,
                         lz_stream stream) {
@@ -436,6 +477,8 @@ lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const vo
   LZ_PTR(dO, nz); LZ_PTR(dq, nz); LZ_PTR(dk, nz); LZ_PTR(dv, nz); LZ_PTR(dg, nz);
   LZ_PTR(meta_k, d->M > 0 && d->H > 0); LZ_PTR(meta_v, false); LZ_PTR(h0, false); LZ_PTR(dhT, false);
   LZ_PTR(dh0, false); LZ_PTR(dmeta_k, false); LZ_PTR(dmeta_v, false); LZ_PTR(o_swa, false);
+  st = check_saved_states(d, dhT, &chunk_states, hT);
+  if (st != LZ_OK) return st;
   if (dalpha && (reinterpret_cast<uintptr_t>(dalpha) & 3u))
     return fail(LZ_ERR_INVALID_ARG, "dalpha must be 4-byte aligned");
   st = check_ws(d, LZ_WS_HYBRID_BWD, ws, ws_bytes_);
@@ -453,8 +496,8 @@ lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const vo
   p.dmk = dmeta_k; p.dmv = dmeta_v; p.dalpha = dalpha;
   cudaError_t e = swa_backward(p, d->io == LZ_BF16, s);
   if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (window branch)");
-  return cuda_status(gla_bwd_launch(d, q, k, v, g, h0, dO, dhT, dq, dk, dv, dg, dh0, w.gla,
-                                    w.dq, w.dk, w.dv, mma, s),
+  return cuda_status(gla_bwd_launch(d, q, k, v, g, h0, dO, dhT, chunk_states, hT, dq, dk, dv,
+                                    dg, dh0, w.gla, w.dq, w.dk, w.dv, mma, s),
                      "lz_hybrid_bwd (gated branch)");
 }
 

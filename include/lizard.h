@@ -77,18 +77,27 @@ typedef struct {
 
 /* Bytes of scratch the call needs (0 is possible); `which` is one of the
  * LZ_WS_* values.  The scratch is caller-owned device memory, 256-byte
- * aligned, and may be reused once the call's stream work has finished. */
+ * aligned, and may be reused once the call's stream work has finished.
+ * LZ_WS_CHUNK_STATES is not scratch but the size of the optional
+ * `chunk_states` buffer of the gated forward and backward calls: the state
+ * before every 64-token chunk, [B, H, ceil(T/64), dk, dv] bf16, kept by the
+ * forward so that the backward need not walk the sequence again.  It is 0
+ * where the kernels keep no such states (fp32 I/O, d = 64); the pointers
+ * are then ignored. */
 enum { LZ_WS_GLA_FWD = 0, LZ_WS_HYBRID_FWD = 1, LZ_WS_GLA_BWD = 2,
-       LZ_WS_SWA_BWD = 3, LZ_WS_HYBRID_BWD = 4 };
+       LZ_WS_SWA_BWD = 3, LZ_WS_HYBRID_BWD = 4, LZ_WS_CHUNK_STATES = 5 };
 size_t lz_workspace_bytes(const lz_dims* d, int which);
 
 /* Gated linear attention forward (section 2a, state update equation).
  *   o = q^T S_t per token; h0 (nullable = zeros) is the state before token 0;
- *   hT (nullable) receives the state after the last token.  Fields used: B,
- *   H, T, dk, dv, chunk, io. */
+ *   hT (nullable) receives the state after the last token; chunk_states
+ *   (nullable) receives the state before every 64-token chunk (see
+ *   LZ_WS_CHUNK_STATES) for lz_gla_bwd.  Fields used: B, H, T, dk, dv,
+ *   chunk, io. */
 lz_status lz_gla_fwd(const lz_dims* d, const void* q, const void* k,
                      const void* v, const float* g, const float* h0, void* o,
-                     float* hT, void* ws, size_t ws_bytes, lz_stream stream);
+                     float* hT, void* chunk_states, void* ws, size_t ws_bytes,
+                     lz_stream stream);
 
 /* Sliding-window softmax with meta-memory sinks (section 2a, anchor window
  * attention).  meta_k may be NULL only when M == 0.  meta_v == NULL selects
@@ -101,22 +110,26 @@ lz_status lz_swa_meta_fwd(const lz_dims* d, const void* q, const void* k,
                           lz_stream stream);
 
 /* Hybrid forward o = o_gla + alpha * o_swa (section 2a, final output).
- *   hT, lse, o_swa are nullable extra outputs (lse and o_swa are what
- *   lz_hybrid_bwd needs).  All lz_dims fields are used. */
+ *   hT, lse, o_swa, chunk_states are nullable extra outputs (lse is what
+ *   lz_hybrid_bwd needs; o_swa and chunk_states let it skip work).  All
+ *   lz_dims fields are used. */
 lz_status lz_hybrid_fwd(const lz_dims* d, const void* q, const void* k,
                         const void* v, const float* g, const void* meta_k,
                         const void* meta_v, const float* h0, void* o,
-                        float* hT, float* lse, void* o_swa, void* ws,
-                        size_t ws_bytes, lz_stream stream);
+                        float* hT, float* lse, void* o_swa, void* chunk_states,
+                        void* ws, size_t ws_bytes, lz_stream stream);
 
 /* Gradient of lz_gla_fwd (needed by the attention-distillation stage,
  * section 2b).  dO = dL/do; dhT (nullable) = dL/dhT.  Writes dq, dk, dv (io
- * dtype), dg (fp32) and dh0 (nullable, fp32).  h0 may be NULL (zeros). */
+ * dtype), dg (fp32) and dh0 (nullable, fp32).  h0 may be NULL (zeros).
+ * chunk_states (nullable): the forward's chunk states for these inputs;
+ * with them the backward skips its own state pass, and then hT (the
+ * forward's final state) must be given too when dhT is. */
 lz_status lz_gla_bwd(const lz_dims* d, const void* q, const void* k,
                      const void* v, const float* g, const float* h0,
-                     const void* dO, const float* dhT, void* dq, void* dk,
-                     void* dv, float* dg, float* dh0, void* ws,
-                     size_t ws_bytes, lz_stream stream);
+                     const void* dO, const float* dhT, const void* chunk_states,
+                     const float* hT, void* dq, void* dk, void* dv, float* dg,
+                     float* dh0, void* ws, size_t ws_bytes, lz_stream stream);
 
 /* Gradient of lz_swa_meta_fwd.  dO = dL/d(o_swa); lse from the forward.
  * o (nullable) is the forward's output o_swa: when given, the softmax
@@ -163,12 +176,14 @@ lz_status lz_swa_meta_bwd_noalloc(const lz_dims* d, const void* q,
 
 /* Gradient of lz_hybrid_fwd in one call: the gated branch sees dO, the
  * window branch alpha * dO.  lse from the forward; o_swa (nullable) the
- * forward's window output, used as in lz_swa_meta_bwd.  dalpha (nullable,
- * one fp32) receives sum over (b,h,t) of dO_t . o_swa_t. */
+ * forward's window output, used as in lz_swa_meta_bwd; chunk_states and hT
+ * (nullable) the forward's, used as in lz_gla_bwd.  dalpha (nullable, one
+ * fp32) receives sum over (b,h,t) of dO_t . o_swa_t. */
 lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k,
                         const void* v, const float* g, const void* meta_k,
                         const void* meta_v, const float* h0, const float* lse,
-                        const void* o_swa, const void* dO, const float* dhT,
+                        const void* o_swa, const void* chunk_states,
+                        const float* hT, const void* dO, const float* dhT,
                         void* dq, void* dk,
                         void* dv, float* dg, float* dh0, float* dmeta_k,
                         float* dmeta_v, float* dalpha, void* ws,
@@ -191,6 +206,25 @@ lz_status lz_gla_decode_step(int Bd, int H, int dk, int dv, int w, int M,
                              const void* v, const float* g,
                              const void* meta_k, const void* meta_v, void* o,
                              lz_stream stream);
+
+/* Device-side status (no counterpart on the pages; a robustness aid).  The
+ * tcgen05 kernels wait on mbarriers for their tensor-core work; every such
+ * wait is bounded (0.2 s) and, when it gives up, adds one to a status word
+ * of the library on that device instead of spinning on (the kernel then
+ * skips the rest of its work and releases its tensor memory).
+ * lz_device_check synchronizes `stream`, reads and clears the word of the
+ * current device and returns LZ_ERR_TIMEOUT if any wait gave up since the
+ * last check (LZ_OK otherwise; LZ_ERR_CUDA if the read failed). */
+lz_status lz_device_check(lz_stream stream);
+
+/* Window-forward kernel choice for the calling host thread (no counterpart
+ * on the pages).  bf16 with dk = dv = 128 has two tensor-core kernels:
+ * warp-level mma.sync with an online softmax (any w; the default, faster
+ * today) and tcgen05 with the scores of the whole band in tensor memory
+ * (w <= 129).  lz_prefer_tcgen05(1) selects the tcgen05 kernel where it
+ * applies; both give the same result up to rounding.  Returns the previous
+ * setting; never fails. */
+int lz_prefer_tcgen05(int on);
 
 /* Per-launch device timing for benchmarks (no counterpart on the pages; a
  * measurement aid).  lz_timing_enable(1) makes every later kernel launch of

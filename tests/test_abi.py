@@ -59,7 +59,7 @@ def _call_hybrid(lib, d, **ptrs):
              lse=None, osw=None, ws=FAKE)
     p.update(ptrs)
     return lib.lz_hybrid_fwd(ctypes.byref(d), p["q"], p["k"], p["v"], p["g"], p["mk"], p["mv"],
-                             p["h0"], p["o"], p["hT"], p["lse"], p["osw"], p["ws"],
+                             p["h0"], p["o"], p["hT"], p["lse"], p["osw"], None, p["ws"],
                              ptrs.get("ws_bytes", 1 << 40), 0)
 
 
@@ -131,14 +131,33 @@ def test_decode_validation(lib):
 
 def test_backward_validation(lib):
     d = _dims()
-    P = [FAKE] * 19
+    P = [FAKE] * 21
     # lse is required by the hybrid backward
     P2 = list(P)
     P2[7] = None
     assert lib.lz_hybrid_bwd(ctypes.byref(d), *P2, FAKE, 1 << 40, 0) == L.LZ_ERR_INVALID_ARG
     # dalpha only needs 4-byte alignment, but not 2
     P3 = list(P)
-    P3[18] = FAKE + 2
+    P3[20] = FAKE + 2
     assert lib.lz_hybrid_bwd(ctypes.byref(d), *P3, FAKE, 1 << 40, 0) == L.LZ_ERR_INVALID_ARG
-    assert lib.lz_gla_bwd(ctypes.byref(_dims(dk=32)), *([FAKE] * 12), FAKE, 1 << 40, 0) == \
+    assert lib.lz_gla_bwd(ctypes.byref(_dims(dk=32)), *([FAKE] * 14), FAKE, 1 << 40, 0) == \
         L.LZ_ERR_UNSUPPORTED
+
+
+def test_chunk_states_size_and_validation(lib):
+    """The forward's chunk states exist for bf16 with d = 128 only; handing
+    them to a backward that gets dL/dhT also needs the final state."""
+    d = _dims(T=200, dk=128, dv=128)
+    assert L.lz_workspace_bytes(d, L.LZ_WS_CHUNK_STATES) == 1 * 2 * 4 * 128 * 128 * 2
+    assert L.lz_workspace_bytes(_dims(T=200, dk=128, dv=128, io=L.LZ_F32),
+                                L.LZ_WS_CHUNK_STATES) == 0
+    assert L.lz_workspace_bytes(_dims(T=200), L.LZ_WS_CHUNK_STATES) == 0
+    P = [FAKE] * 21
+    P[12] = FAKE  # dhT given
+    P[10] = None  # hT missing
+    assert lib.lz_hybrid_bwd(ctypes.byref(d), *P, FAKE, 1 << 40, 0) == L.LZ_ERR_INVALID_ARG
+    assert b"hT" in lib.lz_last_error()
+    # the same for the gated-only backward (chunk_states at 8, hT at 9)
+    G = [FAKE] * 14
+    G[9] = None
+    assert lib.lz_gla_bwd(ctypes.byref(d), *G, FAKE, 1 << 40, 0) == L.LZ_ERR_INVALID_ARG

@@ -20,11 +20,18 @@ DTYPES = [torch.float32, torch.bfloat16]
 @pytest.mark.parametrize("T,dk,dv", [(1, 64, 64), (37, 64, 64), (130, 128, 128),
                                      (200, 64, 128), (257, 128, 64)])
 @pytest.mark.parametrize("with_state", [False, True])
-def test_gla_bwd(dtype, T, dk, dv, with_state):
+@pytest.mark.parametrize("saved", [False, True], ids=["state-pass", "saved-states"])
+def test_gla_bwd(dtype, T, dk, dv, with_state, saved):
+    """saved: the backward gets the forward's chunk states and final state
+    (used by the bf16 d = 128 kernels, ignored elsewhere)."""
     cpu, dev = small_problem(20 + T, 2, 2, T, dk, dv, 0, dtype, train=True, h0=with_state)
     dhT = dev["dhT"] if with_state else None
+    cs = hT = None
+    if saved:
+        _, hT, cs = L.gla_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev.get("h0"),
+                              want_hT=True, want_chunk_states=True)
     res = L.gla_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["dO"], dev.get("h0"), dhT,
-                    want_dh0=True)
+                    chunk_states=cs, hT=hT, want_dh0=True)
     x = oracle_inputs(cpu, ("q", "k", "v", "g", "dO", "h0", "dhT"))
     ref = oracle.gla_bwd(x["q"], x["k"], x["v"], x["g"], x["dO"], x["h0"],
                          x["dhT"] if with_state else None)
@@ -60,15 +67,19 @@ def test_swa_meta_bwd(dtype, T, w, M, sink, with_o):
 
 @pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
 @pytest.mark.parametrize("alpha", [0.0, 0.5, 2.0])
-@pytest.mark.parametrize("saved", [False, True], ids=["rebuild-D", "saved-o_swa"])
+@pytest.mark.parametrize("saved", ["none", "o_swa", "all"])
 def test_hybrid_bwd(dtype, alpha, saved):
+    """saved: which forward results the backward gets (window output; also
+    the gated chunk states and final state)."""
     T, w, M = 210, 40, 6
     cpu, dev = small_problem(77, 2, 2, T, 128, 128, M, dtype, train=True, h0=True)
     fwd = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
-                       w=w, alpha=alpha, h0=dev["h0"], want_lse=True, want_o_swa=saved)
+                       w=w, alpha=alpha, h0=dev["h0"], want_lse=True, want_o_swa=saved != "none",
+                       want_hT=saved == "all", want_chunk_states=saved == "all")
     res = L.hybrid_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
                        fwd["lse"], dev["dO"], w=w, alpha=alpha, h0=dev["h0"], dhT=dev["dhT"],
-                       o_swa=fwd["o_swa"], want_dh0=True)
+                       o_swa=fwd["o_swa"], chunk_states=fwd["chunk_states"], hT=fwd["hT"],
+                       want_dh0=True)
     x = oracle_inputs(cpu, ("q", "k", "v", "g", "meta_k", "meta_v", "dO", "h0", "dhT"))
     ref = oracle.hybrid_bwd(x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], x["dO"], w,
                             1 / math.sqrt(128), alpha, x["h0"], x["dhT"])
@@ -107,10 +118,11 @@ def test_workload_train_sampled():
     x = I.make_inputs(wl, seed=0, device="cpu")
     dev = {k: v.cuda() for k, v in x.items()}
     fwd = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
-                       w=wl.w, alpha=wl.alpha, chunk=wl.chunk, want_lse=True, want_o_swa=True)
+                       w=wl.w, alpha=wl.alpha, chunk=wl.chunk, want_lse=True, want_o_swa=True,
+                       want_chunk_states=True)
     res = L.hybrid_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
                        fwd["lse"], dev["dO"], w=wl.w, alpha=wl.alpha, chunk=wl.chunk,
-                       o_swa=fwd["o_swa"])
+                       o_swa=fwd["o_swa"], chunk_states=fwd["chunk_states"])
     torch.cuda.synchronize()
     h = 5
     for b in range(wl.B):
