@@ -206,8 +206,10 @@ def algorithmic_bytes(kernel: str, wl) -> float | None:
         return n * (4 * d * e + 4)
     if kernel.startswith("gla_bwd") or kernel.startswith("hybrid_bwd"):
         return n * (7 * d * e + 8 * d)
-    if kernel.startswith("gla_state_pass"):
+    if kernel.startswith("gla_states"):  # state pass: reads k, v, g
         return n * (2 * d * e + 4 * d)
+    if kernel.startswith("gla_out"):  # output pass: reads q, k, v, g, writes o
+        return n * (4 * d * e + 4 * d)
     if kernel.startswith("swa_bwd_q"):
         return n * (3 * d * e + 4 + 4)
     if kernel.startswith("swa_bwd_kv"):
@@ -302,7 +304,28 @@ def kernel_table(records):
     return tab
 
 
-def roofline_for(tab, wl, peaks, traffic=None):
+TRAFFIC_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
+                            "traffic.json")
+
+
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes (read + write) per launch of `kernel` on `workload` from the
+    committed ncu summary, or None when there is none or the kernel's source
+    has changed since the counters were taken (sha256 of the file)."""
+    import hashlib
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)[kernel]
+        src = os.path.join(os.path.dirname(TRAFFIC_FILE), "..", rec["source"])
+        with open(src, "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != rec["sha256"]:
+                return None
+        return rec["bytes_per_launch"].get(workload)
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+def roofline_for(tab, wl, peaks):
     """Roofline object for the kernel with the largest total device time."""
     if not tab:
         return None, None
@@ -312,6 +335,7 @@ def roofline_for(tab, wl, peaks, traffic=None):
     by = algorithmic_bytes(dom, wl)
     if by is None:
         return dom, None
+    traffic = measured_traffic(dom, wl.name)
     achieved = by / (avg_ms * 1e-3) / 1e9
     return dom, {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
                  "peak": peaks["hbm_gbs"], "unit": "GB/s",

@@ -54,7 +54,7 @@ constexpr int DKH = 64;        // key dims per CTA
 constexpr int NT = 256;
 constexpr int KP = DKH + 8;    // padded row of the [rows][64 dims] operands
 constexpr int VP = DV + 8;     // padded row of the v / dO tiles
-constexpr int RP = DKH + 2;    // dg staging row (even: float2 access)
+constexpr int RP = DKH;        // dg staging row (64 floats, see rsw)
 constexpr int NPAIR = NSB * (NSB + 1) / 2;
 __device__ constexpr float kMinBlockDecay = 8.75651076e-27f;  // e^-60
 
@@ -65,6 +65,12 @@ __device__ __forceinline__ int swz(int row, int col) {
 // [rows][64] bf16 tile, same idea (8 chunks per row)
 __device__ __forceinline__ int swz64(int row, int col) {
   return row * 64 + ((((col >> 3) ^ row) & 7) << 3) + (col & 7);
+}
+// [rows][64] fp32 staging tile: 8-float groups XOR-swizzled by row % 4, so
+// that the float2 accesses of an MMA fragment (rows g, columns 2c) and the
+// column scans (one row, consecutive columns) are both free of bank conflicts
+__device__ __forceinline__ int rsw(int row, int col) {
+  return row * RP + (col ^ ((row & 3) << 3));
 }
 
 struct BwdSmem {
@@ -474,7 +480,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
         const float2 xv = unpack_bf16(*reinterpret_cast<const uint32_t*>(
             &(role == 0 ? sm.q[st] : sm.k[st])[swz64(t, il)]));
         if (role == 0) {
-          *reinterpret_cast<float2*>(&sm.red[t * RP + il]) = make_float2(xv.x * x0, xv.y * x1);
+          *reinterpret_cast<float2*>(&sm.red[rsw(t, il)]) = make_float2(xv.x * x0, xv.y * x1);
         } else {
           kdk[nt][2 * hh] = xv.x * x0;
           kdk[nt][2 * hh + 1] = xv.y * x1;
@@ -613,7 +619,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int t = 16 * I + gr + 8 * hh, il = nt * 8 + gc;
-          float2* r = reinterpret_cast<float2*>(&sm.red[t * RP + il]);
+          float2* r = reinterpret_cast<float2*>(&sm.red[rsw(t, il)]);
           const float2 x = *r;
           *r = make_float2(x.x - kdk[nt][2 * hh], x.y - kdk[nt][2 * hh + 1]);
         }
@@ -628,7 +634,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
 #pragma unroll
       for (int r = 0; r < SB; ++r) {  // exclusive prefix of q*dq - k*dk
         loc[r] = run;
-        run += sm.red[(16 * qq + r) * RP + col];
+        run += sm.red[rsw(16 * qq + r, col)];
       }
       sm.tot[qq][col] = run;
       __syncthreads();
@@ -651,7 +657,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int t = 16 * Iv + gr + 8 * hh, cl = nt * 8 + gc;
-          *reinterpret_cast<float2*>(&peer_red[t * RP + cl]) = make_float2(dvh[nt][2 * hh], dvh[nt][2 * hh + 1]);
+          *reinterpret_cast<float2*>(&peer_red[rsw(t, cl)]) = make_float2(dvh[nt][2 * hh], dvh[nt][2 * hh + 1]);
         }
     }
     cluster.sync();  // the peer's share has landed in red
@@ -663,7 +669,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
         for (int hh = 0; hh < 2; ++hh) {
           const int t = 16 * Iv + gr + 8 * hh, cl = nt * 8 + gc;
           if (c0 + t >= T) continue;
-          const float2 pr = *reinterpret_cast<const float2*>(&sm.red[t * RP + cl]);
+          const float2 pr = *reinterpret_cast<const float2*>(&sm.red[rsw(t, cl)]);
           float y0 = dvh[nt][2 * hh] + pr.x, y1 = dvh[nt][2 * hh + 1] + pr.y;
           const size_t off = tv + (size_t)(c0 + t) * DV + mcol + cl;
           if (p.add_dv) {
