@@ -348,7 +348,7 @@ def roofline_for(tab, wl, peaks):
 # --------------------------------------------------------------------------
 # sub-measurements
 # --------------------------------------------------------------------------
-def measure_fwd(wl, device, steps, warmup, peaks, seed, tcgen05_window=False):
+def measure_fwd(wl, device, steps, warmup, peaks, seed, tcgen05_window=True):
     import gated_linear_sliding_chunked_b200 as L
     from gated_linear_sliding_chunked_b200 import inputs as I
     x = I.make_inputs(wl, seed=seed, device=device)
@@ -517,7 +517,7 @@ def run_profile_case(args):
     L.load()
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
-    L.lz_prefer_tcgen05(args.tcgen05_window)
+    L.lz_prefer_tcgen05(not args.warp_mma_window)
     case = args.profile_case
     if case in ("train", "train-small"):
         wl = I.TRAIN_BF16 if case == "train" else I.FWD_BF16.with_(train=True)
@@ -567,8 +567,8 @@ def main(argv=None):
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
                     help="run only this workload's step (warm-up + steps) for a profiler "
                          "and print one status line; no measurement")
-    ap.add_argument("--tcgen05-window", action="store_true",
-                    help="with --profile-case: run the window forward on the tcgen05 kernel")
+    ap.add_argument("--warp-mma-window", action="store_true",
+                    help="with --profile-case: run the window forward on the warp-level kernel")
     args = ap.parse_args(argv)
     if args.profile_case:
         return run_profile_case(args)
@@ -641,11 +641,11 @@ def main(argv=None):
     if not args.no_extras:
         extras["fwd_bf16_T2048"] = measure_fwd(I.FWD_BF16, device, 10, 3, peaks, seed=rank)
         extras["long_T65536"] = measure_fwd(I.LONG_BF16, device, 3, 1, peaks, seed=rank)
-        # the same forwards with the tcgen05 window kernel (a comparison)
-        extras["fwd_bf16_T2048_tcgen05_window"] = measure_fwd(I.FWD_BF16, device, 10, 3, peaks,
-                                                              seed=rank, tcgen05_window=True)
-        extras["long_T65536_tcgen05_window"] = measure_fwd(I.LONG_BF16, device, 3, 1, peaks,
-                                                           seed=rank, tcgen05_window=True)
+        # the same forwards with the warp-level window kernel (a comparison)
+        extras["fwd_bf16_T2048_warp_mma_window"] = measure_fwd(I.FWD_BF16, device, 10, 3, peaks,
+                                                               seed=rank, tcgen05_window=False)
+        extras["long_T65536_warp_mma_window"] = measure_fwd(I.LONG_BF16, device, 3, 1, peaks,
+                                                            seed=rank, tcgen05_window=False)
         extras["decode"] = measure_decode(device, 1, 1, peaks, seed=rank)
         extras["train_step_breakdown"] = {k: [c // args.steps, round(t / c, 4)]
                                           for k, (c, t) in tab.items()}

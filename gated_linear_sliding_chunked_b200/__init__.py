@@ -142,8 +142,9 @@ def lz_device_check(stream=None):
 
 
 def lz_prefer_tcgen05(on: bool) -> bool:
-    """Selects the tcgen05 window-forward kernel (where it applies) for the
-    calling thread; returns the previous setting."""
+    """Window forward on the tcgen05 kernel where it applies (the default) or,
+    with False, on the warp-level kernel, for the calling thread; returns the
+    previous setting."""
     return bool(load().lz_prefer_tcgen05(1 if on else 0))
 
 

@@ -141,6 +141,8 @@ struct SwaBwdParams {
   float* dalpha;     // nullable [1]
   int B, H, T, dkd, dvd, w, M;
   float scale;
+  bool tc;               // key side on the tcgen05 kernel (bf16, d = 128)
+  unsigned int* status;  // device status word (set by the tcgen05 launcher)
 };
 // query rows per CTA of the meta-gradient pass (one partial per slab)
 constexpr int kSwaBwdSlab = 512;
@@ -152,6 +154,9 @@ cudaError_t launch_swa_bwd_reduce(const SwaBwdParams& p, int nparts, int nalpha,
 // tensor-core backward (bf16 I/O, dk = dv = 128); same scratch layout
 bool swa_bwd_mma_supported(int dk, int dv, bool bf16);
 cudaError_t launch_swa_bwd_mma(const SwaBwdParams& p, cudaStream_t s);
+// key side (dk, dv) on tcgen05 with TMA-fed operands
+bool swa_bwd_kv_tc_supported(int dk, int dv, bool bf16);
+cudaError_t launch_swa_bwd_kv_tc(const SwaBwdParams& p, cudaStream_t s);
 
 // ---- decode --------------------------------------------------------------
 struct DecodeParams {

@@ -11,11 +11,11 @@
 namespace {
 
 thread_local std::string g_err;
-thread_local bool g_prefer_tc = false;  // lz_prefer_tcgen05
+thread_local bool g_prefer_tc = true;  // lz_prefer_tcgen05
 
-// The window branch's forward: warp-level MMA for bf16 with dk = dv = 128
-// (tcgen05 instead when the calling thread prefers it and w <= 129), fp32
-// SIMT otherwise.
+// The window branch's forward for bf16 with dk = dv = 128: tcgen05 for
+// w <= 129 (unless the calling thread asked for the warp-level kernel),
+// warp-level MMA otherwise; fp32 SIMT for the other shapes.
 cudaError_t swa_forward(const lz::SwaFwdParams& p, bool bf16, cudaStream_t s) {
   if (g_prefer_tc && lz::swa_fwd_tc_supported(p.dk, p.dv, bf16, p.w)) return lz::launch_swa_fwd_tc(p, s);
   if (lz::swa_fwd_mma_supported(p.dk, p.dv, bf16)) return lz::launch_swa_fwd_mma(p, s);
@@ -292,6 +292,7 @@ lz::SwaBwdParams swa_bwd_params(const lz_dims* d, const void* q, const void* k, 
   lz::SwaBwdParams p{};
   p.q = q; p.k = k; p.v = v; p.mk = mk; p.mv = d->M > 0 ? mv : nullptr; p.lse = lse; p.dO = dO;
   p.osw = osw;
+  p.tc = g_prefer_tc;
   p.Dbuf = w.Dbuf; p.alpha_part = w.alpha_part; p.meta_part = w.meta_part;
   p.B = d->B; p.H = d->H; p.T = d->T; p.dkd = d->dk; p.dvd = d->dv; p.w = d->w; p.M = d->M;
   p.scale = d->scale;

@@ -1,0 +1,279 @@
+// Key side of the window + meta softmax backward on the Blackwell tensor
+// cores: tcgen05.mma with dK, dV accumulated in tensor memory, operands
+// brought in by TMA (bf16 I/O, fp32 accumulation, dk = dv = 128).
+//
+// Lizard technical summary, section 2a: key j is seen by queries
+// t in [j, j + w - 1].  With P = exp(logit - lse), the window branch's share
+// gscale * dO of the output gradient and D_t = dO_t . o_t:
+//   dV_j = gscale * sum_t P_tj dO_t,   dK_j = scale * gscale * sum_t dS_tj q_t,
+//   dS_tj = P_tj (dO_t . v_j - D_t).
+// One CTA = 128 keys of one (batch, head), 8 warps; it walks the 64-query
+// tiles that see them.  Per tile:
+//   thread 0: the NEXT tile's S^T = K Q^T and dP^T = V dO^T (M = 128 keys,
+//             N = 64 queries) into the other half of a double-buffered TMEM
+//             pair, so that they run while this tile's softmax does;
+//   all:      each key row's two threads read 32 query columns of this
+//             tile's scores, form P^T and dS^T (bf16) in shared memory;
+//   thread 0: dV += P^T dO, dK += dS^T Q (M = 128, N = 128, K = 64), commit.
+// Q / dO tiles rotate through three shared-memory buffers, loaded by TMA
+// two tiles ahead.
+// K, V (K-major) and the Q / dO tiles sit in shared memory 128-byte
+// swizzled as TMA writes them; the gradient MMAs read Q / dO as MN-major B
+// operands (rows = queries, the reduction dim) from the same tiles.
+#include <cstddef>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "mma.cuh"
+#include "tc05.cuh"
+#include "tma_host.h"
+
+namespace lz {
+namespace {
+
+constexpr int KR = 128;   // keys per CTA (MMA M)
+constexpr int QT = 64;    // queries per tile
+constexpr int D = 128;
+constexpr int NTH = 256;
+constexpr uint32_t kHalf = 64 * 2;  // bytes of one swizzled row (64 dims)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColDK = 0, kColDV = 128, kColS = 256, kColDP = 384;  // S^T, dP^T: + 64 * buffer
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct KvSmem {
+  uint8_t k[2][KR * kHalf];       // dims [0,64), [64,128): 128 key rows each
+  uint8_t v[2][KR * kHalf];
+  uint8_t q[3][2][QT * kHalf];    // [buffer][dim half]: 64 query rows
+  uint8_t dO[3][2][QT * kHalf];
+  uint8_t pt[KR * QT * 2];        // P^T, bf16, no-swizzle K-major
+  uint8_t dst[KR * QT * 2];       // dS^T
+  float lse2[3][QT];              // lse * log2(e) of the tile's queries
+  float dq[3][QT];                // D of the tile's queries
+  uint64_t bar_kv;
+  uint64_t bar_ld[3];
+  uint64_t bar_s[2];
+  uint64_t bar_o;
+  uint32_t tmem_base;
+};
+static_assert(sizeof(KvSmem) + 1024 <= 232448, "shared memory per block exceeds 227 KB");
+static_assert(offsetof(KvSmem, v) % 1024 == 0 && offsetof(KvSmem, q) % 1024 == 0 &&
+                  offsetof(KvSmem, dO) % 1024 == 0 && offsetof(KvSmem, pt) % 1024 == 0,
+              "swizzled tiles must be 1024-byte aligned");
+
+__global__ void __launch_bounds__(NTH, 1)
+    swa_bwd_kv_tc_kernel(SwaBwdParams p, const __grid_constant__ CUtensorMap tk,
+                         const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tq,
+                         const __grid_constant__ CUtensorMap tdo) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  KvSmem& sm = *reinterpret_cast<KvSmem*>(smem_raw + ((1024u - (raw & 1023u)) & 1023u));
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int bh = blockIdx.y;
+  const int T = p.T, w = p.w;
+  const int j0 = blockIdx.x * KR;
+  const int tq_hi = min(T - 1, j0 + KR - 1 + w - 1);
+  const int nq = (tq_hi - j0 + QT) / QT;  // >= 1
+  const float* lse = p.lse + (size_t)bh * T;
+  const float* Db = p.Dbuf + (size_t)bh * T;
+  const float c2 = p.scale * kLog2e;
+
+  const uint32_t s_k = smem_u32(sm.k), s_v = smem_u32(sm.v), s_q = smem_u32(sm.q);
+  const uint32_t s_do = smem_u32(sm.dO), s_pt = smem_u32(sm.pt), s_dst = smem_u32(sm.dst);
+  const uint32_t bar_kv = smem_u32(&sm.bar_kv), bar_o = smem_u32(&sm.bar_o);
+  const uint32_t bar_ld0 = smem_u32(&sm.bar_ld[0]), bar_s0 = smem_u32(&sm.bar_s[0]);  // + 8 per buffer
+  constexpr uint32_t kTileBytes = 2 * 2 * QT * kHalf;                               // Q and dO, both halves
+
+  // query tile i -> buffer i % 3: Q / dO by TMA (thread 0), lse and D by threads
+  auto issue_tile = [&](int i) {
+    const int b = i % 3, t = j0 + i * QT;
+    mbar_expect_tx(bar_ld0 + 8 * b, kTileBytes);
+    for (int hf = 0; hf < 2; ++hf) {
+      tma_load_3d(s_q + (2 * b + hf) * QT * kHalf, &tq, bar_ld0 + 8 * b, hf * 64, t, bh);
+      tma_load_3d(s_do + (2 * b + hf) * QT * kHalf, &tdo, bar_ld0 + 8 * b, hf * 64, t, bh);
+    }
+  };
+  auto load_stats = [&](int i) {
+    const int b = i % 3, t = j0 + i * QT;
+    if (tid < QT) sm.lse2[b][tid] = t + tid < T ? lse[t + tid] * kLog2e : 0.f;
+    else if (tid < 2 * QT) sm.dq[b][tid - QT] = t + tid - QT < T ? Db[t + tid - QT] : 0.f;
+  };
+  // S^T and dP^T of tile i (shared-memory buffer i % 3) into TMEM buffer i & 1
+  auto issue_scores = [&](int i, uint32_t tmem) {
+    const int b = i % 3, tb = i & 1;
+    constexpr uint32_t idS = idesc_bf16(KR, QT, false);
+#pragma unroll 1
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t hf = kk >> 2, ko = (kk & 3) * 32;
+      mma_bf16_ss(tmem + kColS + QT * tb, sdesc_sw128(s_k + hf * KR * kHalf + ko, 16, 1024),
+                  sdesc_sw128(s_q + (2 * b + hf) * QT * kHalf + ko, 16, 1024), idS, kk > 0);
+      mma_bf16_ss(tmem + kColDP + QT * tb, sdesc_sw128(s_v + hf * KR * kHalf + ko, 16, 1024),
+                  sdesc_sw128(s_do + (2 * b + hf) * QT * kHalf + ko, 16, 1024), idS, kk > 0);
+    }
+    mma_commit(bar_s0 + 8 * tb);
+  };
+
+  if (warp == 0) tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
+  if (tid == 0) {
+    mbar_init(bar_kv, 1);
+    mbar_init(bar_ld0, 1);
+    mbar_init(bar_ld0 + 8, 1);
+    mbar_init(bar_ld0 + 16, 1);
+    mbar_init(bar_s0, 1);
+    mbar_init(bar_s0 + 8, 1);
+    mbar_init(bar_o, 1);
+    mbar_init_fence();
+  }
+  for (int i = 0; i < 3 && i < nq; ++i) load_stats(i);
+  tc_fence_before();
+  __syncthreads();  // barriers, TMEM address, first statistics
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  bool alive = true;
+  if (tid == 0) {
+    mbar_expect_tx(bar_kv, 2 * 2 * KR * kHalf);
+    for (int hf = 0; hf < 2; ++hf) {
+      tma_load_3d(s_k + hf * KR * kHalf, &tk, bar_kv, hf * 64, j0, bh);
+      tma_load_3d(s_v + hf * KR * kHalf, &tv, bar_kv, hf * 64, j0, bh);
+    }
+    for (int i = 0; i < 3 && i < nq; ++i) issue_tile(i);
+    alive = mbar_wait(bar_kv, 0, p.status) && mbar_wait(bar_ld0, 0, p.status);
+    if (alive) issue_scores(0, tmem);
+  }
+
+  // this thread: key row kr (TMEM lane), query columns [32 hf, 32 hf + 32)
+  const int kr = tid & (KR - 1), hf = tid >> 7;
+  const int j = j0 + kr;
+  const uint32_t lrow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+#pragma unroll 1
+  for (int i = 0; i < nq; ++i) {
+    const int b = i % 3, tb = i & 1;
+    const int t0c = j0 + i * QT + hf * 32;  // first query column of this thread
+    // the next tile's scores run on the tensor cores during this softmax
+    // (TMEM buffer (i + 1) & 1 was last read before the previous barrier)
+    if (tid == 0 && alive && i + 1 < nq) {
+      alive = mbar_wait(bar_ld0 + 8 * ((i + 1) % 3), ((i + 1) / 3) & 1, p.status);
+      if (alive) issue_scores(i + 1, tmem);
+    }
+    if (alive) alive = mbar_wait(bar_s0 + 8 * tb, (i >> 1) & 1, p.status);
+    tc_fence_after();
+    uint32_t s[32], dp[32];
+    tmem_ld32(lrow + kColS + QT * tb + hf * 32, s);
+    tmem_ld32(lrow + kColDP + QT * tb + hf * 32, dp);
+    tmem_ld_wait();
+    if (i > 0) {  // tile i-1's gradient MMAs are done: P^T, dS^T and its buffer are free
+      if (alive) alive = mbar_wait(bar_o, (i - 1) & 1, p.status);
+      if (i + 2 < nq) {
+        if (tid == 0 && alive) issue_tile(i + 2);
+        load_stats(i + 2);
+      }
+    }
+    // P^T, dS^T of this thread's 32 columns
+    uint32_t pk[16], dk2[16];
+#pragma unroll
+    for (int c = 0; c < 32; c += 2) {
+      float pr[2], ds[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int t = t0c + c + e, cl = hf * 32 + c + e;
+        const bool ok = j < T && t < T && (unsigned)(t - j) < (unsigned)w;
+        const float P = ok ? exp2f(fmaf(__uint_as_float(s[c + e]), c2, -sm.lse2[b][cl])) : 0.f;
+        pr[e] = P;
+        ds[e] = P * (__uint_as_float(dp[c + e]) - sm.dq[b][cl]);
+      }
+      pk[c / 2] = pack_bf16(pr[0], pr[1]);
+      dk2[c / 2] = pack_bf16(ds[0], ds[1]);
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {  // K-major [128 keys][64 queries], 8-row groups 1024 bytes apart
+      const uint32_t off = (kr >> 3) * 1024 + (hf * 4 + x) * 128 + (kr & 7) * 16;
+      *reinterpret_cast<uint4*>(sm.pt + off) = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+      *reinterpret_cast<uint4*>(sm.dst + off) =
+          make_uint4(dk2[4 * x], dk2[4 * x + 1], dk2[4 * x + 2], dk2[4 * x + 3]);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    alive = __syncthreads_and(alive);
+    if (tid == 0 && alive) {
+      tc_fence_after();
+      constexpr uint32_t idG = idesc_bf16(KR, D, true);
+#pragma unroll
+      for (int kk = 0; kk < QT / 16; ++kk) {  // B: Q / dO as MN-major, 16 queries = 2048 bytes
+        const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+        mma_bf16_ss(tmem + kColDV, sdesc(s_pt + kk * 256, 128, 1024),
+                    sdesc_sw128(s_do + 2 * b * QT * kHalf + kk * 2048, QT * kHalf, 1024), idG, acc);
+        mma_bf16_ss(tmem + kColDK, sdesc(s_dst + kk * 256, 128, 1024),
+                    sdesc_sw128(s_q + 2 * b * QT * kHalf + kk * 2048, QT * kHalf, 1024), idG, acc);
+      }
+      mma_commit(bar_o);
+    }
+  }
+  if (alive) alive = mbar_wait(bar_o, (nq - 1) & 1, p.status);
+  tc_fence_after();
+
+  // ---- epilogue: dK, dV rows of this CTA's keys, 64 columns per thread ------
+  const size_t off = ((size_t)bh * T + j) * D;
+  const float sk = p.scale * p.gscale, sv = p.gscale;
+#pragma unroll 1
+  for (int g = 0; g < 2; ++g) {  // 0: dK, 1: dV
+#pragma unroll 1
+    for (int c0 = hf * 64; c0 < hf * 64 + 64; c0 += 32) {
+      uint32_t r[32];
+      tmem_ld32(lrow + (g == 0 ? kColDK : kColDV) + c0, r);
+      tmem_ld_wait();
+      if (!alive || j >= T) continue;
+      const float sc = g == 0 ? sk : sv;
+      float* f32 = g == 0 ? p.dk_f32 : p.dv_f32;
+      if (f32) {
+        float4* dst = reinterpret_cast<float4*>(f32 + off + c0);
+#pragma unroll
+        for (int x = 0; x < 8; ++x)
+          dst[x] = make_float4(__uint_as_float(r[4 * x]) * sc, __uint_as_float(r[4 * x + 1]) * sc,
+                               __uint_as_float(r[4 * x + 2]) * sc, __uint_as_float(r[4 * x + 3]) * sc);
+      } else {
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2)
+          pk[c / 2] = pack_bf16(__uint_as_float(r[c]) * sc, __uint_as_float(r[c + 1]) * sc);
+        uint4* dst = reinterpret_cast<uint4*>((bf16*)(g == 0 ? p.dk : p.dv) + off + c0);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+bool swa_bwd_kv_tc_supported(int dk, int dv, bool bf16) { return bf16 && dk == D && dv == D; }
+
+cudaError_t launch_swa_bwd_kv_tc(const SwaBwdParams& p, cudaStream_t s) {
+  if (p.B * p.H == 0 || p.T == 0) return cudaSuccess;
+  const size_t bytes = sizeof(KvSmem) + 1024;  // + room to align the base to 1024
+  cudaError_t e = cudaFuncSetAttribute(swa_bwd_kv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)bytes);
+  if (e != cudaSuccess) return e;
+  SwaBwdParams pp = p;
+  pp.status = device_status_word();
+  if (pp.status == nullptr) return cudaErrorInvalidDevicePointer;
+  const uint64_t bh = (uint64_t)p.B * p.H;
+  CUtensorMap tk, tv, tq, tdo;
+  if (!tma_map_rows128(&tk, p.k, p.T, bh, KR) || !tma_map_rows128(&tv, p.v, p.T, bh, KR) ||
+      !tma_map_rows128(&tq, p.q, p.T, bh, QT) || !tma_map_rows128(&tdo, p.dO, p.T, bh, QT))
+    return cudaErrorInvalidValue;
+  dim3 grid((p.T + KR - 1) / KR, p.B * p.H);
+  {
+    ScopedTiming tm("swa_bwd_kv_tc", s);
+    swa_bwd_kv_tc_kernel<<<grid, NTH, bytes, s>>>(pp, tk, tv, tq, tdo);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace lz

@@ -535,14 +535,18 @@ cudaError_t launch_swa_bwd_mma(const SwaBwdParams& p, cudaStream_t s) {
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const size_t b2 = sizeof(KVSmem);
-    e = cudaFuncSetAttribute(swa_bwd_kv_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)b2);
-    if (e != cudaSuccess) return e;
-    {
-      ScopedTiming tm("swa_bwd_kv_mma", s);
-      swa_bwd_kv_mma_kernel<<<dim3((p.T + KT2 - 1) / KT2, p.B * p.H), NT, b2, s>>>(p);
+    if (p.tc && swa_bwd_kv_tc_supported(p.dkd, p.dvd, true)) {
+      e = launch_swa_bwd_kv_tc(p, s);
+    } else {
+      const size_t b2 = sizeof(KVSmem);
+      e = cudaFuncSetAttribute(swa_bwd_kv_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)b2);
+      if (e != cudaSuccess) return e;
+      {
+        ScopedTiming tm("swa_bwd_kv_mma", s);
+        swa_bwd_kv_mma_kernel<<<dim3((p.T + KT2 - 1) / KT2, p.B * p.H), NT, b2, s>>>(p);
+      }
+      e = cudaGetLastError();
     }
-    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   const int nparts = (p.M > 0 && !empty) ? p.B * nslab : 0;

@@ -3,15 +3,19 @@
 // single-thread tcgen05.mma issue with completion on an mbarrier, and the
 // TMEM -> register loads of the accumulators.
 //
-// Shared-memory operands use the canonical no-swizzle ("interleaved")
-// layout: the unit is a core matrix of 8 rows x 16 bytes stored as 128
-// contiguous bytes.
+// Shared-memory operands written by threads use the canonical no-swizzle
+// ("interleaved") layout: the unit is a core matrix of 8 rows x 16 bytes
+// stored as 128 contiguous bytes.
 //   K-major operand (rows = M or N, 16-byte chunks along K):
 //     byte(row, kc) = (row / 8) * SBO + kc * LBO + (row % 8) * 16
 //   MN-major operand (16-byte chunks along M/N, rows along K):
 //     byte(kr, nc)  = nc * SBO + (kr / 8) * LBO + (kr % 8) * 16
 // One kind::f16 MMA consumes K = 16 (two core matrices along K), so the next
-// K step starts 2 * LBO bytes further.
+// K step starts 2 * LBO bytes further.  Operands loaded by TMA use the
+// 128-byte swizzle instead (sdesc_sw128): a [rows][64] bf16 box is rows of
+// 128 bytes; K-major, a K step of 16 moves the start 32 bytes along the row
+// and SBO = 1024 steps 8 rows; MN-major (rows = K), a K step of 16 moves 2048
+// bytes, SBO = 1024 steps 8 K-rows and LBO steps to the next 64-wide block.
 //
 // The accumulator D of an M = 128, cta_group::1 MMA sits in TMEM lanes
 // 0..127 (lane = row), one fp32 column per output column.  Warp w of the CTA
@@ -65,6 +69,25 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
   return false;
 }
 
+// ---- TMA (tensor copies global -> shared, no multicast) --------------------
+// The issuing thread announces the bytes the barrier's current phase waits
+// for (and arrives once); every tensor copy then completes part of them.
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+// Box at (c0, c1, c2) of the 3-D tensor map `map` (a __grid_constant__
+// kernel parameter) into shared memory at dst; rows outside the tensor read
+// as zeros.  c0 * element size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* map, uint32_t bar, int c0, int c1,
+                                            int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
 // ---- proxies and ordering -------------------------------------------------
 // Makes this thread's generic-proxy shared-memory writes (st.shared,
 // cp.async) visible to the tensor core's async proxy.
@@ -94,6 +117,12 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+// The same with the 128-byte swizzle of TMA tiles: 8 rows of 128 bytes form
+// a 1024-byte atom whose 16-byte chunks are XOR-permuted by row % 8; atoms
+// must start 1024-byte aligned.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return sdesc(saddr, lbo, sbo) | (2ull << 61);
 }
 // Instruction descriptor of kind::f16 with bf16 A and B, fp32 accumulation,
 // K-major A; B K-major (b_mn = false) or MN-major (b_mn = true).

@@ -1,0 +1,15 @@
+// Host-side TMA tensor maps for the tcgen05 kernels.
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+namespace lz {
+
+// 3-D map over a contiguous bf16 tensor [d2][d1][128] (rows of 128 elements),
+// boxes of 64 elements x `rows` rows x 1 with the 128-byte swizzle; rows
+// outside the tensor read as zeros.  False if the driver's encoder is not
+// available or rejects the map.
+bool tma_map_rows128(CUtensorMap* map, const void* base, uint64_t d1, uint64_t d2, uint32_t rows);
+
+}  // namespace lz

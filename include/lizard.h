@@ -217,13 +217,14 @@ lz_status lz_gla_decode_step(int Bd, int H, int dk, int dv, int w, int M,
  * last check (LZ_OK otherwise; LZ_ERR_CUDA if the read failed). */
 lz_status lz_device_check(lz_stream stream);
 
-/* Window-forward kernel choice for the calling host thread (no counterpart
- * on the pages).  bf16 with dk = dv = 128 has two tensor-core kernels:
- * warp-level mma.sync with an online softmax (any w; the default, faster
- * today) and tcgen05 with the scores of the whole band in tensor memory
- * (w <= 129).  lz_prefer_tcgen05(1) selects the tcgen05 kernel where it
- * applies; both give the same result up to rounding.  Returns the previous
- * setting; never fails. */
+/* Kernel choice of the window branch for the calling host thread (no
+ * counterpart on the pages).  bf16 with dk = dv = 128 has tcgen05 kernels
+ * with TMA-fed operands and accumulators in tensor memory (the default) and
+ * warp-level mma.sync kernels: the forward uses tcgen05 for w <= 129 (the
+ * scores of the whole band fit in tensor memory), the key side of the
+ * backward (dk, dv) for every w.  lz_prefer_tcgen05(0) selects the
+ * warp-level kernels; both give the same result up to rounding.  Returns
+ * the previous setting; never fails. */
 int lz_prefer_tcgen05(int on);
 
 /* Per-launch device timing for benchmarks (no counterpart on the pages; a

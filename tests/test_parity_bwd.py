@@ -65,6 +65,28 @@ def test_swa_meta_bwd(dtype, T, w, M, sink, with_o):
             assert_close("dmeta_v", res["dmeta_v"], ref["dmeta_v"], dtype)
 
 
+@pytest.mark.parametrize("T,w,M", [(1, 1, 2), (300, 64, 4), (1100, 128, 8), (260, 700, 0)])
+@pytest.mark.parametrize("tc", [True, False], ids=["tcgen05", "warp-mma"])
+def test_swa_meta_bwd_kernels(T, w, M, tc):
+    """Both bf16 key-side kernels (tcgen05 and warp-level) against the oracle,
+    with a clean device status word afterwards."""
+    cpu, dev = small_problem(90 + T + w, 2, 2, T, 128, 128, M, torch.bfloat16, train=True)
+    mk = dev["meta_k"] if M else None
+    mv = dev["meta_v"] if M else None
+    prev = L.lz_prefer_tcgen05(tc)
+    try:
+        o, lse = L.swa_meta_fwd(dev["q"], dev["k"], dev["v"], mk, mv, w=w)
+        res = L.swa_meta_bwd(dev["q"], dev["k"], dev["v"], mk, mv, lse, dev["dO"], w=w, o=o)
+    finally:
+        L.lz_prefer_tcgen05(prev)
+    L.lz_device_check()
+    x = oracle_inputs(cpu, ("q", "k", "v", "meta_k", "meta_v", "dO"))
+    ref = oracle.swa_meta_bwd(x["q"], x["k"], x["v"], x["meta_k"] if M else None,
+                              x["meta_v"] if M else None, x["dO"], w, 1 / math.sqrt(128))
+    for name in ("dq", "dk", "dv"):
+        assert_close(name, res[name], ref[name], torch.bfloat16)
+
+
 @pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
 @pytest.mark.parametrize("alpha", [0.0, 0.5, 2.0])
 @pytest.mark.parametrize("saved", ["none", "o_swa", "all"])

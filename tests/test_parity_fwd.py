@@ -152,14 +152,15 @@ def test_workload_long_context_sampled():
 
 
 def test_window_forward_dispatch_and_device_status():
-    """bf16, d = 128: the warp-level kernel by default; the tcgen05 kernel
-    when preferred and w <= 129; no bounded device wait gives up."""
+    """bf16, d = 128: the tcgen05 kernel by default for w <= 129, the
+    warp-level one for wider windows or when asked for; no bounded device
+    wait gives up."""
     cpu, dev = small_problem(21, 2, 2, 700, 128, 128, 8, torch.bfloat16)
     L.lz_timing_read()
     L.lz_timing_enable(True)
-    prev = L.lz_prefer_tcgen05(False)
+    prev = L.lz_prefer_tcgen05(True)
     try:
-        for tc in (False, True):
+        for tc in (True, False):
             L.lz_prefer_tcgen05(tc)
             for w in (129, 300):
                 L.swa_meta_fwd(dev["q"], dev["k"], dev["v"], dev["meta_k"], dev["meta_v"], w=w)
@@ -167,18 +168,19 @@ def test_window_forward_dispatch_and_device_status():
     finally:
         L.lz_timing_enable(False)
         L.lz_prefer_tcgen05(prev)
-    assert names == ["swa_fwd_mma", "swa_fwd_mma", "swa_fwd_tc", "swa_fwd_mma"], names
+    assert names == ["swa_fwd_tc", "swa_fwd_mma", "swa_fwd_mma", "swa_fwd_mma"], names
     L.lz_device_check()
 
 
 @pytest.mark.parametrize("T,w,M,sink", [(1, 1, 0, False), (77, 7, 0, False), (130, 64, 4, True),
                                         (333, 128, 16, False), (700, 129, 8, False)])
-def test_swa_meta_fwd_tcgen05(T, w, M, sink):
-    """The tcgen05 window forward against the oracle."""
+@pytest.mark.parametrize("tc", [True, False], ids=["tcgen05", "warp-mma"])
+def test_swa_meta_fwd_kernels(T, w, M, sink, tc):
+    """Both bf16 window forwards against the oracle."""
     cpu, dev = small_problem(7 + T + w, 1, 3, T, 128, 128, M, torch.bfloat16)
     mk = dev["meta_k"] if M else None
     mv = dev["meta_v"] if (M and not sink) else None
-    prev = L.lz_prefer_tcgen05(True)
+    prev = L.lz_prefer_tcgen05(tc)
     try:
         o, lse = L.swa_meta_fwd(dev["q"], dev["k"], dev["v"], mk, mv, w=w)
     finally:
