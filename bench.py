@@ -62,6 +62,15 @@ def max_over_ranks(x: float, device) -> float:
     return float(t.item())
 
 
+def aggregate_step(ms: float, tokens_per_rank_step: int, device):
+    """(job step time, whole-job tokens/s): every rank runs its own replica
+    (weak scaling, no data-path collective), the job's step takes as long as
+    the slowest rank, and the job's tokens are all ranks' tokens."""
+    world = dist.get_world_size() if (dist.is_available() and dist.is_initialized()) else 1
+    ms_max = max_over_ranks(ms, device)
+    return ms_max, tokens_per_rank_step * world / (ms_max * 1e-3)
+
+
 def sum_over_ranks(x: float, device) -> float:
     if not (dist.is_available() and dist.is_initialized()):
         return float(x)
@@ -609,9 +618,8 @@ def main(argv=None):
         ms = time_region(step.run, args.steps, device)
     L.lz_timing_enable(False)
     records = L.lz_timing_read()
-    ms_max = max_over_ranks(ms, device)
     tokens_step = wl.B * wl.T
-    value = tokens_step * world / (ms_max * 1e-3)
+    ms_max, value = aggregate_step(ms, tokens_step, device)
     tab = kernel_table(records)
     launches = len(records)
     dom, roof = roofline_for(tab, wl, peaks)
@@ -633,8 +641,7 @@ def main(argv=None):
 
     e2e_steps = max(3, min(args.steps, 10))
     e2e_step()
-    ms_e2e = max_over_ranks(time_region(e2e_step, e2e_steps, device), device)
-    e2e_val = tokens_step * world / (ms_e2e * 1e-3)
+    ms_e2e, e2e_val = aggregate_step(time_region(e2e_step, e2e_steps, device), tokens_step, device)
     del xe
 
     extras = {}
