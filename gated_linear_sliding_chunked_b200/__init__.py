@@ -32,7 +32,7 @@ LZ_F32, LZ_BF16 = 0, 1
 EXPORTS = ("lz_gla_fwd", "lz_gla_bwd", "lz_swa_meta_fwd", "lz_hybrid_fwd", "lz_swa_meta_bwd",
            "lz_hybrid_bwd", "lz_gla_decode_step", "lz_workspace_bytes", "lz_last_error",
            "lz_version", "lz_timing_enable", "lz_timing_read", "lz_swa_meta_bwd_noalloc",
-           "lz_device_check", "lz_prefer_tcgen05")
+           "lz_device_check", "lz_prefer_tcgen05", "lz_decode_prefill")
 
 # size of the static scratch array behind lz_swa_meta_bwd_noalloc
 LZ_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -78,6 +78,7 @@ def load(path: str = LIB_PATH):
     lib.lz_gla_decode_step.argtypes = ([ctypes.c_int] * 7 + [ctypes.c_float] * 2 +
                                        [_P] * 11 + [_P])
     lib.lz_device_check.argtypes = [_P]
+    lib.lz_decode_prefill.argtypes = [ctypes.c_int] * 7 + [_P] * 7 + [_P]
     lib.lz_prefer_tcgen05.argtypes = [ctypes.c_int]
     lib.lz_timing_enable.argtypes = [ctypes.c_int]
     lib.lz_timing_read.argtypes = [ctypes.c_char_p, sz, ctypes.POINTER(ctypes.c_float),
@@ -342,6 +343,27 @@ def hybrid_bwd(q, k, v, g, meta_k, meta_v, lse, dO, *, w, alpha, scale=None, chu
                   dk, dv, dg, dh0, dmk, dmv, dalpha, ws, n, stream)
     return {"dq": dq, "dk": dk, "dv": dv, "dg": dg, "dh0": dh0, "dmeta_k": dmk,
             "dmeta_v": dmv, "dalpha": dalpha[:1]}
+
+
+def lz_decode_prefill(Bd, H, T, dk, dv, w, io, k, v, hT, state, kring, vring, pos, stream=None):
+    _check(load().lz_decode_prefill(Bd, H, T, dk, dv, w, io, _ptr(k), _ptr(v), _ptr(hT),
+                                    _ptr(state), _ptr(kring), _ptr(vring), _ptr(pos),
+                                    _stream(stream)))
+
+
+def decode_prefill(k, v, hT, *, w, stream=None):
+    """Decode buffers after a prefill of k, v [Bd, H, T, 128] with final state
+    hT: returns (state, kring, vring, pos) ready for decode_step."""
+    Bd, H, T, dk = k.shape
+    dv = v.shape[-1]
+    dev = k.device
+    state = torch.empty(Bd, H, dk, dv, dtype=torch.float32, device=dev)
+    kring = torch.zeros(Bd, H, w, dk, dtype=k.dtype, device=dev)
+    vring = torch.zeros(Bd, H, w, dv, dtype=v.dtype, device=dev)
+    pos = torch.empty(Bd, dtype=torch.int64, device=dev)
+    lz_decode_prefill(Bd, H, T, dk, dv, w, io_of(k.dtype), k, v, hT, state, kring, vring, pos,
+                      stream)
+    return state, kring, vring, pos
 
 
 def decode_step(state, kring, vring, pos, q, k, v, g, meta_k, meta_v, *, alpha, scale=None,

@@ -181,12 +181,47 @@ __global__ void __launch_bounds__(NT) decode_kernel(DecodeParams p) {
   }
 }
 
+// Prefill -> decode hand-off: the state becomes the prefill's final state,
+// the ring slot t mod w holds token t of the last min(T, w) prompt tokens,
+// pos = T.  One CTA per (sequence, head).
+template <typename IO>
+__global__ void __launch_bounds__(NT) decode_prefill_kernel(DecodePrefillParams p) {
+  const int tid = threadIdx.x;
+  const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
+  const int T = p.T, w = p.w;
+  float4* st = reinterpret_cast<float4*>(p.state + (size_t)bh * D * D);
+  const float4* src = p.hT ? reinterpret_cast<const float4*>(p.hT + (size_t)bh * D * D) : nullptr;
+  for (int x = tid; x < D * D / 4; x += NT) st[x] = src ? src[x] : make_float4(0.f, 0.f, 0.f, 0.f);
+  const int t0 = T > w ? T - w : 0;
+  constexpr int CH = D * (int)sizeof(IO) / 16;  // 16-byte chunks per row
+  const uint4* ks = reinterpret_cast<const uint4*>((const IO*)p.k + (size_t)bh * T * D);
+  const uint4* vs = reinterpret_cast<const uint4*>((const IO*)p.v + (size_t)bh * T * D);
+  uint4* kr = reinterpret_cast<uint4*>((IO*)p.kring + (size_t)bh * w * D);
+  uint4* vr = reinterpret_cast<uint4*>((IO*)p.vring + (size_t)bh * w * D);
+  for (int x = tid; x < (T - t0) * CH; x += NT) {
+    const int t = t0 + x / CH, c = x % CH, slot = t % w;
+    kr[(size_t)slot * CH + c] = ks[(size_t)t * CH + c];
+    vr[(size_t)slot * CH + c] = vs[(size_t)t * CH + c];
+  }
+  if (h == 0 && tid == 0) p.pos[b] = T;
+}
+
 __global__ void decode_pos_kernel(int64_t* pos, int Bd) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < Bd) pos[b] = (pos[b] < 0 ? 0 : pos[b]) + 1;
 }
 
 }  // namespace
+
+cudaError_t launch_decode_prefill(const DecodePrefillParams& p, bool bf16, cudaStream_t s) {
+  if (p.Bd == 0 || p.H == 0) return cudaSuccess;
+  {
+    ScopedTiming tm("decode_prefill", s);
+    if (bf16) decode_prefill_kernel<lz::bf16><<<p.Bd * p.H, NT, 0, s>>>(p);
+    else decode_prefill_kernel<float><<<p.Bd * p.H, NT, 0, s>>>(p);
+  }
+  return cudaGetLastError();
+}
 
 cudaError_t launch_decode(const DecodeParams& p, bool bf16, cudaStream_t s) {
   if (p.Bd == 0 || p.H == 0) return cudaSuccess;

@@ -174,6 +174,17 @@ struct DecodeParams {
   const void* mv;
   void* o;
 };
+struct DecodePrefillParams {
+  int Bd, H, T, w;
+  const void* k;     // [Bd,H,T,128] io dtype
+  const void* v;
+  const float* hT;   // [Bd,H,128,128], nullable = zeros
+  float* state;
+  void* kring;
+  void* vring;
+  int64_t* pos;
+};
+cudaError_t launch_decode_prefill(const DecodePrefillParams& p, bool bf16, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams& p, bool bf16, cudaStream_t s);
 
 }  // namespace lz

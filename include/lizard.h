@@ -207,6 +207,19 @@ lz_status lz_gla_decode_step(int Bd, int H, int dk, int dv, int w, int M,
                              const void* meta_k, const void* meta_v, void* o,
                              lz_stream stream);
 
+/* Hand-off from a prefill to lz_gla_decode_step (section 2a: generation
+ * continues from the fixed-size state and the last w keys/values).  For Bd
+ * prompts of T tokens each: state = hT (the prefill's final state from
+ * lz_gla_fwd / lz_hybrid_fwd, [Bd,H,dk,dv] fp32; NULL = zeros); ring slot
+ * (t mod w) = k_t, v_t for the last min(T, w) prompt tokens (k, v
+ * [Bd,H,T,dk/dv] io dtype, the prefill's layout); pos = T.  Ring slots not
+ * written keep their contents (the decode step never reads them).
+ * Supported: dk = dv = 128, 1 <= w <= 1024. */
+lz_status lz_decode_prefill(int Bd, int H, int T, int dk, int dv, int w,
+                            lz_dtype io, const void* k, const void* v,
+                            const float* hT, float* state, void* kring,
+                            void* vring, int64_t* pos, lz_stream stream);
+
 /* Device-side status (no counterpart on the pages; a robustness aid).  The
  * tcgen05 kernels wait on mbarriers for their tensor-core work; every such
  * wait is bounded (0.2 s) and, when it gives up, adds one to a status word

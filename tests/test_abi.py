@@ -161,3 +161,17 @@ def test_chunk_states_size_and_validation(lib):
     G = [FAKE] * 14
     G[9] = None
     assert lib.lz_gla_bwd(ctypes.byref(d), *G, FAKE, 1 << 40, 0) == L.LZ_ERR_INVALID_ARG
+
+
+def test_decode_prefill_validation(lib):
+    f = lib.lz_decode_prefill
+    args = [FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE]  # k, v, hT, state, kring, vring, pos
+    assert f(2, 2, 10, 64, 128, 16, L.LZ_BF16, *args, 0) == L.LZ_ERR_UNSUPPORTED
+    assert f(2, 2, 10, 128, 128, 0, L.LZ_BF16, *args, 0) == L.LZ_ERR_UNSUPPORTED
+    assert f(2, 2, -1, 128, 128, 16, L.LZ_BF16, *args, 0) == L.LZ_ERR_INVALID_ARG
+    bad = list(args)
+    bad[0] = None  # k missing with T > 0
+    assert f(2, 2, 10, 128, 128, 16, L.LZ_BF16, *bad, 0) == L.LZ_ERR_INVALID_ARG
+    bad = list(args)
+    bad[6] = FAKE + 8  # pos misaligned
+    assert f(2, 2, 10, 128, 128, 16, L.LZ_BF16, *bad, 0) == L.LZ_ERR_INVALID_ARG

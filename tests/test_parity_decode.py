@@ -105,3 +105,40 @@ def test_decode_state_save_restore_bitwise():
         assert torch.equal(x, y)
     for x, y in zip(a, saved):
         assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("T,w", [(0, 8), (5, 16), (150, 64), (300, 128)])
+def test_prefill_hand_off_then_decode(dtype, T, w):
+    """A chunked prefill of T tokens, the hand-off (state = hT, ring = the last
+    w keys and values, pos = T), then n decode steps reproduce the oracle's
+    hybrid forward over all T + n tokens."""
+    Bd, H, M, n, alpha = 2, 2, 4, 6, 0.5
+    cpu, dev = small_problem(70 + T + w, Bd, H, T + n, 128, 128, M, dtype)
+    pre = {k: dev[k][:, :, :T].contiguous() for k in ("q", "k", "v", "g")}
+    if T:
+        fwd = L.hybrid_fwd(pre["q"], pre["k"], pre["v"], pre["g"], dev["meta_k"], dev["meta_v"],
+                           w=w, alpha=alpha, want_hT=True)
+        hT = fwd["hT"]
+    else:
+        hT = None
+    state, kring, vring, pos = L.decode_prefill(pre["k"], pre["v"], hT, w=w)
+    torch.cuda.synchronize()
+    assert torch.all(pos.cpu() == T)
+    if T:
+        assert torch.equal(state, hT)
+        for t in range(max(0, T - w), T):  # ring contents: copies, bit-exact
+            assert torch.equal(kring[:, :, t % w], pre["k"][:, :, t])
+            assert torch.equal(vring[:, :, t % w], pre["v"][:, :, t])
+    outs = []
+    for t in range(T, T + n):
+        sl = lambda name: dev[name][:, :, t].contiguous()
+        outs.append(L.decode_step(state, kring, vring, pos, sl("q"), sl("k"), sl("v"), sl("g"),
+                                  dev["meta_k"], dev["meta_v"], alpha=alpha).clone())
+    dec = torch.stack(outs, dim=2)
+    x = {k: np64(v) for k, v in cpu.items()}
+    ref = oracle.hybrid_fwd(x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], w,
+                            1 / math.sqrt(128), alpha)
+    assert_close("decode o after hand-off", dec, ref["o"][:, :, T:], dtype)
+    assert_close("decode state after hand-off", state, ref["hT"], dtype)
+    assert torch.all(pos.cpu() == T + n)
