@@ -215,7 +215,7 @@ def algorithmic_bytes(kernel: str, wl) -> float | None:
         return n * (4 * d * e + 4)
     if kernel.startswith("gla_bwd") or kernel.startswith("hybrid_bwd"):
         return n * (7 * d * e + 8 * d)
-    if kernel.startswith("gla_states"):  # state pass: reads k, v, g
+    if kernel.startswith("gla_states") or kernel.startswith("gla_delta"):  # state pass: reads k, v, g
         return n * (2 * d * e + 4 * d)
     if kernel.startswith("gla_out"):  # output pass: reads q, k, v, g, writes o
         return n * (4 * d * e + 4 * d)

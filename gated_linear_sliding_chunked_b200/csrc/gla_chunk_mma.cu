@@ -213,6 +213,176 @@ __global__ void __launch_bounds__(NT, 2) gla_states_kernel(GlaFwdParams p) {
 }
 
 // ===========================================================================
+// Pass 1, two-level variant for long sequences: every chunk's own state
+// increment in parallel, then an elementwise scan over the chunks
+// ===========================================================================
+//   dS_c = (k e^{b_l - b})^T v over the chunk,  E_c = e^{b_l} per key dim,
+//   S_{c+1} = diag(E_c) S_c + dS_c.
+// dS_c goes through memory in bf16 (the states the output pass reads are
+// bf16 as well); the scan keeps S in fp32.
+// Measured on B200 it beats the sequential pass at 32 chunks x 64 heads
+// (0.079 vs 0.096 ms), 128 x 64 (0.276 vs 0.363 ms) and 1024 x 32 (1.14 vs
+// 1.81 ms); a single chunk has nothing to scan.
+constexpr int kScanMinChunks = 2;
+
+struct DeltaSmem {
+  bf16 k[C * QKP];
+  bf16 v[C * VP];
+  float g[C * DK];
+  bf16 ks[C * QKP];
+  float dec[NSB][DK];
+};
+static_assert(sizeof(DeltaSmem) <= 115712, "two delta CTAs must fit one SM");
+
+__global__ void __launch_bounds__(NT, 2) gla_delta_kernel(GlaFwdParams p) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  DeltaSmem& sm = *reinterpret_cast<DeltaSmem*>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gr = lane >> 2, gc = (lane & 3) * 2;
+  const int c = blockIdx.x, bh = blockIdx.y;
+  const int T = p.T, nchunks = gridDim.x;
+  const int c0 = c * C, rows = min(C, T - c0);
+  const bf16* k = (const bf16*)p.k + ((size_t)bh * T + c0) * DK;
+  const bf16* v = (const bf16*)p.v + ((size_t)bh * T + c0) * DV;
+  const float* g = p.g + ((size_t)bh * T + c0) * DK;
+  for (int x = tid; x < C * DK / 8; x += NT) {
+    const int r = x / (DK / 8), cc = x % (DK / 8);
+    const bool ok = r < rows;
+    cp_async16(&sm.k[r * QKP + cc * 8], k + (size_t)(ok ? r : 0) * DK + cc * 8, ok ? 16 : 0);
+    cp_async16(&sm.v[r * VP + cc * 8], v + (size_t)(ok ? r : 0) * DV + cc * 8, ok ? 16 : 0);
+  }
+  for (int x = tid; x < C * DK / 4; x += NT) {
+    const int r = x / (DK / 4), cc = x % (DK / 4);
+    const bool ok = r < rows;
+    cp_async16(&sm.g[r * DK + cc * 4], g + (size_t)(ok ? r : 0) * DK + cc * 4, ok ? 16 : 0);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+  // prep: thread -> (sub-block K, key dims i2, i2+1); rows past the end have
+  // g = 0 (no decay) and k = 0
+  const int K = tid >> 6, i2 = (tid & 63) * 2, r0 = K * SB;
+  float2 kfac[SB];
+  {
+    float2 run = make_float2(1.f, 1.f);
+#pragma unroll
+    for (int r = SB - 1; r >= 0; --r) {
+      kfac[r] = run;
+      const float2 gg = *reinterpret_cast<const float2*>(&sm.g[(r0 + r) * DK + i2]);
+      run.x *= __expf(gg.x);
+      run.y *= __expf(gg.y);
+    }
+    *reinterpret_cast<float2*>(&sm.dec[K][i2]) = run;
+  }
+  __syncthreads();
+  {
+    float2 f = make_float2(1.f, 1.f), e = make_float2(1.f, 1.f);
+#pragma unroll
+    for (int J = 0; J < NSB; ++J) {
+      const float2 d = *reinterpret_cast<const float2*>(&sm.dec[J][i2]);
+      if (J > K) {
+        f.x *= d.x;
+        f.y *= d.y;
+      }
+      e.x *= d.x;
+      e.y *= d.y;
+    }
+    if (K == 0)
+      *reinterpret_cast<float2*>(&p.decay[((size_t)bh * nchunks + c) * DK + i2]) = e;
+#pragma unroll
+    for (int r = 0; r < SB; ++r) {
+      const float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.k[(r0 + r) * QKP + i2]));
+      *reinterpret_cast<uint32_t*>(&sm.ks[(r0 + r) * QKP + i2]) =
+          pack_bf16(kv.x * kfac[r].x * f.x, kv.y * kfac[r].y * f.y);
+    }
+  }
+  __syncthreads();
+  // dS rows 16w .. 16w+15, all 128 value columns
+  float acc[DV / 8][4];
+#pragma unroll
+  for (int nt = 0; nt < DV / 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < C / 16; ++kk) {
+    uint32_t a[4];
+    ldsm_x4_t(smem_u32(&sm.ks[(16 * kk + (lane & 7) + ((lane >> 4) << 3)) * QKP + 16 * warp +
+                              ((lane >> 3) & 1) * 8]),
+              a[0], a[1], a[2], a[3]);
+#pragma unroll
+    for (int ntp = 0; ntp < DV / 16; ++ntp) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(smem_u32(&sm.v[(16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8) * VP + ntp * 16 + (lane >> 4) * 8]),
+                b0, b1, b2, b3);
+      mma_bf16(acc[2 * ntp], a, b0, b1);
+      mma_bf16(acc[2 * ntp + 1], a, b2, b3);
+    }
+  }
+  bf16* dst = (bf16*)p.delta16 + ((size_t)bh * nchunks + c) * DK * DV;
+#pragma unroll
+  for (int nt = 0; nt < DV / 8; ++nt)
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int i = 16 * warp + gr + 8 * hh, j = nt * 8 + gc;
+      *reinterpret_cast<uint32_t*>(&dst[(size_t)i * DV + j]) = pack_bf16(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
+    }
+}
+
+// thread -> (batch-head, key dim i, 8 value columns); walks the chunks
+constexpr int SCAN_NT = 128;
+constexpr int SCAN_U = 4;  // chunks whose loads are in flight together
+
+__global__ void __launch_bounds__(SCAN_NT) gla_scan_kernel(GlaFwdParams p, int nchunks) {
+  const size_t id = (size_t)blockIdx.x * SCAN_NT + threadIdx.x;
+  const size_t per_bh = (size_t)DK * (DV / 8);
+  if (id >= (size_t)p.B * p.H * per_bh) return;
+  const size_t bh = id / per_bh;
+  const int i = (int)((id / (DV / 8)) % DK), j8 = (int)(id % (DV / 8)) * 8;
+  float s[8];
+  if (p.h0) {
+    const float4* hp = reinterpret_cast<const float4*>(p.h0 + (bh * DK + i) * DV + j8);
+    const float4 a = hp[0], b = hp[1];
+    s[0] = a.x; s[1] = a.y; s[2] = a.z; s[3] = a.w; s[4] = b.x; s[5] = b.y; s[6] = b.z; s[7] = b.w;
+  } else {
+#pragma unroll
+    for (int x = 0; x < 8; ++x) s[x] = 0.f;
+  }
+  const size_t stride = (size_t)DK * DV;  // one chunk's state
+  const bf16* dl = (const bf16*)p.delta16 + bh * nchunks * stride + (size_t)i * DV + j8;
+  bf16* out = (bf16*)p.states16 + bh * nchunks * stride + (size_t)i * DV + j8;
+  const float* ec = p.decay + bh * nchunks * DK + i;
+  for (int c0 = 0; c0 < nchunks; c0 += SCAN_U) {
+    uint4 d[SCAN_U];
+    float e[SCAN_U];
+#pragma unroll
+    for (int u = 0; u < SCAN_U; ++u) {
+      const int c = c0 + u;
+      d[u] = c < nchunks ? __ldcs(reinterpret_cast<const uint4*>(dl + c * stride)) : make_uint4(0, 0, 0, 0);
+      e[u] = c < nchunks ? __ldcs(ec + (size_t)c * DK) : 1.f;
+    }
+#pragma unroll
+    for (int u = 0; u < SCAN_U; ++u) {
+      const int c = c0 + u;
+      if (c >= nchunks) break;
+      *reinterpret_cast<uint4*>(out + c * stride) =
+          make_uint4(pack_bf16(s[0], s[1]), pack_bf16(s[2], s[3]), pack_bf16(s[4], s[5]), pack_bf16(s[6], s[7]));
+      const uint32_t dw[4] = {d[u].x, d[u].y, d[u].z, d[u].w};
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const float2 f = unpack_bf16(dw[x]);
+        s[2 * x] = fmaf(e[u], s[2 * x], f.x);
+        s[2 * x + 1] = fmaf(e[u], s[2 * x + 1], f.y);
+      }
+    }
+  }
+  if (p.hT) {
+    float4* hp = reinterpret_cast<float4*>(p.hT + (bh * DK + i) * DV + j8);
+    hp[0] = make_float4(s[0], s[1], s[2], s[3]);
+    hp[1] = make_float4(s[4], s[5], s[6], s[7]);
+  }
+}
+
+// ===========================================================================
 // Pass 2: chunk outputs, all chunks in parallel
 // ===========================================================================
 struct OutSmem {
@@ -476,8 +646,29 @@ __global__ void __launch_bounds__(NT, 2) gla_out_kernel(GlaFwdParams p) {
 
 bool gla_chunk_mma_supported(int dk, int dv, bool bf16) { return bf16 && dk == DK && dv == DV; }
 
+bool gla_states_scan_wanted(int T) { return (T + C - 1) / C >= kScanMinChunks; }
+
 cudaError_t launch_gla_states(const GlaFwdParams& p, cudaStream_t s) {
   if (p.B * p.H == 0) return cudaSuccess;
+  const int nchunks = (p.T + C - 1) / C;
+  if (p.delta16 && p.decay && nchunks >= kScanMinChunks) {
+    const size_t bytes = sizeof(DeltaSmem);
+    cudaError_t e = cudaFuncSetAttribute(gla_delta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)bytes);
+    if (e != cudaSuccess) return e;
+    {
+      ScopedTiming tm("gla_delta_mma", s);
+      gla_delta_kernel<<<dim3(nchunks, p.B * p.H), NT, bytes, s>>>(p);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t threads = (size_t)p.B * p.H * DK * (DV / 8);
+    {
+      ScopedTiming tm("gla_scan", s);
+      gla_scan_kernel<<<(unsigned)((threads + SCAN_NT - 1) / SCAN_NT), SCAN_NT, 0, s>>>(p, nchunks);
+    }
+    return cudaGetLastError();
+  }
   const size_t bytes = sizeof(StateSmem);
   cudaError_t e = cudaFuncSetAttribute(gla_states_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)bytes);

@@ -47,6 +47,8 @@ struct GlaFwdParams {
   const void* add16;   // nullable (tensor-core kernel): the same in bf16; may alias o
   float alpha;
   int B, H, T, dk, dv;
+  void* delta16;       // nullable scratch of the two-level state pass: [BH][nchunks][dk][dv] bf16
+  float* decay;        // and [BH][nchunks][dk] fp32
 };
 constexpr int kSimtChunk = 16;
 cudaError_t launch_gla_fwd_simt(const GlaFwdParams& p, bool bf16, cudaStream_t s);
@@ -87,6 +89,8 @@ cudaError_t launch_gla_bwd_simt(const GlaBwdParams& p, bool bf16, cudaStream_t s
 // alpha * add16 when set) from them, all chunks in parallel.
 bool gla_chunk_mma_supported(int dk, int dv, bool bf16);
 cudaError_t launch_gla_states(const GlaFwdParams& p, cudaStream_t s);
+// whether launch_gla_states takes the two-level path (given delta16 / decay)
+bool gla_states_scan_wanted(int T);
 cudaError_t launch_gla_out(const GlaFwdParams& p, cudaStream_t s);
 
 // ---- gated branch, tensor-core backward (bf16 I/O, dk = dv = 128) --------

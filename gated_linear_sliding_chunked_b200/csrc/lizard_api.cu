@@ -32,9 +32,18 @@ cudaError_t swa_backward(const lz::SwaBwdParams& p, bool bf16, cudaStream_t s) {
 // (bf16 states into `states16` scratch) then all chunks' outputs in
 // parallel; bf16 with dk = 128 and other dv: the single-pass tensor-core
 // kernel; otherwise fp32 SIMT.
-cudaError_t gla_forward(lz::GlaFwdParams p, bool bf16, void* states16, cudaStream_t s) {
+// Scratch of the two-level state pass (long sequences): per-chunk increments
+// and decays; both NULL when the sequential pass is used.
+struct ScanWs {
+  void* delta16 = nullptr;
+  float* decay = nullptr;
+};
+
+cudaError_t gla_forward(lz::GlaFwdParams p, bool bf16, void* states16, ScanWs scan, cudaStream_t s) {
   if (lz::gla_chunk_mma_supported(p.dk, p.dv, bf16)) {
     p.states16 = states16;
+    p.delta16 = scan.delta16;
+    p.decay = scan.decay;
     cudaError_t e = lz::launch_gla_states(p, s);
     if (e != cudaSuccess) return e;
     return lz::launch_gla_out(p, s);
@@ -146,6 +155,15 @@ size_t states16_count(const lz_dims* d) {
   const size_t n64 = (size_t)((d->T + lz::gla_fwd_mma_chunk() - 1) / lz::gla_fwd_mma_chunk());
   return (size_t)d->B * d->H * n64 * d->dk * d->dv;
 }
+// the two-level state pass's scratch, carved right after the states
+ScanWs carve_scan(Carver& c, const lz_dims* d) {
+  ScanWs w;
+  if (!lz::gla_states_scan_wanted(d->T)) return w;
+  const size_t n64 = (size_t)((d->T + lz::gla_fwd_mma_chunk() - 1) / lz::gla_fwd_mma_chunk());
+  w.delta16 = c.take<uint16_t>(states16_count(d));
+  w.decay = c.take<float>((size_t)d->B * d->H * n64 * d->dk);
+  return w;
+}
 size_t nchunks16(const lz_dims* d) {
   return (size_t)((d->T + lz::kSimtChunk - 1) / lz::kSimtChunk);
 }
@@ -170,12 +188,14 @@ struct GlaBwdWs {
   float* states;
   void* states16;
   float* hT;
+  ScanWs scan;
 };
 GlaBwdWs carve_gla_bwd(Carver& c, const lz_dims* d) {
   GlaBwdWs w{};
   const size_t bh = (size_t)d->B * d->H;
   if (bwd_uses_mma(d)) {
     w.states16 = c.take<uint16_t>(states16_count(d));  // bf16
+    w.scan = carve_scan(c, d);
   } else {
     w.states = c.take<float>(bh * nchunks16(d) * d->dk * d->dv);
   }
@@ -220,11 +240,17 @@ size_t ws_bytes(const lz_dims* d, int which) {
   Carver c(nullptr);
   switch (which) {
     case LZ_WS_GLA_FWD:
-      if (fwd_uses_chunks(d)) c.take<uint16_t>(states16_count(d));
+      if (fwd_uses_chunks(d)) {
+        c.take<uint16_t>(states16_count(d));
+        carve_scan(c, d);
+      }
       return c.off;
     case LZ_WS_HYBRID_FWD:
       if (!hybrid_uses_mma(d)) c.take<float>(bht(d) * d->dv);  // fp32 window output
-      if (fwd_uses_chunks(d)) c.take<uint16_t>(states16_count(d));
+      if (fwd_uses_chunks(d)) {
+        c.take<uint16_t>(states16_count(d));
+        carve_scan(c, d);
+      }
       return c.off;
     case LZ_WS_GLA_BWD:
       carve_gla_bwd(c, d);
@@ -333,8 +359,9 @@ lz_status lz_gla_fwd(const lz_dims* d, const void* q, const void* k, const void*
   p.hT = hT;
   Carver c(ws);
   void* states16 = fwd_uses_chunks(d) ? c.take<uint16_t>(states16_count(d)) : nullptr;
+  const ScanWs scan = fwd_uses_chunks(d) ? carve_scan(c, d) : ScanWs{};
   if (states16 && chunk_states && ws_bytes(d, LZ_WS_CHUNK_STATES) > 0) states16 = chunk_states;
-  return cuda_status(gla_forward(p, d->io == LZ_BF16, states16, as_stream(stream)), "lz_gla_fwd");
+  return cuda_status(gla_forward(p, d->io == LZ_BF16, states16, scan, as_stream(stream)), "lz_gla_fwd");
 }
 
 lz_status lz_swa_meta_fwd(const lz_dims* d, const void* q, const void* k, const void* v,
@@ -369,6 +396,7 @@ lz_status lz_hybrid_fwd(const lz_dims* d, const void* q, const void* k, const vo
   Carver c(ws);
   float* osw = mma ? nullptr : c.take<float>(bht(d) * d->dv);
   void* states16 = fwd_uses_chunks(d) ? c.take<uint16_t>(states16_count(d)) : nullptr;
+  const ScanWs scan = fwd_uses_chunks(d) ? carve_scan(c, d) : ScanWs{};
   if (states16 && chunk_states && ws_bytes(d, LZ_WS_CHUNK_STATES) > 0) states16 = chunk_states;
   lz::SwaFwdParams sp = swa_fwd_params(d, q, k, v, meta_k, meta_v);
   // tensor-core path: bf16 window output into o_swa if requested, else into o
@@ -383,7 +411,7 @@ lz_status lz_hybrid_fwd(const lz_dims* d, const void* q, const void* k, const vo
   gp.add = osw;
   gp.add16 = mma ? sp.o : nullptr;
   gp.alpha = d->alpha;
-  return cuda_status(gla_forward(gp, bf, states16, s), "lz_hybrid_fwd (gated branch)");
+  return cuda_status(gla_forward(gp, bf, states16, scan, s), "lz_hybrid_fwd (gated branch)");
 }
 
 static cudaError_t gla_bwd_launch(const lz_dims* d, const void* q, const void* k, const void* v,
@@ -405,6 +433,8 @@ static cudaError_t gla_bwd_launch(const lz_dims* d, const void* q, const void* k
     fp.states = w.states;
     fp.states16 = w.states16;
     fp.hT = w.hT;
+    fp.delta16 = w.scan.delta16;
+    fp.decay = w.scan.decay;
     cudaError_t e = mma ? lz::launch_gla_states(fp, s) : lz::launch_gla_fwd_simt(fp, bf, s);
     if (e != cudaSuccess) return e;
   }
