@@ -70,7 +70,8 @@ def _bind(lib):
     lib.oracle_hybrid_bwd.argtypes = [_i] * 7 + [_f, _f] + [_D] * 17 + [_i]
     lib.oracle_decode_step.argtypes = ([_i] * 6 + [_f, _f] + [_D] * 3 + [_I64] +
                                        [_D] * 7 + [_i])
-    for name in ("oracle_gla_fwd", "oracle_gla_chunked_fwd", "oracle_swa_meta_fwd",
+    lib.oracle_mse_loss.argtypes = [ctypes.c_int64] + [_D] * 4
+    for name in ("oracle_mse_loss", "oracle_gla_fwd", "oracle_gla_chunked_fwd", "oracle_swa_meta_fwd",
                  "oracle_hybrid_fwd", "oracle_gla_bwd", "oracle_swa_meta_bwd",
                  "oracle_hybrid_bwd", "oracle_decode_step"):
         getattr(lib, name).restype = ctypes.c_int
@@ -244,3 +245,17 @@ def decode_step(state, kring, vring, pos, q, k, v, g, meta_k, meta_v, scale, alp
                                   vring.ctypes.data_as(_D), pos.ctypes.data_as(_I64),
                                   pq, pk, pv, pg, pmk, pmv, po, nthreads), "decode_step")
     return {"o": o, "state": state, "kring": kring, "vring": vring, "pos": pos}
+
+
+def mse_loss(o, target, *, lib=None):
+    """Stage-1 distillation loss: mean over every element of (o - target)^2.
+
+    Returns (loss, dO) with dO = dloss/do = 2 (o - target) / o.size."""
+    lib = lib or load()
+    (o, po), (t, pt) = _in(o), _in(target)
+    if o.shape != t.shape:
+        raise ValueError("mse_loss: o and target differ in shape")
+    loss, pl = _out((1,))
+    dO, pd = _out(o.shape)
+    _check(lib.oracle_mse_loss(int(o.size), po, pt, pl, pd), "mse_loss")
+    return float(loss[0]), dO

@@ -639,4 +639,24 @@ int oracle_decode_step(int Bd, int H, int dk, int dv, int w, int M,
   return 0;
 }
 
+// Stage-1 distillation loss (section 2b, "training strategy": the first
+// stage trains the hybrid attention to reproduce the teacher's attention
+// output under a mean-squared-error loss).  Reading: the mean runs over every
+// element of the output tensor (n = B*H*T*dv elements):
+//   loss = (1/n) sum_x (o_x - target_x)^2,   dO_x = dloss/do_x = 2 (o_x - target_x) / n.
+// dO may be NULL.  n == 0 gives loss 0.
+int oracle_mse_loss(int64_t n, const double* o, const double* target, double* loss,
+                    double* dO) {
+  if (n < 0 || !loss) return -1;
+  if (n > 0 && (!o || !target)) return -1;
+  double s = 0.0;
+  for (int64_t x = 0; x < n; ++x) {
+    const double diff = o[x] - target[x];
+    s += diff * diff;
+    if (dO) dO[x] = 2.0 * diff / (double)n;
+  }
+  *loss = n > 0 ? s / (double)n : 0.0;
+  return 0;
+}
+
 }  // extern "C"

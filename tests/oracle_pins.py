@@ -339,9 +339,85 @@ def pin_decode_matches_prefill(lib):
         assert np.array_equal(st["kring"][:, :, tok % w], k[:, :, tok])
 
 
+# ----------------------------------------------------------------------------
+# stage-1 distillation loss (section 2b): MSE to the teacher's attention output
+# ----------------------------------------------------------------------------
+def pin_mse_closed_form(lib):
+    """A constant offset c between output and target gives loss c^2 and the
+    gradient -2c/n everywhere; a target equal to the output gives zero."""
+    r = RNG(21)
+    o = r.standard_normal((2, 3, 5, 4))
+    n = o.size
+    for c in (0.0, 0.37, -1.5):
+        loss, dO = oracle.mse_loss(o, o + c, lib=lib)
+        assert abs(loss - c * c) <= 1e-12 * max(1.0, c * c), (c, loss)
+        assert np.allclose(dO, -2.0 * c / n, rtol=0, atol=1e-15), c
+    # a single differing element: loss = e^2 / n
+    t = o.copy()
+    t[1, 2, 3, 0] += 3.0
+    loss, dO = oracle.mse_loss(o, t, lib=lib)
+    assert abs(loss - 9.0 / n) < 1e-12
+    assert abs(dO[1, 2, 3, 0] + 6.0 / n) < 1e-15 and np.count_nonzero(dO) == 1
+    assert oracle.mse_loss(np.zeros((0, 4)), np.zeros((0, 4)), lib=lib)[0] == 0.0
+
+
+def pin_mse_grad_fd(lib):
+    """dO equals central differences of the loss with respect to o."""
+    r = RNG(22)
+    o = r.standard_normal((1, 2, 6, 3))
+    t = r.standard_normal(o.shape)
+    _, dO = oracle.mse_loss(o, t, lib=lib)
+    eps = 1e-6
+    num = np.zeros(o.size)
+    for idx in range(o.size):
+        op = o.reshape(-1).copy()
+        om = op.copy()
+        op[idx] += eps
+        om[idx] -= eps
+        num[idx] = (oracle.mse_loss(op.reshape(o.shape), t, lib=lib)[0] -
+                    oracle.mse_loss(om.reshape(o.shape), t, lib=lib)[0]) / (2 * eps)
+    assert _rel(dO.reshape(-1), num) < 1e-7, _rel(dO.reshape(-1), num)
+
+
+def _stage1_loss(lib, x, target, w, scale):
+    res = oracle.hybrid_fwd(x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], w,
+                            scale, float(x["alpha"]), x["h0"], lib=lib)
+    return oracle.mse_loss(res["o"], target, lib=lib)
+
+
+def pin_stage1_chain_fd(lib):
+    """The stage-1 step (hybrid forward, MSE to a teacher output, hybrid
+    backward fed with the loss gradient) gives the central differences of the
+    loss with respect to every operator input."""
+    x, _, _ = _tiny_case(23)
+    target = RNG(24).standard_normal(np.shape(x["v"]))
+    w, scale, eps = 4, 0.5, 1e-6
+    _, dO = _stage1_loss(lib, x, target, w, scale)
+    an = oracle.hybrid_bwd(x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], dO, w,
+                           scale, float(x["alpha"]), x["h0"], None, lib=lib)
+    names = {"q": "dq", "k": "dk", "v": "dv", "g": "dg", "meta_k": "dmeta_k",
+             "alpha": "dalpha"}
+    for key, gname in names.items():
+        base = np.array(x[key], dtype=np.float64)
+        num = np.zeros(base.size)
+        for idx in range(base.size):
+            bp = base.reshape(-1).copy()
+            bm = bp.copy()
+            bp[idx] += eps
+            bm[idx] -= eps
+            xp, xm = dict(x), dict(x)
+            xp[key] = bp.reshape(base.shape)
+            xm[key] = bm.reshape(base.shape)
+            num[idx] = (_stage1_loss(lib, xp, target, w, scale)[0] -
+                        _stage1_loss(lib, xm, target, w, scale)[0]) / (2 * eps)
+        got = np.asarray(an[gname], dtype=np.float64).reshape(-1)
+        assert _rel(got, num) < 1e-6, (key, _rel(got, num))
+
+
 ALL_PINS = [
     pin_gla_closed_form, pin_gla_unit_gates, pin_gla_full_forgetting,
     pin_gla_initial_state, pin_gla_chunked_identity, pin_swa_full_causal,
     pin_swa_band_meta, pin_swa_sinks, pin_hybrid_affine, pin_hybrid_grad_fd,
     pin_swa_grad_fd, pin_gla_dg_identity, pin_decode_matches_prefill,
+    pin_mse_closed_form, pin_mse_grad_fd, pin_stage1_chain_fd,
 ]

@@ -36,6 +36,9 @@ MUTANTS = [
     ("decode_wrong_slot", "int slot = (int)(p % w);", "int slot = (int)((p + 1) % w);"),
     ("decode_window_short", "int nwin = (int)std::min<int64_t>(p + 1, w);",
      "int nwin = (int)std::min<int64_t>(p, w);"),
+    ("mse_gradient_drops_two", "if (dO) dO[x] = 2.0 * diff / (double)n;", "if (dO) dO[x] = diff / (double)n;"),
+    ("mse_sum_not_mean", "*loss = n > 0 ? s / (double)n : 0.0;", "*loss = n > 0 ? s : 0.0;"),
+    ("mse_gradient_sign", "const double diff = o[x] - target[x];", "const double diff = target[x] - o[x];"),
 ]
 
 
