@@ -289,6 +289,32 @@ class TrainStep:
         return [self.o, self.dq, self.dk, self.dv, self.dg, self.dmk, self.dmv, self.dalpha]
 
 
+class Stage1Step(TrainStep):
+    """The first training stage's step: hybrid forward with the MSE loss to a
+    teacher output fused into its epilogue, then the backward fed with the
+    loss gradient."""
+
+    def __init__(self, wl, x, target, device):
+        super().__init__(wl, x, device)
+        L = self.L
+        self.target = target
+        self.dO = torch.empty_like(self.o)
+        self.loss = torch.empty((), dtype=torch.float32, device=device)
+        n = L.lz_workspace_bytes(self.dims, L.LZ_WS_HYBRID_FWD_MSE)
+        self.wsm, self.nm = torch.empty(max(n, 1), dtype=torch.uint8, device=device), n
+
+    def run(self, x=None):
+        x = x or self.x
+        L, d = self.L, self.dims
+        L.lz_hybrid_fwd_mse(d, x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], None,
+                            self.target, self.o, None, self.lse, self.osw, self.cs, self.loss,
+                            self.dO, self.wsm, self.nm)
+        L.lz_hybrid_bwd(d, x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], None,
+                        self.lse, self.osw, self.cs, None, self.dO, None, self.dq, self.dk,
+                        self.dv, self.dg, None, self.dmk, self.dmv, self.dalpha, self.wsb,
+                        self.nb)
+
+
 def time_region(fn, steps, device):
     """Device time of ``steps`` calls of fn (barrier + synchronize on both
     sides, CUDA events on the current stream); returns ms per step."""
@@ -389,6 +415,27 @@ def measure_fwd(wl, device, steps, warmup, peaks, seed, tcgen05_window=True):
             "l2": "256 MB flush between iterations (not counted in ms_per_call)",
             "kernels": {k: [c // steps, round(t / c, 4)] for k, (c, t) in tab.items()},
             "roofline": roof}
+
+
+def measure_stage1(wl, x, device, steps, warmup, seed):
+    """Stage-1 distillation step (forward + fused MSE loss + backward) on the
+    training workload, with a synthetic teacher output."""
+    import gated_linear_sliding_chunked_b200 as L
+    from gated_linear_sliding_chunked_b200 import inputs as I
+    target = I.make_teacher_output(wl, seed=1000 + seed, device=device)
+    st = Stage1Step(wl, x, target, device)
+    for _ in range(warmup):
+        st.run()
+    torch.cuda.synchronize(device)
+    L.lz_timing_enable(True)
+    ms = time_region(st.run, steps, device)
+    L.lz_timing_enable(False)
+    tab = kernel_table(L.lz_timing_read())
+    L.lz_device_check()
+    return {"workload": wl.name + " + MSE to a synthetic teacher output (N(0, 0.25))",
+            "tokens_per_s": wl.B * wl.T / (ms * 1e-3), "ms_per_step": round(ms, 4),
+            "loss": float(st.loss.cpu()),
+            "kernels": {k: [c // steps, round(t / c, 4)] for k, (c, t) in tab.items()}}
 
 
 def measure_decode(device, steps, warmup, peaks, seed, n_steps=1000):
@@ -656,6 +703,7 @@ def main(argv=None):
         extras["decode"] = measure_decode(device, 1, 1, peaks, seed=rank)
         extras["train_step_breakdown"] = {k: [c // args.steps, round(t / c, 4)]
                                           for k, (c, t) in tab.items()}
+        extras["stage1_step"] = measure_stage1(wl, xd, device, 10, 3, seed=rank)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -27,12 +27,12 @@ LIB_PATH = os.path.join(_PKG, "liblizard.so")
 LZ_OK, LZ_ERR_INVALID_ARG, LZ_ERR_UNSUPPORTED, LZ_ERR_CUDA, LZ_ERR_TIMEOUT = range(5)
 LZ_F32, LZ_BF16 = 0, 1
 (LZ_WS_GLA_FWD, LZ_WS_HYBRID_FWD, LZ_WS_GLA_BWD, LZ_WS_SWA_BWD, LZ_WS_HYBRID_BWD,
- LZ_WS_CHUNK_STATES) = range(6)
+ LZ_WS_CHUNK_STATES, LZ_WS_HYBRID_FWD_MSE) = range(7)
 
 EXPORTS = ("lz_gla_fwd", "lz_gla_bwd", "lz_swa_meta_fwd", "lz_hybrid_fwd", "lz_swa_meta_bwd",
            "lz_hybrid_bwd", "lz_gla_decode_step", "lz_workspace_bytes", "lz_last_error",
            "lz_version", "lz_timing_enable", "lz_timing_read", "lz_swa_meta_bwd_noalloc",
-           "lz_device_check", "lz_prefer_tcgen05", "lz_decode_prefill")
+           "lz_device_check", "lz_prefer_tcgen05", "lz_decode_prefill", "lz_hybrid_fwd_mse")
 
 # size of the static scratch array behind lz_swa_meta_bwd_noalloc
 LZ_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -71,6 +71,7 @@ def load(path: str = LIB_PATH):
     lib.lz_gla_fwd.argtypes = [D] + [_P] * 8 + [_P, sz, _P]
     lib.lz_swa_meta_fwd.argtypes = [D] + [_P] * 7 + [_P]
     lib.lz_hybrid_fwd.argtypes = [D] + [_P] * 12 + [_P, sz, _P]
+    lib.lz_hybrid_fwd_mse.argtypes = [D] + [_P] * 15 + [_P, sz, _P]
     lib.lz_gla_bwd.argtypes = [D] + [_P] * 14 + [_P, sz, _P]
     lib.lz_swa_meta_bwd.argtypes = [D] + [_P] * 13 + [_P, sz, _P]
     lib.lz_hybrid_bwd.argtypes = [D] + [_P] * 21 + [_P, sz, _P]
@@ -176,6 +177,14 @@ def lz_gla_fwd(dims, q, k, v, g, h0, o, hT, chunk_states, ws, ws_bytes, stream=N
 def lz_swa_meta_fwd(dims, q, k, v, meta_k, meta_v, o, lse, stream=None):
     _check(load().lz_swa_meta_fwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(meta_k),
                                   _ptr(meta_v), _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def lz_hybrid_fwd_mse(dims, q, k, v, g, meta_k, meta_v, h0, target, o, hT, lse, o_swa,
+                      chunk_states, loss, dO, ws, ws_bytes, stream=None):
+    _check(load().lz_hybrid_fwd_mse(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                    _ptr(meta_k), _ptr(meta_v), _ptr(h0), _ptr(target), _ptr(o),
+                                    _ptr(hT), _ptr(lse), _ptr(o_swa), _ptr(chunk_states),
+                                    _ptr(loss), _ptr(dO), _ptr(ws), ws_bytes, _stream(stream)))
 
 
 def lz_hybrid_fwd(dims, q, k, v, g, meta_k, meta_v, h0, o, hT, lse, o_swa, chunk_states, ws,
@@ -293,6 +302,28 @@ def hybrid_fwd(q, k, v, g, meta_k, meta_v, *, w, alpha, scale=None, chunk=64, h0
     ws, n = _ws(d, LZ_WS_HYBRID_FWD, dev)
     lz_hybrid_fwd(d, q, k, v, g, meta_k, meta_v, h0, o, hT, lse, osw, cs, ws, n, stream)
     return {"o": o, "hT": hT, "lse": lse, "o_swa": osw, "chunk_states": cs}
+
+
+def hybrid_fwd_mse(q, k, v, g, meta_k, meta_v, target, *, w, alpha, scale=None, chunk=64,
+                   h0=None, want_dO=True, want_hT=False, want_lse=False, want_o_swa=False,
+                   want_chunk_states=False, stream=None):
+    """hybrid_fwd plus the stage-1 loss mean((o - target)^2); the result adds
+    "loss" (0-dim fp32 tensor on the device) and "dO" (its gradient, or None)."""
+    d = _dims_from(q, v, chunk=chunk, w=w, M=_M(meta_k), scale=scale, alpha=alpha)
+    dev = q.device
+    o = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=dev)
+    hT = torch.empty(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], dtype=torch.float32,
+                     device=dev) if want_hT else None
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=dev) if want_lse else None
+    osw = torch.empty_like(o) if want_o_swa else None
+    cs = _chunk_states(d, dev) if want_chunk_states else None
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    dO = torch.empty_like(o) if want_dO else None
+    ws, n = _ws(d, LZ_WS_HYBRID_FWD_MSE, dev)
+    lz_hybrid_fwd_mse(d, q, k, v, g, meta_k, meta_v, h0, target, o, hT, lse, osw, cs, loss, dO,
+                      ws, n, stream)
+    return {"o": o, "hT": hT, "lse": lse, "o_swa": osw, "chunk_states": cs, "loss": loss,
+            "dO": dO}
 
 
 def gla_bwd(q, k, v, g, dO, h0=None, dhT=None, *, chunk=64, chunk_states=None, hT=None,

@@ -393,6 +393,7 @@ struct OutSmem {
   bf16 sp[DK * VP];    // state before the chunk
   float dec[NSB][DK];
   float fac[NPAIR][DK];
+  float lsum[NT / 32];  // per-warp sums of the fused loss
 };
 static_assert(sizeof(OutSmem) <= 115712, "two output CTAs must fit one SM");
 
@@ -409,6 +410,9 @@ __device__ __noinline__ float diag_score_global(const bf16* q, const bf16* k, co
   return a;
 }
 
+// LOSS: the stage-1 loss epilogue (p.target set), a separate instantiation so
+// that the plain forward keeps its registers and schedule.
+template <bool LOSS>
 __global__ void __launch_bounds__(NT, 2) gla_out_kernel(GlaFwdParams p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   OutSmem& sm = *reinterpret_cast<OutSmem*>(smem_raw);
@@ -626,6 +630,27 @@ __global__ void __launch_bounds__(NT, 2) gla_out_kernel(GlaFwdParams p) {
     }
   }
   // epilogue: o = o_gla + alpha * add
+  if (p.add16) {
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        o[nt][2 * hh] += p.alpha * addv[nt][hh].x;
+        o[nt][2 * hh + 1] += p.alpha * addv[nt][hh].y;
+      }
+  }
+  float lsq = 0.f;
+  uint32_t tg[8][2];
+  if constexpr (LOSS) {  // all target loads in flight before the first store
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int t = 16 * I + gr + 8 * hh;
+        const size_t off = ((size_t)bh * T + c0 + t) * DV + 64 * nh + nt * 8 + gc;
+        tg[nt][hh] = t < rows ? __ldg(reinterpret_cast<const unsigned int*>(&((const bf16*)p.target)[off])) : 0u;
+      }
+  }
 #pragma unroll
   for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
@@ -633,13 +658,28 @@ __global__ void __launch_bounds__(NT, 2) gla_out_kernel(GlaFwdParams p) {
       const int t = 16 * I + gr + 8 * hh;
       if (t >= rows) continue;
       const size_t off = ((size_t)bh * T + c0 + t) * DV + 64 * nh + nt * 8 + gc;
-      float x0 = o[nt][2 * hh], x1 = o[nt][2 * hh + 1];
-      if (p.add16) {
-        x0 += p.alpha * addv[nt][hh].x;
-        x1 += p.alpha * addv[nt][hh].y;
+      const float x0 = o[nt][2 * hh], x1 = o[nt][2 * hh + 1];
+      if constexpr (LOSS) {  // stage-1 loss on the fp32 output, before its rounding
+        const float2 tv = unpack_bf16(tg[nt][hh]);
+        const float e0 = x0 - tv.x, e1 = x1 - tv.y;
+        lsq = fmaf(e0, e0, fmaf(e1, e1, lsq));
+        if (p.dO_loss)
+          *reinterpret_cast<uint32_t*>(&((bf16*)p.dO_loss)[off]) = pack_bf16(p.loss_scale * e0, p.loss_scale * e1);
       }
       *reinterpret_cast<uint32_t*>(&((bf16*)p.o)[off]) = pack_bf16(x0, x1);
     }
+  if constexpr (LOSS) {  // fixed-order reduction: lanes, then warps
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) lsq += __shfl_xor_sync(0xffffffffu, lsq, m);
+    if (lane == 0) sm.lsum[warp] = lsq;
+    __syncthreads();
+    if (tid == 0) {
+      float tot = 0.f;
+#pragma unroll
+      for (int w = 0; w < NT / 32; ++w) tot += sm.lsum[w];
+      p.loss_part[(size_t)bh * nchunks + c] = tot;
+    }
+  }
 }
 
 }  // namespace
@@ -680,16 +720,18 @@ cudaError_t launch_gla_states(const GlaFwdParams& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+size_t gla_out_loss_parts(int B, int H, int T) { return (size_t)B * H * ((T + C - 1) / C); }
+
 cudaError_t launch_gla_out(const GlaFwdParams& p, cudaStream_t s) {
   const int nchunks = (p.T + C - 1) / C;
   if (p.B * p.H == 0 || nchunks == 0) return cudaSuccess;
   const size_t bytes = sizeof(OutSmem);
-  cudaError_t e =
-      cudaFuncSetAttribute(gla_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  const auto kern = p.target ? gla_out_kernel<true> : gla_out_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
   {
-    ScopedTiming tm("gla_out_mma", s);
-    gla_out_kernel<<<dim3(nchunks, p.B * p.H), NT, bytes, s>>>(p);
+    ScopedTiming tm(p.target ? "gla_out_mma_loss" : "gla_out_mma", s);
+    kern<<<dim3(nchunks, p.B * p.H), NT, bytes, s>>>(p);
   }
   return cudaGetLastError();
 }

@@ -49,6 +49,14 @@ struct GlaFwdParams {
   int B, H, T, dk, dv;
   void* delta16;       // nullable scratch of the two-level state pass: [BH][nchunks][dk][dv] bf16
   float* decay;        // and [BH][nchunks][dk] fp32
+  // stage-1 distillation loss, fused into the output pass's epilogue (bf16
+  // path): target [B,H,T,dv] (nullable = no loss); loss_part[bh * nchunks + c]
+  // receives each chunk's sum of (o - target)^2 taken on the fp32 output;
+  // dO_loss (nullable) receives loss_scale * (o - target)
+  const void* target;
+  void* dO_loss;
+  float loss_scale;
+  float* loss_part;
 };
 constexpr int kSimtChunk = 16;
 cudaError_t launch_gla_fwd_simt(const GlaFwdParams& p, bool bf16, cudaStream_t s);
@@ -92,6 +100,20 @@ cudaError_t launch_gla_states(const GlaFwdParams& p, cudaStream_t s);
 // whether launch_gla_states takes the two-level path (given delta16 / decay)
 bool gla_states_scan_wanted(int T);
 cudaError_t launch_gla_out(const GlaFwdParams& p, cudaStream_t s);
+// partial sums the fused loss epilogue writes: one per 64-token chunk and head
+size_t gla_out_loss_parts(int B, int H, int T);
+
+// ---- stage-1 distillation loss (loss.cu) ------------------------------------
+// Any layout: n elements of o and target (bf16 or fp32); part[0, nparts)
+// receives block partial sums of (o - target)^2 in a fixed order; dO
+// (nullable) receives scale * (o - target).
+constexpr int kMseParts = 592;  // 4 blocks per SM on 148 SMs
+cudaError_t launch_mse_generic(const void* o, const void* target, void* dO, float scale, size_t n,
+                               bool bf16, float* part, cudaStream_t s);
+int mse_generic_parts(size_t n);
+// loss[0] = inv_n * (sum of part[0, nparts)), summed in fp64 in a fixed order
+cudaError_t launch_loss_reduce(const float* part, size_t nparts, double inv_n, float* loss,
+                               cudaStream_t s);
 
 // ---- gated branch, tensor-core backward (bf16 I/O, dk = dv = 128) --------
 // Needs states16 and hT from the tensor-core forward run as a state pass.

@@ -181,6 +181,15 @@ bool hybrid_uses_mma(const lz_dims* d) {
          lz::swa_bwd_mma_supported(d->dk, d->dv, bf) && lz::gla_bwd_mma_supported(d->dk, d->dv, bf);
 }
 
+// Stage-1 loss: fused into the gated output kernel's epilogue on the
+// tensor-core path; partial sums per (chunk, head) there, per block of the
+// generic loss kernel otherwise.
+bool loss_fused(const lz_dims* d) { return hybrid_uses_mma(d) && fwd_uses_chunks(d); }
+size_t loss_parts(const lz_dims* d) {
+  if (loss_fused(d)) return lz::gla_out_loss_parts(d->B, d->H, d->T);
+  return (size_t)lz::mse_generic_parts(bht(d) * d->dv);
+}
+
 // Gated backward scratch: the states before every chunk (fp32 per 16-token
 // chunk for the SIMT kernel, bf16 per 64-token chunk for the tensor-core
 // kernel) and the final state.
@@ -251,6 +260,10 @@ size_t ws_bytes(const lz_dims* d, int which) {
         c.take<uint16_t>(states16_count(d));
         carve_scan(c, d);
       }
+      return c.off;
+    case LZ_WS_HYBRID_FWD_MSE:
+      c.off = ws_bytes(d, LZ_WS_HYBRID_FWD);
+      c.take<float>(loss_parts(d));
       return c.off;
     case LZ_WS_GLA_BWD:
       carve_gla_bwd(c, d);
@@ -378,17 +391,34 @@ lz_status lz_swa_meta_fwd(const lz_dims* d, const void* q, const void* k, const 
   return cuda_status(swa_forward(p, d->io == LZ_BF16, as_stream(stream)), "lz_swa_meta_fwd");
 }
 
-lz_status lz_hybrid_fwd(const lz_dims* d, const void* q, const void* k, const void* v,
-                        const float* g, const void* meta_k, const void* meta_v,
-                        const float* h0, void* o, float* hT, float* lse, void* o_swa,
-                        void* chunk_states, void* ws, size_t ws_bytes_, lz_stream stream) {
+// The stage-1 loss of lz_hybrid_fwd_mse (NULL for the plain forward).
+struct LossArgs {
+  const void* target;
+  float* loss;
+  void* dO;
+};
+
+static lz_status hybrid_fwd_impl(const char* name, const lz_dims* d, const void* q, const void* k,
+                                 const void* v, const float* g, const void* meta_k,
+                                 const void* meta_v, const float* h0, void* o, float* hT,
+                                 float* lse, void* o_swa, void* chunk_states, const LossArgs* la,
+                                 void* ws, size_t ws_bytes_, lz_stream stream) {
   lz_status st = check_dims(d, true);
   if (st != LZ_OK) return st;
   const bool nz = bht(d) > 0;  // empty tensors may have NULL data
   LZ_PTR(q, nz); LZ_PTR(k, nz); LZ_PTR(v, nz); LZ_PTR(g, nz); LZ_PTR(o, nz);
   LZ_PTR(meta_k, d->M > 0 && d->H > 0); LZ_PTR(meta_v, false); LZ_PTR(h0, false); LZ_PTR(hT, false);
   LZ_PTR(lse, false); LZ_PTR(o_swa, false); LZ_PTR(chunk_states, false);
-  st = check_ws(d, LZ_WS_HYBRID_FWD, ws, ws_bytes_);
+  if (la) {
+    const void* target = la->target;
+    const float* loss = la->loss;
+    LZ_PTR(target, nz); LZ_PTR(loss, true);
+    const size_t ob = bht(d) * d->dv * (d->io == LZ_BF16 ? 2 : 4);
+    const char* oc = (const char*)o;
+    const char* dc = (const char*)la->dO;
+    LZ_REQUIRE(!dc || !nz || dc + ob <= oc || oc + ob <= dc, "dO must not overlap o");
+  }
+  st = check_ws(d, la ? LZ_WS_HYBRID_FWD_MSE : LZ_WS_HYBRID_FWD, ws, ws_bytes_);
   if (st != LZ_OK) return st;
   const cudaStream_t s = as_stream(stream);
   const bool bf = d->io == LZ_BF16;
@@ -397,6 +427,7 @@ lz_status lz_hybrid_fwd(const lz_dims* d, const void* q, const void* k, const vo
   float* osw = mma ? nullptr : c.take<float>(bht(d) * d->dv);
   void* states16 = fwd_uses_chunks(d) ? c.take<uint16_t>(states16_count(d)) : nullptr;
   const ScanWs scan = fwd_uses_chunks(d) ? carve_scan(c, d) : ScanWs{};
+  float* parts = la ? c.take<float>(loss_parts(d)) : nullptr;
   if (states16 && chunk_states && ws_bytes(d, LZ_WS_CHUNK_STATES) > 0) states16 = chunk_states;
   lz::SwaFwdParams sp = swa_fwd_params(d, q, k, v, meta_k, meta_v);
   // tensor-core path: bf16 window output into o_swa if requested, else into o
@@ -411,7 +442,43 @@ lz_status lz_hybrid_fwd(const lz_dims* d, const void* q, const void* k, const vo
   gp.add = osw;
   gp.add16 = mma ? sp.o : nullptr;
   gp.alpha = d->alpha;
-  return cuda_status(gla_forward(gp, bf, states16, scan, s), "lz_hybrid_fwd (gated branch)");
+  const size_t n = bht(d) * d->dv;
+  const float lscale = n > 0 ? (float)(2.0 / (double)n) : 0.f;
+  const bool fused = la && loss_fused(d);
+  if (fused) {
+    gp.target = la->target;
+    gp.dO_loss = la->dO;
+    gp.loss_scale = lscale;
+    gp.loss_part = parts;
+  }
+  e = gla_forward(gp, bf, states16, scan, s);
+  if (e != cudaSuccess || !la) return cuda_status(e, name);
+  size_t nparts = loss_parts(d);
+  if (!fused) {
+    e = lz::launch_mse_generic(o, la->target, la->dO, lscale, n, bf, parts, s);
+    if (e != cudaSuccess) return cuda_status(e, name);
+    nparts = (size_t)lz::mse_generic_parts(n);
+  }
+  return cuda_status(lz::launch_loss_reduce(parts, nparts, n > 0 ? 1.0 / (double)n : 0.0, la->loss, s),
+                     name);
+}
+
+lz_status lz_hybrid_fwd(const lz_dims* d, const void* q, const void* k, const void* v,
+                        const float* g, const void* meta_k, const void* meta_v,
+                        const float* h0, void* o, float* hT, float* lse, void* o_swa,
+                        void* chunk_states, void* ws, size_t ws_bytes_, lz_stream stream) {
+  return hybrid_fwd_impl("lz_hybrid_fwd", d, q, k, v, g, meta_k, meta_v, h0, o, hT, lse, o_swa,
+                         chunk_states, nullptr, ws, ws_bytes_, stream);
+}
+
+lz_status lz_hybrid_fwd_mse(const lz_dims* d, const void* q, const void* k, const void* v,
+                            const float* g, const void* meta_k, const void* meta_v,
+                            const float* h0, const void* target, void* o, float* hT, float* lse,
+                            void* o_swa, void* chunk_states, float* loss, void* dO, void* ws,
+                            size_t ws_bytes_, lz_stream stream) {
+  const LossArgs la{target, loss, dO};
+  return hybrid_fwd_impl("lz_hybrid_fwd_mse", d, q, k, v, g, meta_k, meta_v, h0, o, hT, lse, o_swa,
+                         chunk_states, &la, ws, ws_bytes_, stream);
 }
 
 static cudaError_t gla_bwd_launch(const lz_dims* d, const void* q, const void* k, const void* v,

@@ -128,6 +128,14 @@ def make_inputs(wl: Workload, seed: int = 0, device="cpu") -> dict:
     return out
 
 
+def make_teacher_output(wl: Workload, seed: int = 0, device="cpu", std: float = 0.5):
+    """Synthetic stand-in for a teacher's attention output [B, H, T, dv] (the
+    target of the first training stage; no teacher weights are available)."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    return (_randn(gen, (wl.B, wl.H, wl.T, wl.dv), device) * std).to(wl.torch_dtype)
+
+
 def make_decode_state(wl: DecodeWorkload, seed: int = 0, device="cpu") -> dict:
     """Initial decode state: fp32 state, bf16 K/V rings, positions, meta."""
     gen = torch.Generator(device=device)

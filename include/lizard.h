@@ -85,7 +85,8 @@ typedef struct {
  * where the kernels keep no such states (fp32 I/O, d = 64); the pointers
  * are then ignored. */
 enum { LZ_WS_GLA_FWD = 0, LZ_WS_HYBRID_FWD = 1, LZ_WS_GLA_BWD = 2,
-       LZ_WS_SWA_BWD = 3, LZ_WS_HYBRID_BWD = 4, LZ_WS_CHUNK_STATES = 5 };
+       LZ_WS_SWA_BWD = 3, LZ_WS_HYBRID_BWD = 4, LZ_WS_CHUNK_STATES = 5,
+       LZ_WS_HYBRID_FWD_MSE = 6 };
 size_t lz_workspace_bytes(const lz_dims* d, int which);
 
 /* Gated linear attention forward (section 2a, state update equation).
@@ -118,6 +119,27 @@ lz_status lz_hybrid_fwd(const lz_dims* d, const void* q, const void* k,
                         const void* meta_v, const float* h0, void* o,
                         float* hT, float* lse, void* o_swa, void* chunk_states,
                         void* ws, size_t ws_bytes, lz_stream stream);
+
+/* lz_hybrid_fwd followed by the first training stage's loss (section 2b,
+ * training strategy: the hybrid attention learns to reproduce the teacher's
+ * attention output under a mean-squared-error loss).
+ *   target: the teacher's output, [B, H, T, dv], io dtype.
+ *   loss:   device float[1], receives (1/n) sum (o - target)^2 over all
+ *           n = B*H*T*dv elements (0 when n == 0).
+ *   dO:     nullable, [B, H, T, dv], io dtype: receives dloss/do =
+ *           2 (o - target) / n, the dO that lz_hybrid_bwd takes.
+ * With bf16 I/O and dk = dv = 128 the loss and dO are formed in the output
+ * kernel's epilogue from the fp32 output before it is rounded to bf16;
+ * otherwise a separate kernel reads the stored output.  The partial sums are
+ * added in a fixed order, so the loss is the same bit for bit on every run.
+ * dO must not overlap o.  Scratch: lz_workspace_bytes(d, LZ_WS_HYBRID_FWD_MSE).
+ * All other arguments as in lz_hybrid_fwd. */
+lz_status lz_hybrid_fwd_mse(const lz_dims* d, const void* q, const void* k,
+                            const void* v, const float* g, const void* meta_k,
+                            const void* meta_v, const float* h0,
+                            const void* target, void* o, float* hT, float* lse,
+                            void* o_swa, void* chunk_states, float* loss, void* dO,
+                            void* ws, size_t ws_bytes, lz_stream stream);
 
 /* Gradient of lz_gla_fwd (needed by the attention-distillation stage,
  * section 2b).  dO = dL/do; dhT (nullable) = dL/dhT.  Writes dq, dk, dv (io

@@ -175,3 +175,36 @@ def test_decode_prefill_validation(lib):
     bad = list(args)
     bad[6] = FAKE + 8  # pos misaligned
     assert f(2, 2, 10, 128, 128, 16, L.LZ_BF16, *bad, 0) == L.LZ_ERR_INVALID_ARG
+
+
+def _call_hybrid_mse(lib, d, **ptrs):
+    p = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, mk=FAKE, mv=FAKE, h0=None, target=FAKE,
+             o=FAKE, hT=None, lse=None, osw=None, loss=FAKE, dO=None, ws=FAKE)
+    p.update(ptrs)
+    return lib.lz_hybrid_fwd_mse(ctypes.byref(d), p["q"], p["k"], p["v"], p["g"], p["mk"],
+                                 p["mv"], p["h0"], p["target"], p["o"], p["hT"], p["lse"],
+                                 p["osw"], None, p["loss"], p["dO"], p["ws"],
+                                 ptrs.get("ws_bytes", 1 << 40), 0)
+
+
+@pytest.mark.parametrize("which", ["target", "loss", "o", "q"])
+def test_stage1_loss_null_pointer_rejected(lib, which):
+    assert _call_hybrid_mse(lib, _dims(), **{which: None}) == L.LZ_ERR_INVALID_ARG
+    assert b"NULL" in lib.lz_last_error()
+
+
+def test_stage1_loss_validation(lib):
+    d = _dims(dk=128, dv=128)
+    # the loss gradient may not overlap the output
+    nbytes = d.B * d.H * d.T * d.dv * 2
+    assert _call_hybrid_mse(lib, d, dO=FAKE + nbytes // 2) == L.LZ_ERR_INVALID_ARG
+    assert b"overlap" in lib.lz_last_error()
+    assert _call_hybrid_mse(lib, d, target=FAKE + 2) == L.LZ_ERR_INVALID_ARG
+    # its scratch adds the partial sums to the forward's
+    need = L.lz_workspace_bytes(d, L.LZ_WS_HYBRID_FWD_MSE)
+    assert need > L.lz_workspace_bytes(d, L.LZ_WS_HYBRID_FWD)
+    assert _call_hybrid_mse(lib, d, dO=FAKE + nbytes, ws_bytes=need - 1) == L.LZ_ERR_INVALID_ARG
+    assert b"too small" in lib.lz_last_error()
+    # empty problem: scratch of the partial sums only, no data pointers needed
+    e = _dims(T=0)
+    assert L.lz_workspace_bytes(e, L.LZ_WS_HYBRID_FWD_MSE) == 0
