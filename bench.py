@@ -89,7 +89,7 @@ CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.a
 
 class ClockSampler:
     """SM clocks and throttle reasons sampled while the timed region runs:
-    NVML read from a background thread every 10 ms (read-only queries),
+    NVML read from a background thread every 2 ms (read-only queries),
     else nvidia-smi every 100 ms."""
 
     # clocks-event-reason bits (nvml.h): the slowdowns that reject a run,
@@ -116,7 +116,7 @@ class ClockSampler:
                                      {n for n, b in self.REASONS.items() if bits & b}))
             except Exception:
                 pass
-            time.sleep(0.01)
+            time.sleep(0.002)
 
     def __enter__(self):
         import threading
@@ -131,7 +131,7 @@ class ClockSampler:
             self.stop = threading.Event()
             self.thread = threading.Thread(target=self._nvml_loop, args=(handle, nv), daemon=True)
             self.thread.start()
-            self.source = "nvml, 10 ms"
+            self.source = "nvml, 2 ms"
             return self
         except Exception:
             self.thread = None
@@ -213,6 +213,10 @@ def algorithmic_bytes(kernel: str, wl) -> float | None:
         return n * (4 * d * e + 4 * d)
     if kernel.startswith("swa_fwd"):
         return n * (4 * d * e + 4)
+    if kernel.startswith("gla_bwd_delta"):  # backward's first level: reads q, dO, g
+        return n * (2 * d * e + 4 * d)
+    if kernel.startswith("gla_bwd_scan"):  # moves scratch only
+        return None
     if kernel.startswith("gla_bwd") or kernel.startswith("hybrid_bwd"):
         return n * (7 * d * e + 8 * d)
     if kernel.startswith("gla_states") or kernel.startswith("gla_delta"):  # state pass: reads k, v, g

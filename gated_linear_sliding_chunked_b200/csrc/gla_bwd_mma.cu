@@ -3,26 +3,29 @@
 //
 // Gradient of S_t = diag(exp(g_t)) S_{t-1} + k_t v_t^T, o_t = q_t^T S_t (the
 // attention-output regression of the first training stage, Lizard technical
-// summary section 2b, needs it).  Reverse walk over 64-token chunks with
-// b_t the running log-gate inside the chunk, b_l its last value, G the
-// gradient carried in from later chunks (dL/dhT at the end), S_prev the state
-// before the chunk, B[t][s] = dO_t . v_s and A[t][s] = sum_i q_t k_s e^{b_t-b_s}
-// (both for s <= t):
+// summary section 2b, needs it).  Per 64-token chunk, with b_t the running
+// log-gate inside the chunk, b_l its last value, G the state gradient entering
+// the chunk from the later chunks (dL/dhT after the last one), S_prev the
+// state before the chunk, B[t][s] = dO_t . v_s and A[t][s] = sum_i q_t k_s
+// e^{b_t-b_s} (both for s <= t):
 //   dq_t = e^{b_t} (S_prev dO_t) + sum_{s<=t} B[t][s] k_s e^{b_t - b_s}
 //   dk_t = e^{b_l - b_t} (G v_t) + sum_{u>=t} B[u][t] q_u e^{b_u - b_t}
 //   dv_t = (k_t e^{b_l - b_t})^T G + sum_{u>=t} A[u][t] dO_u
-//   G   <- diag(e^{b_l}) G + sum_u (q_u e^{b_u})^T dO_u
+//   G_new = diag(e^{b_l}) G + sum_u (q_u e^{b_u})^T dO_u  (G of the previous chunk)
 //   dg   : the gate's direct gradient is dg_t = e^{g_t} <dS_t, S_{t-1}> per key
-//          dim; at the chunk's first row that is <G_new, S_prev> with G_new
-//          the carried gradient after this chunk's update, and inside the
-//          chunk dg_t = dg_first - sum_{u<t} (q_u dq_u - k_u dk_u), so
+//          dim; at the chunk's first row that is <G_new, S_prev>, and inside
+//          the chunk dg_t = dg_first - sum_{u<t} (q_u dq_u - k_u dk_u), so
 //          rounding errors add up over one chunk, not the whole sequence.
 //
-// Work split: a cluster of two CTAs per (batch, head); CTA r owns key dims
-// [64r, 64r+64).  dq, dk, dg and its half of G are complete inside the CTA;
-// dv is a sum over key dims, so each CTA sends the partial dv of the peer's
-// 64 value columns through distributed shared memory every chunk and adds
-// the peer's share to its own before storing.
+// Two levels: launch_gla_bwd_scan (gla_chunk_mma.cu) forms every chunk's
+// increment of G in parallel and scans them in reverse, giving G and
+// <G_new, S_prev> for every chunk; the kernel here then takes all chunks at
+// once.  Work split: a cluster of two CTAs per (chunk, batch-head); CTA r owns
+// key dims [64r, 64r+64).  dq, dk and dg are complete inside the CTA; dv is a
+// sum over key dims, so each CTA sends the partial dv of the peer's 64 value
+// columns through distributed shared memory and adds the peer's share to its
+// own before storing.  Staging tiles reuse buffers that are dead by then, so
+// that two CTAs fit one SM.
 //
 // Gate factors follow the forward kernel: per key dim, one reference row
 // (the end of the chunk's first half) when each 32-row half decays by at
@@ -73,32 +76,6 @@ __device__ __forceinline__ int rsw(int row, int col) {
   return row * RP + (col ^ ((row & 3) << 3));
 }
 
-struct BwdSmem {
-  bf16 q[2][C * DKH];
-  bf16 k[2][C * DKH];
-  bf16 v[2][C * VP];
-  bf16 dO[2][C * VP];
-  float g[C * DKH];
-  bf16 sp[DKH * DV];   // state before the chunk, rows = this CTA's key dims (swizzled)
-  bf16 qf[C * KP];
-  bf16 kf[C * KP];
-  bf16 qi[C * KP];     // q e^{b}
-  bf16 ks[C * KP];     // k e^{b_l - b}
-  bf16 eqf[C * KP];    // Eq
-  bf16 ekf[C * KP];    // Ek
-  bf16 g16[DKH * DV];  // carried gradient G, bf16 (swizzled)
-  float red[C * RP];   // q*dq - k*dk for the dg scan; then the peer's dv share
-  float dec[NSB][DKH];
-  float fac[NPAIR][DKH];
-  float ci[NSB][DKH];
-  float ck[NSB][DKH];
-  float ec[DKH];
-  float gsp[2][DKH];     // <G_new, S_prev> per key dim, two value halves
-  float tot[NSB][DKH];
-};
-
-static_assert(sizeof(BwdSmem) <= 232448, "shared memory per block exceeds 227 KB");
-
 __device__ __forceinline__ int pair_index(int I, int J) { return I * (I + 1) / 2 + J; }
 
 // exp(sum_{x = s+1 .. t} g_x,i) for chunk rows s <= t (g: global, the
@@ -111,397 +88,397 @@ __device__ __noinline__ float gate_ratio(const float* g, int rows, int t, int s,
   return __expf(lg);
 }
 
+struct ChunkSmem {
+  bf16 v[C * VP];       // then k * dk (fp32, rsw layout)
+  bf16 dO[C * VP];
+  bf16 sp[DKH * DV];    // S_prev (swizzled); then q * dq (fp32, rsw layout)
+  bf16 g16[DKH * DV];   // G entering the chunk (swizzled)
+  bf16 qf[C * KP];      // qf and kf: then the peer's dv share (fp32, rsw layout)
+  bf16 kf[C * KP];
+  bf16 eqf[C * KP];
+  bf16 ekf[C * KP];
+  float dec[NSB][DKH];
+  float fac[NPAIR][DKH];
+  float ci[NSB][DKH];
+  float ck[NSB][DKH];
+  float ksr[NSB][DKH];  // (k e^{b_l - b}) / kf per (sub-block, key dim)
+  float tot[NSB][DKH];
+};
+static_assert(sizeof(ChunkSmem) + 1024 <= 232448 / 2, "two chunk CTAs must fit one SM");
+static_assert(sizeof(float) * C * RP <= sizeof(bf16) * C * VP, "k*dk staging must fit the v tile");
+static_assert(sizeof(float) * C * RP <= sizeof(bf16) * DKH * DV, "q*dq staging must fit the state tile");
+static_assert(sizeof(float) * C * RP <= 2 * sizeof(bf16) * C * KP, "dv share must fit qf + kf");
+
 // Diagonal-block intra term of a strong-decay chunk at (row t, key dim il):
 // role 0 (dq): sum_{s in block, s <= t} (dO_t . v_s) k_s,il exp(b_t - b_s)
 // role 1 (dk): sum_{u in block, u >= t} (dO_u . v_t) q_u,il exp(b_u - b_t)
+// (dO, v: shared tiles; kq, g: global, the chunk's first row, offset to this
+// CTA's key dims)
 __device__ __noinline__ float diag_intra_term(const bf16* dO, const bf16* v, const bf16* kq,
-                                              const float* g, int rows, int I, int t, int il,
-                                              int role) {
+                                                 const float* g, int rows, int I, int t, int il,
+                                                 int role) {
   float x = 0.f;
   const int lo = role == 0 ? SB * I : t, hi = role == 0 ? t : SB * I + SB - 1;
-  for (int r = lo; r <= hi; ++r) {
+  for (int r = lo; r <= hi && r < rows; ++r) {
     const int rq = role == 0 ? t : r, rv = role == 0 ? r : t;
     float b = 0.f;
     for (int j = 0; j < DV; ++j) b += __bfloat162float(dO[rq * VP + j]) * __bfloat162float(v[rv * VP + j]);
-    x += b * __bfloat162float(kq[swz64(r, il)]) *
+    x += b * __bfloat162float(kq[(size_t)r * DK + il]) *
          (role == 0 ? gate_ratio(g, rows, t, r, il) : gate_ratio(g, rows, r, t, il));
   }
   return x;
 }
 
 // A^T[t][u] = sum_i q_u,i k_t,i exp(b_u,i - b_t,i) over this CTA's key dims,
-// chunk rows t <= u < rows (strong-decay fallback of the diagonal blocks).
+// chunk rows t <= u < rows (strong-decay fallback of the diagonal blocks)
 __device__ __noinline__ float diag_at_entry(const bf16* q, const bf16* k, const float* g, int rows,
-                                            int t, int u) {
+                                               int t, int u) {
   float a = 0.f;
   for (int i = 0; i < DKH; ++i) {
     float lg = 0.f;
     for (int x = t + 1; x <= u && x < rows; ++x) lg += g[(size_t)x * DK + i];
-    a += __bfloat162float(q[swz64(u, i)]) * __bfloat162float(k[swz64(t, i)]) * __expf(lg);
+    a += __bfloat162float(q[(size_t)u * DK + i]) * __bfloat162float(k[(size_t)t * DK + i]) * __expf(lg);
   }
   return a;
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
-    gla_bwd_mma_kernel(GlaBwdParams p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
+    gla_bwd_chunk_kernel(GlaBwdParams p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  BwdSmem& sm = *reinterpret_cast<BwdSmem*>(smem_raw);
+  ChunkSmem& sm = *reinterpret_cast<ChunkSmem*>(smem_raw);
   cg::cluster_group cluster = cg::this_cluster();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gr = lane >> 2, gc = (lane & 3) * 2;
-  const int half = blockIdx.x;  // == rank in the cluster
-  const int i0 = half * DKH;    // first key dim of this CTA
-  const int bh = blockIdx.y;
-  const int T = p.T;
+  const int half = blockIdx.x & 1;  // == rank in the cluster
+  const int i0 = half * DKH;        // first key dim of this CTA
+  const int T = p.T, nchunks = (T + C - 1) / C;
+  const int c = (int)((blockIdx.x >> 1) % (unsigned)nchunks), bh = (int)((blockIdx.x >> 1) / (unsigned)nchunks);
+  const int c0 = c * C;
+  const int rows = min(C, T - c0);
   const size_t tk = (size_t)bh * T * DK, tv = (size_t)bh * T * DV;
-  const bf16* q = (const bf16*)p.q + tk;
-  const bf16* k = (const bf16*)p.k + tk;
-  const bf16* v = (const bf16*)p.v + tv;
-  const bf16* dO = (const bf16*)p.dO + tv;
-  const float* g = p.g + tk;
-  const bf16* st16 = (const bf16*)p.states16;
-  const int nchunks = (T + C - 1) / C;
-  float* peer_red = cluster.map_shared_rank(sm.red, half ^ 1);
+  // this chunk's first row, this CTA's key dims
+  const bf16* qc = (const bf16*)p.q + tk + (size_t)c0 * DK + i0;
+  const bf16* kc = (const bf16*)p.k + tk + (size_t)c0 * DK + i0;
+  const float* gch = p.g + tk + (size_t)c0 * DK + i0;
+  float* stq = reinterpret_cast<float*>(sm.sp);   // q * dq
+  float* stk = reinterpret_cast<float*>(sm.v);    // k * dk
+  float* xch = reinterpret_cast<float*>(sm.qf);   // the peer's dv share
+  float* peer_xch = cluster.map_shared_rank(xch, half ^ 1);
 
-  auto issue_tiles = [&](int c, int st) {
-    const int c0 = c * C;
-    for (int x = tid; x < C * DKH / 8; x += NT) {
-      const int r = x / (DKH / 8), cc = x % (DKH / 8);
-      const bool ok = c0 + r < T;
-      const size_t off = (size_t)(ok ? c0 + r : 0) * DK + i0 + cc * 8;
-      cp_async16(&sm.q[st][swz64(r, cc * 8)], q + off, ok ? 16 : 0);
-      cp_async16(&sm.k[st][swz64(r, cc * 8)], k + off, ok ? 16 : 0);
-    }
-    for (int x = tid; x < C * DV / 8; x += NT) {
-      const int r = x / (DV / 8), cc = x % (DV / 8);
-      const bool ok = c0 + r < T;
-      const size_t off = (size_t)(ok ? c0 + r : 0) * DV + cc * 8;
-      cp_async16(&sm.v[st][r * VP + cc * 8], v + off, ok ? 16 : 0);
-      cp_async16(&sm.dO[st][r * VP + cc * 8], dO + off, ok ? 16 : 0);
-    }
-    cp_async_commit();
-  };
-  auto issue_g = [&](int c) {
-    const int c0 = c * C;
+  // raw g, q, k of this CTA's key dims, staged where qf / kf and eqf / ekf go
+  // once the prep has read them (rows past the end read as zeros)
+  float* gs = reinterpret_cast<float*>(sm.qf);  // [C][DKH] fp32
+  bf16* qs = sm.eqf;                            // [C][DKH] bf16 (swz64)
+  bf16* ks = sm.ekf;
+  {
     for (int x = tid; x < C * DKH / 4; x += NT) {
       const int r = x / (DKH / 4), cc = x % (DKH / 4);
-      const bool ok = c0 + r < T;
-      const size_t off = (size_t)(ok ? c0 + r : 0) * DK + i0 + cc * 4;
-      cp_async16(&sm.g[r * DKH + cc * 4], g + off, ok ? 16 : 0);
+      const bool ok = r < rows;
+      cp_async16(&gs[r * DKH + cc * 4], gch + (size_t)(ok ? r : 0) * DK + cc * 4, ok ? 16 : 0);
+    }
+    for (int x = tid; x < C * DKH / 8; x += NT) {
+      const int r = x / (DKH / 8), cc = x % (DKH / 8);
+      const bool ok = r < rows;
+      const size_t off = (size_t)(ok ? r : 0) * DK + cc * 8;
+      cp_async16(&qs[swz64(r, cc * 8)], qc + off, ok ? 16 : 0);
+      cp_async16(&ks[swz64(r, cc * 8)], kc + off, ok ? 16 : 0);
     }
     cp_async_commit();
-  };
-  auto issue_sp = [&](int c) {
-    const bf16* src = st16 + ((size_t)bh * nchunks + c) * DK * DV + (size_t)i0 * DV;
+  }
+  {  // tiles: v, dO, S_prev and G rows of this CTA's key dims
+    const bf16* v = (const bf16*)p.v + tv + (size_t)c0 * DV;
+    const bf16* dO = (const bf16*)p.dO + tv + (size_t)c0 * DV;
+    for (int x = tid; x < C * DV / 8; x += NT) {
+      const int r = x / (DV / 8), cc = x % (DV / 8);
+      const bool ok = r < rows;
+      const size_t off = (size_t)(ok ? r : 0) * DV + cc * 8;
+      cp_async16(&sm.v[r * VP + cc * 8], v + off, ok ? 16 : 0);
+      cp_async16(&sm.dO[r * VP + cc * 8], dO + off, ok ? 16 : 0);
+    }
+    const size_t so = ((size_t)bh * nchunks + c) * DK * DV + (size_t)i0 * DV;
+    const bf16* sp = (const bf16*)p.states16 + so;
+    const bf16* gi = (const bf16*)p.gin16 + so;
     for (int x = tid; x < DKH * DV / 8; x += NT) {
       const int r = x / (DV / 8), cc = x % (DV / 8);
-      cp_async16(&sm.sp[swz(r, cc * 8)], src + (size_t)r * DV + cc * 8, 16);
+      cp_async16(&sm.sp[swz(r, cc * 8)], sp + (size_t)r * DV + cc * 8, 16);
+      cp_async16(&sm.g16[swz(r, cc * 8)], gi + (size_t)r * DV + cc * 8, 16);
     }
     cp_async_commit();
-  };
+  }
+  cp_async_wait<1>();
+  __syncthreads();
 
-  // ---- carried gradient G: warp -> (key-dim tile mt, value half nh) --------
-  const int mt = warp & 3, gnh = warp >> 2;
-  float G[8][4];
+  // ---- prep 1: per key dim cumulative gate products ------------------------
+  const int K = tid >> 6, i = tid & 63, r0 = K * SB;
+  float qfac[SB], kfac[SB];
+  {
+    float e[SB];
+#pragma unroll
+    for (int r = 0; r < SB; ++r) e[r] = __expf(gs[(r0 + r) * DKH + i]);
+    float run = 1.f;
+#pragma unroll
+    for (int r = SB - 1; r >= 0; --r) {
+      kfac[r] = run;
+      run *= e[r];
+    }
+    run = 1.f;
+#pragma unroll
+    for (int r = 0; r < SB; ++r) {
+      run *= e[r];
+      qfac[r] = run;
+    }
+    sm.dec[K][i] = run;
+  }
+  __syncthreads();
+  // ---- prep 2: operands and factor tables -------------------------------
+  int flags;
+  {
+    const float d0 = sm.dec[0][i], d1 = sm.dec[1][i], d2 = sm.dec[2][i], d3 = sm.dec[3][i];
+    const float dk4[NSB] = {d0, d1, d2, d3};
+    const bool tame = (d0 * d1 >= kMinBlockDecay) && (d2 * d3 >= kMinBlockDecay);
+    const bool bad = !tame && !(d0 >= kMinBlockDecay && d1 >= kMinBlockDecay &&
+                                d2 >= kMinBlockDecay && d3 >= kMinBlockDecay);
+    float rq = 1.f, rk = 1.f;
+    if (tame) {
+      rq = K == 0 ? 1.f / (d0 * d1) : K == 1 ? 1.f / d1 : K == 2 ? 1.f : d2;
+      rk = K == 0 ? d1 : K == 1 ? 1.f : K == 2 ? 1.f / d2 : 1.f / (d2 * d3);
+    }
+    float eqk = 1.f, ksk = 1.f;
+#pragma unroll
+    for (int J = 0; J < NSB; ++J) {
+      if (J < K) eqk *= dk4[J];
+      if (J > K) ksk *= dk4[J];
+    }
+    // inter factors for sub-block K: e^{b_t}/Eq and e^{b_l - b_t}/Ek
+    sm.ci[K][i] = tame ? d0 * d1 : eqk;
+    sm.ck[K][i] = tame ? d2 * d3 : ksk;
+    sm.ksr[K][i] = ksk / rk;
+#pragma unroll
+    for (int I = 0; I < NSB; ++I)
+#pragma unroll
+      for (int J = 0; J <= I; ++J) {
+        if (pair_index(I, J) % NSB != K) continue;
+        float f = 1.f;
+        if (!tame) {
+          if (J == I) {
+            f = 1.f / fmaxf(dk4[I], 1e-30f);
+          } else {
+#pragma unroll
+            for (int Kp = 0; Kp < NSB; ++Kp)
+              if (Kp > J && Kp < I) f *= dk4[Kp];
+          }
+        }
+        sm.fac[pair_index(I, J)][i] = f;
+      }
+    // qf / kf go over the staged gates (read before the last barrier); the
+    // output scales go over the raw q / k once every thread has read them
+#pragma unroll
+    for (int r = 0; r < SB; ++r) {
+      const int o = (r0 + r) * KP + i;
+      sm.qf[o] = __float2bfloat16_rn(__bfloat162float(qs[swz64(r0 + r, i)]) * (qfac[r] * rq));
+      sm.kf[o] = __float2bfloat16_rn(__bfloat162float(ks[swz64(r0 + r, i)]) * (kfac[r] * rk));
+    }
+    const int w = __syncthreads_or(!tame);
+#pragma unroll
+    for (int r = 0; r < SB; ++r) {
+      const int o = (r0 + r) * KP + i;
+      sm.eqf[o] = __float2bfloat16_rn(qfac[r] * rq);
+      sm.ekf[o] = __float2bfloat16_rn(kfac[r] * rk);
+    }
+    cp_async_wait<0>();
+    const int b = __syncthreads_or(bad);
+    flags = (w ? 1 : 0) | (b ? 2 : 0);
+  }
+  const bool scaled = flags & 1, slow = flags & 2;
+
+  // warp -> (row block I, role): role 0 computes dq and dv of value columns
+  // [0, 64); role 1 computes dk and dv of value columns [64, 128)
+  const int I = warp & 3, role = warp >> 2;
+  const bf16* arows = role == 0 ? sm.dO : sm.v;
+  const bf16* prows = role == 0 ? sm.v : sm.dO;
+  const bf16* inter_b = role == 0 ? sm.sp : sm.g16;
+  const bf16* intra_b = role == 0 ? sm.kf : sm.qf;
+  const float* colf = role == 0 ? sm.ci[I] : sm.ck[I];
+  const bf16* oscale = role == 0 ? sm.eqf : sm.ekf;
+  float acc[8][4];
 #pragma unroll
   for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int i = i0 + 16 * mt + gr + 8 * hh, j = 64 * gnh + nt * 8 + gc;
-      float a = 0.f, b = 0.f;
-      if (p.dhT) {
-        const float* src = p.dhT + ((size_t)bh * DK + i) * DV + j;
-        a = src[0];
-        b = src[1];
-      }
-      G[nt][2 * hh] = a;
-      G[nt][2 * hh + 1] = b;
+    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+  // ---- inter: (dO S_prev^T | v G^T), then per-dim factor (ci | ck) --------
+#pragma unroll 2
+  for (int kk = 0; kk < 8; ++kk) {
+    uint32_t a[4];
+    ldsm_x4(smem_u32(&arows[(16 * I + (lane & 15)) * VP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
+            a[3]);
+#pragma unroll
+    for (int ntp = 0; ntp < 4; ++ntp) {
+      uint32_t b0, b1, b2, b3;
+      const int n = ntp * 16 + (lane & 7) + ((lane >> 4) << 3);
+      ldsm_x4(smem_u32(&inter_b[swz(n, kk * 16 + ((lane >> 3) & 1) * 8)]), b0, b1, b2, b3);
+      mma_bf16(acc[2 * ntp], a, b0, b1);
+      mma_bf16(acc[2 * ntp + 1], a, b2, b3);
     }
-  auto write_g16 = [&]() {
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int r = 16 * mt + gr + 8 * hh, j = 64 * gnh + nt * 8 + gc;
-        *reinterpret_cast<uint32_t*>(&sm.g16[swz(r, j)]) = pack_bf16(G[nt][2 * hh], G[nt][2 * hh + 1]);
-      }
-  };
-  write_g16();
-  if (nchunks > 0) {
-    issue_tiles(nchunks - 1, 0);
-    issue_g(nchunks - 1);
-    issue_sp(nchunks - 1);
   }
-  for (int it = 0; it < nchunks; ++it) {
-    const int c = nchunks - 1 - it;
-    const int st = it & 1;
-    const int c0 = c * C;
-    const int rows = T - c0;  // valid rows in this chunk (may exceed C)
-    cp_async_wait<0>();
-    __syncthreads();
-    if (c > 0) issue_tiles(c - 1, st ^ 1);
-
-    // ---- prep 1: per key dim cumulative gate products -----------------------
-    const int K = tid >> 6, i = tid & 63, r0 = K * SB;
-    float qfac[SB], kfac[SB];
-    {
-      float e[SB];
 #pragma unroll
-      for (int r = 0; r < SB; ++r) e[r] = __expf(sm.g[(r0 + r) * DKH + i]);
-      float run = 1.f;
+  for (int nt = 0; nt < 8; ++nt) {
+    const float2 f = *reinterpret_cast<const float2*>(&colf[nt * 8 + gc]);
+    acc[nt][0] *= f.x;
+    acc[nt][1] *= f.y;
+    acc[nt][2] *= f.x;
+    acc[nt][3] *= f.y;
+  }
+  // ---- intra: one 16x16 score block at a time, consumed right away -------
+  const int jlo = role == 0 ? 0 : I, jhi = role == 0 ? I : NSB - 1;
+  for (int J = jlo; J <= jhi; ++J) {
+    float sc[2][4], sc2[2][4];  // two partial sums over k for independent MMA chains
 #pragma unroll
-      for (int r = SB - 1; r >= 0; --r) {
-        kfac[r] = run;
-        run *= e[r];
-      }
-      run = 1.f;
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int r = 0; r < SB; ++r) {
-        run *= e[r];
-        qfac[r] = run;
-      }
-      sm.dec[K][i] = run;
+      for (int e = 0; e < 4; ++e) sc[nt][e] = sc2[nt][e] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < 8; kk += 2) {
+      uint32_t a[4], b0, b1, b2, b3, cc[4], d0, d1, d2, d3;
+      ldsm_x4(smem_u32(&arows[(16 * I + (lane & 15)) * VP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
+              a[3]);
+      ldsm_x4(smem_u32(&prows[(16 * J + (lane & 7) + ((lane >> 4) << 3)) * VP + kk * 16 +
+                              ((lane >> 3) & 1) * 8]),
+              b0, b1, b2, b3);
+      ldsm_x4(smem_u32(&arows[(16 * I + (lane & 15)) * VP + kk * 16 + 16 + (lane >> 4) * 8]), cc[0], cc[1],
+              cc[2], cc[3]);
+      ldsm_x4(smem_u32(&prows[(16 * J + (lane & 7) + ((lane >> 4) << 3)) * VP + kk * 16 + 16 +
+                              ((lane >> 3) & 1) * 8]),
+              d0, d1, d2, d3);
+      mma_bf16(sc[0], a, b0, b1);
+      mma_bf16(sc[1], a, b2, b3);
+      mma_bf16(sc2[0], cc, d0, d1);
+      mma_bf16(sc2[1], cc, d2, d3);
     }
-    __syncthreads();
-    if (c > 0) issue_g(c - 1);
-    // ---- prep 2: operands and factor tables -------------------------------
-    int flags;
-    {
-      const float d0 = sm.dec[0][i], d1 = sm.dec[1][i], d2 = sm.dec[2][i], d3 = sm.dec[3][i];
-      const float dk4[NSB] = {d0, d1, d2, d3};
-      const bool tame = (d0 * d1 >= kMinBlockDecay) && (d2 * d3 >= kMinBlockDecay);
-      const bool bad = !tame && !(d0 >= kMinBlockDecay && d1 >= kMinBlockDecay &&
-                                  d2 >= kMinBlockDecay && d3 >= kMinBlockDecay);
-      float rq = 1.f, rk = 1.f;
-      if (tame) {
-        rq = K == 0 ? 1.f / (d0 * d1) : K == 1 ? 1.f / d1 : K == 2 ? 1.f : d2;
-        rk = K == 0 ? d1 : K == 1 ? 1.f : K == 2 ? 1.f / d2 : 1.f / (d2 * d3);
-      }
-      float eqk = 1.f, ksk = 1.f;
 #pragma unroll
-      for (int J = 0; J < NSB; ++J) {
-        if (J < K) eqk *= dk4[J];
-        if (J > K) ksk *= dk4[J];
-      }
-      // inter factors for sub-block K: e^{b_t}/Eq and e^{b_l - b_t}/Ek
-      sm.ci[K][i] = tame ? d0 * d1 : eqk;
-      sm.ck[K][i] = tame ? d2 * d3 : ksk;
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int I = 0; I < NSB; ++I)
+      for (int e = 0; e < 4; ++e) sc[nt][e] += sc2[nt][e];
+    if (J == I) {
+      if (slow) continue;  // the diagonal block of a strong-decay chunk: below
 #pragma unroll
-        for (int J = 0; J <= I; ++J) {
-          if (pair_index(I, J) % NSB != K) continue;
-          float f = 1.f;
-          if (!tame) {
-            if (J == I) {
-              f = 1.f / fmaxf(dk4[I], 1e-30f);
-            } else {
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-              for (int Kp = 0; Kp < NSB; ++Kp)
-                if (Kp > J && Kp < I) f *= dk4[Kp];
-            }
-          }
-          sm.fac[pair_index(I, J)][i] = f;
+        for (int e = 0; e < 4; ++e) {
+          const int t = gr + (e >> 1) * 8, u = nt * 8 + gc + (e & 1);
+          if (role == 0 ? (u > t) : (u < t)) sc[nt][e] = 0.f;
         }
-      if (K == 0) sm.ec[i] = d0 * d1 * d2 * d3;
-#pragma unroll
-      for (int r = 0; r < SB; ++r) {
-        const float qv = __bfloat162float(sm.q[st][swz64(r0 + r, i)]);
-        const float kv = __bfloat162float(sm.k[st][swz64(r0 + r, i)]);
-        const float eq = qfac[r] * rq, ek = kfac[r] * rk;
-        const int o = (r0 + r) * KP + i;
-        sm.qf[o] = __float2bfloat16_rn(qv * eq);
-        sm.kf[o] = __float2bfloat16_rn(kv * ek);
-        sm.qi[o] = __float2bfloat16_rn(qv * qfac[r] * eqk);
-        sm.ks[o] = __float2bfloat16_rn(kv * kfac[r] * ksk);
-        sm.eqf[o] = __float2bfloat16_rn(eq);
-        sm.ekf[o] = __float2bfloat16_rn(ek);
-      }
-      const int w = __syncthreads_or(!tame);
-      const int b = __syncthreads_or(bad);
-      flags = (w ? 1 : 0) | (b ? 2 : 0);
     }
-    const bool scaled = flags & 1, slow = flags & 2;
-
-    // warp -> (row block I, role): role 0 computes dq and dv of value columns
-    // [0, 64); role 1 computes dk and dv of value columns [64, 128)
-    const int I = warp & 3, role = warp >> 2;
-    const int Ivp = role == 0 ? I : NSB - 1 - I;  // dv row block (see below)
-    const float* gch = g + (size_t)c0 * DK + i0;  // this chunk, this CTA's dims
-    // in-place terms (the window branch's gradients) for this warp's outputs,
-    // loaded now so that the loads overlap the products below
-    uint32_t pre[8][2], prev[8][2];
-    if (p.add_in_place) {
-      const bf16* src = (const bf16*)(role == 0 ? p.dq : p.dk);
+    const uint32_t pa[4] = {pack_bf16(sc[0][0], sc[0][1]), pack_bf16(sc[0][2], sc[0][3]),
+                            pack_bf16(sc[1][0], sc[1][1]), pack_bf16(sc[1][2], sc[1][3])};
+    const float* fac = sm.fac[role == 0 ? pair_index(I, J) : pair_index(J, I)];
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
+    for (int ntp = 0; ntp < 4; ++ntp) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(smem_u32(&intra_b[(16 * J + (lane & 7) + ((lane >> 3) & 1) * 8) * KP + ntp * 16 +
+                                  (lane >> 4) * 8]),
+                b0, b1, b2, b3);
+      if (scaled) {
+        const float f0 = fac[ntp * 16 + gr], f1 = fac[ntp * 16 + 8 + gr];
+        b0 = scale_bf16x2(b0, f0, f0);
+        b1 = scale_bf16x2(b1, f0, f0);
+        b2 = scale_bf16x2(b2, f1, f1);
+        b3 = scale_bf16x2(b3, f1, f1);
+      }
+      mma_bf16(acc[2 * ntp], pa, b0, b1);
+      mma_bf16(acc[2 * ntp + 1], pa, b2, b3);
+    }
+  }
+  // ---- finalize (dq | dk) = (Eq | Ek) * acc, store; keep (q dq | k dk) -----
+  {
+    const bf16* raw = role == 0 ? qc : kc;
+    bf16* outp = (bf16*)(role == 0 ? p.dq : p.dk);
+    const float* addf = role == 0 ? p.add_dq : p.add_dk;
+    // two rounds of four column tiles; each round issues its global loads
+    // before its first store
+#pragma unroll
+    for (int n0 = 0; n0 < 8; n0 += 4) {
+      uint32_t rv[4][2], inp[4][2];
+#pragma unroll
+      for (int n = 0; n < 4; ++n)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int t = 16 * I + gr + 8 * hh;
-          pre[nt][hh] = c0 + t < T ? *reinterpret_cast<const uint32_t*>(
-                                         &src[tk + (size_t)(c0 + t) * DK + i0 + nt * 8 + gc])
-                                   : 0u;
-          const int tv2 = 16 * Ivp + gr + 8 * hh;
-          prev[nt][hh] = (role == half && c0 + tv2 < T)
-                             ? *reinterpret_cast<const uint32_t*>(
-                                   &((const bf16*)p.dv)[tv + (size_t)(c0 + tv2) * DV + 64 * half + nt * 8 + gc])
-                             : 0u;
+          const int il = (n0 + n) * 8 + gc;
+          const bool ok = t < rows;
+          rv[n][hh] = ok ? __ldg(reinterpret_cast<const unsigned int*>(&raw[(size_t)t * DK + il])) : 0u;
+          inp[n][hh] = ok && p.add_in_place && !addf
+                           ? *reinterpret_cast<const uint32_t*>(&outp[tk + (size_t)(c0 + t) * DK + i0 + il])
+                           : 0u;
         }
-    }
-    // role 0: A rows = dO rows I, score partner = v rows J <= I, inter B = S_prev,
-    //         intra B = Kf_J (factor F_IJ), output scale Eq
-    // role 1: A rows = v rows I,  score partner = dO rows J >= I, inter B = G,
-    //         intra B = Qf_J (factor F_JI), output scale Ek
-    const bf16* arows = role == 0 ? sm.dO[st] : sm.v[st];
-    const bf16* prows = role == 0 ? sm.v[st] : sm.dO[st];
-    const bf16* inter_b = role == 0 ? sm.sp : sm.g16;
-    const bf16* intra_b = role == 0 ? sm.kf : sm.qf;
-    const float* colf = role == 0 ? sm.ci[I] : sm.ck[I];
-    const bf16* oscale = role == 0 ? sm.eqf : sm.ekf;
-    float acc[8][4];
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+      for (int n = 0; n < 4; ++n)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-    // ---- inter: (dO S_prev^T | v G^T), then per-dim factor (ci | ck) --------
-#pragma unroll 2
-    for (int kk = 0; kk < 8; ++kk) {
-      uint32_t a[4];
-      ldsm_x4(smem_u32(&arows[(16 * I + (lane & 15)) * VP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
-              a[3]);
-#pragma unroll
-      for (int ntp = 0; ntp < 4; ++ntp) {
-        uint32_t b0, b1, b2, b3;
-        const int n = ntp * 16 + (lane & 7) + ((lane >> 4) << 3);
-        ldsm_x4(smem_u32(&inter_b[swz(n, kk * 16 + ((lane >> 3) & 1) * 8)]), b0, b1, b2, b3);
-        mma_bf16(acc[2 * ntp], a, b0, b1);
-        mma_bf16(acc[2 * ntp + 1], a, b2, b3);
-      }
-    }
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const float2 f = *reinterpret_cast<const float2*>(&colf[nt * 8 + gc]);
-      acc[nt][0] *= f.x;
-      acc[nt][1] *= f.y;
-      acc[nt][2] *= f.x;
-      acc[nt][3] *= f.y;
-    }
-    // ---- intra: one 16x16 score block at a time, consumed right away -------
-    const int jlo = role == 0 ? 0 : I, jhi = role == 0 ? I : NSB - 1;
-    for (int J = jlo; J <= jhi; ++J) {
-      float sc[2][4], sc2[2][4];  // two partial sums over k for independent MMA chains
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sc[nt][e] = sc2[nt][e] = 0.f;
-#pragma unroll
-      for (int kk = 0; kk < 8; kk += 2) {
-        uint32_t a[4], b0, b1, b2, b3, c[4], d0, d1, d2, d3;
-        ldsm_x4(smem_u32(&arows[(16 * I + (lane & 15)) * VP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
-                a[3]);
-        ldsm_x4(smem_u32(&prows[(16 * J + (lane & 7) + ((lane >> 4) << 3)) * VP + kk * 16 +
-                                ((lane >> 3) & 1) * 8]),
-                b0, b1, b2, b3);
-        ldsm_x4(smem_u32(&arows[(16 * I + (lane & 15)) * VP + kk * 16 + 16 + (lane >> 4) * 8]), c[0], c[1],
-                c[2], c[3]);
-        ldsm_x4(smem_u32(&prows[(16 * J + (lane & 7) + ((lane >> 4) << 3)) * VP + kk * 16 + 16 +
-                                ((lane >> 3) & 1) * 8]),
-                d0, d1, d2, d3);
-        mma_bf16(sc[0], a, b0, b1);
-        mma_bf16(sc[1], a, b2, b3);
-        mma_bf16(sc2[0], c, d0, d1);
-        mma_bf16(sc2[1], c, d2, d3);
-      }
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sc[nt][e] += sc2[nt][e];
-      if (J == I) {
-        if (slow) continue;  // the diagonal block of a strong-decay chunk: below
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int t = gr + (e >> 1) * 8, u = nt * 8 + gc + (e & 1);
-            if (role == 0 ? (u > t) : (u < t)) sc[nt][e] = 0.f;
+        for (int hh = 0; hh < 2; ++hh) {
+          const int nt = n0 + n;
+          const int t = 16 * I + gr + 8 * hh;
+          const int il = nt * 8 + gc;
+          const float2 os = unpack_bf16(*reinterpret_cast<const uint32_t*>(&oscale[t * KP + il]));
+          float x0 = acc[nt][2 * hh] * os.x, x1 = acc[nt][2 * hh + 1] * os.y;
+          if (slow) {
+            x0 += diag_intra_term(sm.dO, sm.v, role == 0 ? kc : qc, gch, rows, I, t, il, role);
+            x1 += diag_intra_term(sm.dO, sm.v, role == 0 ? kc : qc, gch, rows, I, t, il + 1, role);
           }
-      }
-      const uint32_t pa[4] = {pack_bf16(sc[0][0], sc[0][1]), pack_bf16(sc[0][2], sc[0][3]),
-                              pack_bf16(sc[1][0], sc[1][1]), pack_bf16(sc[1][2], sc[1][3])};
-      const float* fac = sm.fac[role == 0 ? pair_index(I, J) : pair_index(J, I)];
-#pragma unroll
-      for (int ntp = 0; ntp < 4; ++ntp) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(smem_u32(&intra_b[(16 * J + (lane & 7) + ((lane >> 3) & 1) * 8) * KP + ntp * 16 +
-                                    (lane >> 4) * 8]),
-                  b0, b1, b2, b3);
-        if (scaled) {
-          const float f0 = fac[ntp * 16 + gr], f1 = fac[ntp * 16 + 8 + gr];
-          b0 = scale_bf16x2(b0, f0, f0);
-          b1 = scale_bf16x2(b1, f0, f0);
-          b2 = scale_bf16x2(b2, f1, f1);
-          b3 = scale_bf16x2(b3, f1, f1);
+          if (t < rows) {
+            const size_t off = tk + (size_t)(c0 + t) * DK + i0 + il;
+            float y0 = x0, y1 = x1;
+            if (addf) {
+              const float2 a = *reinterpret_cast<const float2*>(&addf[off]);
+              y0 += a.x;
+              y1 += a.y;
+            } else {
+              const float2 a = unpack_bf16(inp[n][hh]);
+              y0 += a.x;
+              y1 += a.y;
+            }
+            *reinterpret_cast<uint32_t*>(&outp[off]) = pack_bf16(y0, y1);
+          }
+          const float2 xv = unpack_bf16(rv[n][hh]);
+          acc[nt][2 * hh] = xv.x * x0;
+          acc[nt][2 * hh + 1] = xv.y * x1;
         }
-        mma_bf16(acc[2 * ntp], pa, b0, b1);
-        mma_bf16(acc[2 * ntp + 1], pa, b2, b3);
-      }
     }
-    // ---- finalize (dq | dk) = (Eq | Ek) * acc, store, stage for dg ---------
-    float kdk[8][4];  // role 1: k * dk, subtracted into red after a barrier
+  }
+  __syncthreads();  // every reader of S_prev and v is done
+  {
+    float* st = role == 0 ? stq : stk;
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
-        const int t = 16 * I + gr + 8 * hh;
-        const int il = nt * 8 + gc;
-        const float2 os = unpack_bf16(*reinterpret_cast<const uint32_t*>(&oscale[t * KP + il]));
-        float x0 = acc[nt][2 * hh] * os.x, x1 = acc[nt][2 * hh + 1] * os.y;
-        if (slow) {
-          x0 += diag_intra_term(sm.dO[st], sm.v[st], role == 0 ? sm.k[st] : sm.q[st], gch, rows, I, t, il,
-                                role);
-          x1 += diag_intra_term(sm.dO[st], sm.v[st], role == 0 ? sm.k[st] : sm.q[st], gch, rows, I, t,
-                                il + 1, role);
-        }
-        if (c0 + t < T) {
-          const size_t off = tk + (size_t)(c0 + t) * DK + i0 + il;
-          const float* addf = role == 0 ? p.add_dq : p.add_dk;
-          float y0 = x0, y1 = x1;
-          if (addf) {
-            const float2 a = *reinterpret_cast<const float2*>(&addf[off]);
-            y0 += a.x;
-            y1 += a.y;
-          } else if (p.add_in_place) {
-            const float2 a = unpack_bf16(pre[nt][hh]);
-            y0 += a.x;
-            y1 += a.y;
-          }
-          *reinterpret_cast<uint32_t*>(&((bf16*)(role == 0 ? p.dq : p.dk))[off]) = pack_bf16(y0, y1);
-        }
-        const float2 xv = unpack_bf16(*reinterpret_cast<const uint32_t*>(
-            &(role == 0 ? sm.q[st] : sm.k[st])[swz64(t, il)]));
-        if (role == 0) {
-          *reinterpret_cast<float2*>(&sm.red[rsw(t, il)]) = make_float2(xv.x * x0, xv.y * x1);
-        } else {
-          kdk[nt][2 * hh] = xv.x * x0;
-          kdk[nt][2 * hh + 1] = xv.y * x1;
-        }
+        const int t = 16 * I + gr + 8 * hh, il = nt * 8 + gc;
+        *reinterpret_cast<float2*>(&st[rsw(t, il)]) = make_float2(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
       }
+  }
 
-    // ---- partial dv of row block Iv, value columns [64 role, 64 role + 64) ---
-    // (role 1 takes the mirrored row block so that every warp multiplies
-    // 5 score blocks: dq/dk of I take I+1 / 4-I, dv of Iv takes 4-Iv)
-    const int Iv = role == 0 ? I : NSB - 1 - I;
-    float dvh[8][4];
+  // ---- partial dv of row block Iv, value columns [64 role, 64 role + 64) ---
+  // (role 1 takes the mirrored row block so that every warp multiplies
+  // 5 score blocks)
+  const int Iv = role == 0 ? I : NSB - 1 - I;
+  float dvh[8][4];
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+  for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) dvh[nt][e] = 0.f;
-    // inter: (k e^{b_l - b})_Iv G[:, this role's columns]
+    for (int e = 0; e < 4; ++e) dvh[nt][e] = 0.f;
+  // inter: (k e^{b_l - b})_Iv G[:, this role's columns], the k operand as kf
+  // rescaled per key dim
+  {
+    const float* ksr = sm.ksr[Iv];
 #pragma unroll
     for (int kk = 0; kk < DKH / 16; ++kk) {
       uint32_t a[4];
-      ldsm_x4(smem_u32(&sm.ks[(16 * Iv + (lane & 15)) * KP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
+      ldsm_x4(smem_u32(&sm.kf[(16 * Iv + (lane & 15)) * KP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
               a[3]);
+      const float2 f0 = *reinterpret_cast<const float2*>(&ksr[kk * 16 + gc]);
+      const float2 f1 = *reinterpret_cast<const float2*>(&ksr[kk * 16 + 8 + gc]);
+      a[0] = scale_bf16x2(a[0], f0.x, f0.y);
+      a[1] = scale_bf16x2(a[1], f0.x, f0.y);
+      a[2] = scale_bf16x2(a[2], f1.x, f1.y);
+      a[3] = scale_bf16x2(a[3], f1.x, f1.y);
 #pragma unroll
       for (int ntp = 0; ntp < 4; ++ntp) {
         uint32_t b0, b1, b2, b3;
@@ -511,208 +488,147 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
         mma_bf16(dvh[2 * ntp + 1], a, b2, b3);
       }
     }
-    // intra: A^T[Iv][J] dO_J for J >= Iv, one score block at a time
-    for (int J = Iv; J < NSB; ++J) {
-      float at[2][4];
+  }
+  // intra: A^T[Iv][J] dO_J for J >= Iv, one score block at a time
+  for (int J = Iv; J < NSB; ++J) {
+    float at[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) at[nt][e] = 0.f;
+    const float* fac = sm.fac[pair_index(J, Iv)];
+#pragma unroll
+    for (int kk = 0; kk < DKH / 16; ++kk) {
+      uint32_t a[4];
+      ldsm_x4(smem_u32(&sm.kf[(16 * Iv + (lane & 15)) * KP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
+              a[3]);
+      if (scaled) {
+        const float2 f0 = *reinterpret_cast<const float2*>(&fac[kk * 16 + gc]);
+        const float2 f1 = *reinterpret_cast<const float2*>(&fac[kk * 16 + 8 + gc]);
+        a[0] = scale_bf16x2(a[0], f0.x, f0.y);
+        a[1] = scale_bf16x2(a[1], f0.x, f0.y);
+        a[2] = scale_bf16x2(a[2], f1.x, f1.y);
+        a[3] = scale_bf16x2(a[3], f1.x, f1.y);
+      }
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(smem_u32(&sm.qf[(16 * J + (lane & 7) + ((lane >> 4) << 3)) * KP + kk * 16 +
+                              ((lane >> 3) & 1) * 8]),
+              b0, b1, b2, b3);
+      mma_bf16(at[0], a, b0, b1);
+      mma_bf16(at[1], a, b2, b3);
+    }
+    if (J == Iv) {
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) at[nt][e] = 0.f;
-      const float* fac = sm.fac[pair_index(J, Iv)];
-#pragma unroll
-      for (int kk = 0; kk < DKH / 16; ++kk) {
-        uint32_t a[4];
-        ldsm_x4(smem_u32(&sm.kf[(16 * Iv + (lane & 15)) * KP + kk * 16 + (lane >> 4) * 8]), a[0], a[1], a[2],
-                a[3]);
-        if (scaled) {
-          const float2 f0 = *reinterpret_cast<const float2*>(&fac[kk * 16 + gc]);
-          const float2 f1 = *reinterpret_cast<const float2*>(&fac[kk * 16 + 8 + gc]);
-          a[0] = scale_bf16x2(a[0], f0.x, f0.y);
-          a[1] = scale_bf16x2(a[1], f0.x, f0.y);
-          a[2] = scale_bf16x2(a[2], f1.x, f1.y);
-          a[3] = scale_bf16x2(a[3], f1.x, f1.y);
+        for (int e = 0; e < 4; ++e) {
+          const int t = gr + (e >> 1) * 8, u = nt * 8 + gc + (e & 1);
+          const int rt = 16 * Iv + t, ru = 16 * Iv + u;
+          if (u < t) at[nt][e] = 0.f;
+          else if (slow) at[nt][e] = ru < rows ? diag_at_entry(qc, kc, gch, rows, rt, ru) : 0.f;
         }
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(smem_u32(&sm.qf[(16 * J + (lane & 7) + ((lane >> 4) << 3)) * KP + kk * 16 +
-                                ((lane >> 3) & 1) * 8]),
+    }
+    const uint32_t pa[4] = {pack_bf16(at[0][0], at[0][1]), pack_bf16(at[0][2], at[0][3]),
+                            pack_bf16(at[1][0], at[1][1]), pack_bf16(at[1][2], at[1][3])};
+#pragma unroll
+    for (int ntp = 0; ntp < 4; ++ntp) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(smem_u32(&sm.dO[(16 * J + (lane & 7) + ((lane >> 3) & 1) * 8) * VP + 64 * role + ntp * 16 +
+                                (lane >> 4) * 8]),
                 b0, b1, b2, b3);
-        mma_bf16(at[0], a, b0, b1);
-        mma_bf16(at[1], a, b2, b3);
-      }
-      if (J == Iv) {
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int t = gr + (e >> 1) * 8, u = nt * 8 + gc + (e & 1);
-            const int rt = 16 * Iv + t, ru = 16 * Iv + u;
-            if (u < t) at[nt][e] = 0.f;
-            else if (slow) at[nt][e] = ru < rows ? diag_at_entry(sm.q[st], sm.k[st], gch, rows, rt, ru) : 0.f;
-          }
-      }
-      const uint32_t pa[4] = {pack_bf16(at[0][0], at[0][1]), pack_bf16(at[0][2], at[0][3]),
-                              pack_bf16(at[1][0], at[1][1]), pack_bf16(at[1][2], at[1][3])};
-#pragma unroll
-      for (int ntp = 0; ntp < 4; ++ntp) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(smem_u32(&sm.dO[st][(16 * J + (lane & 7) + ((lane >> 3) & 1) * 8) * VP + 64 * role +
-                                      ntp * 16 + (lane >> 4) * 8]),
-                  b0, b1, b2, b3);
-        mma_bf16(dvh[2 * ntp], pa, b0, b1);
-        mma_bf16(dvh[2 * ntp + 1], pa, b2, b3);
-      }
-    }
-
-    // ---- carried gradient: G = diag(e^{b_l}) G + (q e^{b})^T dO --------------
-    {
-      const float d0 = sm.ec[16 * mt + gr], d1 = sm.ec[16 * mt + gr + 8];
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        G[nt][0] *= d0;
-        G[nt][1] *= d0;
-        G[nt][2] *= d1;
-        G[nt][3] *= d1;
-      }
-#pragma unroll
-      for (int kk = 0; kk < C / 16; ++kk) {
-        uint32_t a[4];
-        ldsm_x4_t(smem_u32(&sm.qi[(16 * kk + (lane & 7) + ((lane >> 4) << 3)) * KP + 16 * mt +
-                                  ((lane >> 3) & 1) * 8]),
-                  a[0], a[1], a[2], a[3]);
-#pragma unroll
-        for (int ntp = 0; ntp < 4; ++ntp) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(smem_u32(&sm.dO[st][(16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8) * VP + 64 * gnh +
-                                        ntp * 16 + (lane >> 4) * 8]),
-                    b0, b1, b2, b3);
-          mma_bf16(G[2 * ntp], a, b0, b1);
-          mma_bf16(G[2 * ntp + 1], a, b2, b3);
-        }
-      }
-    }
-    // ---- <G_new, S_prev> per key dim: dg at the chunk's first row -----------
-    {
-      float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        const int j = 64 * gnh + nt * 8 + gc;
-        const float2 s0 = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.sp[swz(16 * mt + gr, j)]));
-        const float2 s1 = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.sp[swz(16 * mt + gr + 8, j)]));
-        a0 += G[nt][0] * s0.x + G[nt][1] * s0.y;
-        a1 += G[nt][2] * s1.x + G[nt][3] * s1.y;
-      }
-      a0 += __shfl_xor_sync(0xffffffffu, a0, 1);
-      a0 += __shfl_xor_sync(0xffffffffu, a0, 2);
-      a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
-      a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
-      if ((lane & 3) == 0) {
-        sm.gsp[gnh][16 * mt + gr] = a0;
-        sm.gsp[gnh][16 * mt + gr + 8] = a1;
-      }
-    }
-    __syncthreads();  // q*dq staged; every reader of sp, g16 and the operands is done
-    if (c > 0) issue_sp(c - 1);
-    write_g16();
-    if (role == 1) {
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int t = 16 * I + gr + 8 * hh, il = nt * 8 + gc;
-          float2* r = reinterpret_cast<float2*>(&sm.red[rsw(t, il)]);
-          const float2 x = *r;
-          *r = make_float2(x.x - kdk[nt][2 * hh], x.y - kdk[nt][2 * hh + 1]);
-        }
-    }
-    __syncthreads();
-
-    // ---- dg: exact seed at the chunk's first row, then a running sum inside --
-    {
-      const int col = tid & 63, qq = tid >> 6;
-      float loc[SB];
-      float run = 0.f;
-#pragma unroll
-      for (int r = 0; r < SB; ++r) {  // exclusive prefix of q*dq - k*dk
-        loc[r] = run;
-        run += sm.red[rsw(16 * qq + r, col)];
-      }
-      sm.tot[qq][col] = run;
-      __syncthreads();
-      float base = sm.gsp[0][col] + sm.gsp[1][col];
-#pragma unroll
-      for (int q2 = 0; q2 < NSB; ++q2)
-        if (q2 < qq) base -= sm.tot[q2][col];
-#pragma unroll
-      for (int r = 0; r < SB; ++r) {
-        const int t = c0 + 16 * qq + r;
-        if (t < T) p.dg[tk + (size_t)t * DK + i0 + col] = base - loc[r];
-      }
-    }
-
-    // ---- dv: exchange the peer's 64 columns through distributed smem --------
-    cluster.sync();  // both CTAs are done with red
-    if (role != half) {  // these warps hold the peer's value columns
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int t = 16 * Iv + gr + 8 * hh, cl = nt * 8 + gc;
-          *reinterpret_cast<float2*>(&peer_red[rsw(t, cl)]) = make_float2(dvh[nt][2 * hh], dvh[nt][2 * hh + 1]);
-        }
-    }
-    cluster.sync();  // the peer's share has landed in red
-    if (role == half) {
-      const int mcol = 64 * half;
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int t = 16 * Iv + gr + 8 * hh, cl = nt * 8 + gc;
-          if (c0 + t >= T) continue;
-          const float2 pr = *reinterpret_cast<const float2*>(&sm.red[rsw(t, cl)]);
-          float y0 = dvh[nt][2 * hh] + pr.x, y1 = dvh[nt][2 * hh + 1] + pr.y;
-          const size_t off = tv + (size_t)(c0 + t) * DV + mcol + cl;
-          if (p.add_dv) {
-            const float2 a = *reinterpret_cast<const float2*>(&p.add_dv[off]);
-            y0 += a.x;
-            y1 += a.y;
-          } else if (p.add_in_place) {
-            const float2 a = unpack_bf16(prev[nt][hh]);
-            y0 += a.x;
-            y1 += a.y;
-          }
-          *reinterpret_cast<uint32_t*>(&((bf16*)p.dv)[off]) = pack_bf16(y0, y1);
-        }
+      mma_bf16(dvh[2 * ntp], pa, b0, b1);
+      mma_bf16(dvh[2 * ntp + 1], pa, b2, b3);
     }
   }
-  // dh0 = G carried to before token 0
-  if (p.dh0) {
+  // the gate gradient at the chunk's first row, from the reverse scan (loaded
+  // here so that the load overlaps the cluster barrier)
+  const float dg_first = p.gsp[((size_t)bh * nchunks + c) * DK + i0 + (tid & 63)];
+  cluster.sync();  // both CTAs: staging complete, qf / kf no longer read
+
+  // ---- dv: the peer's 64 columns go to its exchange tile -------------------
+  if (role != half) {
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
-        const int ii = i0 + 16 * mt + gr + 8 * hh, j = 64 * gnh + nt * 8 + gc;
-        *reinterpret_cast<float2*>(&p.dh0[((size_t)bh * DK + ii) * DV + j]) =
-            make_float2(G[nt][2 * hh], G[nt][2 * hh + 1]);
+        const int t = 16 * Iv + gr + 8 * hh, cl = nt * 8 + gc;
+        *reinterpret_cast<float2*>(&peer_xch[rsw(t, cl)]) = make_float2(dvh[nt][2 * hh], dvh[nt][2 * hh + 1]);
       }
   }
-  cluster.sync();  // keep this CTA's shared memory alive until the peer is done with it
+  // ---- dg: the scan's value at the chunk's first row, then a running sum ---
+  {
+    const int col = tid & 63, qq = tid >> 6;
+    float loc[SB];
+    float run = 0.f;
+#pragma unroll
+    for (int r = 0; r < SB; ++r) {  // exclusive prefix of q*dq - k*dk
+      loc[r] = run;
+      run += stq[rsw(16 * qq + r, col)] - stk[rsw(16 * qq + r, col)];
+    }
+    sm.tot[qq][col] = run;
+    __syncthreads();
+    float base = dg_first;
+#pragma unroll
+    for (int q2 = 0; q2 < NSB; ++q2)
+      if (q2 < qq) base -= sm.tot[q2][col];
+#pragma unroll
+    for (int r = 0; r < SB; ++r) {
+      const int t = 16 * qq + r;
+      if (t < rows) p.dg[tk + (size_t)(c0 + t) * DK + i0 + col] = base - loc[r];
+    }
+  }
+  if (role == half && p.add_in_place && !p.add_dv) {  // loads ahead of the stores below
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int t = 16 * Iv + gr + 8 * hh, cl = nt * 8 + gc;
+        const uint32_t a = t < rows ? *reinterpret_cast<const uint32_t*>(
+                                          &((const bf16*)p.dv)[tv + (size_t)(c0 + t) * DV + 64 * half + cl])
+                                    : 0u;
+        const float2 f = unpack_bf16(a);
+        dvh[nt][2 * hh] += f.x;
+        dvh[nt][2 * hh + 1] += f.y;
+      }
+  }
+  cluster.sync();  // the peer's share has landed
+  if (role == half) {
+    const int mcol = 64 * half;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int t = 16 * Iv + gr + 8 * hh, cl = nt * 8 + gc;
+        if (t >= rows) continue;
+        const float2 pr = *reinterpret_cast<const float2*>(&xch[rsw(t, cl)]);
+        float y0 = dvh[nt][2 * hh] + pr.x, y1 = dvh[nt][2 * hh + 1] + pr.y;
+        const size_t off = tv + (size_t)(c0 + t) * DV + mcol + cl;
+        if (p.add_dv) {
+          const float2 a = *reinterpret_cast<const float2*>(&p.add_dv[off]);
+          y0 += a.x;
+          y1 += a.y;
+        }
+        *reinterpret_cast<uint32_t*>(&((bf16*)p.dv)[off]) = pack_bf16(y0, y1);
+      }
+  }
 }
 
 }  // namespace
 
 bool gla_bwd_mma_supported(int dk, int dv, bool bf16) { return bf16 && dk == DK && dv == DV; }
 
-cudaError_t launch_gla_bwd_mma(const GlaBwdParams& p, cudaStream_t s) {
-  if (p.B * p.H == 0) return cudaSuccess;
-  const size_t bytes = sizeof(BwdSmem);
-  cudaError_t e = cudaFuncSetAttribute(gla_bwd_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+
+cudaError_t launch_gla_bwd_chunks(const GlaBwdParams& p, cudaStream_t s) {
+  const int nchunks = (p.T + C - 1) / C;
+  if (p.B * p.H == 0 || nchunks == 0) return cudaSuccess;
+  if (2 * (size_t)nchunks * p.B * p.H > 0x7fffffffu) return cudaErrorInvalidConfiguration;
+  const size_t bytes = sizeof(ChunkSmem);
+  cudaError_t e = cudaFuncSetAttribute(gla_bwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)bytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(2, p.B * p.H);
   {
-    ScopedTiming tm("gla_bwd_mma", s);
-    gla_bwd_mma_kernel<<<grid, NT, bytes, s>>>(p);
+    ScopedTiming tm("gla_bwd_chunks", s);
+    gla_bwd_chunk_kernel<<<(unsigned)(2 * (size_t)nchunks * p.B * p.H), NT, bytes, s>>>(p);
   }
   return cudaGetLastError();
 }

@@ -234,7 +234,23 @@ struct DeltaSmem {
 };
 static_assert(sizeof(DeltaSmem) <= 115712, "two delta CTAs must fit one SM");
 
-__global__ void __launch_bounds__(NT, 2) gla_delta_kernel(GlaFwdParams p) {
+// One chunk's increment of a carried [dk][dv] matrix, X^T Y over the chunk
+// with X the key-side or query-side operand scaled by its in-chunk decay:
+//   forward (key side):   dS_c = (k e^{b_l - b})^T v,   S_{c+1} = diag(E_c) S_c + dS_c
+//   backward (query side): dG_c = (q e^{b})^T dO,       G_{c-1} = diag(E_c) G_c + dG_c
+// with b the running log-gate from the chunk's start (inclusive) and E_c =
+// e^{b_l} per key dim.  Every factor is a product of per-row gates, so <= 1.
+struct DeltaArgs {
+  const bf16* x;   // k or q  [BH][T][DK]
+  const bf16* y;   // v or dO [BH][T][DV]
+  const float* g;  // [BH][T][DK]
+  bf16* delta;     // [BH][nchunks][DK][DV]
+  float* decay;    // [BH][nchunks][DK]
+  int T;
+};
+
+template <bool QSIDE>
+__global__ void __launch_bounds__(NT, 2) gla_delta_kernel(DeltaArgs p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   DeltaSmem& sm = *reinterpret_cast<DeltaSmem*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -242,8 +258,8 @@ __global__ void __launch_bounds__(NT, 2) gla_delta_kernel(GlaFwdParams p) {
   const int c = blockIdx.x, bh = blockIdx.y;
   const int T = p.T, nchunks = gridDim.x;
   const int c0 = c * C, rows = min(C, T - c0);
-  const bf16* k = (const bf16*)p.k + ((size_t)bh * T + c0) * DK;
-  const bf16* v = (const bf16*)p.v + ((size_t)bh * T + c0) * DV;
+  const bf16* k = p.x + ((size_t)bh * T + c0) * DK;
+  const bf16* v = p.y + ((size_t)bh * T + c0) * DV;
   const float* g = p.g + ((size_t)bh * T + c0) * DK;
   for (int x = tid; x < C * DK / 8; x += NT) {
     const int r = x / (DK / 8), cc = x % (DK / 8);
@@ -260,27 +276,31 @@ __global__ void __launch_bounds__(NT, 2) gla_delta_kernel(GlaFwdParams p) {
   cp_async_wait<0>();
   __syncthreads();
   // prep: thread -> (sub-block K, key dims i2, i2+1); rows past the end have
-  // g = 0 (no decay) and k = 0
+  // g = 0 (no decay) and x = 0.  fac[r]: the in-sub-block part of the row's
+  // factor (key side: gates after the row; query side: gates up to it)
   const int K = tid >> 6, i2 = (tid & 63) * 2, r0 = K * SB;
-  float2 kfac[SB];
+  float2 fac[SB];
   {
     float2 run = make_float2(1.f, 1.f);
 #pragma unroll
-    for (int r = SB - 1; r >= 0; --r) {
-      kfac[r] = run;
+    for (int rr = 0; rr < SB; ++rr) {
+      const int r = QSIDE ? rr : SB - 1 - rr;
+      if (!QSIDE) fac[r] = run;
       const float2 gg = *reinterpret_cast<const float2*>(&sm.g[(r0 + r) * DK + i2]);
       run.x *= __expf(gg.x);
       run.y *= __expf(gg.y);
+      if (QSIDE) fac[r] = run;
     }
     *reinterpret_cast<float2*>(&sm.dec[K][i2]) = run;
   }
   __syncthreads();
   {
+    // f: the other sub-blocks' part (key side: later ones; query side: earlier)
     float2 f = make_float2(1.f, 1.f), e = make_float2(1.f, 1.f);
 #pragma unroll
     for (int J = 0; J < NSB; ++J) {
       const float2 d = *reinterpret_cast<const float2*>(&sm.dec[J][i2]);
-      if (J > K) {
+      if (QSIDE ? (J < K) : (J > K)) {
         f.x *= d.x;
         f.y *= d.y;
       }
@@ -293,11 +313,11 @@ __global__ void __launch_bounds__(NT, 2) gla_delta_kernel(GlaFwdParams p) {
     for (int r = 0; r < SB; ++r) {
       const float2 kv = unpack_bf16(*reinterpret_cast<const uint32_t*>(&sm.k[(r0 + r) * QKP + i2]));
       *reinterpret_cast<uint32_t*>(&sm.ks[(r0 + r) * QKP + i2]) =
-          pack_bf16(kv.x * kfac[r].x * f.x, kv.y * kfac[r].y * f.y);
+          pack_bf16(kv.x * fac[r].x * f.x, kv.y * fac[r].y * f.y);
     }
   }
   __syncthreads();
-  // dS rows 16w .. 16w+15, all 128 value columns
+  // increment rows 16w .. 16w+15, all 128 value columns
   float acc[DV / 8][4];
 #pragma unroll
   for (int nt = 0; nt < DV / 8; ++nt)
@@ -318,7 +338,7 @@ __global__ void __launch_bounds__(NT, 2) gla_delta_kernel(GlaFwdParams p) {
       mma_bf16(acc[2 * ntp + 1], a, b2, b3);
     }
   }
-  bf16* dst = (bf16*)p.delta16 + ((size_t)bh * nchunks + c) * DK * DV;
+  bf16* dst = p.delta + ((size_t)bh * nchunks + c) * DK * DV;
 #pragma unroll
   for (int nt = 0; nt < DV / 8; ++nt)
 #pragma unroll
@@ -328,42 +348,65 @@ __global__ void __launch_bounds__(NT, 2) gla_delta_kernel(GlaFwdParams p) {
     }
 }
 
-// thread -> (batch-head, key dim i, 8 value columns); walks the chunks
+// Elementwise scan over the chunks; thread -> (batch-head, key dim i, 8 value
+// columns).  Forward: out[c] = S before chunk c, S <- E_c S + dS_c, fin = S
+// after the last chunk.  Reverse: out[c] = G entering chunk c from the later
+// chunks, G <- E_c G + dG_c, gsp[c][i] = <G, S_prev[c]> over the value
+// columns with the updated G (the gate gradient at the chunk's first row),
+// fin = G before token 0.
+struct ScanArgs {
+  const bf16* delta;   // [BH][nchunks][DK][DV]
+  const float* decay;  // [BH][nchunks][DK]
+  const float* init;   // nullable [BH][DK][DV]
+  bf16* out;           // [BH][nchunks][DK][DV]
+  float* fin;          // nullable [BH][DK][DV]
+  const bf16* sprev;   // reverse only: the forward states [BH][nchunks][DK][DV]
+  float* gsp;          // reverse only: [BH][nchunks][DK]
+  int BH, nchunks;
+};
 constexpr int SCAN_NT = 128;
 constexpr int SCAN_U = 4;  // chunks whose loads are in flight together
 
-__global__ void __launch_bounds__(SCAN_NT) gla_scan_kernel(GlaFwdParams p, int nchunks) {
+template <bool REV>
+__global__ void __launch_bounds__(SCAN_NT) gla_scan_kernel(ScanArgs p) {
   const size_t id = (size_t)blockIdx.x * SCAN_NT + threadIdx.x;
   const size_t per_bh = (size_t)DK * (DV / 8);
-  if (id >= (size_t)p.B * p.H * per_bh) return;
+  // whole warps only: the thread count is a multiple of DK * DV / 8
+  if (id >= (size_t)p.BH * per_bh) return;
+  const int nchunks = p.nchunks;
   const size_t bh = id / per_bh;
   const int i = (int)((id / (DV / 8)) % DK), j8 = (int)(id % (DV / 8)) * 8;
   float s[8];
-  if (p.h0) {
-    const float4* hp = reinterpret_cast<const float4*>(p.h0 + (bh * DK + i) * DV + j8);
+  if (p.init) {
+    const float4* hp = reinterpret_cast<const float4*>(p.init + (bh * DK + i) * DV + j8);
     const float4 a = hp[0], b = hp[1];
     s[0] = a.x; s[1] = a.y; s[2] = a.z; s[3] = a.w; s[4] = b.x; s[5] = b.y; s[6] = b.z; s[7] = b.w;
   } else {
 #pragma unroll
     for (int x = 0; x < 8; ++x) s[x] = 0.f;
   }
-  const size_t stride = (size_t)DK * DV;  // one chunk's state
-  const bf16* dl = (const bf16*)p.delta16 + bh * nchunks * stride + (size_t)i * DV + j8;
-  bf16* out = (bf16*)p.states16 + bh * nchunks * stride + (size_t)i * DV + j8;
+  const size_t stride = (size_t)DK * DV;  // one chunk's matrix
+  const size_t base = bh * nchunks * stride + (size_t)i * DV + j8;
+  const bf16* dl = p.delta + base;
+  bf16* out = p.out + base;
   const float* ec = p.decay + bh * nchunks * DK + i;
-  for (int c0 = 0; c0 < nchunks; c0 += SCAN_U) {
-    uint4 d[SCAN_U];
+  for (int it0 = 0; it0 < nchunks; it0 += SCAN_U) {
+    uint4 d[SCAN_U], sv[SCAN_U];
     float e[SCAN_U];
 #pragma unroll
     for (int u = 0; u < SCAN_U; ++u) {
-      const int c = c0 + u;
-      d[u] = c < nchunks ? __ldcs(reinterpret_cast<const uint4*>(dl + c * stride)) : make_uint4(0, 0, 0, 0);
-      e[u] = c < nchunks ? __ldcs(ec + (size_t)c * DK) : 1.f;
+      const int it = it0 + u;
+      const int c = REV ? nchunks - 1 - it : it;
+      const bool ok = it < nchunks;
+      d[u] = ok ? __ldcs(reinterpret_cast<const uint4*>(dl + c * stride)) : make_uint4(0, 0, 0, 0);
+      e[u] = ok ? __ldcs(ec + (size_t)c * DK) : 1.f;
+      if (REV) sv[u] = ok ? __ldcs(reinterpret_cast<const uint4*>(p.sprev + base + c * stride)) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int u = 0; u < SCAN_U; ++u) {
-      const int c = c0 + u;
-      if (c >= nchunks) break;
+      const int it = it0 + u;
+      if (it >= nchunks) break;
+      const int c = REV ? nchunks - 1 - it : it;
       *reinterpret_cast<uint4*>(out + c * stride) =
           make_uint4(pack_bf16(s[0], s[1]), pack_bf16(s[2], s[3]), pack_bf16(s[4], s[5]), pack_bf16(s[6], s[7]));
       const uint32_t dw[4] = {d[u].x, d[u].y, d[u].z, d[u].w};
@@ -373,13 +416,49 @@ __global__ void __launch_bounds__(SCAN_NT) gla_scan_kernel(GlaFwdParams p, int n
         s[2 * x] = fmaf(e[u], s[2 * x], f.x);
         s[2 * x + 1] = fmaf(e[u], s[2 * x + 1], f.y);
       }
+      if (REV) {
+        const uint32_t pw[4] = {sv[u].x, sv[u].y, sv[u].z, sv[u].w};
+        float dot = 0.f;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const float2 f = unpack_bf16(pw[x]);
+          dot = fmaf(s[2 * x], f.x, fmaf(s[2 * x + 1], f.y, dot));
+        }
+        // the 16 threads of key dim i are 16 consecutive lanes
+#pragma unroll
+        for (int m = 8; m >= 1; m >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, m);
+        if ((threadIdx.x & 15) == 0) p.gsp[(bh * nchunks + c) * DK + i] = dot;
+      }
     }
   }
-  if (p.hT) {
-    float4* hp = reinterpret_cast<float4*>(p.hT + (bh * DK + i) * DV + j8);
+  if (p.fin) {
+    float4* hp = reinterpret_cast<float4*>(p.fin + (bh * DK + i) * DV + j8);
     hp[0] = make_float4(s[0], s[1], s[2], s[3]);
     hp[1] = make_float4(s[4], s[5], s[6], s[7]);
   }
+}
+
+template <bool QSIDE>
+cudaError_t run_delta(const DeltaArgs& a, int nchunks, int BH, const char* name, cudaStream_t s) {
+  const size_t bytes = sizeof(DeltaSmem);
+  cudaError_t e = cudaFuncSetAttribute(gla_delta_kernel<QSIDE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)bytes);
+  if (e != cudaSuccess) return e;
+  {
+    ScopedTiming tm(name, s);
+    gla_delta_kernel<QSIDE><<<dim3(nchunks, BH), NT, bytes, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+template <bool REV>
+cudaError_t run_scan(const ScanArgs& a, const char* name, cudaStream_t s) {
+  const size_t threads = (size_t)a.BH * DK * (DV / 8);
+  {
+    ScopedTiming tm(name, s);
+    gla_scan_kernel<REV><<<(unsigned)((threads + SCAN_NT - 1) / SCAN_NT), SCAN_NT, 0, s>>>(a);
+  }
+  return cudaGetLastError();
 }
 
 // ===========================================================================
@@ -692,22 +771,12 @@ cudaError_t launch_gla_states(const GlaFwdParams& p, cudaStream_t s) {
   if (p.B * p.H == 0) return cudaSuccess;
   const int nchunks = (p.T + C - 1) / C;
   if (p.delta16 && p.decay && nchunks >= kScanMinChunks) {
-    const size_t bytes = sizeof(DeltaSmem);
-    cudaError_t e = cudaFuncSetAttribute(gla_delta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)bytes);
+    DeltaArgs da{(const bf16*)p.k, (const bf16*)p.v, p.g, (bf16*)p.delta16, p.decay, p.T};
+    cudaError_t e = run_delta<false>(da, nchunks, p.B * p.H, "gla_delta_mma", s);
     if (e != cudaSuccess) return e;
-    {
-      ScopedTiming tm("gla_delta_mma", s);
-      gla_delta_kernel<<<dim3(nchunks, p.B * p.H), NT, bytes, s>>>(p);
-    }
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    const size_t threads = (size_t)p.B * p.H * DK * (DV / 8);
-    {
-      ScopedTiming tm("gla_scan", s);
-      gla_scan_kernel<<<(unsigned)((threads + SCAN_NT - 1) / SCAN_NT), SCAN_NT, 0, s>>>(p, nchunks);
-    }
-    return cudaGetLastError();
+    ScanArgs sa{(const bf16*)p.delta16, p.decay, p.h0, (bf16*)p.states16, p.hT, nullptr, nullptr,
+                p.B * p.H, nchunks};
+    return run_scan<false>(sa, "gla_scan", s);
   }
   const size_t bytes = sizeof(StateSmem);
   cudaError_t e = cudaFuncSetAttribute(gla_states_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -721,6 +790,20 @@ cudaError_t launch_gla_states(const GlaFwdParams& p, cudaStream_t s) {
 }
 
 size_t gla_out_loss_parts(int B, int H, int T) { return (size_t)B * H * ((T + C - 1) / C); }
+
+cudaError_t launch_gla_bwd_scan(const GlaBwdScanParams& p, cudaStream_t s) {
+  const int nchunks = (p.T + C - 1) / C;
+  const int BH = p.B * p.H;
+  if (BH == 0) return cudaSuccess;
+  if (nchunks > 0) {
+    DeltaArgs da{(const bf16*)p.q, (const bf16*)p.dO, p.g, (bf16*)p.delta16, p.decay, p.T};
+    cudaError_t e = run_delta<true>(da, nchunks, BH, "gla_bwd_delta", s);
+    if (e != cudaSuccess) return e;
+  }
+  ScanArgs sa{(const bf16*)p.delta16, p.decay, p.dhT, (bf16*)p.gin16, p.dh0, (const bf16*)p.states16,
+              p.gsp, BH, nchunks};
+  return run_scan<true>(sa, "gla_bwd_scan", s);
+}
 
 cudaError_t launch_gla_out(const GlaFwdParams& p, cudaStream_t s) {
   const int nchunks = (p.T + C - 1) / C;

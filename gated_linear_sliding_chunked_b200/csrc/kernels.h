@@ -88,6 +88,8 @@ struct GlaBwdParams {
   float* dg;
   float* dh0;            // nullable
   int B, H, T, dkd, dvd;
+  const void* gin16;     // two-level tensor-core backward: launch_gla_bwd_scan's outputs
+  const float* gsp;
 };
 cudaError_t launch_gla_bwd_simt(const GlaBwdParams& p, bool bf16, cudaStream_t s);
 
@@ -100,6 +102,28 @@ cudaError_t launch_gla_states(const GlaFwdParams& p, cudaStream_t s);
 // whether launch_gla_states takes the two-level path (given delta16 / decay)
 bool gla_states_scan_wanted(int T);
 cudaError_t launch_gla_out(const GlaFwdParams& p, cudaStream_t s);
+
+// ---- gated backward, two-level (bf16, dk = dv = 128) ------------------------
+// launch_gla_bwd_scan: every chunk's dG_c = (q e^{b})^T dO and decay e^{b_l}
+// in parallel, then a reverse elementwise scan writing gin16[c] (the state
+// gradient entering chunk c from the later chunks, bf16), gsp[c][i] =
+// <G_new, S_prev>_i (the gate gradient at the chunk's first row) and dh0.
+// launch_gla_bwd_chunks then computes every chunk's dq, dk, dv, dg from
+// them, all chunks in parallel.
+struct GlaBwdScanParams {
+  const void* q;
+  const void* dO;
+  const float* g;
+  const void* states16;  // the forward's states before every 64-token chunk
+  const float* dhT;      // nullable
+  void* delta16;         // scratch [BH][nchunks][dk][dv] bf16
+  float* decay;          // scratch [BH][nchunks][dk]
+  void* gin16;           // [BH][nchunks][dk][dv] bf16
+  float* gsp;            // [BH][nchunks][dk]
+  float* dh0;            // nullable
+  int B, H, T;
+};
+cudaError_t launch_gla_bwd_scan(const GlaBwdScanParams& p, cudaStream_t s);
 // partial sums the fused loss epilogue writes: one per 64-token chunk and head
 size_t gla_out_loss_parts(int B, int H, int T);
 
@@ -116,9 +140,10 @@ cudaError_t launch_loss_reduce(const float* part, size_t nparts, double inv_n, f
                                cudaStream_t s);
 
 // ---- gated branch, tensor-core backward (bf16 I/O, dk = dv = 128) --------
-// Needs states16 and hT from the tensor-core forward run as a state pass.
+// Needs states16 (the forward's states before every 64-token chunk) and
+// launch_gla_bwd_scan's gin16 / gsp; all chunks in parallel.
 bool gla_bwd_mma_supported(int dk, int dv, bool bf16);
-cudaError_t launch_gla_bwd_mma(const GlaBwdParams& p, cudaStream_t s);
+cudaError_t launch_gla_bwd_chunks(const GlaBwdParams& p, cudaStream_t s);
 
 // ---- window + meta softmax, SIMT path ------------------------------------
 struct SwaFwdParams {

@@ -156,9 +156,10 @@ size_t states16_count(const lz_dims* d) {
   return (size_t)d->B * d->H * n64 * d->dk * d->dv;
 }
 // the two-level state pass's scratch, carved right after the states
-ScanWs carve_scan(Carver& c, const lz_dims* d) {
+// (always carved for the two-level backward, whose first step uses it too)
+ScanWs carve_scan(Carver& c, const lz_dims* d, bool always = false) {
   ScanWs w;
-  if (!lz::gla_states_scan_wanted(d->T)) return w;
+  if (!always && !lz::gla_states_scan_wanted(d->T)) return w;
   const size_t n64 = (size_t)((d->T + lz::gla_fwd_mma_chunk() - 1) / lz::gla_fwd_mma_chunk());
   w.delta16 = c.take<uint16_t>(states16_count(d));
   w.decay = c.take<float>((size_t)d->B * d->H * n64 * d->dk);
@@ -198,13 +199,18 @@ struct GlaBwdWs {
   void* states16;
   float* hT;
   ScanWs scan;
+  void* gin16;  // two-level backward: state gradient entering every chunk (bf16)
+  float* gsp;   // and <G_new, S_prev> per chunk and key dim
 };
 GlaBwdWs carve_gla_bwd(Carver& c, const lz_dims* d) {
   GlaBwdWs w{};
   const size_t bh = (size_t)d->B * d->H;
   if (bwd_uses_mma(d)) {
     w.states16 = c.take<uint16_t>(states16_count(d));  // bf16
-    w.scan = carve_scan(c, d);
+    w.scan = carve_scan(c, d, true);
+    w.gin16 = c.take<uint16_t>(states16_count(d));
+    const size_t n64 = (size_t)((d->T + lz::gla_fwd_mma_chunk() - 1) / lz::gla_fwd_mma_chunk());
+    w.gsp = c.take<float>(bh * n64 * d->dk);
   } else {
     w.states = c.take<float>(bh * nchunks16(d) * d->dk * d->dv);
   }
@@ -512,7 +518,18 @@ static cudaError_t gla_bwd_launch(const lz_dims* d, const void* q, const void* k
   p.add_in_place = add_in_place;
   p.dq = dq; p.dk = dk; p.dv = dv; p.dg = dg; p.dh0 = dh0;
   p.B = d->B; p.H = d->H; p.T = d->T; p.dkd = d->dk; p.dvd = d->dv;
-  return mma ? lz::launch_gla_bwd_mma(p, s) : lz::launch_gla_bwd_simt(p, bf, s);
+  if (!mma) return lz::launch_gla_bwd_simt(p, bf, s);
+  // two-level: reverse scan of the state gradient, then every chunk at once
+  lz::GlaBwdScanParams sp{};
+  sp.q = q; sp.dO = dO; sp.g = g; sp.states16 = states16; sp.dhT = dhT;
+  sp.delta16 = w.scan.delta16; sp.decay = w.scan.decay;
+  sp.gin16 = w.gin16; sp.gsp = w.gsp; sp.dh0 = dh0;
+  sp.B = d->B; sp.H = d->H; sp.T = d->T;
+  cudaError_t e = lz::launch_gla_bwd_scan(sp, s);
+  if (e != cudaSuccess) return e;
+  p.gin16 = w.gin16;
+  p.gsp = w.gsp;
+  return lz::launch_gla_bwd_chunks(p, s);
 }
 
 lz_status lz_gla_bwd(const lz_dims* d, const void* q, const void* k, const void* v,
