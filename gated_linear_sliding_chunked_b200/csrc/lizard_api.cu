@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <string>
+#include <unordered_map>
 
 #include "../../include/lizard.h"
 #include "kernels.h"
@@ -487,13 +488,18 @@ lz_status lz_hybrid_fwd_mse(const lz_dims* d, const void* q, const void* k, cons
                          chunk_states, &la, ws, ws_bytes_, stream);
 }
 
-static cudaError_t gla_bwd_launch(const lz_dims* d, const void* q, const void* k, const void* v,
+// The gated backward in two phases: the first (state pass when the forward's
+// chunk states are not given; on the tensor-core path also the reverse scan of
+// the state gradient) depends only on the inputs, so lz_hybrid_bwd runs it on
+// a side stream while the window backward runs; the second computes the
+// gradients (and adds them in place to the window branch's).
+static cudaError_t gla_bwd_phase1(const lz_dims* d, const void* q, const void* k, const void* v,
                                   const float* g, const float* h0, const void* dO,
                                   const float* dhT, const void* saved_states,
                                   const float* saved_hT, void* dq, void* dk, void* dv, float* dg,
                                   float* dh0, const GlaBwdWs& w, const float* add_dq,
                                   const float* add_dk, const float* add_dv, bool add_in_place,
-                                  cudaStream_t s) {
+                                  lz::GlaBwdParams& p, cudaStream_t s) {
   const bool bf = d->io == LZ_BF16;
   const bool mma = bwd_uses_mma(d);
   const void* states16 = w.states16;
@@ -511,25 +517,73 @@ static cudaError_t gla_bwd_launch(const lz_dims* d, const void* q, const void* k
     cudaError_t e = mma ? lz::launch_gla_states(fp, s) : lz::launch_gla_fwd_simt(fp, bf, s);
     if (e != cudaSuccess) return e;
   }
-  lz::GlaBwdParams p{};
+  p = lz::GlaBwdParams{};
   p.q = q; p.k = k; p.v = v; p.g = g; p.dO = dO; p.dhT = dhT;
   p.states = w.states; p.states16 = states16; p.hT = hT;
   p.add_dq = add_dq; p.add_dk = add_dk; p.add_dv = add_dv;
   p.add_in_place = add_in_place;
   p.dq = dq; p.dk = dk; p.dv = dv; p.dg = dg; p.dh0 = dh0;
   p.B = d->B; p.H = d->H; p.T = d->T; p.dkd = d->dk; p.dvd = d->dv;
-  if (!mma) return lz::launch_gla_bwd_simt(p, bf, s);
-  // two-level: reverse scan of the state gradient, then every chunk at once
+  if (!mma) return cudaSuccess;
+  // two-level: reverse scan of the state gradient
   lz::GlaBwdScanParams sp{};
   sp.q = q; sp.dO = dO; sp.g = g; sp.states16 = states16; sp.dhT = dhT;
   sp.delta16 = w.scan.delta16; sp.decay = w.scan.decay;
   sp.gin16 = w.gin16; sp.gsp = w.gsp; sp.dh0 = dh0;
   sp.B = d->B; sp.H = d->H; sp.T = d->T;
-  cudaError_t e = lz::launch_gla_bwd_scan(sp, s);
-  if (e != cudaSuccess) return e;
   p.gin16 = w.gin16;
   p.gsp = w.gsp;
-  return lz::launch_gla_bwd_chunks(p, s);
+  return lz::launch_gla_bwd_scan(sp, s);
+}
+
+static cudaError_t gla_bwd_phase2(const lz_dims* d, const lz::GlaBwdParams& p, cudaStream_t s) {
+  if (!bwd_uses_mma(d)) return lz::launch_gla_bwd_simt(p, d->io == LZ_BF16, s);
+  return lz::launch_gla_bwd_chunks(p, s);  // every chunk at once
+}
+
+static cudaError_t gla_bwd_launch(const lz_dims* d, const void* q, const void* k, const void* v,
+                                  const float* g, const float* h0, const void* dO,
+                                  const float* dhT, const void* saved_states,
+                                  const float* saved_hT, void* dq, void* dk, void* dv, float* dg,
+                                  float* dh0, const GlaBwdWs& w, const float* add_dq,
+                                  const float* add_dk, const float* add_dv, bool add_in_place,
+                                  cudaStream_t s) {
+  lz::GlaBwdParams p;
+  cudaError_t e = gla_bwd_phase1(d, q, k, v, g, h0, dO, dhT, saved_states, saved_hT, dq, dk, dv, dg,
+                                 dh0, w, add_dq, add_dk, add_dv, add_in_place, p, s);
+  if (e != cudaSuccess) return e;
+  return gla_bwd_phase2(d, p, s);
+}
+
+// A high-priority stream and two events per (host thread, device), created on
+// first use and kept for the life of the process: lz_hybrid_bwd forks the
+// gated backward's first phase onto it and joins it back before the second.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t join = nullptr;
+};
+
+static cudaError_t side_stream(SideStream** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  thread_local std::unordered_map<int, SideStream> streams;
+  SideStream& ss = streams[dev];
+  if (!ss.stream) {
+    int lo = 0, hi = 0;
+    e = cudaDeviceGetStreamPriorityRange(&lo, &hi);
+    if (e != cudaSuccess) return e;
+    e = cudaStreamCreateWithPriority(&ss.stream, cudaStreamNonBlocking, hi);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      ss = SideStream{};
+      return e;
+    }
+  }
+  *out = &ss;
+  return cudaSuccess;
 }
 
 lz_status lz_gla_bwd(const lz_dims* d, const void* q, const void* k, const void* v,
@@ -609,11 +663,36 @@ lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const vo
   p.dq = dq; p.dk = dk; p.dv = dv;
   p.dq_f32 = w.dq; p.dk_f32 = w.dk; p.dv_f32 = w.dv;
   p.dmk = dmeta_k; p.dmv = dmeta_v; p.dalpha = dalpha;
-  cudaError_t e = swa_backward(p, d->io == LZ_BF16, s);
+  if (!mma || bht(d) == 0) {
+    cudaError_t e = swa_backward(p, d->io == LZ_BF16, s);
+    if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (window branch)");
+    return cuda_status(gla_bwd_launch(d, q, k, v, g, h0, dO, dhT, chunk_states, hT, dq, dk, dv,
+                                      dg, dh0, w.gla, w.dq, w.dk, w.dv, mma, s),
+                       "lz_hybrid_bwd (gated branch)");
+  }
+  // tensor-core path: the gated backward's first phase (it reads only the
+  // inputs and writes only its scratch and dh0) runs on the side stream while
+  // the window backward runs here; the second phase adds to the window
+  // branch's gradients, so it waits for both
+  SideStream* ss = nullptr;
+  cudaError_t e = side_stream(&ss);
+  if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (side stream)");
+  e = cudaEventRecord(ss->fork, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->fork, 0);
+  if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (fork)");
+  lz::GlaBwdParams gp;
+  e = gla_bwd_phase1(d, q, k, v, g, h0, dO, dhT, chunk_states, hT, dq, dk, dv, dg, dh0, w.gla,
+                     w.dq, w.dk, w.dv, mma, gp, ss->stream);
+  // the join is recorded even after a failed launch, so that the caller's
+  // stream never depends on an unrecorded event
+  const cudaError_t ej = cudaEventRecord(ss->join, ss->stream);
+  if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (gated branch, first phase)");
+  if (ej != cudaSuccess) return cuda_status(ej, "lz_hybrid_bwd (join)");
+  e = swa_backward(p, d->io == LZ_BF16, s);
+  const cudaError_t ew = cudaStreamWaitEvent(s, ss->join, 0);
   if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (window branch)");
-  return cuda_status(gla_bwd_launch(d, q, k, v, g, h0, dO, dhT, chunk_states, hT, dq, dk, dv,
-                                    dg, dh0, w.gla, w.dq, w.dk, w.dv, mma, s),
-                     "lz_hybrid_bwd (gated branch)");
+  if (ew != cudaSuccess) return cuda_status(ew, "lz_hybrid_bwd (join)");
+  return cuda_status(gla_bwd_phase2(d, gp, s), "lz_hybrid_bwd (gated branch)");
 }
 
 lz_status lz_decode_prefill(int Bd, int H, int T, int dk, int dv, int w, lz_dtype io,

@@ -18,8 +18,11 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  * - Every pointer is DEVICE memory owned by the caller.  The library never
- *   allocates, frees or synchronizes; every call is asynchronous on `stream`
- *   (a cudaStream_t passed as void*; NULL means the legacy default stream).
+ *   allocates device memory, frees or synchronizes; every call is
+ *   asynchronous on `stream` (a cudaStream_t passed as void*; NULL means the
+ *   legacy default stream).  The one resource it creates itself is a
+ *   high-priority side stream with two events per (host thread, device),
+ *   made on the first lz_hybrid_bwd call and kept: see lz_hybrid_bwd.
  * - Layouts are contiguous row-major:
  *     q, k, g, dq, dk, dg     [B, H, T, dk]
  *     v, o, o_swa, dO, dv     [B, H, T, dv]
@@ -200,7 +203,13 @@ lz_status lz_swa_meta_bwd_noalloc(const lz_dims* d, const void* q,
  * window branch alpha * dO.  lse from the forward; o_swa (nullable) the
  * forward's window output, used as in lz_swa_meta_bwd; chunk_states and hT
  * (nullable) the forward's, used as in lz_gla_bwd.  dalpha (nullable, one
- * fp32) receives sum over (b,h,t) of dO_t . o_swa_t. */
+ * fp32) receives sum over (b,h,t) of dO_t . o_swa_t.
+ * On the bf16, dk = dv = 128 path the part of the gated backward that reads
+ * only the inputs (the reverse scan of the state gradient) runs on the side
+ * stream, forked from `stream` by an event and joined back by another before
+ * the gradients are written, so it overlaps the window backward; to the
+ * caller the call is still ordered on `stream` alone (also under CUDA graph
+ * capture). */
 lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k,
                         const void* v, const float* g, const void* meta_k,
                         const void* meta_v, const float* h0, const float* lse,
