@@ -319,6 +319,76 @@ class Stage1Step(TrainStep):
                         self.nb)
 
 
+class E2EPipeline:
+    """The training step end to end through the C ABI with pinned host
+    buffers: every step copies its inputs host -> device and its outputs
+    device -> host.  Two sets of device buffers let the copies of one step
+    overlap the compute of its neighbours (inputs of step i+1 and outputs of
+    step i-1 move while step i computes; the two copy directions run on
+    their own streams), as a training loop that prefetches its next batch
+    does."""
+
+    def __init__(self, wl, xh, in_keys, step0, device):
+        self.xh, self.in_keys, self.device = xh, in_keys, device
+        self.steps = [step0, TrainStep(wl, {k: torch.empty_like(v, device=device)
+                                            for k, v in xh.items()}, device)]
+        self.xe = [{k: torch.empty_like(v, device=device) for k, v in xh.items()}
+                   for _ in range(2)]
+        self.outs_h = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in st.outputs()]
+                       for st in self.steps]
+        self.s_in = torch.cuda.Stream(device)
+        self.s_out = torch.cuda.Stream(device)
+        ev = lambda: [torch.cuda.Event() for _ in range(2)]
+        self.ev_in, self.ev_comp, self.ev_out = ev(), ev(), ev()
+        self.used = [False, False]
+
+    def _step(self, i):
+        b = i % 2
+        comp = torch.cuda.current_stream(self.device)
+        with torch.cuda.stream(self.s_in):
+            if self.used[b]:
+                self.s_in.wait_event(self.ev_comp[b])  # step i-2 is done reading xe[b]
+            for k in self.in_keys:
+                self.xe[b][k].copy_(self.xh[k], non_blocking=True)
+            self.ev_in[b].record(self.s_in)
+        comp.wait_event(self.ev_in[b])
+        if self.used[b]:
+            comp.wait_event(self.ev_out[b])  # step i-2's outputs have left the device
+        self.steps[b].run(self.xe[b])
+        self.ev_comp[b].record(comp)
+        with torch.cuda.stream(self.s_out):
+            self.s_out.wait_event(self.ev_comp[b])
+            for hbuf, dbuf in zip(self.outs_h[b], self.steps[b].outputs()):
+                hbuf.copy_(dbuf, non_blocking=True)
+            self.ev_out[b].record(self.s_out)
+        self.used[b] = True
+
+    def run(self, n):
+        for i in range(n):
+            self._step(i)
+        comp = torch.cuda.current_stream(self.device)
+        for b in range(2):
+            comp.wait_event(self.ev_out[b])
+
+    def timed(self, n):
+        """ms per step over n pipelined steps, from the first input copy to
+        the last output copy (events on the compute stream, which the copy
+        streams join at both ends)."""
+        barrier()
+        torch.cuda.synchronize(self.device)
+        comp = torch.cuda.current_stream(self.device)
+        a = torch.cuda.Event(enable_timing=True)
+        z = torch.cuda.Event(enable_timing=True)
+        a.record(comp)
+        self.s_in.wait_event(a)
+        self.s_out.wait_event(a)
+        self.run(n)
+        z.record(comp)
+        torch.cuda.synchronize(self.device)
+        barrier()
+        return a.elapsed_time(z) / n
+
+
 def time_region(fn, steps, device):
     """Device time of ``steps`` calls of fn (barrier + synchronize on both
     sides, CUDA events on the current stream); returns ms per step."""
@@ -397,11 +467,17 @@ def measure_fwd(wl, device, steps, warmup, peaks, seed, tcgen05_window=True):
     n = L.lz_workspace_bytes(dims, L.LZ_WS_HYBRID_FWD)
     ws = torch.empty(max(n, 1), dtype=torch.uint8, device=device)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    spans = []
 
     def fn():
         flush.zero_()  # 256 MB write: evicts L2 between iterations
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
         L.lz_hybrid_fwd(dims, x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], None,
                         o, None, None, None, None, ws, n)
+        b.record()
+        spans.append((a, b))
 
     prev = L.lz_prefer_tcgen05(tcgen05_window)
     for _ in range(warmup):
@@ -411,13 +487,21 @@ def measure_fwd(wl, device, steps, warmup, peaks, seed, tcgen05_window=True):
     L.lz_timing_enable(False)
     L.lz_prefer_tcgen05(prev)
     tab = kernel_table(L.lz_timing_read())
-    lib_ms = sum(t for (c, t) in tab.values()) / steps
-    dom, roof = roofline_for(tab, wl, peaks)
+    # the call's own span (after the flush): its gated state pass overlaps the
+    # window forward on the library's side stream, so kernel times do not add up
+    call_ms = sum(a.elapsed_time(b) for a, b in spans[-steps:]) / steps
+    by = algorithmic_bytes("hybrid_fwd", wl)
+    achieved = by / (call_ms * 1e-3) / 1e9
+    roof = {"kernel": "lz_hybrid_fwd (whole call)", "bound": "hbm", "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "algorithmic_bytes_per_call": by, "avg_ms": round(call_ms, 4),
+            "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs copy)"}
     del x, o, ws, flush
-    return {"workload": wl.name, "tokens_per_s": wl.B * wl.T / (lib_ms * 1e-3),
-            "ms_per_call": round(lib_ms, 4), "ms_per_iter_incl_l2_flush": round(ms, 4),
+    return {"workload": wl.name, "tokens_per_s": wl.B * wl.T / (call_ms * 1e-3),
+            "ms_per_call": round(call_ms, 4), "ms_per_iter_incl_l2_flush": round(ms, 4),
             "l2": "256 MB flush between iterations (not counted in ms_per_call)",
             "kernels": {k: [c // steps, round(t / c, 4)] for k, (c, t) in tab.items()},
+            "kernel_note": "per-launch event times; the state pass overlaps the window forward",
             "roofline": roof}
 
 
@@ -679,21 +763,12 @@ def main(argv=None):
     # ---- end to end through the C ABI with host buffers --------------------
     in_keys = ("q", "k", "v", "g", "meta_k", "meta_v", "dO")
     h2d = sum(xh[k].numel() * xh[k].element_size() for k in in_keys)
-    outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in step.outputs()]
-    d2h = sum(t.numel() * t.element_size() for t in outs_h)
-    xe = {k: torch.empty_like(v) for k, v in xd.items()}
-
-    def e2e_step():
-        for k in in_keys:
-            xe[k].copy_(xh[k], non_blocking=True)
-        step.run(xe)
-        for hbuf, dbuf in zip(outs_h, step.outputs()):
-            hbuf.copy_(dbuf, non_blocking=True)
-
-    e2e_steps = max(3, min(args.steps, 10))
-    e2e_step()
-    ms_e2e, e2e_val = aggregate_step(time_region(e2e_step, e2e_steps, device), tokens_step, device)
-    del xe
+    d2h = sum(t.numel() * t.element_size() for t in step.outputs())
+    e2e = E2EPipeline(wl, xh, in_keys, step, device)
+    e2e_steps = max(4, min(args.steps, 10))
+    e2e.run(2)  # fills and drains the pipeline once
+    ms_e2e, e2e_val = aggregate_step(e2e.timed(e2e_steps), tokens_step, device)
+    del e2e
 
     extras = {}
     if not args.no_extras:
@@ -707,6 +782,10 @@ def main(argv=None):
         extras["decode"] = measure_decode(device, 1, 1, peaks, seed=rank)
         extras["train_step_breakdown"] = {k: [c // args.steps, round(t / c, 4)]
                                           for k, (c, t) in tab.items()}
+        extras["train_step_breakdown_note"] = (
+            "per-launch event times; the gated state pass overlaps the window forward and the "
+            "gated backward's first level overlaps the window backward (library side stream), "
+            "so the times of those kernels include the overlap and do not add up to the step")
         extras["stage1_step"] = measure_stage1(wl, xd, device, 10, 3, seed=rank)
 
     cpu = None
@@ -729,7 +808,10 @@ def main(argv=None):
             "effective_tflops": flops / (ms_max * 1e-3) / 1e12,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+                    "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
+                    "pipeline": "pinned host buffers; inputs of step i+1 and outputs of step "
+                                "i-1 copied while step i computes (2 device buffer sets, "
+                                "one stream per copy direction)"},
             "gpu_launches": launches,
             "clocks": clocks,
             "extras": extras,

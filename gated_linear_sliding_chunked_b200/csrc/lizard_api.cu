@@ -53,6 +53,38 @@ cudaError_t gla_forward(lz::GlaFwdParams p, bool bf16, void* states16, ScanWs sc
   return lz::launch_gla_fwd_simt(p, bf16, s);
 }
 
+// A high-priority stream and two events per (host thread, device), created on
+// first use and kept for the life of the process.  lz_hybrid_fwd forks the
+// gated state pass onto it while the window forward runs; lz_hybrid_bwd forks
+// the gated backward's first phase onto it while the window backward runs.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t join = nullptr;
+};
+
+static cudaError_t side_stream(SideStream** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  thread_local std::unordered_map<int, SideStream> streams;
+  SideStream& ss = streams[dev];
+  if (!ss.stream) {
+    int lo = 0, hi = 0;
+    e = cudaDeviceGetStreamPriorityRange(&lo, &hi);
+    if (e != cudaSuccess) return e;
+    e = cudaStreamCreateWithPriority(&ss.stream, cudaStreamNonBlocking, hi);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      ss = SideStream{};
+      return e;
+    }
+  }
+  *out = &ss;
+  return cudaSuccess;
+}
+
 lz_status fail(lz_status st, const char* fmt, ...) {
   char buf[512];
   va_list ap;
@@ -436,16 +468,37 @@ static lz_status hybrid_fwd_impl(const char* name, const lz_dims* d, const void*
   const ScanWs scan = fwd_uses_chunks(d) ? carve_scan(c, d) : ScanWs{};
   float* parts = la ? c.take<float>(loss_parts(d)) : nullptr;
   if (states16 && chunk_states && ws_bytes(d, LZ_WS_CHUNK_STATES) > 0) states16 = chunk_states;
+  lz::GlaFwdParams gp = gla_fwd_params(d, q, k, v, g, h0);
+  gp.o = o;
+  gp.hT = hT;
+  // tensor-core path: the gated state pass (reads k, v, g; writes the chunk
+  // states and hT) runs on the side stream while the window forward runs here
+  SideStream* side = nullptr;
+  if (mma && fwd_uses_chunks(d) && bht(d) > 0) {
+    cudaError_t e = side_stream(&side);
+    if (e == cudaSuccess) e = cudaEventRecord(side->fork, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side->stream, side->fork, 0);
+    if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_fwd (fork)");
+    gp.states16 = states16;
+    gp.delta16 = scan.delta16;
+    gp.decay = scan.decay;
+    e = lz::launch_gla_states(gp, side->stream);
+    // recorded even after a failed launch: the caller's stream never waits
+    // on an unrecorded event
+    const cudaError_t ej = cudaEventRecord(side->join, side->stream);
+    if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_fwd (gated state pass)");
+    if (ej != cudaSuccess) return cuda_status(ej, "lz_hybrid_fwd (join)");
+  }
   lz::SwaFwdParams sp = swa_fwd_params(d, q, k, v, meta_k, meta_v);
   // tensor-core path: bf16 window output into o_swa if requested, else into o
   sp.o = mma ? (o_swa ? o_swa : o) : o_swa;
   sp.o_f32 = osw;
   sp.lse = lse;
   cudaError_t e = swa_forward(sp, bf, s);
-  if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_fwd (window branch)");
-  lz::GlaFwdParams gp = gla_fwd_params(d, q, k, v, g, h0);
-  gp.o = o;
-  gp.hT = hT;
+  if (e != cudaSuccess) {
+    if (side) cudaStreamWaitEvent(s, side->join, 0);
+    return cuda_status(e, "lz_hybrid_fwd (window branch)");
+  }
   gp.add = osw;
   gp.add16 = mma ? sp.o : nullptr;
   gp.alpha = d->alpha;
@@ -458,7 +511,12 @@ static lz_status hybrid_fwd_impl(const char* name, const lz_dims* d, const void*
     gp.loss_scale = lscale;
     gp.loss_part = parts;
   }
-  e = gla_forward(gp, bf, states16, scan, s);
+  if (side) {  // the state pass ran on the side stream: join it, then the outputs
+    e = cudaStreamWaitEvent(s, side->join, 0);
+    if (e == cudaSuccess) e = lz::launch_gla_out(gp, s);
+  } else {
+    e = gla_forward(gp, bf, states16, scan, s);
+  }
   if (e != cudaSuccess || !la) return cuda_status(e, name);
   size_t nparts = loss_parts(d);
   if (!fused) {
@@ -555,36 +613,6 @@ static cudaError_t gla_bwd_launch(const lz_dims* d, const void* q, const void* k
   return gla_bwd_phase2(d, p, s);
 }
 
-// A high-priority stream and two events per (host thread, device), created on
-// first use and kept for the life of the process: lz_hybrid_bwd forks the
-// gated backward's first phase onto it and joins it back before the second.
-struct SideStream {
-  cudaStream_t stream = nullptr;
-  cudaEvent_t fork = nullptr;
-  cudaEvent_t join = nullptr;
-};
-
-static cudaError_t side_stream(SideStream** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  thread_local std::unordered_map<int, SideStream> streams;
-  SideStream& ss = streams[dev];
-  if (!ss.stream) {
-    int lo = 0, hi = 0;
-    e = cudaDeviceGetStreamPriorityRange(&lo, &hi);
-    if (e != cudaSuccess) return e;
-    e = cudaStreamCreateWithPriority(&ss.stream, cudaStreamNonBlocking, hi);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming);
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming);
-    if (e != cudaSuccess) {
-      ss = SideStream{};
-      return e;
-    }
-  }
-  *out = &ss;
-  return cudaSuccess;
-}
 
 lz_status lz_gla_bwd(const lz_dims* d, const void* q, const void* k, const void* v,
                      const float* g, const float* h0, const void* dO, const float* dhT,

@@ -207,3 +207,39 @@ def test_workload_train_sampled():
     dal = float(np.sum(xs["dO"] * o_swa))
     assert_close("dalpha", res["dalpha"].cpu().double().numpy(), np.array([dal]),
                  torch.bfloat16)
+
+
+def test_training_step_under_cuda_graph():
+    """The forward + backward step (whose gated passes fork onto the library's
+    side stream and join back) captured into a CUDA graph and replayed gives
+    the eager results bit for bit."""
+    cpu, dev = small_problem(55, 2, 2, 333, 128, 128, 4, torch.bfloat16, train=True, h0=True)
+
+    def step():
+        f = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
+                         w=64, alpha=0.5, h0=dev["h0"], want_hT=True, want_lse=True,
+                         want_o_swa=True, want_chunk_states=True)
+        b = L.hybrid_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
+                         f["lse"], dev["dO"], w=64, alpha=0.5, h0=dev["h0"], dhT=dev["dhT"],
+                         o_swa=f["o_swa"], chunk_states=f["chunk_states"], hT=f["hT"],
+                         want_dh0=True)
+        return f, b
+
+    f0, b0 = step()
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        f1, b1 = step()
+    graph.replay()
+    torch.cuda.synchronize()
+    for name in ("o", "hT", "lse", "o_swa"):
+        assert torch.equal(f1[name], f0[name]), name
+    for name in ("dq", "dk", "dv", "dg", "dh0", "dmeta_k", "dmeta_v", "dalpha"):
+        assert torch.equal(b1[name], b0[name]), name
+    L.lz_device_check()
