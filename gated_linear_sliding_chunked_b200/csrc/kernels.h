@@ -196,7 +196,7 @@ struct SwaBwdParams {
   unsigned int* status;  // device status word (set by the tcgen05 launcher)
 };
 // query rows per CTA of the meta-gradient pass (one partial per slab)
-constexpr int kSwaBwdSlab = 512;
+constexpr int kSwaBwdSlab = 256;
 int swa_bwd_n_qblocks(int B, int H, int T);
 int swa_bwd_n_meta_parts(int B, int T);
 cudaError_t launch_swa_bwd_simt(const SwaBwdParams& p, bool bf16, cudaStream_t s);
