@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(NT) decode_kernel(DecodeParams p) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) x[e] = ks[l16 * 8 + e];
     } else if (key < nwin) {
-      const int sl = (int)((pos - key) % w);
+      const int sl = slot >= key ? slot - key : slot - key + w;  // (pos - key) mod w, 0 < key < w
       load8(kring + (size_t)sl * D + l16 * 8, x);
     } else {
       load8(mk + (size_t)(key - nwin) * D + l16 * 8, x);
@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(NT) decode_kernel(DecodeParams p) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) x[e] = vs[l * 8 + e];
       } else if (key < nwin) {
-        const int sl = (int)((pos - key) % w);
+        const int sl = slot >= key ? slot - key : slot - key + w;  // (pos - key) mod w
         load8(vring + (size_t)sl * D + l * 8, x);
       } else {
         if (!mv) continue;
