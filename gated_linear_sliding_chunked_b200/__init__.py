@@ -32,7 +32,8 @@ LZ_F32, LZ_BF16 = 0, 1
 EXPORTS = ("lz_gla_fwd", "lz_gla_bwd", "lz_swa_meta_fwd", "lz_hybrid_fwd", "lz_swa_meta_bwd",
            "lz_hybrid_bwd", "lz_gla_decode_step", "lz_workspace_bytes", "lz_last_error",
            "lz_version", "lz_timing_enable", "lz_timing_read", "lz_swa_meta_bwd_noalloc",
-           "lz_device_check", "lz_prefer_tcgen05", "lz_decode_prefill", "lz_hybrid_fwd_mse")
+           "lz_device_check", "lz_prefer_tcgen05", "lz_decode_prefill", "lz_hybrid_fwd_mse",
+           "lz_selftest_bounded_wait")
 
 # size of the static scratch array behind lz_swa_meta_bwd_noalloc
 LZ_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -79,6 +80,7 @@ def load(path: str = LIB_PATH):
     lib.lz_gla_decode_step.argtypes = ([ctypes.c_int] * 7 + [ctypes.c_float] * 2 +
                                        [_P] * 11 + [_P])
     lib.lz_device_check.argtypes = [_P]
+    lib.lz_selftest_bounded_wait.argtypes = [_P]
     lib.lz_decode_prefill.argtypes = [ctypes.c_int] * 7 + [_P] * 7 + [_P]
     lib.lz_prefer_tcgen05.argtypes = [ctypes.c_int]
     lib.lz_timing_enable.argtypes = [ctypes.c_int]
@@ -141,6 +143,13 @@ def lz_device_check(stream=None):
     """Raises LzError(LZ_ERR_TIMEOUT) if a bounded device wait of a library
     kernel gave up since the last check (synchronizes the stream)."""
     _check(load().lz_device_check(_stream(stream)))
+
+
+def lz_selftest_bounded_wait(stream=None):
+    """Launches the library's failure-path self-test: a bounded device wait
+    that nothing completes gives up after 0.2 s; the next lz_device_check
+    raises LzError(LZ_ERR_TIMEOUT)."""
+    _check(load().lz_selftest_bounded_wait(_stream(stream)))
 
 
 def lz_prefer_tcgen05(on: bool) -> bool:

@@ -9,6 +9,8 @@
 
 #include "../../include/lizard.h"
 #include "kernels.h"
+#include "mma.cuh"
+#include "tc05.cuh"
 
 namespace {
 
@@ -54,6 +56,39 @@ extern "C" lz_status lz_device_check(lz_stream stream) {
     char msg[256];
     std::snprintf(msg, sizeof(msg), "lz_device_check: %u bounded device wait(s) gave up", n);
     return (lz_status)lz::set_last_error(LZ_ERR_TIMEOUT, msg);
+  }
+  lz::set_last_error(LZ_OK, "");
+  return LZ_OK;
+}
+
+namespace {
+
+// The failure path on purpose: an mbarrier that nothing arrives on.  The
+// bounded wait gives up after its time limit, counts itself in the status
+// word and the kernel returns; no fault, no hang.
+__global__ void bounded_wait_selftest_kernel(unsigned int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = lz::smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    lz::mbar_init(b, 1);
+    lz::mbar_init_fence();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) lz::mbar_wait(b, 0, status);
+}
+
+}  // namespace
+
+extern "C" lz_status lz_selftest_bounded_wait(lz_stream stream) {
+  unsigned int* word = lz::device_status_word();
+  if (word == nullptr)
+    return (lz_status)lz::set_last_error(LZ_ERR_CUDA, "lz_selftest_bounded_wait: no device status word");
+  bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(word);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    char msg[256];
+    std::snprintf(msg, sizeof(msg), "lz_selftest_bounded_wait: %s", cudaGetErrorString(e));
+    return (lz_status)lz::set_last_error(LZ_ERR_CUDA, msg);
   }
   lz::set_last_error(LZ_OK, "");
   return LZ_OK;

@@ -261,6 +261,13 @@ lz_status lz_decode_prefill(int Bd, int H, int T, int dk, int dv, int w,
  * last check (LZ_OK otherwise; LZ_ERR_CUDA if the read failed). */
 lz_status lz_device_check(lz_stream stream);
 
+/* Test hook of that failure path: launches one block on `stream` that waits
+ * on an mbarrier nothing arrives on.  The wait gives up after its 0.2 s limit
+ * and counts itself in the status word, so the next lz_device_check returns
+ * LZ_ERR_TIMEOUT (and clears it); the device stays usable.  Asynchronous;
+ * LZ_ERR_CUDA if the launch failed. */
+lz_status lz_selftest_bounded_wait(lz_stream stream);
+
 /* Kernel choice of the window branch for the calling host thread (no
  * counterpart on the pages).  bf16 with dk = dv = 128 has tcgen05 kernels
  * with TMA-fed operands and accumulators in tensor memory (the default) and

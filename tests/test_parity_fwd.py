@@ -172,6 +172,26 @@ def test_window_forward_dispatch_and_device_status():
     L.lz_device_check()
 
 
+def test_bounded_wait_failure_path_is_reported_and_device_stays_usable():
+    """A bounded device wait that nothing completes (the library's self-test
+    kernel) gives up, the status word reports it once, and the next kernels
+    run and match the oracle."""
+    L.lz_device_check()  # start from a clean word
+    L.lz_selftest_bounded_wait()
+    with pytest.raises(L.LzError) as err:
+        L.lz_device_check()
+    assert err.value.status == L.LZ_ERR_TIMEOUT
+    L.lz_device_check()  # cleared by the read
+    cpu, dev = small_problem(23, 1, 2, 150, 128, 128, 4, torch.bfloat16)
+    res = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
+                       w=64, alpha=0.5)
+    x = oracle_inputs(cpu, ("q", "k", "v", "g", "meta_k", "meta_v"))
+    ref = oracle.hybrid_fwd(x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], 64,
+                            1 / math.sqrt(128), 0.5)
+    assert_close("o", res["o"], ref["o"], torch.bfloat16)
+    L.lz_device_check()
+
+
 @pytest.mark.parametrize("T,w,M,sink", [(1, 1, 0, False), (77, 7, 0, False), (130, 64, 4, True),
                                         (333, 128, 16, False), (700, 129, 8, False)])
 @pytest.mark.parametrize("tc", [True, False], ids=["tcgen05", "warp-mma"])
