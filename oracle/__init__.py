@@ -71,7 +71,9 @@ def _bind(lib):
     lib.oracle_decode_step.argtypes = ([_i] * 6 + [_f, _f] + [_D] * 3 + [_I64] +
                                        [_D] * 7 + [_i])
     lib.oracle_mse_loss.argtypes = [ctypes.c_int64] + [_D] * 4
-    for name in ("oracle_mse_loss", "oracle_gla_fwd", "oracle_gla_chunked_fwd", "oracle_swa_meta_fwd",
+    lib.oracle_gate_from_logits.argtypes = [ctypes.c_int64, _D, ctypes.c_double, _D]
+    lib.oracle_dlogits.argtypes = [ctypes.c_int64, _D, ctypes.c_double, _D, _D]
+    for name in ("oracle_gate_from_logits", "oracle_dlogits", "oracle_mse_loss", "oracle_gla_fwd", "oracle_gla_chunked_fwd", "oracle_swa_meta_fwd",
                  "oracle_hybrid_fwd", "oracle_gla_bwd", "oracle_swa_meta_bwd",
                  "oracle_hybrid_bwd", "oracle_decode_step"):
         getattr(lib, name).restype = ctypes.c_int
@@ -259,3 +261,23 @@ def mse_loss(o, target, *, lib=None):
     dO, pd = _out(o.shape)
     _check(lib.oracle_mse_loss(int(o.size), po, pt, pl, pd), "mse_loss")
     return float(loss[0]), dO
+
+
+def gate_from_logits(z, scale=1.0, *, lib=None):
+    """Log-gate g = scale * log sigma(z) from the gate logit z (same shape)."""
+    lib = lib or load()
+    z, pz = _in(z)
+    g, pg = _out(z.shape)
+    _check(lib.oracle_gate_from_logits(int(z.size), pz, float(scale), pg), "gate_from_logits")
+    return g
+
+
+def dlogits(z, dg, scale=1.0, *, lib=None):
+    """dL/dz from dL/dg through g = scale * log sigma(z)."""
+    lib = lib or load()
+    (z, pz), (dg, pdg) = _in(z), _in(dg)
+    if z.shape != dg.shape:
+        raise ValueError("dlogits: z and dg differ in shape")
+    dz, pdz = _out(z.shape)
+    _check(lib.oracle_dlogits(int(z.size), pz, float(scale), pdg, pdz), "dlogits")
+    return dz

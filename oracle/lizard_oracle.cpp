@@ -639,6 +639,36 @@ int oracle_decode_step(int Bd, int H, int dk, int dv, int w, int M,
   return 0;
 }
 
+// Gate from its logit (section 2a: the learnable gate is Gamma_i =
+// sigma(W_gamma x_i), so the logit z = W_gamma x_i arrives from the
+// projection upstream).  The log-gate the recurrence uses is
+//   g = scale * log sigma(z)  (<= 0; scale > 0 a temperature, 1 on the page)
+// with log sigma(z) = -log(1 + e^{-z}) taken in the form that does not
+// overflow for either sign of z.  n elements; g_out may alias nothing.
+int oracle_gate_from_logits(int64_t n, const double* z, double scale, double* g_out) {
+  if (n < 0 || !(scale > 0.0)) return -1;
+  if (n > 0 && (!z || !g_out)) return -1;
+  for (int64_t x = 0; x < n; ++x) {
+    const double v = z[x];
+    const double ls = v >= 0.0 ? -std::log1p(std::exp(-v)) : v - std::log1p(std::exp(v));
+    g_out[x] = scale * ls;
+  }
+  return 0;
+}
+
+// Chain rule through that map: dL/dz = dL/dg * scale * sigma(-z), with
+// sigma(-z) = 1 / (1 + e^{z}) taken without overflow.
+int oracle_dlogits(int64_t n, const double* z, double scale, const double* dg, double* dz) {
+  if (n < 0 || !(scale > 0.0)) return -1;
+  if (n > 0 && (!z || !dg || !dz)) return -1;
+  for (int64_t x = 0; x < n; ++x) {
+    const double v = z[x];
+    const double sneg = v >= 0.0 ? std::exp(-v) / (1.0 + std::exp(-v)) : 1.0 / (1.0 + std::exp(v));
+    dz[x] = dg[x] * scale * sneg;
+  }
+  return 0;
+}
+
 // Stage-1 distillation loss (section 2b, "training strategy": the first
 // stage trains the hybrid attention to reproduce the teacher's attention
 // output under a mean-squared-error loss).  Reading: the mean runs over every

@@ -414,10 +414,57 @@ def pin_stage1_chain_fd(lib):
         assert _rel(got, num) < 1e-6, (key, _rel(got, num))
 
 
+# ----------------------------------------------------------------------------
+# gate from its logit (section 2a: Gamma = sigma(W_gamma x))
+# ----------------------------------------------------------------------------
+def pin_gate_logits_closed_form(lib):
+    """exp(g / scale) is the logistic function of z (written here as
+    1 / (1 + e^{-z}) directly); z = 0 gives -scale log 2; far tails behave
+    as -scale e^{-z} and scale z."""
+    z = np.array([-40.0, -5.0, -0.5, 0.0, 0.7, 3.0, 30.0])
+    for scale in (1.0, 1.0 / 16):
+        g = oracle.gate_from_logits(z, scale, lib=lib)
+        assert np.all(g <= 0.0)
+        mid = np.abs(z) < 10
+        assert np.allclose(np.exp(g[mid] / scale), 1.0 / (1.0 + np.exp(-z[mid])), rtol=1e-13)
+        assert abs(g[3] + scale * np.log(2.0)) < 1e-15
+        assert abs(g[-1] / scale + np.exp(-30.0)) < 1e-25
+        assert abs(g[0] / scale - (-40.0)) < 1e-15
+
+
+def pin_gate_logits_grad_fd(lib):
+    """dz through the gate map composed with the hybrid operator equals the
+    central differences of sum(o * dO) + sum(hT * dhT) with respect to z."""
+    x, dO, dhT = _tiny_case(31)
+    r = RNG(32)
+    z = r.standard_normal(np.shape(x["g"])) * 2.0
+    w, scale, s, eps = 3, 0.6, 0.25, 1e-6
+
+    def loss(zz):
+        xx = dict(x)
+        xx["g"] = oracle.gate_from_logits(zz, s, lib=lib)
+        return _hybrid_loss(lib, xx, dO, dhT, w, scale)
+
+    xx = dict(x)
+    xx["g"] = oracle.gate_from_logits(z, s, lib=lib)
+    an = oracle.hybrid_bwd(xx["q"], xx["k"], xx["v"], xx["g"], xx["meta_k"], xx["meta_v"], dO, w,
+                           scale, float(xx["alpha"]), xx["h0"], dhT, lib=lib)
+    dz = oracle.dlogits(z, an["dg"], s, lib=lib).reshape(-1)
+    num = np.zeros(z.size)
+    for idx in range(z.size):
+        zp = z.reshape(-1).copy()
+        zm = zp.copy()
+        zp[idx] += eps
+        zm[idx] -= eps
+        num[idx] = (loss(zp.reshape(z.shape)) - loss(zm.reshape(z.shape))) / (2 * eps)
+    assert _rel(dz, num) < 1e-6, _rel(dz, num)
+
+
 ALL_PINS = [
     pin_gla_closed_form, pin_gla_unit_gates, pin_gla_full_forgetting,
     pin_gla_initial_state, pin_gla_chunked_identity, pin_swa_full_causal,
     pin_swa_band_meta, pin_swa_sinks, pin_hybrid_affine, pin_hybrid_grad_fd,
     pin_swa_grad_fd, pin_gla_dg_identity, pin_decode_matches_prefill,
     pin_mse_closed_form, pin_mse_grad_fd, pin_stage1_chain_fd,
+    pin_gate_logits_closed_form, pin_gate_logits_grad_fd,
 ]

@@ -39,6 +39,8 @@ MUTANTS = [
     ("mse_gradient_drops_two", "if (dO) dO[x] = 2.0 * diff / (double)n;", "if (dO) dO[x] = diff / (double)n;"),
     ("mse_sum_not_mean", "*loss = n > 0 ? s / (double)n : 0.0;", "*loss = n > 0 ? s : 0.0;"),
     ("mse_gradient_sign", "const double diff = o[x] - target[x];", "const double diff = target[x] - o[x];"),
+    ("gate_logit_unscaled", "g_out[x] = scale * ls;", "g_out[x] = ls;"),
+    ("dlogits_sigmoid_of_z", "dz[x] = dg[x] * scale * sneg;", "dz[x] = dg[x] * scale * (1.0 - sneg);"),
 ]
 
 
