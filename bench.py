@@ -253,14 +253,15 @@ def train_flops(wl) -> float:
 class TrainStep:
     """Buffers and one fwd+bwd pass through the C ABI."""
 
-    def __init__(self, wl, x, device):
+    def __init__(self, wl, x, device, gate_logits=False, gate_scale=1.0):
         import gated_linear_sliding_chunked_b200 as L
         self.L = L
         self.wl = wl
         self.x = x
         B, H, T, dk, dv, M = wl.B, wl.H, wl.T, wl.dk, wl.dv, wl.M
         self.dims = L.make_dims(B, H, T, dk, dv, chunk=wl.chunk, w=wl.w, M=M,
-                                io=L.io_of(wl.torch_dtype), scale=wl.scale, alpha=wl.alpha)
+                                io=L.io_of(wl.torch_dtype), scale=wl.scale, alpha=wl.alpha,
+                                gate_logits=gate_logits, gate_scale=gate_scale)
         dt = wl.torch_dtype
         mk = lambda *s, dtype=dt: torch.empty(*s, dtype=dtype, device=device)
         self.o = mk(B, H, T, dv)
@@ -526,6 +527,30 @@ def measure_stage1(wl, x, device, steps, warmup, seed):
             "kernels": {k: [c // steps, round(t / c, 4)] for k, (c, t) in tab.items()}}
 
 
+def measure_train_gate_logits(wl, x, device, steps, warmup, seed):
+    """The training step with the gates given as bf16 logits z (log-gate =
+    log sigma(z) / 16, the workload's gate distribution with z ~ N(0, 1)),
+    formed inside the kernels instead of read as fp32 log-gates."""
+    import gated_linear_sliding_chunked_b200 as L
+    gen = torch.Generator(device=device)
+    gen.manual_seed(2000 + seed)
+    z = torch.randn(x["g"].shape, generator=gen, device=device).to(torch.bfloat16)
+    xz = dict(x)
+    xz["g"] = z
+    st = TrainStep(wl, xz, device, gate_logits=True, gate_scale=1.0 / 16)
+    for _ in range(warmup):
+        st.run()
+    torch.cuda.synchronize(device)
+    L.lz_timing_enable(True)
+    ms = time_region(st.run, steps, device)
+    L.lz_timing_enable(False)
+    tab = kernel_table(L.lz_timing_read())
+    L.lz_device_check()
+    return {"workload": wl.name + " with bf16 gate logits (log-gate = log sigma(z) / 16, z ~ N(0, 1))",
+            "tokens_per_s": wl.B * wl.T / (ms * 1e-3), "ms_per_step": round(ms, 4),
+            "kernels": {k: [c // steps, round(t / c, 4)] for k, (c, t) in tab.items()}}
+
+
 def measure_decode(device, steps, warmup, peaks, seed, n_steps=1000):
     import gated_linear_sliding_chunked_b200 as L
     from gated_linear_sliding_chunked_b200 import inputs as I
@@ -787,6 +812,7 @@ def main(argv=None):
             "gated backward's first level overlaps the window backward (library side stream), "
             "so the times of those kernels include the overlap and do not add up to the step")
         extras["stage1_step"] = measure_stage1(wl, xd, device, 10, 3, seed=rank)
+        extras["train_step_gate_logits"] = measure_train_gate_logits(wl, xd, device, 10, 3, seed=rank)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

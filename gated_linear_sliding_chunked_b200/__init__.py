@@ -49,7 +49,8 @@ class LzDims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int),
                 ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("chunk", ctypes.c_int),
                 ("w", ctypes.c_int), ("M", ctypes.c_int), ("io", ctypes.c_int),
-                ("scale", ctypes.c_float), ("alpha", ctypes.c_float)]
+                ("scale", ctypes.c_float), ("alpha", ctypes.c_float),
+                ("gate_logits", ctypes.c_int), ("gate_scale", ctypes.c_float)]
 
 
 _lib = None
@@ -126,10 +127,13 @@ def io_of(dtype) -> int:
 
 
 def make_dims(B, H, T, dk, dv, *, chunk=64, w=1, M=0, io=LZ_BF16, scale=None,
-              alpha=0.5) -> LzDims:
+              alpha=0.5, gate_logits=False, gate_scale=1.0) -> LzDims:
+    """gate_logits: the `g` tensors of the calls are bf16 gate logits z (the
+    log-gate is gate_scale * log sigma(z)) instead of fp32 log-gates."""
     if scale is None:
         scale = 1.0 / math.sqrt(dk)
-    return LzDims(B, H, T, dk, dv, chunk, w, M, io, float(scale), float(alpha))
+    return LzDims(B, H, T, dk, dv, chunk, w, M, io, float(scale), float(alpha),
+                  int(bool(gate_logits)), float(gate_scale))
 
 
 # --------------------------------------------------------------------------
@@ -254,10 +258,13 @@ def lz_gla_decode_step(Bd, H, dk, dv, w, M, io, scale, alpha, state, kring, vrin
 # --------------------------------------------------------------------------
 # Allocating helpers (torch owns memory; the library computes)
 # --------------------------------------------------------------------------
-def _dims_from(q, v, *, chunk, w, M, scale, alpha):
+def _dims_from(q, v, *, chunk, w, M, scale, alpha, g=None, gate_scale=1.0):
+    """A bf16 `g` is read as gate logits (log-gate = gate_scale * log sigma(g));
+    an fp32 `g` as log-gates."""
     B, H, T, dk = q.shape
+    logits = g is not None and g.dtype != torch.float32
     return make_dims(B, H, T, dk, v.shape[-1], chunk=chunk, w=w, M=M, io=io_of(q.dtype),
-                     scale=scale, alpha=alpha)
+                     scale=scale, alpha=alpha, gate_logits=logits, gate_scale=gate_scale)
 
 
 def _ws(dims, which, device):
@@ -276,10 +283,11 @@ def _chunk_states(dims, device):
     return torch.empty(n, dtype=torch.uint8, device=device) if n else None
 
 
-def gla_fwd(q, k, v, g, h0=None, *, chunk=64, want_hT=False, want_chunk_states=False,
+def gla_fwd(q, k, v, g, h0=None, *, chunk=64, gate_scale=1.0, want_hT=False, want_chunk_states=False,
             stream=None):
-    """Returns (o, hT), or (o, hT, chunk_states) with want_chunk_states."""
-    d = _dims_from(q, v, chunk=chunk, w=1, M=0, scale=None, alpha=0.0)
+    """Returns (o, hT), or (o, hT, chunk_states) with want_chunk_states.  A bf16
+    g holds gate logits (log-gate = gate_scale * log sigma(g))."""
+    d = _dims_from(q, v, chunk=chunk, w=1, M=0, scale=None, alpha=0.0, g=g, gate_scale=gate_scale)
     o = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=q.device)
     hT = torch.empty(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], dtype=torch.float32,
                      device=q.device) if want_hT else None
@@ -298,9 +306,11 @@ def swa_meta_fwd(q, k, v, meta_k, meta_v, *, w, scale=None, want_lse=True, strea
 
 
 def hybrid_fwd(q, k, v, g, meta_k, meta_v, *, w, alpha, scale=None, chunk=64, h0=None,
-               want_hT=False, want_lse=False, want_o_swa=False, want_chunk_states=False,
-               stream=None):
-    d = _dims_from(q, v, chunk=chunk, w=w, M=_M(meta_k), scale=scale, alpha=alpha)
+               gate_scale=1.0, want_hT=False, want_lse=False, want_o_swa=False,
+               want_chunk_states=False, stream=None):
+    """A bf16 g holds gate logits (log-gate = gate_scale * log sigma(g))."""
+    d = _dims_from(q, v, chunk=chunk, w=w, M=_M(meta_k), scale=scale, alpha=alpha, g=g,
+                   gate_scale=gate_scale)
     dev = q.device
     o = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=dev)
     hT = torch.empty(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], dtype=torch.float32,
@@ -314,11 +324,12 @@ def hybrid_fwd(q, k, v, g, meta_k, meta_v, *, w, alpha, scale=None, chunk=64, h0
 
 
 def hybrid_fwd_mse(q, k, v, g, meta_k, meta_v, target, *, w, alpha, scale=None, chunk=64,
-                   h0=None, want_dO=True, want_hT=False, want_lse=False, want_o_swa=False,
+                   h0=None, gate_scale=1.0, want_dO=True, want_hT=False, want_lse=False, want_o_swa=False,
                    want_chunk_states=False, stream=None):
     """hybrid_fwd plus the stage-1 loss mean((o - target)^2); the result adds
     "loss" (0-dim fp32 tensor on the device) and "dO" (its gradient, or None)."""
-    d = _dims_from(q, v, chunk=chunk, w=w, M=_M(meta_k), scale=scale, alpha=alpha)
+    d = _dims_from(q, v, chunk=chunk, w=w, M=_M(meta_k), scale=scale, alpha=alpha, g=g,
+                   gate_scale=gate_scale)
     dev = q.device
     o = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=dev)
     hT = torch.empty(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], dtype=torch.float32,
@@ -336,12 +347,12 @@ def hybrid_fwd_mse(q, k, v, g, meta_k, meta_v, target, *, w, alpha, scale=None, 
 
 
 def gla_bwd(q, k, v, g, dO, h0=None, dhT=None, *, chunk=64, chunk_states=None, hT=None,
-            want_dh0=False, stream=None):
+            gate_scale=1.0, want_dh0=False, stream=None):
     """chunk_states, hT: the forward's (optional; see lz_gla_bwd)."""
-    d = _dims_from(q, v, chunk=chunk, w=1, M=0, scale=None, alpha=0.0)
+    d = _dims_from(q, v, chunk=chunk, w=1, M=0, scale=None, alpha=0.0, g=g, gate_scale=gate_scale)
     dev = q.device
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    dg = torch.empty_like(g)
+    dg = torch.empty(g.shape, dtype=torch.float32, device=dev)  # dL/dz for gate logits
     dh0 = torch.empty(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], dtype=torch.float32,
                       device=dev) if want_dh0 else None
     ws, n = _ws(d, LZ_WS_GLA_BWD, dev)
@@ -364,14 +375,16 @@ def swa_meta_bwd(q, k, v, meta_k, meta_v, lse, dO, *, w, scale=None, o=None, str
 
 
 def hybrid_bwd(q, k, v, g, meta_k, meta_v, lse, dO, *, w, alpha, scale=None, chunk=64,
-               h0=None, dhT=None, o_swa=None, chunk_states=None, hT=None, want_dh0=False,
-               stream=None):
-    """o_swa, chunk_states, hT: the forward's (optional; see lz_hybrid_bwd)."""
+               h0=None, dhT=None, o_swa=None, chunk_states=None, hT=None, gate_scale=1.0,
+               want_dh0=False, stream=None):
+    """o_swa, chunk_states, hT: the forward's (optional; see lz_hybrid_bwd).  A bf16
+    g holds gate logits; dg then receives dL/dg_logits (fp32)."""
     M = _M(meta_k)
-    d = _dims_from(q, v, chunk=chunk, w=w, M=M, scale=scale, alpha=alpha)
+    d = _dims_from(q, v, chunk=chunk, w=w, M=M, scale=scale, alpha=alpha, g=g,
+                   gate_scale=gate_scale)
     dev = q.device
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    dg = torch.empty_like(g)
+    dg = torch.empty(g.shape, dtype=torch.float32, device=dev)  # dL/dz for gate logits
     dh0 = torch.empty(q.shape[0], q.shape[1], q.shape[-1], v.shape[-1], dtype=torch.float32,
                       device=dev) if want_dh0 else None
     dmk = torch.empty(q.shape[1], M, q.shape[-1], dtype=torch.float32, device=dev) if M else None

@@ -38,6 +38,7 @@
 // with ci = e^{b_t}/Eq and ck = e^{b_l - b_t}/Ek constant per (sub-block,
 // key dim).
 #include <cooperative_groups.h>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -78,13 +79,14 @@ __device__ __forceinline__ int rsw(int row, int col) {
 
 __device__ __forceinline__ int pair_index(int I, int J) { return I * (I + 1) / 2 + J; }
 
-// exp(sum_{x = s+1 .. t} g_x,i) for chunk rows s <= t (g: global, the
-// chunk's first row, already offset to this CTA's key dims).  Used only by
-// the strong-decay fallback of the diagonal blocks; it returns a scalar so
-// that no register array of the caller has its address taken.
-__device__ __noinline__ float gate_ratio(const float* g, int rows, int t, int s, int i) {
+// exp(sum_{x = s+1 .. t} g_x,i) for chunk rows s <= t (g, or the logits gz:
+// global, the chunk's first row, already offset to this CTA's key dims).
+// Used only by the strong-decay fallback of the diagonal blocks; it returns a
+// scalar so that no register array of the caller has its address taken.
+template <class Gates>
+__device__ __noinline__ float gate_ratio(Gates g, int rows, int t, int s, int i) {
   float lg = 0.f;
-  for (int x = s + 1; x <= t && x < rows; ++x) lg += g[(size_t)x * DK + i];
+  for (int x = s + 1; x <= t && x < rows; ++x) lg += g.at((size_t)x * DK + i);
   return __expf(lg);
 }
 
@@ -114,9 +116,9 @@ static_assert(sizeof(float) * C * RP <= 2 * sizeof(bf16) * C * KP, "dv share mus
 // role 1 (dk): sum_{u in block, u >= t} (dO_u . v_t) q_u,il exp(b_u - b_t)
 // (dO, v: shared tiles; kq, g: global, the chunk's first row, offset to this
 // CTA's key dims)
-__device__ __noinline__ float diag_intra_term(const bf16* dO, const bf16* v, const bf16* kq,
-                                                 const float* g, int rows, int I, int t, int il,
-                                                 int role) {
+template <class Gates>
+__device__ __noinline__ float diag_intra_term(const bf16* dO, const bf16* v, const bf16* kq, Gates g,
+                                              int rows, int I, int t, int il, int role) {
   float x = 0.f;
   const int lo = role == 0 ? SB * I : t, hi = role == 0 ? t : SB * I + SB - 1;
   for (int r = lo; r <= hi && r < rows; ++r) {
@@ -131,17 +133,21 @@ __device__ __noinline__ float diag_intra_term(const bf16* dO, const bf16* v, con
 
 // A^T[t][u] = sum_i q_u,i k_t,i exp(b_u,i - b_t,i) over this CTA's key dims,
 // chunk rows t <= u < rows (strong-decay fallback of the diagonal blocks)
-__device__ __noinline__ float diag_at_entry(const bf16* q, const bf16* k, const float* g, int rows,
-                                               int t, int u) {
+template <class Gates>
+__device__ __noinline__ float diag_at_entry(const bf16* q, const bf16* k, Gates g, int rows, int t,
+                                            int u) {
   float a = 0.f;
   for (int i = 0; i < DKH; ++i) {
     float lg = 0.f;
-    for (int x = t + 1; x <= u && x < rows; ++x) lg += g[(size_t)x * DK + i];
+    for (int x = t + 1; x <= u && x < rows; ++x) lg += g.at((size_t)x * DK + i);
     a += __bfloat162float(q[(size_t)u * DK + i]) * __bfloat162float(k[(size_t)t * DK + i]) * __expf(lg);
   }
   return a;
 }
 
+// LOGITS: the gates arrive as logits (p.gz set) and dg receives dL/dz; a
+// separate instantiation, so that the log-gate path keeps its schedule.
+template <bool LOGITS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
     gla_bwd_chunk_kernel(GlaBwdParams p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -159,7 +165,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
   // this chunk's first row, this CTA's key dims
   const bf16* qc = (const bf16*)p.q + tk + (size_t)c0 * DK + i0;
   const bf16* kc = (const bf16*)p.k + tk + (size_t)c0 * DK + i0;
-  const float* gch = p.g + tk + (size_t)c0 * DK + i0;
+  // log-gates, or the gate logits (then dg receives dL/dz)
+  const float* gch = LOGITS ? nullptr : p.g + tk + (size_t)c0 * DK + i0;
+  const bf16* gzc = LOGITS ? (const bf16*)p.gz + tk + (size_t)c0 * DK + i0 : nullptr;
+  using Gates = typename std::conditional<LOGITS, LogitGates, LogGates>::type;
+  Gates gsrc;
+  if constexpr (LOGITS) gsrc = LogitGates{gzc, p.gs};
+  else gsrc = LogGates{gch};
   float* stq = reinterpret_cast<float*>(sm.sp);   // q * dq
   float* stk = reinterpret_cast<float*>(sm.v);    // k * dk
   float* xch = reinterpret_cast<float*>(sm.qf);   // the peer's dv share
@@ -170,11 +182,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
   float* gs = reinterpret_cast<float*>(sm.qf);  // [C][DKH] fp32
   bf16* qs = sm.eqf;                            // [C][DKH] bf16 (swz64)
   bf16* ks = sm.ekf;
+  // logits: staged in the upper half of the log-gate tile, converted below
+  bf16* zs = reinterpret_cast<bf16*>(reinterpret_cast<unsigned char*>(gs) + sizeof(bf16) * C * DKH);
   {
-    for (int x = tid; x < C * DKH / 4; x += NT) {
-      const int r = x / (DKH / 4), cc = x % (DKH / 4);
-      const bool ok = r < rows;
-      cp_async16(&gs[r * DKH + cc * 4], gch + (size_t)(ok ? r : 0) * DK + cc * 4, ok ? 16 : 0);
+    if constexpr (LOGITS) {
+      for (int x = tid; x < C * DKH / 8; x += NT) {
+        const int r = x / (DKH / 8), cc = x % (DKH / 8);
+        const bool ok = r < rows;
+        cp_async16(&zs[r * DKH + cc * 8], gzc + (size_t)(ok ? r : 0) * DK + cc * 8, ok ? 16 : 0);
+      }
+    } else {
+      for (int x = tid; x < C * DKH / 4; x += NT) {
+        const int r = x / (DKH / 4), cc = x % (DKH / 4);
+        const bool ok = r < rows;
+        cp_async16(&gs[r * DKH + cc * 4], gch + (size_t)(ok ? r : 0) * DK + cc * 4, ok ? 16 : 0);
+      }
     }
     for (int x = tid; x < C * DKH / 8; x += NT) {
       const int r = x / (DKH / 8), cc = x % (DKH / 8);
@@ -207,6 +229,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
   }
   cp_async_wait<1>();
   __syncthreads();
+  if constexpr (LOGITS) {  // log-gates from the logits (each thread 16 consecutive elements);
+              // rows past the end: g = 0
+    const uint4 za = *reinterpret_cast<const uint4*>(&zs[tid * 16]);
+    const uint4 zb = *reinterpret_cast<const uint4*>(&zs[tid * 16 + 8]);
+    __syncthreads();  // every logit is read before the log-gates overwrite them
+    const bool ok = (tid * 16) / DKH < rows;
+    const uint32_t zw[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+    float gv[16];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+      const float2 f = unpack_bf16(zw[x]);
+      gv[2 * x] = ok ? gate_from_logit(f.x, p.gs) : 0.f;
+      gv[2 * x + 1] = ok ? gate_from_logit(f.y, p.gs) : 0.f;
+    }
+    float4* gd = reinterpret_cast<float4*>(&gs[tid * 16]);
+#pragma unroll
+    for (int x = 0; x < 4; ++x) gd[x] = make_float4(gv[4 * x], gv[4 * x + 1], gv[4 * x + 2], gv[4 * x + 3]);
+    __syncthreads();
+  }
 
   // ---- prep 1: per key dim cumulative gate products ------------------------
   const int K = tid >> 6, i = tid & 63, r0 = K * SB;
@@ -420,8 +461,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
           const float2 os = unpack_bf16(*reinterpret_cast<const uint32_t*>(&oscale[t * KP + il]));
           float x0 = acc[nt][2 * hh] * os.x, x1 = acc[nt][2 * hh + 1] * os.y;
           if (slow) {
-            x0 += diag_intra_term(sm.dO, sm.v, role == 0 ? kc : qc, gch, rows, I, t, il, role);
-            x1 += diag_intra_term(sm.dO, sm.v, role == 0 ? kc : qc, gch, rows, I, t, il + 1, role);
+            x0 += diag_intra_term(sm.dO, sm.v, role == 0 ? kc : qc, gsrc, rows, I, t, il, role);
+            x1 += diag_intra_term(sm.dO, sm.v, role == 0 ? kc : qc, gsrc, rows, I, t, il + 1, role);
           }
           if (t < rows) {
             const size_t off = tk + (size_t)(c0 + t) * DK + i0 + il;
@@ -525,7 +566,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
           const int t = gr + (e >> 1) * 8, u = nt * 8 + gc + (e & 1);
           const int rt = 16 * Iv + t, ru = 16 * Iv + u;
           if (u < t) at[nt][e] = 0.f;
-          else if (slow) at[nt][e] = ru < rows ? diag_at_entry(qc, kc, gch, rows, rt, ru) : 0.f;
+          else if (slow) at[nt][e] = ru < rows ? diag_at_entry(qc, kc, gsrc, rows, rt, ru) : 0.f;
         }
     }
     const uint32_t pa[4] = {pack_bf16(at[0][0], at[0][1]), pack_bf16(at[0][2], at[0][3]),
@@ -574,7 +615,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
 #pragma unroll
     for (int r = 0; r < SB; ++r) {
       const int t = 16 * qq + r;
-      if (t < rows) p.dg[tk + (size_t)(c0 + t) * DK + i0 + col] = base - loc[r];
+      if (t < rows) {
+        float x = base - loc[r];
+        if constexpr (LOGITS) x = dlogit(x, __bfloat162float(__ldg(&gzc[(size_t)t * DK + col])), p.gs);
+        p.dg[tk + (size_t)(c0 + t) * DK + i0 + col] = x;
+      }
     }
   }
   if (role == half && p.add_in_place && !p.add_dv) {  // loads ahead of the stores below
@@ -623,12 +668,12 @@ cudaError_t launch_gla_bwd_chunks(const GlaBwdParams& p, cudaStream_t s) {
   if (p.B * p.H == 0 || nchunks == 0) return cudaSuccess;
   if (2 * (size_t)nchunks * p.B * p.H > 0x7fffffffu) return cudaErrorInvalidConfiguration;
   const size_t bytes = sizeof(ChunkSmem);
-  cudaError_t e = cudaFuncSetAttribute(gla_bwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)bytes);
+  const auto kern = p.gz ? gla_bwd_chunk_kernel<true> : gla_bwd_chunk_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
   {
     ScopedTiming tm("gla_bwd_chunks", s);
-    gla_bwd_chunk_kernel<<<(unsigned)(2 * (size_t)nchunks * p.B * p.H), NT, bytes, s>>>(p);
+    kern<<<(unsigned)(2 * (size_t)nchunks * p.B * p.H), NT, bytes, s>>>(p);
   }
   return cudaGetLastError();
 }

@@ -243,7 +243,9 @@ static_assert(sizeof(DeltaSmem) <= 115712, "two delta CTAs must fit one SM");
 struct DeltaArgs {
   const bf16* x;   // k or q  [BH][T][DK]
   const bf16* y;   // v or dO [BH][T][DV]
-  const float* g;  // [BH][T][DK]
+  const float* g;  // [BH][T][DK] log-gates, or NULL with
+  const bf16* gz;  //   the gate logits [BH][T][DK]
+  float gs;        //   and their scale
   bf16* delta;     // [BH][nchunks][DK][DV]
   float* decay;    // [BH][nchunks][DK]
   int T;
@@ -260,21 +262,37 @@ __global__ void __launch_bounds__(NT, 2) gla_delta_kernel(DeltaArgs p) {
   const int c0 = c * C, rows = min(C, T - c0);
   const bf16* k = p.x + ((size_t)bh * T + c0) * DK;
   const bf16* v = p.y + ((size_t)bh * T + c0) * DV;
-  const float* g = p.g + ((size_t)bh * T + c0) * DK;
   for (int x = tid; x < C * DK / 8; x += NT) {
     const int r = x / (DK / 8), cc = x % (DK / 8);
     const bool ok = r < rows;
     cp_async16(&sm.k[r * QKP + cc * 8], k + (size_t)(ok ? r : 0) * DK + cc * 8, ok ? 16 : 0);
     cp_async16(&sm.v[r * VP + cc * 8], v + (size_t)(ok ? r : 0) * DV + cc * 8, ok ? 16 : 0);
   }
-  for (int x = tid; x < C * DK / 4; x += NT) {
-    const int r = x / (DK / 4), cc = x % (DK / 4);
-    const bool ok = r < rows;
-    cp_async16(&sm.g[r * DK + cc * 4], g + (size_t)(ok ? r : 0) * DK + cc * 4, ok ? 16 : 0);
+  if (p.gz) {  // logits go through ks (written only after the prep's first barrier)
+    const bf16* z = p.gz + ((size_t)bh * T + c0) * DK;
+    for (int x = tid; x < C * DK / 8; x += NT) {
+      const int r = x / (DK / 8), cc = x % (DK / 8);
+      const bool ok = r < rows;
+      cp_async16(&sm.ks[r * QKP + cc * 8], z + (size_t)(ok ? r : 0) * DK + cc * 8, ok ? 16 : 0);
+    }
+  } else {
+    const float* g = p.g + ((size_t)bh * T + c0) * DK;
+    for (int x = tid; x < C * DK / 4; x += NT) {
+      const int r = x / (DK / 4), cc = x % (DK / 4);
+      const bool ok = r < rows;
+      cp_async16(&sm.g[r * DK + cc * 4], g + (size_t)(ok ? r : 0) * DK + cc * 4, ok ? 16 : 0);
+    }
   }
   cp_async_commit();
   cp_async_wait<0>();
   __syncthreads();
+  if (p.gz) {  // log-gates from the logits; rows past the end: g = 0
+    for (int x = tid; x < C * DK; x += NT) {
+      const int r = x / DK, c = x % DK;
+      sm.g[r * DK + c] = r < rows ? gate_from_logit(__bfloat162float(sm.ks[r * QKP + c]), p.gs) : 0.f;
+    }
+    __syncthreads();
+  }
   // prep: thread -> (sub-block K, key dims i2, i2+1); rows past the end have
   // g = 0 (no decay) and x = 0.  fac[r]: the in-sub-block part of the row's
   // factor (key side: gates after the row; query side: gates up to it)
@@ -478,20 +496,21 @@ static_assert(sizeof(OutSmem) <= 115712, "two output CTAs must fit one SM");
 
 // A[t][s] with one exponential per key dim (strong-decay diagonal blocks);
 // q, k, g: global rows of the chunk.
-__device__ __noinline__ float diag_score_global(const bf16* q, const bf16* k, const float* g, int rt,
-                                                int rs) {
+template <class Gates>
+__device__ __noinline__ float diag_score_global(const bf16* q, const bf16* k, Gates g, int rt, int rs) {
   float a = 0.f;
   for (int i = 0; i < DK; ++i) {
     float lg = 0.f;
-    for (int u = rs + 1; u <= rt; ++u) lg += g[(size_t)u * DK + i];
+    for (int u = rs + 1; u <= rt; ++u) lg += g.at((size_t)u * DK + i);
     a += __bfloat162float(q[(size_t)rt * DK + i]) * __bfloat162float(k[(size_t)rs * DK + i]) * __expf(lg);
   }
   return a;
 }
 
-// LOSS: the stage-1 loss epilogue (p.target set), a separate instantiation so
-// that the plain forward keeps its registers and schedule.
-template <bool LOSS>
+// LOSS: the stage-1 loss epilogue (p.target set); LOGITS: the gates arrive as
+// logits (p.gz set).  Separate instantiations, so that the plain forward keeps
+// its registers and schedule.
+template <bool LOSS, bool LOGITS>
 __global__ void __launch_bounds__(NT, 2) gla_out_kernel(GlaFwdParams p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   OutSmem& sm = *reinterpret_cast<OutSmem*>(smem_raw);
@@ -505,7 +524,8 @@ __global__ void __launch_bounds__(NT, 2) gla_out_kernel(GlaFwdParams p) {
   const bf16* q = (const bf16*)p.q + ((size_t)bh * T + c0) * DK;
   const bf16* k = (const bf16*)p.k + ((size_t)bh * T + c0) * DK;
   const bf16* v = (const bf16*)p.v + ((size_t)bh * T + c0) * DV;
-  const float* g = p.g + ((size_t)bh * T + c0) * DK;
+  const float* g = LOGITS ? nullptr : p.g + ((size_t)bh * T + c0) * DK;
+  const bf16* gz = LOGITS ? (const bf16*)p.gz + ((size_t)bh * T + c0) * DK : nullptr;
   const bf16* sp = (const bf16*)p.states16 + ((size_t)bh * nchunks + c) * DK * DV;
 
   for (int x = tid; x < C * DK / 8; x += NT) {
@@ -533,8 +553,15 @@ __global__ void __launch_bounds__(NT, 2) gla_out_kernel(GlaFwdParams p) {
     float2 e[SB];
 #pragma unroll
     for (int r = 0; r < SB; ++r) {
-      const float2 gg = r0 + r < rows ? *reinterpret_cast<const float2*>(&g[(size_t)(r0 + r) * DK + i2])
-                                      : make_float2(0.f, 0.f);
+      float2 gg = make_float2(0.f, 0.f);
+      if (r0 + r < rows) {
+        if constexpr (LOGITS) {
+          const float2 zz = unpack_bf16(*reinterpret_cast<const uint32_t*>(&gz[(size_t)(r0 + r) * DK + i2]));
+          gg = make_float2(gate_from_logit(zz.x, p.gs), gate_from_logit(zz.y, p.gs));
+        } else {
+          gg = *reinterpret_cast<const float2*>(&g[(size_t)(r0 + r) * DK + i2]);
+        }
+      }
       e[r] = make_float2(__expf(gg.x), __expf(gg.y));
     }
     float2 run = make_float2(1.f, 1.f);
@@ -692,7 +719,11 @@ __global__ void __launch_bounds__(NT, 2) gla_out_kernel(GlaFwdParams p) {
         float x = sc[nt][e] + sc2[nt][e];
         if (J == I) {
           if (sk > t) x = 0.f;
-          else if (slow) x = 16 * I + t < rows ? diag_score_global(q, k, g, 16 * I + t, 16 * I + sk) : 0.f;
+          else if (slow) {
+            if (16 * I + t >= rows) x = 0.f;
+            else if constexpr (LOGITS) x = diag_score_global(q, k, LogitGates{gz, p.gs}, 16 * I + t, 16 * I + sk);
+            else x = diag_score_global(q, k, LogGates{g}, 16 * I + t, 16 * I + sk);
+          }
         }
         sc[nt][e] = x;
       }
@@ -770,8 +801,10 @@ bool gla_states_scan_wanted(int T) { return (T + C - 1) / C >= kScanMinChunks; }
 cudaError_t launch_gla_states(const GlaFwdParams& p, cudaStream_t s) {
   if (p.B * p.H == 0) return cudaSuccess;
   const int nchunks = (p.T + C - 1) / C;
-  if (p.delta16 && p.decay && nchunks >= kScanMinChunks) {
-    DeltaArgs da{(const bf16*)p.k, (const bf16*)p.v, p.g, (bf16*)p.delta16, p.decay, p.T};
+  if (p.gz && !(p.delta16 && p.decay)) return cudaErrorInvalidValue;  // logits need the scratch
+  if (p.delta16 && p.decay && (nchunks >= kScanMinChunks || p.gz)) {
+    DeltaArgs da{(const bf16*)p.k, (const bf16*)p.v, p.g, (const bf16*)p.gz, p.gs, (bf16*)p.delta16,
+                 p.decay, p.T};
     cudaError_t e = run_delta<false>(da, nchunks, p.B * p.H, "gla_delta_mma", s);
     if (e != cudaSuccess) return e;
     ScanArgs sa{(const bf16*)p.delta16, p.decay, p.h0, (bf16*)p.states16, p.hT, nullptr, nullptr,
@@ -796,7 +829,8 @@ cudaError_t launch_gla_bwd_scan(const GlaBwdScanParams& p, cudaStream_t s) {
   const int BH = p.B * p.H;
   if (BH == 0) return cudaSuccess;
   if (nchunks > 0) {
-    DeltaArgs da{(const bf16*)p.q, (const bf16*)p.dO, p.g, (bf16*)p.delta16, p.decay, p.T};
+    DeltaArgs da{(const bf16*)p.q, (const bf16*)p.dO, p.g, (const bf16*)p.gz, p.gs, (bf16*)p.delta16,
+                 p.decay, p.T};
     cudaError_t e = run_delta<true>(da, nchunks, BH, "gla_bwd_delta", s);
     if (e != cudaSuccess) return e;
   }
@@ -809,7 +843,8 @@ cudaError_t launch_gla_out(const GlaFwdParams& p, cudaStream_t s) {
   const int nchunks = (p.T + C - 1) / C;
   if (p.B * p.H == 0 || nchunks == 0) return cudaSuccess;
   const size_t bytes = sizeof(OutSmem);
-  const auto kern = p.target ? gla_out_kernel<true> : gla_out_kernel<false>;
+  const auto kern = p.target ? (p.gz ? gla_out_kernel<true, true> : gla_out_kernel<true, false>)
+                             : (p.gz ? gla_out_kernel<false, true> : gla_out_kernel<false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
   {

@@ -57,6 +57,10 @@ struct GlaFwdParams {
   void* dO_loss;
   float loss_scale;
   float* loss_part;
+  // gate logits (tensor-core kernels): when set, g is NULL and the log-gate
+  // is gs * log sigma(gz) with gz bf16 [B,H,T,dk]
+  const void* gz;
+  float gs;
 };
 constexpr int kSimtChunk = 16;
 cudaError_t launch_gla_fwd_simt(const GlaFwdParams& p, bool bf16, cudaStream_t s);
@@ -90,6 +94,8 @@ struct GlaBwdParams {
   int B, H, T, dkd, dvd;
   const void* gin16;     // two-level tensor-core backward: launch_gla_bwd_scan's outputs
   const float* gsp;
+  const void* gz;        // gate logits (see GlaFwdParams); dg then receives dL/dz
+  float gs;
 };
 cudaError_t launch_gla_bwd_simt(const GlaBwdParams& p, bool bf16, cudaStream_t s);
 
@@ -122,6 +128,8 @@ struct GlaBwdScanParams {
   float* gsp;            // [BH][nchunks][dk]
   float* dh0;            // nullable
   int B, H, T;
+  const void* gz;        // gate logits (see GlaFwdParams)
+  float gs;
 };
 cudaError_t launch_gla_bwd_scan(const GlaBwdScanParams& p, cudaStream_t s);
 // partial sums the fused loss epilogue writes: one per 64-token chunk and head

@@ -173,6 +173,13 @@ lz_status check_dims(const lz_dims* d, bool need_window) {
     if (d->M < 0 || d->M > 16)
       return fail(LZ_ERR_UNSUPPORTED, "meta tokens M must be in [0, 16] (got %d)", d->M);
   }
+  LZ_REQUIRE(d->gate_logits == 0 || d->gate_logits == 1, "gate_logits must be 0 or 1 (got %d)",
+             d->gate_logits);
+  if (d->gate_logits) {
+    if (d->io != LZ_BF16 || d->dk != 128 || d->dv != 128)
+      return fail(LZ_ERR_UNSUPPORTED, "gate logits need bf16 I/O and dk = dv = 128");
+    LZ_REQUIRE(d->gate_scale > 0.f && d->gate_scale < 3.0e38f, "gate_scale must be finite and > 0");
+  }
   const double elems = (double)d->B * d->H * d->T * (d->dk > d->dv ? d->dk : d->dv);
   LZ_REQUIRE(elems < 9.0e15, "problem too large");
   return LZ_OK;
@@ -192,7 +199,8 @@ size_t states16_count(const lz_dims* d) {
 // (always carved for the two-level backward, whose first step uses it too)
 ScanWs carve_scan(Carver& c, const lz_dims* d, bool always = false) {
   ScanWs w;
-  if (!always && !lz::gla_states_scan_wanted(d->T)) return w;
+  // (gate logits: always, the one-chunk state pass takes only log-gates)
+  if (!always && !d->gate_logits && !lz::gla_states_scan_wanted(d->T)) return w;
   const size_t n64 = (size_t)((d->T + lz::gla_fwd_mma_chunk() - 1) / lz::gla_fwd_mma_chunk());
   w.delta16 = c.take<uint16_t>(states16_count(d));
   w.decay = c.take<float>((size_t)d->B * d->H * n64 * d->dk);
@@ -359,7 +367,13 @@ lz::SwaFwdParams swa_fwd_params(const lz_dims* d, const void* q, const void* k, 
 lz::GlaFwdParams gla_fwd_params(const lz_dims* d, const void* q, const void* k, const void* v,
                                 const float* g, const float* h0) {
   lz::GlaFwdParams p{};
-  p.q = q; p.k = k; p.v = v; p.g = g; p.h0 = h0;
+  p.q = q; p.k = k; p.v = v; p.h0 = h0;
+  if (d->gate_logits) {  // `g` carries bf16 logits
+    p.gz = g;
+    p.gs = d->gate_scale;
+  } else {
+    p.g = g;
+  }
   p.B = d->B; p.H = d->H; p.T = d->T; p.dk = d->dk; p.dv = d->dv;
   return p;
 }
@@ -576,7 +590,13 @@ static cudaError_t gla_bwd_phase1(const lz_dims* d, const void* q, const void* k
     if (e != cudaSuccess) return e;
   }
   p = lz::GlaBwdParams{};
-  p.q = q; p.k = k; p.v = v; p.g = g; p.dO = dO; p.dhT = dhT;
+  p.q = q; p.k = k; p.v = v; p.dO = dO; p.dhT = dhT;
+  if (d->gate_logits) {
+    p.gz = g;
+    p.gs = d->gate_scale;
+  } else {
+    p.g = g;
+  }
   p.states = w.states; p.states16 = states16; p.hT = hT;
   p.add_dq = add_dq; p.add_dk = add_dk; p.add_dv = add_dv;
   p.add_in_place = add_in_place;
@@ -585,7 +605,7 @@ static cudaError_t gla_bwd_phase1(const lz_dims* d, const void* q, const void* k
   if (!mma) return cudaSuccess;
   // two-level: reverse scan of the state gradient
   lz::GlaBwdScanParams sp{};
-  sp.q = q; sp.dO = dO; sp.g = g; sp.states16 = states16; sp.dhT = dhT;
+  sp.q = q; sp.dO = dO; sp.g = p.g; sp.gz = p.gz; sp.gs = p.gs; sp.states16 = states16; sp.dhT = dhT;
   sp.delta16 = w.scan.delta16; sp.decay = w.scan.decay;
   sp.gin16 = w.gin16; sp.gsp = w.gsp; sp.dh0 = dh0;
   sp.B = d->B; sp.H = d->H; sp.T = d->T;

@@ -76,6 +76,15 @@ typedef struct {
   lz_dtype io;    /* dtype of q, k, v, o, meta, dO, dq, dk, dv */
   float scale;    /* softmax logit scale (usually 1/sqrt(dk)); meta logits too */
   float alpha;    /* weight of the window branch in the hybrid sum */
+  int gate_logits;   /* 0: `g` holds fp32 log-gates.  1: `g` holds the gate
+                      * LOGITS z, bf16 [B,H,T,dk] (section 2a: the gate is
+                      * sigma(W_gamma x), z = W_gamma x); the kernels form the
+                      * log-gate gate_scale * log sigma(z) as they load it, and
+                      * the backward's dg receives dL/dz (fp32).  Needs
+                      * io = LZ_BF16 and dk = dv = 128 (LZ_ERR_UNSUPPORTED
+                      * otherwise).  Zero-initialised dims keep mode 0. */
+  float gate_scale;  /* > 0, used when gate_logits = 1 (a temperature; 1 is
+                      * the page's gate) */
 } lz_dims;
 
 /* Bytes of scratch the call needs (0 is possible); `which` is one of the

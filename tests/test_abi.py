@@ -49,7 +49,7 @@ FAKE = 0x7F0000000000  # never dereferenced: validation fails first
 
 def _dims(**kw):
     base = dict(B=1, H=2, T=64, dk=64, dv=64, chunk=64, w=8, M=2, io=L.LZ_BF16, scale=0.125,
-                alpha=0.5)
+                alpha=0.5, gate_logits=0, gate_scale=1.0)
     base.update(kw)
     return L.LzDims(*[base[f] for f, _ in L.LzDims._fields_])
 
@@ -208,3 +208,23 @@ def test_stage1_loss_validation(lib):
     # empty problem: scratch of the partial sums only, no data pointers needed
     e = _dims(T=0)
     assert L.lz_workspace_bytes(e, L.LZ_WS_HYBRID_FWD_MSE) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(gate_logits=1, io=L.LZ_F32, dk=128, dv=128), L.LZ_ERR_UNSUPPORTED),
+    (dict(gate_logits=1, dk=64, dv=64), L.LZ_ERR_UNSUPPORTED),
+    (dict(gate_logits=2, dk=128, dv=128), L.LZ_ERR_INVALID_ARG),
+    (dict(gate_logits=1, dk=128, dv=128, gate_scale=0.0), L.LZ_ERR_INVALID_ARG),
+    (dict(gate_logits=1, dk=128, dv=128, gate_scale=float("nan")), L.LZ_ERR_INVALID_ARG),
+])
+def test_gate_logits_validation(lib, kw, status):
+    assert _call_hybrid(lib, _dims(**kw)) == status
+    assert lib.lz_last_error()
+
+
+def test_gate_logits_workspace(lib):
+    """Gate logits take the two-level state pass for any length, so its
+    scratch is there even for one chunk."""
+    d0 = _dims(dk=128, dv=128, T=64)
+    d1 = _dims(dk=128, dv=128, T=64, gate_logits=1, gate_scale=0.0625)
+    assert L.lz_workspace_bytes(d1, L.LZ_WS_HYBRID_FWD) > L.lz_workspace_bytes(d0, L.LZ_WS_HYBRID_FWD)
