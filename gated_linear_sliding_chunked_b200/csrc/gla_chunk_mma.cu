@@ -8,12 +8,18 @@
 //   S_next = diag(e^{b_l}) S_prev + sum_s (k_s e^{b_l - b_s}) v_s^T
 //   o_t    = (q_t e^{b_t})^T S_prev + sum_{s<=t} A[t][s] v_s,
 //   A[t][s] = sum_i q_t,i k_s,i e^{b_t,i - b_s,i}.
-// Only the state carries a dependence between chunks, so the work is split:
-//   pass 1 (gla_states_kernel): one CTA per (batch, head, 32 value columns)
-//     walks the chunks and writes the bf16 state before every chunk (and the
-//     final fp32 state);
+// Only the state carries a dependence between chunks, and its recurrence
+// over chunks is linear, so the work is split:
+//   pass 1, two levels: gla_delta_kernel<0> forms every chunk's increment
+//     (k e^{b_l - b})^T v and decay e^{b_l} at once; gla_scan_kernel<0> walks
+//     the chunks elementwise and writes the bf16 state before every chunk
+//     (and the final fp32 state).  gla_states_kernel, one CTA per (batch,
+//     head, 32 value columns) walking the chunks with the state in
+//     registers, serves one-chunk sequences;
 //   pass 2 (gla_out_kernel): one CTA per (chunk, batch, head) computes the
 //     chunk's outputs from its incoming state, all chunks in parallel.
+// The backward's first level reuses the pass-1 kernels on the query side
+// (gla_delta_kernel<1>, gla_scan_kernel<1>, launch_gla_bwd_scan).
 // Gate factors are the bounded ones of the single-pass kernel: per key dim
 // one reference row when each 32-row half decays by at most e^-60 ("tame"),
 // else 16-row sub-block references with per-pair factors F_IJ; diagonal
