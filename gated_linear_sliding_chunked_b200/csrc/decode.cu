@@ -36,7 +36,7 @@ __device__ __forceinline__ void load8(const bf16* p, float* x) {
 }
 
 template <typename IO>
-__global__ void __launch_bounds__(NT) decode_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(NT, 5) decode_kernel(DecodeParams p) {
   __shared__ float qs[D], ks[D], vs[D], eg[D];
   __shared__ float red[16][D];
   __shared__ float sc[WMAX + MMAX];
