@@ -807,8 +807,10 @@ bool gla_states_scan_wanted(int T) { return (T + C - 1) / C >= kScanMinChunks; }
 cudaError_t launch_gla_states(const GlaFwdParams& p, cudaStream_t s) {
   if (p.B * p.H == 0) return cudaSuccess;
   const int nchunks = (p.T + C - 1) / C;
-  if (p.gz && !(p.delta16 && p.decay)) return cudaErrorInvalidValue;  // logits need the scratch
-  if (p.delta16 && p.decay && (nchunks >= kScanMinChunks || p.gz)) {
+  // gate logits take the two-level path for every non-empty sequence (the
+  // sequential pass reads log-gates); an empty one only passes h0 to hT
+  if (p.gz && nchunks > 0 && !(p.delta16 && p.decay)) return cudaErrorInvalidValue;
+  if (p.delta16 && p.decay && nchunks > 0 && (nchunks >= kScanMinChunks || p.gz)) {
     DeltaArgs da{(const bf16*)p.k, (const bf16*)p.v, p.g, (const bf16*)p.gz, p.gs, (bf16*)p.delta16,
                  p.decay, p.T};
     cudaError_t e = run_delta<false>(da, nchunks, p.B * p.H, "gla_delta_mma", s);

@@ -99,3 +99,15 @@ def test_gla_fwd_bwd_with_gate_logits_strong_decay():
         for name in ("dq", "dk", "dv", "dh0"):
             assert_close(f"{name} (saved={saved})", b[name], rb[name], torch.bfloat16)
     L.lz_device_check()
+
+
+def test_gate_logits_empty_sequence_keeps_state():
+    """T = 0 with gate logits: no chunk, hT = h0, dh0 = dhT."""
+    cpu, dev, z, x = _case(91, 0)
+    o, hT = L.gla_fwd(dev["q"], dev["k"], dev["v"], z.cuda(), dev["h0"], gate_scale=0.5,
+                      want_hT=True)
+    assert o.numel() == 0
+    assert torch.equal(hT, dev["h0"])
+    b = L.gla_bwd(dev["q"], dev["k"], dev["v"], z.cuda(), dev["dO"], dev["h0"], dev["dhT"],
+                  gate_scale=0.5, want_dh0=True)
+    assert torch.equal(b["dh0"], dev["dhT"])
