@@ -155,7 +155,8 @@ lz_status lz_hybrid_fwd_mse(const lz_dims* d, const void* q, const void* k,
 
 /* Gradient of lz_gla_fwd (needed by the attention-distillation stage,
  * section 2b).  dO = dL/do; dhT (nullable) = dL/dhT.  Writes dq, dk, dv (io
- * dtype), dg (fp32) and dh0 (nullable, fp32).  h0 may be NULL (zeros).
+ * dtype), dg (fp32; dL/dz of the gate logits when d->gate_logits) and dh0
+ * (nullable, fp32).  h0 may be NULL (zeros).
  * chunk_states (nullable): the forward's chunk states for these inputs;
  * with them the backward skips its own state pass, and then hT (the
  * forward's final state) must be given too when dhT is. */
