@@ -228,3 +228,17 @@ def test_gate_logits_workspace(lib):
     d0 = _dims(dk=128, dv=128, T=64)
     d1 = _dims(dk=128, dv=128, T=64, gate_logits=1, gate_scale=0.0625)
     assert L.lz_workspace_bytes(d1, L.LZ_WS_HYBRID_FWD) > L.lz_workspace_bytes(d0, L.LZ_WS_HYBRID_FWD)
+
+
+def test_binding_reads_bf16_gates_as_logits():
+    """The helpers pass fp32 gates as log-gates and bf16 gates as logits."""
+    import torch
+    q = torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16)
+    v = torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16)
+    d = L._dims_from(q, v, chunk=64, w=4, M=0, scale=None, alpha=0.5,
+                     g=torch.zeros(1, 2, 8, 128, dtype=torch.float32))
+    assert d.gate_logits == 0
+    d = L._dims_from(q, v, chunk=64, w=4, M=0, scale=None, alpha=0.5,
+                     g=torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16), gate_scale=0.25)
+    assert d.gate_logits == 1 and abs(d.gate_scale - 0.25) < 1e-7
+    assert L.lz_workspace_bytes(d, L.LZ_WS_HYBRID_BWD) > 0
