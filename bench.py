@@ -237,6 +237,15 @@ def decode_bytes_per_step(dwl) -> float:
     return dwl.Bd * dwl.H * per
 
 
+def train_step_bytes(wl) -> float:
+    """Algorithmic bytes of one hybrid fwd+bwd step: the forward reads q, k, v
+    (I/O size) and g (fp32) and writes o; the backward reads q, k, v, dO, o,
+    g and the LSE and writes dq, dk, dv (I/O size) and dg (fp32)."""
+    e = 2 if wl.io == "bf16" else 4
+    d = wl.dk
+    return wl.B * wl.H * wl.T * ((4 * d * e + 4 * d) + (8 * d * e + 8 * d + 4))
+
+
 def train_flops(wl) -> float:
     """Algorithmic flops of one fwd+bwd step (causal half of intra tiles,
     valid window keys only)."""
@@ -551,7 +560,10 @@ def measure_train_gate_logits(wl, x, device, steps, warmup, seed):
             "kernels": {k: [c // steps, round(t / c, 4)] for k, (c, t) in tab.items()}}
 
 
-def measure_decode(device, steps, warmup, peaks, seed, n_steps=1000):
+def measure_decode(device, peaks, seed, n_steps=1000):
+    """1000 consecutive decode steps (one kernel launch each), captured in one
+    CUDA graph and timed by its replay; per-kernel event times come from a
+    separate eager pass."""
     import gated_linear_sliding_chunked_b200 as L
     from gated_linear_sliding_chunked_b200 import inputs as I
     dwl = I.DECODE
@@ -568,23 +580,38 @@ def measure_decode(device, steps, warmup, peaks, seed, n_steps=1000):
 
     run_all()  # warm-up pass over all steps
     L.lz_timing_enable(True)
-    ms = time_region(run_all, 1, device)
+    eager_ms = time_region(run_all, 1, device)
     L.lz_timing_enable(False)
     tab = kernel_table(L.lz_timing_read())
+    launches_per_step = sum(c for c, _ in tab.values()) / n_steps
+    side = torch.cuda.Stream(device)
+    side.wait_stream(torch.cuda.current_stream(device))
+    torch.cuda.synchronize(device)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        run_all()
+    graph.replay()  # warm-up replay
+    ms = time_region(graph.replay, 1, device)
     per_step_ms = ms / n_steps
     bytes_step = decode_bytes_per_step(dwl)
+    ach = bytes_step / (per_step_ms * 1e-3) / 1e9
     c, t = tab.get("decode_step", (1, per_step_ms))
     k_ms = t / c
-    ach = bytes_step / (k_ms * 1e-3) / 1e9
-    del st, toks
+    del graph, st, toks
     return {"workload": dwl.name, "steps": n_steps,
+            "timing": f"{n_steps} steps captured in one CUDA graph, one replay timed "
+                      "(CUDA events); no per-launch events inside",
+            "launches_per_step": launches_per_step,
             "tokens_per_s": dwl.Bd / (per_step_ms * 1e-3), "ms_per_step": round(per_step_ms, 5),
+            "eager_ms_per_step_with_launch_events": round(eager_ms / n_steps, 5),
             "kernels": {k: [c2 // n_steps, round(t2 / c2, 5)] for k, (c2, t2) in tab.items()},
-            "roofline": {"kernel": "decode_step", "bound": "hbm", "achieved": round(ach, 1),
-                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "kernel_avg_ms": round(k_ms, 5),
+            "roofline": {"kernel": "decode step (graph replay, whole step)", "bound": "hbm",
+                         "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(ach / peaks["hbm_gbs"], 4),
-                         "algorithmic_bytes_per_launch": bytes_step,
-                         "avg_ms": round(k_ms, 5)}}
+                         "algorithmic_bytes_per_step": bytes_step,
+                         "avg_ms": round(per_step_ms, 5),
+                         "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs copy)"}}
 
 
 # --------------------------------------------------------------------------
@@ -608,27 +635,57 @@ def oracle_train_step(small, xs, nthreads):
     return fwd
 
 
-def cpu_baseline(wl, budget_s=20.0):
-    """Time the oracle as it stands on this host's cores on a bounded sample;
-    report tokens/s in the workload's units (a token = one position over all
-    H heads, so a sample of P head-sequences of T tokens is P*T/H tokens)."""
-    cores = os.cpu_count() or 1
-    pairs = max(1, min(cores, 16))
-    T = 1024
-    small, xs = oracle_sample(wl, pairs, T)
-    t0 = time.perf_counter()
-    oracle_train_step(small, xs, pairs)
-    dt = time.perf_counter() - t0
-    reps = 1
-    while time.perf_counter() - t0 < min(budget_s, 4 * dt) and reps < 3:
+def host_cpu():
+    """(logical cores, CPU model) of this host."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return os.cpu_count() or 1, model
+
+
+ORACLE_T = 2048  # tokens per (batch, head) problem of the oracle's sample
+
+
+def oracle_timer(wl):
+    """The oracle's bounded sample of the training workload and a function
+    that runs one fwd+bwd over it: one (batch, head) problem of the first
+    ORACLE_T tokens per host core, every core a thread (std::thread inside the
+    oracle).  Both the CPU baseline and the reference arm use it, so they
+    time the same program on the same sample."""
+    cores, model = host_cpu()
+    pairs = cores
+    small, xs = oracle_sample(wl, pairs, ORACLE_T)
+    tokens = pairs * ORACLE_T / wl.H  # a token = one position over all H heads
+
+    def run():
         oracle_train_step(small, xs, pairs)
+
+    desc = (f"{pairs} (batch, head) problems x first {ORACLE_T} tokens of the training "
+            f"workload ({wl.name}), fwd+bwd in fp64, {pairs} threads (one per core) on "
+            f"{cores} cores of '{model}'; tokens = problems*T/H")
+    return run, tokens, pairs, cores, model, desc
+
+
+def cpu_baseline(wl, min_s=12.0, max_reps=100):
+    """Time the oracle as it stands on this host's cores on its bounded
+    sample, repeated until about min_s seconds of work; tokens/s in the
+    workload's units."""
+    run, tokens, threads, cores, model, desc = oracle_timer(wl)
+    t0 = time.perf_counter()
+    reps = 0
+    while reps < max_reps and (reps == 0 or time.perf_counter() - t0 < min_s):
+        run()
         reps += 1
     wall = (time.perf_counter() - t0) / reps
-    tokens = pairs * T / wl.H
-    return {"value": tokens / wall, "unit": "tokens/s", "cores": pairs, "kind": "oracle",
-            "sample": f"{pairs} (batch, head) problems x first {T} tokens of the training "
-                      f"workload, fwd+bwd, fp64, std::thread over pairs; {reps} rep(s), "
-                      f"{wall:.2f} s each; tokens = pairs*T/H"}
+    return {"value": tokens / wall, "unit": "tokens/s", "cores": threads, "nproc": cores,
+            "cpu_model": model, "kind": "oracle",
+            "sample": f"{desc}; {reps} rep(s), {wall:.2f} s each"}
 
 
 def run_reference(args):
@@ -637,17 +694,13 @@ def run_reference(args):
     if rank != 0:
         return 0
     wl = I.TRAIN_BF16
-    cores = os.cpu_count() or 1
-    pairs = max(1, min(cores, 8))
-    T = 512
-    small, xs = oracle_sample(wl, pairs, T)
+    run, tokens, threads, cores, model, desc = oracle_timer(wl)
     for _ in range(args.warmup):
-        oracle_train_step(small, xs, pairs)
+        run()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_train_step(small, xs, pairs)
+        run()
     wall = (time.perf_counter() - t0) / max(args.steps, 1)
-    tokens = pairs * T / wl.H
     val = tokens / wall
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
             "higher_is_better": True, "n_gpus": args.gpus, "steps": args.steps,
@@ -655,9 +708,9 @@ def run_reference(args):
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": wl.name, "global_batch": wl.B, "seq_len": wl.T,
                        "parallelism": "host cores (oracle)"},
-            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": pairs, "kind": "oracle",
-                             "sample": f"{pairs} (batch, head) problems x first {T} tokens per "
-                                       f"step, fwd+bwd in fp64; tokens = pairs*T/H"},
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": threads, "nproc": cores,
+                             "cpu_model": model, "kind": "oracle",
+                             "sample": f"{desc}; one pass per step"},
             "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -784,6 +837,17 @@ def main(argv=None):
     launches = len(records)
     dom, roof = roofline_for(tab, wl, peaks)
     flops = train_flops(wl)
+    # the whole step against its attainable roofline max(F / P_tc, bytes / BW)
+    sbytes = train_step_bytes(wl)
+    t_hbm = sbytes / (peaks["hbm_gbs"] * 1e9) * 1e3
+    t_tc = flops / (peaks["bf16_tflops_sustained"] * 1e12) * 1e3
+    step_roof = {"bound": "hbm" if t_hbm >= t_tc else "tensor",
+                 "achieved": round(sbytes / (ms_max * 1e-3) / 1e9, 1), "peak": peaks["hbm_gbs"],
+                 "unit": "GB/s", "frac": round(max(t_hbm, t_tc) / ms_max, 4),
+                 "algorithmic_bytes_per_step": sbytes, "flops_per_step": flops,
+                 "t_roof_ms": round(max(t_hbm, t_tc), 4),
+                 "note": "whole fwd+bwd step; frac = max(F / sustained bf16 peak, "
+                         "bytes / HBM copy bandwidth) / measured step time"}
 
     # ---- end to end through the C ABI with host buffers --------------------
     in_keys = ("q", "k", "v", "g", "meta_k", "meta_v", "dO")
@@ -804,7 +868,7 @@ def main(argv=None):
                                                                seed=rank, tcgen05_window=False)
         extras["long_T65536_warp_mma_window"] = measure_fwd(I.LONG_BF16, device, 3, 1, peaks,
                                                             seed=rank, tcgen05_window=False)
-        extras["decode"] = measure_decode(device, 1, 1, peaks, seed=rank)
+        extras["decode"] = measure_decode(device, peaks, seed=rank)
         extras["train_step_breakdown"] = {k: [c // args.steps, round(t / c, 4)]
                                           for k, (c, t) in tab.items()}
         extras["train_step_breakdown_note"] = (
@@ -831,6 +895,7 @@ def main(argv=None):
                        "parallelism": f"replicas x{world} (no data-path collective)",
                        "l2": "inputs larger than L2 (~0.8 GB read per step), no flush"},
             "roofline": roof,
+            "step_roofline": step_roof,
             "effective_tflops": flops / (ms_max * 1e-3) / 1e12,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,

@@ -82,7 +82,7 @@ def load(path: str = LIB_PATH):
                                        [_P] * 11 + [_P])
     lib.lz_device_check.argtypes = [_P]
     lib.lz_selftest_bounded_wait.argtypes = [_P]
-    lib.lz_decode_prefill.argtypes = [ctypes.c_int] * 7 + [_P] * 7 + [_P]
+    lib.lz_decode_prefill.argtypes = [ctypes.c_int] * 7 + [_P] * 8 + [_P]
     lib.lz_prefer_tcgen05.argtypes = [ctypes.c_int]
     lib.lz_timing_enable.argtypes = [ctypes.c_int]
     lib.lz_timing_read.argtypes = [ctypes.c_char_p, sz, ctypes.POINTER(ctypes.c_float),
@@ -398,24 +398,31 @@ def hybrid_bwd(q, k, v, g, meta_k, meta_v, lse, dO, *, w, alpha, scale=None, chu
             "dmeta_v": dmv, "dalpha": dalpha[:1]}
 
 
-def lz_decode_prefill(Bd, H, T, dk, dv, w, io, k, v, hT, state, kring, vring, pos, stream=None):
-    _check(load().lz_decode_prefill(Bd, H, T, dk, dv, w, io, _ptr(k), _ptr(v), _ptr(hT),
-                                    _ptr(state), _ptr(kring), _ptr(vring), _ptr(pos),
+def lz_decode_prefill(Bd, H, T, dk, dv, w, io, k, v, lens, hT, state, kring, vring, pos,
+                      stream=None):
+    _check(load().lz_decode_prefill(Bd, H, T, dk, dv, w, io, _ptr(k), _ptr(v), _ptr(lens),
+                                    _ptr(hT), _ptr(state), _ptr(kring), _ptr(vring), _ptr(pos),
                                     _stream(stream)))
 
 
-def decode_prefill(k, v, hT, *, w, stream=None):
+def decode_prefill(k, v, hT, *, w, lens=None, stream=None):
     """Decode buffers after a prefill of k, v [Bd, H, T, 128] with final state
-    hT: returns (state, kring, vring, pos) ready for decode_step."""
+    hT: returns (state, kring, vring, pos) ready for decode_step.  lens: an
+    int64 tensor [Bd] of per-sequence prompt lengths (right-padded prompts,
+    padding with k = 0 and g = 0), or None for T each."""
     Bd, H, T, dk = k.shape
     dv = v.shape[-1]
     dev = k.device
+    if lens is not None:
+        lens = lens.to(device=dev, dtype=torch.int64).contiguous()
+        if lens.shape != (Bd,):
+            raise ValueError(f"lens must have shape ({Bd},), got {tuple(lens.shape)}")
     state = torch.empty(Bd, H, dk, dv, dtype=torch.float32, device=dev)
     kring = torch.zeros(Bd, H, w, dk, dtype=k.dtype, device=dev)
     vring = torch.zeros(Bd, H, w, dv, dtype=v.dtype, device=dev)
     pos = torch.empty(Bd, dtype=torch.int64, device=dev)
-    lz_decode_prefill(Bd, H, T, dk, dv, w, io_of(k.dtype), k, v, hT, state, kring, vring, pos,
-                      stream)
+    lz_decode_prefill(Bd, H, T, dk, dv, w, io_of(k.dtype), k, v, lens, hT, state, kring, vring,
+                      pos, stream)
     return state, kring, vring, pos
 
 

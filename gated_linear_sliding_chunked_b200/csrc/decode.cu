@@ -6,6 +6,13 @@
 // 128x128 fp32 state once in and once out (128-bit loads/stores, 16 rows x 4
 // columns per thread), reads the w-slot K/V ring and the M meta tokens once,
 // and writes one output row.  It is bound by HBM bandwidth.
+//
+// The step is one launch: the H CTAs of a sequence read and advance its
+// position through one 64-bit atomic on pos[b], whose bits 48 and up count
+// the CTAs of the current step that have read it.  A CTA adds 2^48 and takes
+// the position from the low bits of the old value; the H-th arrival writes
+// position + 1 with a clear count.  Between steps the word is the plain
+// position.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -16,6 +23,8 @@ constexpr int D = 128;
 constexpr int NT = 256;
 constexpr int WMAX = 1024;
 constexpr int MMAX = 16;
+constexpr int kPosBits = 48;  // position bits of pos[b]; the arrival count sits above
+constexpr unsigned long long kPosMask = (1ull << kPosBits) - 1;
 
 __device__ __forceinline__ void load8(const float* p, float* x) {
   const float4 a = *reinterpret_cast<const float4*>(p);
@@ -41,14 +50,17 @@ __global__ void __launch_bounds__(NT, 5) decode_kernel(DecodeParams p) {
   __shared__ float red[16][D];
   __shared__ float sc[WMAX + MMAX];
   __shared__ float stat[2];
+  __shared__ long long spos;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
   const int w = p.w, M = p.M;
-  int64_t pos = p.pos[b];
-  if (pos < 0) pos = 0;  // negative positions are treated as an empty history
-  const int slot = (int)(pos % w);
-  const int nwin = (int)((pos + 1) < (int64_t)w ? (pos + 1) : (int64_t)w);
-
+  if (tid == 0) {  // read the position and count this CTA in (one atomic)
+    unsigned long long* pw = reinterpret_cast<unsigned long long*>(p.pos + b);
+    const unsigned long long old = atomicAdd(pw, 1ull << kPosBits);
+    const unsigned long long cur = old & kPosMask;
+    if ((old >> kPosBits) == (unsigned long long)(p.H - 1)) atomicExch(pw, cur + 1);  // last of the H
+    spos = (long long)cur;
+  }
   if (tid < D) {
     const size_t off = (size_t)bh * D + tid;
     qs[tid] = ldf((const IO*)p.q + off);
@@ -57,6 +69,9 @@ __global__ void __launch_bounds__(NT, 5) decode_kernel(DecodeParams p) {
     eg[tid] = expf(p.g[off]);
   }
   __syncthreads();
+  const long long pos = spos;
+  const int slot = (int)(pos % w);
+  const int nwin = (int)((pos + 1) < (long long)w ? (pos + 1) : (long long)w);
 
   // ---- gated state: S <- diag(e^g) S + k v^T ; o_gla = q^T S -------------
   {
@@ -182,33 +197,34 @@ __global__ void __launch_bounds__(NT, 5) decode_kernel(DecodeParams p) {
 }
 
 // Prefill -> decode hand-off: the state becomes the prefill's final state,
-// the ring slot t mod w holds token t of the last min(T, w) prompt tokens,
-// pos = T.  One CTA per (sequence, head).
+// the ring slot t mod w holds token t of the last min(L, w) prompt tokens,
+// pos = L, with L = T or the sequence's own prompt length (lens[b], clamped
+// to [0, T]).  One CTA per (sequence, head).
 template <typename IO>
 __global__ void __launch_bounds__(NT) decode_prefill_kernel(DecodePrefillParams p) {
   const int tid = threadIdx.x;
   const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
   const int T = p.T, w = p.w;
+  int L = T;
+  if (p.lens) {
+    const long long l = p.lens[b];
+    L = l < 0 ? 0 : (l > T ? T : (int)l);
+  }
   float4* st = reinterpret_cast<float4*>(p.state + (size_t)bh * D * D);
   const float4* src = p.hT ? reinterpret_cast<const float4*>(p.hT + (size_t)bh * D * D) : nullptr;
   for (int x = tid; x < D * D / 4; x += NT) st[x] = src ? src[x] : make_float4(0.f, 0.f, 0.f, 0.f);
-  const int t0 = T > w ? T - w : 0;
+  const int t0 = L > w ? L - w : 0;
   constexpr int CH = D * (int)sizeof(IO) / 16;  // 16-byte chunks per row
   const uint4* ks = reinterpret_cast<const uint4*>((const IO*)p.k + (size_t)bh * T * D);
   const uint4* vs = reinterpret_cast<const uint4*>((const IO*)p.v + (size_t)bh * T * D);
   uint4* kr = reinterpret_cast<uint4*>((IO*)p.kring + (size_t)bh * w * D);
   uint4* vr = reinterpret_cast<uint4*>((IO*)p.vring + (size_t)bh * w * D);
-  for (int x = tid; x < (T - t0) * CH; x += NT) {
+  for (int x = tid; x < (L - t0) * CH; x += NT) {
     const int t = t0 + x / CH, c = x % CH, slot = t % w;
     kr[(size_t)slot * CH + c] = ks[(size_t)t * CH + c];
     vr[(size_t)slot * CH + c] = vs[(size_t)t * CH + c];
   }
-  if (h == 0 && tid == 0) p.pos[b] = T;
-}
-
-__global__ void decode_pos_kernel(int64_t* pos, int Bd) {
-  const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b < Bd) pos[b] = (pos[b] < 0 ? 0 : pos[b]) + 1;
+  if (h == 0 && tid == 0) p.pos[b] = L;
 }
 
 }  // namespace
@@ -229,12 +245,6 @@ cudaError_t launch_decode(const DecodeParams& p, bool bf16, cudaStream_t s) {
     ScopedTiming tm("decode_step", s);
     if (bf16) decode_kernel<lz::bf16><<<p.Bd * p.H, NT, 0, s>>>(p);
     else decode_kernel<float><<<p.Bd * p.H, NT, 0, s>>>(p);
-  }
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  {
-    ScopedTiming tm("decode_pos", s);
-    decode_pos_kernel<<<(p.Bd + 255) / 256, 256, 0, s>>>(p.pos, p.Bd);
   }
   return cudaGetLastError();
 }

@@ -17,6 +17,16 @@
 //          the chunk dg_t = dg_first - sum_{u<t} (q_u dq_u - k_u dk_u), so
 //          rounding errors add up over one chunk, not the whole sequence.
 //
+// The running sum cancels: every intra-chunk pair (u, s) enters q_u dq_u and
+// k_s dk_s with the same value, and only the pairs that straddle t survive.
+// Under fast forgetting the surviving part is small, so the two copies of a
+// pair must round identically.  Hence (a) the diagonal pairs (s = u, whose
+// copies cancel exactly) stay out of the MMAs and are added to dq and dk in
+// fp32 only, and (b) the products entering the sum are taken from the bf16
+// MMA operands themselves, Qf_u * acc_q,u and Kf_s * acc_k,s, in which a pair
+// is the same product Qf_u B[u][s] Kf_s on both sides, instead of q * dq and
+// k * dk, whose output scales round differently on the two sides.
+//
 // Two levels: launch_gla_bwd_scan (gla_chunk_mma.cu) forms every chunk's
 // increment of G in parallel and scans them in reverse, giving G and
 // <G_new, S_prev> for every chunk; the kernel here then takes all chunks at
@@ -91,9 +101,9 @@ __device__ __noinline__ float gate_ratio(Gates g, int rows, int t, int s, int i)
 }
 
 struct ChunkSmem {
-  bf16 v[C * VP];       // then k * dk (fp32, rsw layout)
+  bf16 v[C * VP];       // then the k-side dg products (fp32, rsw layout)
   bf16 dO[C * VP];
-  bf16 sp[DKH * DV];    // S_prev (swizzled); then q * dq (fp32, rsw layout)
+  bf16 sp[DKH * DV];    // S_prev (swizzled); then the q-side dg products (fp32, rsw)
   bf16 g16[DKH * DV];   // G entering the chunk (swizzled)
   bf16 qf[C * KP];      // qf and kf: then the peer's dv share (fp32, rsw layout)
   bf16 kf[C * KP];
@@ -107,20 +117,21 @@ struct ChunkSmem {
   float tot[NSB][DKH];
 };
 static_assert(sizeof(ChunkSmem) + 1024 <= 232448 / 2, "two chunk CTAs must fit one SM");
-static_assert(sizeof(float) * C * RP <= sizeof(bf16) * C * VP, "k*dk staging must fit the v tile");
-static_assert(sizeof(float) * C * RP <= sizeof(bf16) * DKH * DV, "q*dq staging must fit the state tile");
+static_assert(sizeof(float) * C * RP <= sizeof(bf16) * C * VP, "dg staging must fit the v tile");
+static_assert(sizeof(float) * C * RP <= sizeof(bf16) * DKH * DV, "dg staging must fit the state tile");
 static_assert(sizeof(float) * C * RP <= 2 * sizeof(bf16) * C * KP, "dv share must fit qf + kf");
 
-// Diagonal-block intra term of a strong-decay chunk at (row t, key dim il):
-// role 0 (dq): sum_{s in block, s <= t} (dO_t . v_s) k_s,il exp(b_t - b_s)
-// role 1 (dk): sum_{u in block, u >= t} (dO_u . v_t) q_u,il exp(b_u - b_t)
+// Diagonal-block intra term of a strong-decay chunk at (row t, key dim il),
+// without the pair s = u = t (added separately, in fp32, for every chunk):
+// role 0 (dq): sum_{s in block, s < t} (dO_t . v_s) k_s,il exp(b_t - b_s)
+// role 1 (dk): sum_{u in block, u > t} (dO_u . v_t) q_u,il exp(b_u - b_t)
 // (dO, v: shared tiles; kq, g: global, the chunk's first row, offset to this
 // CTA's key dims)
 template <class Gates>
 __device__ __noinline__ float diag_intra_term(const bf16* dO, const bf16* v, const bf16* kq, Gates g,
                                               int rows, int I, int t, int il, int role) {
   float x = 0.f;
-  const int lo = role == 0 ? SB * I : t, hi = role == 0 ? t : SB * I + SB - 1;
+  const int lo = role == 0 ? SB * I : t + 1, hi = role == 0 ? t - 1 : SB * I + SB - 1;
   for (int r = lo; r <= hi && r < rows; ++r) {
     const int rq = role == 0 ? t : r, rv = role == 0 ? r : t;
     float b = 0.f;
@@ -172,8 +183,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
   Gates gsrc;
   if constexpr (LOGITS) gsrc = LogitGates{gzc, p.gs};
   else gsrc = LogGates{gch};
-  float* stq = reinterpret_cast<float*>(sm.sp);   // q * dq
-  float* stk = reinterpret_cast<float*>(sm.v);    // k * dk
+  float* stq = reinterpret_cast<float*>(sm.sp);   // Qf * acc_q (q dq without the diagonal pairs)
+  float* stk = reinterpret_cast<float*>(sm.v);    // Kf * acc_k
   float* xch = reinterpret_cast<float*>(sm.qf);   // the peer's dv share
   float* peer_xch = cluster.map_shared_rank(xch, half ^ 1);
 
@@ -371,6 +382,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
   }
   // ---- intra: one 16x16 score block at a time, consumed right away -------
   const int jlo = role == 0 ? 0 : I, jhi = role == 0 ? I : NSB - 1;
+  float bdiag[2] = {0.f, 0.f};  // fp32 dO_t . v_t of rows 16I + gr and 16I + gr + 8
   for (int J = jlo; J <= jhi; ++J) {
     float sc[2][4], sc2[2][4];  // two partial sums over k for independent MMA chains
 #pragma unroll
@@ -400,13 +412,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
 #pragma unroll
       for (int e = 0; e < 4; ++e) sc[nt][e] += sc2[nt][e];
     if (J == I) {
+      // the diagonal (t, t) of row gr (gr + 8) sits in lane 4 gr + gr / 2,
+      // fragment element (gr & 1) of column tile 0 (1)
+      const int src = gr * 4 + (gr >> 1);
+      bdiag[0] = __shfl_sync(0xffffffffu, (gr & 1) ? sc[0][1] : sc[0][0], src);
+      bdiag[1] = __shfl_sync(0xffffffffu, (gr & 1) ? sc[1][3] : sc[1][2], src);
       if (slow) continue;  // the diagonal block of a strong-decay chunk: below
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int t = gr + (e >> 1) * 8, u = nt * 8 + gc + (e & 1);
-          if (role == 0 ? (u > t) : (u < t)) sc[nt][e] = 0.f;
+          if (role == 0 ? (u >= t) : (u <= t)) sc[nt][e] = 0.f;
         }
     }
     const uint32_t pa[4] = {pack_bf16(sc[0][0], sc[0][1]), pack_bf16(sc[0][2], sc[0][3]),
@@ -429,9 +446,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
       mma_bf16(acc[2 * ntp + 1], pa, b2, b3);
     }
   }
-  // ---- finalize (dq | dk) = (Eq | Ek) * acc, store; keep (q dq | k dk) -----
+  // ---- finalize (dq | dk) = (Eq | Ek) * acc + diagonal, store; keep the
+  // products (Qf acc_q | Kf acc_k) for dg -----------------------------------
   {
-    const bf16* raw = role == 0 ? qc : kc;
+    const bf16* raw = role == 0 ? kc : qc;  // the other factor of the diagonal pair
+    const bf16* same = role == 0 ? qc : kc;
+    const bf16* fop = role == 0 ? sm.qf : sm.kf;
     bf16* outp = (bf16*)(role == 0 ? p.dq : p.dk);
     const float* addf = role == 0 ? p.add_dq : p.add_dk;
     // two rounds of four column tiles; each round issues its global loads
@@ -459,10 +479,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
           const int t = 16 * I + gr + 8 * hh;
           const int il = nt * 8 + gc;
           const float2 os = unpack_bf16(*reinterpret_cast<const uint32_t*>(&oscale[t * KP + il]));
-          float x0 = acc[nt][2 * hh] * os.x, x1 = acc[nt][2 * hh + 1] * os.y;
+          const float2 fq = unpack_bf16(*reinterpret_cast<const uint32_t*>(&fop[t * KP + il]));
+          const float2 xo = unpack_bf16(rv[n][hh]);
+          const float a0 = acc[nt][2 * hh], a1 = acc[nt][2 * hh + 1];
+          float p0 = fq.x * a0, p1 = fq.y * a1;
+          float x0 = a0 * os.x + bdiag[hh] * xo.x, x1 = a1 * os.y + bdiag[hh] * xo.y;
           if (slow) {
-            x0 += diag_intra_term(sm.dO, sm.v, role == 0 ? kc : qc, gsrc, rows, I, t, il, role);
-            x1 += diag_intra_term(sm.dO, sm.v, role == 0 ? kc : qc, gsrc, rows, I, t, il + 1, role);
+            const float d0 = diag_intra_term(sm.dO, sm.v, raw, gsrc, rows, I, t, il, role);
+            const float d1 = diag_intra_term(sm.dO, sm.v, raw, gsrc, rows, I, t, il + 1, role);
+            x0 += d0;
+            x1 += d1;
+            if (t < rows) {
+              const float2 sv =
+                  unpack_bf16(__ldg(reinterpret_cast<const unsigned int*>(&same[(size_t)t * DK + il])));
+              p0 += sv.x * d0;
+              p1 += sv.y * d1;
+            }
           }
           if (t < rows) {
             const size_t off = tk + (size_t)(c0 + t) * DK + i0 + il;
@@ -478,9 +510,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
             }
             *reinterpret_cast<uint32_t*>(&outp[off]) = pack_bf16(y0, y1);
           }
-          const float2 xv = unpack_bf16(rv[n][hh]);
-          acc[nt][2 * hh] = xv.x * x0;
-          acc[nt][2 * hh + 1] = xv.y * x1;
+          acc[nt][2 * hh] = p0;
+          acc[nt][2 * hh + 1] = p1;
         }
     }
   }
@@ -602,7 +633,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
     float loc[SB];
     float run = 0.f;
 #pragma unroll
-    for (int r = 0; r < SB; ++r) {  // exclusive prefix of q*dq - k*dk
+    for (int r = 0; r < SB; ++r) {  // exclusive prefix of the q-side minus the k-side products
       loc[r] = run;
       run += stq[rsw(16 * qq + r, col)] - stk[rsw(16 * qq + r, col)];
     }

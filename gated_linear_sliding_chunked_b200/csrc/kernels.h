@@ -242,6 +242,7 @@ struct DecodePrefillParams {
   void* kring;
   void* vring;
   int64_t* pos;
+  const int64_t* lens;  // [Bd] prompt lengths, nullable = all T
 };
 cudaError_t launch_decode_prefill(const DecodePrefillParams& p, bool bf16, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams& p, bool bf16, cudaStream_t s);

@@ -393,6 +393,11 @@ lz::SwaBwdParams swa_bwd_params(const lz_dims* d, const void* q, const void* k, 
 
 }  // namespace
 
+namespace lz {
+// Shape and dtype checks of the window entry points (records the error).
+int check_window_dims(const lz_dims* d) { return check_dims(d, true); }
+}  // namespace lz
+
 extern "C" {
 
 const char* lz_last_error(void) { return g_err.c_str(); }
@@ -744,8 +749,9 @@ lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const vo
 }
 
 lz_status lz_decode_prefill(int Bd, int H, int T, int dk, int dv, int w, lz_dtype io,
-                            const void* k, const void* v, const float* hT, float* state,
-                            void* kring, void* vring, int64_t* pos, lz_stream stream) {
+                            const void* k, const void* v, const int64_t* lens, const float* hT,
+                            float* state, void* kring, void* vring, int64_t* pos,
+                            lz_stream stream) {
   LZ_REQUIRE(Bd >= 0 && H >= 0 && T >= 0, "Bd, H, T must be >= 0 (got %d, %d, %d)", Bd, H, T);
   if (io != LZ_F32 && io != LZ_BF16)
     return fail(LZ_ERR_UNSUPPORTED, "io dtype %d is not LZ_F32 or LZ_BF16", (int)io);
@@ -754,11 +760,12 @@ lz_status lz_decode_prefill(int Bd, int H, int T, int dk, int dv, int w, lz_dtyp
   if (w < 1 || w > 1024) return fail(LZ_ERR_UNSUPPORTED, "w must be in [1, 1024] (got %d)", w);
   const bool nz = (size_t)Bd * H > 0;
   const bool nzt = nz && T > 0;
-  LZ_PTR(k, nzt); LZ_PTR(v, nzt); LZ_PTR(hT, false);
+  LZ_PTR(k, nzt); LZ_PTR(v, nzt); LZ_PTR(hT, false); LZ_PTR(lens, false);
   LZ_PTR(state, nz); LZ_PTR(kring, nz); LZ_PTR(vring, nz); LZ_PTR(pos, Bd > 0);
   lz::DecodePrefillParams p{};
   p.Bd = Bd; p.H = H; p.T = T; p.w = w;
   p.k = k; p.v = v; p.hT = hT; p.state = state; p.kring = kring; p.vring = vring; p.pos = pos;
+  p.lens = lens;
   return cuda_status(lz::launch_decode_prefill(p, io == LZ_BF16, as_stream(stream)),
                      "lz_decode_prefill");
 }
@@ -773,6 +780,7 @@ lz_status lz_gla_decode_step(int Bd, int H, int dk, int dv, int w, int M, lz_dty
     return fail(LZ_ERR_UNSUPPORTED, "io dtype %d is not LZ_F32 or LZ_BF16", (int)io);
   if (dk != 128 || dv != 128)
     return fail(LZ_ERR_UNSUPPORTED, "decode supports dk = dv = 128 (got %d, %d)", dk, dv);
+  if (H > 32767) return fail(LZ_ERR_UNSUPPORTED, "decode supports H <= 32767 (got %d)", H);
   if (w < 1 || w > 1024) return fail(LZ_ERR_UNSUPPORTED, "w must be in [1, 1024] (got %d)", w);
   if (M < 0 || M > 16) return fail(LZ_ERR_UNSUPPORTED, "M must be in [0, 16] (got %d)", M);
   const bool nz = (size_t)Bd * H > 0;  // empty tensors may have NULL data

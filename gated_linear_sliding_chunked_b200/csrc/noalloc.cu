@@ -20,6 +20,12 @@
 #include "../../include/lizard.h"
 #include "kernels.h"
 
+namespace lz {
+// The window entry points' checks of a dims struct (lizard_api.cu): LZ_OK, or
+// the status they return, with the error recorded.
+int check_window_dims(const lz_dims* d);
+}  // namespace lz
+
 namespace {
 
 constexpr size_t kScratchBytes = LZ_NOALLOC_SCRATCH_BYTES;
@@ -37,10 +43,9 @@ extern "C" lz_status lz_swa_meta_bwd_noalloc(const lz_dims* d, const void* q, co
                                             const void* o, const void* dO, void* dq,
                                             void* dk, void* dv,
                                             float* dmeta_k, float* dmeta_v, lz_stream stream) {
-  if (d == nullptr)
-    return (lz_status)lz::set_last_error(LZ_ERR_INVALID_ARG, "dims must not be NULL");
-  // lz_workspace_bytes returns 0 for invalid dims; lz_swa_meta_bwd then
-  // reports the precise shape error below.
+  // shapes first, so that a bad call touches no device state
+  const int chk = lz::check_window_dims(d);
+  if (chk != LZ_OK) return (lz_status)chk;
   const size_t need = lz_workspace_bytes(d, LZ_WS_SWA_BWD);
   if (need > kScratchBytes) {
     char msg[256];
@@ -63,9 +68,13 @@ extern "C" lz_status lz_swa_meta_bwd_noalloc(const lz_dims* d, const void* q, co
     std::lock_guard<std::mutex> lock(g_mu);
     auto it = g_addr.find(dev);
     if (it == g_addr.end()) {
-      // First call on this device: look up the array's device address (this
-      // may load the module onto the device, so it must not happen inside a
-      // stream capture).
+      // First call on this device: look up the array's device address.  With
+      // lazy module loading (the CUDA 12 default) this is also where the
+      // module, and with it the 16 MiB array, is loaded onto the device, so it
+      // can fail if the device's memory is exhausted, and it must not happen
+      // inside a stream capture.  The address stays valid until the process
+      // exits or the device is reset (cudaDeviceReset unloads the module:
+      // after that this entry point must not be used in the process).
       e = cudaGetSymbolAddress(&scratch, g_swa_bwd_scratch);
       if (e != cudaSuccess || scratch == nullptr) {
         char msg[256];

@@ -195,7 +195,14 @@ lz_status lz_swa_meta_bwd(const lz_dims* d, const void* q, const void* k,
  *
  * The first call on a device (the device current on the calling thread,
  * which must be the stream's device) looks up the array's device address
- * once; make that first call before any stream capture.  All calls share
+ * once; make that first call before any stream capture.  With lazy module
+ * loading (the CUDA 12 default) that first call is also where the library's
+ * module, and with it the 16 MiB array, is loaded onto the device: it can
+ * fail with LZ_ERR_CUDA if the device's memory is exhausted, so a caller
+ * that pools all device memory should make it before reserving its pool.
+ * Later calls reserve nothing more.  After cudaDeviceReset the array is gone
+ * and this entry point must not be used again in the process.  Invalid
+ * dims are rejected before the device is touched.  All calls share
  * the one array: calls that may overlap on the GPU (different streams, or
  * several host threads, on the same device) race and must be serialized by
  * the caller.  The array keeps the previous call's contents; every part of
@@ -237,9 +244,15 @@ lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k,
  * Per sequence with p = pos[b]: k, v go to ring slot p mod w; the state is
  * decayed by exp(g) and gets k v^T; o_gla = q^T S; the window is the last
  * min(p+1, w) tokens (the new one included) plus the M meta tokens; o =
- * o_gla + alpha * o_swa; pos[b] = p + 1.
+ * o_gla + alpha * o_swa; pos[b] = p + 1.  Sequences may sit at different
+ * positions.  One kernel launch per call: the H blocks of a sequence read
+ * and advance pos[b] with 64-bit atomics, using its bits 48..62 as an arrival
+ * count during the call, so pos[b] must lie in [0, 2^48) and 8-byte aligned
+ * (a value outside that range gives undefined results, with every memory
+ * access still in bounds); calls that overlap on the GPU and share pos race.
  *   q, k [Bd,H,dk], v, o [Bd,H,dv] io dtype; g [Bd,H,dk] fp32.  meta_v NULL
- *   = sink-only.  Supported: dk = dv = 128, io = LZ_BF16 or LZ_F32. */
+ *   = sink-only.  Supported: dk = dv = 128, H <= 32767, io = LZ_BF16 or
+ *   LZ_F32. */
 lz_status lz_gla_decode_step(int Bd, int H, int dk, int dv, int w, int M,
                              lz_dtype io, float scale, float alpha,
                              float* state, void* kring, void* vring,
@@ -250,16 +263,23 @@ lz_status lz_gla_decode_step(int Bd, int H, int dk, int dv, int w, int M,
 
 /* Hand-off from a prefill to lz_gla_decode_step (section 2a: generation
  * continues from the fixed-size state and the last w keys/values).  For Bd
- * prompts of T tokens each: state = hT (the prefill's final state from
+ * prompts of L_b tokens: state = hT (the prefill's final state from
  * lz_gla_fwd / lz_hybrid_fwd, [Bd,H,dk,dv] fp32; NULL = zeros); ring slot
- * (t mod w) = k_t, v_t for the last min(T, w) prompt tokens (k, v
- * [Bd,H,T,dk/dv] io dtype, the prefill's layout); pos = T.  Ring slots not
- * written keep their contents (the decode step never reads them).
+ * (t mod w) = k_t, v_t for the last min(L_b, w) prompt tokens (k, v
+ * [Bd,H,T,dk/dv] io dtype, the prefill's layout); pos[b] = L_b.  Ring slots
+ * not written keep their contents (the decode step never reads them).
+ *   lens: [Bd] int64 device array of prompt lengths L_b (clamped to
+ *   [0, T]), or NULL for L_b = T.  Prompts of different lengths share one
+ *   prefill by right-padding to T with k = 0 and g = 0 (log-gate 0, i.e. no
+ *   decay): the padded tokens then leave the state unchanged, so hT is each
+ *   prompt's state after its own L_b tokens (q and v of the padding are
+ *   free; their outputs are to be ignored).
  * Supported: dk = dv = 128, 1 <= w <= 1024. */
 lz_status lz_decode_prefill(int Bd, int H, int T, int dk, int dv, int w,
                             lz_dtype io, const void* k, const void* v,
-                            const float* hT, float* state, void* kring,
-                            void* vring, int64_t* pos, lz_stream stream);
+                            const int64_t* lens, const float* hT,
+                            float* state, void* kring, void* vring,
+                            int64_t* pos, lz_stream stream);
 
 /* Device-side status (no counterpart on the pages; a robustness aid).  The
  * tcgen05 kernels wait on mbarriers for their tensor-core work; every such

@@ -120,6 +120,8 @@ def test_decode_validation(lib):
     assert f(4, 2, 64, 128, 16, 2, L.LZ_BF16, 0.1, 0.5, *args, 0) == L.LZ_ERR_UNSUPPORTED
     assert f(4, 2, 128, 128, 0, 2, L.LZ_BF16, 0.1, 0.5, *args, 0) == L.LZ_ERR_UNSUPPORTED
     assert f(4, 2, 128, 128, 16, 17, L.LZ_BF16, 0.1, 0.5, *args, 0) == L.LZ_ERR_UNSUPPORTED
+    # the position word holds a 15-bit arrival count of the heads during a step
+    assert f(4, 32768, 128, 128, 16, 2, L.LZ_BF16, 0.1, 0.5, *args, 0) == L.LZ_ERR_UNSUPPORTED
     assert f(-1, 2, 128, 128, 16, 2, L.LZ_BF16, 0.1, 0.5, *args, 0) == L.LZ_ERR_INVALID_ARG
     bad = list(args)
     bad[0] = None  # state
@@ -165,7 +167,8 @@ def test_chunk_states_size_and_validation(lib):
 
 def test_decode_prefill_validation(lib):
     f = lib.lz_decode_prefill
-    args = [FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE]  # k, v, hT, state, kring, vring, pos
+    # k, v, lens, hT, state, kring, vring, pos
+    args = [FAKE, FAKE, None, None, FAKE, FAKE, FAKE, FAKE]
     assert f(2, 2, 10, 64, 128, 16, L.LZ_BF16, *args, 0) == L.LZ_ERR_UNSUPPORTED
     assert f(2, 2, 10, 128, 128, 0, L.LZ_BF16, *args, 0) == L.LZ_ERR_UNSUPPORTED
     assert f(2, 2, -1, 128, 128, 16, L.LZ_BF16, *args, 0) == L.LZ_ERR_INVALID_ARG
@@ -173,7 +176,10 @@ def test_decode_prefill_validation(lib):
     bad[0] = None  # k missing with T > 0
     assert f(2, 2, 10, 128, 128, 16, L.LZ_BF16, *bad, 0) == L.LZ_ERR_INVALID_ARG
     bad = list(args)
-    bad[6] = FAKE + 8  # pos misaligned
+    bad[7] = FAKE + 8  # pos misaligned
+    assert f(2, 2, 10, 128, 128, 16, L.LZ_BF16, *bad, 0) == L.LZ_ERR_INVALID_ARG
+    bad = list(args)
+    bad[2] = FAKE + 8  # lens misaligned
     assert f(2, 2, 10, 128, 128, 16, L.LZ_BF16, *bad, 0) == L.LZ_ERR_INVALID_ARG
 
 

@@ -128,7 +128,9 @@ def test_gla_bwd_gate_edge_cases_bf16(fill):
     decay), g = -30 (full forgetting: elementwise diagonal blocks), a mixture
     inside each chunk, one fast-decaying key dim among slow ones (per-pair
     sub-block factors), and the long-context distribution logsigmoid(N(-1,
-    1.5)) with no /16."""
+    1.5)) with no /16.  Every gradient, dg included, meets the plain
+    relative-L2 bar in every regime (dg's in-chunk running sum cancels
+    exactly in the kernel, so fast forgetting does not amplify rounding)."""
     T = 200
     cpu, dev = small_problem(31, 1, 2, T, 128, 128, 0, torch.bfloat16, train=True, h0=True)
     gen = torch.Generator().manual_seed(5)
@@ -146,18 +148,23 @@ def test_gla_bwd_gate_edge_cases_bf16(fill):
                     want_dh0=True)
     x = oracle_inputs(cpu, ("q", "k", "v", "dO", "h0", "dhT"))
     ref = oracle.gla_bwd(x["q"], x["k"], x["v"], g.double().numpy(), x["dO"], x["h0"], x["dhT"])
-    for name in ("dq", "dk", "dv", "dh0"):
+    for name in ("dq", "dk", "dv", "dh0", "dg"):
         assert_close(f"{name}[g={fill}]", res[name], ref[name], torch.bfloat16)
-    if fill in (0.0, "mixed", "one-dim"):
-        assert_close(f"dg[g={fill}]", res["dg"], ref["dg"], torch.bfloat16)
-    else:
-        # Fast forgetting: dg (reading R11) is a running sum, inside each chunk,
-        # of q*dq - k*dk, terms that cancel there, so the bf16 kernel's dg error
-        # is bounded relative to those terms rather than to dg itself (whose
-        # plain rel-L2 is ~4e-2 for logsigmoid(N(-1, 1.5)) gates; ~0 at -30).
-        terms = np.sqrt(np.sum((x["q"] * ref["dq"]) ** 2) + np.sum((x["k"] * ref["dk"]) ** 2))
-        err = np.sqrt(np.sum((np64(res["dg"]) - ref["dg"]) ** 2))
-        assert err / (np.sqrt(np.sum(ref["dg"] ** 2)) + terms) <= 2e-2, (fill, err, terms)
+
+
+def test_gla_bwd_long_context_gates_full_length():
+    """One head over the long-context workload's whole length (T = 65536)
+    with its fast-forgetting gates logsigmoid(N(-1, 1.5)) and a synthetic
+    dO ~ N(0, 1): every gradient of the bf16 tensor-core backward, dg with
+    the plain relative-L2 bar."""
+    wl = I.LONG_BF16.with_(H=1, M=0, train=True)
+    x = I.make_inputs(wl, seed=3, device="cpu")
+    dev = {k: v.cuda() for k, v in x.items()}
+    res = L.gla_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["dO"])
+    xs = {k: np64(v) for k, v in x.items()}
+    ref = oracle.gla_bwd(xs["q"], xs["k"], xs["v"], xs["g"], xs["dO"])
+    for name in ("dq", "dk", "dv", "dg"):
+        assert_close(f"{name}[T=65536]", res[name], ref[name], torch.bfloat16)
 
 
 def test_bwd_determinism():

@@ -80,6 +80,128 @@ def test_decode_workload_sampled():
     assert torch.all(d["pos"].cpu() == wl.pos0 + 6)
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("w", [8, 128])
+def test_decode_mixed_positions(dtype, w):
+    """Sequences at different positions in one batch (an empty history, a
+    partly filled window, exactly full, one past full, several wraps) step
+    together; every step's output is checked against the oracle's step, the
+    state at the end, the rings bit for bit and pos after every step."""
+    pos0 = [0, 3, w - 1, w, 5 * w + 2]
+    Bd, H, M, n = len(pos0), 2, 4, 7
+    cpu, dev = small_problem(400 + w, Bd, H, n, 128, 128, M, dtype)
+    gen = torch.Generator().manual_seed(401 + w)
+    st0 = torch.randn(Bd, H, 128, 128, generator=gen) * 0.1
+    kr0 = (torch.randn(Bd, H, w, 128, generator=gen) * 0.1).to(dtype)
+    vr0 = torch.randn(Bd, H, w, 128, generator=gen).to(dtype)
+    state, kring, vring = st0.cuda(), kr0.cuda(), vr0.cuda()
+    pos = torch.tensor(pos0, dtype=torch.int64, device="cuda")
+    ost = {"state": np64(st0), "kring": np64(kr0), "vring": np64(vr0),
+           "pos": np.array(pos0, dtype=np.int64)}
+    x = {k: np64(v) for k, v in cpu.items()}
+    for t in range(n):
+        sl = lambda name: dev[name][:, :, t].contiguous()
+        o = L.decode_step(state, kring, vring, pos, sl("q"), sl("k"), sl("v"), sl("g"),
+                          dev["meta_k"], dev["meta_v"], alpha=0.5)
+        ost = oracle.decode_step(ost["state"], ost["kring"], ost["vring"], ost["pos"],
+                                 x["q"][:, :, t], x["k"][:, :, t], x["v"][:, :, t],
+                                 x["g"][:, :, t], x["meta_k"], x["meta_v"],
+                                 1 / math.sqrt(128), 0.5)
+        assert_close(f"o step {t}", o, ost["o"], dtype)
+        assert np.array_equal(pos.cpu().numpy(), ost["pos"]), (t, pos.cpu(), ost["pos"])
+    assert_close("state", state, ost["state"], dtype)
+    assert np.array_equal(np64(kring), ost["kring"])
+    assert np.array_equal(np64(vring), ost["vring"])
+
+
+def test_decode_one_launch_per_step_in_a_graph():
+    """The step is one kernel launch (the position advances inside it), so a
+    run of steps captures into one CUDA graph; replaying it from the same
+    starting buffers gives the eager run's outputs, state, rings and pos bit
+    for bit."""
+    Bd, H, w, M, n = 3, 4, 16, 2, 5
+    cpu, dev = small_problem(420, Bd, H, n, 128, 128, M, torch.bfloat16)
+    gen = torch.Generator().manual_seed(421)
+    init = [(torch.randn(Bd, H, 128, 128, generator=gen) * 0.1).cuda(),
+            (torch.randn(Bd, H, w, 128, generator=gen) * 0.1).bfloat16().cuda(),
+            torch.randn(Bd, H, w, 128, generator=gen).bfloat16().cuda(),
+            torch.tensor([0, 9, 40], dtype=torch.int64, device="cuda")]
+    toks = {k: [dev[k][:, :, t].contiguous() for t in range(n)] for k in ("q", "k", "v", "g")}
+    outs = [torch.empty(Bd, H, 128, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+
+    def steps(bufs):
+        for t in range(n):
+            L.decode_step(*bufs, toks["q"][t], toks["k"][t], toks["v"][t], toks["g"][t],
+                          dev["meta_k"], dev["meta_v"], alpha=0.5, o=outs[t])
+
+    eager = [x.clone() for x in init]
+    steps(eager)
+    eager_out = [o.clone() for o in outs]
+    bufs = [x.clone() for x in init]
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        steps([x.clone() for x in init])  # warm-up off the capture
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        steps(bufs)
+    for x, y in zip(bufs, init):
+        x.copy_(y)
+    graph.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(outs, eager_out):
+        assert torch.equal(a, b)
+    for a, b in zip(bufs, eager):
+        assert torch.equal(a, b)
+    assert torch.equal(bufs[3].cpu(), torch.tensor([n, 9 + n, 40 + n]))
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_variable_length_prefill_then_decode(dtype):
+    """Prompts of different lengths share one right-padded prefill (padding
+    with k = 0 and g = 0, so the state stops at each prompt's end), the
+    hand-off takes the per-sequence lengths, and the batch then decodes with
+    every sequence at its own position: each sequence's outputs and final
+    state match the oracle's forward over its own prompt plus the new tokens."""
+    T, w, M, n, alpha, H = 150, 64, 4, 5, 0.5, 2
+    lens = [150, 113, 5, 0, 64]
+    Bd = len(lens)
+    cpu, dev = small_problem(430, Bd, H, T + n, 128, 128, M, dtype)
+    pk = cpu["k"][:, :, :T].clone()
+    pg = cpu["g"][:, :, :T].clone()
+    for b, l in enumerate(lens):  # padding: no key, no decay
+        pk[b, :, l:] = 0
+        pg[b, :, l:] = 0
+    pre = {"q": dev["q"][:, :, :T].contiguous(), "k": pk.cuda(),
+           "v": dev["v"][:, :, :T].contiguous(), "g": pg.cuda()}
+    fwd = L.hybrid_fwd(pre["q"], pre["k"], pre["v"], pre["g"], dev["meta_k"], dev["meta_v"],
+                       w=w, alpha=alpha, want_hT=True)
+    state, kring, vring, pos = L.decode_prefill(pre["k"], pre["v"], fwd["hT"], w=w,
+                                                lens=torch.tensor(lens))
+    torch.cuda.synchronize()
+    assert pos.cpu().tolist() == lens
+    # decode token j of sequence b is its token lens[b] + j
+    x = {k: np64(v) for k, v in cpu.items()}
+    outs = []
+    for j in range(n):
+        idx = [l + j for l in lens]
+        tok = {name: torch.stack([cpu[name][b, :, idx[b]] for b in range(Bd)]).cuda()
+               for name in ("q", "k", "v", "g")}
+        outs.append(L.decode_step(state, kring, vring, pos, tok["q"], tok["k"], tok["v"],
+                                  tok["g"], dev["meta_k"], dev["meta_v"], alpha=alpha).clone())
+    torch.cuda.synchronize()
+    assert pos.cpu().tolist() == [l + n for l in lens]
+    for b, l in enumerate(lens):
+        sl = lambda name: x[name][b:b + 1, :, :l + n]  # its prompt, then its new tokens
+        ref = oracle.hybrid_fwd(sl("q"), sl("k"), sl("v"), sl("g"), x["meta_k"], x["meta_v"],
+                                w, 1 / math.sqrt(128), alpha)
+        got = torch.stack([o[b] for o in outs], dim=1)[None]
+        assert_close(f"decode o [seq {b}, prompt {l}]", got, ref["o"][:, :, l:], dtype)
+        assert_close(f"state [seq {b}]", state[b:b + 1], ref["hT"], dtype)
+
+
 def test_decode_state_save_restore_bitwise():
     Bd, H, w, M = 4, 2, 8, 2
     cpu, dev = small_problem(90, Bd, H, 12, 128, 128, M, torch.bfloat16)

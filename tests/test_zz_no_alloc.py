@@ -22,11 +22,14 @@ from gated_linear_sliding_chunked_b200 import build as lbuild
 from parity_util import assert_close, small_problem
 
 
-def _noalloc(dims, dev, mk, mv, lse):
-    out = {"dq": torch.empty_like(dev["q"]), "dk": torch.empty_like(dev["k"]),
-           "dv": torch.empty_like(dev["v"]),
-           "dmeta_k": torch.empty(mk.shape, dtype=torch.float32, device="cuda"),
-           "dmeta_v": torch.empty(mv.shape, dtype=torch.float32, device="cuda")}
+def _outputs(dev, mk, mv):
+    return {"dq": torch.empty_like(dev["q"]), "dk": torch.empty_like(dev["k"]),
+            "dv": torch.empty_like(dev["v"]),
+            "dmeta_k": torch.empty(mk.shape, dtype=torch.float32, device="cuda"),
+            "dmeta_v": torch.empty(mv.shape, dtype=torch.float32, device="cuda")}
+
+
+def _noalloc(dims, dev, mk, mv, lse, out):
     L.lz_swa_meta_bwd_noalloc(dims, dev["q"], dev["k"], dev["v"], mk, mv, lse, None, dev["dO"],
                               out["dq"], out["dk"], out["dv"], out["dmeta_k"], out["dmeta_v"])
     return out
@@ -36,9 +39,14 @@ def _noalloc(dims, dev, mk, mv, lse):
 def test_noalloc_matches_allocating_backward_twice():
     lbuild.build()
     L.load()
-    # two different problems back to back through the same static scratch
-    cases = [(3, 2, 4, 700, 64, 8, torch.bfloat16), (4, 1, 3, 513, 33, 3, torch.float32)]
-    for seed, B, H, T, w, M, dtype in cases:
+    # problems back to back through the same static scratch: a larger bf16
+    # case (more 256-query slabs of per-slab partials), a smaller one on the
+    # same tensor-core path, an fp32 one on the SIMT path, then the first
+    # again, which must reproduce its first result bit for bit
+    cases = [(3, 2, 4, 700, 64, 8, torch.bfloat16), (5, 2, 4, 300, 64, 8, torch.bfloat16),
+             (4, 1, 3, 513, 33, 3, torch.float32), (3, 2, 4, 700, 64, 8, torch.bfloat16)]
+    first = None
+    for i, (seed, B, H, T, w, M, dtype) in enumerate(cases):
         cpu, dev = small_problem(seed, B, H, T, 128, 128, M, dtype, train=True)
         mk, mv = dev["meta_k"], dev["meta_v"]
         dims = L.make_dims(B, H, T, 128, 128, chunk=64, w=w, M=M, io=L.io_of(dtype),
@@ -46,10 +54,22 @@ def test_noalloc_matches_allocating_backward_twice():
         assert L.lz_workspace_bytes(dims, L.LZ_WS_SWA_BWD) <= L.LZ_NOALLOC_SCRATCH_BYTES
         _, lse = L.swa_meta_fwd(dev["q"], dev["k"], dev["v"], mk, mv, w=w)
         ref = L.swa_meta_bwd(dev["q"], dev["k"], dev["v"], mk, mv, lse, dev["dO"], w=w)
-        got = _noalloc(dims, dev, mk, mv, lse)
+        out = _outputs(dev, mk, mv)
         torch.cuda.synchronize()
+        free0 = torch.cuda.mem_get_info()[0]
+        got = _noalloc(dims, dev, mk, mv, lse, out)
+        torch.cuda.synchronize()
+        # the first call may load the library's module (and its array);
+        # every later call leaves the device's free memory as it found it
+        if i > 0:
+            assert torch.cuda.mem_get_info()[0] == free0, (i, free0)
         for name in ("dq", "dk", "dv", "dmeta_k", "dmeta_v"):
             assert_close(f"{name} (T={T})", got[name], ref[name].double().cpu().numpy(), dtype)
+        if i == 0:
+            first = {k: v.clone() for k, v in got.items()}
+        if i == len(cases) - 1:
+            for name, x in got.items():
+                assert torch.equal(x, first[name]), name
 
 
 def test_noalloc_rejects_problem_larger_than_its_scratch():
