@@ -33,7 +33,7 @@ EXPORTS = ("lz_gla_fwd", "lz_gla_bwd", "lz_swa_meta_fwd", "lz_hybrid_fwd", "lz_s
            "lz_hybrid_bwd", "lz_gla_decode_step", "lz_workspace_bytes", "lz_last_error",
            "lz_version", "lz_timing_enable", "lz_timing_read", "lz_swa_meta_bwd_noalloc",
            "lz_device_check", "lz_prefer_tcgen05", "lz_decode_prefill", "lz_hybrid_fwd_mse",
-           "lz_selftest_bounded_wait")
+           "lz_selftest_bounded_wait", "lz_cp_segment_decay", "lz_cp_fold", "lz_cp_rows")
 
 # size of the static scratch array behind lz_swa_meta_bwd_noalloc
 LZ_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -84,6 +84,11 @@ def load(path: str = LIB_PATH):
     lib.lz_selftest_bounded_wait.argtypes = [_P]
     lib.lz_decode_prefill.argtypes = [ctypes.c_int] * 7 + [_P] * 8 + [_P]
     lib.lz_prefer_tcgen05.argtypes = [ctypes.c_int]
+    ci = ctypes.c_int
+    lib.lz_cp_segment_decay.argtypes = [ci, ci, ci, _P, _P, _P]
+    lib.lz_cp_fold.argtypes = [ci] * 6 + [_P] * 4 + [_P]
+    lib.lz_cp_rows.argtypes = ([ci] * 4 + [_P, ci, ci, ctypes.c_float, _P, ci, ci, _P, ci, ci] +
+                               [_P])
     lib.lz_timing_enable.argtypes = [ctypes.c_int]
     lib.lz_timing_read.argtypes = [ctypes.c_char_p, sz, ctypes.POINTER(ctypes.c_float),
                                    ctypes.c_int]
@@ -440,3 +445,53 @@ def decode_step(state, kring, vring, pos, q, k, v, g, meta_k, meta_v, *, alpha, 
     lz_gla_decode_step(Bd, H, dk, dv, w, M, io_of(q.dtype), scale, alpha, state, kring, vring,
                        pos, q, k, v, g, meta_k, meta_v, o, stream)
     return o
+
+
+# ---- context parallelism (one sequence over several ranks) -----------------
+def lz_cp_segment_decay(BH, T, dk, g, E, stream=None):
+    _check(load().lz_cp_segment_decay(BH, T, dk, _ptr(g), _ptr(E), _stream(stream)))
+
+
+def lz_cp_fold(R, r, direction, BH, dk, dv, E, X, init, out, stream=None):
+    _check(load().lz_cp_fold(R, r, direction, BH, dk, dv, _ptr(E), _ptr(X), _ptr(init),
+                             _ptr(out), _stream(stream)))
+
+
+def lz_cp_rows(BH, d, io, n, A, a_T, a_off, a_scale, B, b_T, b_off, dst, dst_T, dst_off,
+               stream=None):
+    _check(load().lz_cp_rows(BH, d, io, n, _ptr(A), a_T, a_off, float(a_scale), _ptr(B), b_T,
+                             b_off, _ptr(dst), dst_T, dst_off, _stream(stream)))
+
+
+def segment_decay(g):
+    """Per (batch, head, key dim) product of a segment's gates: g [B, H, T, dk]
+    fp32 log-gates -> [B, H, dk] fp32."""
+    B, H, T, dk = g.shape
+    E = torch.empty(B, H, dk, dtype=torch.float32, device=g.device)
+    lz_cp_segment_decay(B * H, T, dk, g, E)
+    return E
+
+
+def cp_fold(E_all, X_all, r, direction, init=None):
+    """Fold over segments (see lz_cp_fold): E_all [R, B, H, dk], X_all
+    [R, B, H, dk, dv] fp32 -> [B, H, dk, dv]."""
+    R, B, H, dk, dv = X_all.shape
+    out = torch.empty(B, H, dk, dv, dtype=torch.float32, device=X_all.device)
+    lz_cp_fold(R, r, direction, B * H, dk, dv, E_all.contiguous(), X_all.contiguous(),
+               None if init is None else init.contiguous(), out)
+    return out
+
+
+def cp_rows(dst, dst_off, n, A=None, a_off=0, a_scale=1.0, B=None, b_off=0):
+    """dst[:, :, dst_off + t] = a_scale * A[:, :, a_off + t] + B[:, :, b_off + t]
+    for t < n, in place on dst ([batch, head, rows, d] tensors of one dtype;
+    None = zeros).  Returns dst."""
+    Bb, H, dT, d = dst.shape
+    for x in (A, B):
+        if x is not None and (x.dtype != dst.dtype or x.shape[:2] != dst.shape[:2]
+                              or x.shape[3] != d):
+            raise ValueError("cp_rows: tensors must share dtype, batch, heads and d")
+    lz_cp_rows(Bb * H, d, io_of(dst.dtype), n, A, 0 if A is None else A.shape[2], a_off, a_scale,
+               B, 0 if B is None else B.shape[2], b_off, dst, dT, dst_off)
+    return dst
+

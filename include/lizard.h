@@ -281,6 +281,50 @@ lz_status lz_decode_prefill(int Bd, int H, int T, int dk, int dv, int w,
                             float* state, void* kring, void* vring,
                             int64_t* pos, lz_stream stream);
 
+/* ---- Context parallelism: one sequence over R ranks ----------------------
+ * The pages run each layer on one device; splitting a long sequence into R
+ * contiguous segments (rank r holds tokens [r Ts, (r+1) Ts) of every
+ * (batch, head)) rests on section 2a's state update S_t = Gamma_t S_{t-1} +
+ * k_t v_t^T being linear: a segment maps the state it receives to
+ * diag(E) h + S, with E the product of its gates per key dim and S its
+ * final state from a zero start.  These three calls are that arithmetic;
+ * moving data between ranks is the caller's (e.g. torch.distributed).  All
+ * pointers are device memory owned by the caller; calls are asynchronous on
+ * `stream`; bad arguments return LZ_ERR_INVALID_ARG / LZ_ERR_UNSUPPORTED
+ * before any launch, launch failures LZ_ERR_CUDA. */
+
+/* E[bh][i] = exp(sum over the T tokens of g[bh][t][i]): the segment's gate
+ * product per key dim.  g [BH,T,dk] fp32 log-gates, E [BH,dk] fp32 (T = 0
+ * gives 1).  dk = 64 or 128; 16-byte aligned pointers. */
+lz_status lz_cp_segment_decay(int BH, int T, int dk, const float* g, float* E,
+                              lz_stream stream);
+
+/* The fold over segments, elementwise on [BH,dk,dv] fp32 states:
+ *   dir 0 (forward): h = init; for q = 0 .. r-1: h = diag(E_q) h + X_q.
+ *     With X_q = segment q's final state from a zero start, out is the
+ *     state entering segment r (init = the sequence's h0, NULL = 0).
+ *   dir 1 (reverse): h = init; for q = R-1 down to r+1: h = X_q + diag(E_q) h.
+ *     With X_q = the gradient of segment q's outputs with respect to the
+ *     state it received (its dh0 from a backward with dhT = 0), out is the
+ *     state gradient leaving segment r (init = the sequence's dhT, NULL = 0).
+ * E [R,BH,dk], X [R,BH,dk,dv] (segment-major, as an all-gather stacks them);
+ * out [BH,dk,dv] may not alias X.  dv a multiple of 4; 16-byte aligned. */
+lz_status lz_cp_fold(int R, int r, int dir, int BH, int dk, int dv,
+                     const float* E, const float* X, const float* init,
+                     float* out, lz_stream stream);
+
+/* Row-block copy and sum over [BH, rows, d] tensors of the io dtype:
+ *   dst[bh][dst_off + t] = a_scale * A[bh][a_off + t] + B[bh][b_off + t]
+ * for t < n, with A or B NULL standing for zeros; each tensor has its own
+ * row count (a_T, b_T, dst_T).  Summed in fp32, rounded once.  Used to cut
+ * the window halo (the last w - 1 rows) out of a segment, to prepend it, and
+ * to add the window branch's rows to the gated branch's.  dst may alias A or
+ * B row for row (same offsets); other overlaps are not allowed. */
+lz_status lz_cp_rows(int BH, int d, lz_dtype io, int n, const void* A,
+                     int a_T, int a_off, float a_scale, const void* B,
+                     int b_T, int b_off, void* dst, int dst_T, int dst_off,
+                     lz_stream stream);
+
 /* Device-side status (no counterpart on the pages; a robustness aid).  The
  * tcgen05 kernels wait on mbarriers for their tensor-core work; every such
  * wait is bounded (0.2 s) and, when it gives up, adds one to a status word

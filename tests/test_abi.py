@@ -248,3 +248,24 @@ def test_binding_reads_bf16_gates_as_logits():
                      g=torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16), gate_scale=0.25)
     assert d.gate_logits == 1 and abs(d.gate_scale - 0.25) < 1e-7
     assert L.lz_workspace_bytes(d, L.LZ_WS_HYBRID_BWD) > 0
+
+
+def test_context_parallel_validation(lib):
+    """The context-parallel calls refuse bad arguments before any launch."""
+    assert lib.lz_cp_segment_decay(4, 16, 96, FAKE, FAKE, 0) == L.LZ_ERR_UNSUPPORTED
+    assert lib.lz_cp_segment_decay(4, -1, 128, FAKE, FAKE, 0) == L.LZ_ERR_INVALID_ARG
+    assert lib.lz_cp_segment_decay(4, 16, 128, FAKE + 4, FAKE, 0) == L.LZ_ERR_INVALID_ARG
+    f = lib.lz_cp_fold
+    assert f(2, 2, 0, 4, 128, 128, FAKE, FAKE, None, FAKE, 0) == L.LZ_ERR_INVALID_ARG  # r >= R
+    assert f(2, 0, 2, 4, 128, 128, FAKE, FAKE, None, FAKE, 0) == L.LZ_ERR_INVALID_ARG  # dir
+    assert f(2, 0, 0, 4, 128, 126, FAKE, FAKE, None, FAKE, 0) == L.LZ_ERR_UNSUPPORTED
+    assert f(2, 1, 0, 4, 128, 128, FAKE, None, None, FAKE, 0) == L.LZ_ERR_INVALID_ARG
+    assert b"NULL" in lib.lz_last_error()
+    r = lib.lz_cp_rows
+    # rows [10, 20) of a 15-row source
+    assert r(4, 128, L.LZ_BF16, 10, FAKE, 15, 10, 1.0, None, 0, 0, FAKE, 64, 0, 0) == \
+        L.LZ_ERR_INVALID_ARG
+    assert b"outside" in lib.lz_last_error()
+    assert r(4, 128, 7, 10, FAKE, 64, 0, 1.0, None, 0, 0, FAKE, 64, 0, 0) == L.LZ_ERR_UNSUPPORTED
+    assert r(4, 128, L.LZ_BF16, 0, None, 0, 0, 1.0, None, 0, 0, FAKE, 64, 0, 0) == L.LZ_OK
+
