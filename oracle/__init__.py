@@ -73,7 +73,8 @@ def _bind(lib):
     lib.oracle_mse_loss.argtypes = [ctypes.c_int64] + [_D] * 4
     lib.oracle_gate_from_logits.argtypes = [ctypes.c_int64, _D, ctypes.c_double, _D]
     lib.oracle_dlogits.argtypes = [ctypes.c_int64, _D, ctypes.c_double, _D, _D]
-    for name in ("oracle_gate_from_logits", "oracle_dlogits", "oracle_mse_loss", "oracle_gla_fwd", "oracle_gla_chunked_fwd", "oracle_swa_meta_fwd",
+    lib.oracle_qkg_projection.argtypes = [_i] * 5 + [_D] * 4 + [ctypes.c_double] + [_D] * 3
+    for name in ("oracle_qkg_projection", "oracle_gate_from_logits", "oracle_dlogits", "oracle_mse_loss", "oracle_gla_fwd", "oracle_gla_chunked_fwd", "oracle_swa_meta_fwd",
                  "oracle_hybrid_fwd", "oracle_gla_bwd", "oracle_swa_meta_bwd",
                  "oracle_hybrid_bwd", "oracle_decode_step"):
         getattr(lib, name).restype = ctypes.c_int
@@ -281,3 +282,19 @@ def dlogits(z, dg, scale=1.0, *, lib=None):
     dz, pdz = _out(z.shape)
     _check(lib.oracle_dlogits(int(z.size), pz, float(scale), pdg, pdz), "dlogits")
     return dz
+
+
+def qkg_projection(x, Wq, Wk, Wg, H, dk, scale=1.0, *, lib=None):
+    """q = x Wq^T, k = x Wk^T (phi = identity), g = scale * log sigma(x Wg^T),
+    each [B, H, T, dk] (None where its weight is None).  x [B, T, Dm], W
+    [H*dk, Dm]."""
+    lib = lib or load()
+    (x, px) = _in(x)
+    B, T, Dm = x.shape
+    ws = [_in(w) for w in (Wq, Wk, Wg)]
+    outs = [(_out((B, H, T, dk)) if w is not None else (None, None)) for w in (Wq, Wk, Wg)]
+    _check(lib.oracle_qkg_projection(B, T, Dm, H, dk, px, ws[0][1], ws[1][1], ws[2][1],
+                                     float(scale), outs[0][1], outs[1][1], outs[2][1]),
+           "qkg_projection")
+    return outs[0][0], outs[1][0], outs[2][0]
+

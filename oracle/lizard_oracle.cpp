@@ -669,6 +669,46 @@ int oracle_dlogits(int64_t n, const double* z, double scale, const double* dg, d
   return 0;
 }
 
+// The projections in front of the operator (section 2a: the gate is
+// Gamma_i = sigma(W_gamma x_i); the state update takes phi(k_i) and the output
+// reads q_i).  For hidden states x [B][T][Dm] and weights W [H*dk][Dm] (one
+// row per output feature): q = x Wq^T and k = x Wk^T with phi the identity
+// (the pages do not define phi; reading: the operator receives the featurised
+// keys), g = scale * log sigma(x Wg^T) through oracle_gate_from_logits.
+// Outputs in the operator's layout [B][H][T][dk]; a NULL weight skips its
+// output.
+int oracle_qkg_projection(int B, int T, int Dm, int H, int dk, const double* x, const double* Wq,
+                          const double* Wk, const double* Wg, double scale, double* q, double* k,
+                          double* g) {
+  if (B < 0 || T < 0 || Dm < 1 || H < 1 || dk < 1 || !(scale > 0.0)) return -1;
+  const double* W[3] = {Wq, Wk, Wg};
+  double* out[3] = {q, k, g};
+  std::vector<double> z((size_t)dk);
+  for (int which = 0; which < 3; ++which) {
+    if (!W[which]) continue;
+    if (!out[which] || (B * T > 0 && !x)) return -1;
+    for (int b = 0; b < B; ++b)
+      for (int t = 0; t < T; ++t) {
+        const double* xr = x + ((size_t)b * T + t) * Dm;
+        for (int h = 0; h < H; ++h) {
+          for (int i = 0; i < dk; ++i) {
+            const double* wr = W[which] + ((size_t)h * dk + i) * Dm;
+            double acc = 0.0;
+            for (int c = 0; c < Dm; ++c) acc += xr[c] * wr[c];
+            z[i] = acc;
+          }
+          double* dst = out[which] + (((size_t)b * H + h) * T + t) * dk;
+          if (which == 2) {
+            if (oracle_gate_from_logits(dk, z.data(), scale, dst) != 0) return -1;
+          } else {
+            for (int i = 0; i < dk; ++i) dst[i] = z[i];
+          }
+        }
+      }
+  }
+  return 0;
+}
+
 // Stage-1 distillation loss (section 2b, "training strategy": the first
 // stage trains the hybrid attention to reproduce the teacher's attention
 // output under a mean-squared-error loss).  Reading: the mean runs over every

@@ -460,11 +460,58 @@ def pin_gate_logits_grad_fd(lib):
     assert _rel(dz, num) < 1e-6, _rel(dz, num)
 
 
+# ----------------------------------------------------------------------------
+# the projections in front of the operator (section 2a: Gamma = sigma(W_gamma x),
+# phi(k); reading: phi is the identity)
+# ----------------------------------------------------------------------------
+def _proj_x(seed, B=2, T=5, Dm=24):
+    return RNG(seed).standard_normal((B, T, Dm))
+
+
+def pin_projection_selection(lib):
+    """One-hot weight rows pick single hidden features: q[b, h, t, i] is
+    x[b, t, perm(h, i)], in the operator's [B, H, T, dk] layout."""
+    H, dk, Dm = 3, 4, 24
+    x = _proj_x(41, Dm=Dm)
+    perm = RNG(42).permutation(Dm)[: H * dk]
+    W = np.zeros((H * dk, Dm))
+    W[np.arange(H * dk), perm] = 1.0
+    q, k, g = oracle.qkg_projection(x, W, None, None, H, dk, lib=lib)
+    assert k is None and g is None
+    want = x[:, :, perm].reshape(x.shape[0], x.shape[1], H, dk).transpose(0, 2, 1, 3)
+    assert np.array_equal(q, want)
+
+
+def pin_projection_rank_one(lib):
+    """W = a c^T (rank one) gives y = (x . c) a: keys through the identity
+    feature map, gates through the logistic written out directly."""
+    H, dk, Dm, s = 2, 3, 24, 0.5
+    x = _proj_x(43, Dm=Dm)
+    r = RNG(44)
+    a, c = r.standard_normal(H * dk), r.standard_normal(Dm) * 0.3
+    W = np.outer(a, c)
+    _, k, g = oracle.qkg_projection(x, None, W, W, H, dk, s, lib=lib)
+    xc = np.einsum("btd,d->bt", x, c)
+    y = (xc[:, :, None] * a[None, None, :]).reshape(x.shape[0], x.shape[1], H, dk)
+    y = y.transpose(0, 2, 1, 3)
+    assert _rel(k, y) < 1e-13
+    assert np.allclose(np.exp(g / s), 1.0 / (1.0 + np.exp(-y)), rtol=1e-12)
+
+
+def pin_projection_zero_gate_weights(lib):
+    """A zero gate projection gives sigma(0) = 1/2 everywhere: g = -scale log 2."""
+    H, dk, Dm, s = 2, 4, 24, 1.0 / 16
+    x = _proj_x(45, Dm=Dm)
+    _, _, g = oracle.qkg_projection(x, None, None, np.zeros((H * dk, Dm)), H, dk, s, lib=lib)
+    assert np.allclose(g, -s * np.log(2.0), rtol=0, atol=1e-16)
+
+
 ALL_PINS = [
     pin_gla_closed_form, pin_gla_unit_gates, pin_gla_full_forgetting,
     pin_gla_initial_state, pin_gla_chunked_identity, pin_swa_full_causal,
     pin_swa_band_meta, pin_swa_sinks, pin_hybrid_affine, pin_hybrid_grad_fd,
     pin_swa_grad_fd, pin_gla_dg_identity, pin_decode_matches_prefill,
     pin_mse_closed_form, pin_mse_grad_fd, pin_stage1_chain_fd,
-    pin_gate_logits_closed_form, pin_gate_logits_grad_fd,
+    pin_gate_logits_closed_form, pin_gate_logits_grad_fd, pin_projection_selection,
+    pin_projection_rank_one, pin_projection_zero_gate_weights,
 ]

@@ -41,6 +41,11 @@ MUTANTS = [
     ("mse_gradient_sign", "const double diff = o[x] - target[x];", "const double diff = target[x] - o[x];"),
     ("gate_logit_unscaled", "g_out[x] = scale * ls;", "g_out[x] = ls;"),
     ("dlogits_sigmoid_of_z", "dz[x] = dg[x] * scale * sneg;", "dz[x] = dg[x] * scale * (1.0 - sneg);"),
+    ("proj_layout_token_major", "double* dst = out[which] + (((size_t)b * H + h) * T + t) * dk;",
+     "double* dst = out[which] + (((size_t)b * T + t) * H + h) * dk;"),
+    ("proj_gate_map_on_keys", "if (which == 2) {", "if (which == 1) {"),
+    ("proj_weight_rows_of_head0", "const double* wr = W[which] + ((size_t)h * dk + i) * Dm;",
+     "const double* wr = W[which] + ((size_t)i) * Dm;"),
 ]
 
 
