@@ -560,6 +560,42 @@ def measure_train_gate_logits(wl, x, device, steps, warmup, seed):
             "kernels": {k: [c // steps, round(t / c, 4)] for k, (c, t) in tab.items()}}
 
 
+def measure_projection(device, peaks, seed, steps=10, warmup=3):
+    """The q, k, gate projections in front of the operator (one launch) at the
+    training layer's shape: hidden states [2, 8192, 4096] (the Llama-3-8B
+    hidden size), three [4096, 4096] weights; tensor-core bound."""
+    import gated_linear_sliding_chunked_b200 as L
+    from gated_linear_sliding_chunked_b200 import inputs as I
+    wl = I.TRAIN_BF16
+    Dm = 4096
+    gen = torch.Generator(device=device)
+    gen.manual_seed(3000 + seed)
+    x = (torch.randn(wl.B, wl.T, Dm, generator=gen, device=device)).to(torch.bfloat16)
+    W = [(torch.randn(wl.H * wl.dk, Dm, generator=gen, device=device) / Dm ** 0.5).to(torch.bfloat16)
+         for _ in range(3)]
+    q = torch.empty(wl.B, wl.H, wl.T, wl.dk, dtype=torch.bfloat16, device=device)
+    k = torch.empty_like(q)
+    g = torch.empty(wl.B, wl.H, wl.T, wl.dk, dtype=torch.float32, device=device)
+
+    def fn():
+        L.lz_qkg_projection(wl.B, wl.T, Dm, wl.H, wl.dk, x, W[0], W[1], W[2], 1.0 / 16, q, k, g)
+
+    for _ in range(warmup):
+        fn()
+    ms = time_region(fn, steps, device)
+    L.lz_device_check()
+    flops = 2.0 * wl.B * wl.T * Dm * 3 * wl.H * wl.dk
+    tf = flops / (ms * 1e-3) / 1e12
+    del x, W, q, k, g
+    return {"workload": f"x [{wl.B}, {wl.T}, {Dm}] bf16 -> q, k bf16 and fp32 log-gates "
+                        f"[{wl.B}, {wl.H}, {wl.T}, {wl.dk}], three [{wl.H * wl.dk}, {Dm}] weights",
+            "ms_per_call": round(ms, 4), "tokens_per_s": wl.B * wl.T / (ms * 1e-3),
+            "roofline": {"kernel": "qkg_projection_tc", "bound": "tensor", "achieved": round(tf, 1),
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": round(tf / peaks["bf16_tflops"], 4), "flops_per_call": flops,
+                         "peak_source": peaks["source"] + " (bf16_tflops, burst: timed alone)"}}
+
+
 def measure_decode(device, peaks, seed, n_steps=1000):
     """1000 consecutive decode steps (one kernel launch each), captured in one
     CUDA graph and timed by its replay; per-kernel event times come from a
@@ -726,6 +762,8 @@ PROFILE_CASES = {
     "fwd": "hybrid fwd, B4 H16 T2048",
     "long": "hybrid fwd, B1 H32 T65536",
     "decode": "one decode step, Bd128 H32",
+    "proj": "q, k, gate projections, x [1, 2048, 4096] -> [1, 32, 2048, 128] (three 4096^2 weights)",
+    "train-small-tc": "hybrid fwd + bwd, B4 H16 T2048 w64 M4, the gated backward on tcgen05",
 }
 
 
@@ -741,10 +779,24 @@ def run_profile_case(args):
     torch.cuda.set_device(device)
     L.lz_prefer_tcgen05(not args.warp_mma_window)
     case = args.profile_case
-    if case in ("train", "train-small"):
+    if case in ("train", "train-small", "train-small-tc"):
         wl = I.TRAIN_BF16 if case == "train" else I.FWD_BF16.with_(train=True)
         step = TrainStep(wl, I.make_inputs(wl, seed=0, device=device), device)
         fn = step.run
+        L.lz_gated_bwd_tcgen05(case == "train-small-tc")
+    elif case == "proj":
+        H, dk, Dm, T = 32, 128, 4096, 2048
+        gen = torch.Generator(device=device)
+        gen.manual_seed(0)
+        x = torch.randn(1, T, Dm, generator=gen, device=device).to(torch.bfloat16)
+        W = [(torch.randn(H * dk, Dm, generator=gen, device=device) / Dm ** 0.5).to(torch.bfloat16)
+             for _ in range(3)]
+        q = torch.empty(1, H, T, dk, dtype=torch.bfloat16, device=device)
+        k = torch.empty_like(q)
+        g = torch.empty(1, H, T, dk, dtype=torch.float32, device=device)
+
+        def fn():
+            L.lz_qkg_projection(1, T, Dm, H, dk, x, W[0], W[1], W[2], 1.0 / 16, q, k, g)
     elif case in ("fwd", "long"):
         wl = I.FWD_BF16 if case == "fwd" else I.LONG_BF16
         x = I.make_inputs(wl, seed=0, device=device)
@@ -877,6 +929,9 @@ def main(argv=None):
             "so the times of those kernels include the overlap and do not add up to the step")
         extras["stage1_step"] = measure_stage1(wl, xd, device, 10, 3, seed=rank)
         extras["train_step_gate_logits"] = measure_train_gate_logits(wl, xd, device, 10, 3, seed=rank)
+        # last: a dense GEMM at full tensor-core load draws the most power, and
+        # the power cap would lower the clocks of whatever runs right after it
+        extras["qkg_projection"] = measure_projection(device, peaks, seed=rank)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

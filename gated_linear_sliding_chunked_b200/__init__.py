@@ -33,7 +33,8 @@ EXPORTS = ("lz_gla_fwd", "lz_gla_bwd", "lz_swa_meta_fwd", "lz_hybrid_fwd", "lz_s
            "lz_hybrid_bwd", "lz_gla_decode_step", "lz_workspace_bytes", "lz_last_error",
            "lz_version", "lz_timing_enable", "lz_timing_read", "lz_swa_meta_bwd_noalloc",
            "lz_device_check", "lz_prefer_tcgen05", "lz_decode_prefill", "lz_hybrid_fwd_mse",
-           "lz_selftest_bounded_wait", "lz_cp_segment_decay", "lz_cp_fold", "lz_cp_rows")
+           "lz_selftest_bounded_wait", "lz_cp_segment_decay", "lz_cp_fold", "lz_cp_rows",
+           "lz_gated_bwd_tcgen05", "lz_qkg_projection")
 
 # size of the static scratch array behind lz_swa_meta_bwd_noalloc
 LZ_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -85,6 +86,8 @@ def load(path: str = LIB_PATH):
     lib.lz_decode_prefill.argtypes = [ctypes.c_int] * 7 + [_P] * 8 + [_P]
     lib.lz_prefer_tcgen05.argtypes = [ctypes.c_int]
     ci = ctypes.c_int
+    lib.lz_gated_bwd_tcgen05.argtypes = [ci]
+    lib.lz_qkg_projection.argtypes = [ci] * 5 + [_P] * 4 + [ctypes.c_float] + [_P] * 3 + [_P]
     lib.lz_cp_segment_decay.argtypes = [ci, ci, ci, _P, _P, _P]
     lib.lz_cp_fold.argtypes = [ci] * 6 + [_P] * 4 + [_P]
     lib.lz_cp_rows.argtypes = ([ci] * 4 + [_P, ci, ci, ctypes.c_float, _P, ci, ci, _P, ci, ci] +
@@ -162,10 +165,17 @@ def lz_selftest_bounded_wait(stream=None):
 
 
 def lz_prefer_tcgen05(on: bool) -> bool:
-    """Window forward on the tcgen05 kernel where it applies (the default) or,
-    with False, on the warp-level kernel, for the calling thread; returns the
+    """Window kernels on tcgen05 where they apply (the default) or, with
+    False, on the warp-level ones, for the calling thread; returns the
     previous setting."""
     return bool(load().lz_prefer_tcgen05(1 if on else 0))
+
+
+def lz_gated_bwd_tcgen05(on: bool) -> bool:
+    """Gated backward's per-chunk gradients on the tcgen05 kernel (True) or
+    the warp-level one (False, the default), for the calling thread; returns
+    the previous setting."""
+    return bool(load().lz_gated_bwd_tcgen05(1 if on else 0))
 
 
 def lz_timing_enable(on: bool):
@@ -494,4 +504,26 @@ def cp_rows(dst, dst_off, n, A=None, a_off=0, a_scale=1.0, B=None, b_off=0):
     lz_cp_rows(Bb * H, d, io_of(dst.dtype), n, A, 0 if A is None else A.shape[2], a_off, a_scale,
                B, 0 if B is None else B.shape[2], b_off, dst, dT, dst_off)
     return dst
+
+
+# ---- the projections in front of the operator ------------------------------
+def lz_qkg_projection(B, T, Dm, H, dk, x, Wq, Wk, Wg, gate_scale, q, k, g, stream=None):
+    _check(load().lz_qkg_projection(B, T, Dm, H, dk, _ptr(x), _ptr(Wq), _ptr(Wk), _ptr(Wg),
+                                    float(gate_scale), _ptr(q), _ptr(k), _ptr(g),
+                                    _stream(stream)))
+
+
+def qkg_projection(x, Wq=None, Wk=None, Wg=None, *, heads, gate_scale=1.0, stream=None):
+    """x [B, T, Dm] bf16, W [heads * dk, Dm] bf16 -> (q, k, g): q, k [B, heads,
+    T, dk] bf16 and g = gate_scale * logsigmoid(x Wg^T) [B, heads, T, dk] fp32
+    (None where the weight is None)."""
+    B, T, Dm = x.shape
+    Wany = next(w for w in (Wq, Wk, Wg) if w is not None)
+    dk = Wany.shape[0] // heads
+    dev = x.device
+    q = torch.empty(B, heads, T, dk, dtype=torch.bfloat16, device=dev) if Wq is not None else None
+    k = torch.empty(B, heads, T, dk, dtype=torch.bfloat16, device=dev) if Wk is not None else None
+    g = torch.empty(B, heads, T, dk, dtype=torch.float32, device=dev) if Wg is not None else None
+    lz_qkg_projection(B, T, Dm, heads, dk, x, Wq, Wk, Wg, gate_scale, q, k, g, stream)
+    return q, k, g
 

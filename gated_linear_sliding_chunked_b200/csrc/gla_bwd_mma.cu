@@ -115,6 +115,7 @@ struct ChunkSmem {
   float ck[NSB][DKH];
   float ksr[NSB][DKH];  // (k e^{b_l - b}) / kf per (sub-block, key dim)
   float tot[NSB][DKH];
+  float bdg[2][C];      // fp32 dO_t . v_t (the diagonal pairs), per role
 };
 static_assert(sizeof(ChunkSmem) + 1024 <= 232448 / 2, "two chunk CTAs must fit one SM");
 static_assert(sizeof(float) * C * RP <= sizeof(bf16) * C * VP, "dg staging must fit the v tile");
@@ -170,6 +171,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
   const int i0 = half * DKH;        // first key dim of this CTA
   const int T = p.T, nchunks = (T + C - 1) / C;
   const int c = (int)((blockIdx.x >> 1) % (unsigned)nchunks), bh = (int)((blockIdx.x >> 1) / (unsigned)nchunks);
+  // chunks the tcgen05 kernel has computed (both CTAs of the cluster leave)
+  if (p.tc_flags && p.tc_flags[(size_t)bh * ((T + 2 * C - 1) / (2 * C)) + c / 2] == 0) return;
   const int c0 = c * C;
   const int rows = min(C, T - c0);
   const size_t tk = (size_t)bh * T * DK, tv = (size_t)bh * T * DV;
@@ -382,7 +385,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
   }
   // ---- intra: one 16x16 score block at a time, consumed right away -------
   const int jlo = role == 0 ? 0 : I, jhi = role == 0 ? I : NSB - 1;
-  float bdiag[2] = {0.f, 0.f};  // fp32 dO_t . v_t of rows 16I + gr and 16I + gr + 8
+
   for (int J = jlo; J <= jhi; ++J) {
     float sc[2][4], sc2[2][4];  // two partial sums over k for independent MMA chains
 #pragma unroll
@@ -414,9 +417,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
     if (J == I) {
       // the diagonal (t, t) of row gr (gr + 8) sits in lane 4 gr + gr / 2,
       // fragment element (gr & 1) of column tile 0 (1)
-      const int src = gr * 4 + (gr >> 1);
-      bdiag[0] = __shfl_sync(0xffffffffu, (gr & 1) ? sc[0][1] : sc[0][0], src);
-      bdiag[1] = __shfl_sync(0xffffffffu, (gr & 1) ? sc[1][3] : sc[1][2], src);
+      // the diagonal (t, t) of row gr (gr + 8) sits in lane 4 gr + gr / 2,
+      // fragment element (gr & 1) of column tile 0 (1)
+      if ((lane & 3) == (gr >> 1)) {
+        sm.bdg[role][16 * I + gr] = (gr & 1) ? sc[0][1] : sc[0][0];
+        sm.bdg[role][16 * I + gr + 8] = (gr & 1) ? sc[1][3] : sc[1][2];
+      }
       if (slow) continue;  // the diagonal block of a strong-decay chunk: below
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
@@ -446,6 +452,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
       mma_bf16(acc[2 * ntp + 1], pa, b2, b3);
     }
   }
+  __syncwarp();
   // ---- finalize (dq | dk) = (Eq | Ek) * acc + diagonal, store; keep the
   // products (Qf acc_q | Kf acc_k) for dg -----------------------------------
   {
@@ -483,7 +490,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
           const float2 xo = unpack_bf16(rv[n][hh]);
           const float a0 = acc[nt][2 * hh], a1 = acc[nt][2 * hh + 1];
           float p0 = fq.x * a0, p1 = fq.y * a1;
-          float x0 = a0 * os.x + bdiag[hh] * xo.x, x1 = a1 * os.y + bdiag[hh] * xo.y;
+          const float bd = sm.bdg[role][t];
+          float x0 = a0 * os.x + bd * xo.x, x1 = a1 * os.y + bd * xo.y;
           if (slow) {
             const float d0 = diag_intra_term(sm.dO, sm.v, raw, gsrc, rows, I, t, il, role);
             const float d1 = diag_intra_term(sm.dO, sm.v, raw, gsrc, rows, I, t, il + 1, role);

@@ -96,6 +96,9 @@ struct GlaBwdParams {
   const float* gsp;
   const void* gz;        // gate logits (see GlaFwdParams); dg then receives dL/dz
   float gs;
+  const int* tc_flags;   // nullable: [BH][ceil(T/128)] from launch_gla_bwd_tc; the
+                         // per-64-row kernel then runs only the chunks flagged 1
+  unsigned int* status;  // device status word (tcgen05 kernel; set by its launcher)
 };
 cudaError_t launch_gla_bwd_simt(const GlaBwdParams& p, bool bf16, cudaStream_t s);
 
@@ -152,6 +155,14 @@ cudaError_t launch_loss_reduce(const float* part, size_t nparts, double inv_n, f
 // launch_gla_bwd_scan's gin16 / gsp; all chunks in parallel.
 bool gla_bwd_mma_supported(int dk, int dv, bool bf16);
 cudaError_t launch_gla_bwd_chunks(const GlaBwdParams& p, cudaStream_t s);
+// The same gradients on tcgen05 for 128-token chunks whose gates keep each
+// 64-row half's decay within e^-60 in every key dim (fp32 log-gates, bf16,
+// dk = dv = 128, after launch_gla_bwd_scan): flags[bh][c] = 0 for a chunk it
+// computed, 1 for one it left to launch_gla_bwd_chunks (run next with
+// p.tc_flags = flags).
+bool gla_bwd_tc_supported(const GlaBwdParams& p);
+int gla_bwd_tc_nchunks(int T);
+cudaError_t launch_gla_bwd_tc(const GlaBwdParams& p, int* flags, cudaStream_t s);
 
 // ---- window + meta softmax, SIMT path ------------------------------------
 struct SwaFwdParams {

@@ -13,6 +13,7 @@ namespace {
 
 thread_local std::string g_err;
 thread_local bool g_prefer_tc = true;  // lz_prefer_tcgen05
+thread_local bool g_gated_bwd_tc = false;  // lz_gated_bwd_tcgen05
 
 // The window branch's forward for bf16 with dk = dv = 128: tcgen05 for
 // w <= 129 (unless the calling thread asked for the warp-level kernel),
@@ -242,6 +243,7 @@ struct GlaBwdWs {
   ScanWs scan;
   void* gin16;  // two-level backward: state gradient entering every chunk (bf16)
   float* gsp;   // and <G_new, S_prev> per chunk and key dim
+  int* tcflags; // per 128-token chunk: left by the tcgen05 kernel to the per-64-row one
 };
 GlaBwdWs carve_gla_bwd(Carver& c, const lz_dims* d) {
   GlaBwdWs w{};
@@ -252,6 +254,7 @@ GlaBwdWs carve_gla_bwd(Carver& c, const lz_dims* d) {
     w.gin16 = c.take<uint16_t>(states16_count(d));
     const size_t n64 = (size_t)((d->T + lz::gla_fwd_mma_chunk() - 1) / lz::gla_fwd_mma_chunk());
     w.gsp = c.take<float>(bh * n64 * d->dk);
+    w.tcflags = c.take<int>(bh * (size_t)lz::gla_bwd_tc_nchunks(d->T));
   } else {
     w.states = c.take<float>(bh * nchunks16(d) * d->dk * d->dv);
   }
@@ -407,6 +410,12 @@ const char* lz_version(void) { return "lizard-b200 0.1 (sm_100a)"; }
 int lz_prefer_tcgen05(int on) {
   const int prev = g_prefer_tc ? 1 : 0;
   g_prefer_tc = on != 0;
+  return prev;
+}
+
+int lz_gated_bwd_tcgen05(int on) {
+  const int prev = g_gated_bwd_tc ? 1 : 0;
+  g_gated_bwd_tc = on != 0;
   return prev;
 }
 
@@ -619,9 +628,19 @@ static cudaError_t gla_bwd_phase1(const lz_dims* d, const void* q, const void* k
   return lz::launch_gla_bwd_scan(sp, s);
 }
 
-static cudaError_t gla_bwd_phase2(const lz_dims* d, const lz::GlaBwdParams& p, cudaStream_t s) {
+static cudaError_t gla_bwd_phase2(const lz_dims* d, const lz::GlaBwdParams& p, int* tcflags,
+                                  cudaStream_t s) {
   if (!bwd_uses_mma(d)) return lz::launch_gla_bwd_simt(p, d->io == LZ_BF16, s);
-  return lz::launch_gla_bwd_chunks(p, s);  // every chunk at once
+  // every chunk at once: tcgen05 for the chunks whose gate factors stay
+  // bounded over 128 tokens, then the per-64-row kernel for the others
+  if (g_gated_bwd_tc && tcflags && lz::gla_bwd_tc_supported(p)) {
+    cudaError_t e = lz::launch_gla_bwd_tc(p, tcflags, s);
+    if (e != cudaSuccess) return e;
+    lz::GlaBwdParams q = p;
+    q.tc_flags = tcflags;
+    return lz::launch_gla_bwd_chunks(q, s);
+  }
+  return lz::launch_gla_bwd_chunks(p, s);
 }
 
 static cudaError_t gla_bwd_launch(const lz_dims* d, const void* q, const void* k, const void* v,
@@ -635,7 +654,7 @@ static cudaError_t gla_bwd_launch(const lz_dims* d, const void* q, const void* k
   cudaError_t e = gla_bwd_phase1(d, q, k, v, g, h0, dO, dhT, saved_states, saved_hT, dq, dk, dv, dg,
                                  dh0, w, add_dq, add_dk, add_dv, add_in_place, p, s);
   if (e != cudaSuccess) return e;
-  return gla_bwd_phase2(d, p, s);
+  return gla_bwd_phase2(d, p, w.tcflags, s);
 }
 
 
@@ -745,7 +764,7 @@ lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const vo
   const cudaError_t ew = cudaStreamWaitEvent(s, ss->join, 0);
   if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (window branch)");
   if (ew != cudaSuccess) return cuda_status(ew, "lz_hybrid_bwd (join)");
-  return cuda_status(gla_bwd_phase2(d, gp, s), "lz_hybrid_bwd (gated branch)");
+  return cuda_status(gla_bwd_phase2(d, gp, w.gla.tcflags, s), "lz_hybrid_bwd (gated branch)");
 }
 
 lz_status lz_decode_prefill(int Bd, int H, int T, int dk, int dv, int w, lz_dtype io,

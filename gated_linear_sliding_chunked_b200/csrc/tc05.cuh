@@ -88,6 +88,15 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* map, uint3
       : "memory");
 }
 
+// Box at (c0, c1) of the 2-D tensor map `map`; same rules.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* map, uint32_t bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+
 // ---- proxies and ordering -------------------------------------------------
 // Makes this thread's generic-proxy shared-memory writes (st.shared,
 // cp.async) visible to the tensor core's async proxy.
@@ -125,10 +134,17 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return sdesc(saddr, lbo, sbo) | (2ull << 61);
 }
 // Instruction descriptor of kind::f16 with bf16 A and B, fp32 accumulation,
-// K-major A; B K-major (b_mn = false) or MN-major (b_mn = true).
+// K-major A (bit 15 clear); B K-major (b_mn = false) or MN-major (b_mn =
+// true, bit 16).
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn ? 1u : 0u) << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// The same with A MN-major as well (A read transposed from a tile whose rows
+// run along K).
+__host__ __device__ constexpr uint32_t idesc_bf16_at(int M, int N, bool b_mn) {
+  return idesc_bf16(M, N, b_mn) | (1u << 15);
 }
 
 // D[tmem] (+)= A[smem] * B[smem]; issued by one thread.

@@ -12,4 +12,9 @@ namespace lz {
 // available or rejects the map.
 bool tma_map_rows128(CUtensorMap* map, const void* base, uint64_t d1, uint64_t d2, uint32_t rows);
 
+// 2-D map over a row-major bf16 matrix [rows][cols] (cols * 2 a multiple of
+// 16 bytes), boxes of 64 columns x `box_rows` rows with the 128-byte swizzle;
+// elements outside the matrix read as zeros.
+bool tma_map_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows);
+
 }  // namespace lz

@@ -281,6 +281,26 @@ lz_status lz_decode_prefill(int Bd, int H, int T, int dk, int dv, int w,
                             float* state, void* kring, void* vring,
                             int64_t* pos, lz_stream stream);
 
+/* The projections in front of the operator (section 2a: the gate is
+ * Gamma_i = sigma(W_gamma x_i) and the state update takes phi(k_i); the pages
+ * do not define phi, read here as the identity, the featurised keys being
+ * the operator's input).  From hidden states x [B,T,Dm] (bf16, row-major)
+ * and weights W [H*dk, Dm] (bf16, one row per output feature, as a linear
+ * layer stores them), one launch computes any of
+ *   q = x Wq^T,  k = x Wk^T  -> [B,H,T,dk] bf16 (rounded once),
+ *   g = gate_scale * log sigma(x Wg^T) -> [B,H,T,dk] fp32 log-gates,
+ * on tcgen05 tensor cores (fp32 accumulation), the gate's logit never
+ * leaving the chip.  A NULL weight skips its output (its output pointer must
+ * then be NULL too).  Requirements: Dm a multiple of 8, dk = 64 or 128, H*dk
+ * a multiple of 256, gate_scale > 0, 16-byte aligned pointers.  Caller-owned
+ * device memory; asynchronous on `stream`; bad arguments return
+ * LZ_ERR_INVALID_ARG / LZ_ERR_UNSUPPORTED before any launch.  A bounded
+ * device wait that gives up is reported by lz_device_check. */
+lz_status lz_qkg_projection(int B, int T, int Dm, int H, int dk, const void* x,
+                            const void* Wq, const void* Wk, const void* Wg,
+                            float gate_scale, void* q, void* k, float* g,
+                            lz_stream stream);
+
 /* ---- Context parallelism: one sequence over R ranks ----------------------
  * The pages run each layer on one device; splitting a long sequence into R
  * contiguous segments (rank r holds tokens [r Ts, (r+1) Ts) of every
@@ -342,15 +362,27 @@ lz_status lz_device_check(lz_stream stream);
  * LZ_ERR_CUDA if the launch failed. */
 lz_status lz_selftest_bounded_wait(lz_stream stream);
 
-/* Kernel choice of the window branch for the calling host thread (no
- * counterpart on the pages).  bf16 with dk = dv = 128 has tcgen05 kernels
- * with TMA-fed operands and accumulators in tensor memory (the default) and
- * warp-level mma.sync kernels: the forward uses tcgen05 for w <= 129 (the
- * scores of the whole band fit in tensor memory), the key side of the
- * backward (dk, dv) for every w.  lz_prefer_tcgen05(0) selects the
- * warp-level kernels; both give the same result up to rounding.  Returns
- * the previous setting; never fails. */
+/* Kernel choice for the calling host thread (no counterpart on the pages).
+ * bf16 with dk = dv = 128 has tcgen05 kernels with TMA-fed operands and
+ * accumulators in tensor memory (the default) and warp-level mma.sync
+ * kernels: the window forward uses tcgen05 for w <= 129 (the scores of the
+ * whole band fit in tensor memory) and the key side of the window backward
+ * (dk, dv) for every w.  lz_prefer_tcgen05(0) selects the warp-level
+ * kernels; both give the same result up to rounding.  Returns the previous
+ * setting; never fails. */
 int lz_prefer_tcgen05(int on);
+
+/* Kernel choice of the gated backward's per-chunk gradients for the calling
+ * host thread (no counterpart on the pages).  bf16 with dk = dv = 128 has a
+ * warp-level mma.sync kernel over 64-token chunks (the default: faster on
+ * B200, see the design notes) and a tcgen05 kernel over 128-token chunks
+ * (TMA-fed operands, every contraction with M = 128 and its accumulator in
+ * tensor memory).  With lz_gated_bwd_tcgen05(1) the tcgen05 kernel takes
+ * every 128-token chunk whose fp32 log-gates decay each 64-token half by at
+ * most e^-60 in every key dim; faster-decaying chunks, and gates given as
+ * logits, stay on the warp-level kernel.  Both give the same result up to
+ * rounding.  Returns the previous setting; never fails. */
+int lz_gated_bwd_tcgen05(int on);
 
 /* Per-launch device timing for benchmarks (no counterpart on the pages; a
  * measurement aid).  lz_timing_enable(1) makes every later kernel launch of

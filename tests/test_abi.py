@@ -269,3 +269,21 @@ def test_context_parallel_validation(lib):
     assert r(4, 128, 7, 10, FAKE, 64, 0, 1.0, None, 0, 0, FAKE, 64, 0, 0) == L.LZ_ERR_UNSUPPORTED
     assert r(4, 128, L.LZ_BF16, 0, None, 0, 0, 1.0, None, 0, 0, FAKE, 64, 0, 0) == L.LZ_OK
 
+
+def test_projection_validation(lib):
+    """The projection refuses bad arguments before any launch."""
+    f = lib.lz_qkg_projection
+    ok = dict(B=2, T=8, Dm=256, H=2, dk=128)
+    args = lambda **kw: [kw.get(n, ok[n]) for n in ("B", "T", "Dm", "H", "dk")]
+    P = [FAKE, FAKE, FAKE, FAKE]  # x, Wq, Wk, Wg
+    O = [FAKE, FAKE, FAKE]        # q, k, g
+    assert f(*args(Dm=100), *P, ctypes.c_float(1.0), *O, 0) == L.LZ_ERR_UNSUPPORTED
+    assert f(*args(dk=96), *P, ctypes.c_float(1.0), *O, 0) == L.LZ_ERR_UNSUPPORTED
+    assert f(*args(H=1), *P, ctypes.c_float(1.0), *O, 0) == L.LZ_ERR_UNSUPPORTED  # H*dk = 128
+    assert f(*args(), *P, ctypes.c_float(0.0), *O, 0) == L.LZ_ERR_INVALID_ARG
+    assert f(*args(), FAKE, FAKE, None, FAKE, ctypes.c_float(1.0), *O, 0) == L.LZ_ERR_INVALID_ARG
+    assert b"both" in lib.lz_last_error()
+    assert f(*args(), FAKE + 8, FAKE, FAKE, FAKE, ctypes.c_float(1.0), *O, 0) == \
+        L.LZ_ERR_INVALID_ARG
+    assert f(*args(T=0), *P, ctypes.c_float(1.0), *O, 0) == L.LZ_OK
+

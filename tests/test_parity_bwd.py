@@ -110,6 +110,31 @@ def test_hybrid_bwd(dtype, alpha, saved):
     assert_close("dalpha", res["dalpha"].cpu().double().numpy(), np.array([ref["dalpha"]]), dtype)
 
 
+@pytest.mark.parametrize("T", [1, 64, 128, 129, 300, 700])
+@pytest.mark.parametrize("tc", [True, False], ids=["tcgen05", "warp-mma"])
+def test_gla_bwd_kernels(T, tc):
+    """Both bf16 per-chunk backward kernels (tcgen05 over 128-token chunks and
+    warp-level over 64-token chunks) against the oracle, with the kernel that
+    ran named by the library's launch timing and a clean status word."""
+    cpu, dev = small_problem(300 + T, 2, 2, T, 128, 128, 0, torch.bfloat16, train=True, h0=True)
+    prev = L.lz_gated_bwd_tcgen05(tc)
+    L.lz_timing_enable(True)
+    try:
+        res = L.gla_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["dO"], dev["h0"], dev["dhT"],
+                        want_dh0=True)
+        torch.cuda.synchronize()
+    finally:
+        L.lz_timing_enable(False)
+        L.lz_gated_bwd_tcgen05(prev)
+    ran = {name for name, _ in L.lz_timing_read()}
+    assert ("gla_bwd_chunks_tc" in ran) == tc, ran
+    L.lz_device_check()
+    x = oracle_inputs(cpu, ("q", "k", "v", "g", "dO", "h0", "dhT"))
+    ref = oracle.gla_bwd(x["q"], x["k"], x["v"], x["g"], x["dO"], x["h0"], x["dhT"])
+    for name in ("dq", "dk", "dv", "dg", "dh0"):
+        assert_close(name, res[name], ref[name], torch.bfloat16)
+
+
 def test_gla_bwd_full_forgetting():
     """g = -30 everywhere: the elementwise-exponent path of the backward."""
     cpu, dev = small_problem(3, 1, 2, 45, 64, 64, 0, torch.float32, train=True)
@@ -122,8 +147,9 @@ def test_gla_bwd_full_forgetting():
         assert_close(name, res[name], ref[name], torch.float32)
 
 
+@pytest.mark.parametrize("tc", [False, True], ids=["warp-mma", "tcgen05"])
 @pytest.mark.parametrize("fill", [0.0, -30.0, "mixed", "one-dim", "strong"])
-def test_gla_bwd_gate_edge_cases_bf16(fill):
+def test_gla_bwd_gate_edge_cases_bf16(fill, tc):
     """The tensor-core backward's gate paths (bf16, d = 128): g = 0 (no
     decay), g = -30 (full forgetting: elementwise diagonal blocks), a mixture
     inside each chunk, one fast-decaying key dim among slow ones (per-pair
@@ -144,8 +170,12 @@ def test_gla_bwd_gate_edge_cases_bf16(fill):
         g = torch.nn.functional.logsigmoid(torch.randn(1, 2, T, 128, generator=gen) * 1.5 - 1.0)
     else:
         g = torch.full((1, 2, T, 128), float(fill))
-    res = L.gla_bwd(dev["q"], dev["k"], dev["v"], g.cuda(), dev["dO"], dev["h0"], dev["dhT"],
-                    want_dh0=True)
+    prev = L.lz_gated_bwd_tcgen05(tc)  # tcgen05: the fast-decaying chunks fall back
+    try:
+        res = L.gla_bwd(dev["q"], dev["k"], dev["v"], g.cuda(), dev["dO"], dev["h0"], dev["dhT"],
+                        want_dh0=True)
+    finally:
+        L.lz_gated_bwd_tcgen05(prev)
     x = oracle_inputs(cpu, ("q", "k", "v", "dO", "h0", "dhT"))
     ref = oracle.gla_bwd(x["q"], x["k"], x["v"], g.double().numpy(), x["dO"], x["h0"], x["dhT"])
     for name in ("dq", "dk", "dv", "dh0", "dg"):
@@ -177,20 +207,27 @@ def test_bwd_determinism():
         assert torch.equal(runs[0][name], runs[1][name]), name
 
 
-def test_workload_train_sampled():
+@pytest.mark.parametrize("tc", [False, True], ids=["warp-mma", "tcgen05"])
+def test_workload_train_sampled(tc):
     """Llama-3-8B-shaped training layer (B=2, H=32, T=8192): fwd + bwd at full
     size on the GPU; every per-token gradient checked on sampled heads, meta
-    gradients for one head exactly (both batch rows), dalpha over all heads."""
+    gradients for one head exactly (both batch rows), dalpha over all heads.
+    tc: the gated backward's per-chunk gradients on the tcgen05 kernel."""
     wl = I.TRAIN_BF16
     x = I.make_inputs(wl, seed=0, device="cpu")
     dev = {k: v.cuda() for k, v in x.items()}
     fwd = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
                        w=wl.w, alpha=wl.alpha, chunk=wl.chunk, want_lse=True, want_o_swa=True,
                        want_chunk_states=True)
-    res = L.hybrid_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
-                       fwd["lse"], dev["dO"], w=wl.w, alpha=wl.alpha, chunk=wl.chunk,
-                       o_swa=fwd["o_swa"], chunk_states=fwd["chunk_states"])
+    prev = L.lz_gated_bwd_tcgen05(tc)
+    try:
+        res = L.hybrid_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
+                           fwd["lse"], dev["dO"], w=wl.w, alpha=wl.alpha, chunk=wl.chunk,
+                           o_swa=fwd["o_swa"], chunk_states=fwd["chunk_states"])
+    finally:
+        L.lz_gated_bwd_tcgen05(prev)
     torch.cuda.synchronize()
+    L.lz_device_check()
     h = 5
     for b in range(wl.B):
         sl = lambda t: np64(t[b:b + 1, h:h + 1])

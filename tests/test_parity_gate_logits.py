@@ -57,20 +57,26 @@ def test_hybrid_fwd_bwd_with_gate_logits(T):
 
 def test_gate_logits_equal_the_log_gates_they_stand_for():
     """The same problem given as logits and as the fp32 log-gates they map
-    to: outputs and gradients agree to far below the bf16 bar, and dz is the
-    chain rule applied to the log-gate run's dg."""
+    to, through the same kernels (the warp-level ones: gates given as logits
+    always take them): outputs and gradients agree to far below the bf16 bar,
+    and dz is the chain rule applied to the log-gate run's dg."""
     s, w, alpha, T = 0.25, 64, 0.5, 300
     cpu, dev, z, x = _case(71, T, mu=1.0, sigma=1.5, s=s)
     zd = z.cuda()
     g32 = torch.from_numpy(x["g"]).float().cuda()
     out = {}
-    for key, gate in (("z", zd), ("g", g32)):
-        f = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], gate, dev["meta_k"], dev["meta_v"], w=w,
-                         alpha=alpha, h0=dev["h0"], gate_scale=s, want_hT=True, want_lse=True)
-        b = L.hybrid_bwd(dev["q"], dev["k"], dev["v"], gate, dev["meta_k"], dev["meta_v"],
-                         f["lse"], dev["dO"], w=w, alpha=alpha, h0=dev["h0"], dhT=dev["dhT"],
-                         gate_scale=s, want_dh0=True)
-        out[key] = (f, b)
+    prev = L.lz_prefer_tcgen05(False)
+    try:
+        for key, gate in (("z", zd), ("g", g32)):
+            f = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], gate, dev["meta_k"], dev["meta_v"],
+                             w=w, alpha=alpha, h0=dev["h0"], gate_scale=s, want_hT=True,
+                             want_lse=True)
+            b = L.hybrid_bwd(dev["q"], dev["k"], dev["v"], gate, dev["meta_k"], dev["meta_v"],
+                             f["lse"], dev["dO"], w=w, alpha=alpha, h0=dev["h0"],
+                             dhT=dev["dhT"], gate_scale=s, want_dh0=True)
+            out[key] = (f, b)
+    finally:
+        L.lz_prefer_tcgen05(prev)
     (fz, bz), (fg, bg) = out["z"], out["g"]
     for name in ("o", "hT"):
         assert_close(name, fz[name], np64(fg[name]), torch.bfloat16, factor=0.1)
