@@ -783,7 +783,7 @@ def run_profile_case(args):
         wl = I.TRAIN_BF16 if case == "train" else I.FWD_BF16.with_(train=True)
         step = TrainStep(wl, I.make_inputs(wl, seed=0, device=device), device)
         fn = step.run
-        L.lz_gated_bwd_tcgen05(case == "train-small-tc")
+        L.lz_tcgen05_all(case == "train-small-tc")
     elif case == "proj":
         H, dk, Dm, T = 32, 128, 4096, 2048
         gen = torch.Generator(device=device)

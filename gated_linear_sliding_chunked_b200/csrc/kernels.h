@@ -212,6 +212,7 @@ struct SwaBwdParams {
   int B, H, T, dkd, dvd, w, M;
   float scale;
   bool tc;               // key side on the tcgen05 kernel (bf16, d = 128)
+  bool tc_q;             // query side on the tcgen05 kernel where it applies
   unsigned int* status;  // device status word (set by the tcgen05 launcher)
 };
 // query rows per CTA of the meta-gradient pass (one partial per slab)
@@ -227,6 +228,10 @@ cudaError_t launch_swa_bwd_mma(const SwaBwdParams& p, cudaStream_t s);
 // key side (dk, dv) on tcgen05 with TMA-fed operands
 bool swa_bwd_kv_tc_supported(int dk, int dv, bool bf16);
 cudaError_t launch_swa_bwd_kv_tc(const SwaBwdParams& p, cudaStream_t s);
+// query side (dq, D, meta-gradient and dalpha partials) on tcgen05: bf16,
+// dk = dv = 128, w <= 129, M <= 16, the forward output (osw) given
+bool swa_bwd_q_tc_supported(const SwaBwdParams& p);
+cudaError_t launch_swa_bwd_q_tc(const SwaBwdParams& p, cudaStream_t s);
 
 // ---- decode --------------------------------------------------------------
 struct DecodeParams {

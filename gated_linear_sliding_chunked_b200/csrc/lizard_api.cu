@@ -13,7 +13,7 @@ namespace {
 
 thread_local std::string g_err;
 thread_local bool g_prefer_tc = true;  // lz_prefer_tcgen05
-thread_local bool g_gated_bwd_tc = false;  // lz_gated_bwd_tcgen05
+thread_local bool g_tc_all = false;  // lz_tcgen05_all
 
 // The window branch's forward for bf16 with dk = dv = 128: tcgen05 for
 // w <= 129 (unless the calling thread asked for the warp-level kernel),
@@ -388,6 +388,7 @@ lz::SwaBwdParams swa_bwd_params(const lz_dims* d, const void* q, const void* k, 
   p.q = q; p.k = k; p.v = v; p.mk = mk; p.mv = d->M > 0 ? mv : nullptr; p.lse = lse; p.dO = dO;
   p.osw = osw;
   p.tc = g_prefer_tc;
+  p.tc_q = g_prefer_tc && g_tc_all;
   p.Dbuf = w.Dbuf; p.alpha_part = w.alpha_part; p.meta_part = w.meta_part;
   p.B = d->B; p.H = d->H; p.T = d->T; p.dkd = d->dk; p.dvd = d->dv; p.w = d->w; p.M = d->M;
   p.scale = d->scale;
@@ -413,9 +414,9 @@ int lz_prefer_tcgen05(int on) {
   return prev;
 }
 
-int lz_gated_bwd_tcgen05(int on) {
-  const int prev = g_gated_bwd_tc ? 1 : 0;
-  g_gated_bwd_tc = on != 0;
+int lz_tcgen05_all(int on) {
+  const int prev = g_tc_all ? 1 : 0;
+  g_tc_all = on != 0;
   return prev;
 }
 
@@ -633,7 +634,7 @@ static cudaError_t gla_bwd_phase2(const lz_dims* d, const lz::GlaBwdParams& p, i
   if (!bwd_uses_mma(d)) return lz::launch_gla_bwd_simt(p, d->io == LZ_BF16, s);
   // every chunk at once: tcgen05 for the chunks whose gate factors stay
   // bounded over 128 tokens, then the per-64-row kernel for the others
-  if (g_gated_bwd_tc && tcflags && lz::gla_bwd_tc_supported(p)) {
+  if (g_tc_all && tcflags && lz::gla_bwd_tc_supported(p)) {
     cudaError_t e = lz::launch_gla_bwd_tc(p, tcflags, s);
     if (e != cudaSuccess) return e;
     lz::GlaBwdParams q = p;

@@ -526,14 +526,18 @@ cudaError_t launch_swa_bwd_mma(const SwaBwdParams& p, cudaStream_t s) {
   const int nslab = (p.T + SLAB - 1) / SLAB;
   cudaError_t e = cudaSuccess;
   if (!empty) {
-    const size_t b1 = sizeof(QSmem);
-    e = cudaFuncSetAttribute(swa_bwd_q_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)b1);
-    if (e != cudaSuccess) return e;
-    {
-      ScopedTiming tm("swa_bwd_q_mma", s);
-      swa_bwd_q_mma_kernel<<<dim3(p.H, p.B, nslab), NT, b1, s>>>(p);
+    if (p.tc_q && swa_bwd_q_tc_supported(p)) {
+      e = launch_swa_bwd_q_tc(p, s);
+    } else {
+      const size_t b1 = sizeof(QSmem);
+      e = cudaFuncSetAttribute(swa_bwd_q_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)b1);
+      if (e != cudaSuccess) return e;
+      {
+        ScopedTiming tm("swa_bwd_q_mma", s);
+        swa_bwd_q_mma_kernel<<<dim3(p.H, p.B, nslab), NT, b1, s>>>(p);
+      }
+      e = cudaGetLastError();
     }
-    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (p.tc && swa_bwd_kv_tc_supported(p.dkd, p.dvd, true)) {
       e = launch_swa_bwd_kv_tc(p, s);

@@ -372,17 +372,21 @@ lz_status lz_selftest_bounded_wait(lz_stream stream);
  * setting; never fails. */
 int lz_prefer_tcgen05(int on);
 
-/* Kernel choice of the gated backward's per-chunk gradients for the calling
- * host thread (no counterpart on the pages).  bf16 with dk = dv = 128 has a
- * warp-level mma.sync kernel over 64-token chunks (the default: faster on
- * B200, see the design notes) and a tcgen05 kernel over 128-token chunks
- * (TMA-fed operands, every contraction with M = 128 and its accumulator in
- * tensor memory).  With lz_gated_bwd_tcgen05(1) the tcgen05 kernel takes
- * every 128-token chunk whose fp32 log-gates decay each 64-token half by at
- * most e^-60 in every key dim; faster-decaying chunks, and gates given as
- * logits, stay on the warp-level kernel.  Both give the same result up to
- * rounding.  Returns the previous setting; never fails. */
-int lz_gated_bwd_tcgen05(int on);
+/* tcgen05 kernels where the warp-level ones measured faster on B200, for the
+ * calling host thread (no counterpart on the pages; default off).  With
+ * lz_tcgen05_all(1):
+ *  - the gated backward's per-chunk gradients run on a tcgen05 kernel over
+ *    128-token chunks (TMA-fed operands, every contraction with M = 128 and
+ *    its accumulator in tensor memory) for every chunk whose fp32 log-gates
+ *    decay each 64-token half by at most e^-60 in every key dim
+ *    (faster-decaying chunks, and gates given as logits, stay on the
+ *    warp-level kernel over 64-token chunks);
+ *  - the query side of the window backward (dq, D, the meta-gradient and
+ *    dalpha partials) runs on a tcgen05 kernel when lz_prefer_tcgen05 is on,
+ *    w <= 129, M <= 16 and the forward's window output is given.
+ * Both choices give the same result up to rounding.  Returns the previous
+ * setting; never fails. */
+int lz_tcgen05_all(int on);
 
 /* Per-launch device timing for benchmarks (no counterpart on the pages; a
  * measurement aid).  lz_timing_enable(1) makes every later kernel launch of

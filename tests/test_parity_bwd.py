@@ -65,25 +65,35 @@ def test_swa_meta_bwd(dtype, T, w, M, sink, with_o):
             assert_close("dmeta_v", res["dmeta_v"], ref["dmeta_v"], dtype)
 
 
-@pytest.mark.parametrize("T,w,M", [(1, 1, 2), (300, 64, 4), (1100, 128, 8), (260, 700, 0)])
-@pytest.mark.parametrize("tc", [True, False], ids=["tcgen05", "warp-mma"])
-def test_swa_meta_bwd_kernels(T, w, M, tc):
-    """Both bf16 key-side kernels (tcgen05 and warp-level) against the oracle,
-    with a clean device status word afterwards."""
+@pytest.mark.parametrize("T,w,M", [(1, 1, 2), (300, 64, 4), (1100, 128, 8), (260, 700, 0),
+                                   (513, 129, 16), (700, 33, 0)])
+@pytest.mark.parametrize("mode", ["tcgen05", "warp-mma", "tcgen05-all"])
+def test_swa_meta_bwd_kernels(T, w, M, mode):
+    """The bf16 window-backward kernels against the oracle: the key side on
+    tcgen05 (default) or warp-level, and with lz_tcgen05_all also the query
+    side on tcgen05 (w <= 129); a clean device status word afterwards."""
     cpu, dev = small_problem(90 + T + w, 2, 2, T, 128, 128, M, torch.bfloat16, train=True)
     mk = dev["meta_k"] if M else None
     mv = dev["meta_v"] if M else None
-    prev = L.lz_prefer_tcgen05(tc)
+    prev = L.lz_prefer_tcgen05(mode != "warp-mma")
+    prev_all = L.lz_tcgen05_all(mode == "tcgen05-all")
     try:
         o, lse = L.swa_meta_fwd(dev["q"], dev["k"], dev["v"], mk, mv, w=w)
+        L.lz_timing_enable(True)
         res = L.swa_meta_bwd(dev["q"], dev["k"], dev["v"], mk, mv, lse, dev["dO"], w=w, o=o)
+        torch.cuda.synchronize()
     finally:
+        L.lz_timing_enable(False)
         L.lz_prefer_tcgen05(prev)
+        L.lz_tcgen05_all(prev_all)
+    ran = {name for name, _ in L.lz_timing_read()}
+    if T > 0:
+        assert ("swa_bwd_q_tc" in ran) == (mode == "tcgen05-all" and w <= 129), ran
     L.lz_device_check()
     x = oracle_inputs(cpu, ("q", "k", "v", "meta_k", "meta_v", "dO"))
     ref = oracle.swa_meta_bwd(x["q"], x["k"], x["v"], x["meta_k"] if M else None,
                               x["meta_v"] if M else None, x["dO"], w, 1 / math.sqrt(128))
-    for name in ("dq", "dk", "dv"):
+    for name in ("dq", "dk", "dv") + (("dmeta_k", "dmeta_v") if M else ()):
         assert_close(name, res[name], ref[name], torch.bfloat16)
 
 
@@ -117,7 +127,7 @@ def test_gla_bwd_kernels(T, tc):
     warp-level over 64-token chunks) against the oracle, with the kernel that
     ran named by the library's launch timing and a clean status word."""
     cpu, dev = small_problem(300 + T, 2, 2, T, 128, 128, 0, torch.bfloat16, train=True, h0=True)
-    prev = L.lz_gated_bwd_tcgen05(tc)
+    prev = L.lz_tcgen05_all(tc)
     L.lz_timing_enable(True)
     try:
         res = L.gla_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["dO"], dev["h0"], dev["dhT"],
@@ -125,7 +135,7 @@ def test_gla_bwd_kernels(T, tc):
         torch.cuda.synchronize()
     finally:
         L.lz_timing_enable(False)
-        L.lz_gated_bwd_tcgen05(prev)
+        L.lz_tcgen05_all(prev)
     ran = {name for name, _ in L.lz_timing_read()}
     assert ("gla_bwd_chunks_tc" in ran) == tc, ran
     L.lz_device_check()
@@ -170,12 +180,12 @@ def test_gla_bwd_gate_edge_cases_bf16(fill, tc):
         g = torch.nn.functional.logsigmoid(torch.randn(1, 2, T, 128, generator=gen) * 1.5 - 1.0)
     else:
         g = torch.full((1, 2, T, 128), float(fill))
-    prev = L.lz_gated_bwd_tcgen05(tc)  # tcgen05: the fast-decaying chunks fall back
+    prev = L.lz_tcgen05_all(tc)  # tcgen05: the fast-decaying chunks fall back
     try:
         res = L.gla_bwd(dev["q"], dev["k"], dev["v"], g.cuda(), dev["dO"], dev["h0"], dev["dhT"],
                         want_dh0=True)
     finally:
-        L.lz_gated_bwd_tcgen05(prev)
+        L.lz_tcgen05_all(prev)
     x = oracle_inputs(cpu, ("q", "k", "v", "dO", "h0", "dhT"))
     ref = oracle.gla_bwd(x["q"], x["k"], x["v"], g.double().numpy(), x["dO"], x["h0"], x["dhT"])
     for name in ("dq", "dk", "dv", "dh0", "dg"):
@@ -219,13 +229,13 @@ def test_workload_train_sampled(tc):
     fwd = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
                        w=wl.w, alpha=wl.alpha, chunk=wl.chunk, want_lse=True, want_o_swa=True,
                        want_chunk_states=True)
-    prev = L.lz_gated_bwd_tcgen05(tc)
+    prev = L.lz_tcgen05_all(tc)
     try:
         res = L.hybrid_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
                            fwd["lse"], dev["dO"], w=wl.w, alpha=wl.alpha, chunk=wl.chunk,
                            o_swa=fwd["o_swa"], chunk_states=fwd["chunk_states"])
     finally:
-        L.lz_gated_bwd_tcgen05(prev)
+        L.lz_tcgen05_all(prev)
     torch.cuda.synchronize()
     L.lz_device_check()
     h = 5
