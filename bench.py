@@ -201,6 +201,12 @@ def load_peaks():
                 "source": "fallback"}
 
 
+def hbm_peak_source(peaks) -> str:
+    if peaks["source"] == "measured":
+        return "of measured (MEASURED_PEAKS.json hbm_gbs copy)"
+    return "of fallback (6.65 TB/s copy bandwidth; MEASURED_PEAKS.json absent)"
+
+
 def algorithmic_bytes(kernel: str, wl) -> float | None:
     """Bytes the method must move per launch of ``kernel`` on workload ``wl``
     (per (batch, head, token): q, k, v, o at the I/O size, g in fp32; the
@@ -461,7 +467,7 @@ def roofline_for(tab, wl, peaks):
                  "frac": round(achieved / peaks["hbm_gbs"], 4),
                  "traffic": traffic, "launches": count, "avg_ms": round(avg_ms, 4),
                  "algorithmic_bytes_per_launch": by,
-                 "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs copy)"}
+                 "peak_source": hbm_peak_source(peaks)}
 
 
 # --------------------------------------------------------------------------
@@ -505,7 +511,7 @@ def measure_fwd(wl, device, steps, warmup, peaks, seed, tcgen05_window=True):
     roof = {"kernel": "lz_hybrid_fwd (whole call)", "bound": "hbm", "achieved": round(achieved, 1),
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
             "algorithmic_bytes_per_call": by, "avg_ms": round(call_ms, 4),
-            "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs copy)"}
+            "peak_source": hbm_peak_source(peaks)}
     del x, o, ws, flush
     return {"workload": wl.name, "tokens_per_s": wl.B * wl.T / (call_ms * 1e-3),
             "ms_per_call": round(call_ms, 4), "ms_per_iter_incl_l2_flush": round(ms, 4),
@@ -593,7 +599,9 @@ def measure_projection(device, peaks, seed, steps=10, warmup=3):
             "roofline": {"kernel": "qkg_projection_tc", "bound": "tensor", "achieved": round(tf, 1),
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": round(tf / peaks["bf16_tflops"], 4), "flops_per_call": flops,
-                         "peak_source": peaks["source"] + " (bf16_tflops, burst: timed alone)"}}
+                         "peak_source": ("of measured" if peaks["source"] == "measured" else
+                                         "of fallback (1.59 PFLOP/s)") +
+                                        " (bf16 burst figure: timed alone)"}}
 
 
 def measure_decode(device, peaks, seed, n_steps=1000):
@@ -647,7 +655,7 @@ def measure_decode(device, peaks, seed, n_steps=1000):
                          "frac": round(ach / peaks["hbm_gbs"], 4),
                          "algorithmic_bytes_per_step": bytes_step,
                          "avg_ms": round(per_step_ms, 5),
-                         "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs copy)"}}
+                         "peak_source": hbm_peak_source(peaks)}}
 
 
 # --------------------------------------------------------------------------

@@ -5,7 +5,8 @@
 // One CTA per (sequence, head).  Per step and head the kernel streams the
 // 128x128 fp32 state once in and once out (128-bit loads/stores, 16 rows x 4
 // columns per thread), reads the w-slot K/V ring and the M meta tokens once,
-// and writes one output row.  It is bound by HBM bandwidth.
+// and writes one output row.  It is bound by HBM bandwidth.  The ring rows
+// are prefetched into L2 at entry so that their reads overlap the state pass.
 //
 // The step is one launch: the H CTAs of a sequence read and advance its
 // position through one 64-bit atomic on pos[b], whose bits 48 and up count
@@ -54,6 +55,16 @@ __global__ void __launch_bounds__(NT, 5) decode_kernel(DecodeParams p) {
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
   const int w = p.w, M = p.M;
+  {  // the ring rows the window reads after the state pass: into L2 now, so that
+     // they stream from HBM beside the state instead of after it
+    constexpr int kLines = D * (int)sizeof(IO) / 128;  // 128-byte lines per ring row
+    const int n = 2 * w * kLines;
+    for (int x = tid; x < n; x += NT) {
+      const int which = x / (w * kLines), r = (x / kLines) % w, ln = x % kLines;
+      const IO* ring = (const IO*)(which ? p.vring : p.kring) + ((size_t)bh * w + r) * D;
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(ring) + ln * 128));
+    }
+  }
   if (tid == 0) {  // read the position and count this CTA in (one atomic)
     unsigned long long* pw = reinterpret_cast<unsigned long long*>(p.pos + b);
     const unsigned long long old = atomicAdd(pw, 1ull << kPosBits);

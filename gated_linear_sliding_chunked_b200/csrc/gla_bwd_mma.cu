@@ -221,6 +221,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
     }
     cp_async_commit();
   }
+  if (p.add_in_place && !p.add_dq) {
+    // the window branch's gradients, added in the epilogue, were written long
+    // before this kernel and have left L2: start bringing them back now (one
+    // 128-byte line per row: this CTA's 64 dims of dq and dk, its 64 value
+    // columns of dv)
+    const int r = tid & 63, which = tid >> 6;  // 4 x 64 threads: dq, dk, dv
+    if (which < 3 && r < rows) {
+      const bf16* base = which == 0 ? (const bf16*)p.dq : which == 1 ? (const bf16*)p.dk : (const bf16*)p.dv;
+      const size_t off = which < 2 ? tk + (size_t)(c0 + r) * DK + i0 : tv + (size_t)(c0 + r) * DV + 64 * half;
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(base + off));
+    }
+  }
   {  // tiles: v, dO, S_prev and G rows of this CTA's key dims
     const bf16* v = (const bf16*)p.v + tv + (size_t)c0 * DV;
     const bf16* dO = (const bf16*)p.dO + tv + (size_t)c0 * DV;
@@ -415,8 +427,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
 #pragma unroll
       for (int e = 0; e < 4; ++e) sc[nt][e] += sc2[nt][e];
     if (J == I) {
-      // the diagonal (t, t) of row gr (gr + 8) sits in lane 4 gr + gr / 2,
-      // fragment element (gr & 1) of column tile 0 (1)
       // the diagonal (t, t) of row gr (gr + 8) sits in lane 4 gr + gr / 2,
       // fragment element (gr & 1) of column tile 0 (1)
       if ((lane & 3) == (gr >> 1)) {
