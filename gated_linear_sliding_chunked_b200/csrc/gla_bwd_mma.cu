@@ -395,6 +395,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
     acc[nt][2] *= f.x;
     acc[nt][3] *= f.y;
   }
+  {  // the finalize's lines (raw operand and previous gradient, rows t and t + 8), into L1
+    const int tr = 16 * I + gr + ((lane & 2) ? 8 : 0);
+    if (tr < rows) {
+      if ((lane & 1) == 0)
+        asm volatile("prefetch.global.L1 [%0];" ::"l"((role == 0 ? kc : qc) + (size_t)tr * DK));
+      else if (p.add_in_place && !(role == 0 ? p.add_dq : p.add_dk))
+        asm volatile("prefetch.global.L1 [%0];" ::"l"((const bf16*)(role == 0 ? p.dq : p.dk) + tk +
+                                                      (size_t)(c0 + tr) * DK + i0));
+    }
+  }
   // ---- intra: one 16x16 score block at a time, consumed right away -------
   const int jlo = role == 0 ? 0 : I, jhi = role == 0 ? I : NSB - 1;
 
