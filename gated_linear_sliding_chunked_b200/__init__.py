@@ -31,10 +31,10 @@ LZ_F32, LZ_BF16 = 0, 1
 
 EXPORTS = ("lz_gla_fwd", "lz_gla_bwd", "lz_swa_meta_fwd", "lz_hybrid_fwd", "lz_swa_meta_bwd",
            "lz_hybrid_bwd", "lz_gla_decode_step", "lz_workspace_bytes", "lz_last_error",
-           "lz_version", "lz_timing_enable", "lz_timing_read", "lz_swa_meta_bwd_noalloc",
-           "lz_device_check", "lz_prefer_tcgen05", "lz_decode_prefill", "lz_hybrid_fwd_mse",
-           "lz_selftest_bounded_wait", "lz_cp_segment_decay", "lz_cp_fold", "lz_cp_rows",
-           "lz_tcgen05_all", "lz_qkg_projection")
+           "lz_version", "lz_timing_enable", "lz_timing_only", "lz_timing_read",
+           "lz_swa_meta_bwd_noalloc", "lz_device_check", "lz_prefer_tcgen05", "lz_decode_prefill",
+           "lz_hybrid_fwd_mse", "lz_selftest_bounded_wait", "lz_cp_segment_decay", "lz_cp_fold",
+           "lz_cp_rows", "lz_tcgen05_all", "lz_qkg_projection")
 
 # size of the static scratch array behind lz_swa_meta_bwd_noalloc
 LZ_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -93,6 +93,7 @@ def load(path: str = LIB_PATH):
     lib.lz_cp_rows.argtypes = ([ci] * 4 + [_P, ci, ci, ctypes.c_float, _P, ci, ci, _P, ci, ci] +
                                [_P])
     lib.lz_timing_enable.argtypes = [ctypes.c_int]
+    lib.lz_timing_only.argtypes = [ctypes.c_char_p]
     lib.lz_timing_read.argtypes = [ctypes.c_char_p, sz, ctypes.POINTER(ctypes.c_float),
                                    ctypes.c_int]
     for name in EXPORTS:
@@ -181,6 +182,11 @@ def lz_tcgen05_all(on: bool) -> bool:
 
 def lz_timing_enable(on: bool):
     load().lz_timing_enable(1 if on else 0)
+
+
+def lz_timing_only(name: str | None):
+    """Time only the launches of kernel `name` (None: every launch)."""
+    load().lz_timing_only(name.encode() if name else None)
 
 
 def lz_timing_read(max_records: int = 1 << 16):

@@ -9,6 +9,19 @@ namespace lz {
 
 using bf16 = __nv_bfloat16;
 
+// CTAs of `kern` resident on the device at once (SMs x blocks per SM), or 0
+template <class Kern>
+inline int resident_ctas(Kern kern, int threads, size_t smem) {
+  int dev = 0, sms = 0, per = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kern, threads, smem) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  return sms * per;
+}
+
 // Exponent span (in nats) of the cumulative log-gate inside one 16-row
 // sub-block above which the factorized gate product q*exp(b_t-b_r) .
 // k*exp(b_r-b_s) could leave the normal fp32/bf16 range; blocks beyond it

@@ -513,6 +513,13 @@ __device__ __noinline__ float diag_score_global(const bf16* q, const bf16* k, Ga
   return a;
 }
 
+// the CTA's threads request the 128-byte lines of [base, base + bytes) into L2
+__device__ __forceinline__ void prefetch_l2_lines(const void* base, size_t bytes, int tid) {
+  const char* b = static_cast<const char*>(base);
+  for (size_t off = (size_t)tid * 128; off < bytes; off += (size_t)NT * 128)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(b + off));
+}
+
 // LOSS: the stage-1 loss epilogue (p.target set); LOGITS: the gates arrive as
 // logits (p.gz set).  Separate instantiations, so that the plain forward keeps
 // its registers and schedule.
@@ -551,6 +558,24 @@ __global__ void __launch_bounds__(NT, 2) gla_out_kernel(GlaFwdParams p) {
     cp_async16(&sm.sp[r * VP + cc * 8], sp + (size_t)r * DV + cc * 8, 16);
   }
   cp_async_commit();
+  if (p.wave > 0) {
+    // CTAs start in linear-index order, so the one `wave` places on starts
+    // about when this one ends: its inputs go to L2 now, and its loads find
+    // them there instead of waiting on HBM
+    const size_t L = (size_t)blockIdx.y * gridDim.x + blockIdx.x + (size_t)p.wave;
+    if (L < (size_t)gridDim.x * gridDim.y) {
+      const int cn = (int)(L % gridDim.x), bhn = (int)(L / gridDim.x);
+      const int rn = min(C, T - cn * C);
+      const size_t row = (size_t)bhn * T + (size_t)cn * C;
+      prefetch_l2_lines((const bf16*)p.q + row * DK, (size_t)rn * DK * 2, tid);
+      prefetch_l2_lines((const bf16*)p.k + row * DK, (size_t)rn * DK * 2, tid);
+      prefetch_l2_lines((const bf16*)p.v + row * DV, (size_t)rn * DV * 2, tid);
+      if (LOGITS) prefetch_l2_lines((const bf16*)p.gz + row * DK, (size_t)rn * DK * 2, tid);
+      else prefetch_l2_lines(p.g + row * DK, (size_t)rn * DK * 4, tid);
+      if (p.add16) prefetch_l2_lines((const bf16*)p.add16 + row * DV, (size_t)rn * DV * 2, tid);
+      prefetch_l2_lines((const bf16*)p.states16 + ((size_t)bhn * nchunks + cn) * DK * DV, (size_t)DK * DV * 2, tid);
+    }
+  }
 
   // ---- prep 1 (gates straight from global): thread -> (sub-block K, dims i2, i2+1)
   const int K = tid >> 6, i2 = (tid & 63) * 2, r0 = K * SB;
@@ -855,9 +880,11 @@ cudaError_t launch_gla_out(const GlaFwdParams& p, cudaStream_t s) {
                              : (p.gz ? gla_out_kernel<false, true> : gla_out_kernel<false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e != cudaSuccess) return e;
+  GlaFwdParams pp = p;
+  pp.wave = resident_ctas(kern, NT, bytes);
   {
     ScopedTiming tm(p.target ? "gla_out_mma_loss" : "gla_out_mma", s);
-    kern<<<dim3(nchunks, p.B * p.H), NT, bytes, s>>>(p);
+    kern<<<dim3(nchunks, p.B * p.H), NT, bytes, s>>>(pp);
   }
   return cudaGetLastError();
 }

@@ -61,6 +61,7 @@ struct GlaFwdParams {
   // is gs * log sigma(gz) with gz bf16 [B,H,T,dk]
   const void* gz;
   float gs;
+  int wave;  // CTAs resident at once (0: no prefetch of the next wave's inputs)
 };
 constexpr int kSimtChunk = 16;
 cudaError_t launch_gla_fwd_simt(const GlaFwdParams& p, bool bf16, cudaStream_t s);

@@ -121,6 +121,9 @@ __global__ void __launch_bounds__(NT, 2) swa_bwd_q_mma_kernel(SwaBwdParams p) {
     for (int x = tid; x < QTILE; x += NT)
       sm.lse2[x] = t0 + x < T ? lse[t0 + x] * kLog2e : 0.f;
     cp_async_commit();
+    if (p.osw && tid < 2 * QTILE && t0 + (tid >> 1) < T)  // the output rows D reads: into L1 meanwhile
+      asm volatile("prefetch.global.L1 [%0];" ::"l"((const bf16*)p.osw + ((size_t)bh * T + t0 + (tid >> 1)) * D +
+                                                    (tid & 1) * 64));
     cp_async_wait<0>();
     __syncthreads();
     if (p.osw) {  // D_t = dO_t . o_t, two threads per row

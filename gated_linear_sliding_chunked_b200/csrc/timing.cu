@@ -3,6 +3,7 @@
 // recorded on the launch's own stream.  Benchmarks read the elapsed times
 // back with lz_timing_read.  Off by default; costs nothing when off.
 #include <cstring>
+#include <string>
 #include <vector>
 
 #include "../../include/lizard.h"
@@ -17,6 +18,7 @@ struct Rec {
 };
 
 thread_local bool g_on = false;
+thread_local std::string g_only;  // empty: every launch; else only launches of this name
 thread_local std::vector<Rec> g_recs;
 thread_local std::vector<cudaEvent_t> g_pool;
 
@@ -33,7 +35,8 @@ cudaEvent_t take_event() {
 
 }  // namespace
 
-ScopedTiming::ScopedTiming(const char* name, cudaStream_t s) : s_(s), on_(g_on) {
+ScopedTiming::ScopedTiming(const char* name, cudaStream_t s)
+    : s_(s), on_(g_on && (g_only.empty() || g_only == name)) {
   if (!on_) return;
   name_ = name;
   a_ = take_event();
@@ -57,6 +60,11 @@ extern "C" {
 
 int lz_timing_enable(int on) {
   lz::g_on = on != 0;
+  return 0;
+}
+
+int lz_timing_only(const char* name) {
+  lz::g_only = name ? name : "";
   return 0;
 }
 

@@ -395,9 +395,14 @@ int lz_tcgen05_all(int on);
  * default).  lz_timing_read waits for the recorded launches, writes up to
  * max_records kernel names (NUL-terminated, name_stride bytes apart; names
  * may be NULL) and elapsed milliseconds (ms may be NULL), clears the record
- * and returns how many launches were recorded.  Both return 0 / a count and
- * never fail. */
+ * and returns how many launches were recorded.  lz_timing_only(name)
+ * narrows the timing to the launches of that kernel name (as lz_timing_read
+ * reports it; NULL or "" times every launch again), so that a benchmark can
+ * time one kernel inside a step without an event pair around every other
+ * launch.  All three return 0 / a count and never fail; the settings are per
+ * host thread. */
 int lz_timing_enable(int on);
+int lz_timing_only(const char* name);
 int lz_timing_read(char* names, size_t name_stride, float* ms, int max_records);
 
 /* Thread-local description of the last non-OK status ("" if none). */

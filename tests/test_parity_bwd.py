@@ -120,6 +120,27 @@ def test_hybrid_bwd(dtype, alpha, saved):
     assert_close("dalpha", res["dalpha"].cpu().double().numpy(), np.array([ref["dalpha"]]), dtype)
 
 
+def test_launch_timing_filter():
+    """lz_timing_only narrows the launch timing to one kernel name; None
+    restores timing of every launch."""
+    cpu, dev = small_problem(41, 2, 2, 200, 128, 128, 0, torch.bfloat16, train=True)
+    L.lz_timing_read()
+    runs = {}
+    for only in ("gla_bwd_chunks", None):
+        L.lz_timing_only(only)
+        L.lz_timing_enable(True)
+        try:
+            L.gla_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["dO"])
+            torch.cuda.synchronize()
+        finally:
+            L.lz_timing_enable(False)
+            L.lz_timing_only(None)
+        runs[only] = [name for name, _ in L.lz_timing_read()]
+    assert runs["gla_bwd_chunks"] == ["gla_bwd_chunks"], runs
+    assert "gla_bwd_chunks" in runs[None] and len(set(runs[None])) > 1, runs
+    L.lz_device_check()
+
+
 @pytest.mark.parametrize("T", [1, 64, 128, 129, 300, 700])
 @pytest.mark.parametrize("tc", [True, False], ids=["tcgen05", "warp-mma"])
 def test_gla_bwd_kernels(T, tc):
