@@ -643,18 +643,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
   // the gate gradient at the chunk's first row, from the reverse scan (loaded
   // here so that the load overlaps the cluster barrier)
   const float dg_first = p.gsp[((size_t)bh * nchunks + c) * DK + i0 + (tid & 63)];
-  cluster.sync();  // both CTAs: staging complete, qf / kf no longer read
-
-  // ---- dv: the peer's 64 columns go to its exchange tile -------------------
-  if (role != half) {
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int t = 16 * Iv + gr + 8 * hh, cl = nt * 8 + gc;
-        *reinterpret_cast<float2*>(&peer_xch[rsw(t, cl)]) = make_float2(dvh[nt][2 * hh], dvh[nt][2 * hh + 1]);
-      }
-  }
+  // this CTA no longer reads qf / kf (the peer's dv share lands over them):
+  // arrive now, and compute dg before waiting for the peer to do the same
+  auto done_reading = cluster.barrier_arrive();
+  __syncthreads();  // the dg products staged by every warp
   // ---- dg: the scan's value at the chunk's first row, then a running sum ---
   {
     const int col = tid & 63, qq = tid >> 6;
@@ -681,6 +673,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
       }
     }
   }
+  cluster.barrier_wait(std::move(done_reading));
+  // ---- dv: the peer's 64 columns go to its exchange tile -------------------
+  if (role != half) {
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int t = 16 * Iv + gr + 8 * hh, cl = nt * 8 + gc;
+        *reinterpret_cast<float2*>(&peer_xch[rsw(t, cl)]) = make_float2(dvh[nt][2 * hh], dvh[nt][2 * hh + 1]);
+      }
+  }
+  auto share_sent = cluster.barrier_arrive();
   if (role == half && p.add_in_place && !p.add_dv) {  // loads ahead of the stores below
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
@@ -695,7 +699,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 2)
         dvh[nt][2 * hh + 1] += f.y;
       }
   }
-  cluster.sync();  // the peer's share has landed
+  cluster.barrier_wait(std::move(share_sent));  // the peer's share has landed
   if (role == half) {
     const int mcol = 64 * half;
 #pragma unroll
