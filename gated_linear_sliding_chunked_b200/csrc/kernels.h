@@ -215,9 +215,18 @@ struct SwaBwdParams {
   bool tc;               // key side on the tcgen05 kernel (bf16, d = 128)
   bool tc_q;             // query side on the tcgen05 kernel where it applies
   unsigned int* status;  // device status word (set by the tcgen05 launcher)
+  // Split query side (used when both are set, the key side runs on tcgen05,
+  // the forward output is given and dq is bf16): the key side also stores its
+  // bf16 dS^T tiles, the query-side pass keeps only D, the meta tokens' dS and
+  // the meta gradients, and swa_bwd_dq forms dq = scale * gscale * dS [K; MK].
+  void* ds_tiles;        // [B*H][ceil(T/128)][ds_nq][128 keys][64 queries] bf16
+  void* ds_meta;         // [B*H][T][16] bf16: the meta tokens' dS / gscale
+  int ds_nq;             // query tiles per 128-key block (swa_bwd_ds_nq(w))
 };
 // query rows per CTA of the meta-gradient pass (one partial per slab)
 constexpr int kSwaBwdSlab = 256;
+// 64-query tiles that see one 128-key block of a window of w keys
+inline int swa_bwd_ds_nq(int w) { return (127 + w - 1 + 64) / 64; }
 int swa_bwd_n_qblocks(int B, int H, int T);
 int swa_bwd_n_meta_parts(int B, int T);
 cudaError_t launch_swa_bwd_simt(const SwaBwdParams& p, bool bf16, cudaStream_t s);

@@ -282,11 +282,18 @@ struct HybridBwdWs {
   float* dq;  // fp32 window-branch gradients (SIMT path only)
   float* dk;
   float* dv;
+  void* ds_tiles;  // tensor-core path: the key side's bf16 dS^T tiles ...
+  void* ds_meta;   // ... and the meta tokens' dS, for the split query side
 };
 HybridBwdWs carve_hybrid_bwd(Carver& c, const lz_dims* d) {
   HybridBwdWs w{};
   w.swa = carve_swa_bwd(c, d);
   w.gla = carve_gla_bwd(c, d);
+  if (hybrid_uses_mma(d) && d->w <= 129) {  // windows of up to 129 keys: at most 4 tiles per block
+    const size_t nblk = (size_t)((d->T + 127) / 128);
+    w.ds_tiles = c.take<uint16_t>((size_t)d->B * d->H * nblk * lz::swa_bwd_ds_nq(d->w) * 128 * 64);
+    w.ds_meta = c.take<uint16_t>(bht(d) * 16);
+  }
   if (!hybrid_uses_mma(d)) {
     w.dq = c.take<float>(bht(d) * d->dk);
     w.dk = c.take<float>(bht(d) * d->dk);
@@ -736,6 +743,7 @@ lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const vo
   p.dq = dq; p.dk = dk; p.dv = dv;
   p.dq_f32 = w.dq; p.dk_f32 = w.dk; p.dv_f32 = w.dv;
   p.dmk = dmeta_k; p.dmv = dmeta_v; p.dalpha = dalpha;
+  p.ds_tiles = w.ds_tiles; p.ds_meta = w.ds_meta;
   if (!mma || bht(d) == 0) {
     cudaError_t e = swa_backward(p, d->io == LZ_BF16, s);
     if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (window branch)");

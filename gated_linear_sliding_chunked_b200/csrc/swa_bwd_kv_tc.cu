@@ -16,7 +16,9 @@
 //             tile's scores, form P^T and dS^T (bf16) in shared memory;
 //   thread 0: dV += P^T dO, dK += dS^T Q (M = 128, N = 128, K = 64), commit.
 // Q / dO tiles rotate through three shared-memory buffers, loaded by TMA
-// two tiles ahead.
+// two tiles ahead.  With p.ds_tiles set the threads also store their bf16
+// dS^T rows of every tile to global memory, from which swa_bwd_dq forms dq
+// (so that the query side does not form the band's scores a second time).
 // K, V (K-major) and the Q / dO tiles sit in shared memory 128-byte
 // swizzled as TMA writes them; the gradient MMAs read Q / dO as MN-major B
 // operands (rows = queries, the reduction dim) from the same tiles.
@@ -183,6 +185,13 @@ __global__ void __launch_bounds__(NTH, 1)
       }
       pk[c / 2] = pack_bf16(pr[0], pr[1]);
       dk2[c / 2] = pack_bf16(ds[0], ds[1]);
+    }
+    if (p.ds_tiles) {  // dS^T of this tile for the split query side: [bh][block][tile][key][query]
+      uint4* dst = reinterpret_cast<uint4*>((bf16*)p.ds_tiles +
+                                            ((((size_t)bh * gridDim.x + blockIdx.x) * p.ds_nq + i) * KR + kr) * QT +
+                                            hf * 32);
+#pragma unroll
+      for (int x = 0; x < 4; ++x) dst[x] = make_uint4(dk2[4 * x], dk2[4 * x + 1], dk2[4 * x + 2], dk2[4 * x + 3]);
     }
 #pragma unroll
     for (int x = 0; x < 4; ++x) {  // K-major [128 keys][64 queries], 8-row groups 1024 bytes apart

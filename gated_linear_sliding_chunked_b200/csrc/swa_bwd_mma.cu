@@ -75,6 +75,10 @@ __device__ __forceinline__ void qk_scores(const uint32_t (*qa)[4], const bf16* k
     }
 }
 
+// WINDOW = false: the split query side (the forward output is given): no key
+// sweep and no dq; the meta tokens' dS goes to p.ds_meta for swa_bwd_dq, and
+// D and the meta gradients are formed as in the full pass.
+template <bool WINDOW>
 __global__ void __launch_bounds__(NT, 2) swa_bwd_q_mma_kernel(SwaBwdParams p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   QSmem& sm = *reinterpret_cast<QSmem*>(smem_raw);
@@ -214,17 +218,29 @@ __global__ void __launch_bounds__(NT, 2) swa_bwd_q_mma_kernel(SwaBwdParams p) {
           for (int nt = 0; nt < MT / 8; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) ds[nt][e] = p.gscale * s[nt][e] * (dp[nt][e] - Drow[e >> 1]);
-          // dq += dS_meta mk
-          const uint32_t pa[4] = {pack_bf16(ds[0][0], ds[0][1]), pack_bf16(ds[0][2], ds[0][3]),
-                                  pack_bf16(ds[1][0], ds[1][1]), pack_bf16(ds[1][2], ds[1][3])};
+          if constexpr (WINDOW) {  // dq += dS_meta mk
+            const uint32_t pa[4] = {pack_bf16(ds[0][0], ds[0][1]), pack_bf16(ds[0][2], ds[0][3]),
+                                    pack_bf16(ds[1][0], ds[1][1]), pack_bf16(ds[1][2], ds[1][3])};
 #pragma unroll
-          for (int ntp = 0; ntp < D / 16; ++ntp) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(smem_u32(&sm.mk[((lane & 7) + ((lane >> 3) & 1) * 8) * RPAD + ntp * 16 +
-                                      (lane >> 4) * 8]),
-                      b0, b1, b2, b3);
-            mma_bf16(dq[2 * ntp], pa, b0, b1);
-            mma_bf16(dq[2 * ntp + 1], pa, b2, b3);
+            for (int ntp = 0; ntp < D / 16; ++ntp) {
+              uint32_t b0, b1, b2, b3;
+              ldsm_x4_t(smem_u32(&sm.mk[((lane & 7) + ((lane >> 3) & 1) * 8) * RPAD + ntp * 16 +
+                                        (lane >> 4) * 8]),
+                        b0, b1, b2, b3);
+              mma_bf16(dq[2 * ntp], pa, b0, b1);
+              mma_bf16(dq[2 * ntp + 1], pa, b2, b3);
+            }
+          } else {  // the meta tokens' dS without the gscale factor, for swa_bwd_dq
+#pragma unroll
+            for (int nt = 0; nt < MT / 8; ++nt)
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                const int t = row0 + 8 * hh, j = nt * 8 + gc;
+                if (t < T)
+                  *reinterpret_cast<uint32_t*>(&((bf16*)p.ds_meta)[((size_t)bh * T + t) * MT + j]) =
+                      pack_bf16(s[nt][2 * hh] * (dp[nt][2 * hh] - Drow[hh]),
+                                s[nt][2 * hh + 1] * (dp[nt][2 * hh + 1] - Drow[hh]));
+              }
           }
           // stage dS_meta and P_meta for the meta-gradient products
 #pragma unroll
@@ -237,46 +253,48 @@ __global__ void __launch_bounds__(NT, 2) swa_bwd_q_mma_kernel(SwaBwdParams p) {
             }
         }
       }
-      // window tiles, double-buffered
-      load_rows(sm.k[0], k, lo, hi - lo + 1, KT1);
-      load_rows(sm.v[0], v, lo, hi - lo + 1, KT1);
-      cp_async_commit();
-      for (int it = 0; it < ntiles; ++it) {
-        const int stg = it & 1, kb = lo + it * KT1;
-        cp_async_wait<0>();
-        __syncthreads();
-        if (it + 1 < ntiles) {
-          const int nb = kb + KT1;
-          load_rows(sm.k[stg ^ 1], k, nb, hi - nb + 1, KT1);
-          load_rows(sm.v[stg ^ 1], v, nb, hi - nb + 1, KT1);
-          cp_async_commit();
-        }
-        float s[KT1 / 8][4], dp[KT1 / 8][4];
-        tile_pdp(sm.k[stg], sm.v[stg], IntTag<KT1>{}, window_valid(kb), s, dp);
-        if (sweep == 0) {
-#pragma unroll
-          for (int nt = 0; nt < KT1 / 8; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) Drow[e >> 1] += s[nt][e] * dp[nt][e];
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < KT1 / 16; ++kk) {
-            float d0[4], d1[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              d0[e] = p.gscale * s[2 * kk][e] * (dp[2 * kk][e] - Drow[e >> 1]);
-              d1[e] = p.gscale * s[2 * kk + 1][e] * (dp[2 * kk + 1][e] - Drow[e >> 1]);
-            }
-            const uint32_t pa[4] = {pack_bf16(d0[0], d0[1]), pack_bf16(d0[2], d0[3]),
-                                    pack_bf16(d1[0], d1[1]), pack_bf16(d1[2], d1[3])};
-#pragma unroll
-            for (int ntp = 0; ntp < D / 16; ++ntp) {
-              uint32_t b0, b1, b2, b3;
-              ldsm_x4_t(smem_u32(&sm.k[stg][(kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * RPAD +
-                                            ntp * 16 + (lane >> 4) * 8]),
-                        b0, b1, b2, b3);
-              mma_bf16(dq[2 * ntp], pa, b0, b1);
-              mma_bf16(dq[2 * ntp + 1], pa, b2, b3);
+      if constexpr (WINDOW) {
+        // window tiles, double-buffered
+        load_rows(sm.k[0], k, lo, hi - lo + 1, KT1);
+        load_rows(sm.v[0], v, lo, hi - lo + 1, KT1);
+        cp_async_commit();
+        for (int it = 0; it < ntiles; ++it) {
+          const int stg = it & 1, kb = lo + it * KT1;
+          cp_async_wait<0>();
+          __syncthreads();
+          if (it + 1 < ntiles) {
+            const int nb = kb + KT1;
+            load_rows(sm.k[stg ^ 1], k, nb, hi - nb + 1, KT1);
+            load_rows(sm.v[stg ^ 1], v, nb, hi - nb + 1, KT1);
+            cp_async_commit();
+          }
+          float s[KT1 / 8][4], dp[KT1 / 8][4];
+          tile_pdp(sm.k[stg], sm.v[stg], IntTag<KT1>{}, window_valid(kb), s, dp);
+          if (sweep == 0) {
+  #pragma unroll
+            for (int nt = 0; nt < KT1 / 8; ++nt)
+  #pragma unroll
+              for (int e = 0; e < 4; ++e) Drow[e >> 1] += s[nt][e] * dp[nt][e];
+          } else {
+  #pragma unroll
+            for (int kk = 0; kk < KT1 / 16; ++kk) {
+              float d0[4], d1[4];
+  #pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                d0[e] = p.gscale * s[2 * kk][e] * (dp[2 * kk][e] - Drow[e >> 1]);
+                d1[e] = p.gscale * s[2 * kk + 1][e] * (dp[2 * kk + 1][e] - Drow[e >> 1]);
+              }
+              const uint32_t pa[4] = {pack_bf16(d0[0], d0[1]), pack_bf16(d0[2], d0[3]),
+                                      pack_bf16(d1[0], d1[1]), pack_bf16(d1[2], d1[3])};
+  #pragma unroll
+              for (int ntp = 0; ntp < D / 16; ++ntp) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(smem_u32(&sm.k[stg][(kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * RPAD +
+                                              ntp * 16 + (lane >> 4) * 8]),
+                          b0, b1, b2, b3);
+                mma_bf16(dq[2 * ntp], pa, b0, b1);
+                mma_bf16(dq[2 * ntp + 1], pa, b2, b3);
+              }
             }
           }
         }
@@ -296,12 +314,14 @@ __global__ void __launch_bounds__(NT, 2) swa_bwd_q_mma_kernel(SwaBwdParams p) {
       const int t = row0 + 8 * hh;
       if (t >= T) continue;
       const size_t off = ((size_t)bh * T + t) * D;
+      if constexpr (WINDOW) {
 #pragma unroll
-      for (int nt = 0; nt < D / 8; ++nt) {
-        const int j = nt * 8 + gc;
-        const float x0 = dq[nt][2 * hh] * p.scale, x1 = dq[nt][2 * hh + 1] * p.scale;
-        if (p.dq_f32) *reinterpret_cast<float2*>(&p.dq_f32[off + j]) = make_float2(x0, x1);
-        else *reinterpret_cast<uint32_t*>(&((bf16*)p.dq)[off + j]) = pack_bf16(x0, x1);
+        for (int nt = 0; nt < D / 8; ++nt) {
+          const int j = nt * 8 + gc;
+          const float x0 = dq[nt][2 * hh] * p.scale, x1 = dq[nt][2 * hh + 1] * p.scale;
+          if (p.dq_f32) *reinterpret_cast<float2*>(&p.dq_f32[off + j]) = make_float2(x0, x1);
+          else *reinterpret_cast<uint32_t*>(&((bf16*)p.dq)[off + j]) = pack_bf16(x0, x1);
+        }
       }
       if ((lane & 3) == 0) {
         p.Dbuf[(size_t)bh * T + t] = Drow[hh];
@@ -520,6 +540,121 @@ __global__ void __launch_bounds__(NT, 2) swa_bwd_kv_mma_kernel(SwaBwdParams p) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Kernel 3 (split query side): dq from the key side's dS tiles
+// ---------------------------------------------------------------------------
+// The tcgen05 key side forms, for every 128-key block b and every 64-query
+// tile i that sees it, dS^T = P^T (dP^T - D) without the gscale factor and
+// stores it in bf16: ds_tiles[bh][b][i][key][query].  A query tile q0 takes
+// those of the blocks its window reaches and the meta tokens' dS:
+//   dq = scale * gscale * (sum_b dS_b K_b + dS_meta MK)
+// (Lizard technical summary, section 2a: the window keys and the always-visible
+// meta tokens share one softmax, so they share its Jacobian).
+constexpr int QT3 = 64;        // query rows per CTA (4 warps x 16)
+constexpr int KB3 = 128;       // keys per block of the key side
+constexpr int DSP = QT3 + 8;   // padded row of the [key][query] dS tile
+
+struct DqSmem {
+  bf16 ds[KB3 * DSP];
+  bf16 k[KB3 * RPAD];
+  bf16 mk[MT * RPAD];
+  bf16 dsm[QT3 * 24];          // the meta tokens' dS, [query][16] (+8 pad)
+};
+static_assert(sizeof(DqSmem) <= 232448 / 3, "three dq CTAs must fit one SM");
+
+__global__ void __launch_bounds__(NT, 3) swa_bwd_dq_kernel(SwaBwdParams p) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  DqSmem& sm = *reinterpret_cast<DqSmem*>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gr = lane >> 2, gc = (lane & 3) * 2;
+  const int q0 = blockIdx.x * QT3, bh = blockIdx.y, h = bh % p.H;
+  const int T = p.T, w = p.w, M = p.M;
+  const int nblk = (T + KB3 - 1) / KB3;
+  float dq[D / 8][4];
+#pragma unroll
+  for (int nt = 0; nt < D / 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dq[nt][e] = 0.f;
+
+  if (M > 0) {  // dq += dS_meta MK
+    const bf16* dsm = (const bf16*)p.ds_meta + ((size_t)bh * T + q0) * MT;
+    for (int x = tid; x < QT3 * MT / 8; x += NT) {
+      const int r = x / (MT / 8), cc = x % (MT / 8);
+      const bool ok = q0 + r < T;
+      cp_async16(&sm.dsm[r * 24 + cc * 8], dsm + (size_t)(ok ? r : 0) * MT + cc * 8, ok ? 16 : 0);
+    }
+    const bf16* mk = (const bf16*)p.mk + (size_t)h * M * D;
+    for (int x = tid; x < MT * D / 8; x += NT) {
+      const int r = x / (D / 8), cc = x % (D / 8);
+      const bool ok = r < M;
+      cp_async16(&sm.mk[r * RPAD + cc * 8], mk + (size_t)(ok ? r : 0) * D + cc * 8, ok ? 16 : 0);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    uint32_t a[4];
+    ldsm_x4(smem_u32(&sm.dsm[(16 * warp + (lane & 15)) * 24 + (lane >> 4) * 8]), a[0], a[1], a[2], a[3]);
+#pragma unroll
+    for (int ntp = 0; ntp < D / 16; ++ntp) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(smem_u32(&sm.mk[((lane & 7) + ((lane >> 3) & 1) * 8) * RPAD + ntp * 16 + (lane >> 4) * 8]),
+                b0, b1, b2, b3);
+      mma_bf16(dq[2 * ntp], a, b0, b1);
+      mma_bf16(dq[2 * ntp + 1], a, b2, b3);
+    }
+  }
+  // the key blocks whose window reaches the tile: keys >= q0 - w + 1, <= q0 + 63
+  const int b_lo = max(0, q0 - w + 1) / KB3, b_hi = min(q0 / KB3, nblk - 1);
+  for (int b = b_lo; b <= b_hi; ++b) {
+    const int j0 = b * KB3, i = (q0 - j0) / QT3;
+    const int nq = (min(T - 1, j0 + KB3 - 1 + w - 1) - j0 + QT3) / QT3;  // tiles the key side formed
+    if (i >= nq) continue;
+    __syncthreads();  // the previous block's readers are done
+    const bf16* ds = (const bf16*)p.ds_tiles + (((size_t)bh * nblk + b) * p.ds_nq + i) * KB3 * QT3;
+    for (int x = tid; x < KB3 * QT3 / 8; x += NT) {
+      const int r = x / (QT3 / 8), cc = x % (QT3 / 8);
+      cp_async16(&sm.ds[r * DSP + cc * 8], ds + (size_t)r * QT3 + cc * 8, 16);
+    }
+    const bf16* k = (const bf16*)p.k + ((size_t)bh * T + j0) * D;
+    const int rows = min(KB3, T - j0);
+    for (int x = tid; x < KB3 * D / 8; x += NT) {
+      const int r = x / (D / 8), cc = x % (D / 8);
+      const bool ok = r < rows;
+      cp_async16(&sm.k[r * RPAD + cc * 8], k + (size_t)(ok ? r : 0) * D + cc * 8, ok ? 16 : 0);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+#pragma unroll 2
+    for (int kk = 0; kk < KB3 / 16; ++kk) {
+      uint32_t a[4];  // A = dS (queries x keys) from the [key][query] tile, transposed
+      ldsm_x4_t(smem_u32(&sm.ds[(kk * 16 + (lane & 7) + ((lane >> 4) << 3)) * DSP + 16 * warp +
+                                ((lane >> 3) & 1) * 8]),
+                a[0], a[1], a[2], a[3]);
+#pragma unroll
+      for (int ntp = 0; ntp < D / 16; ++ntp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(smem_u32(&sm.k[(kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * RPAD + ntp * 16 +
+                                 (lane >> 4) * 8]),
+                  b0, b1, b2, b3);
+        mma_bf16(dq[2 * ntp], a, b0, b1);
+        mma_bf16(dq[2 * ntp + 1], a, b2, b3);
+      }
+    }
+  }
+  const float sc = p.scale * p.gscale;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int t = q0 + 16 * warp + gr + 8 * hh;
+    if (t >= T) continue;
+    const size_t off = ((size_t)bh * T + t) * D;
+#pragma unroll
+    for (int nt = 0; nt < D / 8; ++nt)
+      *reinterpret_cast<uint32_t*>(&((bf16*)p.dq)[off + nt * 8 + gc]) =
+          pack_bf16(dq[nt][2 * hh] * sc, dq[nt][2 * hh + 1] * sc);
+  }
+}
+
 }  // namespace
 
 bool swa_bwd_mma_supported(int dk, int dv, bool bf16) { return bf16 && dk == D && dv == D; }
@@ -528,33 +663,52 @@ cudaError_t launch_swa_bwd_mma(const SwaBwdParams& p, cudaStream_t s) {
   const bool empty = p.T == 0 || p.B * p.H == 0;
   const int nslab = (p.T + SLAB - 1) / SLAB;
   cudaError_t e = cudaSuccess;
+  const bool kv_tc = p.tc && swa_bwd_kv_tc_supported(p.dkd, p.dvd, true);
+  const bool q_tc = p.tc_q && swa_bwd_q_tc_supported(p);
+  // split query side: D and the meta terms here, dq from the key side's dS tiles
+  const bool split = p.ds_tiles && p.ds_meta && p.osw && p.dq && !p.dq_f32 && kv_tc && !q_tc;
+  SwaBwdParams pp = p;
+  if (split) pp.ds_nq = swa_bwd_ds_nq(p.w);
+  else pp.ds_tiles = nullptr;
   if (!empty) {
-    if (p.tc_q && swa_bwd_q_tc_supported(p)) {
-      e = launch_swa_bwd_q_tc(p, s);
+    if (q_tc) {
+      e = launch_swa_bwd_q_tc(pp, s);
     } else {
+      const auto kern = split ? swa_bwd_q_mma_kernel<false> : swa_bwd_q_mma_kernel<true>;
       const size_t b1 = sizeof(QSmem);
-      e = cudaFuncSetAttribute(swa_bwd_q_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)b1);
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)b1);
       if (e != cudaSuccess) return e;
       {
-        ScopedTiming tm("swa_bwd_q_mma", s);
-        swa_bwd_q_mma_kernel<<<dim3(p.H, p.B, nslab), NT, b1, s>>>(p);
+        ScopedTiming tm(split ? "swa_bwd_meta" : "swa_bwd_q_mma", s);
+        kern<<<dim3(p.H, p.B, nslab), NT, b1, s>>>(pp);
       }
       e = cudaGetLastError();
     }
     if (e != cudaSuccess) return e;
-    if (p.tc && swa_bwd_kv_tc_supported(p.dkd, p.dvd, true)) {
-      e = launch_swa_bwd_kv_tc(p, s);
+    if (kv_tc) {
+      e = launch_swa_bwd_kv_tc(pp, s);
     } else {
       const size_t b2 = sizeof(KVSmem);
       e = cudaFuncSetAttribute(swa_bwd_kv_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)b2);
       if (e != cudaSuccess) return e;
       {
         ScopedTiming tm("swa_bwd_kv_mma", s);
-        swa_bwd_kv_mma_kernel<<<dim3((p.T + KT2 - 1) / KT2, p.B * p.H), NT, b2, s>>>(p);
+        swa_bwd_kv_mma_kernel<<<dim3((p.T + KT2 - 1) / KT2, p.B * p.H), NT, b2, s>>>(pp);
       }
       e = cudaGetLastError();
     }
     if (e != cudaSuccess) return e;
+    if (split) {
+      const size_t b3 = sizeof(DqSmem);
+      e = cudaFuncSetAttribute(swa_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)b3);
+      if (e != cudaSuccess) return e;
+      {
+        ScopedTiming tm("swa_bwd_dq", s);
+        swa_bwd_dq_kernel<<<dim3((p.T + QT3 - 1) / QT3, p.B * p.H), NT, b3, s>>>(pp);
+      }
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
   }
   const int nparts = (p.M > 0 && !empty) ? p.B * nslab : 0;
   const int nalpha = empty ? 0 : p.B * p.H * nslab;

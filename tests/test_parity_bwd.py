@@ -228,6 +228,50 @@ def test_gla_bwd_long_context_gates_full_length():
         assert_close(f"{name}[T=65536]", res[name], ref[name], torch.bfloat16)
 
 
+@pytest.mark.parametrize("T,w,M,sink", [(1, 1, 2, False), (64, 64, 0, False), (127, 129, 8, False),
+                                         (129, 33, 3, True), (300, 128, 16, False),
+                                         (700, 100, 4, True)])
+def test_hybrid_bwd_split_query_side(T, w, M, sink):
+    """bf16 hybrid backward given the window output: the query side keeps D
+    and the meta terms, the tcgen05 key side stores its dS tiles and dq is
+    formed from them (swa_bwd_dq), for ragged lengths, windows up to 129
+    keys, sink-only meta tokens and none; run twice, bit-identical."""
+    alpha = 0.7
+    cpu, dev = small_problem(500 + T + w, 2, 2, T, 128, 128, M, torch.bfloat16, train=True)
+    mk = dev["meta_k"] if M else None
+    mv = dev["meta_v"] if (M and not sink) else None
+    fwd = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], mk, mv, w=w, alpha=alpha,
+                       want_lse=True, want_o_swa=True)
+    L.lz_timing_read()
+    L.lz_timing_enable(True)
+    try:
+        runs = [L.hybrid_bwd(dev["q"], dev["k"], dev["v"], dev["g"], mk, mv, fwd["lse"],
+                             dev["dO"], w=w, alpha=alpha, o_swa=fwd["o_swa"]) for _ in range(2)]
+        torch.cuda.synchronize()
+    finally:
+        L.lz_timing_enable(False)
+    ran = {name for name, _ in L.lz_timing_read()}
+    assert {"swa_bwd_meta", "swa_bwd_kv_tc", "swa_bwd_dq"} <= ran, ran
+    assert "swa_bwd_q_mma" not in ran, ran
+    L.lz_device_check()
+    x = oracle_inputs(cpu, ("q", "k", "v", "g", "meta_k", "meta_v", "dO"))
+    ref = oracle.hybrid_bwd(x["q"], x["k"], x["v"], x["g"], x["meta_k"] if M else None,
+                            x["meta_v"] if (M and not sink) else None, x["dO"], w,
+                            1 / math.sqrt(128), alpha)
+    res = runs[0]
+    for name in ("dq", "dk", "dv", "dg"):
+        assert_close(name, res[name], ref[name], torch.bfloat16)
+    if M > 0:
+        assert_close("dmeta_k", res["dmeta_k"], ref["dmeta_k"], torch.bfloat16)
+        if not sink:
+            assert_close("dmeta_v", res["dmeta_v"], ref["dmeta_v"], torch.bfloat16)
+    assert_close("dalpha", res["dalpha"].cpu().double().numpy(), np.array([ref["dalpha"]]),
+                 torch.bfloat16)
+    for name in ("dq", "dk", "dv", "dg", "dmeta_k", "dmeta_v", "dalpha"):
+        if runs[0].get(name) is not None:
+            assert torch.equal(runs[0][name], runs[1][name]), name
+
+
 def test_bwd_determinism():
     cpu, dev = small_problem(8, 2, 2, 300, 128, 128, 4, torch.bfloat16, train=True)
     fwd = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
