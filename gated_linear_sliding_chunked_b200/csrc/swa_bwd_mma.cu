@@ -42,17 +42,42 @@ struct IntTag {
 struct QSmem {
   bf16 q[QTILE * RPAD];
   bf16 dO[QTILE * RPAD];
-  bf16 k[2][KT1 * RPAD];
-  bf16 v[2][KT1 * RPAD];
   bf16 mk[MT * RPAD];
   bf16 mv[MT * RPAD];
   bf16 dsm[QTILE * 24];   // meta dS (bf16), rows x 16 (+8 pad)
   bf16 pm[QTILE * 24];    // meta P (bf16)
   float lse2[QTILE];
   float drow[QTILE];      // D_t from the saved forward output
+  // last, so that the split pass (no key sweep) launches without them
+  bf16 k[2][KT1 * RPAD];
+  bf16 v[2][KT1 * RPAD];
 };
 
 static_assert(sizeof(QSmem) <= 232448, "shared memory per block exceeds 227 KB");
+
+// the same with the A fragments read from shared memory as they are used
+// (arow: this lane's ldmatrix row of the warp's 16 query rows)
+template <int NK>
+__device__ __forceinline__ void qk_scores_sm(const bf16* arow, const bf16* ks, int lane, float (*s)[4]) {
+#pragma unroll
+  for (int nt = 0; nt < NK / 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    uint32_t a[4];
+    ldsm_x4(smem_u32(arow + kk * 16), a[0], a[1], a[2], a[3]);
+#pragma unroll
+    for (int ntp = 0; ntp < NK / 16; ++ntp) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(smem_u32(&ks[(ntp * 16 + (lane & 7) + ((lane >> 4) << 3)) * RPAD + kk * 16 +
+                           ((lane >> 3) & 1) * 8]),
+              b0, b1, b2, b3);
+      mma_bf16(s[2 * ntp], a, b0, b1);
+      mma_bf16(s[2 * ntp + 1], a, b2, b3);
+    }
+  }
+}
 
 // scores of 16 query rows (A fragments qa) against NK keys stored row-major
 template <int NK>
@@ -79,7 +104,7 @@ __device__ __forceinline__ void qk_scores(const uint32_t (*qa)[4], const bf16* k
 // sweep and no dq; the meta tokens' dS goes to p.ds_meta for swa_bwd_dq, and
 // D and the meta gradients are formed as in the full pass.
 template <bool WINDOW>
-__global__ void __launch_bounds__(NT, 2) swa_bwd_q_mma_kernel(SwaBwdParams p) {
+__global__ void __launch_bounds__(NT, WINDOW ? 2 : 4) swa_bwd_q_mma_kernel(SwaBwdParams p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   QSmem& sm = *reinterpret_cast<QSmem*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -153,13 +178,17 @@ __global__ void __launch_bounds__(NT, 2) swa_bwd_q_mma_kernel(SwaBwdParams p) {
       __syncthreads();
     }
     const int row0 = t0 + 16 * warp + gr;
-    uint32_t qa[D / 16][4], da[D / 16][4];
+    // the key sweep keeps the warp's q / dO fragments in registers; the split
+    // pass (one 16-key meta tile) reads them from shared memory instead
+    uint32_t qa[WINDOW ? D / 16 : 1][4], da[WINDOW ? D / 16 : 1][4];
+    const bf16* qrow = &sm.q[(16 * warp + (lane & 15)) * RPAD + (lane >> 4) * 8];
+    const bf16* drow_a = &sm.dO[(16 * warp + (lane & 15)) * RPAD + (lane >> 4) * 8];
+    if constexpr (WINDOW) {
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      ldsm_x4(smem_u32(&sm.q[(16 * warp + (lane & 15)) * RPAD + kk * 16 + (lane >> 4) * 8]),
-              qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
-      ldsm_x4(smem_u32(&sm.dO[(16 * warp + (lane & 15)) * RPAD + kk * 16 + (lane >> 4) * 8]),
-              da[kk][0], da[kk][1], da[kk][2], da[kk][3]);
+      for (int kk = 0; kk < D / 16; ++kk) {
+        ldsm_x4(smem_u32(qrow + kk * 16), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
+        ldsm_x4(smem_u32(drow_a + kk * 16), da[kk][0], da[kk][1], da[kk][2], da[kk][3]);
+      }
     }
     const float l2[2] = {sm.lse2[16 * warp + gr], sm.lse2[16 * warp + gr + 8]};
     float Drow[2] = {0.f, 0.f};
@@ -177,9 +206,11 @@ __global__ void __launch_bounds__(NT, 2) swa_bwd_q_mma_kernel(SwaBwdParams p) {
     auto tile_pdp = [&](const bf16* ks, const bf16* vs, auto nk_tag, auto valid, float (*s)[4],
                         float (*dp)[4]) {
       constexpr int NK = decltype(nk_tag)::value;
-      qk_scores<NK>(qa, ks, lane, s);
+      if constexpr (WINDOW) qk_scores<NK>(qa, ks, lane, s);
+      else qk_scores_sm<NK>(qrow, ks, lane, s);
       if (vs) {
-        qk_scores<NK>(da, vs, lane, dp);
+        if constexpr (WINDOW) qk_scores<NK>(da, vs, lane, dp);
+        else qk_scores_sm<NK>(drow_a, vs, lane, dp);
       } else {
 #pragma unroll
         for (int nt = 0; nt < NK / 8; ++nt)
@@ -550,86 +581,113 @@ __global__ void __launch_bounds__(NT, 2) swa_bwd_kv_mma_kernel(SwaBwdParams p) {
 //   dq = scale * gscale * (sum_b dS_b K_b + dS_meta MK)
 // (Lizard technical summary, section 2a: the window keys and the always-visible
 // meta tokens share one softmax, so they share its Jacobian).
-constexpr int QT3 = 64;        // query rows per CTA (4 warps x 16)
+constexpr int QT3 = 64;        // query rows per dS tile
+constexpr int QR3 = 128;       // query rows per CTA (8 warps x 16): two tiles, one key block
+constexpr int NT3 = 256;
 constexpr int KB3 = 128;       // keys per block of the key side
-constexpr int DSP = QT3 + 8;   // padded row of the [key][query] dS tile
+constexpr int DSP = QT3 + 8;   // padded row of a [key][query] dS tile
 
 struct DqSmem {
-  bf16 ds[KB3 * DSP];
+  bf16 ds[2][KB3 * DSP];       // the block's dS tiles of the CTA's two query tiles
   bf16 k[KB3 * RPAD];
   bf16 mk[MT * RPAD];
-  bf16 dsm[QT3 * 24];          // the meta tokens' dS, [query][16] (+8 pad)
+  bf16 dsm[QR3 * 24];          // the meta tokens' dS, [query][16] (+8 pad)
 };
-static_assert(sizeof(DqSmem) <= 232448 / 3, "three dq CTAs must fit one SM");
+static_assert(sizeof(DqSmem) <= 232448 / 2, "two dq CTAs must fit one SM");
 
-__global__ void __launch_bounds__(NT, 3) swa_bwd_dq_kernel(SwaBwdParams p) {
+// one CTA = 128 query rows q0 .. q0 + 127 (q0 a multiple of 128, so its two
+// 64-row tiles see the same key blocks); warp wq takes rows 16 wq .. 16 wq + 15
+__global__ void __launch_bounds__(NT3, 2) swa_bwd_dq_kernel(SwaBwdParams p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   DqSmem& sm = *reinterpret_cast<DqSmem*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gr = lane >> 2, gc = (lane & 3) * 2;
-  const int q0 = blockIdx.x * QT3, bh = blockIdx.y, h = bh % p.H;
+  const int q0 = blockIdx.x * QR3, bh = blockIdx.y, h = bh % p.H;
   const int T = p.T, w = p.w, M = p.M;
   const int nblk = (T + KB3 - 1) / KB3;
+  const int half = warp >> 2, rw = 16 * (warp & 3);  // the warp's tile and its rows in it
+  // the key blocks whose window reaches the CTA's rows: keys >= q0 - w + 1, <= q0 + 127
+  const int b_lo = max(0, q0 - w + 1) / KB3, b_hi = min(q0 / KB3, nblk - 1);
+  // tiles the key side formed for block b (the same count as its own loop)
+  auto tiles_of = [&](int b) { return (min(T - 1, b * KB3 + KB3 - 1 + w - 1) - b * KB3 + QT3) / QT3; };
+  auto load_block = [&](int b) {
+    const int j0 = b * KB3, nq = tiles_of(b);
+    for (int hf = 0; hf < 2; ++hf) {
+      const int i = (q0 - j0) / QT3 + hf;
+      if (i >= nq) continue;  // no query of this tile sees the block: its rows read as zeros below
+      const bf16* ds = (const bf16*)p.ds_tiles + (((size_t)bh * nblk + b) * p.ds_nq + i) * KB3 * QT3;
+      for (int x = tid; x < KB3 * QT3 / 8; x += NT3) {
+        const int r = x / (QT3 / 8), cc = x % (QT3 / 8);
+        cp_async16(&sm.ds[hf][r * DSP + cc * 8], ds + (size_t)r * QT3 + cc * 8, 16);
+      }
+    }
+    const bf16* k = (const bf16*)p.k + ((size_t)bh * T + j0) * D;
+    const int rows = min(KB3, T - j0);
+    for (int x = tid; x < KB3 * D / 8; x += NT3) {
+      const int r = x / (D / 8), cc = x % (D / 8);
+      const bool ok = r < rows;
+      cp_async16(&sm.k[r * RPAD + cc * 8], k + (size_t)(ok ? r : 0) * D + cc * 8, ok ? 16 : 0);
+    }
+  };
+  if (b_lo < b_hi) {  // the last block's tiles and keys into L2 while the first is used
+    const int b = b_hi, j0 = b * KB3, nq = tiles_of(b);
+    for (int hf = 0; hf < 2; ++hf) {
+      const int i = (q0 - j0) / QT3 + hf;
+      if (i >= nq) continue;
+      const char* t = (const char*)p.ds_tiles + (((size_t)bh * nblk + b) * p.ds_nq + i) * KB3 * QT3 * 2;
+      for (int x = tid; x < KB3 * QT3 * 2 / 128; x += NT3)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(t + x * 128));
+    }
+    const char* k = (const char*)((const bf16*)p.k + ((size_t)bh * T + j0) * D);
+    for (int x = tid; x < min(KB3, T - j0) * D * 2 / 128; x += NT3)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(k + (size_t)x * 128));
+  }
+
   float dq[D / 8][4];
 #pragma unroll
   for (int nt = 0; nt < D / 8; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) dq[nt][e] = 0.f;
 
-  if (M > 0) {  // dq += dS_meta MK
+  if (M > 0) {  // the meta tokens' dS and MK ride with the first block's copies
     const bf16* dsm = (const bf16*)p.ds_meta + ((size_t)bh * T + q0) * MT;
-    for (int x = tid; x < QT3 * MT / 8; x += NT) {
+    for (int x = tid; x < QR3 * MT / 8; x += NT3) {
       const int r = x / (MT / 8), cc = x % (MT / 8);
       const bool ok = q0 + r < T;
       cp_async16(&sm.dsm[r * 24 + cc * 8], dsm + (size_t)(ok ? r : 0) * MT + cc * 8, ok ? 16 : 0);
     }
     const bf16* mk = (const bf16*)p.mk + (size_t)h * M * D;
-    for (int x = tid; x < MT * D / 8; x += NT) {
+    for (int x = tid; x < MT * D / 8; x += NT3) {
       const int r = x / (D / 8), cc = x % (D / 8);
       const bool ok = r < M;
       cp_async16(&sm.mk[r * RPAD + cc * 8], mk + (size_t)(ok ? r : 0) * D + cc * 8, ok ? 16 : 0);
     }
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
-    uint32_t a[4];
-    ldsm_x4(smem_u32(&sm.dsm[(16 * warp + (lane & 15)) * 24 + (lane >> 4) * 8]), a[0], a[1], a[2], a[3]);
-#pragma unroll
-    for (int ntp = 0; ntp < D / 16; ++ntp) {
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(smem_u32(&sm.mk[((lane & 7) + ((lane >> 3) & 1) * 8) * RPAD + ntp * 16 + (lane >> 4) * 8]),
-                b0, b1, b2, b3);
-      mma_bf16(dq[2 * ntp], a, b0, b1);
-      mma_bf16(dq[2 * ntp + 1], a, b2, b3);
-    }
   }
-  // the key blocks whose window reaches the tile: keys >= q0 - w + 1, <= q0 + 63
-  const int b_lo = max(0, q0 - w + 1) / KB3, b_hi = min(q0 / KB3, nblk - 1);
   for (int b = b_lo; b <= b_hi; ++b) {
-    const int j0 = b * KB3, i = (q0 - j0) / QT3;
-    const int nq = (min(T - 1, j0 + KB3 - 1 + w - 1) - j0 + QT3) / QT3;  // tiles the key side formed
-    if (i >= nq) continue;
-    __syncthreads();  // the previous block's readers are done
-    const bf16* ds = (const bf16*)p.ds_tiles + (((size_t)bh * nblk + b) * p.ds_nq + i) * KB3 * QT3;
-    for (int x = tid; x < KB3 * QT3 / 8; x += NT) {
-      const int r = x / (QT3 / 8), cc = x % (QT3 / 8);
-      cp_async16(&sm.ds[r * DSP + cc * 8], ds + (size_t)r * QT3 + cc * 8, 16);
-    }
-    const bf16* k = (const bf16*)p.k + ((size_t)bh * T + j0) * D;
-    const int rows = min(KB3, T - j0);
-    for (int x = tid; x < KB3 * D / 8; x += NT) {
-      const int r = x / (D / 8), cc = x % (D / 8);
-      const bool ok = r < rows;
-      cp_async16(&sm.k[r * RPAD + cc * 8], k + (size_t)(ok ? r : 0) * D + cc * 8, ok ? 16 : 0);
-    }
+    if (b > b_lo) __syncthreads();  // the previous block's readers are done
+    load_block(b);
     cp_async_commit();
     cp_async_wait<0>();
     __syncthreads();
+    if (M > 0 && b == b_lo) {  // dq += dS_meta MK
+      uint32_t a[4];
+      ldsm_x4(smem_u32(&sm.dsm[(16 * warp + (lane & 15)) * 24 + (lane >> 4) * 8]), a[0], a[1], a[2], a[3]);
+#pragma unroll
+      for (int ntp = 0; ntp < D / 16; ++ntp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(smem_u32(&sm.mk[((lane & 7) + ((lane >> 3) & 1) * 8) * RPAD + ntp * 16 + (lane >> 4) * 8]),
+                  b0, b1, b2, b3);
+        mma_bf16(dq[2 * ntp], a, b0, b1);
+        mma_bf16(dq[2 * ntp + 1], a, b2, b3);
+      }
+    }
+    const int j0 = b * KB3;
+    if ((q0 - j0) / QT3 + half >= tiles_of(b)) continue;  // this warp's tile does not see the block
 #pragma unroll 2
     for (int kk = 0; kk < KB3 / 16; ++kk) {
       uint32_t a[4];  // A = dS (queries x keys) from the [key][query] tile, transposed
-      ldsm_x4_t(smem_u32(&sm.ds[(kk * 16 + (lane & 7) + ((lane >> 4) << 3)) * DSP + 16 * warp +
-                                ((lane >> 3) & 1) * 8]),
+      ldsm_x4_t(smem_u32(&sm.ds[half][(kk * 16 + (lane & 7) + ((lane >> 4) << 3)) * DSP + rw +
+                                      ((lane >> 3) & 1) * 8]),
                 a[0], a[1], a[2], a[3]);
 #pragma unroll
       for (int ntp = 0; ntp < D / 16; ++ntp) {
@@ -675,7 +733,7 @@ cudaError_t launch_swa_bwd_mma(const SwaBwdParams& p, cudaStream_t s) {
       e = launch_swa_bwd_q_tc(pp, s);
     } else {
       const auto kern = split ? swa_bwd_q_mma_kernel<false> : swa_bwd_q_mma_kernel<true>;
-      const size_t b1 = sizeof(QSmem);
+      const size_t b1 = split ? offsetof(QSmem, k) : sizeof(QSmem);
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)b1);
       if (e != cudaSuccess) return e;
       {
@@ -704,7 +762,7 @@ cudaError_t launch_swa_bwd_mma(const SwaBwdParams& p, cudaStream_t s) {
       if (e != cudaSuccess) return e;
       {
         ScopedTiming tm("swa_bwd_dq", s);
-        swa_bwd_dq_kernel<<<dim3((p.T + QT3 - 1) / QT3, p.B * p.H), NT, b3, s>>>(pp);
+        swa_bwd_dq_kernel<<<dim3((p.T + QR3 - 1) / QR3, p.B * p.H), NT3, b3, s>>>(pp);
       }
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
