@@ -18,6 +18,11 @@
 // Kernel 2 (key-major): CTA = 64 keys of one (batch, head), 4 warps x 16
 // keys, walking the 32-row query tiles that see them; dk, dv in registers.
 // A fixed-order reduction (shared with the SIMT path) sums the partials.
+// Split query side (kernel 1 with WINDOW = false, the tcgen05 key side and
+// kernel 3): when the forward output is given and the key side runs on
+// tcgen05, the key side stores the dS^T tiles it forms anyway, kernel 1 keeps
+// only D, the meta tokens' dS and the meta gradients, and kernel 3 forms dq
+// from the stored tiles, so the band's scores are formed once.
 #include "common.cuh"
 #include "kernels.h"
 #include "mma.cuh"
