@@ -230,12 +230,14 @@ def test_gla_bwd_long_context_gates_full_length():
 
 @pytest.mark.parametrize("T,w,M,sink", [(1, 1, 2, False), (64, 64, 0, False), (127, 129, 8, False),
                                          (129, 33, 3, True), (300, 128, 16, False),
-                                         (700, 100, 4, True)])
+                                         (700, 100, 4, True), (300, 130, 4, False),
+                                         (260, 300, 2, False)])
 def test_hybrid_bwd_split_query_side(T, w, M, sink):
     """bf16 hybrid backward given the window output: the query side keeps D
     and the meta terms, the tcgen05 key side stores its dS tiles and dq is
     formed from them (swa_bwd_dq), for ragged lengths, windows up to 129
-    keys, sink-only meta tokens and none; run twice, bit-identical."""
+    keys, sink-only meta tokens and none; wider windows take the unsplit
+    query side.  Run twice, bit-identical."""
     alpha = 0.7
     cpu, dev = small_problem(500 + T + w, 2, 2, T, 128, 128, M, torch.bfloat16, train=True)
     mk = dev["meta_k"] if M else None
@@ -251,8 +253,11 @@ def test_hybrid_bwd_split_query_side(T, w, M, sink):
     finally:
         L.lz_timing_enable(False)
     ran = {name for name, _ in L.lz_timing_read()}
-    assert {"swa_bwd_meta", "swa_bwd_kv_tc", "swa_bwd_dq"} <= ran, ran
-    assert "swa_bwd_q_mma" not in ran, ran
+    if w <= 129:
+        assert {"swa_bwd_meta", "swa_bwd_kv_tc", "swa_bwd_dq"} <= ran, ran
+        assert "swa_bwd_q_mma" not in ran, ran
+    else:
+        assert "swa_bwd_q_mma" in ran and not {"swa_bwd_meta", "swa_bwd_dq"} & ran, ran
     L.lz_device_check()
     x = oracle_inputs(cpu, ("q", "k", "v", "g", "meta_k", "meta_v", "dO"))
     ref = oracle.hybrid_bwd(x["q"], x["k"], x["v"], x["g"], x["meta_k"] if M else None,
