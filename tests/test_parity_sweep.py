@@ -1,0 +1,85 @@
+"""Seeded sweep of the hybrid operator's forward and backward over mixed
+configurations (bf16, d = 128): lengths around the chunk and tile sizes,
+windows from one key to wider than the tcgen05 band, meta tokens from none to
+the maximum with and without meta values, mix weights, initial states, gate
+strengths, and which forward results the backward is handed.  Every case is
+checked against the fp64 oracle at the bf16 bar.  The configurations are drawn
+from a fixed seed, so the sweep is the same on every run."""
+import math
+import random
+
+import numpy as np
+import pytest
+import torch
+
+import gated_linear_sliding_chunked_b200 as L
+import oracle
+from parity_util import assert_close, oracle_inputs, small_problem
+
+pytestmark = pytest.mark.gpu
+
+
+def _configs(seed=2027):
+    """Twelve cases: every length of the list once, windows and meta counts
+    cycled through shuffled lists, the other choices drawn per case."""
+    rng = random.Random(seed)
+    Ts = [1, 2, 63, 64, 65, 127, 128, 129, 191, 256, 333, 517]
+    ws = [1, 2, 17, 64, 100, 128, 129, 130, 200, 256]
+    Ms = [0, 1, 4, 8, 16]
+    for lst in (Ts, ws, Ms):
+        rng.shuffle(lst)
+    out = []
+    for i, T in enumerate(Ts):
+        M = Ms[i % len(Ms)]
+        out.append(dict(idx=i, T=T, w=ws[i % len(ws)], M=M, sink=M > 0 and rng.random() < 0.3,
+                        alpha=rng.choice([0.0, 0.25, 0.5, 1.0, 2.0]),
+                        h0=rng.random() < 0.5, g_mu=rng.choice([2.0, 0.0, -1.0]),
+                        g_div=rng.choice([16.0, 1.0]),
+                        saved=["none", "o_swa", "all"][i % 3]))
+    return out
+
+
+@pytest.mark.parametrize("cfg", _configs(), ids=lambda c: "case{idx}-T{T}-w{w}-M{M}".format(**c))
+def test_hybrid_sweep(cfg):
+    T, w, M, sink, alpha = cfg["T"], cfg["w"], cfg["M"], cfg["sink"], cfg["alpha"]
+    cpu, dev = small_problem(9000 + cfg["idx"], 2, 2, T, 128, 128, M, torch.bfloat16, train=True,
+                             h0=cfg["h0"], g_mu=cfg["g_mu"], g_div=cfg["g_div"])
+    mk = dev["meta_k"] if M else None
+    mv = dev["meta_v"] if (M and not sink) else None
+    h0 = dev["h0"] if cfg["h0"] else None
+    saved = cfg["saved"]
+    f = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], mk, mv, w=w, alpha=alpha, h0=h0,
+                     want_hT=True, want_lse=True, want_o_swa=saved != "none",
+                     want_chunk_states=saved == "all")
+    b = L.hybrid_bwd(dev["q"], dev["k"], dev["v"], dev["g"], mk, mv, f["lse"], dev["dO"], w=w,
+                     alpha=alpha, h0=h0, dhT=dev["dhT"], o_swa=f["o_swa"],
+                     chunk_states=f["chunk_states"], hT=f["hT"] if saved == "all" else None,
+                     want_dh0=True)
+    L.lz_device_check()
+    x = oracle_inputs(cpu, ("q", "k", "v", "g", "meta_k", "meta_v", "dO", "h0", "dhT"))
+    mko = x["meta_k"] if M else None
+    mvo = x["meta_v"] if (M and not sink) else None
+    h0o = x["h0"] if cfg["h0"] else None
+    sc = 1 / math.sqrt(128)
+    rf = oracle.hybrid_fwd(x["q"], x["k"], x["v"], x["g"], mko, mvo, w, sc, alpha, h0o)
+    rb = oracle.hybrid_bwd(x["q"], x["k"], x["v"], x["g"], mko, mvo, x["dO"], w, sc, alpha, h0o,
+                           x["dhT"])
+    assert_close("o", f["o"], rf["o"], torch.bfloat16)
+    assert_close("hT", f["hT"], rf["hT"], torch.bfloat16)
+    for name in ("dq", "dk", "dv", "dg", "dh0"):
+        assert_close(name, b[name], rb[name], torch.bfloat16)
+    if M:
+        assert_close("dmeta_k", b["dmeta_k"], rb["dmeta_k"], torch.bfloat16)
+        if not sink:
+            assert_close("dmeta_v", b["dmeta_v"], rb["dmeta_v"], torch.bfloat16)
+    if saved == "none":  # D rebuilt from the scores in fp32
+        assert_close("dalpha", b["dalpha"].cpu().double().numpy(), np.array([rb["dalpha"]]),
+                     torch.bfloat16)
+    else:
+        # D_t = dO_t . o_swa_t read off the saved bf16 window output: dalpha
+        # carries its rounding, |err| <= 2^-9 sum |dO| |o_swa| (elementwise),
+        # which a relative bar misses when the sum cancels.  The bar is that
+        # bound (x 2), or the relative one where it is wider.
+        bound = 2.0 * 2.0 ** -9 * float(np.sum(np.abs(x["dO"]) * np.abs(rf["o_swa"])))
+        err = abs(float(b["dalpha"].item()) - rb["dalpha"])
+        assert err <= max(bound, 2e-2 * abs(rb["dalpha"])), (err, bound, rb["dalpha"])
