@@ -39,7 +39,8 @@ def _configs(seed=2027):
     return out
 
 
-@pytest.mark.parametrize("cfg", _configs(), ids=lambda c: "case{idx}-T{T}-w{w}-M{M}".format(**c))
+@pytest.mark.parametrize("cfg", _configs(),
+                         ids=lambda c: "case{idx}-T{T}-w{w}-M{M}".format(**c))
 def test_hybrid_sweep(cfg):
     T, w, M, sink, alpha = cfg["T"], cfg["w"], cfg["M"], cfg["sink"], cfg["alpha"]
     cpu, dev = small_problem(9000 + cfg["idx"], 2, 2, T, 128, 128, M, torch.bfloat16, train=True,
@@ -83,3 +84,51 @@ def test_hybrid_sweep(cfg):
         bound = 2.0 * 2.0 ** -9 * float(np.sum(np.abs(x["dO"]) * np.abs(rf["o_swa"])))
         err = abs(float(b["dalpha"].item()) - rb["dalpha"])
         assert err <= max(bound, 2e-2 * abs(rb["dalpha"])), (err, bound, rb["dalpha"])
+
+
+def _configs_f32(seed=2028):
+    rng = random.Random(seed)
+    out = []
+    for i, (T, d) in enumerate([(1, 64), (37, 128), (64, 64), (129, 128), (200, 64), (257, 128)]):
+        M = rng.choice([0, 2, 5, 16])
+        out.append(dict(idx=i, T=T, d=d, w=rng.choice([1, 16, 64, 100, 130, 300]), M=M,
+                        sink=M > 0 and rng.random() < 0.3, alpha=rng.choice([0.0, 0.5, 1.5]),
+                        h0=rng.random() < 0.5, g_mu=rng.choice([2.0, 0.0, -1.0]),
+                        g_div=rng.choice([16.0, 1.0])))
+    return out
+
+
+@pytest.mark.parametrize("cfg", _configs_f32(),
+                         ids=lambda c: "f32-case{idx}-T{T}-d{d}-w{w}-M{M}".format(**c))
+def test_hybrid_sweep_f32(cfg):
+    """The fp32 I/O kernels (SIMT) over the same kinds of mixed cases, at the
+    fp32 bar."""
+    T, d, w, M, sink, alpha = cfg["T"], cfg["d"], cfg["w"], cfg["M"], cfg["sink"], cfg["alpha"]
+    cpu, dev = small_problem(9500 + cfg["idx"], 1, 2, T, d, d, M, torch.float32, train=True,
+                             h0=cfg["h0"], g_mu=cfg["g_mu"], g_div=cfg["g_div"])
+    mk = dev["meta_k"] if M else None
+    mv = dev["meta_v"] if (M and not sink) else None
+    h0 = dev["h0"] if cfg["h0"] else None
+    f = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], mk, mv, w=w, alpha=alpha, h0=h0,
+                     want_hT=True, want_lse=True)
+    b = L.hybrid_bwd(dev["q"], dev["k"], dev["v"], dev["g"], mk, mv, f["lse"], dev["dO"], w=w,
+                     alpha=alpha, h0=h0, dhT=dev["dhT"], want_dh0=True)
+    L.lz_device_check()
+    x = oracle_inputs(cpu, ("q", "k", "v", "g", "meta_k", "meta_v", "dO", "h0", "dhT"))
+    mko = x["meta_k"] if M else None
+    mvo = x["meta_v"] if (M and not sink) else None
+    h0o = x["h0"] if cfg["h0"] else None
+    sc = 1 / math.sqrt(d)
+    rf = oracle.hybrid_fwd(x["q"], x["k"], x["v"], x["g"], mko, mvo, w, sc, alpha, h0o)
+    rb = oracle.hybrid_bwd(x["q"], x["k"], x["v"], x["g"], mko, mvo, x["dO"], w, sc, alpha, h0o,
+                           x["dhT"])
+    assert_close("o", f["o"], rf["o"], torch.float32)
+    assert_close("hT", f["hT"], rf["hT"], torch.float32)
+    for name in ("dq", "dk", "dv", "dg", "dh0"):
+        assert_close(name, b[name], rb[name], torch.float32)
+    if M:
+        assert_close("dmeta_k", b["dmeta_k"], rb["dmeta_k"], torch.float32)
+        if not sink:
+            assert_close("dmeta_v", b["dmeta_v"], rb["dmeta_v"], torch.float32)
+    assert_close("dalpha", b["dalpha"].cpu().double().numpy(), np.array([rb["dalpha"]]),
+                 torch.float32)
