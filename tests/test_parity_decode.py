@@ -1,6 +1,7 @@
 """Decode-step parity: the constant-memory generation step vs the oracle, the
 decode-equals-prefill identity on the GPU, and save/restore of the state."""
 import math
+import random
 
 import numpy as np
 import pytest
@@ -264,3 +265,63 @@ def test_prefill_hand_off_then_decode(dtype, T, w):
     assert_close("decode o after hand-off", dec, ref["o"][:, :, T:], dtype)
     assert_close("decode state after hand-off", state, ref["hT"], dtype)
     assert torch.all(pos.cpu() == T + n)
+
+
+def _decode_configs(seed=2029):
+    rng = random.Random(seed)
+    out = []
+    for i, T in enumerate([1, 63, 65, 128, 150, 257]):
+        Bd = rng.choice([1, 2, 3, 5])
+        M = rng.choice([0, 1, 4, 16])
+        out.append(dict(idx=i, dtype=[torch.bfloat16, torch.float32][i % 2], T=T,
+                        lens=[rng.randint(0, T) for _ in range(Bd)],
+                        w=rng.choice([1, 2, 16, 64, 128, 129, 200]), M=M,
+                        sink=M > 0 and rng.random() < 0.3, n=rng.choice([1, 3, 8]),
+                        alpha=rng.choice([0.0, 0.5, 2.0]), H=rng.choice([1, 2, 3])))
+    return out
+
+
+@pytest.mark.parametrize("cfg", _decode_configs(),
+                         ids=lambda c: "case{idx}-T{T}-w{w}-M{M}-Bd{}".format(len(c["lens"]), **c))
+def test_decode_sweep(cfg):
+    """Seeded mixed cases of the prefill hand-off with per-sequence prompt
+    lengths (zero included) followed by n decode steps: windows from one key
+    to wider than the ring's prompt part, meta tokens with and without
+    values, several mix weights and head counts; every sequence's outputs
+    and final state match the oracle's forward over its prompt and new
+    tokens."""
+    dtype, T, lens, w, M = cfg["dtype"], cfg["T"], cfg["lens"], cfg["w"], cfg["M"]
+    sink, n, alpha, H = cfg["sink"], cfg["n"], cfg["alpha"], cfg["H"]
+    Bd = len(lens)
+    cpu, dev = small_problem(7600 + cfg["idx"], Bd, H, T + n, 128, 128, M, dtype)
+    pk = cpu["k"][:, :, :T].clone()
+    pg = cpu["g"][:, :, :T].clone()
+    for b, l in enumerate(lens):  # padding: no key, no decay
+        pk[b, :, l:] = 0
+        pg[b, :, l:] = 0
+    mk = dev["meta_k"] if M else None
+    mv = dev["meta_v"] if (M and not sink) else None
+    pre = {"q": dev["q"][:, :, :T].contiguous(), "k": pk.cuda(),
+           "v": dev["v"][:, :, :T].contiguous(), "g": pg.cuda()}
+    fwd = L.hybrid_fwd(pre["q"], pre["k"], pre["v"], pre["g"], mk, mv, w=w, alpha=alpha,
+                       want_hT=True)
+    state, kring, vring, pos = L.decode_prefill(pre["k"], pre["v"], fwd["hT"], w=w,
+                                                lens=torch.tensor(lens))
+    x = {k: np64(v) for k, v in cpu.items()}
+    outs = []
+    for j in range(n):
+        idx = [l + j for l in lens]
+        tok = {name: torch.stack([cpu[name][b, :, idx[b]] for b in range(Bd)]).cuda()
+               for name in ("q", "k", "v", "g")}
+        outs.append(L.decode_step(state, kring, vring, pos, tok["q"], tok["k"], tok["v"],
+                                  tok["g"], mk, mv, alpha=alpha).clone())
+    torch.cuda.synchronize()
+    assert pos.cpu().tolist() == [l + n for l in lens]
+    for b, l in enumerate(lens):
+        sl = lambda name: x[name][b:b + 1, :, :l + n]
+        ref = oracle.hybrid_fwd(sl("q"), sl("k"), sl("v"), sl("g"), x["meta_k"] if M else None,
+                                x["meta_v"] if (M and not sink) else None, w,
+                                1 / math.sqrt(128), alpha)
+        got = torch.stack([o[b] for o in outs], dim=1)[None]
+        assert_close(f"decode o [seq {b}, prompt {l}]", got, ref["o"][:, :, l:], dtype)
+        assert_close(f"state [seq {b}]", state[b:b + 1], ref["hT"], dtype)
