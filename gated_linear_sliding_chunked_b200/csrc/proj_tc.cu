@@ -11,8 +11,9 @@
 // One CTA computes a 128-token x 256-feature tile (two heads of 128 or four of
 // 64) of one of the three outputs; consecutive CTAs take consecutive feature
 // tiles of the same 128 tokens, so the x rows they share come from L2.  Warp
-// roles: warp 0 lane 0 issues TMA copies into a 4-stage ring of
-// (x, W) k-tiles (64 hidden dims each, 128-byte swizzle); warp 1 lane 0
+// roles: warp 0 lane 0 issues TMA copies into a 2-stage ring of
+// (x, W) k-tiles (64 hidden dims each, 128-byte swizzle; two CTAs share an
+// SM, so one's epilogue overlaps the other's main loop); warp 1 lane 0
 // issues tcgen05.mma (M = 128, N = 256, K = 16) into a 256-column tensor-memory
 // accumulator and frees each stage with tcgen05.commit; warps 2..5 (one TMEM
 // lane quarter each) read the accumulator and store the tile.  Every wait is
@@ -29,7 +30,7 @@
 namespace lz {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 2;
 constexpr int NTH = 192;                   // 6 warps
 constexpr uint32_t kA = BM * BK * 2;       // bytes of one x k-tile
 constexpr uint32_t kB = BN * BK * 2;       // bytes of one W k-tile
@@ -53,7 +54,7 @@ struct ProjParams {
   unsigned int* status;
 };
 
-__global__ void __launch_bounds__(NTH, 1)
+__global__ void __launch_bounds__(NTH, 2)
     proj_tc_kernel(ProjParams p, const __grid_constant__ CUtensorMap tx,
                    const __grid_constant__ CUtensorMap tw0, const __grid_constant__ CUtensorMap tw1,
                    const __grid_constant__ CUtensorMap tw2) {
