@@ -232,23 +232,26 @@ def test_gla_bwd_long_context_gates_full_length():
                                          (129, 33, 3, True), (300, 128, 16, False),
                                          (700, 100, 4, True), (300, 130, 4, False),
                                          (260, 300, 2, False)])
-def test_hybrid_bwd_split_query_side(T, w, M, sink):
+@pytest.mark.parametrize("states", [False, True], ids=["no-states", "chunk-states"])
+def test_hybrid_bwd_split_query_side(T, w, M, sink, states):
     """bf16 hybrid backward given the window output: the query side keeps D
     and the meta terms, the tcgen05 key side stores its dS tiles and dq is
     formed from them (swa_bwd_dq), for ragged lengths, windows up to 129
     keys, sink-only meta tokens and none; wider windows take the unsplit
-    query side.  Run twice, bit-identical."""
+    query side.  With and without the forward's chunk states (the gated
+    first level then skips its own state pass).  Run twice, bit-identical."""
     alpha = 0.7
     cpu, dev = small_problem(500 + T + w, 2, 2, T, 128, 128, M, torch.bfloat16, train=True)
     mk = dev["meta_k"] if M else None
     mv = dev["meta_v"] if (M and not sink) else None
     fwd = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], mk, mv, w=w, alpha=alpha,
-                       want_lse=True, want_o_swa=True)
+                       want_lse=True, want_o_swa=True, want_chunk_states=states)
     L.lz_timing_read()
     L.lz_timing_enable(True)
     try:
         runs = [L.hybrid_bwd(dev["q"], dev["k"], dev["v"], dev["g"], mk, mv, fwd["lse"],
-                             dev["dO"], w=w, alpha=alpha, o_swa=fwd["o_swa"]) for _ in range(2)]
+                             dev["dO"], w=w, alpha=alpha, o_swa=fwd["o_swa"],
+                             chunk_states=fwd["chunk_states"]) for _ in range(2)]
         torch.cuda.synchronize()
     finally:
         L.lz_timing_enable(False)
