@@ -231,6 +231,13 @@ __global__ void __launch_bounds__(NT, 2) gla_states_kernel(GlaFwdParams p) {
 // 1.81 ms); a single chunk has nothing to scan.
 constexpr int kScanMinChunks = 2;
 
+// the CTA's threads request the 128-byte lines of [base, base + bytes) into L2
+__device__ __forceinline__ void prefetch_l2_lines(const void* base, size_t bytes, int tid) {
+  const char* b = static_cast<const char*>(base);
+  for (size_t off = (size_t)tid * 128; off < bytes; off += (size_t)NT * 128)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(b + off));
+}
+
 struct DeltaSmem {
   bf16 k[C * QKP];
   bf16 v[C * VP];
@@ -255,6 +262,7 @@ struct DeltaArgs {
   bf16* delta;     // [BH][nchunks][DK][DV]
   float* decay;    // [BH][nchunks][DK]
   int T;
+  int wave = 0;    // resident CTAs: the inputs of the CTA this far ahead go to L2
 };
 
 template <bool QSIDE>
@@ -290,6 +298,18 @@ __global__ void __launch_bounds__(NT, 2) gla_delta_kernel(DeltaArgs p) {
     }
   }
   cp_async_commit();
+  if (p.wave > 0) {  // the inputs of the CTA one wave later, into L2 (as in the output pass)
+    const size_t L = (size_t)blockIdx.y * gridDim.x + blockIdx.x + (size_t)p.wave;
+    if (L < (size_t)gridDim.x * gridDim.y) {
+      const int cn = (int)(L % gridDim.x), bhn = (int)(L / gridDim.x);
+      const int rn = min(C, T - cn * C);
+      const size_t row = (size_t)bhn * T + (size_t)cn * C;
+      prefetch_l2_lines(p.x + row * DK, (size_t)rn * DK * 2, tid);
+      prefetch_l2_lines(p.y + row * DV, (size_t)rn * DV * 2, tid);
+      if (p.gz) prefetch_l2_lines(p.gz + row * DK, (size_t)rn * DK * 2, tid);
+      else prefetch_l2_lines(p.g + row * DK, (size_t)rn * DK * 4, tid);
+    }
+  }
   cp_async_wait<0>();
   __syncthreads();
   if (p.gz) {  // log-gates from the logits; rows past the end: g = 0
@@ -468,9 +488,11 @@ cudaError_t run_delta(const DeltaArgs& a, int nchunks, int BH, const char* name,
   cudaError_t e = cudaFuncSetAttribute(gla_delta_kernel<QSIDE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)bytes);
   if (e != cudaSuccess) return e;
+  DeltaArgs aa = a;
+  aa.wave = resident_ctas(gla_delta_kernel<QSIDE>, NT, bytes);
   {
     ScopedTiming tm(name, s);
-    gla_delta_kernel<QSIDE><<<dim3(nchunks, BH), NT, bytes, s>>>(a);
+    gla_delta_kernel<QSIDE><<<dim3(nchunks, BH), NT, bytes, s>>>(aa);
   }
   return cudaGetLastError();
 }
@@ -511,13 +533,6 @@ __device__ __noinline__ float diag_score_global(const bf16* q, const bf16* k, Ga
     a += __bfloat162float(q[(size_t)rt * DK + i]) * __bfloat162float(k[(size_t)rs * DK + i]) * __expf(lg);
   }
   return a;
-}
-
-// the CTA's threads request the 128-byte lines of [base, base + bytes) into L2
-__device__ __forceinline__ void prefetch_l2_lines(const void* base, size_t bytes, int tid) {
-  const char* b = static_cast<const char*>(base);
-  for (size_t off = (size_t)tid * 128; off < bytes; off += (size_t)NT * 128)
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(b + off));
 }
 
 // LOSS: the stage-1 loss epilogue (p.target set); LOGITS: the gates arrive as
