@@ -280,6 +280,42 @@ def test_hybrid_bwd_split_query_side(T, w, M, sink, states):
             assert torch.equal(runs[0][name], runs[1][name]), name
 
 
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)], ids=["bf16", "f32"])
+@pytest.mark.parametrize("B,T", [(2, 0), (0, 70)], ids=["no-tokens", "no-sequences"])
+def test_hybrid_empty_inputs(dtype, d, B, T):
+    """Degenerate shapes through the forward and the backward.  With no
+    tokens the state passes through unchanged both ways (hT = h0, dh0 =
+    dhT), and with either no tokens or no sequences the meta-token gradients
+    and dalpha are exactly zero (the outputs start as uninitialised memory,
+    so the library must write them)."""
+    H, M = 2, 4
+    cpu, dev = small_problem(61 + T, B, H, T, d, d, M, dtype, train=True, h0=True)
+    bf = dtype == torch.bfloat16
+    f = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"], w=16,
+                     alpha=0.5, h0=dev["h0"], want_hT=True, want_lse=True, want_o_swa=bf,
+                     want_chunk_states=bf)
+    b = None
+    for _ in range(2):
+        if b is not None:  # NaN-filled and freed: the next call's outputs reuse these blocks
+            for t in (b["dmeta_k"], b["dmeta_v"], b["dalpha"]):
+                t.fill_(float("nan"))
+            torch.cuda.synchronize()
+            del b
+        b = L.hybrid_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
+                         f["lse"], dev["dO"], w=16, alpha=0.5, h0=dev["h0"], dhT=dev["dhT"],
+                         o_swa=f["o_swa"], chunk_states=f["chunk_states"], want_dh0=True)
+        L.lz_device_check()
+        assert f["o"].numel() == 0 and f["hT"].shape == (B, H, d, d)
+        for name in ("dq", "dk", "dv", "dg"):
+            assert b[name].numel() == 0, name
+        if B:
+            assert torch.equal(f["hT"].cpu(), cpu["h0"])
+            assert torch.equal(b["dh0"].cpu(), cpu["dhT"])
+        assert torch.equal(b["dmeta_k"].cpu(), torch.zeros(H, M, d))
+        assert torch.equal(b["dmeta_v"].cpu(), torch.zeros(H, M, d))
+        assert float(b["dalpha"].item()) == 0.0
+
+
 def test_bwd_determinism():
     cpu, dev = small_problem(8, 2, 2, 300, 128, 128, 4, torch.bfloat16, train=True)
     fwd = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
