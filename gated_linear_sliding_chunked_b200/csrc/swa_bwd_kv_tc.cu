@@ -7,14 +7,18 @@
 // gscale * dO of the output gradient and D_t = dO_t . o_t:
 //   dV_j = gscale * sum_t P_tj dO_t,   dK_j = scale * gscale * sum_t dS_tj q_t,
 //   dS_tj = P_tj (dO_t . v_j - D_t).
-// One CTA = 128 keys of one (batch, head), 8 warps; it walks the 64-query
-// tiles that see them.  Per tile:
-//   thread 0: the NEXT tile's S^T = K Q^T and dP^T = V dO^T (M = 128 keys,
-//             N = 64 queries) into the other half of a double-buffered TMEM
-//             pair, so that they run while this tile's softmax does;
-//   all:      each key row's two threads read 32 query columns of this
-//             tile's scores, form P^T and dS^T (bf16) in shared memory;
-//   thread 0: dV += P^T dO, dK += dS^T Q (M = 128, N = 128, K = 64), commit.
+// One CTA = 128 keys of one (batch, head); it walks the 64-query tiles that
+// see them.  Nine warps:
+//   warp 8, the producer (one lane): the TMA copies, and per tile i the NEXT
+//             tile's S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = 64
+//             queries) into the other half of a double-buffered TMEM pair,
+//             then, once tile i's P^T and dS^T are in shared memory,
+//             dV += P^T dO and dK += dS^T Q (M = 128, N = 128, K = 64) and a
+//             commit;
+//   warps 0-7: each key row's two threads read 32 query columns of tile i's
+//             scores and form P^T and dS^T (bf16) in one of two shared-memory
+//             buffers, so that they wait for the gradient MMAs of tile i - 2,
+//             not of tile i - 1.
 // Q / dO tiles rotate through three shared-memory buffers, loaded by TMA
 // two tiles ahead.  With p.ds_tiles set the threads also store their bf16
 // dS^T rows of every tile to global memory, from which swa_bwd_dq forms dq
@@ -36,7 +40,8 @@ namespace {
 constexpr int KR = 128;   // keys per CTA (MMA M)
 constexpr int QT = 64;    // queries per tile
 constexpr int D = 128;
-constexpr int NTH = 256;
+constexpr int NSW = 256;  // softmax threads (warps 0-7)
+constexpr int NTH = NSW + 32;  // + the producer warp
 constexpr uint32_t kHalf = 64 * 2;  // bytes of one swizzled row (64 dims)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDK = 0, kColDV = 128, kColS = 256, kColDP = 384;  // S^T, dP^T: + 64 * buffer
@@ -47,14 +52,15 @@ struct KvSmem {
   uint8_t v[2][KR * kHalf];
   uint8_t q[3][2][QT * kHalf];    // [buffer][dim half]: 64 query rows
   uint8_t dO[3][2][QT * kHalf];
-  uint8_t pt[KR * QT * 2];        // P^T, bf16, no-swizzle K-major
-  uint8_t dst[KR * QT * 2];       // dS^T
+  uint8_t pt[2][KR * QT * 2];     // P^T of tile i in buffer i & 1, bf16, no-swizzle K-major
+  uint8_t dst[2][KR * QT * 2];    // dS^T
   float lse2[3][QT];              // lse * log2(e) of the tile's queries
   float dq[3][QT];                // D of the tile's queries
   uint64_t bar_kv;
-  uint64_t bar_ld[3];
-  uint64_t bar_s[2];
-  uint64_t bar_o;
+  uint64_t bar_ld[3];             // Q / dO buffer landed
+  uint64_t bar_s[2];              // tile i's scores in TMEM buffer i & 1
+  uint64_t bar_o[2];              // tile i's gradient MMAs done: P^T / dS^T buffer i & 1 free
+  uint64_t bar_p[2];              // tile i's P^T / dS^T written (one arrival per softmax warp)
   uint32_t tmem_base;
 };
 static_assert(sizeof(KvSmem) + 1024 <= 232448, "shared memory per block exceeds 227 KB");
@@ -69,7 +75,7 @@ __global__ void __launch_bounds__(NTH, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   KvSmem& sm = *reinterpret_cast<KvSmem*>(smem_raw + ((1024u - (raw & 1023u)) & 1023u));
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.y;
   const int T = p.T, w = p.w;
   const int j0 = blockIdx.x * KR;
@@ -81,11 +87,14 @@ __global__ void __launch_bounds__(NTH, 1)
 
   const uint32_t s_k = smem_u32(sm.k), s_v = smem_u32(sm.v), s_q = smem_u32(sm.q);
   const uint32_t s_do = smem_u32(sm.dO), s_pt = smem_u32(sm.pt), s_dst = smem_u32(sm.dst);
-  const uint32_t bar_kv = smem_u32(&sm.bar_kv), bar_o = smem_u32(&sm.bar_o);
+  const uint32_t bar_kv = smem_u32(&sm.bar_kv);
   const uint32_t bar_ld0 = smem_u32(&sm.bar_ld[0]), bar_s0 = smem_u32(&sm.bar_s[0]);  // + 8 per buffer
+  const uint32_t bar_o0 = smem_u32(&sm.bar_o[0]), bar_p0 = smem_u32(&sm.bar_p[0]);
   constexpr uint32_t kTileBytes = 2 * 2 * QT * kHalf;                               // Q and dO, both halves
+  constexpr uint32_t kPBytes = KR * QT * 2;                                         // one P^T / dS^T buffer
 
-  // query tile i -> buffer i % 3: Q / dO by TMA (thread 0), lse and D by threads
+  // query tile i -> buffer i % 3: Q / dO by TMA (the producer), lse and D by
+  // softmax threads
   auto issue_tile = [&](int i) {
     const int b = i % 3, t = j0 + i * QT;
     mbar_expect_tx(bar_ld0 + 8 * b, kTileBytes);
@@ -113,16 +122,31 @@ __global__ void __launch_bounds__(NTH, 1)
     }
     mma_commit(bar_s0 + 8 * tb);
   };
+  // dV += P^T dO, dK += dS^T Q of tile i: P^T / dS^T buffer i & 1, Q / dO
+  // buffer i % 3 as MN-major B operands (16 queries = 2048 bytes per step)
+  auto issue_grads = [&](int i, uint32_t tmem) {
+    const int b = i % 3, pb = i & 1;
+    constexpr uint32_t idG = idesc_bf16(KR, D, true);
+#pragma unroll
+    for (int kk = 0; kk < QT / 16; ++kk) {
+      const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+      mma_bf16_ss(tmem + kColDV, sdesc(s_pt + pb * kPBytes + kk * 256, 128, 1024),
+                  sdesc_sw128(s_do + 2 * b * QT * kHalf + kk * 2048, QT * kHalf, 1024), idG, acc);
+      mma_bf16_ss(tmem + kColDK, sdesc(s_dst + pb * kPBytes + kk * 256, 128, 1024),
+                  sdesc_sw128(s_q + 2 * b * QT * kHalf + kk * 2048, QT * kHalf, 1024), idG, acc);
+    }
+    mma_commit(bar_o0 + 8 * pb);
+  };
 
   if (warp == 0) tmem_alloc(smem_u32(&sm.tmem_base), kTmemCols);
   if (tid == 0) {
     mbar_init(bar_kv, 1);
-    mbar_init(bar_ld0, 1);
-    mbar_init(bar_ld0 + 8, 1);
-    mbar_init(bar_ld0 + 16, 1);
-    mbar_init(bar_s0, 1);
-    mbar_init(bar_s0 + 8, 1);
-    mbar_init(bar_o, 1);
+    for (int b = 0; b < 3; ++b) mbar_init(bar_ld0 + 8 * b, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_s0 + 8 * b, 1);
+      mbar_init(bar_o0 + 8 * b, 1);
+      mbar_init(bar_p0 + 8 * b, NSW / 32);
+    }
     mbar_init_fence();
   }
   for (int i = 0; i < 3 && i < nq; ++i) load_stats(i);
@@ -131,122 +155,128 @@ __global__ void __launch_bounds__(NTH, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
+  // Every wait below is on a barrier whose next phase cannot complete before
+  // the wait is satisfied (each ring of barriers is indexed by the tile's
+  // parity and advanced only through the other role), so parity waits never
+  // see a phase ahead of the one they wait for.
   bool alive = true;
-  if (tid == 0) {
-    mbar_expect_tx(bar_kv, 2 * 2 * KR * kHalf);
-    for (int hf = 0; hf < 2; ++hf) {
-      tma_load_3d(s_k + hf * KR * kHalf, &tk, bar_kv, hf * 64, j0, bh);
-      tma_load_3d(s_v + hf * KR * kHalf, &tv, bar_kv, hf * 64, j0, bh);
-    }
-    for (int i = 0; i < 3 && i < nq; ++i) issue_tile(i);
-    alive = mbar_wait(bar_kv, 0, p.status) && mbar_wait(bar_ld0, 0, p.status);
-    if (alive) issue_scores(0, tmem);
-  }
-
-  // this thread: key row kr (TMEM lane), query columns [32 hf, 32 hf + 32)
-  const int kr = tid & (KR - 1), hf = tid >> 7;
-  const int j = j0 + kr;
-  const uint32_t lrow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+  if (warp == NSW / 32) {
+    // ---- producer ---------------------------------------------------------
+    if (lane == 0) {
+      mbar_expect_tx(bar_kv, 2 * 2 * KR * kHalf);
+      for (int hf = 0; hf < 2; ++hf) {
+        tma_load_3d(s_k + hf * KR * kHalf, &tk, bar_kv, hf * 64, j0, bh);
+        tma_load_3d(s_v + hf * KR * kHalf, &tv, bar_kv, hf * 64, j0, bh);
+      }
+      for (int i = 0; i < 3 && i < nq; ++i) issue_tile(i);
+      alive = mbar_wait(bar_kv, 0, p.status) && mbar_wait(bar_ld0, 0, p.status);
+      if (alive) issue_scores(0, tmem);
 #pragma unroll 1
-  for (int i = 0; i < nq; ++i) {
-    const int b = i % 3, tb = i & 1;
-    const int t0c = j0 + i * QT + hf * 32;  // first query column of this thread
-    // the next tile's scores run on the tensor cores during this softmax
-    // (TMEM buffer (i + 1) & 1 was last read before the previous barrier)
-    if (tid == 0 && alive && i + 1 < nq) {
-      alive = mbar_wait(bar_ld0 + 8 * ((i + 1) % 3), ((i + 1) / 3) & 1, p.status);
-      if (alive) issue_scores(i + 1, tmem);
-    }
-    if (alive) alive = mbar_wait(bar_s0 + 8 * tb, (i >> 1) & 1, p.status);
-    tc_fence_after();
-    uint32_t s[32], dp[32];
-    tmem_ld32(lrow + kColS + QT * tb + hf * 32, s);
-    tmem_ld32(lrow + kColDP + QT * tb + hf * 32, dp);
-    tmem_ld_wait();
-    if (i > 0) {  // tile i-1's gradient MMAs are done: P^T, dS^T and its buffer are free
-      if (alive) alive = mbar_wait(bar_o, (i - 1) & 1, p.status);
-      if (i + 2 < nq) {
-        if (tid == 0 && alive) issue_tile(i + 2);
-        load_stats(i + 2);
+      for (int i = 0; i < nq; ++i) {
+        // the next tile's scores run on the tensor cores during this softmax
+        // (TMEM buffer (i + 1) & 1 was last read before tile i - 1's arrival)
+        if (i + 1 < nq) {
+          if (alive) alive = mbar_wait(bar_ld0 + 8 * ((i + 1) % 3), ((i + 1) / 3) & 1, p.status);
+          if (alive) issue_scores(i + 1, tmem);
+        }
+        if (i > 0 && i + 2 < nq) {  // Q / dO buffer (i + 2) % 3: read by tile i - 1's gradient MMAs
+          if (alive) alive = mbar_wait(bar_o0 + 8 * ((i - 1) & 1), ((i - 1) >> 1) & 1, p.status);
+          if (alive) issue_tile(i + 2);
+        }
+        if (alive) alive = mbar_wait(bar_p0 + 8 * (i & 1), (i >> 1) & 1, p.status);
+        tc_fence_after();
+        if (alive) issue_grads(i, tmem);
       }
     }
-    // P^T, dS^T of this thread's 32 columns
-    uint32_t pk[16], dk2[16];
-#pragma unroll
-    for (int c = 0; c < 32; c += 2) {
-      float pr[2], ds[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int t = t0c + c + e, cl = hf * 32 + c + e;
-        const bool ok = j < T && t < T && (unsigned)(t - j) < (unsigned)w;
-        const float P = ok ? exp2f(fmaf(__uint_as_float(s[c + e]), c2, -sm.lse2[b][cl])) : 0.f;
-        pr[e] = P;
-        ds[e] = P * (__uint_as_float(dp[c + e]) - sm.dq[b][cl]);
-      }
-      pk[c / 2] = pack_bf16(pr[0], pr[1]);
-      dk2[c / 2] = pack_bf16(ds[0], ds[1]);
-    }
-    if (p.ds_tiles) {  // dS^T of this tile for the split query side: [bh][block][tile][key][query]
-      uint4* dst = reinterpret_cast<uint4*>((bf16*)p.ds_tiles +
-                                            ((((size_t)bh * gridDim.x + blockIdx.x) * p.ds_nq + i) * KR + kr) * QT +
-                                            hf * 32);
-#pragma unroll
-      for (int x = 0; x < 4; ++x) dst[x] = make_uint4(dk2[4 * x], dk2[4 * x + 1], dk2[4 * x + 2], dk2[4 * x + 3]);
-    }
-#pragma unroll
-    for (int x = 0; x < 4; ++x) {  // K-major [128 keys][64 queries], 8-row groups 1024 bytes apart
-      const uint32_t off = (kr >> 3) * 1024 + (hf * 4 + x) * 128 + (kr & 7) * 16;
-      *reinterpret_cast<uint4*>(sm.pt + off) = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
-      *reinterpret_cast<uint4*>(sm.dst + off) =
-          make_uint4(dk2[4 * x], dk2[4 * x + 1], dk2[4 * x + 2], dk2[4 * x + 3]);
-    }
-    fence_async_smem();
-    tc_fence_before();
-    alive = __syncthreads_and(alive);
-    if (tid == 0 && alive) {
+    __syncwarp();
+  } else {
+    // ---- softmax warps: key row kr (TMEM lane), query columns [32 hf, 32 hf + 32)
+    const int kr = tid & (KR - 1), hf = tid >> 7;
+    const int j = j0 + kr;
+    const uint32_t lrow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+#pragma unroll 1
+    for (int i = 0; i < nq; ++i) {
+      const int b = i % 3, tb = i & 1;
+      const int t0c = j0 + i * QT + hf * 32;  // first query column of this thread
+      // statistics buffer (i + 2) % 3 was last read for tile i - 1, before
+      // the softmax warps' barrier that ended the previous iteration
+      if (i > 0 && i + 2 < nq) load_stats(i + 2);
+      if (alive) alive = mbar_wait(bar_s0 + 8 * tb, (i >> 1) & 1, p.status);
       tc_fence_after();
-      constexpr uint32_t idG = idesc_bf16(KR, D, true);
-#pragma unroll
-      for (int kk = 0; kk < QT / 16; ++kk) {  // B: Q / dO as MN-major, 16 queries = 2048 bytes
-        const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-        mma_bf16_ss(tmem + kColDV, sdesc(s_pt + kk * 256, 128, 1024),
-                    sdesc_sw128(s_do + 2 * b * QT * kHalf + kk * 2048, QT * kHalf, 1024), idG, acc);
-        mma_bf16_ss(tmem + kColDK, sdesc(s_dst + kk * 256, 128, 1024),
-                    sdesc_sw128(s_q + 2 * b * QT * kHalf + kk * 2048, QT * kHalf, 1024), idG, acc);
-      }
-      mma_commit(bar_o);
-    }
-  }
-  if (alive) alive = mbar_wait(bar_o, (nq - 1) & 1, p.status);
-  tc_fence_after();
-
-  // ---- epilogue: dK, dV rows of this CTA's keys, 64 columns per thread ------
-  const size_t off = ((size_t)bh * T + j) * D;
-  const float sk = p.scale * p.gscale, sv = p.gscale;
-#pragma unroll 1
-  for (int g = 0; g < 2; ++g) {  // 0: dK, 1: dV
-#pragma unroll 1
-    for (int c0 = hf * 64; c0 < hf * 64 + 64; c0 += 32) {
-      uint32_t r[32];
-      tmem_ld32(lrow + (g == 0 ? kColDK : kColDV) + c0, r);
+      uint32_t s[32], dp[32];
+      tmem_ld32(lrow + kColS + QT * tb + hf * 32, s);
+      tmem_ld32(lrow + kColDP + QT * tb + hf * 32, dp);
       tmem_ld_wait();
-      if (!alive || j >= T) continue;
-      const float sc = g == 0 ? sk : sv;
-      float* f32 = g == 0 ? p.dk_f32 : p.dv_f32;
-      if (f32) {
-        float4* dst = reinterpret_cast<float4*>(f32 + off + c0);
+      // P^T, dS^T of this thread's 32 columns
+      uint32_t pk[16], dk2[16];
 #pragma unroll
-        for (int x = 0; x < 8; ++x)
-          dst[x] = make_float4(__uint_as_float(r[4 * x]) * sc, __uint_as_float(r[4 * x + 1]) * sc,
-                               __uint_as_float(r[4 * x + 2]) * sc, __uint_as_float(r[4 * x + 3]) * sc);
-      } else {
-        uint32_t pk[16];
+      for (int c = 0; c < 32; c += 2) {
+        float pr[2], ds[2];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2)
-          pk[c / 2] = pack_bf16(__uint_as_float(r[c]) * sc, __uint_as_float(r[c + 1]) * sc);
-        uint4* dst = reinterpret_cast<uint4*>((bf16*)(g == 0 ? p.dk : p.dv) + off + c0);
+        for (int e = 0; e < 2; ++e) {
+          const int t = t0c + c + e, cl = hf * 32 + c + e;
+          const bool ok = j < T && t < T && (unsigned)(t - j) < (unsigned)w;
+          const float P = ok ? exp2f(fmaf(__uint_as_float(s[c + e]), c2, -sm.lse2[b][cl])) : 0.f;
+          pr[e] = P;
+          ds[e] = P * (__uint_as_float(dp[c + e]) - sm.dq[b][cl]);
+        }
+        pk[c / 2] = pack_bf16(pr[0], pr[1]);
+        dk2[c / 2] = pack_bf16(ds[0], ds[1]);
+      }
+      if (p.ds_tiles) {  // dS^T of this tile for the split query side: [bh][block][tile][key][query]
+        uint4* dst = reinterpret_cast<uint4*>((bf16*)p.ds_tiles +
+                                              ((((size_t)bh * gridDim.x + blockIdx.x) * p.ds_nq + i) * KR + kr) * QT +
+                                              hf * 32);
 #pragma unroll
-        for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+        for (int x = 0; x < 4; ++x) dst[x] = make_uint4(dk2[4 * x], dk2[4 * x + 1], dk2[4 * x + 2], dk2[4 * x + 3]);
+      }
+      // buffer tb was read by tile i - 2's gradient MMAs
+      if (i >= 2 && alive) alive = mbar_wait(bar_o0 + 8 * tb, ((i - 2) >> 1) & 1, p.status);
+      uint8_t* ptb = sm.pt[tb];
+      uint8_t* dsb = sm.dst[tb];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {  // K-major [128 keys][64 queries], 8-row groups 1024 bytes apart
+        const uint32_t off = (kr >> 3) * 1024 + (hf * 4 + x) * 128 + (kr & 7) * 16;
+        *reinterpret_cast<uint4*>(ptb + off) = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+        *reinterpret_cast<uint4*>(dsb + off) = make_uint4(dk2[4 * x], dk2[4 * x + 1], dk2[4 * x + 2], dk2[4 * x + 3]);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_p0 + 8 * tb);
+      asm volatile("bar.sync 1, %0;" ::"n"(NSW) : "memory");  // softmax warps only
+    }
+    if (alive) alive = mbar_wait(bar_o0 + 8 * ((nq - 1) & 1), ((nq - 1) >> 1) & 1, p.status);
+    tc_fence_after();
+
+    // ---- epilogue: dK, dV rows of this CTA's keys, 64 columns per thread ----
+    const size_t off = ((size_t)bh * T + j) * D;
+    const float sk = p.scale * p.gscale, sv = p.gscale;
+#pragma unroll 1
+    for (int g = 0; g < 2; ++g) {  // 0: dK, 1: dV
+#pragma unroll 1
+      for (int c0 = hf * 64; c0 < hf * 64 + 64; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(lrow + (g == 0 ? kColDK : kColDV) + c0, r);
+        tmem_ld_wait();
+        if (!alive || j >= T) continue;
+        const float sc = g == 0 ? sk : sv;
+        float* f32 = g == 0 ? p.dk_f32 : p.dv_f32;
+        if (f32) {
+          float4* dst = reinterpret_cast<float4*>(f32 + off + c0);
+#pragma unroll
+          for (int x = 0; x < 8; ++x)
+            dst[x] = make_float4(__uint_as_float(r[4 * x]) * sc, __uint_as_float(r[4 * x + 1]) * sc,
+                                 __uint_as_float(r[4 * x + 2]) * sc, __uint_as_float(r[4 * x + 3]) * sc);
+        } else {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2)
+            pk[c / 2] = pack_bf16(__uint_as_float(r[c]) * sc, __uint_as_float(r[c + 1]) * sc);
+          uint4* dst = reinterpret_cast<uint4*>((bf16*)(g == 0 ? p.dk : p.dv) + off + c0);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+        }
       }
     }
   }
