@@ -607,7 +607,9 @@ __global__ void __launch_bounds__(NT3, 2) swa_bwd_dq_kernel(SwaBwdParams p) {
   DqSmem& sm = *reinterpret_cast<DqSmem*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gr = lane >> 2, gc = (lane & 3) * 2;
-  const int q0 = blockIdx.x * QR3, bh = blockIdx.y, h = bh % p.H;
+  // batch-heads in reverse: the key side wrote the last ones' tiles last, so
+  // they are still in L2 when this pass starts
+  const int q0 = blockIdx.x * QR3, bh = gridDim.y - 1 - blockIdx.y, h = bh % p.H;
   const int T = p.T, w = p.w, M = p.M;
   const int nblk = (T + KB3 - 1) / KB3;
   const int half = warp >> 2, rw = 16 * (warp & 3);  // the warp's tile and its rows in it
