@@ -544,7 +544,9 @@ __global__ void __launch_bounds__(NT, 2) gla_out_kernel(GlaFwdParams p) {
   OutSmem& sm = *reinterpret_cast<OutSmem*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gr = lane >> 2, gc = (lane & 3) * 2;
-  const int c = blockIdx.x, bh = blockIdx.y;
+  // batch-heads in reverse: the window forward wrote the last ones' outputs
+  // last, so they are still in L2 when this pass starts
+  const int c = blockIdx.x, bh = gridDim.y - 1 - blockIdx.y;
   const int T = p.T;
   const int c0 = c * C;
   const int rows = min(C, T - c0);
@@ -579,7 +581,7 @@ __global__ void __launch_bounds__(NT, 2) gla_out_kernel(GlaFwdParams p) {
     // them there instead of waiting on HBM
     const size_t L = (size_t)blockIdx.y * gridDim.x + blockIdx.x + (size_t)p.wave;
     if (L < (size_t)gridDim.x * gridDim.y) {
-      const int cn = (int)(L % gridDim.x), bhn = (int)(L / gridDim.x);
+      const int cn = (int)(L % gridDim.x), bhn = (int)(gridDim.y - 1 - L / gridDim.x);
       const int rn = min(C, T - cn * C);
       const size_t row = (size_t)bhn * T + (size_t)cn * C;
       prefetch_l2_lines((const bf16*)p.q + row * DK, (size_t)rn * DK * 2, tid);
