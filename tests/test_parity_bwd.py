@@ -316,6 +316,32 @@ def test_hybrid_empty_inputs(dtype, d, B, T):
         assert float(b["dalpha"].item()) == 0.0
 
 
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)], ids=["bf16", "f32"])
+def test_hybrid_max_window_and_meta(dtype, d):
+    """The largest window the library takes (w = 1024) and the most meta
+    tokens (M = 16), at a ragged length past the window: forward and every
+    gradient against the oracle."""
+    T, w, M, alpha = 1100, 1024, 16, 0.8
+    cpu, dev = small_problem(1100 + d, 1, 2, T, d, d, M, dtype, train=True, h0=True)
+    f = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"], w=w,
+                     alpha=alpha, h0=dev["h0"], want_hT=True, want_lse=True)
+    b = L.hybrid_bwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],
+                     f["lse"], dev["dO"], w=w, alpha=alpha, h0=dev["h0"], dhT=dev["dhT"],
+                     want_dh0=True)
+    L.lz_device_check()
+    x = oracle_inputs(cpu, ("q", "k", "v", "g", "meta_k", "meta_v", "dO", "h0", "dhT"))
+    sc = 1 / math.sqrt(d)
+    rf = oracle.hybrid_fwd(x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], w, sc,
+                           alpha, x["h0"])
+    rb = oracle.hybrid_bwd(x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], x["dO"], w,
+                           sc, alpha, x["h0"], x["dhT"])
+    assert_close("o", f["o"], rf["o"], dtype)
+    assert_close("hT", f["hT"], rf["hT"], dtype)
+    for name in ("dq", "dk", "dv", "dg", "dh0", "dmeta_k", "dmeta_v"):
+        assert_close(name, b[name], rb[name], dtype)
+    assert_close("dalpha", b["dalpha"].cpu().double().numpy(), np.array([rb["dalpha"]]), dtype)
+
+
 def test_bwd_determinism():
     cpu, dev = small_problem(8, 2, 2, 300, 128, 128, 4, torch.bfloat16, train=True)
     fwd = L.hybrid_fwd(dev["q"], dev["k"], dev["v"], dev["g"], dev["meta_k"], dev["meta_v"],

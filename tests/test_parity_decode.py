@@ -325,3 +325,29 @@ def test_decode_sweep(cfg):
         got = torch.stack([o[b] for o in outs], dim=1)[None]
         assert_close(f"decode o [seq {b}, prompt {l}]", got, ref["o"][:, :, l:], dtype)
         assert_close(f"state [seq {b}]", state[b:b + 1], ref["hT"], dtype)
+
+
+def test_decode_max_window():
+    """The largest window the library takes (w = 1024) with the most meta
+    tokens (M = 16): 1100 decode steps from an empty state, so the ring wraps,
+    against the oracle's forward over the same tokens."""
+    Bd, H, T, w, M = 2, 2, 1100, 1024, 16
+    cpu, dev = small_problem(1024, Bd, H, T, 128, 128, M, torch.bfloat16)
+    alpha = 0.6
+    state = torch.zeros(Bd, H, 128, 128, device="cuda")
+    kring = torch.zeros(Bd, H, w, 128, dtype=torch.bfloat16, device="cuda")
+    vring = torch.zeros_like(kring)
+    pos = torch.zeros(Bd, dtype=torch.int64, device="cuda")
+    outs = []
+    for t in range(T):
+        sl = lambda n: dev[n][:, :, t].contiguous()
+        outs.append(L.decode_step(state, kring, vring, pos, sl("q"), sl("k"), sl("v"), sl("g"),
+                                  dev["meta_k"], dev["meta_v"], alpha=alpha).clone())
+    L.lz_device_check()
+    dec = torch.stack(outs, dim=2)
+    x = {k: np64(v) for k, v in cpu.items()}
+    ref = oracle.hybrid_fwd(x["q"], x["k"], x["v"], x["g"], x["meta_k"], x["meta_v"], w,
+                            1 / math.sqrt(128), alpha)
+    assert_close("decode o", dec, ref["o"], torch.bfloat16)
+    assert_close("decode state", state, ref["hT"], torch.bfloat16)
+    assert torch.all(pos.cpu() == T)
