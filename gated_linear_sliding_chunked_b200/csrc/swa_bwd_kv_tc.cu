@@ -41,6 +41,7 @@ constexpr int KR = 128;   // keys per CTA (MMA M)
 constexpr int QT = 64;    // queries per tile
 constexpr int D = 128;
 constexpr int NSW = 256;  // softmax threads (warps 0-7)
+constexpr int kBlocksPerCta = 4;  // consecutive key blocks one CTA walks
 constexpr int NTH = NSW + 32;  // + the producer warp
 constexpr uint32_t kHalf = 64 * 2;  // bytes of one swizzled row (64 dims)
 constexpr uint32_t kTmemCols = 512;
@@ -78,9 +79,27 @@ __global__ void __launch_bounds__(NTH, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.y;
   const int T = p.T, w = p.w;
-  const int j0 = blockIdx.x * KR;
-  const int tq_hi = min(T - 1, j0 + KR - 1 + w - 1);
-  const int nq = (tq_hi - j0 + QT) / QT;  // >= 1
+  const int nblk = (T + KR - 1) / KR;
+  const int blk0 = blockIdx.x * kBlocksPerCta, blk1 = min(nblk, blk0 + kBlocksPerCta);
+  // query tiles that see key block b (at least one)
+  auto nq_of = [&](int b) {
+    const int j0 = b * KR;
+    return (min(T - 1, j0 + KR - 1 + w - 1) - j0 + QT) / QT;
+  };
+  // the CTA walks the (key block, query tile) pairs of its blocks as one
+  // sequence g = 0 .. npair - 1
+  int npair = 0;
+  for (int b = blk0; b < blk1; ++b) npair += nq_of(b);
+  auto pair_of = [&](int g, int& b, int& i) {
+    b = blk0;
+    i = g;
+    while (b + 1 < blk1) {
+      const int n = nq_of(b);
+      if (i < n) break;
+      i -= n;
+      ++b;
+    }
+  };
   const float* lse = p.lse + (size_t)bh * T;
   const float* Db = p.Dbuf + (size_t)bh * T;
   const float c2 = p.scale * kLog2e;
@@ -93,47 +112,61 @@ __global__ void __launch_bounds__(NTH, 1)
   constexpr uint32_t kTileBytes = 2 * 2 * QT * kHalf;                               // Q and dO, both halves
   constexpr uint32_t kPBytes = KR * QT * 2;                                         // one P^T / dS^T buffer
 
-  // query tile i -> buffer i % 3: Q / dO by TMA (the producer), lse and D by
-  // softmax threads
-  auto issue_tile = [&](int i) {
-    const int b = i % 3, t = j0 + i * QT;
-    mbar_expect_tx(bar_ld0 + 8 * b, kTileBytes);
+  // K, V of key block b (the producer)
+  auto issue_kv = [&](int b) {
+    mbar_expect_tx(bar_kv, 2 * 2 * KR * kHalf);
     for (int hf = 0; hf < 2; ++hf) {
-      tma_load_3d(s_q + (2 * b + hf) * QT * kHalf, &tq, bar_ld0 + 8 * b, hf * 64, t, bh);
-      tma_load_3d(s_do + (2 * b + hf) * QT * kHalf, &tdo, bar_ld0 + 8 * b, hf * 64, t, bh);
+      tma_load_3d(s_k + hf * KR * kHalf, &tk, bar_kv, hf * 64, b * KR, bh);
+      tma_load_3d(s_v + hf * KR * kHalf, &tv, bar_kv, hf * 64, b * KR, bh);
     }
   };
-  auto load_stats = [&](int i) {
-    const int b = i % 3, t = j0 + i * QT;
-    if (tid < QT) sm.lse2[b][tid] = t + tid < T ? lse[t + tid] * kLog2e : 0.f;
-    else if (tid < 2 * QT) sm.dq[b][tid - QT] = t + tid - QT < T ? Db[t + tid - QT] : 0.f;
+  // pair g's query tile -> buffer g % 3: Q / dO by TMA (the producer), lse and
+  // D by softmax threads
+  auto issue_tile = [&](int g) {
+    int b, i;
+    pair_of(g, b, i);
+    const int buf = g % 3, t = b * KR + i * QT;
+    mbar_expect_tx(bar_ld0 + 8 * buf, kTileBytes);
+    for (int hf = 0; hf < 2; ++hf) {
+      tma_load_3d(s_q + (2 * buf + hf) * QT * kHalf, &tq, bar_ld0 + 8 * buf, hf * 64, t, bh);
+      tma_load_3d(s_do + (2 * buf + hf) * QT * kHalf, &tdo, bar_ld0 + 8 * buf, hf * 64, t, bh);
+    }
   };
-  // S^T and dP^T of tile i (shared-memory buffer i % 3) into TMEM buffer i & 1
-  auto issue_scores = [&](int i, uint32_t tmem) {
-    const int b = i % 3, tb = i & 1;
+  auto load_stats = [&](int g) {
+    int b, i;
+    pair_of(g, b, i);
+    const int buf = g % 3, t = b * KR + i * QT;
+    if (tid < QT) sm.lse2[buf][tid] = t + tid < T ? lse[t + tid] * kLog2e : 0.f;
+    else if (tid < 2 * QT) sm.dq[buf][tid - QT] = t + tid - QT < T ? Db[t + tid - QT] : 0.f;
+  };
+  // S^T and dP^T of pair g (shared-memory buffer g % 3, the K / V in shared
+  // memory) into TMEM buffer g & 1
+  auto issue_scores = [&](int g, uint32_t tmem) {
+    const int buf = g % 3, tb = g & 1;
     constexpr uint32_t idS = idesc_bf16(KR, QT, false);
 #pragma unroll 1
     for (int kk = 0; kk < D / 16; ++kk) {
       const uint32_t hf = kk >> 2, ko = (kk & 3) * 32;
       mma_bf16_ss(tmem + kColS + QT * tb, sdesc_sw128(s_k + hf * KR * kHalf + ko, 16, 1024),
-                  sdesc_sw128(s_q + (2 * b + hf) * QT * kHalf + ko, 16, 1024), idS, kk > 0);
+                  sdesc_sw128(s_q + (2 * buf + hf) * QT * kHalf + ko, 16, 1024), idS, kk > 0);
       mma_bf16_ss(tmem + kColDP + QT * tb, sdesc_sw128(s_v + hf * KR * kHalf + ko, 16, 1024),
-                  sdesc_sw128(s_do + (2 * b + hf) * QT * kHalf + ko, 16, 1024), idS, kk > 0);
+                  sdesc_sw128(s_do + (2 * buf + hf) * QT * kHalf + ko, 16, 1024), idS, kk > 0);
     }
     mma_commit(bar_s0 + 8 * tb);
   };
-  // dV += P^T dO, dK += dS^T Q of tile i: P^T / dS^T buffer i & 1, Q / dO
-  // buffer i % 3 as MN-major B operands (16 queries = 2048 bytes per step)
-  auto issue_grads = [&](int i, uint32_t tmem) {
-    const int b = i % 3, pb = i & 1;
+  // dV += P^T dO, dK += dS^T Q of pair g (first: the block's first pair, which
+  // starts the accumulators): P^T / dS^T buffer g & 1, Q / dO buffer g % 3 as
+  // MN-major B operands (16 queries = 2048 bytes per step)
+  auto issue_grads = [&](int g, bool first, uint32_t tmem) {
+    const int buf = g % 3, pb = g & 1;
     constexpr uint32_t idG = idesc_bf16(KR, D, true);
 #pragma unroll
     for (int kk = 0; kk < QT / 16; ++kk) {
-      const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+      const uint32_t acc = (!first || kk > 0) ? 1u : 0u;
       mma_bf16_ss(tmem + kColDV, sdesc(s_pt + pb * kPBytes + kk * 256, 128, 1024),
-                  sdesc_sw128(s_do + 2 * b * QT * kHalf + kk * 2048, QT * kHalf, 1024), idG, acc);
+                  sdesc_sw128(s_do + 2 * buf * QT * kHalf + kk * 2048, QT * kHalf, 1024), idG, acc);
       mma_bf16_ss(tmem + kColDK, sdesc(s_dst + pb * kPBytes + kk * 256, 128, 1024),
-                  sdesc_sw128(s_q + 2 * b * QT * kHalf + kk * 2048, QT * kHalf, 1024), idG, acc);
+                  sdesc_sw128(s_q + 2 * buf * QT * kHalf + kk * 2048, QT * kHalf, 1024), idG, acc);
     }
     mma_commit(bar_o0 + 8 * pb);
   };
@@ -149,59 +182,74 @@ __global__ void __launch_bounds__(NTH, 1)
     }
     mbar_init_fence();
   }
-  for (int i = 0; i < 3 && i < nq; ++i) load_stats(i);
+  for (int g = 0; g < 3 && g < npair; ++g) load_stats(g);
   tc_fence_before();
   __syncthreads();  // barriers, TMEM address, first statistics
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
   // Every wait below is on a barrier whose next phase cannot complete before
-  // the wait is satisfied (each ring of barriers is indexed by the tile's
-  // parity and advanced only through the other role), so parity waits never
-  // see a phase ahead of the one they wait for.
+  // the wait is satisfied (each ring of barriers is indexed by the pair's
+  // parity and advanced only through the other role; bar_kv only by the
+  // producer itself), so parity waits never see a phase ahead of the one
+  // they wait for.
   bool alive = true;
   if (warp == NSW / 32) {
     // ---- producer ---------------------------------------------------------
     if (lane == 0) {
-      mbar_expect_tx(bar_kv, 2 * 2 * KR * kHalf);
-      for (int hf = 0; hf < 2; ++hf) {
-        tma_load_3d(s_k + hf * KR * kHalf, &tk, bar_kv, hf * 64, j0, bh);
-        tma_load_3d(s_v + hf * KR * kHalf, &tv, bar_kv, hf * 64, j0, bh);
-      }
-      for (int i = 0; i < 3 && i < nq; ++i) issue_tile(i);
+      issue_kv(blk0);
+      for (int g = 0; g < 3 && g < npair; ++g) issue_tile(g);
       alive = mbar_wait(bar_kv, 0, p.status) && mbar_wait(bar_ld0, 0, p.status);
       if (alive) issue_scores(0, tmem);
+      int kvb = blk0, kvn = 0;  // the block whose K / V are loaded, and its load count - 1
 #pragma unroll 1
-      for (int i = 0; i < nq; ++i) {
-        // the next tile's scores run on the tensor cores during this softmax
-        // (TMEM buffer (i + 1) & 1 was last read before tile i - 1's arrival)
-        if (i + 1 < nq) {
-          if (alive) alive = mbar_wait(bar_ld0 + 8 * ((i + 1) % 3), ((i + 1) / 3) & 1, p.status);
-          if (alive) issue_scores(i + 1, tmem);
+      for (int g = 0; g < npair; ++g) {
+        int b, i;
+        pair_of(g, b, i);
+        // the next pair's scores run on the tensor cores during this softmax
+        // (TMEM buffer (g + 1) & 1 was last read before pair g - 1's arrival)
+        if (g + 1 < npair) {
+          int b1, i1;
+          pair_of(g + 1, b1, i1);
+          if (b1 != kvb) {  // a new key block: pair g's scores were the last to read K / V
+            if (alive) alive = mbar_wait(bar_s0 + 8 * (g & 1), (g >> 1) & 1, p.status);
+            if (alive) issue_kv(b1);
+            kvb = b1;
+            ++kvn;
+            if (alive) alive = mbar_wait(bar_kv, kvn & 1, p.status);
+          }
+          if (alive) alive = mbar_wait(bar_ld0 + 8 * ((g + 1) % 3), ((g + 1) / 3) & 1, p.status);
+          if (alive) issue_scores(g + 1, tmem);
         }
-        if (i > 0 && i + 2 < nq) {  // Q / dO buffer (i + 2) % 3: read by tile i - 1's gradient MMAs
-          if (alive) alive = mbar_wait(bar_o0 + 8 * ((i - 1) & 1), ((i - 1) >> 1) & 1, p.status);
-          if (alive) issue_tile(i + 2);
+        if (g > 0 && g + 2 < npair) {  // Q / dO buffer (g + 2) % 3: read by pair g - 1's gradient MMAs
+          if (alive) alive = mbar_wait(bar_o0 + 8 * ((g - 1) & 1), ((g - 1) >> 1) & 1, p.status);
+          if (alive) issue_tile(g + 2);
         }
-        if (alive) alive = mbar_wait(bar_p0 + 8 * (i & 1), (i >> 1) & 1, p.status);
+        // pair g's P^T / dS^T written; at a block's first pair this also
+        // means the previous block's dK / dV were read out of TMEM (the same
+        // warps read them before this pair's softmax)
+        if (alive) alive = mbar_wait(bar_p0 + 8 * (g & 1), (g >> 1) & 1, p.status);
         tc_fence_after();
-        if (alive) issue_grads(i, tmem);
+        if (alive) issue_grads(g, i == 0, tmem);
       }
     }
     __syncwarp();
   } else {
     // ---- softmax warps: key row kr (TMEM lane), query columns [32 hf, 32 hf + 32)
     const int kr = tid & (KR - 1), hf = tid >> 7;
-    const int j = j0 + kr;
     const uint32_t lrow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const float sk = p.scale * p.gscale, sv = p.gscale;
 #pragma unroll 1
-    for (int i = 0; i < nq; ++i) {
-      const int b = i % 3, tb = i & 1;
-      const int t0c = j0 + i * QT + hf * 32;  // first query column of this thread
-      // statistics buffer (i + 2) % 3 was last read for tile i - 1, before
+    for (int g = 0; g < npair; ++g) {
+      int b, i;
+      pair_of(g, b, i);
+      const int buf = g % 3, tb = g & 1;
+      const int j = b * KR + kr;
+      const int t0c = b * KR + i * QT + hf * 32;  // first query column of this thread
+      // statistics buffer (g + 2) % 3 was last read for pair g - 1, before
       // the softmax warps' barrier that ended the previous iteration
-      if (i > 0 && i + 2 < nq) load_stats(i + 2);
-      if (alive) alive = mbar_wait(bar_s0 + 8 * tb, (i >> 1) & 1, p.status);
+      if (g > 0 && g + 2 < npair) load_stats(g + 2);
+      if (alive) alive = mbar_wait(bar_s0 + 8 * tb, (g >> 1) & 1, p.status);
       tc_fence_after();
       uint32_t s[32], dp[32];
       tmem_ld32(lrow + kColS + QT * tb + hf * 32, s);
@@ -216,22 +264,21 @@ __global__ void __launch_bounds__(NTH, 1)
         for (int e = 0; e < 2; ++e) {
           const int t = t0c + c + e, cl = hf * 32 + c + e;
           const bool ok = j < T && t < T && (unsigned)(t - j) < (unsigned)w;
-          const float P = ok ? exp2f(fmaf(__uint_as_float(s[c + e]), c2, -sm.lse2[b][cl])) : 0.f;
+          const float P = ok ? exp2f(fmaf(__uint_as_float(s[c + e]), c2, -sm.lse2[buf][cl])) : 0.f;
           pr[e] = P;
-          ds[e] = P * (__uint_as_float(dp[c + e]) - sm.dq[b][cl]);
+          ds[e] = P * (__uint_as_float(dp[c + e]) - sm.dq[buf][cl]);
         }
         pk[c / 2] = pack_bf16(pr[0], pr[1]);
         dk2[c / 2] = pack_bf16(ds[0], ds[1]);
       }
-      if (p.ds_tiles) {  // dS^T of this tile for the split query side: [bh][block][tile][key][query]
+      if (p.ds_tiles) {  // dS^T of this pair for the split query side: [bh][block][tile][key][query]
         uint4* dst = reinterpret_cast<uint4*>((bf16*)p.ds_tiles +
-                                              ((((size_t)bh * gridDim.x + blockIdx.x) * p.ds_nq + i) * KR + kr) * QT +
-                                              hf * 32);
+                                              ((((size_t)bh * nblk + b) * p.ds_nq + i) * KR + kr) * QT + hf * 32);
 #pragma unroll
         for (int x = 0; x < 4; ++x) dst[x] = make_uint4(dk2[4 * x], dk2[4 * x + 1], dk2[4 * x + 2], dk2[4 * x + 3]);
       }
-      // buffer tb was read by tile i - 2's gradient MMAs
-      if (i >= 2 && alive) alive = mbar_wait(bar_o0 + 8 * tb, ((i - 2) >> 1) & 1, p.status);
+      // buffer tb was read by pair g - 2's gradient MMAs
+      if (g >= 2 && alive) alive = mbar_wait(bar_o0 + 8 * tb, ((g - 2) >> 1) & 1, p.status);
       uint8_t* ptb = sm.pt[tb];
       uint8_t* dsb = sm.dst[tb];
 #pragma unroll
@@ -244,40 +291,42 @@ __global__ void __launch_bounds__(NTH, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_p0 + 8 * tb);
-      asm volatile("bar.sync 1, %0;" ::"n"(NSW) : "memory");  // softmax warps only
-    }
-    if (alive) alive = mbar_wait(bar_o0 + 8 * ((nq - 1) & 1), ((nq - 1) >> 1) & 1, p.status);
-    tc_fence_after();
-
-    // ---- epilogue: dK, dV rows of this CTA's keys, 64 columns per thread ----
-    const size_t off = ((size_t)bh * T + j) * D;
-    const float sk = p.scale * p.gscale, sv = p.gscale;
+      if (i == nq_of(b) - 1) {
+        // ---- the block's last pair: dK, dV rows of its keys, 64 columns per thread
+        if (alive) alive = mbar_wait(bar_o0 + 8 * tb, (g >> 1) & 1, p.status);
+        tc_fence_after();
+        const size_t off = ((size_t)bh * T + j) * D;
 #pragma unroll 1
-    for (int g = 0; g < 2; ++g) {  // 0: dK, 1: dV
+        for (int gi = 0; gi < 2; ++gi) {  // 0: dK, 1: dV
 #pragma unroll 1
-      for (int c0 = hf * 64; c0 < hf * 64 + 64; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(lrow + (g == 0 ? kColDK : kColDV) + c0, r);
-        tmem_ld_wait();
-        if (!alive || j >= T) continue;
-        const float sc = g == 0 ? sk : sv;
-        float* f32 = g == 0 ? p.dk_f32 : p.dv_f32;
-        if (f32) {
-          float4* dst = reinterpret_cast<float4*>(f32 + off + c0);
+          for (int c0 = hf * 64; c0 < hf * 64 + 64; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(lrow + (gi == 0 ? kColDK : kColDV) + c0, r);
+            tmem_ld_wait();
+            if (!alive || j >= T) continue;
+            const float sc = gi == 0 ? sk : sv;
+            float* f32 = gi == 0 ? p.dk_f32 : p.dv_f32;
+            if (f32) {
+              float4* dst = reinterpret_cast<float4*>(f32 + off + c0);
 #pragma unroll
-          for (int x = 0; x < 8; ++x)
-            dst[x] = make_float4(__uint_as_float(r[4 * x]) * sc, __uint_as_float(r[4 * x + 1]) * sc,
-                                 __uint_as_float(r[4 * x + 2]) * sc, __uint_as_float(r[4 * x + 3]) * sc);
-        } else {
-          uint32_t pk[16];
+              for (int x = 0; x < 8; ++x)
+                dst[x] = make_float4(__uint_as_float(r[4 * x]) * sc, __uint_as_float(r[4 * x + 1]) * sc,
+                                     __uint_as_float(r[4 * x + 2]) * sc, __uint_as_float(r[4 * x + 3]) * sc);
+            } else {
+              uint32_t pk2[16];
 #pragma unroll
-          for (int c = 0; c < 32; c += 2)
-            pk[c / 2] = pack_bf16(__uint_as_float(r[c]) * sc, __uint_as_float(r[c + 1]) * sc);
-          uint4* dst = reinterpret_cast<uint4*>((bf16*)(g == 0 ? p.dk : p.dv) + off + c0);
+              for (int c = 0; c < 32; c += 2)
+                pk2[c / 2] = pack_bf16(__uint_as_float(r[c]) * sc, __uint_as_float(r[c + 1]) * sc);
+              uint4* dst = reinterpret_cast<uint4*>((bf16*)(gi == 0 ? p.dk : p.dv) + off + c0);
 #pragma unroll
-          for (int x = 0; x < 4; ++x) dst[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+              for (int x = 0; x < 4; ++x)
+                dst[x] = make_uint4(pk2[4 * x], pk2[4 * x + 1], pk2[4 * x + 2], pk2[4 * x + 3]);
+            }
+          }
         }
+        tc_fence_before();  // these TMEM reads precede the next arrival
       }
+      asm volatile("bar.sync 1, %0;" ::"n"(NSW) : "memory");  // softmax warps only
     }
   }
 
@@ -307,7 +356,7 @@ cudaError_t launch_swa_bwd_kv_tc(const SwaBwdParams& p, cudaStream_t s) {
   if (!tma_map_rows128(&tk, p.k, p.T, bh, KR) || !tma_map_rows128(&tv, p.v, p.T, bh, KR) ||
       !tma_map_rows128(&tq, p.q, p.T, bh, QT) || !tma_map_rows128(&tdo, p.dO, p.T, bh, QT))
     return cudaErrorInvalidValue;
-  dim3 grid((p.T + KR - 1) / KR, p.B * p.H);
+  dim3 grid(((p.T + KR - 1) / KR + kBlocksPerCta - 1) / kBlocksPerCta, p.B * p.H);
   {
     ScopedTiming tm("swa_bwd_kv_tc", s);
     swa_bwd_kv_tc_kernel<<<grid, NTH, bytes, s>>>(pp, tk, tv, tq, tdo);
