@@ -590,11 +590,12 @@ constexpr int QT3 = 64;        // query rows per dS tile
 constexpr int QR3 = 128;       // query rows per CTA (8 warps x 16): two tiles, one key block
 constexpr int NT3 = 256;
 constexpr int KB3 = 128;       // keys per block of the key side
+constexpr int KU3 = 64;        // keys per streamed unit (half a block)
 constexpr int DSP = QT3 + 8;   // padded row of a [key][query] dS tile
 
 struct DqSmem {
-  bf16 ds[2][KB3 * DSP];       // the block's dS tiles of the CTA's two query tiles
-  bf16 k[KB3 * RPAD];
+  bf16 ds[2][2][KU3 * DSP];    // [stage][query tile]: a unit's rows of the CTA's two dS tiles
+  bf16 k[2][KU3 * RPAD];       // [stage]: the unit's keys
   bf16 mk[MT * RPAD];
   bf16 dsm[QR3 * 24];          // the meta tokens' dS, [query][16] (+8 pad)
 };
@@ -617,38 +618,30 @@ __global__ void __launch_bounds__(NT3, 2) swa_bwd_dq_kernel(SwaBwdParams p) {
   const int b_lo = max(0, q0 - w + 1) / KB3, b_hi = min(q0 / KB3, nblk - 1);
   // tiles the key side formed for block b (the same count as its own loop)
   auto tiles_of = [&](int b) { return (min(T - 1, b * KB3 + KB3 - 1 + w - 1) - b * KB3 + QT3) / QT3; };
-  auto load_block = [&](int b) {
+  // the blocks stream through two stages in units of 64 keys: unit u = block
+  // b_lo + u / 2, keys [64 (u % 2), 64 (u % 2) + 64) of it
+  const int nu = 2 * (b_hi - b_lo + 1);
+  auto load_unit = [&](int u) {
+    const int b = b_lo + u / 2, st = u & 1, ko = KU3 * (u % 2);
     const int j0 = b * KB3, nq = tiles_of(b);
     for (int hf = 0; hf < 2; ++hf) {
       const int i = (q0 - j0) / QT3 + hf;
-      if (i >= nq) continue;  // no query of this tile sees the block: its rows read as zeros below
-      const bf16* ds = (const bf16*)p.ds_tiles + (((size_t)bh * nblk + b) * p.ds_nq + i) * KB3 * QT3;
-      for (int x = tid; x < KB3 * QT3 / 8; x += NT3) {
+      if (i >= nq) continue;  // no query of this tile sees the block: its warps skip it below
+      const bf16* ds = (const bf16*)p.ds_tiles + (((size_t)bh * nblk + b) * p.ds_nq + i) * KB3 * QT3 +
+                       (size_t)ko * QT3;
+      for (int x = tid; x < KU3 * QT3 / 8; x += NT3) {
         const int r = x / (QT3 / 8), cc = x % (QT3 / 8);
-        cp_async16(&sm.ds[hf][r * DSP + cc * 8], ds + (size_t)r * QT3 + cc * 8, 16);
+        cp_async16(&sm.ds[st][hf][r * DSP + cc * 8], ds + (size_t)r * QT3 + cc * 8, 16);
       }
     }
-    const bf16* k = (const bf16*)p.k + ((size_t)bh * T + j0) * D;
-    const int rows = min(KB3, T - j0);
-    for (int x = tid; x < KB3 * D / 8; x += NT3) {
+    const bf16* k = (const bf16*)p.k + (size_t)bh * T * D;
+    const int rows = min(KU3, T - j0 - ko);  // may be <= 0: all zeros
+    for (int x = tid; x < KU3 * D / 8; x += NT3) {
       const int r = x / (D / 8), cc = x % (D / 8);
-      const bool ok = r < rows;
-      cp_async16(&sm.k[r * RPAD + cc * 8], k + (size_t)(ok ? r : 0) * D + cc * 8, ok ? 16 : 0);
+      const bool ok = r < rows;  // zero-filled rows still name an in-bounds source row
+      cp_async16(&sm.k[st][r * RPAD + cc * 8], k + (size_t)(ok ? j0 + ko + r : j0) * D + cc * 8, ok ? 16 : 0);
     }
   };
-  if (b_lo < b_hi) {  // the last block's tiles and keys into L2 while the first is used
-    const int b = b_hi, j0 = b * KB3, nq = tiles_of(b);
-    for (int hf = 0; hf < 2; ++hf) {
-      const int i = (q0 - j0) / QT3 + hf;
-      if (i >= nq) continue;
-      const char* t = (const char*)p.ds_tiles + (((size_t)bh * nblk + b) * p.ds_nq + i) * KB3 * QT3 * 2;
-      for (int x = tid; x < KB3 * QT3 * 2 / 128; x += NT3)
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(t + x * 128));
-    }
-    const char* k = (const char*)((const bf16*)p.k + ((size_t)bh * T + j0) * D);
-    for (int x = tid; x < min(KB3, T - j0) * D * 2 / 128; x += NT3)
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(k + (size_t)x * 128));
-  }
 
   float dq[D / 8][4];
 #pragma unroll
@@ -656,7 +649,7 @@ __global__ void __launch_bounds__(NT3, 2) swa_bwd_dq_kernel(SwaBwdParams p) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) dq[nt][e] = 0.f;
 
-  if (M > 0) {  // the meta tokens' dS and MK ride with the first block's copies
+  if (M > 0) {  // the meta tokens' dS and MK ride with the first unit's copies
     const bf16* dsm = (const bf16*)p.ds_meta + ((size_t)bh * T + q0) * MT;
     for (int x = tid; x < QR3 * MT / 8; x += NT3) {
       const int r = x / (MT / 8), cc = x % (MT / 8);
@@ -670,13 +663,14 @@ __global__ void __launch_bounds__(NT3, 2) swa_bwd_dq_kernel(SwaBwdParams p) {
       cp_async16(&sm.mk[r * RPAD + cc * 8], mk + (size_t)(ok ? r : 0) * D + cc * 8, ok ? 16 : 0);
     }
   }
-  for (int b = b_lo; b <= b_hi; ++b) {
-    if (b > b_lo) __syncthreads();  // the previous block's readers are done
-    load_block(b);
-    cp_async_commit();
-    cp_async_wait<0>();
+  load_unit(0);
+  cp_async_commit();
+  if (nu > 1) load_unit(1);
+  cp_async_commit();
+  for (int u = 0; u < nu; ++u) {
+    cp_async_wait<1>();  // unit u's group (one group is committed per unit, empty past the end)
     __syncthreads();
-    if (M > 0 && b == b_lo) {  // dq += dS_meta MK
+    if (M > 0 && u == 0) {  // dq += dS_meta MK
       uint32_t a[4];
       ldsm_x4(smem_u32(&sm.dsm[(16 * warp + (lane & 15)) * 24 + (lane >> 4) * 8]), a[0], a[1], a[2], a[3]);
 #pragma unroll
@@ -688,24 +682,29 @@ __global__ void __launch_bounds__(NT3, 2) swa_bwd_dq_kernel(SwaBwdParams p) {
         mma_bf16(dq[2 * ntp + 1], a, b2, b3);
       }
     }
-    const int j0 = b * KB3;
-    if ((q0 - j0) / QT3 + half >= tiles_of(b)) continue;  // this warp's tile does not see the block
+    const int b = b_lo + u / 2, st = u & 1;
+    if ((q0 - b * KB3) / QT3 + half < tiles_of(b)) {  // this warp's tile sees the block
+      const bf16* dsb = sm.ds[st][half];
+      const bf16* kb = sm.k[st];
 #pragma unroll 2
-    for (int kk = 0; kk < KB3 / 16; ++kk) {
-      uint32_t a[4];  // A = dS (queries x keys) from the [key][query] tile, transposed
-      ldsm_x4_t(smem_u32(&sm.ds[half][(kk * 16 + (lane & 7) + ((lane >> 4) << 3)) * DSP + rw +
-                                      ((lane >> 3) & 1) * 8]),
-                a[0], a[1], a[2], a[3]);
+      for (int kk = 0; kk < KU3 / 16; ++kk) {
+        uint32_t a[4];  // A = dS (queries x keys) from the [key][query] tile, transposed
+        ldsm_x4_t(smem_u32(&dsb[(kk * 16 + (lane & 7) + ((lane >> 4) << 3)) * DSP + rw + ((lane >> 3) & 1) * 8]),
+                  a[0], a[1], a[2], a[3]);
 #pragma unroll
-      for (int ntp = 0; ntp < D / 16; ++ntp) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(smem_u32(&sm.k[(kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * RPAD + ntp * 16 +
+        for (int ntp = 0; ntp < D / 16; ++ntp) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(smem_u32(&kb[(kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * RPAD + ntp * 16 +
                                  (lane >> 4) * 8]),
-                  b0, b1, b2, b3);
-        mma_bf16(dq[2 * ntp], a, b0, b1);
-        mma_bf16(dq[2 * ntp + 1], a, b2, b3);
+                    b0, b1, b2, b3);
+          mma_bf16(dq[2 * ntp], a, b0, b1);
+          mma_bf16(dq[2 * ntp + 1], a, b2, b3);
+        }
       }
     }
+    __syncthreads();  // stage st is free
+    if (u + 2 < nu) load_unit(u + 2);
+    cp_async_commit();
   }
   const float sc = p.scale * p.gscale;
 #pragma unroll
