@@ -587,7 +587,7 @@ __global__ void __launch_bounds__(NT, 2) swa_bwd_kv_mma_kernel(SwaBwdParams p) {
 // (Lizard technical summary, section 2a: the window keys and the always-visible
 // meta tokens share one softmax, so they share its Jacobian).
 constexpr int QT3 = 64;        // query rows per dS tile
-constexpr int QR3 = 128;       // query rows per CTA (8 warps x 16): two tiles, one key block
+constexpr int QR3 = 128;       // query rows per CTA (8 warps x 16): two tiles that see the same key blocks
 constexpr int NT3 = 256;
 constexpr int KB3 = 128;       // keys per block of the key side
 constexpr int KU3 = 64;        // keys per streamed unit (half a block)
