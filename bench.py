@@ -542,26 +542,33 @@ def measure_stage1(wl, x, device, steps, warmup, seed):
             "kernels": {k: [c // steps, round(t / c, 4)] for k, (c, t) in tab.items()}}
 
 
-def measure_train_gate_logits(wl, x, device, steps, warmup, seed):
+def measure_train_gate_logits(wl, x, device, steps, warmup, seed, fused=False):
     """The training step with the gates given as bf16 logits z (log-gate =
-    log sigma(z) / 16, the workload's gate distribution with z ~ N(0, 1)),
-    formed inside the kernels instead of read as fp32 log-gates."""
+    log sigma(z) / 16, the workload's gate distribution with z ~ N(0, 1)):
+    mapped once to fp32 log-gates in the workspace and dL/dg mapped back to
+    dL/dz (the default), or (fused) mapped inside every gated kernel."""
     import gated_linear_sliding_chunked_b200 as L
     gen = torch.Generator(device=device)
     gen.manual_seed(2000 + seed)
     z = torch.randn(x["g"].shape, generator=gen, device=device).to(torch.bfloat16)
     xz = dict(x)
     xz["g"] = z
-    st = TrainStep(wl, xz, device, gate_logits=True, gate_scale=1.0 / 16)
-    for _ in range(warmup):
-        st.run()
-    torch.cuda.synchronize(device)
-    L.lz_timing_enable(True)
-    ms = time_region(st.run, steps, device)
-    L.lz_timing_enable(False)
-    tab = kernel_table(L.lz_timing_read())
-    L.lz_device_check()
-    return {"workload": wl.name + " with bf16 gate logits (log-gate = log sigma(z) / 16, z ~ N(0, 1))",
+    prev = L.lz_fused_gate_logits(fused)
+    try:
+        st = TrainStep(wl, xz, device, gate_logits=True, gate_scale=1.0 / 16)
+        for _ in range(warmup):
+            st.run()
+        torch.cuda.synchronize(device)
+        L.lz_timing_enable(True)
+        ms = time_region(st.run, steps, device)
+        L.lz_timing_enable(False)
+        tab = kernel_table(L.lz_timing_read())
+        L.lz_device_check()
+    finally:
+        L.lz_fused_gate_logits(prev)
+    how = "mapped inside every gated kernel" if fused else "mapped once, dL/dz by one more pass"
+    return {"workload": wl.name + " with bf16 gate logits (log-gate = log sigma(z) / 16, z ~ N(0, 1); "
+            + how + ")",
             "tokens_per_s": wl.B * wl.T / (ms * 1e-3), "ms_per_step": round(ms, 4),
             "kernels": {k: [c // steps, round(t / c, 4)] for k, (c, t) in tab.items()}}
 
@@ -951,6 +958,8 @@ def main(argv=None):
             "overlap and do not add up to the step")
         extras["stage1_step"] = measure_stage1(wl, xd, device, 10, 3, seed=rank)
         extras["train_step_gate_logits"] = measure_train_gate_logits(wl, xd, device, 10, 3, seed=rank)
+        extras["train_step_gate_logits_fused"] = measure_train_gate_logits(wl, xd, device, 10, 3,
+                                                                           seed=rank, fused=True)
         # last: a dense GEMM at full tensor-core load draws the most power, and
         # the power cap would lower the clocks of whatever runs right after it
         extras["qkg_projection"] = measure_projection(device, peaks, seed=rank)

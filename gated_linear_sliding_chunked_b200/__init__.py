@@ -34,7 +34,7 @@ EXPORTS = ("lz_gla_fwd", "lz_gla_bwd", "lz_swa_meta_fwd", "lz_hybrid_fwd", "lz_s
            "lz_version", "lz_timing_enable", "lz_timing_only", "lz_timing_read",
            "lz_swa_meta_bwd_noalloc", "lz_device_check", "lz_prefer_tcgen05", "lz_decode_prefill",
            "lz_hybrid_fwd_mse", "lz_selftest_bounded_wait", "lz_cp_segment_decay", "lz_cp_fold",
-           "lz_cp_rows", "lz_tcgen05_all", "lz_qkg_projection")
+           "lz_cp_rows", "lz_tcgen05_all", "lz_qkg_projection", "lz_fused_gate_logits")
 
 # size of the static scratch array behind lz_swa_meta_bwd_noalloc
 LZ_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -87,6 +87,7 @@ def load(path: str = LIB_PATH):
     lib.lz_prefer_tcgen05.argtypes = [ctypes.c_int]
     ci = ctypes.c_int
     lib.lz_tcgen05_all.argtypes = [ci]
+    lib.lz_fused_gate_logits.argtypes = [ci]
     lib.lz_qkg_projection.argtypes = [ci] * 5 + [_P] * 4 + [ctypes.c_float] + [_P] * 3 + [_P]
     lib.lz_cp_segment_decay.argtypes = [ci, ci, ci, _P, _P, _P]
     lib.lz_cp_fold.argtypes = [ci] * 6 + [_P] * 4 + [_P]
@@ -178,6 +179,13 @@ def lz_tcgen05_all(on: bool) -> bool:
     backward's query side), for the calling thread (default False); returns
     the previous setting."""
     return bool(load().lz_tcgen05_all(1 if on else 0))
+
+
+def lz_fused_gate_logits(on: bool) -> bool:
+    """Gates given as logits mapped inside every gated kernel (True) instead
+    of by one pass into the workspace (False, the default), for the calling
+    thread; returns the previous setting."""
+    return bool(load().lz_fused_gate_logits(1 if on else 0))
 
 
 def lz_timing_enable(on: bool):

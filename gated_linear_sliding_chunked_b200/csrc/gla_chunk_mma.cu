@@ -872,6 +872,75 @@ cudaError_t launch_gla_states(const GlaFwdParams& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Gates given as logits (Gamma = sigma(z)): one pass maps them to fp32
+// log-gates g = scale * log sigma(z) for the log-gate kernels, and one maps
+// those kernels' dL/dg to dL/dz = dL/dg * scale * sigma(-z) (the same
+// gate_from_logit / dlogit as the kernels that map them on the fly).
+// Eight elements a thread, one thread per eight elements (grid-stride past
+// 2^31 - 1 blocks), so that every load of the stream is in flight at once.
+__global__ void __launch_bounds__(256) gate_logits_to_log_kernel(const bf16* __restrict__ z, float* __restrict__ g,
+                                                                 size_t n8, float gs) {
+  for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < n8; i += (size_t)gridDim.x * 256) {
+    const uint4 zz = __ldcs(reinterpret_cast<const uint4*>(z) + i);
+    const uint32_t zw[4] = {zz.x, zz.y, zz.z, zz.w};
+    float o[8];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const float2 f = unpack_bf16(zw[x]);
+      o[2 * x] = gate_from_logit(f.x, gs);
+      o[2 * x + 1] = gate_from_logit(f.y, gs);
+    }
+    float4* dst = reinterpret_cast<float4*>(g) + 2 * i;
+    dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+__global__ void __launch_bounds__(256) gate_dlogit_kernel(float* __restrict__ dg, const bf16* __restrict__ z,
+                                                          size_t n8, float gs) {
+  for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < n8; i += (size_t)gridDim.x * 256) {
+    const uint4 zz = __ldcs(reinterpret_cast<const uint4*>(z) + i);
+    const uint32_t zw[4] = {zz.x, zz.y, zz.z, zz.w};
+    float4* d = reinterpret_cast<float4*>(dg) + 2 * i;
+    const float4 a = d[0], b = d[1];
+    float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const float2 f = unpack_bf16(zw[x]);
+      v[2 * x] = dlogit(v[2 * x], f.x, gs);
+      v[2 * x + 1] = dlogit(v[2 * x + 1], f.y, gs);
+    }
+    d[0] = make_float4(v[0], v[1], v[2], v[3]);
+    d[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+}
+
+static unsigned gate_pass_grid(size_t n8) {
+  const size_t want = (n8 + 255) / 256;
+  return (unsigned)(want < 0x7fffffffu ? (want > 0 ? want : 1) : 0x7fffffffu);
+}
+
+cudaError_t launch_gate_logits_to_log(const void* z, float* g, size_t n, float gs, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  if (n % 8) return cudaErrorInvalidValue;
+  {
+    ScopedTiming tm("gate_logits_to_log", s);
+    gate_logits_to_log_kernel<<<gate_pass_grid(n / 8), 256, 0, s>>>((const bf16*)z, g, n / 8, gs);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate_dlogit(float* dg, const void* z, size_t n, float gs, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  if (n % 8) return cudaErrorInvalidValue;
+  {
+    ScopedTiming tm("gate_dlogit", s);
+    gate_dlogit_kernel<<<gate_pass_grid(n / 8), 256, 0, s>>>(dg, (const bf16*)z, n / 8, gs);
+  }
+  return cudaGetLastError();
+}
+
 size_t gla_out_loss_parts(int B, int H, int T) { return (size_t)B * H * ((T + C - 1) / C); }
 
 cudaError_t launch_gla_bwd_scan(const GlaBwdScanParams& p, cudaStream_t s) {

@@ -112,6 +112,10 @@ cudaError_t launch_gla_states(const GlaFwdParams& p, cudaStream_t s);
 // whether launch_gla_states takes the two-level path (given delta16 / decay)
 bool gla_states_scan_wanted(int T);
 cudaError_t launch_gla_out(const GlaFwdParams& p, cudaStream_t s);
+// gates given as bf16 logits z: g = gs * log sigma(z) into fp32 (n elements,
+// a multiple of 8), and dL/dg -> dL/dz = dL/dg * gs * sigma(-z) in place
+cudaError_t launch_gate_logits_to_log(const void* z, float* g, size_t n, float gs, cudaStream_t s);
+cudaError_t launch_gate_dlogit(float* dg, const void* z, size_t n, float gs, cudaStream_t s);
 
 // ---- gated backward, two-level (bf16, dk = dv = 128) ------------------------
 // launch_gla_bwd_scan: every chunk's dG_c = (q e^{b})^T dO and decay e^{b_l}

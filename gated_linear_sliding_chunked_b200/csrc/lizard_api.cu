@@ -14,6 +14,7 @@ namespace {
 thread_local std::string g_err;
 thread_local bool g_prefer_tc = true;  // lz_prefer_tcgen05
 thread_local bool g_tc_all = false;  // lz_tcgen05_all
+thread_local bool g_fused_logits = false;  // lz_fused_gate_logits
 
 // The window branch's forward for bf16 with dk = dv = 128: tcgen05 for
 // w <= 129 (unless the calling thread asked for the warp-level kernel),
@@ -302,6 +303,33 @@ HybridBwdWs carve_hybrid_bwd(Carver& c, const lz_dims* d) {
   return w;
 }
 
+// Gates given as logits: their fp32 log-gates, carved last in the gated and
+// hybrid workspaces (the size depends on the dims alone).
+float* carve_gates(Carver& c, const lz_dims* d) {
+  return d->gate_logits ? c.take<float>(bht(d) * d->dk) : nullptr;
+}
+
+// The gates the kernels read.  Logits are mapped once to fp32 log-gates in
+// the workspace (g32) and the call proceeds as with log-gates, unless the
+// calling thread asked for the kernels that map them on the fly
+// (lz_fused_gate_logits); z is then set for the backward to map dL/dg back
+// to dL/dz.
+struct GateIn {
+  lz_dims d;        // the dims the kernels see
+  const float* g;   // the gates they read
+  const void* z;    // the logits, when they were mapped here
+};
+cudaError_t gate_input(const lz_dims* d, const float* g, float* g32, cudaStream_t s, GateIn& out) {
+  out.d = *d;
+  out.g = g;
+  out.z = nullptr;
+  if (!d->gate_logits || g_fused_logits || g32 == nullptr) return cudaSuccess;
+  out.d.gate_logits = 0;
+  out.g = g32;
+  out.z = g;
+  return lz::launch_gate_logits_to_log(g, g32, bht(d) * d->dk, d->gate_scale, s);
+}
+
 size_t ws_bytes(const lz_dims* d, int which) {
   Carver c(nullptr);
   switch (which) {
@@ -310,6 +338,7 @@ size_t ws_bytes(const lz_dims* d, int which) {
         c.take<uint16_t>(states16_count(d));
         carve_scan(c, d);
       }
+      carve_gates(c, d);
       return c.off;
     case LZ_WS_HYBRID_FWD:
       if (!hybrid_uses_mma(d)) c.take<float>(bht(d) * d->dv);  // fp32 window output
@@ -317,6 +346,7 @@ size_t ws_bytes(const lz_dims* d, int which) {
         c.take<uint16_t>(states16_count(d));
         carve_scan(c, d);
       }
+      carve_gates(c, d);
       return c.off;
     case LZ_WS_HYBRID_FWD_MSE:
       c.off = ws_bytes(d, LZ_WS_HYBRID_FWD);
@@ -324,12 +354,14 @@ size_t ws_bytes(const lz_dims* d, int which) {
       return c.off;
     case LZ_WS_GLA_BWD:
       carve_gla_bwd(c, d);
+      carve_gates(c, d);
       return c.off;
     case LZ_WS_SWA_BWD:
       carve_swa_bwd(c, d);
       return c.off;
     case LZ_WS_HYBRID_BWD:
       carve_hybrid_bwd(c, d);
+      carve_gates(c, d);
       return c.off;
     case LZ_WS_CHUNK_STATES:
       return fwd_uses_chunks(d) && bwd_uses_mma(d) ? states16_count(d) * sizeof(uint16_t) : 0;
@@ -427,6 +459,12 @@ int lz_tcgen05_all(int on) {
   return prev;
 }
 
+int lz_fused_gate_logits(int on) {
+  const int prev = g_fused_logits ? 1 : 0;
+  g_fused_logits = on != 0;
+  return prev;
+}
+
 size_t lz_workspace_bytes(const lz_dims* d, int which) {
   if (check_dims(d, which != LZ_WS_GLA_FWD && which != LZ_WS_GLA_BWD) != LZ_OK) return 0;
   return ws_bytes(d, which);
@@ -442,14 +480,19 @@ lz_status lz_gla_fwd(const lz_dims* d, const void* q, const void* k, const void*
   LZ_PTR(h0, false); LZ_PTR(hT, false); LZ_PTR(chunk_states, false);
   st = check_ws(d, LZ_WS_GLA_FWD, ws, ws_bytes_);
   if (st != LZ_OK) return st;
-  lz::GlaFwdParams p = gla_fwd_params(d, q, k, v, g, h0);
-  p.o = o;
-  p.hT = hT;
+  const cudaStream_t s = as_stream(stream);
   Carver c(ws);
   void* states16 = fwd_uses_chunks(d) ? c.take<uint16_t>(states16_count(d)) : nullptr;
   const ScanWs scan = fwd_uses_chunks(d) ? carve_scan(c, d) : ScanWs{};
+  float* g32 = carve_gates(c, d);
   if (states16 && chunk_states && ws_bytes(d, LZ_WS_CHUNK_STATES) > 0) states16 = chunk_states;
-  return cuda_status(gla_forward(p, d->io == LZ_BF16, states16, scan, as_stream(stream)), "lz_gla_fwd");
+  GateIn gi;
+  cudaError_t e = gate_input(d, g, g32, s, gi);
+  if (e != cudaSuccess) return cuda_status(e, "lz_gla_fwd (gate logits)");
+  lz::GlaFwdParams p = gla_fwd_params(&gi.d, q, k, v, gi.g, h0);
+  p.o = o;
+  p.hT = hT;
+  return cuda_status(gla_forward(p, d->io == LZ_BF16, states16, scan, s), "lz_gla_fwd");
 }
 
 lz_status lz_swa_meta_fwd(const lz_dims* d, const void* q, const void* k, const void* v,
@@ -502,9 +545,15 @@ static lz_status hybrid_fwd_impl(const char* name, const lz_dims* d, const void*
   float* osw = mma ? nullptr : c.take<float>(bht(d) * d->dv);
   void* states16 = fwd_uses_chunks(d) ? c.take<uint16_t>(states16_count(d)) : nullptr;
   const ScanWs scan = fwd_uses_chunks(d) ? carve_scan(c, d) : ScanWs{};
+  float* g32 = carve_gates(c, d);
   float* parts = la ? c.take<float>(loss_parts(d)) : nullptr;
   if (states16 && chunk_states && ws_bytes(d, LZ_WS_CHUNK_STATES) > 0) states16 = chunk_states;
-  lz::GlaFwdParams gp = gla_fwd_params(d, q, k, v, g, h0);
+  GateIn gi;  // before the fork: the side stream's state pass reads the mapped gates
+  {
+    const cudaError_t e = gate_input(d, g, g32, s, gi);
+    if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_fwd (gate logits)");
+  }
+  lz::GlaFwdParams gp = gla_fwd_params(&gi.d, q, k, v, gi.g, h0);
   gp.o = o;
   gp.hT = hT;
   // tensor-core path: the gated state pass (reads k, v, g; writes the chunk
@@ -680,12 +729,17 @@ lz_status lz_gla_bwd(const lz_dims* d, const void* q, const void* k, const void*
   if (st != LZ_OK) return st;
   st = check_ws(d, LZ_WS_GLA_BWD, ws, ws_bytes_);
   if (st != LZ_OK) return st;
+  const cudaStream_t s = as_stream(stream);
   Carver c(ws);
   GlaBwdWs w = carve_gla_bwd(c, d);
-  return cuda_status(gla_bwd_launch(d, q, k, v, g, h0, dO, dhT, chunk_states, hT, dq, dk, dv,
-                                    dg, dh0, w,
-                                    nullptr, nullptr, nullptr, false, as_stream(stream)),
-                     "lz_gla_bwd");
+  float* g32 = carve_gates(c, d);
+  GateIn gi;
+  cudaError_t e = gate_input(d, g, g32, s, gi);
+  if (e != cudaSuccess) return cuda_status(e, "lz_gla_bwd (gate logits)");
+  e = gla_bwd_launch(&gi.d, q, k, v, gi.g, h0, dO, dhT, chunk_states, hT, dq, dk, dv, dg, dh0, w,
+                     nullptr, nullptr, nullptr, false, s);
+  if (e == cudaSuccess && gi.z) e = lz::launch_gate_dlogit(dg, gi.z, bht(d) * d->dk, d->gate_scale, s);
+  return cuda_status(e, "lz_gla_bwd");
 }
 
 lz_status lz_swa_meta_bwd(const lz_dims* d, const void* q, const void* k, const void* v,
@@ -735,6 +789,12 @@ lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const vo
   const cudaStream_t s = as_stream(stream);
   Carver c(ws);
   HybridBwdWs w = carve_hybrid_bwd(c, d);
+  float* g32 = carve_gates(c, d);
+  GateIn gi;  // before the fork: the gated first phase reads the mapped gates
+  {
+    const cudaError_t e = gate_input(d, g, g32, s, gi);
+    if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (gate logits)");
+  }
   const bool mma = hybrid_uses_mma(d);
   lz::SwaBwdParams p = swa_bwd_params(d, q, k, v, meta_k, meta_v, lse, o_swa, dO, w.swa);
   p.gscale = d->alpha;
@@ -747,9 +807,10 @@ lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const vo
   if (!mma || bht(d) == 0) {
     cudaError_t e = swa_backward(p, d->io == LZ_BF16, s);
     if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (window branch)");
-    return cuda_status(gla_bwd_launch(d, q, k, v, g, h0, dO, dhT, chunk_states, hT, dq, dk, dv,
-                                      dg, dh0, w.gla, w.dq, w.dk, w.dv, mma, s),
-                       "lz_hybrid_bwd (gated branch)");
+    e = gla_bwd_launch(&gi.d, q, k, v, gi.g, h0, dO, dhT, chunk_states, hT, dq, dk, dv, dg, dh0,
+                       w.gla, w.dq, w.dk, w.dv, mma, s);
+    if (e == cudaSuccess && gi.z) e = lz::launch_gate_dlogit(dg, gi.z, bht(d) * d->dk, d->gate_scale, s);
+    return cuda_status(e, "lz_hybrid_bwd (gated branch)");
   }
   // tensor-core path: the gated backward's first phase (it reads only the
   // inputs and writes only its scratch and dh0) runs on the side stream while
@@ -762,7 +823,7 @@ lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const vo
   if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->fork, 0);
   if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (fork)");
   lz::GlaBwdParams gp;
-  e = gla_bwd_phase1(d, q, k, v, g, h0, dO, dhT, chunk_states, hT, dq, dk, dv, dg, dh0, w.gla,
+  e = gla_bwd_phase1(&gi.d, q, k, v, gi.g, h0, dO, dhT, chunk_states, hT, dq, dk, dv, dg, dh0, w.gla,
                      w.dq, w.dk, w.dv, mma, gp, ss->stream);
   // the join is recorded even after a failed launch, so that the caller's
   // stream never depends on an unrecorded event
@@ -773,7 +834,9 @@ lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const vo
   const cudaError_t ew = cudaStreamWaitEvent(s, ss->join, 0);
   if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (window branch)");
   if (ew != cudaSuccess) return cuda_status(ew, "lz_hybrid_bwd (join)");
-  return cuda_status(gla_bwd_phase2(d, gp, w.gla.tcflags, s), "lz_hybrid_bwd (gated branch)");
+  e = gla_bwd_phase2(&gi.d, gp, w.gla.tcflags, s);
+  if (e == cudaSuccess && gi.z) e = lz::launch_gate_dlogit(dg, gi.z, bht(d) * d->dk, d->gate_scale, s);
+  return cuda_status(e, "lz_hybrid_bwd (gated branch)");
 }
 
 lz_status lz_decode_prefill(int Bd, int H, int T, int dk, int dv, int w, lz_dtype io,

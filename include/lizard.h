@@ -388,6 +388,17 @@ int lz_prefer_tcgen05(int on);
  * setting; never fails. */
 int lz_tcgen05_all(int on);
 
+/* How gates given as logits (lz_dims.gate_logits = 1) reach the gated
+ * kernels, for the calling host thread (no counterpart on the pages; default
+ * off).  Off: one pass maps the logits to fp32 log-gates in the call's
+ * workspace (the gated and hybrid workspaces hold B*H*T*dk floats for them
+ * whenever gate_logits is set) and the backward maps dL/dg to dL/dz in one
+ * more pass over dg.  On: every gated kernel maps the logits itself as it
+ * reads them (fewer bytes, more special-function work; measured slower on
+ * B200).  Both give the same result up to rounding.  Returns the previous
+ * setting; never fails. */
+int lz_fused_gate_logits(int on);
+
 /* Per-launch device timing for benchmarks (no counterpart on the pages; a
  * measurement aid).  lz_timing_enable(1) makes every later kernel launch of
  * this library from the calling host thread record a pair of CUDA events

@@ -1,7 +1,10 @@
 """Gate logits (the gate as sigma(z), z from the projection upstream): the
-kernels form the log-gate scale * log sigma(z) as they load it and the
-backward returns dL/dz.  CUDA library through the C ABI vs the fp64 oracle
-(the oracle's gate map, then its operator and its chain rule)."""
+log-gate is scale * log sigma(z) and the backward returns dL/dz.  Both ways
+the library takes them: one pass maps them to fp32 log-gates in the
+workspace and one more maps dL/dg to dL/dz (the default), or every gated
+kernel maps them as it loads them (lz_fused_gate_logits).  CUDA library
+through the C ABI vs the fp64 oracle (the oracle's gate map, then its
+operator and its chain rule)."""
 import math
 
 import numpy as np
@@ -15,6 +18,13 @@ from parity_util import assert_close, np64, oracle_inputs, small_problem
 pytestmark = pytest.mark.gpu
 
 D = 128
+
+
+@pytest.fixture(params=[False, True], ids=["mapped-once", "fused"], autouse=True)
+def logits_mode(request):
+    prev = L.lz_fused_gate_logits(request.param)
+    yield request.param
+    L.lz_fused_gate_logits(prev)
 
 
 def _logits(seed, shape, mu, sigma):
