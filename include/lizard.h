@@ -379,7 +379,8 @@ int lz_prefer_tcgen05(int on);
  *    128-token chunks (TMA-fed operands, every contraction with M = 128 and
  *    its accumulator in tensor memory) for every chunk whose fp32 log-gates
  *    decay each 64-token half by at most e^-60 in every key dim
- *    (faster-decaying chunks, and gates given as logits, stay on the
+ *    (faster-decaying chunks, and gates given as logits under
+ *    lz_fused_gate_logits(1), stay on the
  *    warp-level kernel over 64-token chunks);
  *  - the query side of the window backward (dq, D, the meta-gradient and
  *    dalpha partials) runs on a tcgen05 kernel when lz_prefer_tcgen05 is on,
