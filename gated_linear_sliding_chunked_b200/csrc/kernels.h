@@ -192,6 +192,11 @@ bool swa_fwd_tc_supported(int dk, int dv, bool bf16, int w);
 cudaError_t launch_swa_fwd_tc(const SwaFwdParams& p, cudaStream_t s);
 
 struct SwaBwdParams {
+  // the hybrid backward's overlap: an event (cudaEvent_t) recorded right after
+  // the query-side launch, and the partials' reduction left to the caller
+  // (launch_swa_bwd_mma_reduce) on another stream
+  void* query_done = nullptr;
+  bool defer_reduce = false;
   const void* q;
   const void* k;
   const void* v;
@@ -239,6 +244,8 @@ cudaError_t launch_swa_bwd_reduce(const SwaBwdParams& p, int nparts, int nalpha,
 // tensor-core backward (bf16 I/O, dk = dv = 128); same scratch layout
 bool swa_bwd_mma_supported(int dk, int dv, bool bf16);
 cudaError_t launch_swa_bwd_mma(const SwaBwdParams& p, cudaStream_t s);
+// the partials' reduction of launch_swa_bwd_mma (when it was deferred)
+cudaError_t launch_swa_bwd_mma_reduce(const SwaBwdParams& p, cudaStream_t s);
 // key side (dk, dv) on tcgen05 with TMA-fed operands
 bool swa_bwd_kv_tc_supported(int dk, int dv, bool bf16);
 cudaError_t launch_swa_bwd_kv_tc(const SwaBwdParams& p, cudaStream_t s);

@@ -63,6 +63,7 @@ struct SideStream {
   cudaStream_t stream = nullptr;
   cudaEvent_t fork = nullptr;
   cudaEvent_t join = nullptr;
+  cudaEvent_t mid = nullptr;  // lz_hybrid_bwd: the window backward's query side done
 };
 
 static cudaError_t side_stream(SideStream** out) {
@@ -78,6 +79,7 @@ static cudaError_t side_stream(SideStream** out) {
     e = cudaStreamCreateWithPriority(&ss.stream, cudaStreamNonBlocking, hi);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.mid, cudaEventDisableTiming);
     if (e != cudaSuccess) {
       ss = SideStream{};
       return e;
@@ -825,14 +827,25 @@ lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const vo
   lz::GlaBwdParams gp;
   e = gla_bwd_phase1(&gi.d, q, k, v, gi.g, h0, dO, dhT, chunk_states, hT, dq, dk, dv, dg, dh0, w.gla,
                      w.dq, w.dk, w.dv, mma, gp, ss->stream);
+  // the window backward here; its partials' reduction (which needs only the
+  // query side) joins the side stream behind the gated first phase, off the
+  // path to the per-chunk gradients
+  p.query_done = (void*)ss->mid;
+  p.defer_reduce = true;
+  const cudaError_t esw = e == cudaSuccess ? swa_backward(p, d->io == LZ_BF16, s) : cudaSuccess;
+  cudaError_t er = cudaSuccess;
+  if (e == cudaSuccess && esw == cudaSuccess) {
+    er = cudaStreamWaitEvent(ss->stream, ss->mid, 0);
+    if (er == cudaSuccess) er = lz::launch_swa_bwd_mma_reduce(p, ss->stream);
+  }
   // the join is recorded even after a failed launch, so that the caller's
   // stream never depends on an unrecorded event
   const cudaError_t ej = cudaEventRecord(ss->join, ss->stream);
-  if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (gated branch, first phase)");
-  if (ej != cudaSuccess) return cuda_status(ej, "lz_hybrid_bwd (join)");
-  e = swa_backward(p, d->io == LZ_BF16, s);
   const cudaError_t ew = cudaStreamWaitEvent(s, ss->join, 0);
-  if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (window branch)");
+  if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (gated branch, first phase)");
+  if (esw != cudaSuccess) return cuda_status(esw, "lz_hybrid_bwd (window branch)");
+  if (er != cudaSuccess) return cuda_status(er, "lz_hybrid_bwd (window partials)");
+  if (ej != cudaSuccess) return cuda_status(ej, "lz_hybrid_bwd (join)");
   if (ew != cudaSuccess) return cuda_status(ew, "lz_hybrid_bwd (join)");
   e = gla_bwd_phase2(&gi.d, gp, w.gla.tcflags, s);
   if (e == cudaSuccess && gi.z) e = lz::launch_gate_dlogit(dg, gi.z, bht(d) * d->dk, d->gate_scale, s);

@@ -749,6 +749,8 @@ cudaError_t launch_swa_bwd_mma(const SwaBwdParams& p, cudaStream_t s) {
       e = cudaGetLastError();
     }
     if (e != cudaSuccess) return e;
+    if (p.query_done) e = cudaEventRecord((cudaEvent_t)p.query_done, s);
+    if (e != cudaSuccess) return e;
     if (kv_tc) {
       e = launch_swa_bwd_kv_tc(pp, s);
     } else {
@@ -774,6 +776,14 @@ cudaError_t launch_swa_bwd_mma(const SwaBwdParams& p, cudaStream_t s) {
       if (e != cudaSuccess) return e;
     }
   }
+  if (empty && p.query_done) e = cudaEventRecord((cudaEvent_t)p.query_done, s);
+  if (e != cudaSuccess || p.defer_reduce) return e;
+  return launch_swa_bwd_mma_reduce(p, s);
+}
+
+cudaError_t launch_swa_bwd_mma_reduce(const SwaBwdParams& p, cudaStream_t s) {
+  const bool empty = p.T == 0 || p.B * p.H == 0;
+  const int nslab = (p.T + SLAB - 1) / SLAB;
   const int nparts = (p.M > 0 && !empty) ? p.B * nslab : 0;
   const int nalpha = empty ? 0 : p.B * p.H * nslab;
   return launch_swa_bwd_reduce(p, nparts, nalpha, s);
