@@ -78,9 +78,10 @@ typedef struct {
   float alpha;    /* weight of the window branch in the hybrid sum */
   int gate_logits;   /* 0: `g` holds fp32 log-gates.  1: `g` holds the gate
                       * LOGITS z, bf16 [B,H,T,dk] (section 2a: the gate is
-                      * sigma(W_gamma x), z = W_gamma x); the kernels form the
-                      * log-gate gate_scale * log sigma(z) as they load it, and
-                      * the backward's dg receives dL/dz (fp32).  Needs
+                      * sigma(W_gamma x), z = W_gamma x); the log-gate is
+                      * gate_scale * log sigma(z) (mapped once into the call's
+                      * scratch, or inside the kernels: lz_fused_gate_logits),
+                      * and the backward's dg receives dL/dz (fp32).  Needs
                       * io = LZ_BF16 and dk = dv = 128 (LZ_ERR_UNSUPPORTED
                       * otherwise).  Zero-initialised dims keep mode 0. */
   float gate_scale;  /* > 0, used when gate_logits = 1 (a temperature; 1 is
@@ -95,7 +96,8 @@ typedef struct {
  * before every 64-token chunk, [B, H, ceil(T/64), dk, dv] bf16, kept by the
  * forward so that the backward need not walk the sequence again.  It is 0
  * where the kernels keep no such states (fp32 I/O, d = 64); the pointers
- * are then ignored. */
+ * are then ignored.  With gate_logits = 1 the gated and hybrid scratch also
+ * holds B*H*T*dk floats for the mapped log-gates. */
 enum { LZ_WS_GLA_FWD = 0, LZ_WS_HYBRID_FWD = 1, LZ_WS_GLA_BWD = 2,
        LZ_WS_SWA_BWD = 3, LZ_WS_HYBRID_BWD = 4, LZ_WS_CHUNK_STATES = 5,
        LZ_WS_HYBRID_FWD_MSE = 6 };
