@@ -44,7 +44,7 @@ constexpr int KR = 128;   // keys per CTA (MMA M)
 constexpr int QT = 64;    // queries per tile
 constexpr int D = 128;
 constexpr int NSW = 256;  // softmax threads (warps 0-7)
-constexpr int kBlocksPerCta = 2;  // consecutive key blocks one CTA walks (4: 0.392 ms, 8: 0.462 ms alone)
+constexpr int kBlocksPerCta = 2;  // consecutive key blocks one CTA walks (3: 0.410, 4: 0.392, 8: 0.462 ms alone)
 constexpr int NTH = NSW + 32;  // + the producer warp
 constexpr uint32_t kHalf = 64 * 2;  // bytes of one swizzled row (64 dims)
 constexpr uint32_t kTmemCols = 512;
