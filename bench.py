@@ -107,10 +107,13 @@ class ClockSampler:
 
     def _nvml_loop(self, handle, nv):
         import time
+        try:  # a constant: read once, so that each sample costs two calls
+            mx = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
+        except Exception:
+            mx = 0
         while not self.stop.is_set():
             try:
                 sm = nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM)
-                mx = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
                 bits = nv.nvmlDeviceGetCurrentClocksEventReasons(handle)
                 self.samples.append((float(sm), float(mx),
                                      {n for n, b in self.REASONS.items() if bits & b}))
