@@ -550,31 +550,38 @@ static lz_status hybrid_fwd_impl(const char* name, const lz_dims* d, const void*
   float* g32 = carve_gates(c, d);
   float* parts = la ? c.take<float>(loss_parts(d)) : nullptr;
   if (states16 && chunk_states && ws_bytes(d, LZ_WS_CHUNK_STATES) > 0) states16 = chunk_states;
-  GateIn gi;  // before the fork: the side stream's state pass reads the mapped gates
-  {
-    const cudaError_t e = gate_input(d, g, g32, s, gi);
-    if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_fwd (gate logits)");
-  }
-  lz::GlaFwdParams gp = gla_fwd_params(&gi.d, q, k, v, gi.g, h0);
-  gp.o = o;
-  gp.hT = hT;
   // tensor-core path: the gated state pass (reads k, v, g; writes the chunk
-  // states and hT) runs on the side stream while the window forward runs here
+  // states and hT) runs on the side stream while the window forward runs
+  // here; gate logits are mapped there too, ahead of it (the window branch
+  // does not read the gates; the output pass comes after the join)
   SideStream* side = nullptr;
-  if (mma && fwd_uses_chunks(d) && bht(d) > 0) {
+  const bool fork = mma && fwd_uses_chunks(d) && bht(d) > 0;
+  if (fork) {
     cudaError_t e = side_stream(&side);
     if (e == cudaSuccess) e = cudaEventRecord(side->fork, s);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(side->stream, side->fork, 0);
     if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_fwd (fork)");
+  }
+  GateIn gi;
+  cudaError_t eg = gate_input(d, g, g32, fork ? side->stream : s, gi);
+  lz::GlaFwdParams gp = gla_fwd_params(&gi.d, q, k, v, gi.g, h0);
+  gp.o = o;
+  gp.hT = hT;
+  if (fork) {
     gp.states16 = states16;
     gp.delta16 = scan.delta16;
     gp.decay = scan.decay;
-    e = lz::launch_gla_states(gp, side->stream);
+    cudaError_t e = eg == cudaSuccess ? lz::launch_gla_states(gp, side->stream) : eg;
     // recorded even after a failed launch: the caller's stream never waits
     // on an unrecorded event
     const cudaError_t ej = cudaEventRecord(side->join, side->stream);
-    if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_fwd (gated state pass)");
+    if (e != cudaSuccess) {
+      cudaStreamWaitEvent(s, side->join, 0);
+      return cuda_status(e, "lz_hybrid_fwd (gated state pass)");
+    }
     if (ej != cudaSuccess) return cuda_status(ej, "lz_hybrid_fwd (join)");
+  } else if (eg != cudaSuccess) {
+    return cuda_status(eg, "lz_hybrid_fwd (gate logits)");
   }
   lz::SwaFwdParams sp = swa_fwd_params(d, q, k, v, meta_k, meta_v);
   // tensor-core path: bf16 window output into o_swa if requested, else into o
@@ -792,11 +799,7 @@ lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const vo
   Carver c(ws);
   HybridBwdWs w = carve_hybrid_bwd(c, d);
   float* g32 = carve_gates(c, d);
-  GateIn gi;  // before the fork: the gated first phase reads the mapped gates
-  {
-    const cudaError_t e = gate_input(d, g, g32, s, gi);
-    if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (gate logits)");
-  }
+  GateIn gi;
   const bool mma = hybrid_uses_mma(d);
   lz::SwaBwdParams p = swa_bwd_params(d, q, k, v, meta_k, meta_v, lse, o_swa, dO, w.swa);
   p.gscale = d->alpha;
@@ -807,7 +810,9 @@ lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const vo
   p.dmk = dmeta_k; p.dmv = dmeta_v; p.dalpha = dalpha;
   p.ds_tiles = w.ds_tiles; p.ds_meta = w.ds_meta;
   if (!mma || bht(d) == 0) {
-    cudaError_t e = swa_backward(p, d->io == LZ_BF16, s);
+    cudaError_t e = gate_input(d, g, g32, s, gi);
+    if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (gate logits)");
+    e = swa_backward(p, d->io == LZ_BF16, s);
     if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (window branch)");
     e = gla_bwd_launch(&gi.d, q, k, v, gi.g, h0, dO, dhT, chunk_states, hT, dq, dk, dv, dg, dh0,
                        w.gla, w.dq, w.dk, w.dv, mma, s);
@@ -825,8 +830,13 @@ lz_status lz_hybrid_bwd(const lz_dims* d, const void* q, const void* k, const vo
   if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->fork, 0);
   if (e != cudaSuccess) return cuda_status(e, "lz_hybrid_bwd (fork)");
   lz::GlaBwdParams gp;
-  e = gla_bwd_phase1(&gi.d, q, k, v, gi.g, h0, dO, dhT, chunk_states, hT, dq, dk, dv, dg, dh0, w.gla,
-                     w.dq, w.dk, w.dv, mma, gp, ss->stream);
+  // gate logits are mapped on the side stream, ahead of the gated first phase
+  // (the window branch does not read the gates; the second phase comes after
+  // the join)
+  e = gate_input(d, g, g32, ss->stream, gi);
+  if (e == cudaSuccess)
+    e = gla_bwd_phase1(&gi.d, q, k, v, gi.g, h0, dO, dhT, chunk_states, hT, dq, dk, dv, dg, dh0,
+                       w.gla, w.dq, w.dk, w.dv, mma, gp, ss->stream);
   // the window backward here; its partials' reduction (which needs only the
   // query side) joins the side stream behind the gated first phase, off the
   // path to the per-chunk gradients
