@@ -287,3 +287,31 @@ def test_projection_validation(lib):
         L.LZ_ERR_INVALID_ARG
     assert f(*args(T=0), *P, ctypes.c_float(1.0), *O, 0) == L.LZ_OK
 
+
+
+def test_kernel_choice_switches_are_per_thread(lib):
+    """The per-thread switches (tcgen05 kernels, the gate-logit map) return
+    the previous setting and leave other host threads' settings alone.  No
+    device is touched."""
+    import threading
+    switches = (L.lz_prefer_tcgen05, L.lz_tcgen05_all, L.lz_fused_gate_logits)
+    defaults = (True, False, False)
+    for sw, dflt in zip(switches, defaults):
+        assert sw(not dflt) == dflt
+        assert sw(dflt) == (not dflt)
+        assert sw(dflt) == dflt
+    seen = {}
+
+    def other():
+        seen["other"] = [sw(d) for sw, d in zip(switches, defaults)]
+
+    for sw, dflt in zip(switches, defaults):
+        sw(not dflt)
+    try:
+        t = threading.Thread(target=other)
+        t.start()
+        t.join()
+    finally:
+        for sw, dflt in zip(switches, defaults):
+            sw(dflt)
+    assert seen["other"] == list(defaults)
