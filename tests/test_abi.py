@@ -230,10 +230,20 @@ def test_gate_logits_validation(lib, kw, status):
 
 def test_gate_logits_workspace(lib):
     """Gate logits take the two-level state pass for any length, so its
-    scratch is there even for one chunk."""
+    scratch is there even for one chunk; every gated and hybrid workspace
+    also holds the mapped fp32 log-gates (B*H*T*dk floats, 256-byte
+    rounded), the window-only one does not."""
     d0 = _dims(dk=128, dv=128, T=64)
     d1 = _dims(dk=128, dv=128, T=64, gate_logits=1, gate_scale=0.0625)
     assert L.lz_workspace_bytes(d1, L.LZ_WS_HYBRID_FWD) > L.lz_workspace_bytes(d0, L.LZ_WS_HYBRID_FWD)
+    e0 = _dims(dk=128, dv=128, T=300)
+    e1 = _dims(dk=128, dv=128, T=300, gate_logits=1, gate_scale=0.0625)
+    gates = (e1.B * e1.H * e1.T * e1.dk * 4 + 255) // 256 * 256
+    for kind in (L.LZ_WS_GLA_FWD, L.LZ_WS_HYBRID_FWD, L.LZ_WS_HYBRID_FWD_MSE, L.LZ_WS_GLA_BWD,
+                 L.LZ_WS_HYBRID_BWD):
+        assert L.lz_workspace_bytes(e1, kind) - L.lz_workspace_bytes(e0, kind) == gates, kind
+    for kind in (L.LZ_WS_SWA_BWD, L.LZ_WS_CHUNK_STATES):
+        assert L.lz_workspace_bytes(e1, kind) == L.lz_workspace_bytes(e0, kind), kind
 
 
 def test_binding_reads_bf16_gates_as_logits():
