@@ -686,7 +686,7 @@ __global__ void __launch_bounds__(NT3, 2) swa_bwd_dq_kernel(SwaBwdParams p) {
     if ((q0 - b * KB3) / QT3 + half < tiles_of(b)) {  // this warp's tile sees the block
       const bf16* dsb = sm.ds[st][half];
       const bf16* kb = sm.k[st];
-#pragma unroll 2
+#pragma unroll
       for (int kk = 0; kk < KU3 / 16; ++kk) {
         uint32_t a[4];  // A = dS (queries x keys) from the [key][query] tile, transposed
         ldsm_x4_t(smem_u32(&dsb[(kk * 16 + (lane & 7) + ((lane >> 4) << 3)) * DSP + rw + ((lane >> 3) & 1) * 8]),
